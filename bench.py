@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Throughput of the SPIN-4DGS per-Gaussian attribute decoder on B200.
+
+Metric: decoded spatiotemporal positions/s.  One step = one fused decode
+(normalise -> 4D hash encode -> trunk + heads -> activations -> Sigma) of one
+synthetic sports frame (300k positions, 16-level fp16 hash grid with 2^19
+entries per level, 32-64-64-11 fp16 network).  With N GPUs every rank
+decodes its own frame (weak scaling, no collective on the data path); the
+time is the max over ranks.  A second measurement covers fwd+bwd: one
+1M-position training launch (forward, then backward with the scatter-add into
+the tables and the weight gradients).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from spatiotemporal_neural_field_b200 import synthetic as S  # noqa: E402
+
+WORKLOAD = "sports_frame_fp16"
+OUT_WIDTHS = S.DECODE_OUT_WIDTHS
+METRIC = "decoded spatiotemporal positions/s (fwd)"
+UNIT = "positions/s"
+KERNEL_SRC = os.path.join(ROOT, "spatiotemporal_neural_field_b200", "csrc")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-fwd-bwd", action="store_true")
+    p.add_argument("--cpu-sample", type=int, default=150_000, help="positions the oracle decodes for cpu_baseline")
+    return p.parse_args()
+
+
+def workload_config(n_gpus):
+    w = S.WORKLOADS[WORKLOAD]
+    g, m = w["grid"], w["mlp"]
+    return {
+        "workload": "%s: one frame of %d positions per GPU (80%% static, 20%% in 8 fast blobs), "
+                    "L=%d F=%d T=2^%d fp16 tables, spatial res %d-%d, temporal %d-%d, "
+                    "%d-%dx%d-11 fp16 trunk+heads" % (WORKLOAD, w["N"], g.L, g.F, g.log2_T, g.nmin_s, g.nmax_s,
+                                                       g.nmin_t, g.nmax_t, m.in_dim, m.n_hidden, m.hidden),
+        "positions_per_gpu": w["N"],
+        "l2": "flushed before every timed step (256 MiB write, outside the events)",
+        "parallelism": "dp%d (independent frames per rank, no collective)" % n_gpus,
+    }
+
+
+def algorithmic_bytes_per_position():
+    """Useful bytes a position needs: 16 levels x 16 corners x F fp16 features,
+    its 16-byte (x,y,z,t) input and 17 fp32 outputs."""
+    g = S.WORKLOADS[WORKLOAD]["grid"]
+    return g.L * 16 * g.F * 2 + 16 + 17 * 4
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(KERNEL_SRC)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(KERNEL_SRC, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "decode_fwd_sports_frame.traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(n_sample):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    from threadpoolctl import threadpool_limits
+    from oracle import decoder as dec
+    w = S.WORKLOADS[WORKLOAD]
+    frame = S.sports_scene(w["N"]).frame(w["frame"])
+    rows = np.random.default_rng(7).choice(len(frame), n_sample, replace=False)
+    tables = S.hash_tables(w["grid"])
+    weights = S.mlp_weights(w["mlp"])
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        dec.decode_forward(frame[rows], tables, weights, w["grid"], w["mlp"])
+        dt = time.perf_counter() - t0
+    return {"value": n_sample / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d positions of the same frame (numpy fp64, BLAS limited to 1 thread)" % n_sample,
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+    from oracle import decoder as dec
+    w = S.WORKLOADS[WORKLOAD]
+    frame = S.sports_scene(w["N"]).frame(w["frame"])
+    tables = S.hash_tables(w["grid"])
+    weights = S.mlp_weights(w["mlp"])
+    sample = 10_000
+    rng = np.random.default_rng(11)
+    with threadpool_limits(limits=1):
+        for _ in range(args.warmup):
+            dec.decode_forward(frame[rng.choice(len(frame), sample, replace=False)], tables, weights, w["grid"], w["mlp"])
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            dec.decode_forward(frame[rng.choice(len(frame), sample, replace=False)], tables, weights, w["grid"], w["mlp"])
+        dt = time.perf_counter() - t0
+    value = sample * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "%d positions of the frame per step" % sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from spatiotemporal_neural_field_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        dist.barrier()
+    from spatiotemporal_neural_field_b200 import spin4d as sp
+
+    w = S.WORKLOADS[WORKLOAD]
+    grid, mlp, N = w["grid"], w["mlp"], w["N"]
+    scene = S.sports_scene(N)
+    frame_idx = (w["frame"] + rank) % S.N_FRAMES
+    pos_h = scene.frame(frame_idx)
+    tables = torch.from_numpy(S.hash_tables(grid)).to(dev)
+    weights = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
+    pos = torch.from_numpy(pos_h).to(dev)
+    g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+    out = sp.alloc_outputs(N, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sp.decode_fwd(g, m, pos, tables, weights, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    clocks = ClockSampler(uuid)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = N * world * args.steps / (ms_max * 1e-3)
+
+    # ---- end to end: pinned host input -> decode -> pinned host outputs ----
+    pos_pin = torch.from_numpy(pos_h).pin_memory()
+    out_pin = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+    pos_d = torch.empty_like(pos)
+
+    def e2e_step():
+        pos_d.copy_(pos_pin, non_blocking=True)
+        sp.decode_fwd(g, m, pos_d, tables, weights, out=out, stream=stream)
+        for k in out:
+            out_pin[k].copy_(out[k], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e_s.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = N * world * args.steps / (float(te.item()) * 1e-3)
+    h2d = pos_h.nbytes
+    d2h = sum(v.numel() * v.element_size() for v in out.values())
+
+    # ---- fwd+bwd: one 1M-position training launch ----
+    fwd_bwd = None
+    if not args.no_fwd_bwd:
+        wt = S.WORKLOADS["sports_train_fp16"]
+        nb = wt["batch"]
+        pb = torch.from_numpy(scene.frames(range(0, 4))[:nb]).to(dev)
+        gb = {k: torch.randn((nb, wd), device=dev, generator=torch.Generator(device=dev).manual_seed(rank))
+              * wt["grad_std"] for k, wd in OUT_WIDTHS.items()}
+        outb = sp.alloc_outputs(nb, dev)
+        gtab = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), dtype=torch.float32, device=dev)
+        gwt = torch.zeros(mlp.n_params(), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(sp.decode_bwd_workspace(g, m, nb), 1), dtype=torch.uint8, device=dev)
+
+        def fb():
+            sp.decode_fwd(g, m, pb, tables, weights, out=outb, stream=stream)
+            sp.decode_bwd(g, m, pb, tables, weights, gb, gtab, gwt, workspace=ws, stream=stream)
+
+        for _ in range(max(3, args.warmup // 2)):
+            fb()
+        torch.cuda.synchronize()
+        k = max(3, args.steps // 4)
+        evb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        for i in range(k):
+            flush.zero_()
+            evb[i][0].record(stream)
+            fb()
+            evb[i][1].record(stream)
+        torch.cuda.synchronize()
+        tb = torch.tensor([sum(a.elapsed_time(b) for a, b in evb)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(tb, op=dist.ReduceOp.MAX)
+        fwd_bwd = {"metric": "decoded spatiotemporal positions/s (fwd+bwd)", "value": nb * world * k /
+                   (float(tb.item()) * 1e-3), "unit": UNIT, "ms_per_step": float(tb.item()) / k,
+                   "workload": "sports_train_fp16: one 1M-position launch (frames 0-3), decode_fwd + decode_bwd"}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        bpp = algorithmic_bytes_per_position()
+        achieved = bpp * N / (ms_per_step * 1e-3) / 1e9
+        traffic = profiled_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": workload_config(world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                         "bytes_per_position": bpp, "kernel": "decode_fwd"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        }
+        if fwd_bwd:
+            line["fwd_bwd"] = fwd_bwd
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_sample)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

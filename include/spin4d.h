@@ -1,0 +1,289 @@
+/*
+ * spin4d.h -- C ABI of the B200-native SPIN-4DGS per-Gaussian attribute decoder.
+ *
+ * What the library computes (from "Implicit 4D Gaussian Splatting for Fast
+ * Motion with Large Inter-Frame Displacements", SPIN-4DGS, sections 3.1 and
+ * 3.3): each spatiotemporal Gaussian position (x, y, z, t) is normalised
+ * (Eq. 7 scene contraction, Eq. 8 time normalisation), encoded by a 4D
+ * multiresolution hash grid (Eq. 9), decoded by a shared trunk and a
+ * multibranch head (Eq. 10) into scale, rotation, colour and opacity with the
+ * activations of Eq. 11, and turned into a covariance Sigma = R S S^T R^T
+ * (Eq. 2).  The backward pass scatter-adds gradients into the hash tables and
+ * the network weights; Adam (section 4, implementation details) updates them.
+ * A HexPlane encoder with a two-branch deformation network (4D Gaussian
+ * Splatting reading notes, sections 3.1-3.2) is a second encoder behind the
+ * same covariance assembly, and a double-sigmoid temporal window (KineticGS
+ * notes, "learnable energy-flow activation") can gate the opacity.
+ *
+ * Conventions shared by every call:
+ *  - All array pointers are DEVICE pointers owned by the caller unless a
+ *    comment says otherwise.  The library never frees or keeps them.
+ *  - Every compute call is asynchronous on `stream` (NULL = the legacy
+ *    default stream), allocates no memory and never synchronises.
+ *  - Arguments are validated on the host before any launch; on a validation
+ *    failure nothing is launched and SPIN4D_ERR_INVALID (or
+ *    SPIN4D_ERR_UNSUPPORTED for a valid but unimplemented shape) is returned.
+ *    A launch failure returns SPIN4D_ERR_CUDA; spin4d_last_cuda_error() gives
+ *    the cudaError_t value.
+ *  - Gradient outputs ACCUMULATE (+=): the caller zeroes them first.  This is
+ *    what lets many batches add into one gradient before one Adam step.
+ *  - Arrays are row-major; "N x k" means N rows of k contiguous values.
+ *  - Environment variable SPIN4D_FAULT=<name> (for example
+ *    SPIN4D_FAULT=spin4d_decode_fwd) makes that entry point return
+ *    SPIN4D_ERR_INJECTED after validation and before any launch; it exists
+ *    to test callers' error paths without touching the GPU.
+ */
+#ifndef SPIN4D_H
+#define SPIN4D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* spin4d_stream_t;
+
+typedef enum spin4d_status {
+    SPIN4D_OK = 0,
+    SPIN4D_ERR_INVALID = -1,      /* bad argument; nothing launched */
+    SPIN4D_ERR_UNSUPPORTED = -2,  /* valid but not implemented shape; nothing launched */
+    SPIN4D_ERR_CUDA = -3,         /* a CUDA launch or query failed */
+    SPIN4D_ERR_NONFINITE = -4,    /* a kernel met a non-finite value (see spin4d_adam_step) */
+    SPIN4D_ERR_INJECTED = -5      /* SPIN4D_FAULT selected this call */
+} spin4d_status;
+
+typedef enum spin4d_dtype { SPIN4D_F32 = 0, SPIN4D_F16 = 1 } spin4d_dtype;
+
+#define SPIN4D_MAX_LEVELS 16
+#define SPIN4D_MAX_FEATURES 8
+#define SPIN4D_MAX_WIDTH 128
+
+/* grid flag: `pos` already holds x~ in [0,1]^4; skip Eq. 7-8 (values are clamped to [0,1]). */
+#define SPIN4D_INPUT_NORMALISED 1u
+
+/*
+ * 4D multiresolution hash grid (SPIN-4DGS section 3.3, Eq. 9).
+ * Level l owns T = 2^log2_T entries of F features; table memory is
+ * L x T x F values of `table_dtype`, entry-major (the F features of an entry
+ * are contiguous), level after level.  res[l][d] is the number of grid
+ * VERTICES along axis d (x, y, z, t) at level l (>= 2), so a normalised
+ * coordinate u in [0,1] sits at u * (res - 1).  A level whose vertex count
+ * res_x*res_y*res_z*res_t is <= T is indexed densely (x fastest); otherwise by
+ * the spatial hash (v_x*1 ^ v_y*2654435761 ^ v_z*805459861 ^ v_t*3674653429)
+ * mod 2^32, mod T.  Time is normalised by (t - t_min)/(t_max - t_min)
+ * (Eq. 8) and clamped to [0,1].
+ */
+typedef struct spin4d_grid_desc {
+    int32_t L;              /* levels, 1..16 */
+    int32_t F;              /* features per level: 1, 2, 4 or 8 */
+    int32_t log2_T;         /* entries per level = 2^log2_T, 4..24 */
+    int32_t table_dtype;    /* spin4d_dtype of the tables */
+    int32_t res[SPIN4D_MAX_LEVELS][4];
+    float t_min, t_max;     /* t_max > t_min */
+    uint32_t flags;         /* SPIN4D_INPUT_NORMALISED or 0 */
+    int32_t reserved;       /* must be 0 */
+} spin4d_grid_desc;
+
+/*
+ * Fills `g`.  Per-level resolutions follow Instant-NGP's geometric growth,
+ * res_l = floor(Nmin * b^l) with b = exp((ln Nmax - ln Nmin)/(L - 1)),
+ * separately for the spatial axes (nmin_s..nmax_s) and time (nmin_t..nmax_t).
+ * Host only; returns SPIN4D_ERR_INVALID on bad sizes.
+ */
+int spin4d_grid_init(spin4d_grid_desc* g, int L, int F, int log2_T, int table_dtype,
+                     int nmin_s, int nmax_s, int nmin_t, int nmax_t,
+                     float t_min, float t_max);
+
+/*
+ * Decoder network (SPIN-4DGS section 3.3, Eq. 10): a trunk of n_hidden
+ * ReLU layers of width `hidden` on the LF-dimensional latent, then one linear
+ * layer of 11 rows [scale 3 | rotation 4 | rgb 3 | opacity 1].
+ * Weights are ONE packed vector of `w_dtype`: for each layer in order,
+ * W[out][in] row-major followed by b[out].  in_dim must equal L*F.
+ * gate != 0 multiplies the opacity by the double-sigmoid window
+ * sigmoid((t~-(c-r))/tau) * sigmoid(((c+r)-t~)/tau) of the normalised time t~,
+ * with per-Gaussian (c, r) passed in `gate_cr`.
+ */
+typedef struct spin4d_mlp_desc {
+    int32_t in_dim;     /* = L*F, <= 128 */
+    int32_t hidden;     /* trunk width, 1..128 */
+    int32_t n_hidden;   /* trunk layers, 1..4 */
+    int32_t w_dtype;    /* spin4d_dtype of the packed weights */
+    int32_t gate;       /* 0 or 1 */
+    float tau;          /* > 0 when gate != 0 */
+} spin4d_mlp_desc;
+
+/* Number of values in the packed weight vector (or -1 if `m` is invalid). */
+int64_t spin4d_mlp_param_count(const spin4d_mlp_desc* m);
+
+/* Decoded attributes, structure of arrays, fp32, device memory:
+ * scale N x 3, rot N x 4 (unit, (w,x,y,z)), rgb N x 3, opacity N x 1,
+ * cov N x 6 packed (xx, xy, xz, yy, yz, zz).  None may be NULL. */
+typedef struct spin4d_outputs {
+    float* scale;
+    float* rot;
+    float* rgb;
+    float* opacity;
+    float* cov;
+} spin4d_outputs;
+
+/* Upstream gradients on the decoded attributes, same shapes as spin4d_outputs.
+ * A NULL member means a zero gradient for that attribute. */
+typedef struct spin4d_output_grads {
+    const float* scale;
+    const float* rot;
+    const float* rgb;
+    const float* opacity;
+    const float* cov;
+} spin4d_output_grads;
+
+/*
+ * Eq. 7-9: normalise and hash-encode N positions.
+ *   pos     N x 4 fp32 (x, y, z, t), 16-byte aligned
+ *   tables  L x T x F of g->table_dtype, aligned to F * sizeof(dtype)
+ *   z       N x (L*F) fp32 output, level-major (z[n][l*F + f])
+ * N == 0 is valid and launches nothing.
+ */
+int spin4d_encode_fwd(const spin4d_grid_desc* g, const float* pos, int64_t N,
+                      const void* tables, float* z, spin4d_stream_t stream);
+
+/*
+ * Eq. 7-11 and Eq. 2 fused: normalise, encode, trunk + head, activations
+ * s = exp(min(s^, 20)), r = r^/max(||r^||, 1e-12), rgb = sigmoid, o = sigmoid
+ * (times the gate when m->gate), then Sigma.  One kernel, nothing but `out`
+ * written to memory.
+ *   weights  packed vector, see spin4d_mlp_desc, 16-byte aligned
+ *   gate_cr  N x 2 fp32 (c, r) when m->gate, else ignored (may be NULL)
+ */
+int spin4d_decode_fwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
+                      const float* pos, int64_t N, const void* tables, const void* weights,
+                      const float* gate_cr, spin4d_outputs out, spin4d_stream_t stream);
+
+/* Bytes of device workspace spin4d_decode_bwd needs for N positions. */
+size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, int64_t N);
+
+/*
+ * Backward of spin4d_decode_fwd for loss = sum_k <grad_out.k, output_k>:
+ * recomputes the forward, then accumulates
+ *   grad_tables   += dloss/dtables   (L x T x F fp32, scatter-added with atomics)
+ *   grad_weights  += dloss/dweights  (packed like `weights`, fp32)
+ * The gradient of s^ is zero where s^ > 20 (the clip); ReLU passes where its
+ * input is > 0.  `workspace` (device, >= spin4d_decode_bwd_workspace bytes,
+ * 256-byte aligned, contents ignored on entry) holds per-block partial weight
+ * gradients so that grad_weights is summed in a fixed order.
+ */
+int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
+                      const float* pos, int64_t N, const void* tables, const void* weights,
+                      const float* gate_cr, const spin4d_output_grads* grad_out,
+                      float* grad_tables, float* grad_weights,
+                      void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
+ * Eq. 2 alone: Sigma = R(q) diag(s)^2 R(q)^T for unit quaternions q = (w,x,y,z).
+ *   scale N x 3, rot N x 4 (used as given, not renormalised), cov N x 6 packed.
+ */
+int spin4d_cov_assemble(const float* scale, const float* rot, int64_t N, float* cov,
+                        spin4d_stream_t stream);
+
+/*
+ * Adam (Kingma & Ba) with bias correction, step counted from 1:
+ *   m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+ *   p -= lr * (m / (1-b1^step)) / (sqrt(v / (1-b2^step)) + eps)
+ * over n fp32 parameters `params` with fp32 state m, v (zero before step 1).
+ * params_work (may be NULL) receives an fp16 copy of the updated parameters
+ * (the working copy fp16 tables / weights are read from).  zero_grad != 0
+ * clears `grad` after use.  If `nonfinite_flag` is non-NULL (device int32,
+ * caller-zeroed), it is set to 1 when any updated parameter is not finite;
+ * the host reads it when it chooses (the call itself never synchronises).
+ */
+int spin4d_adam_step(float* params, void* params_work, float* grad, float* m, float* v,
+                     int64_t n, int step, float lr, float b1, float b2, float eps,
+                     int zero_grad, int32_t* nonfinite_flag, spin4d_stream_t stream);
+
+/*
+ * HexPlane encoder + deformation network (4D Gaussian Splatting reading
+ * notes, sections 3.1-3.2).  Planes XY, XZ, YZ, XT, YT, ZT at each spatial
+ * resolution scales[s] (time axis: time_res samples), `channels` each,
+ * stored fp32 channel-last [rows = second axis][cols = first axis][C],
+ * scale-major then plane order; sampled bilinearly (align corners) at
+ * x~ = (mu + 1)/2 and t~ = frame/(n_frames - 1); samples concatenated
+ * (scale, plane, channel) into n_scales*6*channels features; trunk of
+ * n_hidden ReLU layers of width `hidden`; one 58-row linear layer
+ * [d_mu 3 | d_q 4 | d_logs 3 | d_sh 48]; weights packed fp32 as in
+ * spin4d_mlp_desc.
+ */
+typedef struct spin4d_hexplane_desc {
+    int32_t n_scales;       /* 1..4 */
+    int32_t scales[4];      /* spatial resolutions (vertices), >= 2 */
+    int32_t time_res;       /* time samples, >= 2 */
+    int32_t channels;       /* 32 (multiple of 4, <= 32) */
+    int32_t n_frames;       /* frames of the sequence, >= 2 */
+    int32_t hidden;         /* trunk width, <= 128 */
+    int32_t n_hidden;       /* trunk layers, 1..4 */
+} spin4d_hexplane_desc;
+
+/* Values in the packed plane array / weight vector (-1 if invalid). */
+int64_t spin4d_hexplane_plane_count(const spin4d_hexplane_desc* h);
+int64_t spin4d_hexplane_param_count(const spin4d_hexplane_desc* h);
+
+/* Deformed Gaussians: mu' N x 3, rot N x 4, scale N x 3, sh N x 48, cov N x 6 (fp32). */
+typedef struct spin4d_hex_outputs {
+    float* mu;
+    float* rot;
+    float* scale;
+    float* sh;
+    float* cov;
+} spin4d_hex_outputs;
+
+typedef struct spin4d_hex_output_grads {
+    const float* mu;
+    const float* rot;
+    const float* scale;
+    const float* sh;
+    const float* cov;
+} spin4d_hex_output_grads;
+
+/*
+ * mu' = mu + d_mu; q' = (q_can + d_q)/max(||q_can + d_q||, 1e-12);
+ * s' = exp(logs_can + d_logs); sh' = sh_can + d_sh; Sigma(s', q').
+ *   mu N x 3, frame N int32 in [0, n_frames), q_can N x 4, logs_can N x 3,
+ *   sh_can N x 48 (all fp32).
+ */
+int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                        int64_t N, const float* planes, const float* weights,
+                        const float* q_can, const float* logs_can, const float* sh_can,
+                        spin4d_hex_outputs out, spin4d_stream_t stream);
+
+size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N);
+
+/* Backward of spin4d_hexplane_fwd: grad_planes += , grad_weights += (fp32). */
+int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                        int64_t N, const float* planes, const float* weights,
+                        const float* q_can, const float* logs_can, const float* sh_can,
+                        const spin4d_hex_output_grads* grad_out,
+                        float* grad_planes, float* grad_weights,
+                        void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
+ * Test hook: the interpolation cell of every position at every level, as the
+ * kernels compute it.  idx N x L x 16 uint32 (corner c selects vertex
+ * base_d + bit d of c, d = 0 x, 1 y, 2 z, 3 t); frac N x L x 4 fp32
+ * (position inside the cell, per axis).
+ */
+int spin4d_debug_corners(const spin4d_grid_desc* g, const float* pos, int64_t N,
+                         uint32_t* idx, float* frac, spin4d_stream_t stream);
+
+/* Static string for a status code. */
+const char* spin4d_status_string(int status);
+/* cudaError_t of the last SPIN4D_ERR_CUDA returned on this thread (0 if none). */
+int spin4d_last_cuda_error(void);
+/* Library version, e.g. "0.1.0". */
+const char* spin4d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPIN4D_H */

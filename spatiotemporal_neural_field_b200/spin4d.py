@@ -1,0 +1,282 @@
+"""Thin ctypes binding of ``libspin4d.so`` (declared in ``include/spin4d.h``).
+
+Argument marshalling only: every step of the decoder runs in the library's
+CUDA kernels.  torch is used for device memory and the current stream.  If
+the library is missing the import fails loudly; there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspin4d.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError("libspin4d.so is not built (run `python -m spatiotemporal_neural_field_b200.build` "
+                      "or __graft_entry__.build()); spin4d has no CPU fallback")
+lib = ctypes.CDLL(_LIB_PATH)
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_INJECTED = 0, -1, -2, -3, -4, -5
+F32, F16 = 0, 1
+INPUT_NORMALISED = 1
+MAX_LEVELS = 16
+HEAD_ROWS = 11
+
+c_i32, c_i64, c_f32, c_u32, c_vp, c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_uint32,
+                                          ctypes.c_void_p, ctypes.c_size_t)
+
+
+class GridDesc(ctypes.Structure):
+    _fields_ = [("L", c_i32), ("F", c_i32), ("log2_T", c_i32), ("table_dtype", c_i32),
+                ("res", (c_i32 * 4) * MAX_LEVELS), ("t_min", c_f32), ("t_max", c_f32),
+                ("flags", c_u32), ("reserved", c_i32)]
+
+    def resolutions(self):
+        return [[self.res[l][d] for d in range(4)] for l in range(self.L)]
+
+
+class MlpDesc(ctypes.Structure):
+    _fields_ = [("in_dim", c_i32), ("hidden", c_i32), ("n_hidden", c_i32), ("w_dtype", c_i32),
+                ("gate", c_i32), ("tau", c_f32)]
+
+
+class Outputs(ctypes.Structure):
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("rgb", c_vp), ("opacity", c_vp), ("cov", c_vp)]
+
+
+class OutputGrads(ctypes.Structure):
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("rgb", c_vp), ("opacity", c_vp), ("cov", c_vp)]
+
+
+class HexDesc(ctypes.Structure):
+    _fields_ = [("n_scales", c_i32), ("scales", c_i32 * 4), ("time_res", c_i32), ("channels", c_i32),
+                ("n_frames", c_i32), ("hidden", c_i32), ("n_hidden", c_i32)]
+
+
+class HexOutputs(ctypes.Structure):
+    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp)]
+
+
+class HexOutputGrads(ctypes.Structure):
+    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp)]
+
+
+P = ctypes.POINTER
+_SIGS = {
+    "spin4d_grid_init": (c_i32, [P(GridDesc), c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_f32, c_f32]),
+    "spin4d_mlp_param_count": (c_i64, [P(MlpDesc)]),
+    "spin4d_encode_fwd": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
+    "spin4d_decode_fwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, Outputs, c_vp]),
+    "spin4d_decode_bwd_workspace": (c_sz, [P(GridDesc), P(MlpDesc), c_i64]),
+    "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, P(OutputGrads),
+                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "spin4d_adam_step": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i32, c_f32, c_f32, c_f32, c_f32, c_i32,
+                                 c_vp, c_vp]),
+    "spin4d_hexplane_plane_count": (c_i64, [P(HexDesc)]),
+    "spin4d_hexplane_param_count": (c_i64, [P(HexDesc)]),
+    "spin4d_hexplane_fwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, HexOutputs, c_vp]),
+    "spin4d_hexplane_bwd_workspace": (c_sz, [P(HexDesc), c_i64]),
+    "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                    P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_debug_corners": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
+    "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
+    "spin4d_last_cuda_error": (c_i32, []),
+    "spin4d_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class Spin4dError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        msg = lib.spin4d_status_string(status).decode()
+        if status == ERR_CUDA:
+            msg += " (cudaError %d)" % lib.spin4d_last_cuda_error()
+        super().__init__("%s failed: %s [%d]" % (call, msg, status))
+        self.status = status
+
+
+def _check(call: str, status: int) -> None:
+    if status != OK:
+        raise Spin4dError(call, status)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+_DT = {"f32": F32, "f16": F16, torch.float32: F32, torch.float16: F16}
+
+
+# ---------------------------------------------------------------------------
+# Descriptors
+# ---------------------------------------------------------------------------
+def grid_desc(L: int, F: int, log2_T: int, dtype, nmin_s: int, nmax_s: int, nmin_t: int, nmax_t: int,
+              t_min: float, t_max: float, normalised_input: bool = False) -> GridDesc:
+    g = GridDesc()
+    _check("spin4d_grid_init", lib.spin4d_grid_init(ctypes.byref(g), L, F, log2_T, _DT[dtype], nmin_s, nmax_s,
+                                                    nmin_t, nmax_t, t_min, t_max))
+    if normalised_input:
+        g.flags |= INPUT_NORMALISED
+    return g
+
+
+def grid_from_spec(spec, normalised_input: bool = False) -> GridDesc:
+    return grid_desc(spec.L, spec.F, spec.log2_T, spec.dtype, spec.nmin_s, spec.nmax_s, spec.nmin_t,
+                     spec.nmax_t, spec.t_min, spec.t_max, normalised_input)
+
+
+def mlp_desc(in_dim: int, hidden: int, n_hidden: int, dtype, gate: bool = False, tau: float = 0.02) -> MlpDesc:
+    return MlpDesc(in_dim, hidden, n_hidden, _DT[dtype], 1 if gate else 0, tau)
+
+
+def mlp_from_spec(spec) -> MlpDesc:
+    return mlp_desc(spec.in_dim, spec.hidden, spec.n_hidden, spec.dtype, spec.gate, spec.tau)
+
+
+def mlp_param_count(m: MlpDesc) -> int:
+    return int(lib.spin4d_mlp_param_count(ctypes.byref(m)))
+
+
+def hex_desc(scales=(64, 128, 256), time_res: int = 75, channels: int = 32, n_frames: int = 150,
+             hidden: int = 64, n_hidden: int = 2) -> HexDesc:
+    h = HexDesc()
+    h.n_scales = len(scales)
+    for i, s in enumerate(scales):
+        h.scales[i] = s
+    h.time_res, h.channels, h.n_frames, h.hidden, h.n_hidden = time_res, channels, n_frames, hidden, n_hidden
+    return h
+
+
+def hex_from_spec(spec) -> HexDesc:
+    return hex_desc(spec.scales, spec.time_res, spec.channels, spec.n_frames, spec.hidden, spec.n_hidden)
+
+
+# ---------------------------------------------------------------------------
+# Calls
+# ---------------------------------------------------------------------------
+def encode_fwd(g: GridDesc, pos: torch.Tensor, tables: torch.Tensor, z: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    N = pos.shape[0]
+    if z is None:
+        z = torch.empty((N, g.L * g.F), dtype=torch.float32, device=pos.device)
+    _check("spin4d_encode_fwd", lib.spin4d_encode_fwd(ctypes.byref(g), _ptr(pos), N, _ptr(tables), _ptr(z),
+                                                      _stream(stream)))
+    return z
+
+
+def alloc_outputs(N: int, device) -> Dict[str, torch.Tensor]:
+    return {k: torch.empty((N, w), dtype=torch.float32, device=device)
+            for k, w in (("scale", 3), ("rot", 4), ("rgb", 3), ("opacity", 1), ("cov", 6))}
+
+
+def decode_fwd(g: GridDesc, m: MlpDesc, pos: torch.Tensor, tables: torch.Tensor, weights: torch.Tensor,
+               gate_cr: Optional[torch.Tensor] = None, out: Optional[Dict[str, torch.Tensor]] = None,
+               stream=None) -> Dict[str, torch.Tensor]:
+    N = pos.shape[0]
+    if out is None:
+        out = alloc_outputs(N, pos.device)
+    o = Outputs(*(_ptr(out[k]) for k in ("scale", "rot", "rgb", "opacity", "cov")))
+    _check("spin4d_decode_fwd", lib.spin4d_decode_fwd(ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables),
+                                                      _ptr(weights), _ptr(gate_cr), o, _stream(stream)))
+    return out
+
+
+def decode_bwd_workspace(g: GridDesc, m: MlpDesc, N: int) -> int:
+    return int(lib.spin4d_decode_bwd_workspace(ctypes.byref(g), ctypes.byref(m), N))
+
+
+def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
+               grad_tables: torch.Tensor, grad_weights: torch.Tensor, gate_cr=None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    N = pos.shape[0]
+    need = decode_bwd_workspace(g, m, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
+    go = OutputGrads(*(_ptr(grads.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov")))
+    _check("spin4d_decode_bwd", lib.spin4d_decode_bwd(ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables),
+                                                      _ptr(weights), _ptr(gate_cr), ctypes.byref(go),
+                                                      _ptr(grad_tables), _ptr(grad_weights), _ptr(workspace),
+                                                      workspace.numel(), _stream(stream)))
+
+
+def cov_assemble(scale: torch.Tensor, rot: torch.Tensor, cov: Optional[torch.Tensor] = None, stream=None):
+    N = scale.shape[0]
+    if cov is None:
+        cov = torch.empty((N, 6), dtype=torch.float32, device=scale.device)
+    _check("spin4d_cov_assemble", lib.spin4d_cov_assemble(_ptr(scale), _ptr(rot), N, _ptr(cov), _stream(stream)))
+    return cov
+
+
+def adam_step(params, grad, m, v, step: int, lr: float, b1: float, b2: float, eps: float,
+              params_work: Optional[torch.Tensor] = None, zero_grad: bool = False,
+              nonfinite_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check("spin4d_adam_step", lib.spin4d_adam_step(_ptr(params), _ptr(params_work), _ptr(grad), _ptr(m), _ptr(v),
+                                                    params.numel(), step, lr, b1, b2, eps, 1 if zero_grad else 0,
+                                                    _ptr(nonfinite_flag), _stream(stream)))
+
+
+def hexplane_plane_count(h: HexDesc) -> int:
+    return int(lib.spin4d_hexplane_plane_count(ctypes.byref(h)))
+
+
+def hexplane_param_count(h: HexDesc) -> int:
+    return int(lib.spin4d_hexplane_param_count(ctypes.byref(h)))
+
+
+HEX_KEYS = (("mu", 3), ("rot", 4), ("scale", 3), ("sh", 48), ("cov", 6))
+
+
+def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=None, stream=None):
+    N = inp["mu"].shape[0]
+    if out is None:
+        out = {k: torch.empty((N, w), dtype=torch.float32, device=planes.device) for k, w in HEX_KEYS}
+    o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS))
+    _check("spin4d_hexplane_fwd", lib.spin4d_hexplane_fwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
+                                                          _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
+                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), o,
+                                                          _stream(stream)))
+    return out
+
+
+def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, stream=None):
+    N = inp["mu"].shape[0]
+    need = int(lib.spin4d_hexplane_bwd_workspace(ctypes.byref(h), N))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=planes.device)
+    go = HexOutputGrads(*(_ptr(grads.get(k)) for k, _ in HEX_KEYS))
+    _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
+                                                          _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
+                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]),
+                                                          ctypes.byref(go), _ptr(grad_planes), _ptr(grad_weights),
+                                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def debug_corners(g: GridDesc, pos: torch.Tensor, stream=None):
+    N = pos.shape[0]
+    idx = torch.empty((N, g.L, 16), dtype=torch.int32, device=pos.device)
+    frac = torch.empty((N, g.L, 4), dtype=torch.float32, device=pos.device)
+    _check("spin4d_debug_corners", lib.spin4d_debug_corners(ctypes.byref(g), _ptr(pos), N, _ptr(idx), _ptr(frac),
+                                                            _stream(stream)))
+    return idx, frac
+
+
+def version() -> str:
+    return lib.spin4d_version().decode()

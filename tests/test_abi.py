@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the header declares, computes the same host-side grid constants as the
+oracle, rejects bad arguments before any launch, and honours the host
+fault-injection hook."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spin4d.h")
+
+
+@pytest.fixture(scope="module")
+def sp():
+    from spatiotemporal_neural_field_b200 import build
+    build.build()
+    from spatiotemporal_neural_field_b200 import spin4d
+    return spin4d
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(spin4d_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(sp):
+    names = declared_functions()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(sp.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", sp._LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (spin4d_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(sp.EXPORTED) == set(names)
+
+
+def test_grid_init_matches_oracle_resolutions(sp):
+    from oracle import hashgrid as hg
+    from spatiotemporal_neural_field_b200 import synthetic as S
+    for spec in (S.GRID_TINY, S.GRID_SPORTS, S.GRID_STRESS):
+        g = sp.grid_from_spec(spec)
+        want = hg.grid_resolutions(spec.L, spec.nmin_s, spec.nmax_s, spec.nmin_t, spec.nmax_t)
+        assert np.array_equal(np.array(g.resolutions()), want)
+        assert g.L == spec.L and g.F == spec.F and g.log2_T == spec.log2_T
+
+
+def test_param_counts(sp):
+    from spatiotemporal_neural_field_b200 import synthetic as S
+    for spec in (S.MLP_TINY, S.MLP_SPORTS, S.MLP_STRESS):
+        assert sp.mlp_param_count(sp.mlp_from_spec(spec)) == spec.n_params()
+        assert S.mlp_weights(spec).size == spec.n_params()
+    h = sp.hex_from_spec(S.HEX)
+    assert sp.hexplane_plane_count(h) == S.HEX.n_plane_floats()
+    assert sp.hexplane_param_count(h) == S.HEX.n_params()
+
+
+FAKE = 1 << 20      # 16-byte aligned, never dereferenced: every call below returns before a launch
+
+
+def _outs(sp):
+    return sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE)
+
+
+def test_invalid_arguments_rejected_on_host(sp):
+    from spatiotemporal_neural_field_b200 import synthetic as S
+    lib = sp.lib
+    g = sp.grid_from_spec(S.GRID_SPORTS)
+    m = sp.mlp_from_spec(S.MLP_SPORTS)
+    ref = ctypes.byref
+    # negative N, null and misaligned pointers
+    assert lib.spin4d_decode_fwd(ref(g), ref(m), FAKE, -1, FAKE, FAKE, None, _outs(sp), None) == sp.ERR_INVALID
+    assert lib.spin4d_decode_fwd(ref(g), ref(m), None, 10, FAKE, FAKE, None, _outs(sp), None) == sp.ERR_INVALID
+    assert lib.spin4d_decode_fwd(ref(g), ref(m), FAKE + 4, 10, FAKE, FAKE, None, _outs(sp), None) == sp.ERR_INVALID
+    assert lib.spin4d_encode_fwd(ref(g), FAKE, 10, FAKE + 2, FAKE, None) == sp.ERR_INVALID
+    # N == 0 is a valid no-op
+    assert lib.spin4d_decode_fwd(ref(g), ref(m), None, 0, None, None, None, sp.Outputs(), None) == sp.OK
+    assert lib.spin4d_encode_fwd(ref(g), None, 0, None, None, None) == sp.OK
+    # descriptor errors
+    bad = sp.grid_from_spec(S.GRID_SPORTS)
+    bad.F = 3
+    assert lib.spin4d_encode_fwd(ref(bad), FAKE, 10, FAKE, FAKE, None) == sp.ERR_INVALID
+    bad = sp.grid_from_spec(S.GRID_SPORTS)
+    bad.res[2][1] = 1
+    assert lib.spin4d_encode_fwd(ref(bad), FAKE, 10, FAKE, FAKE, None) == sp.ERR_INVALID
+    bad = sp.grid_from_spec(S.GRID_SPORTS)
+    bad.t_max = bad.t_min
+    assert lib.spin4d_encode_fwd(ref(bad), FAKE, 10, FAKE, FAKE, None) == sp.ERR_INVALID
+    m2 = sp.mlp_from_spec(S.MLP_SPORTS)
+    m2.in_dim = 31                         # must equal L*F
+    assert lib.spin4d_decode_fwd(ref(g), ref(m2), FAKE, 10, FAKE, FAKE, None, _outs(sp), None) == sp.ERR_INVALID
+    m3 = sp.mlp_desc(32, 64, 2, "f16", gate=True, tau=0.02)
+    assert lib.spin4d_decode_fwd(ref(g), ref(m3), FAKE, 10, FAKE, FAKE, None, _outs(sp), None) == sp.ERR_INVALID
+    m4 = sp.mlp_desc(32, 64, 2, "f16", gate=True, tau=0.0)
+    assert lib.spin4d_decode_fwd(ref(g), ref(m4), FAKE, 10, FAKE, FAKE, FAKE, _outs(sp), None) == sp.ERR_INVALID
+    # bwd: too small a workspace
+    go = sp.OutputGrads()
+    assert lib.spin4d_decode_bwd(ref(g), ref(m), FAKE, 1000, FAKE, FAKE, None, ref(go), FAKE, FAKE, FAKE, 16,
+                                 None) == sp.ERR_INVALID
+    # adam
+    assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 0, 1e-3, 0.9, 0.99, 1e-15, 0, None,
+                                None) == sp.ERR_INVALID
+    assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 1, 1e-3, 1.0, 0.99, 1e-15, 0, None,
+                                None) == sp.ERR_INVALID
+    assert lib.spin4d_grid_init(None, 4, 2, 12, 0, 4, 32, 4, 32, 0.0, 1.0) == sp.ERR_INVALID
+    assert sp.lib.spin4d_status_string(sp.ERR_INVALID) == b"invalid argument"
+
+
+def test_unsupported_hexplane_shape(sp):
+    lib = sp.lib
+    h = sp.hex_desc(channels=16)
+    inp = [FAKE] * 2
+    assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE), None) == sp.ERR_UNSUPPORTED
+
+
+def test_fault_injection_hook_in_subprocess(sp):
+    code = r"""
+import ctypes, sys
+sys.path.insert(0, %r)
+from spatiotemporal_neural_field_b200 import spin4d as sp, synthetic as S
+g = sp.grid_from_spec(S.GRID_SPORTS); m = sp.mlp_from_spec(S.MLP_SPORTS)
+F = 1 << 20
+r1 = sp.lib.spin4d_decode_fwd(ctypes.byref(g), ctypes.byref(m), F, 10, F, F, None, sp.Outputs(F, F, F, F, F), None)
+r2 = sp.lib.spin4d_encode_fwd(ctypes.byref(g), F, -1, F, F, None)
+print(r1, r2)
+""" % ROOT
+    env = dict(os.environ, SPIN4D_FAULT="spin4d_decode_fwd")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, timeout=300)
+    assert out.returncode == 0, out.stderr
+    r1, r2 = map(int, out.stdout.split())
+    assert r1 == -5          # injected after validation, before any launch
+    assert r2 == -1          # other entry points unaffected (still validated)

@@ -46,6 +46,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fwd-bwd", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=150_000, help="positions the oracle decodes for cpu_baseline")
+    p.add_argument("--no-probe", action="store_true", help="skip the random-gather ceiling measurement")
+    p.add_argument("--ncu-case", default=None,
+                   help="profiling driver: run a few untimed launches of one workload and exit "
+                        "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32)")
     return p.parse_args()
 
 
@@ -78,11 +82,14 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+DECODE_SOURCES = ("decode_tc.cu", "common.cuh", "tc.cuh")
+
+
+def kernel_source_hash(files=DECODE_SOURCES):
+    """Hash of the sources the timed decode kernel is built from."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(KERNEL_SRC)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(KERNEL_SRC, f), "rb").read())
+    for f in files:
+        h.update(open(os.path.join(KERNEL_SRC, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -137,6 +144,39 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def table_sectors_per_position(sp, g, pos_dev, F, elem_bytes, sample=20_000):
+    """Distinct 32-byte table sectors one position touches (all levels), from
+    the kernel's own corner indices: the minimum sector traffic of a position
+    when no other position shares its sectors."""
+    idx, _ = sp.debug_corners(g, pos_dev[:sample].contiguous())
+    idx = idx.cpu().numpy().view(np.uint32).astype(np.int64)
+    sec = np.sort((idx * F * elem_bytes) >> 5, axis=2)
+    distinct = 1 + np.count_nonzero(np.diff(sec, axis=2), axis=2)
+    return float(distinct.sum(axis=1).mean())
+
+
+def probe_sector_rates(sp, torch, dev):
+    """Random 16-byte loads (one sector each) from a 32 MiB L2-resident buffer
+    and from a 4 GiB buffer (HBM): the gather ceilings, sectors/s."""
+    out = {}
+    blocks = 4 * torch.cuda.get_device_properties(dev).multi_processor_count
+    for name, nbytes, lpt in (("l2", 32 << 20, 4096), ("hbm", 4 << 30, 1024)):
+        buf = torch.ones(nbytes // 4, dtype=torch.int32, device=dev)
+        best = None
+        for it in range(4):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            n = sp.probe_gather(buf, 16, lpt, blocks, seed=it + 1)
+            b.record()
+            torch.cuda.synchronize()
+            if it:
+                rate = n / (a.elapsed_time(b) * 1e-3)
+                best = rate if best is None else max(best, rate)
+        out[name] = best
+        del buf
+    return out
 
 
 def cpu_baseline(n_sample):
@@ -313,6 +353,18 @@ def run_ours(args):
                    (float(tb.item()) * 1e-3), "unit": UNIT, "ms_per_step": float(tb.item()) / k,
                    "workload": "sports_train_fp16: one 1M-position launch (frames 0-3), decode_fwd + decode_bwd"}
 
+    gather = None
+    if not args.no_probe:
+        rates = probe_sector_rates(sp, torch, dev)
+        spp = table_sectors_per_position(sp, g, pos, grid.F, 2)
+        dec_rate = spp * value / world
+        gather = {"table_sectors_per_position": spp,
+                  "decoder_sector_rate": dec_rate,
+                  "l2_random_sector_rate": rates["l2"], "hbm_random_sector_rate": rates["hbm"],
+                  "frac_of_l2_random": dec_rate / rates["l2"], "unit": "sectors/s per GPU",
+                  "note": "tables (32 MiB) are L2-resident: the gather ceiling is the measured random "
+                          "32-byte-sector rate of an L2-resident buffer (spin4d_probe_gather)"}
+
     if rank == 0:
         peak, peak_kind = measured_peaks()
         bpp = algorithmic_bytes_per_position()
@@ -331,6 +383,8 @@ def run_ours(args):
         }
         if fwd_bwd:
             line["fwd_bwd"] = fwd_bwd
+        if gather:
+            line["gather_roofline"] = gather
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.cpu_sample)
         print(json.dumps(line), flush=True)
@@ -339,8 +393,66 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_ncu_case(name):
+    """A few untimed launches of one workload, for an ncu capture."""
+    import torch
+    from spatiotemporal_neural_field_b200 import build as _b
+    _b.build()
+    from spatiotemporal_neural_field_b200 import spin4d as sp
+    dev = torch.device("cuda", 0)
+    w = S.WORKLOADS[name]
+    if name == "hexplane_fp32":
+        hx = w["hex"]
+        n = w["N"]
+        inp = {k: torch.from_numpy(v).to(dev) for k, v in S.hexplane_inputs(n).items()}
+        planes = torch.from_numpy(S.hexplane_planes(hx)).to(dev)
+        weights = torch.from_numpy(S.hexplane_weights(hx)).to(dev)
+        h = sp.hex_from_spec(hx)
+        grads = {k: torch.randn((n, wd), device=dev) for k, wd in S.HEX_OUT_WIDTHS.items()}
+        gp = torch.zeros(hx.n_plane_floats(), device=dev)
+        gw = torch.zeros(hx.n_params(), device=dev)
+        for _ in range(3):
+            sp.hexplane_fwd(h, inp, planes, weights)
+            sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw)
+    else:
+        grid, mlp = w["grid"], w["mlp"]
+        g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+        if name == "stress_fp16_gate":
+            n = w["N"]
+            pos = S.stress_positions(n)
+        elif name == "sports_train_fp16":
+            n = w["batch"]
+            pos = S.sports_scene(300_000).frames(range(4))[:n]
+        elif name == "tiny_fp32":
+            n = w["N"]
+            pos = S.uniform_positions(n)
+        else:
+            n = w["N"]
+            pos = S.sports_scene(n).frame(w["frame"])
+        P = torch.from_numpy(pos).to(dev)
+        T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+        W = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
+        cr = torch.from_numpy(S.gate_params(n)).to(dev) if mlp.gate else None
+        out = sp.alloc_outputs(n, dev)
+        bwd = name in ("sports_train_fp16", "tiny_fp32")
+        if bwd:
+            grads = {k: torch.randn((n, wd), device=dev) * 1e-2 for k, wd in OUT_WIDTHS.items()}
+            gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
+            gw = torch.zeros(mlp.n_params(), device=dev)
+        for _ in range(3):
+            sp.decode_fwd(g, m, P, T, W, cr, out=out)
+            if bwd:
+                sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr)
+    torch.cuda.synchronize()
+    sp.check_device_errors()
+    print("ncu case done:", name)
+
+
 def main():
     args = parse()
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

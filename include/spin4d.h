@@ -52,7 +52,8 @@ typedef enum spin4d_status {
     SPIN4D_ERR_UNSUPPORTED = -2,  /* valid but not implemented shape; nothing launched */
     SPIN4D_ERR_CUDA = -3,         /* a CUDA launch or query failed */
     SPIN4D_ERR_NONFINITE = -4,    /* a kernel met a non-finite value (see spin4d_adam_step) */
-    SPIN4D_ERR_INJECTED = -5      /* SPIN4D_FAULT selected this call */
+    SPIN4D_ERR_INJECTED = -5,     /* SPIN4D_FAULT selected this call */
+    SPIN4D_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out (see spin4d_check_device_errors) */
 } spin4d_status;
 
 typedef enum spin4d_dtype { SPIN4D_F32 = 0, SPIN4D_F16 = 1 } spin4d_dtype;
@@ -275,6 +276,28 @@ int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const in
  */
 int spin4d_debug_corners(const spin4d_grid_desc* g, const float* pos, int64_t N,
                          uint32_t* idx, float* frac, spin4d_stream_t stream);
+
+/*
+ * Synchronous: reads the library's device error word, set by a kernel whose
+ * bounded wait for its own tensor-core work ran out (the kernel then frees
+ * its tensor memory and exits early, leaving its outputs incomplete).
+ * Returns SPIN4D_OK or SPIN4D_ERR_TIMEOUT; clear != 0 resets the word.
+ * Waits for the current device's legacy default stream.
+ */
+int spin4d_check_device_errors(int clear);
+
+/*
+ * Measurement helper (not part of the decoder): the gather-rate ceiling.
+ * Launches `blocks` x 256 threads; each issues `loads_per_thread` (a multiple
+ * of 8) independent loads of `width` bytes (4 or 16) at pseudo-random,
+ * width-aligned offsets of `buf` (device, 16-byte aligned, `buf_bytes` long),
+ * eight in flight per thread.  Every load touches exactly one 32-byte sector,
+ * so loads / elapsed time is the random-sector rate of wherever `buf` lives:
+ * L2 for a buffer well under the L2 size, HBM for one far above it.
+ * `sink` (device, 4 bytes) is written only to keep the loads alive.
+ */
+int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t loads_per_thread, int blocks,
+                        uint32_t seed, uint32_t* sink, spin4d_stream_t stream);
 
 /* Static string for a status code. */
 const char* spin4d_status_string(int status);

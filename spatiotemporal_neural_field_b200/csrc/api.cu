@@ -195,6 +195,7 @@ const char* spin4d_status_string(int s) {
     case SPIN4D_ERR_CUDA: return "CUDA error";
     case SPIN4D_ERR_NONFINITE: return "non-finite value";
     case SPIN4D_ERR_INJECTED: return "injected fault";
+    case SPIN4D_ERR_TIMEOUT: return "device wait timed out";
     default: return "unknown status";
   }
 }

@@ -182,6 +182,72 @@ __device__ __forceinline__ void encode_level(const float xt[4], const GridParams
     for (int f = 0; f < F; ++f) acc[f] = fmaf(w[c], v[c][f], acc[f]);
 }
 
+// Encode one level of an fp16 table, x-neighbours paired: corners c (x bit 0)
+// and c+1 (x bit 1) usually fall in the same 16-byte group of G = 8/F entries
+// (dense levels: consecutive entries; hashed levels: x enters the hash with
+// prime 1, so x and x+1 differ only in the low bits unless a carry crosses
+// the group).  One 16-byte load then serves both corners; only lanes whose
+// pair straddles two groups issue a second load.  Four pairs per batch bound
+// the registers held by loads in flight.
+template <int F>
+__device__ __forceinline__ uint32_t group_word(const uint4& v, uint32_t i) {
+  // word holding entry i of the group (F = 2: one word per entry)
+  return (i & 2u) ? ((i & 1u) ? v.w : v.z) : ((i & 1u) ? v.y : v.x);
+}
+
+template <int F>
+__device__ __forceinline__ void accumulate_entry(const uint4& v, uint32_t i, float wgt, float acc[F]) {
+  if constexpr (F == 2) {
+    uint32_t u = group_word<F>(v, i);
+    float2 a = __half22float2(*reinterpret_cast<__half2*>(&u));
+    acc[0] = fmaf(wgt, a.x, acc[0]);
+    acc[1] = fmaf(wgt, a.y, acc[1]);
+  } else if constexpr (F == 4) {
+    uint32_t u0 = (i & 1u) ? v.z : v.x, u1 = (i & 1u) ? v.w : v.y;
+    float2 a = __half22float2(*reinterpret_cast<__half2*>(&u0));
+    float2 b = __half22float2(*reinterpret_cast<__half2*>(&u1));
+    acc[0] = fmaf(wgt, a.x, acc[0]);
+    acc[1] = fmaf(wgt, a.y, acc[1]);
+    acc[2] = fmaf(wgt, b.x, acc[2]);
+    acc[3] = fmaf(wgt, b.y, acc[3]);
+  }
+}
+
+template <int F>
+__device__ __forceinline__ void encode_level_f16_paired(const float xt[4], const GridParams& g, int l,
+                                                        const __half* __restrict__ tables, float acc[F]) {
+  static_assert(F == 2 || F == 4, "paired gather covers F = 2 and 4");
+  constexpr uint32_t G = 8 / F;   // entries per 16-byte group
+  uint32_t base[4];
+  float frac[4];
+  level_cell(xt, g, l, base, frac);
+  uint32_t idx[16];
+  level_indices(base, g, l, idx);
+  float w[16];
+  level_weights(frac, w);
+  const uint4* tab = reinterpret_cast<const uint4*>(tables + ((size_t)l << g.log2_T) * F);
+#pragma unroll
+  for (int f = 0; f < F; ++f) acc[f] = 0.0f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint4 v0[4], v1[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int c = 2 * (4 * b + p);
+      const uint32_t g0 = idx[c] / G, g1 = idx[c + 1] / G;
+      v0[p] = __ldg(tab + g0);
+      v1[p] = v0[p];
+      if (g1 != g0) v1[p] = __ldg(tab + g1);
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int c = 2 * (4 * b + p);
+      accumulate_entry<F>(v0[p], idx[c] % G, w[c], acc);
+      accumulate_entry<F>(v1[p], idx[c + 1] % G, w[c + 1], acc);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Scatter-add of the adjoint: grad_l[idx_c][f] += w_c * dz[f]  (fp32 atomics).
 // ---------------------------------------------------------------------------
@@ -350,6 +416,11 @@ __device__ __forceinline__ void heads_backward(const float y[kHeadRows], float g
   float so = sigmoidf_(y[10]);
   dy[10] = g.o * gate * so * (1.0f - so);
 }
+
+// Floats between consecutive per-block slots of a weight-gradient workspace:
+// n rounded up to a multiple of 4 so every slot starts 16-byte aligned (the
+// slots are updated with vector accesses).
+__host__ __device__ __forceinline__ size_t slot_stride(int n) { return ((size_t)n + 3) & ~(size_t)3; }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }

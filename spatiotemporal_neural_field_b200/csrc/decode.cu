@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
   float* dB = dA + maxw * kBwdBlock;
   float* dy_s = dB + maxw * kBwdBlock;
   const int col = threadIdx.x;
-  float* slot = ws + (size_t)blockIdx.x * n_params;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
   for (int p = threadIdx.x; p < n_params; p += blockDim.x) slot[p] = 0.0f;
 
   // offsets of each layer's packed parameters
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
 __global__ void reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
     float s = 0.0f;
-    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * n_params + p];
+    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * slot_stride(n_params) + p];
     out[p] += s;
   }
 }
@@ -364,6 +364,18 @@ static MlpParams make_mlp(const spin4d_mlp_desc* m) {
 int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                   const void* tables, const void* weights, const float* gate_cr, const spin4d_outputs& out,
                   cudaStream_t s, bool* handled);
+// Tensor-core fused backward (decode_bwd_tc.cu): CTAs per SM, 0 when the shape is not covered.
+int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* m);
+int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
+                  const void* tables, const void* weights, const float* gate_cr, const spin4d_output_grads* go,
+                  float* grad_tables, float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s);
+
+// Thread blocks (= workspace slots) the backward launches for N positions.
+static int bwd_slots(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, int64_t N) {
+  const int c = decode_bwd_tc_ctas_per_sm(g, m);
+  if (c > 0) return persistent_blocks((N + 127) / 128, c);
+  return bwd_blocks(N);
+}
 
 }  // namespace spin4d
 
@@ -389,7 +401,7 @@ extern "C" int spin4d_decode_fwd(const spin4d_grid_desc* g, const spin4d_mlp_des
 
 extern "C" size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, int64_t N) {
   if (validate_grid(g) != SPIN4D_OK || validate_mlp(g, m) != SPIN4D_OK || N <= 0) return 0;
-  return (size_t)bwd_blocks(N) * (size_t)spin4d_mlp_param_count(m) * sizeof(float);
+  return (size_t)bwd_slots(g, m, N) * slot_stride((int)spin4d_mlp_param_count(m)) * sizeof(float);
 }
 
 extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
@@ -403,10 +415,20 @@ extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_des
     return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_decode_bwd_workspace(g, m, N)) return SPIN4D_ERR_INVALID;
   if (grad_out->rot && !aligned(grad_out->rot, 4)) return SPIN4D_ERR_INVALID;
-  if (bwd_smem(m) > 220 * 1024) return SPIN4D_ERR_UNSUPPORTED;
+  const bool tc = decode_bwd_tc_ctas_per_sm(g, m) > 0;
+  if (!tc && bwd_smem(m) > 220 * 1024) return SPIN4D_ERR_UNSUPPORTED;
   if (fault_injected("spin4d_decode_bwd")) return SPIN4D_ERR_INJECTED;
-  GradPtrs go{grad_out->scale, grad_out->rot, grad_out->rgb, grad_out->opacity, grad_out->cov};
   int n_params = (int)spin4d_mlp_param_count(m);
+  if (tc) {
+    cudaStream_t s = (cudaStream_t)stream;
+    const int blocks = bwd_slots(g, m, N);
+    float* ws = static_cast<float*>(workspace);
+    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, grad_out, grad_tables, grad_weights, ws,
+                               n_params, blocks, s));
+    reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
+    return launch_status();
+  }
+  GradPtrs go{grad_out->scale, grad_out->rot, grad_out->rgb, grad_out->opacity, grad_out->cov};
   return dispatch<BwdFn>(g->table_dtype, g->F, m->w_dtype, make_grid_params(g), make_mlp(m), bwd_smem(m), pos,
                          N, tables, weights, gate_cr, go, grad_tables, grad_weights,
                          static_cast<float*>(workspace), n_params, (cudaStream_t)stream);

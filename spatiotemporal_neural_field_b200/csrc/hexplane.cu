@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kHexBwdBlock) hexplane_bwd_kernel(
   float* zc = d1b + kHexH * kHexBwdBlock;
   const int IN = hp.in_dim;
   const int col = threadIdx.x;
-  float* slot = ws + (size_t)blockIdx.x * n_params;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
   for (int p = threadIdx.x; p < n_params; p += blockDim.x) slot[p] = 0.0f;
   const float* W2 = W + kHexH * IN + kHexH;
   const float* W3 = head_weights(W, hp);
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kHexBwdBlock) hexplane_bwd_kernel(
 __global__ void hex_reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
     float s = 0.0f;
-    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * n_params + p];
+    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * slot_stride(n_params) + p];
     out[p] += s;
   }
 }
@@ -419,7 +419,7 @@ extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* m
 
 extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N) {
   if (validate_hex(h) != SPIN4D_OK || N <= 0) return 0;
-  return (size_t)hex_bwd_blocks(N) * (size_t)spin4d_hexplane_param_count(h) * sizeof(float);
+  return (size_t)hex_bwd_blocks(N) * slot_stride((int)spin4d_hexplane_param_count(h)) * sizeof(float);
 }
 
 extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,

@@ -18,7 +18,7 @@ if not os.path.exists(_LIB_PATH):
                       "or __graft_entry__.build()); spin4d has no CPU fallback")
 lib = ctypes.CDLL(_LIB_PATH)
 
-OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_INJECTED = 0, -1, -2, -3, -4, -5
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_INJECTED, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
 F32, F16 = 0, 1
 INPUT_NORMALISED = 1
 MAX_LEVELS = 16
@@ -82,6 +82,8 @@ _SIGS = {
     "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp,
                                     P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_debug_corners": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
+    "spin4d_check_device_errors": (c_i32, [c_i32]),
+    "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
     "spin4d_version": (ctypes.c_char_p, []),
@@ -276,6 +278,22 @@ def debug_corners(g: GridDesc, pos: torch.Tensor, stream=None):
     _check("spin4d_debug_corners", lib.spin4d_debug_corners(ctypes.byref(g), _ptr(pos), N, _ptr(idx), _ptr(frac),
                                                             _stream(stream)))
     return idx, frac
+
+
+def check_device_errors(clear: bool = True) -> None:
+    """Synchronous: raises if a kernel's bounded device wait ran out."""
+    _check("spin4d_check_device_errors", lib.spin4d_check_device_errors(1 if clear else 0))
+
+
+def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: int, seed: int = 1,
+                 sink: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Launches the random-gather probe; returns the number of loads issued."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    _check("spin4d_probe_gather", lib.spin4d_probe_gather(_ptr(buf), buf.numel() * buf.element_size(), width,
+                                                          loads_per_thread, blocks, seed, _ptr(sink),
+                                                          _stream(stream)))
+    return blocks * 256 * loads_per_thread
 
 
 def version() -> str:

@@ -200,6 +200,8 @@ BWD_CASES = {
     "tiny_spec": ("tiny_fp32", 4096, 1e-4, 0.0, 1.0),
     "tiny_stress": ("tiny_fp32", 4099, 1.0, 0.5, 1.0),
     "sports": ("sports_frame_fp16", 20011, 1.0, 0.5, 1e-2),
+    # initial state: 1e-4 tables, so latent and activations are ~1e-5 (fp16-subnormal unless rescaled)
+    "sports_spec_init": ("sports_frame_fp16", 20011, 1e-4, 0.0, 1e-2),
     "stress_gate": ("stress_fp16_gate", 6007, 1.0, 0.5, 1.0),
 }
 
@@ -232,11 +234,30 @@ def test_decode_bwd_matches_oracle(sp, case):
     assert o == gw.size
 
 
+@pytest.mark.parametrize("name,n", [("sports_frame_fp16", 20011), ("stress_fp16_gate", 3001)])
+def test_decode_bwd_covariance_only_gradient(sp, name, n):
+    """Upstream gradient on Sigma alone: Sigma ~ s^2 ~ 1e-5, so the gradients
+    that reach the network are ~1e-7..1e-9, far below fp16's normal range."""
+    grid, mlp, pos, tables, weights, cr = _workload(name, n, 1.0, 0.5)
+    full = S.upstream_grads(n, S.DECODE_OUT_WIDTHS, 1e-2)
+    grads = {"cov": full["cov"]}
+    gt, gw = _bwd(sp, grid, mlp, pos, tables, weights, cr, grads)
+    zeros = {k: np.zeros_like(v) for k, v in full.items()}
+    zeros["cov"] = full["cov"]
+    wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, zeros, gate_cr=cr)
+    tol.normwise(gt, wt, tol.FP16_GRAD_RTOL, "grad_tables")
+    o = 0
+    for (out_d, in_d) in mlp.layer_shapes():
+        tol.normwise(gw[o:o + out_d * in_d], ww[o:o + out_d * in_d], tol.FP16_GRAD_RTOL, "dW %dx%d" % (out_d, in_d))
+        o += out_d * in_d + out_d
+
+
 def test_decode_bwd_null_upstream_means_zero(sp):
     """A NULL upstream pointer is a zero gradient: only rgb given."""
     grid, mlp, pos, tables, weights, _ = _workload("tiny_fp32", 1000, 1.0, 0.5)
     grads = S.upstream_grads(1000, {"rgb": 3}, 1.0)
     gt, gw = _bwd(sp, grid, mlp, pos, tables, weights, None, grads)
+    assert np.any(gt != 0)
     full = {k: np.zeros((1000, w), np.float32) for k, w in S.DECODE_OUT_WIDTHS.items()}
     full["rgb"] = grads["rgb"]
     wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, full)
@@ -264,8 +285,11 @@ def test_decode_bwd_accumulates_and_is_linear_at_full_batch(sp):
     gw2 = torch.zeros_like(gw)
     sp.decode_bwd(g, m, P[:h].contiguous(), T, W, {k: v[:h].contiguous() for k, v in G.items()}, gt2, gw2)
     sp.decode_bwd(g, m, P[h:].contiguous(), T, W, {k: v[h:].contiguous() for k, v in G.items()}, gt2, gw2)
-    tol.normwise(host(gt2), host(gt), 1e-5, "tables: halves vs whole")
-    tol.normwise(host(gw2), host(gw), 1e-5, "weights: halves vs whole")
+    # Same arithmetic per position; only the fp32 accumulation order differs
+    # (atomics, per-block weight slots).  A coarse-level entry receives up to
+    # K ~ 10^3 additions here, so the rounding bound is ~K * 2^-24 ~ 6e-5.
+    tol.normwise(host(gt2), host(gt), 1e-4, "tables: halves vs whole")
+    tol.normwise(host(gw2), host(gw), 1e-4, "weights: halves vs whole")
     # sampled oracle check: the head-bias gradient is a plain sum of dy over
     # positions; check it on a 4000-row subset launched alone
     rows = np.random.default_rng(2).choice(len(pos), 4000, replace=False)

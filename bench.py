@@ -326,14 +326,14 @@ def run_ours(args):
         pb = torch.from_numpy(scene.frames(range(0, 4))[:nb]).to(dev)
         gb = {k: torch.randn((nb, wd), device=dev, generator=torch.Generator(device=dev).manual_seed(rank))
               * wt["grad_std"] for k, wd in OUT_WIDTHS.items()}
-        outb = sp.alloc_outputs(nb, dev)
+        outb = sp.alloc_outputs(nb, dev, latent_dim=grid.L * grid.F)
         gtab = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), dtype=torch.float32, device=dev)
         gwt = torch.zeros(mlp.n_params(), dtype=torch.float32, device=dev)
         ws = torch.empty(max(sp.decode_bwd_workspace(g, m, nb), 1), dtype=torch.uint8, device=dev)
 
         def fb():
             sp.decode_fwd(g, m, pb, tables, weights, out=outb, stream=stream)
-            sp.decode_bwd(g, m, pb, tables, weights, gb, gtab, gwt, workspace=ws, stream=stream)
+            sp.decode_bwd(g, m, pb, tables, weights, gb, gtab, gwt, workspace=ws, latent=outb["latent"], stream=stream)
 
         for _ in range(max(3, args.warmup // 2)):
             fb()
@@ -351,7 +351,7 @@ def run_ours(args):
             dist.all_reduce(tb, op=dist.ReduceOp.MAX)
         fwd_bwd = {"metric": "decoded spatiotemporal positions/s (fwd+bwd)", "value": nb * world * k /
                    (float(tb.item()) * 1e-3), "unit": UNIT, "ms_per_step": float(tb.item()) / k,
-                   "workload": "sports_train_fp16: one 1M-position launch (frames 0-3), decode_fwd + decode_bwd"}
+                   "workload": "sports_train_fp16: one 1M-position launch (frames 0-3), decode_fwd (saving z) + decode_bwd (reading z)"}
 
     gather = None
     if not args.no_probe:
@@ -433,7 +433,7 @@ def run_ncu_case(name):
         T = torch.from_numpy(S.hash_tables(grid)).to(dev)
         W = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
         cr = torch.from_numpy(S.gate_params(n)).to(dev) if mlp.gate else None
-        out = sp.alloc_outputs(n, dev)
+        out = sp.alloc_outputs(n, dev, latent_dim=grid.L * grid.F)
         bwd = name in ("sports_train_fp16", "tiny_fp32")
         if bwd:
             grads = {k: torch.randn((n, wd), device=dev) * 1e-2 for k, wd in OUT_WIDTHS.items()}
@@ -442,7 +442,7 @@ def run_ncu_case(name):
         for _ in range(3):
             sp.decode_fwd(g, m, P, T, W, cr, out=out)
             if bwd:
-                sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr)
+                sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr, latent=out["latent"])
     torch.cuda.synchronize()
     sp.check_device_errors()
     print("ncu case done:", name)

@@ -122,13 +122,17 @@ int64_t spin4d_mlp_param_count(const spin4d_mlp_desc* m);
 
 /* Decoded attributes, structure of arrays, fp32, device memory:
  * scale N x 3, rot N x 4 (unit, (w,x,y,z)), rgb N x 3, opacity N x 1,
- * cov N x 6 packed (xx, xy, xz, yy, yz, zz).  None may be NULL. */
+ * cov N x 6 packed (xx, xy, xz, yy, yz, zz).  None of these may be NULL.
+ * latent (optional, may be NULL): N x (L*F) fp32, 16-byte aligned, receives
+ * the encoder output z (Eq. 9) so that a following spin4d_decode_bwd can
+ * read it instead of gathering the tables again. */
 typedef struct spin4d_outputs {
     float* scale;
     float* rot;
     float* rgb;
     float* opacity;
     float* cov;
+    float* latent;
 } spin4d_outputs;
 
 /* Upstream gradients on the decoded attributes, same shapes as spin4d_outputs.
@@ -168,7 +172,9 @@ size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const spin4d_mlp_d
 
 /*
  * Backward of spin4d_decode_fwd for loss = sum_k <grad_out.k, output_k>:
- * recomputes the forward, then accumulates
+ * recomputes the forward (from `latent`, the z that spin4d_decode_fwd saved
+ * for the same positions and tables, when it is not NULL; otherwise by
+ * gathering the tables again), then accumulates
  *   grad_tables   += dloss/dtables   (L x T x F fp32, scatter-added with atomics)
  *   grad_weights  += dloss/dweights  (packed like `weights`, fp32)
  * The gradient of s^ is zero where s^ > 20 (the clip); ReLU passes where its
@@ -178,7 +184,7 @@ size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const spin4d_mlp_d
  */
 int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                       const float* pos, int64_t N, const void* tables, const void* weights,
-                      const float* gate_cr, const spin4d_output_grads* grad_out,
+                      const float* gate_cr, const float* latent, const spin4d_output_grads* grad_out,
                       float* grad_tables, float* grad_weights,
                       void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 

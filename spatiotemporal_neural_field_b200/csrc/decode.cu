@@ -25,7 +25,7 @@ struct MlpParams {
 };
 
 struct OutPtrs {
-  float *scale, *rot, *rgb, *opacity, *cov;
+  float *scale, *rot, *rgb, *opacity, *cov, *latent;
 };
 struct GradPtrs {
   const float *scale, *rot, *rgb, *opacity, *cov;
@@ -81,6 +81,10 @@ __global__ void __launch_bounds__(kFwdBlock) decode_fwd_simt(GridParams g, MlpPa
       encode_level<T, F>(xt, g, l, tables, acc);
 #pragma unroll
       for (int f = 0; f < F; ++f) buf0[(l * F + f) * kFwdBlock + col] = acc[f];
+      if (out.latent) {
+#pragma unroll
+        for (int f = 0; f < F; ++f) out.latent[n * m.in_dim + l * F + f] = acc[f];
+      }
     }
     const W* wp = weights;
     float* cur = buf0;
@@ -140,7 +144,8 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
                                                              const float4* __restrict__ pos, int64_t N,
                                                              const T* __restrict__ tables,
                                                              const W* __restrict__ weights,
-                                                             const float2* __restrict__ gate_cr, GradPtrs go,
+                                                             const float2* __restrict__ gate_cr,
+                                                             const float* __restrict__ latent, GradPtrs go,
                                                              float* __restrict__ grad_tables,
                                                              float* __restrict__ ws, int n_params) {
   extern __shared__ float smem[];
@@ -172,11 +177,15 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
     // ---- forward, keeping every layer input ----
     if (valid) {
       normalise_position(pos[n], g, xt);
-      for (int l = 0; l < g.L; ++l) {
-        float acc[F];
-        encode_level<T, F>(xt, g, l, tables, acc);
+      if (latent) {
+        for (int k = 0; k < IN; ++k) acts[k * kBwdBlock + col] = __ldg(latent + n * IN + k);
+      } else {
+        for (int l = 0; l < g.L; ++l) {
+          float acc[F];
+          encode_level<T, F>(xt, g, l, tables, acc);
 #pragma unroll
-        for (int f = 0; f < F; ++f) acts[(l * F + f) * kBwdBlock + col] = acc[f];
+          for (int f = 0; f < F; ++f) acts[(l * F + f) * kBwdBlock + col] = acc[f];
+        }
       }
       int din = IN;
       float* cur = acts;
@@ -294,7 +303,7 @@ static int launch_fwd(const GridParams& gp, const MlpParams& mp, size_t smem, co
 
 template <typename T, int F, typename W>
 static int launch_bwd(const GridParams& gp, const MlpParams& mp, size_t smem, const float* pos, int64_t N,
-                      const void* tables, const void* weights, const float* gate_cr, GradPtrs go,
+                      const void* tables, const void* weights, const float* gate_cr, const float* latent, GradPtrs go,
                       float* grad_tables, float* grad_weights, float* ws, int n_params, cudaStream_t s) {
   auto k = decode_bwd_simt<T, F, W>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -302,7 +311,7 @@ static int launch_bwd(const GridParams& gp, const MlpParams& mp, size_t smem, co
   int blocks = bwd_blocks(N);
   k<<<blocks, kBwdBlock, smem, s>>>(gp, mp, reinterpret_cast<const float4*>(pos), N,
                                     static_cast<const T*>(tables), static_cast<const W*>(weights),
-                                    reinterpret_cast<const float2*>(gate_cr), go, grad_tables, ws, n_params);
+                                    reinterpret_cast<const float2*>(gate_cr), latent, go, grad_tables, ws, n_params);
   SPIN4D_CHECK(launch_status());
   int rb = (n_params + 255) / 256;
   reduce_slots<<<rb, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
@@ -367,8 +376,9 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
 // Tensor-core fused backward (decode_bwd_tc.cu): CTAs per SM, 0 when the shape is not covered.
 int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* m);
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
-                  const void* tables, const void* weights, const float* gate_cr, const spin4d_output_grads* go,
-                  float* grad_tables, float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s);
+                  const void* tables, const void* weights, const float* gate_cr, const float* latent,
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_weights, float* ws, int n_params,
+                  int blocks, cudaStream_t s);
 
 // Thread blocks (= workspace slots) the backward launches for N positions.
 static int bwd_slots(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, int64_t N) {
@@ -387,14 +397,15 @@ extern "C" int spin4d_decode_fwd(const spin4d_grid_desc* g, const spin4d_mlp_des
   SPIN4D_CHECK(check_common(g, m, pos, N, tables, weights, gate_cr));
   if (N == 0) return SPIN4D_OK;
   if (!out.scale || !out.rot || !out.rgb || !out.opacity || !out.cov || !aligned(out.rot, 16) ||
-      !aligned(out.scale, 4) || !aligned(out.rgb, 4) || !aligned(out.opacity, 4) || !aligned(out.cov, 4))
+      !aligned(out.scale, 4) || !aligned(out.rgb, 4) || !aligned(out.opacity, 4) || !aligned(out.cov, 4) ||
+      (out.latent && !aligned(out.latent, 16)))
     return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_decode_fwd")) return SPIN4D_ERR_INJECTED;
   cudaStream_t s = (cudaStream_t)stream;
   bool handled = false;
   int st = decode_fwd_tc(g, m, pos, N, tables, weights, gate_cr, out, s, &handled);
   if (handled) return st;
-  OutPtrs o{out.scale, out.rot, out.rgb, out.opacity, out.cov};
+  OutPtrs o{out.scale, out.rot, out.rgb, out.opacity, out.cov, out.latent};
   return dispatch<FwdFn>(g->table_dtype, g->F, m->w_dtype, make_grid_params(g), make_mlp(m), fwd_smem(m), pos,
                          N, tables, weights, gate_cr, o, s);
 }
@@ -405,13 +416,14 @@ extern "C" size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const s
 }
 
 extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
-                                 const void* tables, const void* weights, const float* gate_cr,
+                                 const void* tables, const void* weights, const float* gate_cr, const float* latent,
                                  const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
                                  void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
   SPIN4D_CHECK(check_common(g, m, pos, N, tables, weights, gate_cr));
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_tables || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
-  if (!aligned(grad_tables, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256))
+  if (!aligned(grad_tables, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256) ||
+      (latent && !aligned(latent, 16)))
     return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_decode_bwd_workspace(g, m, N)) return SPIN4D_ERR_INVALID;
   if (grad_out->rot && !aligned(grad_out->rot, 4)) return SPIN4D_ERR_INVALID;
@@ -423,13 +435,13 @@ extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_des
     cudaStream_t s = (cudaStream_t)stream;
     const int blocks = bwd_slots(g, m, N);
     float* ws = static_cast<float*>(workspace);
-    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, grad_out, grad_tables, grad_weights, ws,
-                               n_params, blocks, s));
+    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
+                               ws, n_params, blocks, s));
     reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
     return launch_status();
   }
   GradPtrs go{grad_out->scale, grad_out->rot, grad_out->rgb, grad_out->opacity, grad_out->cov};
   return dispatch<BwdFn>(g->table_dtype, g->F, m->w_dtype, make_grid_params(g), make_mlp(m), bwd_smem(m), pos,
-                         N, tables, weights, gate_cr, go, grad_tables, grad_weights,
+                         N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
                          static_cast<float*>(workspace), n_params, (cudaStream_t)stream);
 }

@@ -11,19 +11,21 @@
 //      the trunk inputs z and h1 split into two fp16 terms (hi + lo) so the
 //      ReLU masks agree with exact arithmetic; then per position the
 //      activations, their adjoint and the upstream gradients give dy;
-//   Every fp16 operand row (z, h1, h2, dy, dpre2, dpre1) is stored scaled by
+//   Every fp16 operand tile (z, h1, h2, dy, dpre2, dpre1) is stored scaled by
 //   a power of two that puts its largest entry in [2^10, 2^11); epilogues and
-//   the weight-gradient reduction undo the scales in fp32.
+//   the weight-gradient readback undo the scales in fp32.
 //   E. dh2 = dy . Wh      (tcgen05, K = 16)  -> dpre2 = dh2 * [h2 > 0]
 //   G. dh1 = dpre2 . W2   (tcgen05, K = H)   -> dpre1 = dh1 * [h1 > 0]
 //   I. dz  = dpre1 . W1   (tcgen05, K = H)   -> scatter-add into the tables
 //      with fp32 vector atomics; an x-neighbour pair that shares a 16-byte
 //      group of the gradient table is one 16-byte atomic;
-//   F/H/J. weight gradients dW = sum_p d_p a_p^T: lanes run over positions,
-//      each lane an 8x8 outer product per pair of 16-byte operand chunks
-//      (conflict-free reads of the K-major tiles), then a butterfly warp
-//      reduction; the sums go to this CTA's slot of the workspace, which a
-//      second kernel adds into grad_weights in slot order (deterministic).
+//   weight gradients dW = sum_p d_p a_p^T on the tensor core too, issued with
+//      the dgrad MMA of the same stage: the K-major-by-feature operand tiles
+//      are read as MN-major operands so that K runs over the tile's 128
+//      positions (M = 64 accumulators sit in lanes 0-15 of each TMEM
+//      quadrant); biases are column sums over positions (SIMT).  Each tile's
+//      result is unscaled and added to this CTA's slot of the workspace,
+//      which a second kernel adds into grad_weights in slot order.
 // The dgrad MMAs use transposed copies of the weights staged as K-major
 // tiles.  Every mbarrier wait is bounded (device error word on timeout).
 #include "host.h"
@@ -60,8 +62,8 @@ struct BLayout {
   static constexpr int h2t = h1t + kTile * H * 2;    // [128][H], later dpre1
   static constexpr int dyt = h2t + kTile * H * 2;    // [128][16]
   static constexpr int d2t = dyt + kTile * kHeadN * 2;   // [128][H] dpre2
-  static constexpr int scales = d2t + kTile * H * 2;   // fp32 [8][128]: inverse row scales, z-max exchange
-  static constexpr int misc = scales + 8 * kTile * 4;
+  static constexpr int scales = d2t + kTile * H * 2;   // fp32 [8]: per-warp maxima
+  static constexpr int misc = scales + 64;
   static constexpr int bytes = misc + 16;
 };
 
@@ -105,92 +107,85 @@ __device__ __forceinline__ void unpack8(const uint4& u, float f[8]) {
   }
 }
 
-// Butterfly reduction of 64 per-lane values: afterwards lane l holds the
-// warp-wide sums of values 2l and 2l+1 in v[0], v[1].
-__device__ __forceinline__ void warp_reduce64(float v[64]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int r = 0; r < 5; ++r) {
-    const int m = 16 >> r;
-    const int c = 64 >> r;
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int i = 0; i < c / 2; ++i) {
-      const float send = upper ? v[i] : v[i + c / 2];
-      const float keep = upper ? v[i + c / 2] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-    }
-  }
-}
-
-// dW[o][i] += sum_p d[p][o] a[p][i] and db[o] += sum_p d[p][o] for one layer:
-// d is a K-major fp16 tile with Kd columns, a one with Ka columns, each row
-// stored multiplied by a power of two whose inverse is inv_d[p] / inv_a[p];
-// `rows` output rows are real (the rest of d's columns are padding).
-__device__ void weight_grad(const uint8_t* sm, int d_off, int Kd, int rows, const float* inv_d, int a_off, int Ka,
-                            const float* inv_a, float* __restrict__ slotW, float* __restrict__ slotB) {
+// db[o] += factor * sum_p d[p][o] for a K-major fp16 tile d with Kd columns
+// (`rows` real): lanes run over positions, 16-byte chunk reads (conflict-free),
+// then a shuffle reduction per output.
+__device__ void bias_grad(const uint8_t* sm, int d_off, int Kd, int rows, float factor, float* __restrict__ slotB) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = kThreads / 32;
-  const int ob_n = Kd / 8, ib_n = Ka / 8;
-  const int n_blocks = ob_n * ib_n + ob_n;
-  for (int b = warp; b < n_blocks; b += n_warps) {
-    if (b < ob_n * ib_n) {
-      const int ob = b / ib_n, ib = b - ob * ib_n;
-      float acc[64];
+  for (int ob = warp; ob < Kd / 8; ob += n_warps) {
+    float acc[8];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTile / 32; ++j) {
-        const int p = lane + 32 * j;
-        float d[8], a[8];
-        unpack8(*reinterpret_cast<const uint4*>(sm + d_off + tc::kmaj_off(p, ob, Kd)), d);
-        unpack8(*reinterpret_cast<const uint4*>(sm + a_off + tc::kmaj_off(p, ib, Ka)), a);
-        const float f = inv_d[p] * inv_a[p];
+    for (int j = 0; j < kTile / 32; ++j) {
+      float d[8];
+      unpack8(*reinterpret_cast<const uint4*>(sm + d_off + tc::kmaj_off(lane + 32 * j, ob, Kd)), d);
 #pragma unroll
-        for (int oo = 0; oo < 8; ++oo) d[oo] *= f;
+      for (int i = 0; i < 8; ++i) acc[i] += d[i];
+    }
 #pragma unroll
-        for (int oo = 0; oo < 8; ++oo)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int ii = 0; ii < 8; ++ii) acc[oo * 8 + ii] = fmaf(d[oo], a[ii], acc[oo * 8 + ii]);
-      }
-      warp_reduce64(acc);
-      const int o = ob * 8 + (2 * lane) / 8, i = ib * 8 + (2 * lane) % 8;
-      if (o < rows) {
-        float2* q = reinterpret_cast<float2*>(slotW + (size_t)o * Ka + i);
-        float2 t = *q;
-        t.x += acc[0];
-        t.y += acc[1];
-        *q = t;
-      }
-    } else {
-      const int ob = b - ob_n * ib_n;
-      float acc[8];
+      for (int m = 16; m >= 1; m >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], m);
+    float mine = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) mine = (lane == i) ? acc[i] : mine;
+    if (lane < 8 && ob * 8 + lane < rows) slotB[ob * 8 + lane] += mine * factor;
+  }
+}
+
+// Weight-gradient MMA over the tile's positions: D[m][n] = sum_p A[p][m] B[p][n]
+// where A and B are the K-major-by-feature operand tiles (rows = positions,
+// Fa / Fb features per row) read as MN-major operands, so K = 128 positions.
+__device__ __forceinline__ void mma_wgrad(uint32_t d_tmem, uint32_t a_tile, int Fa, uint32_t b_tile, int Fb, int M,
+                                          int N) {
+  const uint32_t idesc = tc::idesc_f16_f32(M, N) | (1u << 15) | (1u << 16);   // A and B MN-major
+  for (int s = 0; s < kTile / 16; ++s)
+    tc::mma_f16(d_tmem, tc::smem_desc(a_tile + s * 32 * Fa, (uint32_t)Fa * 16u, 128),
+                tc::smem_desc(b_tile + s * 32 * Fb, (uint32_t)Fb * 16u, 128), idesc, s > 0 ? 1u : 0u);
+}
+
+// Reads an M x N weight-gradient accumulator (M = 64: rows in lanes 0-15 of
+// each warp quadrant; M = 128: one row per lane) and hands every element to
+// fn(row, col, value).  Warps 0-3 take the first half of the columns, 4-7 the
+// second; N = 16 is read by warps 0-3 alone.
+template <int M, int N, typename Fn>
+__device__ __forceinline__ void wgrad_readback(uint32_t tmem, uint32_t col, Fn fn) {
+  const int warp = threadIdx.x >> 5, t = threadIdx.x & 31, q = warp & 3, ch = warp >> 2;
+  const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+  const int row = M == 128 ? q * 32 + t : q * 16 + t;
+  const bool has_row = M == 128 || t < 16;
+  if constexpr (N == 16) {
+    if (ch == 0) {
+      float v[16];
+      tc::tmem_ld16(tmem + lane_addr + col, v);
+      if (has_row)
 #pragma unroll
-      for (int j = 0; j < kTile / 32; ++j) {
-        const int p = lane + 32 * j;
-        float d[8];
-        unpack8(*reinterpret_cast<const uint4*>(sm + d_off + tc::kmaj_off(p, ob, Kd)), d);
-        const float f = inv_d[p];
+        for (int i = 0; i < 16; ++i) fn(row, i, v[i]);
+    }
+  } else if constexpr (N == 32) {
+    float v[16];
+    tc::tmem_ld16(tmem + lane_addr + col + ch * 16, v);
+    if (has_row)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(d[i], f, acc[i]);
-      }
+      for (int i = 0; i < 16; ++i) fn(row, ch * 16 + i, v[i]);
+  } else {
+#pragma unroll 1
+    for (int c0 = ch * (N / 2); c0 < (ch + 1) * (N / 2); c0 += 32) {
+      float v[32];
+      tc::tmem_ld32(tmem + lane_addr + col + c0, v);
+      if (has_row)
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], m);
-      float mine = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mine = (lane == i) ? acc[i] : mine;
-      if (lane < 8 && ob * 8 + lane < rows) slotB[ob * 8 + lane] += mine;
+        for (int i = 0; i < 32; ++i) fn(row, c0 + i, v[i]);
     }
   }
 }
 
-// Power of two that brings a row's largest magnitude m into [2^10, 2^11):
-// every fp16 operand row is stored scaled by it, so values that would be
+// Power of two that brings a tile's largest magnitude m into [2^10, 2^11):
+// every fp16 operand tile is stored scaled by it, so values that would be
 // fp16-subnormal (small upstream gradients, tiny early-training activations)
-// keep their 11-bit precision.  Exact (a power of two); 1 for m = 0.
+// keep their 11-bit precision; rows down to 2^-24 of the tile maximum stay
+// normal.  Exact (a power of two); 1 for m = 0.
 __device__ __forceinline__ float pow2_scale(float m) {
   if (!(m > 0.f) || !isfinite(m)) return 1.0f;
   int e;
@@ -270,11 +265,14 @@ __device__ __forceinline__ void issue_mma_split(uint32_t d_tmem, uint32_t a_hi, 
 template <int F, int IN, int H>
 __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kernel(
     GridParams g, int gate, float tau, const float4* __restrict__ pos, int64_t N, const __half* __restrict__ tables,
-    const __half* __restrict__ weights, const float2* __restrict__ gate_cr, GradIn go, float* __restrict__ grad_tables,
-    float* __restrict__ ws, int n_params) {
+    const __half* __restrict__ weights, const float2* __restrict__ gate_cr, const float* __restrict__ latent, GradIn go,
+    float* __restrict__ grad_tables, float* __restrict__ ws, int n_params) {
   using Lay = BLayout<IN, H>;
-  constexpr uint32_t kCols = tmem_cols(2 * H);
-  static_assert(IN % 16 == 0 && H % 16 == 0 && (F == 2 || F == 4) && IN <= H, "tile shape");
+  // TMEM columns: two per-tile regions of H, then the weight-gradient
+  // accumulators dW1 (IN), dW2 (H), dWh^T (16)
+  constexpr uint32_t colA = 0, colB = H, cW1 = 2 * H, cW2 = 2 * H + IN, cW3 = 2 * H + IN + H;
+  constexpr uint32_t kCols = tmem_cols(2 * H + IN + H + kHeadN);
+  static_assert(IN % 16 == 0 && H % 16 == 0 && (F == 2 || F == 4) && IN <= H && (H == 64 || H == 128), "tile shape");
   extern __shared__ __align__(1024) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & (kTile - 1), half = tid / kTile;
@@ -314,7 +312,6 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t colA = 0, colB = (uint32_t)H;
   uint32_t phase = 0;
   bool failed = false;
   const uint32_t a_zt = tc::smem_u32(sm + Lay::zt), a_h1 = tc::smem_u32(sm + Lay::h1t),
@@ -334,44 +331,47 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
     __syncthreads();
   };
 
-  float* inv = reinterpret_cast<float*>(sm + Lay::scales);
-  float* inv_z = inv, *inv_h1 = inv + kTile, *inv_h2 = inv + 2 * kTile, *inv_dy = inv + 3 * kTile,
-       *inv_d2 = inv + 4 * kTile, *inv_d1 = inv + 5 * kTile, *zmax = inv + 6 * kTile;   // zmax: [2][128]
-
-  // Epilogue helper: the row's values fn(column, accumulator) over all H
-  // columns of TMEM region `col` give the row scale; this thread then stores
-  // its half of the scaled row as fp16 at `dst` and, if dst_lo >= 0, the
-  // rounding remainder as a second fp16 tile at `dst_lo`.
+  float* red = reinterpret_cast<float*>(sm + Lay::scales);   // per-warp maxima
+  const int lane_id = tid & 31;
+  // Largest magnitude over the whole tile (all 256 threads contribute).
+  auto tile_max = [&](float m) -> float {
+    const unsigned u = __reduce_max_sync(0xffffffffu, __float_as_uint(m));   // m >= 0: bit order = value order
+    if (lane_id == 0) red[warp] = __uint_as_float(u);
+    __syncthreads();
+    float t = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) t = fmaxf(t, red[w]);
+    return t;
+  };
+  // Epilogue: this thread's half of the row, fn(column, accumulator) -> value;
+  // one scale for the tile; fp16 hi at `dst`, rounding remainder at `dst_lo`.
   auto store_scaled = [&](uint32_t col, int dst, int dst_lo, auto fn) -> float {
+    constexpr int HH = H / 2;
+    float v[HH];
+#pragma unroll
+    for (int c0 = 0; c0 < HH; c0 += 32) tc::tmem_ld32(tmem + lane + col + half * HH + c0, v + c0);
     float m = 0.f;
-#pragma unroll 1
-    for (int c0 = 0; c0 < H; c0 += 32) {
-      float v[32];
-      tc::tmem_ld32(tmem + lane + col + c0, v);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(fn(c0 + i, v[i])));
+    for (int i = 0; i < HH; ++i) {
+      v[i] = fn(half * HH + i, v[i]);
+      m = fmaxf(m, fabsf(v[i]));
     }
-    const float sc = pow2_scale(m);
-#pragma unroll 1
-    for (int c0 = half * (H / 2); c0 < (half + 1) * (H / 2); c0 += 32) {
-      float v[32];
-      tc::tmem_ld32(tmem + lane + col + c0, v);
+    const float sc = pow2_scale(tile_max(m));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float r[8];
+    for (int q = 0; q < HH / 8; ++q) {
+      float r[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) r[i] = fn(c0 + 8 * q + i, v[8 * q + i]) * sc;
-        store_row8(sm, dst, row, c0 / 8 + q, H, r);
-        if (dst_lo >= 0) {
+      for (int i = 0; i < 8; ++i) r[i] = v[8 * q + i] * sc;
+      store_row8(sm, dst, row, half * (HH / 8) + q, H, r);
+      if (dst_lo >= 0) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) r[i] -= __half2float(__float2half_rn(r[i]));
-          store_row8(sm, dst_lo, row, c0 / 8 + q, H, r);
-        }
+        for (int i = 0; i < 8; ++i) r[i] -= __half2float(__float2half_rn(r[i]));
+        store_row8(sm, dst_lo, row, half * (HH / 8) + q, H, r);
       }
     }
     return sc;
   };
-  // fp16 tile value (unscaled sign test only) of this row at column c
+  // fp16 tile entry of this row at column c (for ReLU masks: sign only)
   auto tile_at = [&](int off, int c) -> float {
     return __half2float(*reinterpret_cast<const __half*>(sm + off + tc::kmaj_off(row, c / 8, H) + (c % 8) * 2));
   };
@@ -380,30 +380,38 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
     const int64_t n = tile * kTile + row;
     const bool valid = n < N;
     float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    // ---- A. gather this thread's half of z; one power-of-two scale per row ----
+    // ---- A. gather this thread's half of z; one power-of-two scale per tile ----
     if (valid) normalise_position(pos[n], g, xt);
     constexpr int HZ = IN / 2;
     float zv[HZ];
+    if (latent) {   // z saved by the forward pass: no second gather
 #pragma unroll
-    for (int q = 0; q < HZ / F; ++q) {
-      float acc[F];
-      if (valid) {
-        encode_level_f16_paired<F>(xt, g, half * (HZ / F) + q, tables, acc);
-      } else {
-#pragma unroll
-        for (int f = 0; f < F; ++f) acc[f] = 0.f;
+      for (int q = 0; q < HZ / 4; ++q) {
+        float4 v = valid ? __ldg(reinterpret_cast<const float4*>(latent + n * IN + half * HZ) + q)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        zv[4 * q] = v.x;
+        zv[4 * q + 1] = v.y;
+        zv[4 * q + 2] = v.z;
+        zv[4 * q + 3] = v.w;
       }
+    } else {
 #pragma unroll
-      for (int f = 0; f < F; ++f) zv[q * F + f] = acc[f];
-    }
-    {
-      float m = 0.f;
+      for (int q = 0; q < HZ / F; ++q) {
+        float acc[F];
+        if (valid) {
+          encode_level_f16_paired<F>(xt, g, half * (HZ / F) + q, tables, acc);
+        } else {
 #pragma unroll
-      for (int i = 0; i < HZ; ++i) m = fmaxf(m, fabsf(zv[i]));
-      zmax[half * kTile + row] = m;
+          for (int f = 0; f < F; ++f) acc[f] = 0.f;
+        }
+#pragma unroll
+        for (int f = 0; f < F; ++f) zv[q * F + f] = acc[f];
+      }
     }
-    __syncthreads();
-    const float s_z = pow2_scale(fmaxf(zmax[row], zmax[kTile + row]));
+    float zm = 0.f;
+#pragma unroll
+    for (int i = 0; i < HZ; ++i) zm = fmaxf(zm, fabsf(zv[i]));
+    const float s_z = pow2_scale(tile_max(zm));
 #pragma unroll
     for (int kc = 0; kc < HZ / 8; ++kc) {
       float r[8];
@@ -415,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
       for (int i = 0; i < 8; ++i) r[i] -= __half2float(__float2half_rn(r[i]));
       store_row8(sm, Lay::h2t, row, half * (HZ / 8) + kc, IN, r);
     }
-    if (half == 0) inv_z[row] = 1.0f / s_z;
     handoff();
     // ---- B. h1 = relu(z W1^T + b1), z as hi + lo: the ReLU masks must match
     //      those of exact arithmetic, or the gradient of a pre-activation near
@@ -425,7 +432,6 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
     const float iz = 1.0f / s_z;
     const float s_h1 = store_scaled(colA, Lay::h1t, Lay::d2t,
                                     [&](int c, float v) { return fmaxf(fmaf(v, iz, bias[c]), 0.f); });
-    if (half == 0) inv_h1[row] = 1.0f / s_h1;
     handoff();
     // ---- C. h2 = relu(h1 W2^T + b2), h1 as hi + lo ----
     if (tid == 0) issue_mma_split(tmem + colB, a_h1, a_d2, tc::smem_u32(sm + Lay::w2), H, H, mbar);
@@ -433,17 +439,16 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
     const float ih1 = 1.0f / s_h1;
     const float s_h2 = store_scaled(colB, Lay::h2t, -1,
                                     [&](int c, float v) { return fmaxf(fmaf(v, ih1, bias[H + c]), 0.f); });
-    if (half == 0) inv_h2[row] = 1.0f / s_h2;
     handoff();
-    // ---- D. head and its adjoint: dy (scaled per row) ----
+    // ---- D. head and its adjoint: dy ----
     if (tid == 0) issue_mma(tmem + colA, a_h2, tc::smem_u32(sm + Lay::wh), H, kHeadN, mbar);
     if (!wait_mma()) { failed = true; break; }
+    float dy[kHeadN];
+#pragma unroll
+    for (int i = 0; i < kHeadN; ++i) dy[i] = 0.f;
     if (half == 0) {
       float v[16];
       tc::tmem_ld16(tmem + lane + colA, v);
-      float dy[kHeadN];
-#pragma unroll
-      for (int i = 0; i < kHeadN; ++i) dy[i] = 0.f;
       if (valid) {
         const float ih2 = 1.0f / s_h2;
         float y[kHeadRows];
@@ -466,10 +471,12 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
         for (int i = 0; i < 6; ++i) ag.cov[i] = g_or0(go.cov, 6 * n + i);
         heads_backward(y, gw, ag, dy);
       }
-      float m = 0.f;
+    }
+    float dm = 0.f;
 #pragma unroll
-      for (int i = 0; i < kHeadN; ++i) m = fmaxf(m, fabsf(dy[i]));
-      const float s_dy = pow2_scale(m);
+    for (int i = 0; i < kHeadN; ++i) dm = fmaxf(dm, fabsf(dy[i]));
+    const float s_dy = pow2_scale(tile_max(dm));
+    if (half == 0) {
 #pragma unroll
       for (int i = 0; i < kHeadN; ++i) dy[i] *= s_dy;
       *reinterpret_cast<uint4*>(sm + Lay::dyt + tc::kmaj_off(row, 0, kHeadN)) =
@@ -478,30 +485,55 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
       *reinterpret_cast<uint4*>(sm + Lay::dyt + tc::kmaj_off(row, 1, kHeadN)) =
           make_uint4(tc::pack_half2(dy[8], dy[9]), tc::pack_half2(dy[10], dy[11]), tc::pack_half2(dy[12], dy[13]),
                      tc::pack_half2(dy[14], dy[15]));
-      inv_dy[row] = 1.0f / s_dy;
     }
     handoff();
-    // ---- E. dpre2 = (dy Wh) * [h2 > 0] ----
-    if (tid == 0) issue_mma(tmem + colB, a_dy, tc::smem_u32(sm + Lay::wht), kHeadN, H, mbar);
-    // ---- F. head weight gradient (overlaps the MMA) ----
-    weight_grad(sm, Lay::dyt, kHeadN, kHeadRows, inv_dy, Lay::h2t, H, inv_h2, slot + oWh, slot + oBh);
+    // ---- E. dpre2 = (dy Wh) * [h2 > 0]; dWh^T = h2^T dy on the tensor core ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma_group(tmem + colB, a_dy, tc::smem_u32(sm + Lay::wht), kHeadN, H, false);
+      mma_wgrad(tmem + cW3, a_h2, H, a_dy, kHeadN, H, kHeadN);
+      tc::mma_commit(mbar);
+    }
+    bias_grad(sm, Lay::dyt, kHeadN, kHeadRows, 1.0f / s_dy, slot + oBh);
     if (!wait_mma()) { failed = true; break; }
-    const float idy = inv_dy[row];
+    {
+      const float f3 = 1.0f / (s_h2 * s_dy);
+      wgrad_readback<H, kHeadN>(tmem, cW3, [&](int i, int o, float v) {
+        if (o < kHeadRows) slot[oWh + o * H + i] += v * f3;
+      });
+    }
+    const float idy = 1.0f / s_dy;
     const float s_d2 = store_scaled(colB, Lay::d2t, -1, [&](int c, float v) { return tile_at(Lay::h2t, c) > 0.f ? v * idy : 0.f; });
-    if (half == 0) inv_d2[row] = 1.0f / s_d2;
     handoff();
-    // ---- G. dpre1 = (dpre2 W2) * [h1 > 0], into the h2 tile ----
-    if (tid == 0) issue_mma(tmem + colA, a_d2, tc::smem_u32(sm + Lay::w2t), H, H, mbar);
+    // ---- G. dpre1 = (dpre2 W2) * [h1 > 0] into the h2 tile; dW2 = dpre2^T h1 ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma_group(tmem + colA, a_d2, tc::smem_u32(sm + Lay::w2t), H, H, false);
+      mma_wgrad(tmem + cW2, a_d2, H, a_h1, H, H, H);
+      tc::mma_commit(mbar);
+    }
+    bias_grad(sm, Lay::d2t, H, H, 1.0f / s_d2, slot + oB2);
     if (!wait_mma()) { failed = true; break; }
+    {
+      const float f2 = 1.0f / (s_d2 * s_h1);
+      wgrad_readback<H, H>(tmem, cW2, [&](int o, int i, float v) { slot[oW2 + o * H + i] += v * f2; });
+    }
     const float id2 = 1.0f / s_d2;
     const float s_d1 = store_scaled(colA, Lay::h2t, -1, [&](int c, float v) { return tile_at(Lay::h1t, c) > 0.f ? v * id2 : 0.f; });
-    if (half == 0) inv_d1[row] = 1.0f / s_d1;
     handoff();
-    // ---- I. dz = dpre1 W1 ----
-    if (tid == 0) issue_mma(tmem + colB, a_h2, tc::smem_u32(sm + Lay::w1t), H, IN, mbar);
-    // ---- H. layer-2 weight gradient (overlaps the MMA) ----
-    weight_grad(sm, Lay::d2t, H, H, inv_d2, Lay::h1t, H, inv_h1, slot + oW2, slot + oB2);
+    // ---- I. dz = dpre1 W1 -> scatter; dW1 = dpre1^T z ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma_group(tmem + colB, a_h2, tc::smem_u32(sm + Lay::w1t), H, IN, false);
+      mma_wgrad(tmem + cW1, a_h2, H, a_zt, IN, H, IN);
+      tc::mma_commit(mbar);
+    }
+    bias_grad(sm, Lay::h2t, H, H, 1.0f / s_d1, slot + oB1);
     if (!wait_mma()) { failed = true; break; }
+    {
+      const float f1 = 1.0f / (s_d1 * s_z);
+      wgrad_readback<H, IN>(tmem, cW1, [&](int o, int i, float v) { slot[oW1 + o * IN + i] += v * f1; });
+    }
     {
       constexpr int HALF_IN = IN / 2;
       float dzv[HALF_IN];
@@ -523,8 +555,6 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
         }
       }
     }
-    // ---- J. layer-1 weight gradient ----
-    weight_grad(sm, Lay::h2t, H, H, inv_d1, Lay::zt, IN, inv_z, slot + oW1, slot + oB1);
     tc::fence_before_sync();
     __syncthreads();
   }
@@ -543,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 
 template <int F, int IN, int H>
 int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* pos, int64_t N, const void* tables,
-                  const void* weights, const float* gate_cr, const spin4d_output_grads* go, float* grad_tables,
-                  float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s) {
+                  const void* weights, const float* gate_cr, const float* latent, const spin4d_output_grads* go,
+                  float* grad_tables, float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s) {
   using Lay = BLayout<IN, H>;
   auto k = decode_bwd_tc_kernel<F, IN, H>;
   const int smem = align_up(Lay::bytes, 128);
@@ -557,13 +587,13 @@ int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* p
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
     if (e != cudaSuccess) return cuda_status(e);
-    if (occ < 1 || occ * (int)tmem_cols(2 * H) > 512) return SPIN4D_ERR_UNSUPPORTED;
+    if (occ < 1 || occ * (int)tmem_cols(3 * H + IN + kHeadN) > 512) return SPIN4D_ERR_UNSUPPORTED;
     configured[dev] = true;
   }
   GradIn gi{go->scale, go->rot, go->rgb, go->opacity, go->cov};
   k<<<blocks, kThreads, smem, s>>>(gp, m->gate, m->tau, reinterpret_cast<const float4*>(pos), N,
                                    static_cast<const __half*>(tables), static_cast<const __half*>(weights),
-                                   reinterpret_cast<const float2*>(gate_cr), gi, grad_tables, ws, n_params);
+                                   reinterpret_cast<const float2*>(gate_cr), latent, gi, grad_tables, ws, n_params);
   return launch_status();
 }
 
@@ -591,15 +621,16 @@ int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* 
 }
 
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
-                  const void* tables, const void* weights, const float* gate_cr, const spin4d_output_grads* go,
-                  float* grad_tables, float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s) {
+                  const void* tables, const void* weights, const float* gate_cr, const float* latent,
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_weights, float* ws, int n_params,
+                  int blocks, cudaStream_t s) {
   const GridParams gp = make_grid_params(g);
   if (g->F == 2 && m->in_dim == 32 && m->hidden == 64)
-    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, go, grad_tables, grad_weights, ws,
-                                    n_params, blocks, s);
+    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
+                                    ws, n_params, blocks, s);
   if (g->F == 4 && m->in_dim == 64 && m->hidden == 128)
-    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, go, grad_tables, grad_weights, ws,
-                                     n_params, blocks, s);
+    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
+                                     ws, n_params, blocks, s);
   return SPIN4D_ERR_UNSUPPORTED;
 }
 

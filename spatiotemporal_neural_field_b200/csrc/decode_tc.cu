@@ -55,7 +55,7 @@ struct Layout {
 };
 
 struct TcOut {
-  float *scale, *rot, *rgb, *opacity, *cov;
+  float *scale, *rot, *rgb, *opacity, *cov, *latent;
 };
 
 // W[rows][K] (fp16, row-major, global) -> K-major tile with `rows_pad` rows.
@@ -144,6 +144,11 @@ __global__ void __launch_bounds__(kThreads, 512 / tmem_cols(2 * H)) decode_fwd_t
         }
 #pragma unroll
         for (int f = 0; f < F; ++f) zv[q * F + f] = acc[f];
+      }
+      if (out.latent && valid) {   // z saved for the backward pass
+        float4* zl = reinterpret_cast<float4*>(out.latent + n * IN + kc * 8);
+        zl[0] = make_float4(zv[0], zv[1], zv[2], zv[3]);
+        zl[1] = make_float4(zv[4], zv[5], zv[6], zv[7]);
       }
       *reinterpret_cast<uint4*>(sm + Lay::zt + tc::kmaj_off(row, kc, IN)) =
           make_uint4(tc::pack_half2(zv[0], zv[1]), tc::pack_half2(zv[2], zv[3]), tc::pack_half2(zv[4], zv[5]),
@@ -278,7 +283,7 @@ int launch_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* pos, 
   }
   const int64_t tiles = (N + kTile - 1) / kTile;
   const int blocks = persistent_blocks(tiles, ctas);
-  TcOut out{o.scale, o.rot, o.rgb, o.opacity, o.cov};
+  TcOut out{o.scale, o.rot, o.rgb, o.opacity, o.cov, o.latent};
   k<<<blocks, kThreads, smem, s>>>(gp, m->n_hidden, m->gate, m->tau, reinterpret_cast<const float4*>(pos), N,
                                 static_cast<const __half*>(tables), static_cast<const __half*>(weights),
                                 reinterpret_cast<const float2*>(gate_cr), out);

@@ -43,7 +43,8 @@ class MlpDesc(ctypes.Structure):
 
 
 class Outputs(ctypes.Structure):
-    _fields_ = [("scale", c_vp), ("rot", c_vp), ("rgb", c_vp), ("opacity", c_vp), ("cov", c_vp)]
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("rgb", c_vp), ("opacity", c_vp), ("cov", c_vp),
+                ("latent", c_vp)]
 
 
 class OutputGrads(ctypes.Structure):
@@ -70,7 +71,7 @@ _SIGS = {
     "spin4d_encode_fwd": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
     "spin4d_decode_fwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, Outputs, c_vp]),
     "spin4d_decode_bwd_workspace": (c_sz, [P(GridDesc), P(MlpDesc), c_i64]),
-    "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, P(OutputGrads),
+    "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
                                   c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "spin4d_adam_step": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i32, c_f32, c_f32, c_f32, c_f32, c_i32,
@@ -184,9 +185,13 @@ def encode_fwd(g: GridDesc, pos: torch.Tensor, tables: torch.Tensor, z: Optional
     return z
 
 
-def alloc_outputs(N: int, device) -> Dict[str, torch.Tensor]:
-    return {k: torch.empty((N, w), dtype=torch.float32, device=device)
-            for k, w in (("scale", 3), ("rot", 4), ("rgb", 3), ("opacity", 1), ("cov", 6))}
+def alloc_outputs(N: int, device, latent_dim: int = 0) -> Dict[str, torch.Tensor]:
+    """Output tensors; latent_dim = L*F also allocates the saved latent z."""
+    out = {k: torch.empty((N, w), dtype=torch.float32, device=device)
+           for k, w in (("scale", 3), ("rot", 4), ("rgb", 3), ("opacity", 1), ("cov", 6))}
+    if latent_dim:
+        out["latent"] = torch.empty((N, latent_dim), dtype=torch.float32, device=device)
+    return out
 
 
 def decode_fwd(g: GridDesc, m: MlpDesc, pos: torch.Tensor, tables: torch.Tensor, weights: torch.Tensor,
@@ -195,7 +200,7 @@ def decode_fwd(g: GridDesc, m: MlpDesc, pos: torch.Tensor, tables: torch.Tensor,
     N = pos.shape[0]
     if out is None:
         out = alloc_outputs(N, pos.device)
-    o = Outputs(*(_ptr(out[k]) for k in ("scale", "rot", "rgb", "opacity", "cov")))
+    o = Outputs(*(_ptr(out.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov", "latent")))
     _check("spin4d_decode_fwd", lib.spin4d_decode_fwd(ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables),
                                                       _ptr(weights), _ptr(gate_cr), o, _stream(stream)))
     return out
@@ -207,14 +212,16 @@ def decode_bwd_workspace(g: GridDesc, m: MlpDesc, N: int) -> int:
 
 def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
                grad_tables: torch.Tensor, grad_weights: torch.Tensor, gate_cr=None,
-               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+               workspace: Optional[torch.Tensor] = None, latent: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    """latent: the z saved by decode_fwd for the same positions (optional)."""
     N = pos.shape[0]
     need = decode_bwd_workspace(g, m, N)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
     go = OutputGrads(*(_ptr(grads.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov")))
     _check("spin4d_decode_bwd", lib.spin4d_decode_bwd(ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables),
-                                                      _ptr(weights), _ptr(gate_cr), ctypes.byref(go),
+                                                      _ptr(weights), _ptr(gate_cr), _ptr(latent), ctypes.byref(go),
                                                       _ptr(grad_tables), _ptr(grad_weights), _ptr(workspace),
                                                       workspace.numel(), _stream(stream)))
 

@@ -64,7 +64,7 @@ FAKE = 1 << 20      # 16-byte aligned, never dereferenced: every call below retu
 
 
 def _outs(sp):
-    return sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE)
+    return sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE, None)
 
 
 def test_invalid_arguments_rejected_on_host(sp):
@@ -100,8 +100,11 @@ def test_invalid_arguments_rejected_on_host(sp):
     assert lib.spin4d_decode_fwd(ref(g), ref(m4), FAKE, 10, FAKE, FAKE, FAKE, _outs(sp), None) == sp.ERR_INVALID
     # bwd: too small a workspace
     go = sp.OutputGrads()
-    assert lib.spin4d_decode_bwd(ref(g), ref(m), FAKE, 1000, FAKE, FAKE, None, ref(go), FAKE, FAKE, FAKE, 16,
+    assert lib.spin4d_decode_bwd(ref(g), ref(m), FAKE, 1000, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, FAKE, 16,
                                  None) == sp.ERR_INVALID
+    # misaligned saved latent
+    assert lib.spin4d_decode_fwd(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None,
+                                 sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4), None) == sp.ERR_INVALID
     # adam
     assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 0, 1e-3, 0.9, 0.99, 1e-15, 0, None,
                                 None) == sp.ERR_INVALID
@@ -126,7 +129,7 @@ sys.path.insert(0, %r)
 from spatiotemporal_neural_field_b200 import spin4d as sp, synthetic as S
 g = sp.grid_from_spec(S.GRID_SPORTS); m = sp.mlp_from_spec(S.MLP_SPORTS)
 F = 1 << 20
-r1 = sp.lib.spin4d_decode_fwd(ctypes.byref(g), ctypes.byref(m), F, 10, F, F, None, sp.Outputs(F, F, F, F, F), None)
+r1 = sp.lib.spin4d_decode_fwd(ctypes.byref(g), ctypes.byref(m), F, 10, F, F, None, sp.Outputs(F, F, F, F, F, None), None)
 r2 = sp.lib.spin4d_encode_fwd(ctypes.byref(g), F, -1, F, F, None)
 print(r1, r2)
 """ % ROOT

@@ -252,6 +252,34 @@ def test_decode_bwd_covariance_only_gradient(sp, name, n):
         o += out_d * in_d + out_d
 
 
+@pytest.mark.parametrize("name,n", [("tiny_fp32", 4099), ("sports_frame_fp16", 20011), ("stress_fp16_gate", 3001)])
+def test_saved_latent_matches_encoder_and_feeds_backward(sp, name, n):
+    """decode_fwd's saved latent equals encode_fwd's z bit for bit, and the
+    backward fed with it matches the oracle (and the re-gathering backward)."""
+    grid, mlp, pos, tables, weights, cr = _workload(name, n, 1.0, 0.5)
+    g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+    P, T, W = dev(pos), dev(tables), dev(weights)
+    C = dev(cr) if cr is not None else None
+    out = sp.decode_fwd(g, m, P, T, W, C, out=sp.alloc_outputs(n, "cuda", latent_dim=grid.L * grid.F))
+    z = sp.encode_fwd(g, P, T)
+    assert torch.equal(out["latent"], z)
+    gstd = 1e-2 if grid.dtype == "f16" else 1.0
+    grads = S.upstream_grads(n, S.DECODE_OUT_WIDTHS, gstd)
+    G = {k: dev(v) for k, v in grads.items()}
+    res = []
+    for lat in (out["latent"], None):
+        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), dtype=torch.float32, device="cuda")
+        gw = torch.zeros(mlp.n_params(), dtype=torch.float32, device="cuda")
+        sp.decode_bwd(g, m, P, T, W, G, gt, gw, gate_cr=C, latent=lat)
+        res.append((host(gt), host(gw)))
+    tol.normwise(res[0][0], res[1][0], 1e-4, "tables: saved latent vs re-gather")
+    tol.normwise(res[0][1], res[1][1], 1e-4, "weights: saved latent vs re-gather")
+    wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr)
+    rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
+    tol.normwise(res[0][0], wt, rtol, "grad_tables")
+    tol.normwise(res[0][1], ww, rtol, "grad_weights")
+
+
 def test_decode_bwd_null_upstream_means_zero(sp):
     """A NULL upstream pointer is a zero gradient: only rgb given."""
     grid, mlp, pos, tables, weights, _ = _workload("tiny_fp32", 1000, 1.0, 0.5)

@@ -189,6 +189,31 @@ int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                       void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 
 /*
+ * spin4d_decode_bwd without a workspace argument, for callers that cannot
+ * allocate device memory (hosts that own all device memory and hand the
+ * library only its input and output buffers, or loops that may not call
+ * cudaMalloc while running).  The paper has no counterpart; this is an
+ * interface convenience of this library.
+ *
+ * The scratch lives in one array of SPIN4D_NOALLOC_SCRATCH_BYTES compiled
+ * into the library; every GPU that loads the library holds it until the
+ * process exits.  Returns SPIN4D_ERR_INVALID, launching nothing, when the
+ * scratch this (g, m, N) needs (spin4d_decode_bwd_workspace) is larger.
+ * The first call on each device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array: calls that
+ * overlap on the GPU (different streams, or different host threads) race and
+ * corrupt each other's weight gradients; serialise them.  Each call writes
+ * every part of the scratch it reads, so nothing needs clearing between calls.
+ * Other arguments, results and errors are those of spin4d_decode_bwd.
+ */
+#define SPIN4D_NOALLOC_SCRATCH_BYTES (16u << 20)
+int spin4d_decode_bwd_noalloc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
+                              const float* pos, int64_t N, const void* tables, const void* weights,
+                              const float* gate_cr, const float* latent, const spin4d_output_grads* grad_out,
+                              float* grad_tables, float* grad_weights, spin4d_stream_t stream);
+
+/*
  * Eq. 2 alone: Sigma = R(q) diag(s)^2 R(q)^T for unit quaternions q = (w,x,y,z).
  *   scale N x 3, rot N x 4 (used as given, not renormalised), cov N x 6 packed.
  */

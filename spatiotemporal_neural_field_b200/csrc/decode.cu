@@ -445,3 +445,61 @@ extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_des
                          N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
                          static_cast<float*>(workspace), n_params, (cudaStream_t)stream);
 }
+
+// ---------------------------------------------------------------------------
+// Backward pass for callers that cannot allocate device memory.
+//
+// Some hosts own every byte of device memory themselves: a renderer or game
+// engine that hands a plugin only the buffers it passes in, or a real-time
+// loop that forbids cudaMalloc once it is running.  Such a caller cannot
+// provide the workspace spin4d_decode_bwd asks for, so this entry point uses
+// a fixed scratch array compiled into the library instead.  The array lives
+// in every GPU that loads the library, for the life of the process.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace spin4d {
+
+constexpr size_t kStaticScratchBytes = (size_t)16 << 20;   // 16 MiB
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (cudaGetSymbolAddress with that device current).
+static int static_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= 64) return SPIN4D_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return SPIN4D_OK;
+}
+
+}  // namespace spin4d
+
+extern "C" int spin4d_decode_bwd_noalloc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos,
+                                         int64_t N, const void* tables, const void* weights, const float* gate_cr,
+                                         const float* latent, const spin4d_output_grads* grad_out,
+                                         float* grad_tables, float* grad_weights, spin4d_stream_t stream) {
+  SPIN4D_CHECK(validate_grid(g));
+  SPIN4D_CHECK(validate_mlp(g, m));
+  if (N < 0) return SPIN4D_ERR_INVALID;
+  if (N == 0) return SPIN4D_OK;
+  // The scratch needed grows with the weight count and (up to a cap) with N.
+  if (spin4d_decode_bwd_workspace(g, m, N) > kStaticScratchBytes) return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_decode_bwd_noalloc")) return SPIN4D_ERR_INJECTED;
+  void* scratch = nullptr;
+  SPIN4D_CHECK(static_scratch_address(&scratch));
+  // Every slot the kernels read is first written by the same call, so the
+  // scratch needs no clearing between calls.
+  return spin4d_decode_bwd(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
+                           scratch, kStaticScratchBytes, stream);
+}

@@ -73,6 +73,8 @@ _SIGS = {
     "spin4d_decode_bwd_workspace": (c_sz, [P(GridDesc), P(MlpDesc), c_i64]),
     "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
                                   c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_decode_bwd_noalloc": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
+                                          P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "spin4d_adam_step": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i32, c_f32, c_f32, c_f32, c_f32, c_i32,
                                  c_vp, c_vp]),
@@ -224,6 +226,22 @@ def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, t
                                                       _ptr(weights), _ptr(gate_cr), _ptr(latent), ctypes.byref(go),
                                                       _ptr(grad_tables), _ptr(grad_weights), _ptr(workspace),
                                                       workspace.numel(), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_bwd_noalloc(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
+                       grad_tables: torch.Tensor, grad_weights: torch.Tensor, gate_cr=None,
+                       latent: Optional[torch.Tensor] = None, stream=None) -> None:
+    """decode_bwd using the library's built-in scratch instead of a caller
+    workspace (for hosts that cannot allocate device memory).  Calls that
+    overlap on the GPU race on that scratch."""
+    go = OutputGrads(*(_ptr(grads.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov")))
+    _check("spin4d_decode_bwd_noalloc",
+           lib.spin4d_decode_bwd_noalloc(ctypes.byref(g), ctypes.byref(m), _ptr(pos), pos.shape[0], _ptr(tables),
+                                         _ptr(weights), _ptr(gate_cr), _ptr(latent), ctypes.byref(go),
+                                         _ptr(grad_tables), _ptr(grad_weights), _stream(stream)))
 
 
 def cov_assemble(scale: torch.Tensor, rot: torch.Tensor, cov: Optional[torch.Tensor] = None, stream=None):

@@ -185,7 +185,9 @@ def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, table
     45 launches of 1M positions, each decode_fwd (saving z) + decode_bwd
     (gradients accumulate), then fused Adam on the fp32 master tables and
     weights, which also rewrites the fp16 working copies and clears the
-    gradients."""
+    gradients.  With N ranks every rank does this on its own upstream
+    gradients and the gradients are summed over ranks before Adam."""
+    from spatiotemporal_neural_field_b200 import dp
     wt = S.WORKLOADS["sports_train_fp16"]
     nb, total = wt["batch"], wt["N"]
     n_batches = total // nb
@@ -211,6 +213,7 @@ def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, table
             sp.decode_bwd(g, m, p, tab16, w16, {k: v[a:e] for k, v in grads.items()}, gtab, gw, workspace=ws,
                           latent=out["latent"], stream=stream)
         state["step"] += 1
+        dp.allreduce_gradients([gtab, gw])     # the step's one exchange (a no-op on one GPU)
         sp.adam_step(tab32, gtab, mt, vt, state["step"], wt["lr"], b1, b2, wt["eps"], params_work=tab16,
                      zero_grad=True, stream=stream)
         sp.adam_step(w32, gw, mw, vw, state["step"], wt["lr"], b1, b2, wt["eps"], params_work=w16,
@@ -227,10 +230,7 @@ def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, table
         step()
         evs[i][1].record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([sum(a.elapsed_time(b) for a, b in evs)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item()) / k
+    ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), device=dev) / k
     return {"metric": "decoded spatiotemporal positions/s (training step: fwd+bwd+Adam)",
             "value": total * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "launches_per_step": 2 * n_batches + 2,
             "workload": "sports_train_fp16: 150 frames x 300k = 45M positions, 45 launches of 1M (decode_fwd saving z "
@@ -303,11 +303,12 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     from spatiotemporal_neural_field_b200 import spin4d as sp
+    from spatiotemporal_neural_field_b200 import dp
 
     w = S.WORKLOADS[WORKLOAD]
     grid, mlp, N = w["grid"], w["mlp"], w["N"]
     scene = S.sports_scene(N)
-    frame_idx = (w["frame"] + rank) % S.N_FRAMES
+    frame_idx = dp.rank_frame(w["frame"], rank, S.N_FRAMES)
     pos_h = scene.frame(frame_idx)
     tables = torch.from_numpy(S.hash_tables(grid)).to(dev)
     weights = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
@@ -340,11 +341,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), device=dev)
     ms_per_step = ms_max / args.steps
     value = N * world * args.steps / (ms_max * 1e-3)
 
@@ -393,10 +390,8 @@ def run_ours(args):
         e2e_step()
     e_e.record(s_out)
     torch.cuda.synchronize()
-    te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = N * world * args.steps / (float(te.item()) * 1e-3)
+    te = dp.max_over_ranks(e_s.elapsed_time(e_e), device=dev)
+    e2e_value = N * world * args.steps / (te * 1e-3)
     h2d = pos_h.nbytes
     d2h = sum(v.numel() * v.element_size() for v in out.values())
 
@@ -428,11 +423,9 @@ def run_ours(args):
             fb()
             evb[i][1].record(stream)
         torch.cuda.synchronize()
-        tb = torch.tensor([sum(a.elapsed_time(b) for a, b in evb)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(tb, op=dist.ReduceOp.MAX)
+        tb = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in evb), device=dev)
         fwd_bwd = {"metric": "decoded spatiotemporal positions/s (fwd+bwd)", "value": nb * world * k /
-                   (float(tb.item()) * 1e-3), "unit": UNIT, "ms_per_step": float(tb.item()) / k,
+                   (tb * 1e-3), "unit": UNIT, "ms_per_step": tb / k,
                    "workload": "sports_train_fp16: one 1M-position launch (frames 0-3), decode_fwd (saving z) + decode_bwd (reading z)"}
 
     # ---- full training step over the 150-frame sequence ----

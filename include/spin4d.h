@@ -330,6 +330,16 @@ int spin4d_check_device_errors(int clear);
 int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t loads_per_thread, int blocks,
                         uint32_t seed, uint32_t* sink, spin4d_stream_t stream);
 
+/*
+ * Test hook for failure detection: one block waits (at most max_iters polls,
+ * 1..2^24) on a barrier that nothing ever arrives at, through the same
+ * bounded-wait path the tensor-core kernels use; the wait runs out, the
+ * kernel sets the device error word and exits.  A following
+ * spin4d_check_device_errors returns SPIN4D_ERR_TIMEOUT.  Nothing hangs and
+ * the context stays usable.
+ */
+int spin4d_selftest_wait_timeout(uint32_t max_iters, spin4d_stream_t stream);
+
 /* Static string for a status code. */
 const char* spin4d_status_string(int status);
 /* cudaError_t of the last SPIN4D_ERR_CUDA returned on this thread (0 if none). */

@@ -86,6 +86,7 @@ _SIGS = {
                                     P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_debug_corners": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
     "spin4d_check_device_errors": (c_i32, [c_i32]),
+    "spin4d_selftest_wait_timeout": (c_i32, [c_u32, c_vp]),
     "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
@@ -308,6 +309,11 @@ def debug_corners(g: GridDesc, pos: torch.Tensor, stream=None):
 def check_device_errors(clear: bool = True) -> None:
     """Synchronous: raises if a kernel's bounded device wait ran out."""
     _check("spin4d_check_device_errors", lib.spin4d_check_device_errors(1 if clear else 0))
+
+
+def selftest_wait_timeout(max_iters: int = 4096, stream=None) -> None:
+    """Launches a kernel whose bounded wait must run out (failure-detection test)."""
+    _check("spin4d_selftest_wait_timeout", lib.spin4d_selftest_wait_timeout(max_iters, _stream(stream)))
 
 
 def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: int, seed: int = 1,

@@ -261,13 +261,16 @@ typedef struct spin4d_hexplane_desc {
 int64_t spin4d_hexplane_plane_count(const spin4d_hexplane_desc* h);
 int64_t spin4d_hexplane_param_count(const spin4d_hexplane_desc* h);
 
-/* Deformed Gaussians: mu' N x 3, rot N x 4, scale N x 3, sh N x 48, cov N x 6 (fp32). */
+/* Deformed Gaussians: mu' N x 3, rot N x 4, scale N x 3, sh N x 48, cov N x 6 (fp32).
+ * latent (optional, may be NULL): N x (n_scales*6*channels) fp32, 16-byte
+ * aligned, receives the concatenated plane samples. */
 typedef struct spin4d_hex_outputs {
     float* mu;
     float* rot;
     float* scale;
     float* sh;
     float* cov;
+    float* latent;
 } spin4d_hex_outputs;
 
 typedef struct spin4d_hex_output_grads {

@@ -310,6 +310,7 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
 }
 
 int bwd_device_error(int clear);   // decode_bwd_tc.cu
+int hex_device_error(int clear);   // hexplane.cu
 
 namespace {
 // Waits on an mbarrier that nothing ever arrives at, with the same bounded
@@ -346,6 +347,8 @@ extern "C" int spin4d_check_device_errors(int clear) {
     if (e != cudaSuccess) return spin4d::cuda_status(e);
   }
   const int b = spin4d::bwd_device_error(clear);
+  const int h = spin4d::hex_device_error(clear);
   if (b != SPIN4D_OK) return b;
+  if (h != SPIN4D_OK) return h;
   return v ? SPIN4D_ERR_TIMEOUT : SPIN4D_OK;
 }

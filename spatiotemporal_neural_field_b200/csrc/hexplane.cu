@@ -17,8 +17,24 @@
 #include <string.h>
 
 #include "host.h"
+#include "tc.cuh"
 
 namespace spin4d {
+
+// Set when a bounded wait of a HexPlane tensor-core kernel runs out.
+__device__ int g_hex_device_error = 0;
+
+int hex_device_error(int clear) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_hex_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (clear && v) {
+    int zero = 0;
+    e = cudaMemcpyToSymbol(g_hex_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return v ? SPIN4D_ERR_TIMEOUT : SPIN4D_OK;
+}
 
 constexpr int kHexC = 32;
 constexpr int kHexH = 64;
@@ -55,9 +71,14 @@ struct PlaneSample {
   float w00, w01, w10, w11;
 };
 
+// xt[a] by selects, so a runtime axis index keeps xt in registers.
+__device__ __forceinline__ float pick_axis(const float xt[4], int a) {
+  return a == 0 ? xt[0] : (a == 1 ? xt[1] : (a == 2 ? xt[2] : xt[3]));
+}
+
 __device__ __forceinline__ PlaneSample plane_sample(const float xt[4], const HexParams& hp, int k) {
-  float pa = __fmul_rn(xt[hp.axis_a[k]], hp.scale_a[k]);
-  float pb = __fmul_rn(xt[hp.axis_b[k]], hp.scale_b[k]);
+  float pa = __fmul_rn(pick_axis(xt, hp.axis_a[k]), hp.scale_a[k]);
+  float pb = __fmul_rn(pick_axis(xt, hp.axis_b[k]), hp.scale_b[k]);
   int ia = min(max((int)floorf(pa), 0), hp.res_a[k] - 2);
   int ib = min(max((int)floorf(pb), 0), hp.res_b[k] - 2);
   float wa = __fsub_rn(pa, (float)ia), wb = __fsub_rn(pb, (float)ib);
@@ -334,6 +355,315 @@ __global__ void hex_reduce_slots(const float* __restrict__ ws, int n_slots, int 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Forward on the tensor cores, fp32-accurate: 3xTF32 (kind::tf32).
+//
+// Every operand x is split into hi = tf32(x) and lo = x - hi, and each
+// product is hi.hi + hi.lo + lo.hi (the dropped lo.lo term is below 2^-21 of
+// the result), which keeps the 1e-5 fp32 parity that plain tf32 misses.
+// Persistent CTAs of 256 threads handle 128-Gaussian tiles.  The 576-wide
+// first layer is streamed one plane sample (32 channels) at a time through
+// two shared-memory stages: while the tensor core multiplies sample k, the
+// threads gather and split sample k+1 (two threads per Gaussian, 16 channels
+// each, 16-byte loads of the channel-last rows) and stage the matching 64x32
+// slice of W1.  Trunk layer 2 and the 58-row head follow from one 128x64
+// activation tile; the epilogue writes mu', q', s', sh' and Sigma.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kHexTile = 128;
+constexpr int kHexThreads = 256;
+constexpr uint32_t kHexWait = 1u << 24;
+
+struct HexTcLayout {
+  static constexpr int A = 0;                      // 2 stages x (hi, lo) [128][32] fp32 = 64 KB; later the H tile
+  static constexpr int A_STAGE = 2 * kHexTile * kHexC * 4;
+  static constexpr int H_LO = kHexTile * kHexH * 4;   // H tile: hi at A, lo at A + H_LO
+  static constexpr int B1 = A + 2 * A_STAGE;       // 2 stages x (hi, lo) [64][32]
+  static constexpr int B1_STAGE = 2 * kHexH * kHexC * 4;
+  static constexpr int W2 = B1 + 2 * B1_STAGE;     // hi, lo [64][64]
+  static constexpr int W3 = W2 + 2 * kHexH * kHexH * 4;   // hi, lo [64][64] (58 rows used)
+  static constexpr int BIAS = W3 + 2 * kHexH * kHexH * 4; // b1 | b2 | b3 (64 each)
+  static constexpr int MISC = BIAS + 3 * kHexH * 4;  // 2 mbarriers + TMEM address
+  static constexpr int BYTES = MISC + 32;
+};
+
+// Stores 4 consecutive values of a row (K-major 32-bit tile with K columns,
+// 4-value chunk kc) as tf32 hi and lo parts.
+__device__ __forceinline__ void store_split4(uint8_t* sm, int hi_off, int lo_off, int r, int kc, int K, float4 v) {
+  float h0, h1, h2, h3, l0, l1, l2, l3;
+  tc::split_tf32(v.x, h0, l0);
+  tc::split_tf32(v.y, h1, l1);
+  tc::split_tf32(v.z, h2, l2);
+  tc::split_tf32(v.w, h3, l3);
+  *reinterpret_cast<float4*>(sm + hi_off + tc::kmaj_off32(r, kc, K)) = make_float4(h0, h1, h2, h3);
+  *reinterpret_cast<float4*>(sm + lo_off + tc::kmaj_off32(r, kc, K)) = make_float4(l0, l1, l2, l3);
+}
+
+// 3xTF32 product over K columns into two fresh accumulators: d_main = A_hi.B_hi
+// and d_corr = A_hi.B_lo + A_lo.B_hi (the dropped lo.lo term is below 2^-21).
+// The tensor core aligns addends to the running sum and truncates, so the
+// small correction terms get an accumulator of their own, and callers keep K
+// short and add the partial results in fp32 on the CUDA cores.
+__device__ __forceinline__ void mma_3xtf32(uint32_t d_main, uint32_t d_corr, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
+                                           uint32_t b_lo, int K, int N) {
+  const uint32_t sbo = (uint32_t)K * 32u;
+  const uint32_t idesc = tc::idesc_tf32_f32(kHexTile, N);
+  for (int s = 0; s < K / 8; ++s) {
+    const uint32_t o = (uint32_t)s * 256u;
+    tc::mma_tf32(d_main, tc::smem_desc(a_hi + o, 128, sbo), tc::smem_desc(b_hi + o, 128, sbo), idesc, s > 0 ? 1u : 0u);
+    tc::mma_tf32(d_corr, tc::smem_desc(a_hi + o, 128, sbo), tc::smem_desc(b_lo + o, 128, sbo), idesc, s > 0 ? 1u : 0u);
+    tc::mma_tf32(d_corr, tc::smem_desc(a_lo + o, 128, sbo), tc::smem_desc(b_hi + o, 128, sbo), idesc, 1u);
+  }
+}
+
+// acc[i] += main[col0 + i] + corr[col0 + i] for this thread's 32 columns.
+__device__ __forceinline__ void add_partial(uint32_t d_main, uint32_t d_corr, float acc[32]) {
+  float a[32], b[32];
+  tc::tmem_ld32(d_main, a);
+  tc::tmem_ld32(d_corr, b);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] += a[i] + b[i];
+}
+
+__global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
+    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
+    const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
+    const float* __restrict__ logs_can, const float* __restrict__ sh_can, HexOutPtrs out, float* __restrict__ latent) {
+  using Lay = HexTcLayout;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kHexTile - 1), half = tid / kHexTile;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  const float* W1 = W;
+  const float* b1 = W1 + kHexH * IN;
+  const float* W2g = b1 + kHexH;
+  const float* b2 = W2g + kHexH * kHexH;
+  const float* W3g = b2 + kHexH;
+  const float* b3 = W3g + kHexHead * kHexH;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::MISC + 16);
+  const uint32_t mbar0 = tc::smem_u32(sm + Lay::MISC), mbar1 = mbar0 + 8;
+  float* bias = reinterpret_cast<float*>(sm + Lay::BIAS);
+
+  // ---- W2, W3 (split) and biases, once per CTA ----
+  for (int i = tid; i < kHexH * (kHexH / 4); i += kHexThreads) {
+    const int r = i / (kHexH / 4), kc = i % (kHexH / 4);
+    store_split4(sm, Lay::W2, Lay::W2 + kHexH * kHexH * 4, r, kc, kHexH,
+                 __ldg(reinterpret_cast<const float4*>(W2g + r * kHexH) + kc));
+    const float4 w3 = r < kHexHead ? __ldg(reinterpret_cast<const float4*>(W3g + r * kHexH) + kc)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    store_split4(sm, Lay::W3, Lay::W3 + kHexH * kHexH * 4, r, kc, kHexH, w3);
+  }
+  for (int o = tid; o < kHexH; o += kHexThreads) {
+    bias[o] = __ldg(b1 + o);
+    bias[kHexH + o] = __ldg(b2 + o);
+    bias[2 * kHexH + o] = o < kHexHead ? __ldg(b3 + o) : 0.f;
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(mbar0, 1);
+    tc::mbar_init(mbar1, 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+  // TMEM regions of 64 columns: R0..R3.  Plane sample k accumulates into
+  // (R0, R1) when k is even and (R2, R3) when odd; layer 2 uses (R0, R1) and
+  // the head (R2, R3).
+  const uint32_t R[4] = {tmem, tmem + 64, tmem + 128, tmem + 192};
+  uint32_t ph0 = 0, ph1 = 0;
+  bool failed = false;
+  auto wait_bar = [&](int b) -> bool {
+    const uint32_t bar = b ? mbar1 : mbar0;
+    uint32_t& ph = b ? ph1 : ph0;
+    const bool ok = tc::mbar_wait_bounded(bar, ph, kHexWait);
+    ph ^= 1u;
+    return ok;
+  };
+  const uint32_t sA = tc::smem_u32(sm + Lay::A), sB1 = tc::smem_u32(sm + Lay::B1);
+  const uint32_t col = (uint32_t)(half * 32);
+
+  for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
+    const int64_t n = tile * kHexTile + row;
+    const bool valid = n < N;
+    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) hex_normalise(mu, frame, n, hp, xt);
+    float acc1[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc1[i] = 0.f;
+    // ---- layer 1, streamed over the plane samples ----
+    // Registers hold sample k+1's global data (its W1 slice and its four
+    // corner rows) while sample k is multiplied, so load latency overlaps
+    // the MMAs and the barriers.
+    float4 wpre[2], cpre[4][4];
+    float cw[4];
+    auto prefetch = [&](int k) {
+      const int r = tid >> 2, c2 = (tid & 3) * 2;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) wpre[q] = __ldg(reinterpret_cast<const float4*>(W1 + (size_t)r * IN + k * kHexC) + c2 + q);
+      if (valid) {
+        const PlaneSample ps = plane_sample(xt, hp, k);
+        cw[0] = ps.w00; cw[1] = ps.w01; cw[2] = ps.w10; cw[3] = ps.w11;
+        const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cpre[c][q] = __ldg(reinterpret_cast<const float4*>(planes + off[c]) + half * 4 + q);
+      }
+    };
+    prefetch(0);
+    for (int k = 0; k < NS; ++k) {
+      const int b = k & 1;
+      if (k >= 2) {   // sample k-2 used this stage: fold its partial sums in, then reuse
+        const bool ok = wait_bar(b);
+        if (__syncthreads_or(!ok)) { failed = true; break; }
+        tc::fence_after_sync();
+        add_partial(R[2 * b] + lane + col, R[2 * b + 1] + lane + col, acc1);
+      }
+      const int a_hi = Lay::A + b * Lay::A_STAGE, a_lo = a_hi + kHexTile * kHexC * 4;
+      const int w_hi = Lay::B1 + b * Lay::B1_STAGE, w_lo = w_hi + kHexH * kHexC * 4;
+      {
+        const int r = tid >> 2, c2 = (tid & 3) * 2;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) store_split4(sm, w_hi, w_lo, r, c2 + q, kHexC, wpre[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c4 = half * 4 + q;
+        float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+          z4.x = cw[0] * cpre[0][q].x + cw[1] * cpre[1][q].x + cw[2] * cpre[2][q].x + cw[3] * cpre[3][q].x;
+          z4.y = cw[0] * cpre[0][q].y + cw[1] * cpre[1][q].y + cw[2] * cpre[2][q].y + cw[3] * cpre[3][q].y;
+          z4.z = cw[0] * cpre[0][q].z + cw[1] * cpre[1][q].z + cw[2] * cpre[2][q].z + cw[3] * cpre[3][q].z;
+          z4.w = cw[0] * cpre[0][q].w + cw[1] * cpre[1][q].w + cw[2] * cpre[2][q].w + cw[3] * cpre[3][q].w;
+          if (latent) reinterpret_cast<float4*>(latent + n * IN + k * kHexC)[c4] = z4;
+        }
+        store_split4(sm, a_hi, a_lo, row, c4, kHexC, z4);
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      __syncthreads();
+      if (tid == 0) {
+        tc::fence_after_sync();
+        mma_3xtf32(R[2 * b], R[2 * b + 1], sA + a_hi, sA + a_lo, sB1 + (w_hi - Lay::B1), sB1 + (w_lo - Lay::B1), kHexC,
+                   kHexH);
+        tc::mma_commit(b ? mbar1 : mbar0);
+      }
+      if (k + 1 < NS) prefetch(k + 1);
+    }
+    if (failed) break;
+    // the last two samples (in the order their barriers completed)
+    for (int k = (NS >= 2 ? NS - 2 : 0); k < NS; ++k) {
+      const int b = k & 1;
+      const bool ok = wait_bar(b);
+      if (__syncthreads_or(!ok)) { failed = true; break; }
+      tc::fence_after_sync();
+      add_partial(R[2 * b] + lane + col, R[2 * b + 1] + lane + col, acc1);
+    }
+    if (failed) break;
+    // ---- h1 = relu(sum + b1) -> split H tile (over the A stages) ----
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 h;
+      h.x = fmaxf(acc1[4 * q] + bias[half * 32 + 4 * q], 0.f);
+      h.y = fmaxf(acc1[4 * q + 1] + bias[half * 32 + 4 * q + 1], 0.f);
+      h.z = fmaxf(acc1[4 * q + 2] + bias[half * 32 + 4 * q + 2], 0.f);
+      h.w = fmaxf(acc1[4 * q + 3] + bias[half * 32 + 4 * q + 3], 0.f);
+      store_split4(sm, Lay::A, Lay::A + Lay::H_LO, row, half * 8 + q, kHexH, h);
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- layer 2 into (R0, R1) ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma_3xtf32(R[0], R[1], sA, sA + Lay::H_LO, tc::smem_u32(sm + Lay::W2), tc::smem_u32(sm + Lay::W2) + kHexH * kHexH * 4,
+                 kHexH, kHexH);
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!wait_bar(0))) { failed = true; break; }
+    tc::fence_after_sync();
+    {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      add_partial(R[0] + lane + col, R[1] + lane + col, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 h;
+        h.x = fmaxf(v[4 * q] + bias[kHexH + half * 32 + 4 * q], 0.f);
+        h.y = fmaxf(v[4 * q + 1] + bias[kHexH + half * 32 + 4 * q + 1], 0.f);
+        h.z = fmaxf(v[4 * q + 2] + bias[kHexH + half * 32 + 4 * q + 2], 0.f);
+        h.w = fmaxf(v[4 * q + 3] + bias[kHexH + half * 32 + 4 * q + 3], 0.f);
+        store_split4(sm, Lay::A, Lay::A + Lay::H_LO, row, half * 8 + q, kHexH, h);
+      }
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- head (58 rows, padded to 64) into (R2, R3) ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma_3xtf32(R[2], R[3], sA, sA + Lay::H_LO, tc::smem_u32(sm + Lay::W3), tc::smem_u32(sm + Lay::W3) + kHexH * kHexH * 4,
+                 kHexH, kHexH);
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!wait_bar(0))) { failed = true; break; }
+    tc::fence_after_sync();
+    {
+      float y[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = bias[2 * kHexH + half * 32 + i];
+      add_partial(R[2] + lane + col, R[3] + lane + col, y);
+      tc::fence_before_sync();
+      if (valid) {
+        if (half == 0) {
+          float qh[4], q[4], s[3], cov[6];
+#pragma unroll
+          for (int i = 0; i < 3; ++i) out.mu[3 * n + i] = __ldg(mu + 3 * n + i) + y[i];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + y[3 + i];
+          normalise_quat(qh, q);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) s[i] = expf(__ldg(logs_can + 3 * n + i) + y[7 + i]);
+          covariance(s, q, cov);
+          reinterpret_cast<float4*>(out.rot)[n] = make_float4(q[0], q[1], q[2], q[3]);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) out.scale[3 * n + i] = s[i];
+#pragma unroll
+          for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
+#pragma unroll
+          for (int i = 10; i < 32; ++i) out.sh[48 * n + (i - 10)] = __ldg(sh_can + 48 * n + (i - 10)) + y[i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < kHexHead - 32; ++i) out.sh[48 * n + 22 + i] = __ldg(sh_can + 48 * n + 22 + i) + y[i];
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  if (failed) {
+    if (tid == 0) atomicExch(&g_hex_device_error, 1);
+    wait_bar(0);
+    wait_bar(1);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
 static const int kAxes[6][2] = {{0, 1}, {0, 2}, {1, 2}, {0, 3}, {1, 3}, {2, 3}};   // XY XZ YZ XT YT ZT
 
 static HexParams make_hex_params(const spin4d_hexplane_desc* h) {
@@ -411,6 +741,26 @@ extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* m
   if (fault_injected("spin4d_hexplane_fwd")) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
+  if (h->n_scales * 6 <= 24) {
+    // tensor cores, 3xTF32
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int smem = HexTcLayout::BYTES;
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(hexplane_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_fwd_tc_kernel, kHexThreads, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      if (occ < 1 || occ * 256 > 512) return SPIN4D_ERR_UNSUPPORTED;
+      configured[dev] = true;
+    }
+    const int blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
+    hexplane_fwd_tc_kernel<<<blocks, kHexThreads, smem, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can,
+                                                                               logs_can, sh_can, o, out.latent);
+    return launch_status();
+  }
   int blocks = persistent_blocks((N + 127) / 128, 4);
   hexplane_fwd_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can, logs_can,
                                                                 sh_can, o);

@@ -57,7 +57,7 @@ class HexDesc(ctypes.Structure):
 
 
 class HexOutputs(ctypes.Structure):
-    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp)]
+    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp), ("latent", c_vp)]
 
 
 class HexOutputGrads(ctypes.Structure):
@@ -276,7 +276,7 @@ def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=
     N = inp["mu"].shape[0]
     if out is None:
         out = {k: torch.empty((N, w), dtype=torch.float32, device=planes.device) for k, w in HEX_KEYS}
-    o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS))
+    o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS), _ptr(out.get("latent")))
     _check("spin4d_hexplane_fwd", lib.spin4d_hexplane_fwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
                                                           _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
                                                           _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), o,

@@ -119,7 +119,7 @@ def test_unsupported_hexplane_shape(sp):
     h = sp.hex_desc(channels=16)
     inp = [FAKE] * 2
     assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE), None) == sp.ERR_UNSUPPORTED
+                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
 
 
 def test_fault_injection_hook_in_subprocess(sp):

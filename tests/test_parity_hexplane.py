@@ -72,3 +72,13 @@ def test_hexplane_bwd_matches_oracle(sp, n):
         o += out_d * in_d
         tol.normwise(gwh[o:o + out_d], ww[o:o + out_d], tol.FP32_GRAD_RTOL, "db %d" % out_d)
         o += out_d
+
+
+def test_hexplane_fwd_saved_latent_matches_oracle_encoder(sp):
+    n = 3001
+    hx, inp, planes, weights = _inputs(n, 0.5)
+    out = {k: torch.empty((n, w), dtype=torch.float32, device="cuda") for k, w in sp.HEX_KEYS}
+    out["latent"] = torch.empty((n, hx.in_dim), dtype=torch.float32, device="cuda")
+    sp.hexplane_fwd(sp.hex_from_spec(hx), {k: dev(v) for k, v in inp.items()}, dev(planes), dev(weights), out=out)
+    z = hp.encode(hp.normalise(inp["mu"], inp["frame"], hx.n_frames), planes, hx)
+    tol.rowwise(host(out["latent"]), z, tol.FP32_RTOL, "latent")

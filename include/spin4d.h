@@ -294,11 +294,22 @@ int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* mu, const in
 
 size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N);
 
-/* Backward of spin4d_hexplane_fwd: grad_planes += , grad_weights += (fp32). */
+/*
+ * Backward of spin4d_hexplane_fwd: grad_planes += dL/dplanes and
+ * grad_weights += dL/dweights (fp32, packed like planes and weights) for
+ * L = sum over outputs of <grad_out.x, x>; a NULL member of grad_out is a
+ * zero gradient.  latent (optional, may be NULL, 16-byte aligned) is the
+ * forward's saved latent for the same inputs; given, the plane samples are
+ * read from it instead of being gathered again.  workspace: device memory
+ * of at least spin4d_hexplane_bwd_workspace(h, N) bytes, 256-byte aligned,
+ * owned by the caller, overwritten.  Plane gradients are accumulated with
+ * fp32 atomics (their order of summation is not fixed); weight gradients
+ * are summed in a fixed order.
+ */
 int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
                         int64_t N, const float* planes, const float* weights,
                         const float* q_can, const float* logs_can, const float* sh_can,
-                        const spin4d_hex_output_grads* grad_out,
+                        const float* latent, const spin4d_hex_output_grads* grad_out,
                         float* grad_planes, float* grad_weights,
                         void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 

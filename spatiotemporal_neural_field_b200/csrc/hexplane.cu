@@ -14,6 +14,7 @@
 // 576-wide feature.  Weight gradients go to the block's workspace slot and
 // are summed in a fixed order by a second kernel; plane gradients are
 // scattered with fp32 vector atomics.
+#include <cuda_bf16.h>
 #include <string.h>
 
 #include "host.h"
@@ -356,18 +357,40 @@ __global__ void hex_reduce_slots(const float* __restrict__ ws, int n_slots, int 
 }
 
 // ---------------------------------------------------------------------------
-// Forward on the tensor cores, fp32-accurate: 3xTF32 (kind::tf32).
+// Forward and backward on the tensor cores, fp32-accurate: bf16x3 split.
 //
-// Every operand x is split into hi = tf32(x) and lo = x - hi, and each
-// product is hi.hi + hi.lo + lo.hi (the dropped lo.lo term is below 2^-21 of
-// the result), which keeps the 1e-5 fp32 parity that plain tf32 misses.
-// Persistent CTAs of 256 threads handle 128-Gaussian tiles.  The 576-wide
-// first layer is streamed one plane sample (32 channels) at a time through
-// two shared-memory stages: while the tensor core multiplies sample k, the
-// threads gather and split sample k+1 (two threads per Gaussian, 16 channels
-// each, 16-byte loads of the channel-last rows) and stage the matching 64x32
-// slice of W1.  Trunk layer 2 and the 58-row head follow from one 128x64
-// activation tile; the epilogue writes mu', q', s', sh' and Sigma.
+// Every operand x is split into three bf16 parts, x0 = bf16(x),
+// x1 = bf16(x - x0), x2 = bf16(x - x0 - x1), so |x - (x0 + x1 + x2)| is below
+// 2^-26 |x|.  A product keeps the six terms x_i.y_j with i + j <= 2: x0.y0 in
+// one TMEM accumulator and the five smaller terms in a second one (the
+// tensor core aligns addends to the running sum and truncates, so the small
+// terms must not share the big one's accumulator); the dropped terms are
+// below 2^-25 of the result.  Accumulators are fresh for every short K (one
+// plane sample, one layer, one tile of Gaussians) and partial results are
+// added in fp32 on the CUDA cores.  kind::f16 takes K = 16 per instruction,
+// so this issues as many MMAs as a 3xTF32 split; unlike kind::tf32, which
+// returned zero products for MN-major (transposed) operand tiles without
+// swizzle here, it reads such tiles, which the weight gradients need.
+//
+// Persistent CTAs of 256 threads handle 128-Gaussian tiles, two threads per
+// Gaussian (32 of its 64 hidden columns, or 16 of a sample's 32 channels,
+// each).  The 576-wide first layer is streamed one plane sample (32
+// channels) at a time through two shared-memory stages: while the tensor
+// core multiplies sample k, the threads gather and split sample k+1 (16-byte
+// loads of the channel-last rows) and stage the matching 64x32 slice of W1.
+//
+// Every operand tile is stored [row][col] in 8-row x 16-byte core matrices:
+// element (r, c) of a tile with L columns sits at byte
+// (r/8)*16L + (c/8)*128 + (r%8)*16 + (c%8)*2 of each of its three planes.
+// Read with rows as M or N and columns as K this is the canonical K-major
+// layout (LBO 128, SBO 16L); read with columns as M or N and rows as K it is
+// the MN-major one (SBO 128 between 8-column blocks, LBO 16L between 8-row
+// blocks).  A tile written once therefore serves a product and its
+// transpose: the z stage is layer 1's A operand (rows = Gaussians) and the
+// W1 gradient's B operand (K = Gaussians), the W1 stage is layer 1's B
+// operand and dz's transposed B operand, and each activation or delta tile
+// is the A operand of a data gradient and a transposed operand of a weight
+// gradient.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -375,45 +398,109 @@ constexpr int kHexTile = 128;
 constexpr int kHexThreads = 256;
 constexpr uint32_t kHexWait = 1u << 24;
 
+// Byte size of one bf16 plane of an R x L tile.
+constexpr int plane_bytes(int R, int L) { return R * L * 2; }
+
 struct HexTcLayout {
-  static constexpr int A = 0;                      // 2 stages x (hi, lo) [128][32] fp32 = 64 KB; later the H tile
-  static constexpr int A_STAGE = 2 * kHexTile * kHexC * 4;
-  static constexpr int H_LO = kHexTile * kHexH * 4;   // H tile: hi at A, lo at A + H_LO
-  static constexpr int B1 = A + 2 * A_STAGE;       // 2 stages x (hi, lo) [64][32]
-  static constexpr int B1_STAGE = 2 * kHexH * kHexC * 4;
-  static constexpr int W2 = B1 + 2 * B1_STAGE;     // hi, lo [64][64]
-  static constexpr int W3 = W2 + 2 * kHexH * kHexH * 4;   // hi, lo [64][64] (58 rows used)
-  static constexpr int BIAS = W3 + 2 * kHexH * kHexH * 4; // b1 | b2 | b3 (64 each)
-  static constexpr int MISC = BIAS + 3 * kHexH * 4;  // 2 mbarriers + TMEM address
+  static constexpr int Z_PLANE = plane_bytes(kHexTile, kHexC);      // 8 KB
+  static constexpr int Z_STAGE = 3 * Z_PLANE;
+  static constexpr int A = 0;                                      // 2 z stages = 48 KB; later the H tile
+  static constexpr int H_PLANE = plane_bytes(kHexTile, kHexH);     // 16 KB: the H tile fills region A
+  static constexpr int W_PLANE = plane_bytes(kHexH, kHexC);        // 4 KB
+  static constexpr int W_STAGE = 3 * W_PLANE;
+  static constexpr int B1 = A + 2 * Z_STAGE;                       // 2 W1 stages = 24 KB
+  static constexpr int S_PLANE = plane_bytes(kHexH, kHexH);        // 8 KB
+  static constexpr int W2 = B1 + 2 * W_STAGE;                      // [64][64] x 3 planes
+  static constexpr int W3 = W2 + 3 * S_PLANE;                      // [64][64] x 3 planes (58 rows used)
+  static constexpr int BIAS = W3 + 3 * S_PLANE;                    // b1 | b2 | b3 (64 each)
+  static constexpr int MISC = BIAS + 3 * kHexH * 4;                // 2 mbarriers + TMEM address
+  static constexpr int BYTES = MISC + 32;
+  static __device__ __forceinline__ int z(int b) { return A + b * Z_STAGE; }
+  static __device__ __forceinline__ int w(int b) { return B1 + b * W_STAGE; }
+};
+static_assert(3 * HexTcLayout::H_PLANE == 2 * HexTcLayout::Z_STAGE, "H tile must fill the z stages");
+
+// Backward: the forward's regions at the same offsets, a second activation
+// tile T1 in place of the forward's bias block, then the biases and the
+// CTA's bias-gradient sums.  The first activation tile T0 is the forward's H
+// tile (over the z stages).
+struct HexBwdLayout {
+  static constexpr int T1 = HexTcLayout::BIAS;               // [128][64] x 3 planes
+  static constexpr int BIAS = T1 + 3 * HexTcLayout::H_PLANE;  // b1 | b2 | b3
+  static constexpr int BACC = BIAS + 3 * kHexH * 4;           // db1 | db2 | db3 over the CTA's tiles
+  static constexpr int MISC = BACC + 3 * kHexH * 4;           // 2 mbarriers + TMEM address
   static constexpr int BYTES = MISC + 32;
 };
+static_assert(HexBwdLayout::BYTES <= 227 * 1024, "backward tiles exceed the shared memory of one CTA");
 
-// Stores 4 consecutive values of a row (K-major 32-bit tile with K columns,
-// 4-value chunk kc) as tf32 hi and lo parts.
-__device__ __forceinline__ void store_split4(uint8_t* sm, int hi_off, int lo_off, int r, int kc, int K, float4 v) {
-  float h0, h1, h2, h3, l0, l1, l2, l3;
-  tc::split_tf32(v.x, h0, l0);
-  tc::split_tf32(v.y, h1, l1);
-  tc::split_tf32(v.z, h2, l2);
-  tc::split_tf32(v.w, h3, l3);
-  *reinterpret_cast<float4*>(sm + hi_off + tc::kmaj_off32(r, kc, K)) = make_float4(h0, h1, h2, h3);
-  *reinterpret_cast<float4*>(sm + lo_off + tc::kmaj_off32(r, kc, K)) = make_float4(l0, l1, l2, l3);
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// Stores 8 consecutive values of row r (8-column chunk kc of a tile with L
+// columns) as its three bf16 planes (plane = bytes between planes).
+__device__ __forceinline__ void store_split8(uint8_t* sm, int off, int plane, int r, int kc, int L, const float v[8]) {
+  uint32_t p0[4], p1[4], p2[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    const float2 f0 = __bfloat1622float2(h0);
+    const float r0 = v[2 * j] - f0.x, r1 = v[2 * j + 1] - f0.y;
+    const __nv_bfloat162 h1 = __floats2bfloat162_rn(r0, r1);
+    const float2 f1 = __bfloat1622float2(h1);
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(r0 - f1.x, r1 - f1.y);
+    p0[j] = bf2_bits(h0);
+    p1[j] = bf2_bits(h1);
+    p2[j] = bf2_bits(h2);
+  }
+  const uint32_t o = (uint32_t)off + tc::kmaj_off(r, kc, L);
+  *reinterpret_cast<uint4*>(sm + o) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+  *reinterpret_cast<uint4*>(sm + o + plane) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+  *reinterpret_cast<uint4*>(sm + o + 2 * plane) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
 }
 
-// 3xTF32 product over K columns into two fresh accumulators: d_main = A_hi.B_hi
-// and d_corr = A_hi.B_lo + A_lo.B_hi (the dropped lo.lo term is below 2^-21).
-// The tensor core aligns addends to the running sum and truncates, so the
-// small correction terms get an accumulator of their own, and callers keep K
-// short and add the partial results in fp32 on the CUDA cores.
-__device__ __forceinline__ void mma_3xtf32(uint32_t d_main, uint32_t d_corr, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
-                                           uint32_t b_lo, int K, int N) {
-  const uint32_t sbo = (uint32_t)K * 32u;
-  const uint32_t idesc = tc::idesc_tf32_f32(kHexTile, N);
-  for (int s = 0; s < K / 8; ++s) {
-    const uint32_t o = (uint32_t)s * 256u;
-    tc::mma_tf32(d_main, tc::smem_desc(a_hi + o, 128, sbo), tc::smem_desc(b_hi + o, 128, sbo), idesc, s > 0 ? 1u : 0u);
-    tc::mma_tf32(d_corr, tc::smem_desc(a_hi + o, 128, sbo), tc::smem_desc(b_lo + o, 128, sbo), idesc, s > 0 ? 1u : 0u);
-    tc::mma_tf32(d_corr, tc::smem_desc(a_lo + o, 128, sbo), tc::smem_desc(b_hi + o, 128, sbo), idesc, 1u);
+__device__ __forceinline__ void store_split8(uint8_t* sm, int off, int plane, int r, int kc, int L, float4 a, float4 b) {
+  const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  store_split8(sm, off, plane, r, kc, L, v);
+}
+
+// Stores this thread's 32 values (columns half*32 ..) of row r of a 64-column tile.
+__device__ __forceinline__ void store_row32(uint8_t* sm, int off, int r, int half, const float v[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store_split8(sm, off, HexTcLayout::H_PLANE, r, half * 4 + q, kHexH, v + 8 * q);
+}
+
+// One operand of a split product: shared-memory address of plane 0, bytes
+// between planes, descriptor strides, and how far the start address moves
+// per 16-deep K slice.
+struct SplitOp {
+  uint32_t base, plane, lbo, sbo, step;
+};
+// Tile with L columns read K-major (rows are M or N, columns are K).
+__device__ __forceinline__ SplitOp kmajor(uint32_t base, int plane, int L) {
+  return {base, (uint32_t)plane, 128u, 16u * (uint32_t)L, 256u};
+}
+// Tile with L columns read MN-major (columns are M or N, rows are K).
+__device__ __forceinline__ SplitOp mnmajor(uint32_t base, int plane, int L) {
+  return {base, (uint32_t)plane, 16u * (uint32_t)L, 128u, 32u * (uint32_t)L};
+}
+
+// Split product over K into two fresh accumulators: d_main = A0.B0 and
+// d_corr = A0.B1 + A1.B0 + A0.B2 + A2.B0 + A1.B1.
+__device__ __forceinline__ void mma6(uint32_t d_main, uint32_t d_corr, const SplitOp& a, const SplitOp& b, int K,
+                                     uint32_t idesc) {
+  for (int s = 0; s < K / 16; ++s) {
+    uint64_t ad[3], bd[3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      ad[i] = tc::smem_desc(a.base + i * a.plane + s * a.step, a.lbo, a.sbo);
+      bd[i] = tc::smem_desc(b.base + i * b.plane + s * b.step, b.lbo, b.sbo);
+    }
+    const uint32_t acc = s > 0 ? 1u : 0u;
+    tc::mma_f16(d_main, ad[0], bd[0], idesc, acc);
+    tc::mma_f16(d_corr, ad[0], bd[1], idesc, acc);
+    tc::mma_f16(d_corr, ad[1], bd[0], idesc, 1u);
+    tc::mma_f16(d_corr, ad[0], bd[2], idesc, 1u);
+    tc::mma_f16(d_corr, ad[2], bd[0], idesc, 1u);
+    tc::mma_f16(d_corr, ad[1], bd[1], idesc, 1u);
   }
 }
 
@@ -426,6 +513,163 @@ __device__ __forceinline__ void add_partial(uint32_t d_main, uint32_t d_corr, fl
   for (int i = 0; i < 32; ++i) acc[i] += a[i] + b[i];
 }
 
+// Sums over a warp: v[i] holds this lane's value of column i; on return the
+// lane holds the sum over the warp's 32 lanes of column `lane`.  Each of the
+// five exchange rounds halves the columns a lane is responsible for.
+__device__ __forceinline__ float warp_column_sum(float v[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// Commit barriers of the two stages; every commit is waited for exactly once.
+struct HexBars {
+  uint32_t bar0, bar1, ph0, ph1;
+  __device__ __forceinline__ uint32_t addr(int b) const { return b ? bar1 : bar0; }
+  __device__ __forceinline__ bool wait(int b) {
+    const bool ok = tc::mbar_wait_bounded(b ? bar1 : bar0, b ? ph1 : ph0, kHexWait);
+    if (b)
+      ph1 ^= 1u;
+    else
+      ph0 ^= 1u;
+    return ok;
+  }
+};
+
+// Streams the plane samples of one tile through the two stages.  Stage
+// b = k & 1 receives sample k: the 64x32 slice of W1 for the sample and the
+// tile's 128x32 feature block z_k (split), z_k read from zsrc (a saved
+// latent) when given, else sampled from the planes (and then copied to zdst
+// when given).  issue(k, b) runs on thread 0 once the stage is written and
+// its MMAs are committed to stage b's barrier; consume(k, b) runs on every
+// thread once they are done, before the stage takes sample k + 2.  Global
+// loads for sample k + 1 are issued right after sample k's MMAs, so their
+// latency overlaps the tensor core.  Returns false if a wait ran out.
+template <class Issue, class Consume>
+__device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
+                                           const float* __restrict__ W1, const float* __restrict__ zsrc,
+                                           float* __restrict__ zdst, int64_t n, bool valid, const float xt[4],
+                                           HexBars& bars, Issue issue, Consume consume) {
+  using Lay = HexTcLayout;
+  const int tid = threadIdx.x, row = tid & (kHexTile - 1), half = tid / kHexTile;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  float4 wpre[2], cpre[4][4];
+  float cw[4] = {0.f, 0.f, 0.f, 0.f};
+  auto prefetch = [&](int k) {
+    const int r = tid >> 2, c8 = tid & 3;   // W1 slice: 64 rows x 4 chunks of 8
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      wpre[q] = __ldg(reinterpret_cast<const float4*>(W1 + (size_t)r * IN + k * kHexC) + 2 * c8 + q);
+    if (!valid) return;
+    if (zsrc) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        cpre[0][q] = __ldg(reinterpret_cast<const float4*>(zsrc + n * IN + k * kHexC) + half * 4 + q);
+    } else {
+      const PlaneSample ps = plane_sample(xt, hp, k);
+      cw[0] = ps.w00;
+      cw[1] = ps.w01;
+      cw[2] = ps.w10;
+      cw[3] = ps.w11;
+      const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cpre[c][q] = __ldg(reinterpret_cast<const float4*>(planes + off[c]) + half * 4 + q);
+    }
+  };
+  prefetch(0);
+  for (int k = 0; k < NS; ++k) {
+    const int b = k & 1;
+    if (k >= 2) {   // sample k-2 used this stage: take its results, then refill
+      const bool ok = bars.wait(b);
+      if (__syncthreads_or(!ok)) return false;
+      tc::fence_after_sync();
+      consume(k - 2, b);
+    }
+    store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, wpre[0], wpre[1]);
+    float4 z4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      z4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (valid) {
+        if (zsrc) {
+          z4[q] = cpre[0][q];
+        } else {
+          z4[q].x = cw[0] * cpre[0][q].x + cw[1] * cpre[1][q].x + cw[2] * cpre[2][q].x + cw[3] * cpre[3][q].x;
+          z4[q].y = cw[0] * cpre[0][q].y + cw[1] * cpre[1][q].y + cw[2] * cpre[2][q].y + cw[3] * cpre[3][q].y;
+          z4[q].z = cw[0] * cpre[0][q].z + cw[1] * cpre[1][q].z + cw[2] * cpre[2][q].z + cw[3] * cpre[3][q].z;
+          z4[q].w = cw[0] * cpre[0][q].w + cw[1] * cpre[1][q].w + cw[2] * cpre[2][q].w + cw[3] * cpre[3][q].w;
+          if (zdst) reinterpret_cast<float4*>(zdst + n * IN + k * kHexC)[half * 4 + q] = z4[q];
+        }
+      }
+    }
+    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2, kHexC, z4[0], z4[1]);
+    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z4[2], z4[3]);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      tc::fence_after_sync();
+      issue(k, b);
+      tc::mma_commit(bars.addr(b));
+    }
+    if (k + 1 < NS) prefetch(k + 1);
+  }
+  for (int k = (NS >= 2 ? NS - 2 : 0); k < NS; ++k) {   // the last two samples
+    const int b = k & 1;
+    const bool ok = bars.wait(b);
+    if (__syncthreads_or(!ok)) return false;
+    tc::fence_after_sync();
+    consume(k, b);
+  }
+  return true;
+}
+
+// Makes every thread's shared-memory tile writes visible to the tensor core
+// and lines the threads up before thread 0 issues the next MMAs.
+__device__ __forceinline__ void tiles_ready() {
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+}
+
+// Stages W2 and W3 (split, W3 padded with zero rows to 64) and the three
+// bias vectors, once per CTA.
+__device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, const float* __restrict__ W2g,
+                                                   const float* __restrict__ b1, const float* __restrict__ b2,
+                                                   const float* __restrict__ W3g, const float* __restrict__ b3) {
+  using Lay = HexTcLayout;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kHexH * (kHexH / 8); i += kHexThreads) {
+    const int r = i / (kHexH / 8), kc = i % (kHexH / 8);
+    const float4* w2 = reinterpret_cast<const float4*>(W2g + r * kHexH) + 2 * kc;
+    store_split8(sm, Lay::W2, Lay::S_PLANE, r, kc, kHexH, __ldg(w2), __ldg(w2 + 1));
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (r < kHexHead) {
+      const float4* w3 = reinterpret_cast<const float4*>(W3g + r * kHexH) + 2 * kc;
+      a = __ldg(w3);
+      b = __ldg(w3 + 1);
+    }
+    store_split8(sm, Lay::W3, Lay::S_PLANE, r, kc, kHexH, a, b);
+  }
+  float* bias = reinterpret_cast<float*>(sm + bias_off);
+  for (int o = tid; o < kHexH; o += kHexThreads) {
+    bias[o] = __ldg(b1 + o);
+    bias[kHexH + o] = __ldg(b2 + o);
+    bias[2 * kHexH + o] = o < kHexHead ? __ldg(b3 + o) : 0.f;
+  }
+}
+
 __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
@@ -434,7 +678,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   extern __shared__ __align__(1024) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & (kHexTile - 1), half = tid / kHexTile;
-  const int IN = hp.in_dim, NS = hp.n_samples;
+  const int IN = hp.in_dim;
   const float* W1 = W;
   const float* b1 = W1 + kHexH * IN;
   const float* W2g = b1 + kHexH;
@@ -443,22 +687,9 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   const float* b3 = W3g + kHexHead * kHexH;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::MISC + 16);
   const uint32_t mbar0 = tc::smem_u32(sm + Lay::MISC), mbar1 = mbar0 + 8;
-  float* bias = reinterpret_cast<float*>(sm + Lay::BIAS);
+  const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
 
-  // ---- W2, W3 (split) and biases, once per CTA ----
-  for (int i = tid; i < kHexH * (kHexH / 4); i += kHexThreads) {
-    const int r = i / (kHexH / 4), kc = i % (kHexH / 4);
-    store_split4(sm, Lay::W2, Lay::W2 + kHexH * kHexH * 4, r, kc, kHexH,
-                 __ldg(reinterpret_cast<const float4*>(W2g + r * kHexH) + kc));
-    const float4 w3 = r < kHexHead ? __ldg(reinterpret_cast<const float4*>(W3g + r * kHexH) + kc)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    store_split4(sm, Lay::W3, Lay::W3 + kHexH * kHexH * 4, r, kc, kHexH, w3);
-  }
-  for (int o = tid; o < kHexH; o += kHexThreads) {
-    bias[o] = __ldg(b1 + o);
-    bias[kHexH + o] = __ldg(b2 + o);
-    bias[2 * kHexH + o] = o < kHexHead ? __ldg(b3 + o) : 0.f;
-  }
+  stage_small_layers(sm, Lay::BIAS, W2g, b1, b2, W3g, b3);
   if (warp == 0) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
     tc::tmem_relinquish();
@@ -473,21 +704,14 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
-  // TMEM regions of 64 columns: R0..R3.  Plane sample k accumulates into
-  // (R0, R1) when k is even and (R2, R3) when odd; layer 2 uses (R0, R1) and
-  // the head (R2, R3).
-  const uint32_t R[4] = {tmem, tmem + 64, tmem + 128, tmem + 192};
-  uint32_t ph0 = 0, ph1 = 0;
-  bool failed = false;
-  auto wait_bar = [&](int b) -> bool {
-    const uint32_t bar = b ? mbar1 : mbar0;
-    uint32_t& ph = b ? ph1 : ph0;
-    const bool ok = tc::mbar_wait_bounded(bar, ph, kHexWait);
-    ph ^= 1u;
-    return ok;
-  };
-  const uint32_t sA = tc::smem_u32(sm + Lay::A), sB1 = tc::smem_u32(sm + Lay::B1);
   const uint32_t col = (uint32_t)(half * 32);
+  const uint32_t sbase = tc::smem_u32(sm);
+  const SplitOp H = kmajor(sbase + Lay::A, Lay::H_PLANE, kHexH);
+  // TMEM: plane sample k accumulates into columns [128b, 128b + 128) of stage
+  // b = k & 1 (main, then correction); layer 2 reuses stage 0's columns and
+  // the head stage 1's.
+  HexBars bars{mbar0, mbar1, 0u, 0u};
+  bool failed = false;
 
   for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
     const int64_t n = tile * kHexTile + row;
@@ -498,129 +722,53 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc1[i] = 0.f;
     // ---- layer 1, streamed over the plane samples ----
-    // Registers hold sample k+1's global data (its W1 slice and its four
-    // corner rows) while sample k is multiplied, so load latency overlaps
-    // the MMAs and the barriers.
-    float4 wpre[2], cpre[4][4];
-    float cw[4];
-    auto prefetch = [&](int k) {
-      const int r = tid >> 2, c2 = (tid & 3) * 2;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) wpre[q] = __ldg(reinterpret_cast<const float4*>(W1 + (size_t)r * IN + k * kHexC) + c2 + q);
-      if (valid) {
-        const PlaneSample ps = plane_sample(xt, hp, k);
-        cw[0] = ps.w00; cw[1] = ps.w01; cw[2] = ps.w10; cw[3] = ps.w11;
-        const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) cpre[c][q] = __ldg(reinterpret_cast<const float4*>(planes + off[c]) + half * 4 + q);
-      }
+    auto issue = [&](int, int b) {
+      mma6(tmem + 128 * b, tmem + 128 * b + 64, kmajor(sbase + Lay::z(b), Lay::Z_PLANE, kHexC),
+           kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
-    prefetch(0);
-    for (int k = 0; k < NS; ++k) {
-      const int b = k & 1;
-      if (k >= 2) {   // sample k-2 used this stage: fold its partial sums in, then reuse
-        const bool ok = wait_bar(b);
-        if (__syncthreads_or(!ok)) { failed = true; break; }
-        tc::fence_after_sync();
-        add_partial(R[2 * b] + lane + col, R[2 * b + 1] + lane + col, acc1);
-      }
-      const int a_hi = Lay::A + b * Lay::A_STAGE, a_lo = a_hi + kHexTile * kHexC * 4;
-      const int w_hi = Lay::B1 + b * Lay::B1_STAGE, w_lo = w_hi + kHexH * kHexC * 4;
-      {
-        const int r = tid >> 2, c2 = (tid & 3) * 2;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) store_split4(sm, w_hi, w_lo, r, c2 + q, kHexC, wpre[q]);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int c4 = half * 4 + q;
-        float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) {
-          z4.x = cw[0] * cpre[0][q].x + cw[1] * cpre[1][q].x + cw[2] * cpre[2][q].x + cw[3] * cpre[3][q].x;
-          z4.y = cw[0] * cpre[0][q].y + cw[1] * cpre[1][q].y + cw[2] * cpre[2][q].y + cw[3] * cpre[3][q].y;
-          z4.z = cw[0] * cpre[0][q].z + cw[1] * cpre[1][q].z + cw[2] * cpre[2][q].z + cw[3] * cpre[3][q].z;
-          z4.w = cw[0] * cpre[0][q].w + cw[1] * cpre[1][q].w + cw[2] * cpre[2][q].w + cw[3] * cpre[3][q].w;
-          if (latent) reinterpret_cast<float4*>(latent + n * IN + k * kHexC)[c4] = z4;
-        }
-        store_split4(sm, a_hi, a_lo, row, c4, kHexC, z4);
-      }
-      tc::fence_proxy_async();
-      tc::fence_before_sync();
-      __syncthreads();
-      if (tid == 0) {
-        tc::fence_after_sync();
-        mma_3xtf32(R[2 * b], R[2 * b + 1], sA + a_hi, sA + a_lo, sB1 + (w_hi - Lay::B1), sB1 + (w_lo - Lay::B1), kHexC,
-                   kHexH);
-        tc::mma_commit(b ? mbar1 : mbar0);
-      }
-      if (k + 1 < NS) prefetch(k + 1);
+    auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
+    if (!hex_stream(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
+      failed = true;
+      break;
     }
-    if (failed) break;
-    // the last two samples (in the order their barriers completed)
-    for (int k = (NS >= 2 ? NS - 2 : 0); k < NS; ++k) {
-      const int b = k & 1;
-      const bool ok = wait_bar(b);
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      tc::fence_after_sync();
-      add_partial(R[2 * b] + lane + col, R[2 * b + 1] + lane + col, acc1);
-    }
-    if (failed) break;
-    // ---- h1 = relu(sum + b1) -> split H tile (over the A stages) ----
+    // ---- h1 = relu(sum + b1) -> H tile (over the z stages) ----
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float4 h;
-      h.x = fmaxf(acc1[4 * q] + bias[half * 32 + 4 * q], 0.f);
-      h.y = fmaxf(acc1[4 * q + 1] + bias[half * 32 + 4 * q + 1], 0.f);
-      h.z = fmaxf(acc1[4 * q + 2] + bias[half * 32 + 4 * q + 2], 0.f);
-      h.w = fmaxf(acc1[4 * q + 3] + bias[half * 32 + 4 * q + 3], 0.f);
-      store_split4(sm, Lay::A, Lay::A + Lay::H_LO, row, half * 8 + q, kHexH, h);
-    }
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- layer 2 into (R0, R1) ----
+    for (int i = 0; i < 32; ++i) acc1[i] = fmaxf(acc1[i] + bias[half * 32 + i], 0.f);
+    store_row32(sm, Lay::A, row, half, acc1);
+    tiles_ready();
+    // ---- layer 2 into stage 0's columns ----
     if (tid == 0) {
       tc::fence_after_sync();
-      mma_3xtf32(R[0], R[1], sA, sA + Lay::H_LO, tc::smem_u32(sm + Lay::W2), tc::smem_u32(sm + Lay::W2) + kHexH * kHexH * 4,
-                 kHexH, kHexH);
+      mma6(tmem, tmem + 64, H, kmajor(sbase + Lay::W2, Lay::S_PLANE, kHexH), kHexH,
+           tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
       tc::mma_commit(mbar0);
     }
-    if (__syncthreads_or(!wait_bar(0))) { failed = true; break; }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
     tc::fence_after_sync();
     {
       float v[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      add_partial(R[0] + lane + col, R[1] + lane + col, v);
+      add_partial(tmem + lane + col, tmem + 64 + lane + col, v);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 h;
-        h.x = fmaxf(v[4 * q] + bias[kHexH + half * 32 + 4 * q], 0.f);
-        h.y = fmaxf(v[4 * q + 1] + bias[kHexH + half * 32 + 4 * q + 1], 0.f);
-        h.z = fmaxf(v[4 * q + 2] + bias[kHexH + half * 32 + 4 * q + 2], 0.f);
-        h.w = fmaxf(v[4 * q + 3] + bias[kHexH + half * 32 + 4 * q + 3], 0.f);
-        store_split4(sm, Lay::A, Lay::A + Lay::H_LO, row, half * 8 + q, kHexH, h);
-      }
+      for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i] + bias[kHexH + half * 32 + i], 0.f);
+      store_row32(sm, Lay::A, row, half, v);
     }
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- head (58 rows, padded to 64) into (R2, R3) ----
+    tiles_ready();
+    // ---- head (58 rows, padded to 64) into stage 1's columns ----
     if (tid == 0) {
       tc::fence_after_sync();
-      mma_3xtf32(R[2], R[3], sA, sA + Lay::H_LO, tc::smem_u32(sm + Lay::W3), tc::smem_u32(sm + Lay::W3) + kHexH * kHexH * 4,
-                 kHexH, kHexH);
+      mma6(tmem + 128, tmem + 192, H, kmajor(sbase + Lay::W3, Lay::S_PLANE, kHexH), kHexH,
+           tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
       tc::mma_commit(mbar0);
     }
-    if (__syncthreads_or(!wait_bar(0))) { failed = true; break; }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
     tc::fence_after_sync();
     {
       float y[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = bias[2 * kHexH + half * 32 + i];
-      add_partial(R[2] + lane + col, R[3] + lane + col, y);
+      add_partial(tmem + 128 + lane + col, tmem + 192 + lane + col, y);
       tc::fence_before_sync();
       if (valid) {
         if (half == 0) {
@@ -651,14 +799,317 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
 
   if (failed) {
     if (tid == 0) atomicExch(&g_hex_device_error, 1);
-    wait_bar(0);
-    wait_bar(1);
+    bars.wait(0);
+    bars.wait(1);
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// RMW of 32 consecutive floats of a workspace slot row.
+__device__ __forceinline__ void slot_add32(float* dst, const float a[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float4 v = d[q];
+    v.x += a[4 * q];
+    v.y += a[4 * q + 1];
+    v.z += a[4 * q + 2];
+    v.w += a[4 * q + 3];
+    d[q] = v;
+  }
+}
+
+// Backward, one 128-Gaussian tile per step of a persistent CTA:
+//   1. forward again (layer 1 streamed as in the forward, z from the saved
+//      latent when given), keeping h1 and h2 in registers;
+//   2. the head's rows 0..15 give q' and s', and with them the head adjoint
+//      dy (58 values, zero padded to 64);
+//   3. dh2 = (dy W3) * [h2 > 0] and dW3 += dy^T h2, then
+//      dh1 = (dh2 W2) * [h1 > 0] and dW2 += dh2^T h1 (one MMA group each);
+//   4. per plane sample k, dz_k = dh1 W1_k and dW1_k += dh1^T z_k; dz_k is
+//      spread over the sample's four bilinear corners with fp32 vector
+//      atomics.
+// Weight gradients are partial sums over one tile (K = 128, fresh
+// accumulators) added in fp32 to the CTA's workspace slot, and bias
+// gradients are warp column sums gathered in shared memory, so they do not
+// depend on scheduling.  TMEM: stages as in the forward, plus the 64-row
+// weight-gradient accumulators at columns 256 (main) and 320 (correction).
+__global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
+    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
+    const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
+    const float* __restrict__ logs_can, const float* __restrict__ latent, HexGradPtrs go,
+    float* __restrict__ grad_planes, float* __restrict__ ws, int n_params) {
+  using Lay = HexTcLayout;
+  using BL = HexBwdLayout;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int row = tid & (kHexTile - 1), half = tid / kHexTile;
+  const int IN = hp.in_dim;
+  const float* W1 = W;
+  const float* b1 = W1 + kHexH * IN;
+  const float* W2g = b1 + kHexH;
+  const float* b2 = W2g + kHexH * kHexH;
+  const float* W3g = b2 + kHexH;
+  const float* b3 = W3g + kHexHead * kHexH;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
+  float* sW1 = slot;
+  float* sb1 = sW1 + kHexH * IN;
+  float* sW2 = sb1 + kHexH;
+  float* sb2 = sW2 + kHexH * kHexH;
+  float* sW3 = sb2 + kHexH;
+  float* sb3 = sW3 + kHexHead * kHexH;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + BL::MISC + 16);
+  const uint32_t mbar0 = tc::smem_u32(sm + BL::MISC), mbar1 = mbar0 + 8;
+  const float* bias = reinterpret_cast<const float*>(sm + BL::BIAS);
+  float* bacc = reinterpret_cast<float*>(sm + BL::BACC);
+
+  for (int p = tid; p < n_params; p += kHexThreads) slot[p] = 0.f;
+  stage_small_layers(sm, BL::BIAS, W2g, b1, b2, W3g, b3);
+  for (int o = tid; o < 3 * kHexH; o += kHexThreads) bacc[o] = 0.f;
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(mbar0, 1);
+    tc::mbar_init(mbar1, 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t col = (uint32_t)(half * 32);
+  const uint32_t sbase = tc::smem_u32(sm);
+  const int T0 = Lay::A;
+  const SplitOp T0k = kmajor(sbase + T0, Lay::H_PLANE, kHexH), T0t = mnmajor(sbase + T0, Lay::H_PLANE, kHexH);
+  const SplitOp T1k = kmajor(sbase + BL::T1, Lay::H_PLANE, kHexH), T1t = mnmajor(sbase + BL::T1, Lay::H_PLANE, kHexH);
+  const SplitOp W2k = kmajor(sbase + Lay::W2, Lay::S_PLANE, kHexH), W2t = mnmajor(sbase + Lay::W2, Lay::S_PLANE, kHexH);
+  const SplitOp W3k = kmajor(sbase + Lay::W3, Lay::S_PLANE, kHexH), W3t = mnmajor(sbase + Lay::W3, Lay::S_PLANE, kHexH);
+  const uint32_t RW = tmem + 256;
+  // Row m of a 64-row accumulator sits in TMEM lane (m % 16) + 32 (m / 16):
+  // warp w reads rows 16 (w % 4) + lane for lanes below 16.
+  const int wrow = (warp & 3) * 16 + lid;
+  const bool wrow_ok = lid < 16;
+  HexBars bars{mbar0, mbar1, 0u, 0u};
+  bool failed = false;
+
+  for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
+    const int64_t n = tile * kHexTile + row;
+    const bool valid = n < N;
+    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) hex_normalise(mu, frame, n, hp, xt);
+    // ---- 1. forward ----
+    float h1[32], h2[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h1[i] = 0.f;
+    auto issue1 = [&](int, int b) {
+      mma6(tmem + 128 * b, tmem + 128 * b + 64, kmajor(sbase + Lay::z(b), Lay::Z_PLANE, kHexC),
+           kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+    };
+    auto consume1 = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, h1); };
+    if (!hex_stream(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
+      failed = true;
+      break;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h1[i] = fmaxf(h1[i] + bias[half * 32 + i], 0.f);
+    store_row32(sm, T0, row, half, h1);
+    tiles_ready();
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma6(tmem, tmem + 64, T0k, W2k, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
+    tc::fence_after_sync();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h2[i] = 0.f;
+    add_partial(tmem + lane + col, tmem + 64 + lane + col, h2);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h2[i] = fmaxf(h2[i] + bias[kHexH + half * 32 + i], 0.f);
+    store_row32(sm, BL::T1, row, half, h2);
+    tiles_ready();
+    // head rows 0..15 (d_mu, d_q, d_logs) into stage 1's columns
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma6(tmem + 128, tmem + 192, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, 16, false, false));
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
+    tc::fence_after_sync();
+    // ---- 2. head adjoint ----
+    float dy[32];
+    if (half == 0) {
+      float a[16], c[16];
+      tc::tmem_ld16(tmem + 128 + lane, a);
+      tc::tmem_ld16(tmem + 192 + lane, c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dy[i] = 0.f;
+      if (valid) {
+        float qh[4], q[4], s[3], gc[6], ds[3], dq[4], dqh[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + (a[3 + i] + c[3 + i] + bias[2 * kHexH + 3 + i]);
+        const float nrm = normalise_quat(qh, q);
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+          s[i] = expf(__ldg(logs_can + 3 * n + i) + (a[7 + i] + c[7 + i] + bias[2 * kHexH + 7 + i]));
+#pragma unroll
+        for (int i = 0; i < 6; ++i) gc[i] = g_or0(go.cov, 6 * n + i);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) ds[i] = g_or0(go.scale, 3 * n + i);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dq[i] = g_or0(go.rot, 4 * n + i);
+        covariance_backward(s, q, gc, ds, dq);
+        normalise_quat_backward(q, nrm, dq, dqh);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) dy[i] = g_or0(go.mu, 3 * n + i);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dy[3 + i] = dqh[i];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) dy[7 + i] = ds[i] * s[i];
+#pragma unroll
+        for (int i = 10; i < 32; ++i) dy[i] = g_or0(go.sh, 48 * n + (i - 10));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dy[i] = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
+    }
+    tc::fence_before_sync();
+    store_row32(sm, T0, row, half, dy);
+    atomicAdd(bacc + 2 * kHexH + half * 32 + lid, warp_column_sum(dy));
+    tiles_ready();
+    // ---- 3. dh2 = dy W3 (masked), dW3 = dy^T h2 ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma6(tmem, tmem + 64, T0k, W3t, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, true));
+      mma6(RW, RW + 64, T0t, T1t, kHexTile, tc::idesc_bf16_f32(64, kHexH, true, true));
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
+    tc::fence_after_sync();
+    float d[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) d[i] = 0.f;
+    add_partial(tmem + lane + col, tmem + 64 + lane + col, d);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) d[i] = h2[i] > 0.f ? d[i] : 0.f;
+    {
+      float a[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = 0.f;
+      add_partial(RW + lane + (warp >> 2) * 32, RW + 64 + lane + (warp >> 2) * 32, a);
+      if (wrow_ok && wrow < kHexHead) slot_add32(sW3 + wrow * kHexH + (warp >> 2) * 32, a);
+    }
+    tc::fence_before_sync();
+    store_row32(sm, T0, row, half, d);
+    store_row32(sm, BL::T1, row, half, h1);
+    {
+      float t[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) t[i] = d[i];
+      atomicAdd(bacc + kHexH + half * 32 + lid, warp_column_sum(t));
+    }
+    tiles_ready();
+    // ---- dh1 = dh2 W2 (masked), dW2 = dh2^T h1 ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      mma6(tmem, tmem + 64, T0k, W2t, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, true));
+      mma6(RW, RW + 64, T0t, T1t, kHexTile, tc::idesc_bf16_f32(64, kHexH, true, true));
+      tc::mma_commit(mbar0);
+    }
+    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
+    tc::fence_after_sync();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) d[i] = 0.f;
+    add_partial(tmem + lane + col, tmem + 64 + lane + col, d);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) d[i] = h1[i] > 0.f ? d[i] : 0.f;
+    {
+      float a[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = 0.f;
+      add_partial(RW + lane + (warp >> 2) * 32, RW + 64 + lane + (warp >> 2) * 32, a);
+      if (wrow_ok) slot_add32(sW2 + wrow * kHexH + (warp >> 2) * 32, a);
+    }
+    tc::fence_before_sync();
+    store_row32(sm, BL::T1, row, half, d);
+    atomicAdd(bacc + half * 32 + lid, warp_column_sum(d));
+    // ---- 4. per plane sample: dz_k = dh1 W1_k, dW1_k = dh1^T z_k ----
+    // Stage b's TMEM columns: dz main | dz correction | dW1 main | dW1 correction (32 each).
+    auto issue2 = [&](int, int b) {
+      const uint32_t S = tmem + 128 * b;
+      mma6(S, S + 32, T1k, mnmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexH,
+           tc::idesc_bf16_f32(kHexTile, kHexC, false, true));
+      mma6(S + 64, S + 96, T1t, mnmajor(sbase + Lay::z(b), Lay::Z_PLANE, kHexC), kHexTile,
+           tc::idesc_bf16_f32(64, kHexC, true, true));
+    };
+    auto consume2 = [&](int k, int b) {
+      const uint32_t S = tmem + 128 * b;
+      float a[16], c[16];
+      tc::tmem_ld16(S + lane + half * 16, a);
+      tc::tmem_ld16(S + 32 + lane + half * 16, c);
+      if (valid) {
+        const PlaneSample ps = plane_sample(xt, hp, k);
+        const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
+        const float w[4] = {ps.w00, ps.w01, ps.w10, ps.w11};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a[i] += c[i];
+#pragma unroll
+        for (int cn = 0; cn < 4; ++cn) {
+          float4* g = reinterpret_cast<float4*>(grad_planes + off[cn]) + half * 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            atomicAdd(g + q, make_float4(w[cn] * a[4 * q], w[cn] * a[4 * q + 1], w[cn] * a[4 * q + 2],
+                                         w[cn] * a[4 * q + 3]));
+        }
+      }
+      tc::tmem_ld16(S + 64 + lane + (warp >> 2) * 16, a);
+      tc::tmem_ld16(S + 96 + lane + (warp >> 2) * 16, c);
+      tc::fence_before_sync();
+      if (wrow_ok) {
+        float4* dst = reinterpret_cast<float4*>(sW1 + (size_t)wrow * IN + k * kHexC + (warp >> 2) * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float4 v = dst[q];
+          v.x += a[4 * q] + c[4 * q];
+          v.y += a[4 * q + 1] + c[4 * q + 1];
+          v.z += a[4 * q + 2] + c[4 * q + 2];
+          v.w += a[4 * q + 3] + c[4 * q + 3];
+          dst[q] = v;
+        }
+      }
+    };
+    if (!hex_stream(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
+      failed = true;
+      break;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+  }
+
+  if (failed) {
+    if (tid == 0) atomicExch(&g_hex_device_error, 1);
+    bars.wait(0);
+    bars.wait(1);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!failed)
+    for (int o = tid; o < kHexH; o += kHexThreads) {
+      sb1[o] += bacc[o];
+      sb2[o] += bacc[kHexH + o];
+      if (o < kHexHead) sb3[o] += bacc[2 * kHexH + o];
+    }
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -774,7 +1225,7 @@ extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, i
 
 extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
                                    const float* planes, const float* weights, const float* q_can,
-                                   const float* logs_can, const float* sh_can,
+                                   const float* logs_can, const float* sh_can, const float* latent,
                                    const spin4d_hex_output_grads* grad_out, float* grad_planes,
                                    float* grad_weights, void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
   (void)sh_can;   // sh' = sh_can + d_sh: the upstream sh gradient flows through unchanged
@@ -782,19 +1233,48 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_planes || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_planes, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256)) return SPIN4D_ERR_INVALID;
+  if (latent && !aligned(latent, 16)) return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_hexplane_bwd_workspace(h, N)) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_hexplane_bwd")) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
   HexGradPtrs go{grad_out->mu, grad_out->rot, grad_out->scale, grad_out->sh, grad_out->cov};
   const int n_params = (int)spin4d_hexplane_param_count(h);
-  const int blocks = hex_bwd_blocks(N);
   cudaStream_t s = (cudaStream_t)stream;
-  const int smem = (4 * kHexH + kHexHead + kHexC) * kHexBwdBlock * (int)sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(hexplane_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return cuda_status(e);
-  hexplane_bwd_kernel<<<blocks, kHexBwdBlock, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, go,
-                                                      grad_planes, static_cast<float*>(workspace), n_params);
-  SPIN4D_CHECK(launch_status());
+  int blocks = 0;
+  {
+    // tensor cores, 3xTF32: one CTA per SM (it holds 512 TMEM columns)
+    static bool configured[64] = {false};
+    static bool usable[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int smem = HexBwdLayout::BYTES;
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(hexplane_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_bwd_tc_kernel, kHexThreads, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      usable[dev] = occ == 1;
+      configured[dev] = true;
+    }
+    if (usable[dev]) {
+      blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
+      hexplane_bwd_tc_kernel<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can,
+                                                              latent, go, grad_planes, static_cast<float*>(workspace),
+                                                              n_params);
+      SPIN4D_CHECK(launch_status());
+    }
+  }
+  if (blocks == 0) {
+    // fp32 SIMT fallback (the saved latent is not used)
+    blocks = hex_bwd_blocks(N);
+    const int smem = (4 * kHexH + kHexHead + kHexC) * kHexBwdBlock * (int)sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(hexplane_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    hexplane_bwd_kernel<<<blocks, kHexBwdBlock, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, go,
+                                                        grad_planes, static_cast<float*>(workspace), n_params);
+    SPIN4D_CHECK(launch_status());
+  }
   hex_reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(static_cast<float*>(workspace), blocks, n_params,
                                                           grad_weights);
   return launch_status();

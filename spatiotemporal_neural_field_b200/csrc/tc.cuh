@@ -43,37 +43,11 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
-// D (+)= A . B^T with tf32 operands (fp32 bit patterns in shared memory; the
-// tensor core reads the top 19 bits), fp32 accumulate, K = 8 per instruction.
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Instruction descriptor, kind::tf32: tf32 A and B (both K-major), fp32 D.
-__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// x = hi + lo with hi a tf32 value (10 explicit mantissa bits, rounded to
-// nearest) and lo the exact fp32 remainder: the 3xTF32 split.
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-  uint32_t h;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
-  hi = __uint_as_float(h);
-  lo = x - hi;
-}
-
-// Byte offset of (row r, 4-element chunk kc) in a K-major tile whose rows hold
-// K 32-bit values: 8-row x 16-byte core matrices, LBO = 128 bytes along K,
-// SBO = K * 32 bytes between 8-row groups.
-__host__ __device__ __forceinline__ uint32_t kmaj_off32(int r, int kc, int K) {
-  return (uint32_t)((r >> 3) * (K * 32) + kc * 128 + (r & 7) * 16);
+// Instruction descriptor, kind::f16 with bf16 A and B and fp32 D; a_mn / b_mn
+// select MN-major (transposed) reads of A / B.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Arrive on `mbar` once every tcgen05.mma issued so far by this thread is done.

@@ -82,7 +82,7 @@ _SIGS = {
     "spin4d_hexplane_param_count": (c_i64, [P(HexDesc)]),
     "spin4d_hexplane_fwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, HexOutputs, c_vp]),
     "spin4d_hexplane_bwd_workspace": (c_sz, [P(HexDesc), c_i64]),
-    "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp,
+    "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                     P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_debug_corners": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
     "spin4d_check_device_errors": (c_i32, [c_i32]),
@@ -284,7 +284,8 @@ def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=
     return out
 
 
-def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, stream=None):
+def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, latent=None,
+                 stream=None):
     N = inp["mu"].shape[0]
     need = int(lib.spin4d_hexplane_bwd_workspace(ctypes.byref(h), N))
     if workspace is None:
@@ -292,7 +293,7 @@ def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weig
     go = HexOutputGrads(*(_ptr(grads.get(k)) for k, _ in HEX_KEYS))
     _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
                                                           _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
-                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]),
+                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), _ptr(latent),
                                                           ctypes.byref(go), _ptr(grad_planes), _ptr(grad_weights),
                                                           _ptr(workspace), workspace.numel(), _stream(stream)))
 

@@ -120,6 +120,11 @@ def test_unsupported_hexplane_shape(sp):
     inp = [FAKE] * 2
     assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
                                    sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
+    # supported shape, misaligned saved latent for the backward
+    h = sp.hex_desc()
+    go = sp.HexOutputGrads()
+    assert lib.spin4d_hexplane_bwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4,
+                                   ctypes.byref(go), FAKE, FAKE, FAKE, 1 << 40, None) == sp.ERR_INVALID
 
 
 def test_fault_injection_hook_in_subprocess(sp):

@@ -494,9 +494,11 @@ def run_ncu_case(name):
         grads = {k: torch.randn((n, wd), device=dev) for k, wd in S.HEX_OUT_WIDTHS.items()}
         gp = torch.zeros(hx.n_plane_floats(), device=dev)
         gw = torch.zeros(hx.n_params(), device=dev)
-        for _ in range(3):
-            sp.hexplane_fwd(h, inp, planes, weights)
-            sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw)
+        out = {k: torch.empty((n, wd), device=dev) for k, wd in sp.HEX_KEYS}
+        out["latent"] = torch.empty((n, hx.in_dim), device=dev)
+        for _ in range(3):   # a training step: forward saving the latent, backward reading it
+            sp.hexplane_fwd(h, inp, planes, weights, out=out)
+            sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, latent=out["latent"])
     else:
         grid, mlp = w["grid"], w["mlp"]
         g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)

@@ -47,6 +47,11 @@ def parse():
     p.add_argument("--no-fwd-bwd", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=150_000, help="positions the oracle decodes for cpu_baseline")
     p.add_argument("--no-probe", action="store_true", help="skip the random-gather ceiling measurement")
+    p.add_argument("--workloads", action="store_true",
+                   help="time every workload (fwd, and fwd+bwd where trained) and the device ceilings; "
+                        "one JSON line each")
+    p.add_argument("--cpu-workloads", action="store_true",
+                   help="time the oracle on every workload (1 thread and all cores); one JSON line each")
     p.add_argument("--ncu-case", default=None,
                    help="profiling driver: run a few untimed launches of one workload and exit "
                         "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32)")
@@ -476,6 +481,208 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def device_ceilings(sp, torch, dev):
+    """Measured ceilings of one GPU: random 32-byte-sector and random 128-byte
+    line gather rates and sequential read bandwidth for an L2-resident
+    (32 MiB) and an HBM-resident (4 GiB) buffer, and the fp32 FMA rate."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def best(fn, reps=4):
+        rate = 0.0
+        for it in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            units = fn(it)
+            b.record()
+            torch.cuda.synchronize()
+            if it:
+                rate = max(rate, units / (a.elapsed_time(b) * 1e-3))
+        return rate
+
+    out = {}
+    for name, nbytes, lpt in (("l2", 32 << 20, 4096), ("hbm", 4 << 30, 1024)):
+        buf = torch.ones(nbytes // 4, dtype=torch.int32, device=dev)
+        out[name + "_random_sector_per_s"] = best(lambda it: sp.probe_gather(buf, 16, lpt, 4 * sms, seed=it + 1))
+        out[name + "_random_line128_per_s"] = best(lambda it: sp.probe_gather(buf, 128, lpt, 4 * sms, seed=it + 1))
+        passes = 64 if name == "l2" else 2
+        out[name + "_sequential_bytes_per_s"] = best(lambda it: sp.probe_stream(buf, passes, 4 * sms))
+        del buf
+    out["fp32_fma_flop_per_s"] = best(lambda it: sp.probe_fma(1 << 16, 8 * sms, dev))
+    return out
+
+
+def run_workloads(args):
+    """Every workload of the build on one GPU: events around each launch (or
+    launch pair), L2 flushed before each, median of the timed reps."""
+    import torch
+    from spatiotemporal_neural_field_b200 import build as _b
+    _b.build()
+    from spatiotemporal_neural_field_b200 import spin4d as sp
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ceil = device_ceilings(sp, torch, dev)
+    print(json.dumps({"ceilings": ceil}), flush=True)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def emit(name, what, n, ms, **extra):
+        line = {"workload": name, "pass": what, "positions": n, "ms": ms, "positions_per_s": n / (ms * 1e-3)}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+    # decoder workloads
+    for name in ("tiny_fp32", "sports_frame_fp16", "sports_train_fp16", "stress_fp16_gate"):
+        w = S.WORKLOADS[name]
+        grid, mlp = w["grid"], w["mlp"]
+        g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+        if name == "tiny_fp32":
+            n, pos = w["N"], S.uniform_positions(w["N"])
+        elif name == "sports_frame_fp16":
+            n, pos = w["N"], S.sports_scene(w["N"]).frame(w["frame"])
+        elif name == "sports_train_fp16":
+            n = w["batch"]
+            pos = S.sports_scene(300_000).frames(range(4))[:n]
+        else:
+            n, pos = w["N"], S.stress_positions(w["N"])
+        P = torch.from_numpy(pos).to(dev)
+        T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+        W = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
+        cr = torch.from_numpy(S.gate_params(n)).to(dev) if mlp.gate else None
+        out = sp.alloc_outputs(n, dev, latent_dim=grid.L * grid.F)
+        fwd_out = {k: v for k, v in out.items() if k != "latent"}
+        reps = 20 if n <= 1_000_000 else 7
+        ms = timed(lambda: sp.decode_fwd(g, m, P, T, W, cr, out=fwd_out), reps)
+        spp = table_sectors_per_position(sp, g, P, grid.F, 2 if grid.dtype == "f16" else 4)
+        rate = spp * n / (ms * 1e-3)
+        where = "hbm" if name == "stress_fp16_gate" else "l2"
+        emit(name, "fwd", n, ms, table_sectors_per_position=spp, sector_rate=rate,
+             frac_of_random_sector_ceiling=rate / ceil[where + "_random_sector_per_s"], ceiling=where)
+        if name == "sports_frame_fp16":
+            continue
+        grads = {k: torch.randn((n, wd), device=dev) * (1e-2 if grid.dtype == "f16" else 1.0)
+                 for k, wd in OUT_WIDTHS.items()}
+        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), dtype=torch.float32, device=dev)
+        gw = torch.zeros(mlp.n_params(), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(sp.decode_bwd_workspace(g, m, n), 1), dtype=torch.uint8, device=dev)
+
+        def fb():
+            sp.decode_fwd(g, m, P, T, W, cr, out=out)
+            sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr, workspace=ws, latent=out["latent"])
+
+        emit(name, "fwd+bwd (saved latent)", n, timed(fb, reps))
+        del P, T, W, out, fwd_out, grads, gt, gw, ws
+        torch.cuda.empty_cache()
+
+    # HexPlane
+    w = S.WORKLOADS["hexplane_fp32"]
+    hx, n = w["hex"], w["N"]
+    h = sp.hex_from_spec(hx)
+    inp = {k: torch.from_numpy(v).to(dev) for k, v in S.hexplane_inputs(n).items()}
+    planes = torch.from_numpy(S.hexplane_planes(hx)).to(dev)
+    weights = torch.from_numpy(S.hexplane_weights(hx)).to(dev)
+    out = {k: torch.empty((n, wd), device=dev) for k, wd in sp.HEX_KEYS}
+    lat = torch.empty((n, hx.in_dim), device=dev)
+    grads = {k: torch.randn((n, wd), device=dev) for k, wd in S.HEX_OUT_WIDTHS.items()}
+    gp = torch.zeros(hx.n_plane_floats(), device=dev)
+    gw = torch.zeros(hx.n_params(), device=dev)
+    ws = torch.empty(max(sp.hexplane_bwd_workspace(h, n), 1), dtype=torch.uint8, device=dev)
+    lines = len(hx.scales) * 6 * 4   # 128-byte plane rows per Gaussian
+    ms = timed(lambda: sp.hexplane_fwd(h, inp, planes, weights, out=out), 20)
+    emit("hexplane_fp32", "fwd", n, ms, plane_lines_per_gaussian=lines,
+         frac_of_l2_random_line_ceiling=lines * n / (ms * 1e-3) / ceil["l2_random_line128_per_s"])
+    out_l = dict(out, latent=lat)
+
+    def hfb():
+        sp.hexplane_fwd(h, inp, planes, weights, out=out_l)
+        sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws, latent=lat)
+
+    emit("hexplane_fp32", "fwd+bwd (saved latent)", n, timed(hfb, 10))
+    emit("hexplane_fp32", "bwd (gathering again)", n,
+         timed(lambda: sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws), 10))
+    sp.check_device_errors()
+
+
+def _oracle_chunk(task):
+    """One worker's share of an oracle timing (runs in a spawned process)."""
+    name, what, rows_seed, n = task
+    from threadpoolctl import threadpool_limits
+    sys.path.insert(0, ROOT)
+    with threadpool_limits(limits=1):
+        fn = _oracle_job(name, what, n, rows_seed)
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+
+def _oracle_job(name, what, n, seed):
+    """The oracle's forward (or forward+backward) on n positions of a workload."""
+    from oracle import decoder as dec, hexplane as hxo
+    rng = np.random.default_rng(seed)
+    if name == "hexplane_fp32":
+        hx = S.WORKLOADS[name]["hex"]
+        inp = S.hexplane_inputs(n, seed)
+        planes, weights = S.hexplane_planes(hx), S.hexplane_weights(hx)
+        if what == "fwd":
+            return lambda: hxo.forward(inp, planes, weights, hx)
+        grads = S.upstream_grads(n, S.HEX_OUT_WIDTHS, 1.0, seed)
+        return lambda: (hxo.forward(inp, planes, weights, hx), hxo.backward(inp, planes, weights, hx, grads))
+    w = S.WORKLOADS[name]
+    grid, mlp = w["grid"], w["mlp"]
+    if name == "tiny_fp32":
+        pos = S.uniform_positions(w["N"])
+    elif name == "stress_fp16_gate":
+        pos = S.stress_positions(1_000_000)
+    else:
+        pos = S.sports_scene(300_000).frame(w.get("frame", 75))
+    pos = pos[rng.choice(len(pos), min(n, len(pos)), replace=False)]
+    tables, weights = S.hash_tables(grid), S.mlp_weights(mlp)
+    cr = S.gate_params(len(pos), seed) if mlp.gate else None
+    if what == "fwd":
+        return lambda: dec.decode_forward(pos, tables, weights, grid, mlp, gate_cr=cr)
+    grads = S.upstream_grads(len(pos), S.DECODE_OUT_WIDTHS, 1e-2, seed)
+    return lambda: (dec.decode_forward(pos, tables, weights, grid, mlp, gate_cr=cr),
+                    dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr))
+
+
+def run_cpu_workloads(args):
+    """The oracle, as it stands, on a bounded sample of every workload: one
+    thread, and a pool of spawned single-threaded processes (one per core, at
+    most 32) over equal shares of a larger sample.  The stress workload gets
+    the single-thread timing only: the oracle widens its 512 MiB of tables to
+    fp64 per call, too much memory to hold once per process."""
+    import multiprocessing as mp
+    procs = min(os.cpu_count() or 1, 32)
+    jobs = [("tiny_fp32", "fwd", 4096), ("tiny_fp32", "fwd+bwd", 4096), ("sports_frame_fp16", "fwd", 20_000),
+            ("sports_train_fp16", "fwd+bwd", 10_000), ("stress_fp16_gate", "fwd", 10_000),
+            ("hexplane_fp32", "fwd", 2_000), ("hexplane_fp32", "fwd+bwd", 1_000)]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(procs) as pool:
+        pool.map(_oracle_chunk, [("tiny_fp32", "fwd", i, 64) for i in range(procs)])   # start every worker
+        for name, what, n in jobs:
+            one = _oracle_chunk((name, what, 1, n))
+            line = {"workload": name, "pass": what, "kind": "oracle", "sample": n,
+                    "positions_per_s_1_thread": n / one, "host_cores": os.cpu_count()}
+            if name != "stress_fp16_gate":
+                t0 = time.perf_counter()
+                pool.map(_oracle_chunk, [(name, what, 100 + i, n) for i in range(procs)])
+                line["positions_per_s_pool"] = n * procs / (time.perf_counter() - t0)
+                line["pool_processes"] = procs
+            print(json.dumps(line), flush=True)
+
+
 def run_ncu_case(name):
     """A few untimed launches of one workload, for an ncu capture."""
     import torch
@@ -537,6 +744,12 @@ def main():
     args = parse()
     if args.ncu_case:
         run_ncu_case(args.ncu_case)
+        return
+    if args.cpu_workloads:
+        run_cpu_workloads(args)
+        return
+    if args.workloads:
+        run_workloads(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -334,15 +334,34 @@ int spin4d_check_device_errors(int clear);
 /*
  * Measurement helper (not part of the decoder): the gather-rate ceiling.
  * Launches `blocks` x 256 threads; each issues `loads_per_thread` (a multiple
- * of 8) independent loads of `width` bytes (4 or 16) at pseudo-random,
- * width-aligned offsets of `buf` (device, 16-byte aligned, `buf_bytes` long),
- * eight in flight per thread.  Every load touches exactly one 32-byte sector,
- * so loads / elapsed time is the random-sector rate of wherever `buf` lives:
- * L2 for a buffer well under the L2 size, HBM for one far above it.
- * `sink` (device, 4 bytes) is written only to keep the loads alive.
+ * of 8) independent loads at pseudo-random, width-aligned offsets of `buf`
+ * (device, `buf_bytes` long, 16-byte aligned; 128-byte aligned for width
+ * 128), eight in flight per thread.  width 4 or 16: every load is its own
+ * 4- or 16-byte access inside one 32-byte sector, so loads / elapsed time is
+ * the random-sector rate of wherever `buf` lives (L2 for a buffer well under
+ * the L2 size, HBM for one far above it).  width 128: each group of 8
+ * consecutive lanes reads one random 128-byte line, 16 bytes per lane, so
+ * (blocks x 256 x loads_per_thread / 8) / elapsed time is the random-line
+ * rate.  `sink` (device, 4 bytes) is written only to keep the loads alive.
  */
 int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t loads_per_thread, int blocks,
                         uint32_t seed, uint32_t* sink, spin4d_stream_t stream);
+
+/*
+ * Measurement helper: reads `buf` (device, 16-byte aligned, buf_bytes a
+ * multiple of 16) front to back `passes` times with 16-byte loads from
+ * `blocks` x 256 threads; passes x buf_bytes / elapsed time is the
+ * sequential read bandwidth of wherever `buf` lives.
+ */
+int spin4d_probe_stream(const void* buf, uint64_t buf_bytes, int passes, int blocks, uint32_t* sink,
+                        spin4d_stream_t stream);
+
+/*
+ * Measurement helper: `blocks` x 256 threads each run 8 independent fp32 FMA
+ * chains for `iters` steps; 16 x iters x blocks x 256 / elapsed time is the
+ * CUDA-core fp32 rate in FLOP/s.
+ */
+int spin4d_probe_fma(int64_t iters, int blocks, uint32_t* sink, spin4d_stream_t stream);
 
 /*
  * Test hook for failure detection: one block waits (at most max_iters polls,

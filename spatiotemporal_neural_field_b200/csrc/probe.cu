@@ -1,12 +1,15 @@
-// Gather-rate probe: the denominator of the decoder's gather roofline.
+// Measurement probes: the denominators of the gather rooflines.
 //
 // The decoder's hash-grid gathers touch one 32-byte sector per table access
-// at effectively random addresses, so neither a streaming copy (HBM peak) nor
-// a dense GEMM describes their ceiling.  This kernel measures it directly:
-// every thread issues independent `width`-byte loads at pseudo-random,
-// width-aligned offsets of a buffer (32 MiB stays resident in L2; 1 GiB and up
-// streams from HBM), eight loads in flight per thread, and folds the loaded
-// words into a sink so nothing is optimised away.
+// at effectively random addresses, and the HexPlane encoder reads whole
+// 128-byte channel rows at random rows, so neither a streaming copy (HBM
+// peak) nor a dense GEMM describes their ceiling.  probe_gather measures it
+// directly: independent loads at pseudo-random, width-aligned offsets of a
+// buffer (32 MiB stays resident in L2; 1 GiB and up streams from HBM), eight
+// in flight per thread, folded into a sink so nothing is optimised away.
+// probe_stream reads a buffer front to back (the sequential ceiling of
+// wherever it lives) and probe_fma runs independent fp32 FMA chains (the
+// CUDA-core arithmetic peak).
 #include "host.h"
 
 namespace spin4d {
@@ -28,7 +31,10 @@ __global__ void __launch_bounds__(256) probe_gather_kernel(const uint8_t* __rest
                                                            uint32_t* __restrict__ sink) {
   const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
   uint32_t acc = 0;
-  uint32_t state = mix32(tid * 0x9E3779B9u ^ seed);
+  // W = 128: the 8 lanes of a group share the random line and each loads one
+  // of its 16-byte chunks, so one warp instruction reads 4 whole lines.
+  const uint32_t key = W == 128 ? tid >> 3 : tid;
+  uint32_t state = mix32(key * 0x9E3779B9u ^ seed);
   for (int64_t i = 0; i < loads_per_thread; i += 8) {
     uint64_t off[8];
 #pragma unroll
@@ -43,14 +49,46 @@ __global__ void __launch_bounds__(256) probe_gather_kernel(const uint8_t* __rest
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc += v[k];
     } else {
+      const uint64_t chunk = W == 128 ? (threadIdx.x & 7) : 0;
       uint4 v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = __ldg(reinterpret_cast<const uint4*>(buf) + off[k]);
+      for (int k = 0; k < 8; ++k) v[k] = __ldg(reinterpret_cast<const uint4*>(buf) + off[k] * (W / 16) + chunk);
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc += v[k].x ^ v[k].w;
     }
   }
   if (acc == 0x12345678u) sink[0] = acc;   // practically never taken; keeps the loads alive
+}
+
+__global__ void __launch_bounds__(256) probe_stream_kernel(const uint4* __restrict__ buf, uint64_t n16, int passes,
+                                                           uint32_t* __restrict__ sink) {
+  uint32_t acc = 0;
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  for (int p = 0; p < passes; ++p) {
+    uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+      const uint4 a = __ldcg(buf + i), b = __ldcg(buf + i + stride), c = __ldcg(buf + i + 2 * stride),
+                  d = __ldcg(buf + i + 3 * stride);
+      acc += (a.x ^ b.y) + (c.z ^ d.w);
+    }
+    for (; i < n16; i += stride) acc += __ldcg(buf + i).x;
+  }
+  if (acc == 0x12345678u) sink[0] = acc;
+}
+
+__global__ void __launch_bounds__(256) probe_fma_kernel(int64_t iters, float seed, uint32_t* __restrict__ sink) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = seed + (float)(threadIdx.x + k);
+  const float m = 0.999999f, c = 1e-7f;
+  for (int64_t i = 0; i < iters; ++i) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmaf(a[k], m, c);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) s += a[k];
+  if (s == 1234.5f) sink[0] = 1;
 }
 
 }  // namespace
@@ -60,15 +98,35 @@ using namespace spin4d;
 
 extern "C" int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t loads_per_thread,
                                    int blocks, uint32_t seed, uint32_t* sink, spin4d_stream_t stream) {
-  if (!buf || !sink || (width != 4 && width != 16) || buf_bytes < (uint64_t)width || loads_per_thread < 8 ||
-      loads_per_thread % 8 || blocks < 1 || !aligned(buf, 16))
+  if (!buf || !sink || (width != 4 && width != 16 && width != 128) || buf_bytes < (uint64_t)width ||
+      loads_per_thread < 8 || loads_per_thread % 8 || blocks < 1 || !aligned(buf, width == 128 ? 128 : 16))
     return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_probe_gather")) return SPIN4D_ERR_INJECTED;
   const uint64_t slots = buf_bytes / (uint64_t)width;
   const uint8_t* b = static_cast<const uint8_t*>(buf);
+  cudaStream_t s = (cudaStream_t)stream;
   if (width == 4)
-    probe_gather_kernel<4><<<blocks, 256, 0, (cudaStream_t)stream>>>(b, slots, loads_per_thread, seed, sink);
+    probe_gather_kernel<4><<<blocks, 256, 0, s>>>(b, slots, loads_per_thread, seed, sink);
+  else if (width == 16)
+    probe_gather_kernel<16><<<blocks, 256, 0, s>>>(b, slots, loads_per_thread, seed, sink);
   else
-    probe_gather_kernel<16><<<blocks, 256, 0, (cudaStream_t)stream>>>(b, slots, loads_per_thread, seed, sink);
+    probe_gather_kernel<128><<<blocks, 256, 0, s>>>(b, slots, loads_per_thread, seed, sink);
+  return launch_status();
+}
+
+extern "C" int spin4d_probe_stream(const void* buf, uint64_t buf_bytes, int passes, int blocks, uint32_t* sink,
+                                   spin4d_stream_t stream) {
+  if (!buf || !sink || buf_bytes < 16 || buf_bytes % 16 || passes < 1 || blocks < 1 || !aligned(buf, 16))
+    return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_probe_stream")) return SPIN4D_ERR_INJECTED;
+  probe_stream_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint4*>(buf), buf_bytes / 16, passes,
+                                                                sink);
+  return launch_status();
+}
+
+extern "C" int spin4d_probe_fma(int64_t iters, int blocks, uint32_t* sink, spin4d_stream_t stream) {
+  if (!sink || iters < 1 || blocks < 1) return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_probe_fma")) return SPIN4D_ERR_INJECTED;
+  probe_fma_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(iters, 1.0f, sink);
   return launch_status();
 }

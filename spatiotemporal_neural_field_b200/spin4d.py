@@ -88,6 +88,8 @@ _SIGS = {
     "spin4d_check_device_errors": (c_i32, [c_i32]),
     "spin4d_selftest_wait_timeout": (c_i32, [c_u32, c_vp]),
     "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
+    "spin4d_probe_stream": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i32, c_vp, c_vp]),
+    "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
     "spin4d_version": (ctypes.c_char_p, []),
@@ -284,12 +286,15 @@ def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=
     return out
 
 
+def hexplane_bwd_workspace(h: HexDesc, N: int) -> int:
+    return int(lib.spin4d_hexplane_bwd_workspace(ctypes.byref(h), N))
+
+
 def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, latent=None,
                  stream=None):
     N = inp["mu"].shape[0]
-    need = int(lib.spin4d_hexplane_bwd_workspace(ctypes.byref(h), N))
     if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=planes.device)
+        workspace = torch.empty(max(hexplane_bwd_workspace(h, N), 1), dtype=torch.uint8, device=planes.device)
     go = HexOutputGrads(*(_ptr(grads.get(k)) for k, _ in HEX_KEYS))
     _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
                                                           _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
@@ -319,13 +324,33 @@ def selftest_wait_timeout(max_iters: int = 4096, stream=None) -> None:
 
 def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: int, seed: int = 1,
                  sink: Optional[torch.Tensor] = None, stream=None) -> int:
-    """Launches the random-gather probe; returns the number of loads issued."""
+    """Launches the random-gather probe; returns the number of `width`-byte
+    units read (sectors for width 4/16, 128-byte lines for width 128)."""
     if sink is None:
         sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
     _check("spin4d_probe_gather", lib.spin4d_probe_gather(_ptr(buf), buf.numel() * buf.element_size(), width,
                                                           loads_per_thread, blocks, seed, _ptr(sink),
                                                           _stream(stream)))
-    return blocks * 256 * loads_per_thread
+    return blocks * 256 * loads_per_thread // (8 if width == 128 else 1)
+
+
+def probe_stream(buf: torch.Tensor, passes: int, blocks: int, sink: Optional[torch.Tensor] = None,
+                 stream=None) -> int:
+    """Sequential-read probe; returns the bytes read."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size()
+    _check("spin4d_probe_stream", lib.spin4d_probe_stream(_ptr(buf), nbytes, passes, blocks, _ptr(sink),
+                                                          _stream(stream)))
+    return passes * nbytes
+
+
+def probe_fma(iters: int, blocks: int, device, sink: Optional[torch.Tensor] = None, stream=None) -> int:
+    """fp32 FMA-chain probe; returns the FLOPs executed."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=device)
+    _check("spin4d_probe_fma", lib.spin4d_probe_fma(iters, blocks, _ptr(sink), _stream(stream)))
+    return 16 * iters * blocks * 256
 
 
 def version() -> str:

@@ -262,7 +262,7 @@ int64_t spin4d_hexplane_plane_count(const spin4d_hexplane_desc* h);
 int64_t spin4d_hexplane_param_count(const spin4d_hexplane_desc* h);
 
 /* Deformed Gaussians: mu' N x 3, rot N x 4, scale N x 3, sh N x 48, cov N x 6 (fp32).
- * latent (optional, may be NULL): N x (n_scales*6*channels) fp32, 16-byte
+ * latent (optional, may be NULL): N x (n_scales*6*channels) fp32, 32-byte
  * aligned, receives the concatenated plane samples. */
 typedef struct spin4d_hex_outputs {
     float* mu;
@@ -285,7 +285,10 @@ typedef struct spin4d_hex_output_grads {
  * mu' = mu + d_mu; q' = (q_can + d_q)/max(||q_can + d_q||, 1e-12);
  * s' = exp(logs_can + d_logs); sh' = sh_can + d_sh; Sigma(s', q').
  *   mu N x 3, frame N int32 in [0, n_frames), q_can N x 4, logs_can N x 3,
- *   sh_can N x 48 (all fp32).
+ *   sh_can N x 48 (all fp32).  planes and weights: device, 32-byte aligned;
+ *   out.rot 16-byte aligned.  Misaligned or NULL arguments return
+ *   SPIN4D_ERR_INVALID; channels other than 32, hidden other than 64 or
+ *   n_hidden other than 2 return SPIN4D_ERR_UNSUPPORTED, before any launch.
  */
 int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
                         int64_t N, const float* planes, const float* weights,
@@ -298,7 +301,7 @@ size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N);
  * Backward of spin4d_hexplane_fwd: grad_planes += dL/dplanes and
  * grad_weights += dL/dweights (fp32, packed like planes and weights) for
  * L = sum over outputs of <grad_out.x, x>; a NULL member of grad_out is a
- * zero gradient.  latent (optional, may be NULL, 16-byte aligned) is the
+ * zero gradient.  latent (optional, may be NULL, 32-byte aligned) is the
  * forward's saved latent for the same inputs; given, the plane samples are
  * read from it instead of being gathered again.  workspace: device memory
  * of at least spin4d_hexplane_bwd_workspace(h, N) bytes, 256-byte aligned,

@@ -506,11 +506,14 @@ __device__ __forceinline__ void mma6(uint32_t d_main, uint32_t d_corr, const Spl
 
 // acc[i] += main[col0 + i] + corr[col0 + i] for this thread's 32 columns.
 __device__ __forceinline__ void add_partial(uint32_t d_main, uint32_t d_corr, float acc[32]) {
-  float a[32], b[32];
-  tc::tmem_ld32(d_main, a);
-  tc::tmem_ld32(d_corr, b);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] += a[i] + b[i];
+  for (int h = 0; h < 2; ++h) {
+    float a[16], b[16];
+    tc::tmem_ld16(d_main + 16 * h, a);
+    tc::tmem_ld16(d_corr + 16 * h, b);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[16 * h + i] += a[i] + b[i];
+  }
 }
 
 // Sums over a warp: v[i] holds this lane's value of column i; on return the
@@ -545,16 +548,37 @@ struct HexBars {
   }
 };
 
+// 32 bytes (one sector) of read-only global data in one 256-bit load; p must
+// be 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const float* p, float v[8]) {
+  asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "l"(p));
+}
+
+// Global data of one plane sample for one thread: its chunk of the W1 slice
+// (row tid/4, 8 columns) and, for its Gaussian, the 16 channels (half*16 ..)
+// of the four corner rows with their bilinear weights, or the 16 values of a
+// saved latent (in c[0]).
+struct SampleRegs {
+  float w[8];
+  float c[4][16];
+  float wt[4];
+};
+
 // Streams the plane samples of one tile through the two stages.  Stage
 // b = k & 1 receives sample k: the 64x32 slice of W1 for the sample and the
 // tile's 128x32 feature block z_k (split), z_k read from zsrc (a saved
 // latent) when given, else sampled from the planes (and then copied to zdst
 // when given).  issue(k, b) runs on thread 0 once the stage is written and
 // its MMAs are committed to stage b's barrier; consume(k, b) runs on every
-// thread once they are done, before the stage takes sample k + 2.  Global
-// loads for sample k + 1 are issued right after sample k's MMAs, so their
-// latency overlaps the tensor core.  Returns false if a wait ran out.
-template <class Issue, class Consume>
+// thread once they are done, before the stage takes sample k + 2.  Each
+// thread reads its half of its Gaussian's four corner rows as 32-byte
+// sectors.  Global loads run DEPTH samples ahead: with DEPTH = 2, two
+// register sets (even and odd samples) keep about 128 KB of row reads per SM
+// in flight while the tensor core and the barriers work.  The sample count
+// is even (6 per scale).  Returns false if a wait ran out.
+template <int DEPTH, class Issue, class Consume>
 __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
                                            const float* __restrict__ W1, const float* __restrict__ zsrc,
                                            float* __restrict__ zdst, int64_t n, bool valid, const float xt[4],
@@ -562,33 +586,28 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
   using Lay = HexTcLayout;
   const int tid = threadIdx.x, row = tid & (kHexTile - 1), half = tid / kHexTile;
   const int IN = hp.in_dim, NS = hp.n_samples;
-  float4 wpre[2], cpre[4][4];
-  float cw[4] = {0.f, 0.f, 0.f, 0.f};
-  auto prefetch = [&](int k) {
-    const int r = tid >> 2, c8 = tid & 3;   // W1 slice: 64 rows x 4 chunks of 8
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-      wpre[q] = __ldg(reinterpret_cast<const float4*>(W1 + (size_t)r * IN + k * kHexC) + 2 * c8 + q);
+  SampleRegs ra, rb;
+  auto prefetch = [&](int k, SampleRegs& r) {
+    ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
     if (!valid) return;
     if (zsrc) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        cpre[0][q] = __ldg(reinterpret_cast<const float4*>(zsrc + n * IN + k * kHexC) + half * 4 + q);
+      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16, r.c[0]);
+      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16 + 8, r.c[0] + 8);
     } else {
       const PlaneSample ps = plane_sample(xt, hp, k);
-      cw[0] = ps.w00;
-      cw[1] = ps.w01;
-      cw[2] = ps.w10;
-      cw[3] = ps.w11;
+      r.wt[0] = ps.w00;
+      r.wt[1] = ps.w01;
+      r.wt[2] = ps.w10;
+      r.wt[3] = ps.w11;
       const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) cpre[c][q] = __ldg(reinterpret_cast<const float4*>(planes + off[c]) + half * 4 + q);
+      for (int c = 0; c < 4; ++c) {
+        ld_nc_v8(planes + off[c] + half * 16, r.c[c]);
+        ld_nc_v8(planes + off[c] + half * 16 + 8, r.c[c] + 8);
+      }
     }
   };
-  prefetch(0);
-  for (int k = 0; k < NS; ++k) {
+  auto step = [&](int k, SampleRegs& r) -> bool {
     const int b = k & 1;
     if (k >= 2) {   // sample k-2 used this stage: take its results, then refill
       const bool ok = bars.wait(b);
@@ -596,25 +615,20 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
       tc::fence_after_sync();
       consume(k - 2, b);
     }
-    store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, wpre[0], wpre[1]);
-    float4 z4[4];
+    store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, r.w);
+    float z[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      z4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (valid) {
-        if (zsrc) {
-          z4[q] = cpre[0][q];
-        } else {
-          z4[q].x = cw[0] * cpre[0][q].x + cw[1] * cpre[1][q].x + cw[2] * cpre[2][q].x + cw[3] * cpre[3][q].x;
-          z4[q].y = cw[0] * cpre[0][q].y + cw[1] * cpre[1][q].y + cw[2] * cpre[2][q].y + cw[3] * cpre[3][q].y;
-          z4[q].z = cw[0] * cpre[0][q].z + cw[1] * cpre[1][q].z + cw[2] * cpre[2][q].z + cw[3] * cpre[3][q].z;
-          z4[q].w = cw[0] * cpre[0][q].w + cw[1] * cpre[1][q].w + cw[2] * cpre[2][q].w + cw[3] * cpre[3][q].w;
-          if (zdst) reinterpret_cast<float4*>(zdst + n * IN + k * kHexC)[half * 4 + q] = z4[q];
-        }
-      }
+    for (int i = 0; i < 16; ++i) {
+      z[i] = 0.f;
+      if (valid) z[i] = zsrc ? r.c[0][i] : r.wt[0] * r.c[0][i] + r.wt[1] * r.c[1][i] + r.wt[2] * r.c[2][i] + r.wt[3] * r.c[3][i];
     }
-    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2, kHexC, z4[0], z4[1]);
-    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z4[2], z4[3]);
+    if (valid && zdst && !zsrc) {
+      float4* d = reinterpret_cast<float4*>(zdst + n * IN + k * kHexC + half * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) d[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+    }
+    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2, kHexC, z);
+    store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z + 8);
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -623,9 +637,21 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
       issue(k, b);
       tc::mma_commit(bars.addr(b));
     }
-    if (k + 1 < NS) prefetch(k + 1);
+    if (k + DEPTH < NS) prefetch(k + DEPTH, r);
+    return true;
+  };
+  prefetch(0, ra);
+  if constexpr (DEPTH == 2) {
+    prefetch(1, rb);
+    for (int k = 0; k < NS; k += 2) {
+      if (!step(k, ra)) return false;
+      if (!step(k + 1, rb)) return false;
+    }
+  } else {
+    for (int k = 0; k < NS; ++k)
+      if (!step(k, ra)) return false;
   }
-  for (int k = (NS >= 2 ? NS - 2 : 0); k < NS; ++k) {   // the last two samples
+  for (int k = NS - 2; k < NS; ++k) {   // the last two samples
     const int b = k & 1;
     const bool ok = bars.wait(b);
     if (__syncthreads_or(!ok)) return false;
@@ -727,7 +753,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
-    if (!hex_stream(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
+    if (!hex_stream<2>(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
       failed = true;
       break;
     }
@@ -914,7 +940,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume1 = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, h1); };
-    if (!hex_stream(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
+    if (!hex_stream<1>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
       failed = true;
       break;
     }
@@ -1086,7 +1112,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
         }
       }
     };
-    if (!hex_stream(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
+    if (!hex_stream<1>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
       failed = true;
       break;
     }
@@ -1151,7 +1177,7 @@ static int hex_check(const spin4d_hexplane_desc* h, const float* mu, const int32
   if (N < 0) return SPIN4D_ERR_INVALID;
   if (N == 0) return SPIN4D_OK;
   if (!mu || !frame || !planes || !weights || !q_can || !logs_can) return SPIN4D_ERR_INVALID;
-  if (!aligned(planes, 16) || !aligned(weights, 16) || !aligned(mu, 4) || !aligned(frame, 4) ||
+  if (!aligned(planes, 32) || !aligned(weights, 32) || !aligned(mu, 4) || !aligned(frame, 4) ||
       !aligned(q_can, 4) || !aligned(logs_can, 4))
     return SPIN4D_ERR_INVALID;
   return hex_supported(h);
@@ -1189,6 +1215,7 @@ extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* m
   if (N == 0) return SPIN4D_OK;
   if (!sh_can || !out.mu || !out.rot || !out.scale || !out.sh || !out.cov || !aligned(out.rot, 16))
     return SPIN4D_ERR_INVALID;
+  if (out.latent && !aligned(out.latent, 32)) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_hexplane_fwd")) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
@@ -1233,7 +1260,7 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_planes || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_planes, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256)) return SPIN4D_ERR_INVALID;
-  if (latent && !aligned(latent, 16)) return SPIN4D_ERR_INVALID;
+  if (latent && !aligned(latent, 32)) return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_hexplane_bwd_workspace(h, N)) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_hexplane_bwd")) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);

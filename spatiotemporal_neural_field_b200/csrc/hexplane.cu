@@ -609,11 +609,14 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
   };
   auto step = [&](int k, SampleRegs& r) -> bool {
     const int b = k & 1;
+    bool ok = true;
     if (k >= 2) {   // sample k-2 used this stage: take its results, then refill
-      const bool ok = bars.wait(b);
-      if (__syncthreads_or(!ok)) return false;
+      // Every thread sees the commit itself, so no block barrier is needed
+      // before reading the results or refilling the stage; a wait that ran
+      // out is reported at the barrier below.
+      ok = bars.wait(b);
       tc::fence_after_sync();
-      consume(k - 2, b);
+      if (ok) consume(k - 2, b);
     }
     store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, r.w);
     float z[16];
@@ -631,7 +634,7 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
     store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z + 8);
     tc::fence_proxy_async();
     tc::fence_before_sync();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) return false;
     if (tid == 0) {
       tc::fence_after_sync();
       issue(k, b);

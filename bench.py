@@ -506,6 +506,12 @@ def device_ceilings(sp, torch, dev):
         out[name + "_random_line128_per_s"] = best(lambda it: sp.probe_gather(buf, 128, lpt, 4 * sms, seed=it + 1))
         passes = 64 if name == "l2" else 2
         out[name + "_sequential_bytes_per_s"] = best(lambda it: sp.probe_stream(buf, passes, 4 * sms))
+        ops = 512 if name == "l2" else 128
+        for wdt in (8, 16):
+            out["%s_random_red%d_per_s" % (name, wdt)] = best(
+                lambda it: sp.probe_atomic(buf, wdt, ops, 4 * sms, seed=it + 1))
+        out[name + "_random_bulk_red128_rows_per_s"] = best(
+            lambda it: sp.probe_bulk_reduce(buf, ops // 4, 8 * sms, seed=it + 1))
         del buf
     out["fp32_fma_flop_per_s"] = best(lambda it: sp.probe_fma(1 << 16, 8 * sms, dev))
     return out

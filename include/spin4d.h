@@ -351,6 +351,27 @@ int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t 
                         uint32_t seed, uint32_t* sink, spin4d_stream_t stream);
 
 /*
+ * Measurement helper: the scatter-add ceiling.  `blocks` x 256 threads each
+ * issue `ops_per_thread` (a multiple of 8) fp32 reductions (red.global.add,
+ * `width` = 4, 8 or 16 bytes: 1, 2 or 4 floats of +1.0) at pseudo-random,
+ * width-aligned offsets of `buf` (device, 16-byte aligned, `buf_bytes`
+ * long, modified); operations / elapsed time is the random-atomic rate of
+ * wherever `buf` lives.
+ */
+int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int64_t ops_per_thread, int blocks,
+                        uint32_t seed, spin4d_stream_t stream);
+
+/*
+ * Measurement helper: the row scatter-add ceiling.  `blocks` x 128 threads
+ * each add a 128-byte row of fp32 ones to `rows_per_thread` pseudo-random
+ * 128-byte rows of `buf` (device, 128-byte aligned, modified) with bulk
+ * asynchronous reductions (cp.reduce.async.bulk .add.f32), up to 8 in flight
+ * per thread; rows / elapsed time is the rate.
+ */
+int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int64_t rows_per_thread, int blocks, uint32_t seed,
+                             spin4d_stream_t stream);
+
+/*
  * Measurement helper: reads `buf` (device, 16-byte aligned, buf_bytes a
  * multiple of 16) front to back `passes` times with 16-byte loads from
  * `blocks` x 256 threads; passes x buf_bytes / elapsed time is the

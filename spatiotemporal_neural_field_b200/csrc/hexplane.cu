@@ -487,12 +487,21 @@ __device__ __forceinline__ SplitOp mnmajor(uint32_t base, int plane, int L) {
 // d_corr = A0.B1 + A1.B0 + A0.B2 + A2.B0 + A1.B1.
 __device__ __forceinline__ void mma6(uint32_t d_main, uint32_t d_corr, const SplitOp& a, const SplitOp& b, int K,
                                      uint32_t idesc) {
-  for (int s = 0; s < K / 16; ++s) {
-    uint64_t ad[3], bd[3];
+  // Descriptors are built once; a K slice moves the start-address field
+  // (address / 16, low bits) by step / 16.
+  uint64_t ad[3], bd[3];
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      ad[i] = tc::smem_desc(a.base + i * a.plane + s * a.step, a.lbo, a.sbo);
-      bd[i] = tc::smem_desc(b.base + i * b.plane + s * b.step, b.lbo, b.sbo);
+  for (int i = 0; i < 3; ++i) {
+    ad[i] = tc::smem_desc(a.base + i * a.plane, a.lbo, a.sbo);
+    bd[i] = tc::smem_desc(b.base + i * b.plane, b.lbo, b.sbo);
+  }
+  for (int s = 0; s < K / 16; ++s) {
+    if (s > 0) {
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        ad[i] += a.step >> 4;
+        bd[i] += b.step >> 4;
+      }
     }
     const uint32_t acc = s > 0 ? 1u : 0u;
     tc::mma_f16(d_main, ad[0], bd[0], idesc, acc);
@@ -557,42 +566,49 @@ __device__ __forceinline__ void ld_nc_v8(const float* p, float v[8]) {
 }
 
 // Global data of one plane sample for one thread: its chunk of the W1 slice
-// (row tid/4, 8 columns) and, for its Gaussian, the 16 channels (half*16 ..)
-// of the four corner rows with their bilinear weights, or the 16 values of a
-// saved latent (in c[0]).
+// (row tid/4, 8 columns) and, for its Gaussian, either the 16 channels
+// (half*16 ..) of the four corner rows with their bilinear weights, or the
+// 16 values of a saved latent.
+template <bool LATENT>
 struct SampleRegs {
   float w[8];
   float c[4][16];
   float wt[4];
 };
+template <>
+struct SampleRegs<true> {
+  float w[8];
+  float z[16];
+};
 
 // Streams the plane samples of one tile through the two stages.  Stage
 // b = k & 1 receives sample k: the 64x32 slice of W1 for the sample and the
 // tile's 128x32 feature block z_k (split), z_k read from zsrc (a saved
-// latent) when given, else sampled from the planes (and then copied to zdst
+// latent) when LATENT, else sampled from the planes (and then copied to zdst
 // when given).  issue(k, b) runs on thread 0 once the stage is written and
 // its MMAs are committed to stage b's barrier; consume(k, b) runs on every
 // thread once they are done, before the stage takes sample k + 2.  Each
-// thread reads its half of its Gaussian's four corner rows as 32-byte
-// sectors.  Global loads run DEPTH samples ahead: with DEPTH = 2, two
-// register sets (even and odd samples) keep about 128 KB of row reads per SM
-// in flight while the tensor core and the barriers work.  The sample count
-// is even (6 per scale).  Returns false if a wait ran out.
-template <int DEPTH, class Issue, class Consume>
+// thread reads its half of its Gaussian's four corner rows (or latent row)
+// as 32-byte sectors.  Global loads run DEPTH samples ahead: with DEPTH = 2,
+// two register sets (even and odd samples) keep about 128 KB of row reads
+// per SM in flight while the tensor core and the barriers work.  The sample
+// count is even (6 per scale).  Returns false if a wait ran out.
+template <int DEPTH, bool LATENT, class Issue, class Consume>
 __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
                                            const float* __restrict__ W1, const float* __restrict__ zsrc,
                                            float* __restrict__ zdst, int64_t n, bool valid, const float xt[4],
                                            HexBars& bars, Issue issue, Consume consume) {
   using Lay = HexTcLayout;
+  using Regs = SampleRegs<LATENT>;
   const int tid = threadIdx.x, row = tid & (kHexTile - 1), half = tid / kHexTile;
   const int IN = hp.in_dim, NS = hp.n_samples;
-  SampleRegs ra, rb;
-  auto prefetch = [&](int k, SampleRegs& r) {
+  Regs ra, rb;
+  auto prefetch = [&](int k, Regs& r) {
     ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
     if (!valid) return;
-    if (zsrc) {
-      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16, r.c[0]);
-      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16 + 8, r.c[0] + 8);
+    if constexpr (LATENT) {
+      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16, r.z);
+      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16 + 8, r.z + 8);
     } else {
       const PlaneSample ps = plane_sample(xt, hp, k);
       r.wt[0] = ps.w00;
@@ -607,7 +623,7 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
       }
     }
   };
-  auto step = [&](int k, SampleRegs& r) -> bool {
+  auto step = [&](int k, Regs& r) -> bool {
     const int b = k & 1;
     bool ok = true;
     if (k >= 2) {   // sample k-2 used this stage: take its results, then refill
@@ -623,12 +639,18 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       z[i] = 0.f;
-      if (valid) z[i] = zsrc ? r.c[0][i] : r.wt[0] * r.c[0][i] + r.wt[1] * r.c[1][i] + r.wt[2] * r.c[2][i] + r.wt[3] * r.c[3][i];
+      if constexpr (LATENT) {
+        if (valid) z[i] = r.z[i];
+      } else {
+        if (valid) z[i] = r.wt[0] * r.c[0][i] + r.wt[1] * r.c[1][i] + r.wt[2] * r.c[2][i] + r.wt[3] * r.c[3][i];
+      }
     }
-    if (valid && zdst && !zsrc) {
-      float4* d = reinterpret_cast<float4*>(zdst + n * IN + k * kHexC + half * 16);
+    if constexpr (!LATENT) {
+      if (valid && zdst) {
+        float4* d = reinterpret_cast<float4*>(zdst + n * IN + k * kHexC + half * 16);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) d[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+        for (int q = 0; q < 4; ++q) d[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+      }
     }
     store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2, kHexC, z);
     store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z + 8);
@@ -756,7 +778,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
-    if (!hex_stream<2>(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
+    if (!hex_stream<2, false>(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
       failed = true;
       break;
     }
@@ -839,18 +861,13 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   }
 }
 
-// RMW of 32 consecutive floats of a workspace slot row.
+// Adds 32 consecutive floats to a workspace slot row with fp32 vector
+// reductions.  Only this thread ever updates these elements, so the adds land
+// in program order and the sum does not depend on scheduling.
 __device__ __forceinline__ void slot_add32(float* dst, const float a[32]) {
   float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    float4 v = d[q];
-    v.x += a[4 * q];
-    v.y += a[4 * q + 1];
-    v.z += a[4 * q + 2];
-    v.w += a[4 * q + 3];
-    d[q] = v;
-  }
+  for (int q = 0; q < 8; ++q) atomicAdd(d + q, make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
 }
 
 // Backward, one 128-Gaussian tile per step of a persistent CTA:
@@ -868,6 +885,7 @@ __device__ __forceinline__ void slot_add32(float* dst, const float a[32]) {
 // gradients are warp column sums gathered in shared memory, so they do not
 // depend on scheduling.  TMEM: stages as in the forward, plus the 64-row
 // weight-gradient accumulators at columns 256 (main) and 320 (correction).
+template <bool LATENT>
 __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
@@ -943,7 +961,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume1 = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, h1); };
-    if (!hex_stream<1>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
+    if (!hex_stream<LATENT ? 2 : 1, LATENT>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
       failed = true;
       break;
     }
@@ -1102,20 +1120,15 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
       tc::tmem_ld16(S + 64 + lane + (warp >> 2) * 16, a);
       tc::tmem_ld16(S + 96 + lane + (warp >> 2) * 16, c);
       tc::fence_before_sync();
-      if (wrow_ok) {
+      if (wrow_ok) {   // this thread alone updates these slot elements: see slot_add32
         float4* dst = reinterpret_cast<float4*>(sW1 + (size_t)wrow * IN + k * kHexC + (warp >> 2) * 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float4 v = dst[q];
-          v.x += a[4 * q] + c[4 * q];
-          v.y += a[4 * q + 1] + c[4 * q + 1];
-          v.z += a[4 * q + 2] + c[4 * q + 2];
-          v.w += a[4 * q + 3] + c[4 * q + 3];
-          dst[q] = v;
-        }
+        for (int q = 0; q < 4; ++q)
+          atomicAdd(dst + q, make_float4(a[4 * q] + c[4 * q], a[4 * q + 1] + c[4 * q + 1], a[4 * q + 2] + c[4 * q + 2],
+                                         a[4 * q + 3] + c[4 * q + 3]));
       }
     };
-    if (!hex_stream<1>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
+    if (!hex_stream<LATENT ? 2 : 1, LATENT>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
       failed = true;
       break;
     }
@@ -1223,7 +1236,7 @@ extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* m
   HexParams p = make_hex_params(h);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
   if (h->n_scales * 6 <= 24) {
-    // tensor cores, 3xTF32
+    // tensor cores, bf16x3 split
     static bool configured[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
@@ -1272,26 +1285,30 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
   cudaStream_t s = (cudaStream_t)stream;
   int blocks = 0;
   {
-    // tensor cores, 3xTF32: one CTA per SM (it holds 512 TMEM columns)
+    // tensor cores, bf16x3 split: one CTA per SM (it holds 512 TMEM columns)
     static bool configured[64] = {false};
     static bool usable[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     const int smem = HexBwdLayout::BYTES;
     if (!configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(hexplane_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      int occ = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_bwd_tc_kernel, kHexThreads, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      usable[dev] = occ == 1;
+      bool ok = true;
+      for (auto* kern : {hexplane_bwd_tc_kernel<false>, hexplane_bwd_tc_kernel<true>}) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        int occ = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kHexThreads, smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        ok = ok && occ == 1;
+      }
+      usable[dev] = ok;
       configured[dev] = true;
     }
     if (usable[dev]) {
       blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
-      hexplane_bwd_tc_kernel<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can,
-                                                              latent, go, grad_planes, static_cast<float*>(workspace),
-                                                              n_params);
+      auto* kern = latent ? hexplane_bwd_tc_kernel<true> : hexplane_bwd_tc_kernel<false>;
+      kern<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, latent, go, grad_planes,
+                                             static_cast<float*>(workspace), n_params);
       SPIN4D_CHECK(launch_status());
     }
   }

@@ -7,7 +7,9 @@
 // directly: independent loads at pseudo-random, width-aligned offsets of a
 // buffer (32 MiB stays resident in L2; 1 GiB and up streams from HBM), eight
 // in flight per thread, folded into a sink so nothing is optimised away.
-// probe_stream reads a buffer front to back (the sequential ceiling of
+// probe_atomic issues fp32 reductions (1, 2 or 4 floats, one 32-byte sector
+// each) at random offsets: the ceiling of a gradient scatter.  probe_stream
+// reads a buffer front to back (the sequential ceiling of
 // wherever it lives) and probe_fma runs independent fp32 FMA chains (the
 // CUDA-core arithmetic peak).
 #include "host.h"
@@ -58,6 +60,50 @@ __global__ void __launch_bounds__(256) probe_gather_kernel(const uint8_t* __rest
     }
   }
   if (acc == 0x12345678u) sink[0] = acc;   // practically never taken; keeps the loads alive
+}
+
+template <int W>
+__global__ void __launch_bounds__(256) probe_atomic_kernel(float* __restrict__ buf, uint64_t n_slots, int64_t ops,
+                                                           uint32_t seed) {
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t state = mix32(tid * 0x9E3779B9u ^ seed);
+  for (int64_t i = 0; i < ops; i += 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      state = mix32(state + 0x6D2B79F5u);
+      const uint64_t slot = ((uint64_t)state * n_slots) >> 32;
+      if constexpr (W == 4)
+        atomicAdd(buf + slot, 1.0f);
+      else if constexpr (W == 8)
+        atomicAdd(reinterpret_cast<float2*>(buf) + slot, make_float2(1.0f, 1.0f));
+      else
+        atomicAdd(reinterpret_cast<float4*>(buf) + slot, make_float4(1.0f, 1.0f, 1.0f, 1.0f));
+    }
+  }
+}
+
+// Each thread owns a 128-byte row of ones in shared memory and adds it to
+// random 128-byte rows of buf with bulk asynchronous reductions, at most 8
+// of its own in flight.
+__global__ void __launch_bounds__(128) probe_bulk_reduce_kernel(float* __restrict__ buf, uint64_t n_rows, int64_t ops,
+                                                                uint32_t seed) {
+  __shared__ __align__(128) float rows[128][32];
+  for (int i = 0; i < 32; ++i) rows[threadIdx.x][i] = 1.0f;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t state = mix32(tid * 0x9E3779B9u ^ seed);
+  const uint32_t src = (uint32_t)__cvta_generic_to_shared(&rows[threadIdx.x][0]);
+  for (int64_t i = 0; i < ops; ++i) {
+    state = mix32(state + 0x6D2B79F5u);
+    const uint64_t r = ((uint64_t)state * n_rows) >> 32;
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 128;" ::"l"(buf + r * 32),
+                 "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 8;" ::: "memory");
+  }
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(256) probe_stream_kernel(const uint4* __restrict__ buf, uint64_t n16, int passes,
@@ -128,5 +174,32 @@ extern "C" int spin4d_probe_fma(int64_t iters, int blocks, uint32_t* sink, spin4
   if (!sink || iters < 1 || blocks < 1) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_probe_fma")) return SPIN4D_ERR_INJECTED;
   probe_fma_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(iters, 1.0f, sink);
+  return launch_status();
+}
+
+extern "C" int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int64_t ops_per_thread, int blocks,
+                                   uint32_t seed, spin4d_stream_t stream) {
+  if (!buf || (width != 4 && width != 8 && width != 16) || buf_bytes < (uint64_t)width || ops_per_thread < 8 ||
+      ops_per_thread % 8 || blocks < 1 || !aligned(buf, 16))
+    return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_probe_atomic")) return SPIN4D_ERR_INJECTED;
+  const uint64_t slots = buf_bytes / (uint64_t)width;
+  float* b = static_cast<float*>(buf);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (width == 4)
+    probe_atomic_kernel<4><<<blocks, 256, 0, s>>>(b, slots, ops_per_thread, seed);
+  else if (width == 8)
+    probe_atomic_kernel<8><<<blocks, 256, 0, s>>>(b, slots, ops_per_thread, seed);
+  else
+    probe_atomic_kernel<16><<<blocks, 256, 0, s>>>(b, slots, ops_per_thread, seed);
+  return launch_status();
+}
+
+extern "C" int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int64_t rows_per_thread, int blocks,
+                                        uint32_t seed, spin4d_stream_t stream) {
+  if (!buf || buf_bytes < 128 || rows_per_thread < 1 || blocks < 1 || !aligned(buf, 128)) return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_probe_bulk_reduce")) return SPIN4D_ERR_INJECTED;
+  probe_bulk_reduce_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(static_cast<float*>(buf), buf_bytes / 128,
+                                                                     rows_per_thread, seed);
   return launch_status();
 }

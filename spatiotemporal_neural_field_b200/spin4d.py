@@ -89,6 +89,8 @@ _SIGS = {
     "spin4d_selftest_wait_timeout": (c_i32, [c_u32, c_vp]),
     "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
     "spin4d_probe_stream": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i32, c_vp, c_vp]),
+    "spin4d_probe_atomic": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
+    "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
@@ -332,6 +334,20 @@ def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: i
                                                           loads_per_thread, blocks, seed, _ptr(sink),
                                                           _stream(stream)))
     return blocks * 256 * loads_per_thread // (8 if width == 128 else 1)
+
+
+def probe_atomic(buf: torch.Tensor, width: int, ops_per_thread: int, blocks: int, seed: int = 1, stream=None) -> int:
+    """Random fp32 reductions of `width` bytes into `buf`; returns the count."""
+    _check("spin4d_probe_atomic", lib.spin4d_probe_atomic(_ptr(buf), buf.numel() * buf.element_size(), width,
+                                                          ops_per_thread, blocks, seed, _stream(stream)))
+    return blocks * 256 * ops_per_thread
+
+
+def probe_bulk_reduce(buf: torch.Tensor, rows_per_thread: int, blocks: int, seed: int = 1, stream=None) -> int:
+    """Random 128-byte bulk fp32 reductions into `buf`; returns the rows added."""
+    _check("spin4d_probe_bulk_reduce", lib.spin4d_probe_bulk_reduce(_ptr(buf), buf.numel() * buf.element_size(),
+                                                                    rows_per_thread, blocks, seed, _stream(stream)))
+    return blocks * 128 * rows_per_thread
 
 
 def probe_stream(buf: torch.Tensor, passes: int, blocks: int, sink: Optional[torch.Tensor] = None,

@@ -510,8 +510,9 @@ def device_ceilings(sp, torch, dev):
         for wdt in (8, 16):
             out["%s_random_red%d_per_s" % (name, wdt)] = best(
                 lambda it: sp.probe_atomic(buf, wdt, ops, 4 * sms, seed=it + 1))
-        out[name + "_random_bulk_red128_rows_per_s"] = best(
-            lambda it: sp.probe_bulk_reduce(buf, ops // 4, 8 * sms, seed=it + 1))
+        for rb in (128, 256):
+            out["%s_random_bulk_red%d_rows_per_s" % (name, rb)] = best(
+                lambda it: sp.probe_bulk_reduce(buf, ops // 4, 8 * sms, seed=it + 1, row_bytes=rb))
         del buf
     out["fp32_fma_flop_per_s"] = best(lambda it: sp.probe_fma(1 << 16, 8 * sms, dev))
     return out

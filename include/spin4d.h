@@ -363,13 +363,14 @@ int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int64_t ops_pe
 
 /*
  * Measurement helper: the row scatter-add ceiling.  `blocks` x 128 threads
- * each add a 128-byte row of fp32 ones to `rows_per_thread` pseudo-random
- * 128-byte rows of `buf` (device, 128-byte aligned, modified) with bulk
- * asynchronous reductions (cp.reduce.async.bulk .add.f32), up to 8 in flight
- * per thread; rows / elapsed time is the rate.
+ * each add a row of fp32 ones (`row_bytes` = 128 or 256) to
+ * `rows_per_thread` pseudo-random, row-aligned rows of `buf` (device,
+ * 128-byte aligned, modified) with bulk asynchronous reductions
+ * (cp.reduce.async.bulk .add.f32), up to 8 in flight per thread; rows /
+ * elapsed time is the rate.
  */
-int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int64_t rows_per_thread, int blocks, uint32_t seed,
-                             spin4d_stream_t stream);
+int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int row_bytes, int64_t rows_per_thread, int blocks,
+                             uint32_t seed, spin4d_stream_t stream);
 
 /*
  * Measurement helper: reads `buf` (device, 16-byte aligned, buf_bytes a

@@ -420,12 +420,18 @@ struct HexTcLayout {
 };
 static_assert(3 * HexTcLayout::H_PLANE == 2 * HexTcLayout::Z_STAGE, "H tile must fill the z stages");
 
-// Backward: the forward's regions at the same offsets, a second activation
-// tile T1 in place of the forward's bias block, then the biases and the
-// CTA's bias-gradient sums.  The first activation tile T0 is the forward's H
-// tile (over the z stages).
+// Backward: the forward's z stages, W1 stages and W2 | W3 at the same
+// offsets, the scatter staging over W2 | W3, a second activation tile T1,
+// then the biases and the CTA's bias-gradient sums.  The first activation
+// tile T0 is the forward's H tile (over the z stages).
 struct HexBwdLayout {
-  static constexpr int T1 = HexTcLayout::BIAS;               // [128][64] x 3 planes
+  // Per plane sample of the dz pass, the 4 bilinear corners' 128-byte rows of
+  // w_c * dz for every Gaussian of the tile, 16 bytes of padding per Gaussian
+  // so that a warp's row stores hit distinct banks.  Overlays W2 | W3, which
+  // are staged again at the start of every tile.
+  static constexpr int SCAT_ROW = 4 * kHexC * 4 + 16;
+  static constexpr int SCAT = HexTcLayout::W2;
+  static constexpr int T1 = SCAT + kHexTile * SCAT_ROW;       // [128][64] x 3 planes
   static constexpr int BIAS = T1 + 3 * HexTcLayout::H_PLANE;  // b1 | b2 | b3
   static constexpr int BACC = BIAS + 3 * kHexH * 4;           // db1 | db2 | db3 over the CTA's tiles
   static constexpr int MISC = BACC + 3 * kHexH * 4;           // 2 mbarriers + TMEM address
@@ -686,6 +692,18 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
   return true;
 }
 
+// grad[0..63] += the 256 bytes at shared address src, asynchronously (one
+// bulk reduction); completion is tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_add_2rows(float* grad, uint32_t src) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 256;" ::"l"(grad), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// This thread's bulk operations have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's bulk operations are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Makes every thread's shared-memory tile writes visible to the tensor core
 // and lines the threads up before thread 0 issues the next MMAs.
 __device__ __forceinline__ void tiles_ready() {
@@ -694,11 +712,8 @@ __device__ __forceinline__ void tiles_ready() {
   __syncthreads();
 }
 
-// Stages W2 and W3 (split, W3 padded with zero rows to 64) and the three
-// bias vectors, once per CTA.
-__device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, const float* __restrict__ W2g,
-                                                   const float* __restrict__ b1, const float* __restrict__ b2,
-                                                   const float* __restrict__ W3g, const float* __restrict__ b3) {
+// Stages W2 and W3 (split, W3 padded with zero rows to 64).
+__device__ __forceinline__ void stage_w23(uint8_t* sm, const float* __restrict__ W2g, const float* __restrict__ W3g) {
   using Lay = HexTcLayout;
   const int tid = threadIdx.x;
   for (int i = tid; i < kHexH * (kHexH / 8); i += kHexThreads) {
@@ -713,6 +728,14 @@ __device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, co
     }
     store_split8(sm, Lay::W3, Lay::S_PLANE, r, kc, kHexH, a, b);
   }
+}
+
+// Stages W2 and W3 and the three bias vectors, once per CTA.
+__device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, const float* __restrict__ W2g,
+                                                   const float* __restrict__ b1, const float* __restrict__ b2,
+                                                   const float* __restrict__ W3g, const float* __restrict__ b3) {
+  const int tid = threadIdx.x;
+  stage_w23(sm, W2g, W3g);
   float* bias = reinterpret_cast<float*>(sm + bias_off);
   for (int o = tid; o < kHexH; o += kHexThreads) {
     bias[o] = __ldg(b1 + o);
@@ -952,6 +975,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     const bool valid = n < N;
     float xt[4] = {0.f, 0.f, 0.f, 0.f};
     if (valid) hex_normalise(mu, frame, n, hp, xt);
+    if (tile != blockIdx.x) stage_w23(sm, W2g, W3g);   // the last tile's scatter staging sat over them
     // ---- 1. forward ----
     float h1[32], h2[32];
 #pragma unroll
@@ -1099,42 +1123,57 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     };
     auto consume2 = [&](int k, int b) {
       const uint32_t S = tmem + 128 * b;
-      float a[16], c[16];
-      tc::tmem_ld16(S + lane + half * 16, a);
-      tc::tmem_ld16(S + 32 + lane + half * 16, c);
-      if (valid) {
-        const PlaneSample ps = plane_sample(xt, hp, k);
-        const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
-        const float w[4] = {ps.w00, ps.w01, ps.w10, ps.w11};
+      float dz[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a[i] += c[i];
+      for (int h = 0; h < 2; ++h) {   // both threads of a Gaussian read its whole dz row
+        float a[16], c[16];
+        tc::tmem_ld16(S + lane + 16 * h, a);
+        tc::tmem_ld16(S + 32 + lane + 16 * h, c);
 #pragma unroll
-        for (int cn = 0; cn < 4; ++cn) {
-          float4* g = reinterpret_cast<float4*>(grad_planes + off[cn]) + half * 4;
+        for (int i = 0; i < 16; ++i) dz[16 * h + i] = a[i] + c[i];
+      }
+      {
+        float a[16], c[16];
+        tc::tmem_ld16(S + 64 + lane + (warp >> 2) * 16, a);
+        tc::tmem_ld16(S + 96 + lane + (warp >> 2) * 16, c);
+        tc::fence_before_sync();
+        if (wrow_ok) {   // this thread alone updates these slot elements: see slot_add32
+          float4* dst = reinterpret_cast<float4*>(sW1 + (size_t)wrow * IN + k * kHexC + (warp >> 2) * 16);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            atomicAdd(g + q, make_float4(w[cn] * a[4 * q], w[cn] * a[4 * q + 1], w[cn] * a[4 * q + 2],
-                                         w[cn] * a[4 * q + 3]));
+            atomicAdd(dst + q, make_float4(a[4 * q] + c[4 * q], a[4 * q + 1] + c[4 * q + 1],
+                                           a[4 * q + 2] + c[4 * q + 2], a[4 * q + 3] + c[4 * q + 3]));
         }
       }
-      tc::tmem_ld16(S + 64 + lane + (warp >> 2) * 16, a);
-      tc::tmem_ld16(S + 96 + lane + (warp >> 2) * 16, c);
-      tc::fence_before_sync();
-      if (wrow_ok) {   // this thread alone updates these slot elements: see slot_add32
-        float4* dst = reinterpret_cast<float4*>(sW1 + (size_t)wrow * IN + k * kHexC + (warp >> 2) * 16);
+      if (valid) {
+        // corners 2*half and 2*half + 1 are neighbouring cells along the
+        // plane's first axis, so their gradient rows are contiguous: w_c * dz
+        // is staged as those two 128-byte rows and added with one bulk
+        // reduction
+        const PlaneSample ps = plane_sample(xt, hp, k);
+        bulk_wait_read();   // this thread's rows of the previous sample have been read
+        uint8_t* rows = sm + BL::SCAT + row * BL::SCAT_ROW;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          atomicAdd(dst + q, make_float4(a[4 * q] + c[4 * q], a[4 * q + 1] + c[4 * q + 1], a[4 * q + 2] + c[4 * q + 2],
-                                         a[4 * q + 3] + c[4 * q + 3]));
+        for (int cc = 0; cc < 2; ++cc) {
+          const float w = half ? (cc ? ps.w11 : ps.w10) : (cc ? ps.w01 : ps.w00);
+          float4* d = reinterpret_cast<float4*>(rows + (2 * half + cc) * (kHexC * 4));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) d[q] = make_float4(w * dz[4 * q], w * dz[4 * q + 1], w * dz[4 * q + 2], w * dz[4 * q + 3]);
+        }
+        tc::fence_proxy_async();
+        bulk_add_2rows(grad_planes + (half ? ps.o10 : ps.o00), tc::smem_u32(rows + 2 * half * (kHexC * 4)));
+        bulk_commit();
       }
     };
     if (!hex_stream<LATENT ? 2 : 1, LATENT>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
       failed = true;
       break;
     }
+    bulk_wait_read();   // the staging rows are W2 | W3 again in the next tile
     tc::fence_before_sync();
     __syncthreads();
   }
+  bulk_wait_all();
 
   if (failed) {
     if (tid == 0) atomicExch(&g_hex_device_error, 1);

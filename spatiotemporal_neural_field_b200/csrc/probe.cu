@@ -82,13 +82,14 @@ __global__ void __launch_bounds__(256) probe_atomic_kernel(float* __restrict__ b
   }
 }
 
-// Each thread owns a 128-byte row of ones in shared memory and adds it to
-// random 128-byte rows of buf with bulk asynchronous reductions, at most 8
-// of its own in flight.
+// Each thread owns a row of ones (RB bytes) in shared memory and adds it to
+// random RB-byte rows of buf with bulk asynchronous reductions, at most 8 of
+// its own in flight.
+template <int RB>
 __global__ void __launch_bounds__(128) probe_bulk_reduce_kernel(float* __restrict__ buf, uint64_t n_rows, int64_t ops,
                                                                 uint32_t seed) {
-  __shared__ __align__(128) float rows[128][32];
-  for (int i = 0; i < 32; ++i) rows[threadIdx.x][i] = 1.0f;
+  __shared__ __align__(128) float rows[128][RB / 4];
+  for (int i = 0; i < RB / 4; ++i) rows[threadIdx.x][i] = 1.0f;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
@@ -97,8 +98,8 @@ __global__ void __launch_bounds__(128) probe_bulk_reduce_kernel(float* __restric
   for (int64_t i = 0; i < ops; ++i) {
     state = mix32(state + 0x6D2B79F5u);
     const uint64_t r = ((uint64_t)state * n_rows) >> 32;
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 128;" ::"l"(buf + r * 32),
-                 "r"(src)
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(buf + r * (RB / 4)),
+                 "r"(src), "n"(RB)
                  : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     asm volatile("cp.async.bulk.wait_group.read 8;" ::: "memory");
@@ -195,11 +196,17 @@ extern "C" int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int
   return launch_status();
 }
 
-extern "C" int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int64_t rows_per_thread, int blocks,
-                                        uint32_t seed, spin4d_stream_t stream) {
-  if (!buf || buf_bytes < 128 || rows_per_thread < 1 || blocks < 1 || !aligned(buf, 128)) return SPIN4D_ERR_INVALID;
+extern "C" int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int row_bytes, int64_t rows_per_thread,
+                                        int blocks, uint32_t seed, spin4d_stream_t stream) {
+  if (!buf || (row_bytes != 128 && row_bytes != 256) || buf_bytes < (uint64_t)row_bytes || rows_per_thread < 1 ||
+      blocks < 1 || !aligned(buf, 128))
+    return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_probe_bulk_reduce")) return SPIN4D_ERR_INJECTED;
-  probe_bulk_reduce_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(static_cast<float*>(buf), buf_bytes / 128,
-                                                                     rows_per_thread, seed);
+  float* b = static_cast<float*>(buf);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (row_bytes == 128)
+    probe_bulk_reduce_kernel<128><<<blocks, 128, 0, s>>>(b, buf_bytes / 128, rows_per_thread, seed);
+  else
+    probe_bulk_reduce_kernel<256><<<blocks, 128, 0, s>>>(b, buf_bytes / 256, rows_per_thread, seed);
   return launch_status();
 }

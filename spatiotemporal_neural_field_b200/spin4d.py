@@ -90,7 +90,7 @@ _SIGS = {
     "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
     "spin4d_probe_stream": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i32, c_vp, c_vp]),
     "spin4d_probe_atomic": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
-    "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i64, c_i32, c_u32, c_vp]),
+    "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
@@ -343,10 +343,12 @@ def probe_atomic(buf: torch.Tensor, width: int, ops_per_thread: int, blocks: int
     return blocks * 256 * ops_per_thread
 
 
-def probe_bulk_reduce(buf: torch.Tensor, rows_per_thread: int, blocks: int, seed: int = 1, stream=None) -> int:
-    """Random 128-byte bulk fp32 reductions into `buf`; returns the rows added."""
+def probe_bulk_reduce(buf: torch.Tensor, rows_per_thread: int, blocks: int, seed: int = 1, row_bytes: int = 128,
+                      stream=None) -> int:
+    """Random bulk fp32 row reductions into `buf`; returns the rows added."""
     _check("spin4d_probe_bulk_reduce", lib.spin4d_probe_bulk_reduce(_ptr(buf), buf.numel() * buf.element_size(),
-                                                                    rows_per_thread, blocks, seed, _stream(stream)))
+                                                                    row_bytes, rows_per_thread, blocks, seed,
+                                                                    _stream(stream)))
     return blocks * 128 * rows_per_thread
 
 

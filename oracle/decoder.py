@@ -238,10 +238,15 @@ def decode_forward(pos, tables, weights, grid, mlp, gate_cr=None, normalised_inp
     return out
 
 
-def decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=None, normalised_input=False):
+def decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=None, normalised_input=False,
+                    want_pos=False):
     """Gradients of sum_k <grads[k], output_k> w.r.t. the tables and weights.
 
-    Returns (grad_tables L x T x F, grad_weights packed like ``weights``)."""
+    Returns (grad_tables L x T x F, grad_weights packed like ``weights``), and
+    with ``want_pos`` also grad_pos N x 3: the gradient w.r.t. the spatial
+    position (x, y, z) through the interpolation weights and Eq. 7 (w.r.t. the
+    normalised coordinates themselves when ``normalised_input``).  The
+    timestamp is data, not a parameter, and gets none."""
     res, xt = _prepare(pos, grid, normalised_input)
     z = hashgrid.encode(xt, tables, res, grid.log2_T)
     layers = unpack_layers(weights, mlp.layer_shapes())
@@ -250,7 +255,15 @@ def decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=None, normal
     dy = heads_backward(y, g64, _gate_for(xt, mlp, gate_cr))
     dz, wgrads = mlp_backward(dy, layers, acts, pres)
     gt = hashgrid.scatter_table_grad(dz, xt, res, grid.log2_T, grid.L, grid.F)
-    return gt, pack_layers(wgrads)
+    if not want_pos:
+        return gt, pack_layers(wgrads)
+    gx = hashgrid.encode_position_grad(dz, xt, tables, res, grid.log2_T)[:, :3]
+    p32 = np.asarray(pos, np.float32)
+    if normalised_input:
+        gpos = gx * hashgrid.clamp_passes(p32[:, :3])
+    else:
+        gpos = np.einsum("ni,nij->nj", gx, hashgrid.contraction_jacobian(p32))
+    return gt, pack_layers(wgrads), gpos
 
 
 def adam_step(p, g, m, v, step: int, lr: float, b1: float, b2: float, eps: float):

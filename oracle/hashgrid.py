@@ -170,3 +170,66 @@ def scatter_table_grad(dz: np.ndarray, xt: np.ndarray, res: np.ndarray, log2_T: 
                                         weights=(wts[:, l, :] * g[:, None]).reshape(-1),
                                         minlength=T)
     return grad
+
+
+# ---------------------------------------------------------------------------
+# Position gradient (trainable Gaussian means, SPIN-4DGS section 3.3: the
+# positions are optimised jointly with the decoder)
+# ---------------------------------------------------------------------------
+def contraction_jacobian(pos: np.ndarray) -> np.ndarray:
+    """d mu_bar / d mu of Eq. 7, N x 3 x 3 fp64, at the fp32 positions.
+
+    Inside the unit ball mu_bar = mu/4 + 1/2, so the Jacobian is I/4.
+    Outside, c = (2 - 1/n) mu / n = (2/n - 1/n^2) mu with n = |mu|, so
+    dc/dmu = (2/n - 1/n^2) I + (2/n^4 - 2/n^3) mu mu^T, and mu_bar = c/4 + 1/2.
+    The branch is the one the fp32 normalisation takes (n <= 1 in fp32)."""
+    mu32 = np.asarray(pos, F32)[:, :3]
+    x, y, z = mu32[:, 0], mu32[:, 1], mu32[:, 2]
+    inside = np.sqrt((x * x + y * y) + z * z) <= F32(1)
+    mu = mu32.astype(np.float64)
+    n = np.sqrt(np.sum(mu * mu, axis=1))
+    eye = np.broadcast_to(np.eye(3), (mu.shape[0], 3, 3))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        g = 2.0 / n - 1.0 / n ** 2
+        h = 2.0 / n ** 4 - 2.0 / n ** 3
+        out = g[:, None, None] * eye + h[:, None, None] * mu[:, :, None] * mu[:, None, :]
+    out = np.where(inside[:, None, None], eye, out)
+    return 0.25 * out
+
+
+def clamp_passes(v: np.ndarray) -> np.ndarray:
+    """Mask of the clamp to [0, 1]: 1 where the value passes unchanged."""
+    v = np.asarray(v)
+    return ((v >= 0) & (v <= 1)).astype(np.float64)
+
+
+def encode_position_grad(dz: np.ndarray, xt: np.ndarray, tables: np.ndarray, res: np.ndarray,
+                         log2_T: int) -> np.ndarray:
+    """Adjoint of ``encode`` w.r.t. the normalised position, N x 4 fp64.
+
+    z_l = sum_c W_c e_c with W_c = prod_d (bit_d ? w_d : 1 - w_d) and
+    w_d = x~_d (res_d - 1) - base_d, so
+    d<dz_l, z_l>/dx~_d = (res_d - 1) sum_c (dz_l . e_c) dW_c/dw_d,
+    dW_c/dw_d = (bit_d ? 1 : -1) prod_{e != d} (bit_e ? w_e : 1 - w_e)
+    (the derivative inside the cell; the interpolant is continuous across
+    cells, its derivative is taken from the cell the position falls in)."""
+    L, T, F = tables.shape
+    _, frac, idx = corner_select(xt, res, log2_T)
+    w = frac.astype(np.float64)
+    N = xt.shape[0]
+    g = np.zeros((N, 4), np.float64)
+    for l in range(L):
+        s = np.zeros((N, 16), np.float64)          # dz_l . e_c per corner
+        for f in range(F):
+            col = np.ascontiguousarray(tables[l, :, f]).astype(np.float64)
+            s += dz[:, l * F + f][:, None] * np.take(col, idx[:, l, :].astype(np.int64))
+        for d in range(4):
+            acc = np.zeros(N, np.float64)
+            for c in range(16):
+                dw = np.ones(N, np.float64) if (c >> d) & 1 else -np.ones(N, np.float64)
+                for e in range(4):
+                    if e != d:
+                        dw = dw * (w[:, l, e] if (c >> e) & 1 else 1.0 - w[:, l, e])
+                acc += s[:, c] * dw
+            g[:, d] += (int(res[l, d]) - 1) * acc
+    return g

@@ -189,6 +189,28 @@ int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                       void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 
 /*
+ * spin4d_decode_bwd that also accumulates the gradient w.r.t. the Gaussian
+ * means (SPIN-4DGS section 3.3 trains the positions jointly with the
+ * decoder):
+ *   grad_pos += dloss/d(x, y, z)   (N x 3 fp32, 4-byte aligned, not NULL)
+ * through the quadrilinear interpolation weights of every level (the
+ * derivative inside the cell the position falls in, times res - 1 per axis)
+ * and the Jacobian of Eq. 7 (I/4 inside the unit ball; outside, the
+ * contracted point 2 - 1/|mu| along the ray of mu).  With
+ * SPIN4D_INPUT_NORMALISED it is the gradient w.r.t. the normalised
+ * coordinates, zero where the clamp to [0, 1] bound.  The timestamp is data,
+ * not a parameter: it gets no gradient.  The corner entries are gathered
+ * again for this even when `latent` is given.  Each position's three values
+ * are written by one thread (no atomics).  Other arguments, results and
+ * errors are those of spin4d_decode_bwd.
+ */
+int spin4d_decode_bwd_pos(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
+                          const float* pos, int64_t N, const void* tables, const void* weights,
+                          const float* gate_cr, const float* latent, const spin4d_output_grads* grad_out,
+                          float* grad_tables, float* grad_weights, float* grad_pos,
+                          void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
  * spin4d_decode_bwd without a workspace argument, for callers that cannot
  * allocate device memory (hosts that own all device memory and hand the
  * library only its input and output buffers, or loops that may not call

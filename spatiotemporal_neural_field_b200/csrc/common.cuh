@@ -249,6 +249,77 @@ __device__ __forceinline__ void encode_level_f16_paired(const float xt[4], const
 }
 
 // ---------------------------------------------------------------------------
+// Position gradient (trainable Gaussian means).
+// ---------------------------------------------------------------------------
+// gx[d] += d<dz, z_l>/dx~_d for one level: inside the position's cell
+// z_l = sum_c W_c e_c with W_c = prod_d (bit_d ? w_d : 1 - w_d) and
+// w_d = x~_d (res_d - 1) - base_d, so the derivative is
+// (res_d - 1) sum_c (dz . e_c) dW_c/dw_d,
+// dW_c/dw_d = (bit_d ? 1 : -1) prod_{e != d} (bit_e ? w_e : 1 - w_e).
+template <typename T, int F>
+__device__ __forceinline__ void level_position_grad(const float xt[4], const GridParams& g, int l,
+                                                    const T* __restrict__ tables, const float dz[F], float gx[4]) {
+  uint32_t base[4];
+  float frac[4];
+  level_cell(xt, g, l, base, frac);
+  uint32_t idx[16];
+  level_indices(base, g, l, idx);
+  const T* tab = tables + ((size_t)l << g.log2_T) * F;
+  float s[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    float v[F];
+    Entry<T, F>::load(tab, idx[c], v);
+    float a = 0.0f;
+#pragma unroll
+    for (int f = 0; f < F; ++f) a = fmaf(dz[f], v[f], a);
+    s[c] = a;
+  }
+#pragma unroll
+  for (int d = 0; d < 4; ++d) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float p = ((c >> d) & 1) ? s[c] : -s[c];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e != d) p *= ((c >> e) & 1) ? frac[e] : 1.0f - frac[e];
+      acc += p;
+    }
+    gx[d] = fmaf(acc, g.scale[l][d], gx[d]);
+  }
+}
+
+// Gradient w.r.t. the raw spatial position from the gradient w.r.t. the
+// normalised coordinates: Eq. 7's Jacobian, I/4 inside the unit ball and
+// (g I + h mu mu^T)/4 outside with g = 2/n - 1/n^2, h = 2/n^4 - 2/n^3 (the
+// contracted point 2 - 1/n along the ray of mu).  For normalised input, the
+// clamp to [0, 1] alone: the gradient passes where the input was in range.
+__device__ __forceinline__ void position_grad_chain(float4 p, const GridParams& g, const float gx[4], float out[3]) {
+  if (g.flags & SPIN4D_INPUT_NORMALISED) {
+    out[0] = (p.x >= 0.0f && p.x <= 1.0f) ? gx[0] : 0.0f;
+    out[1] = (p.y >= 0.0f && p.y <= 1.0f) ? gx[1] : 0.0f;
+    out[2] = (p.z >= 0.0f && p.z <= 1.0f) ? gx[2] : 0.0f;
+    return;
+  }
+  const float n2 = __fadd_rn(__fadd_rn(__fmul_rn(p.x, p.x), __fmul_rn(p.y, p.y)), __fmul_rn(p.z, p.z));
+  const float n = __fsqrt_rn(n2);
+  if (n <= 1.0f) {
+    out[0] = 0.25f * gx[0];
+    out[1] = 0.25f * gx[1];
+    out[2] = 0.25f * gx[2];
+    return;
+  }
+  const float in = 1.0f / n;
+  const float gg = in * (2.0f - in);                 // 2/n - 1/n^2
+  const float hh = 2.0f * in * in * in * (in - 1.0f);   // 2/n^4 - 2/n^3
+  const float dot = p.x * gx[0] + p.y * gx[1] + p.z * gx[2];
+  out[0] = 0.25f * (gg * gx[0] + hh * dot * p.x);
+  out[1] = 0.25f * (gg * gx[1] + hh * dot * p.y);
+  out[2] = 0.25f * (gg * gx[2] + hh * dot * p.z);
+}
+
+// ---------------------------------------------------------------------------
 // Scatter-add of the adjoint: grad_l[idx_c][f] += w_c * dz[f]  (fp32 atomics).
 // ---------------------------------------------------------------------------
 template <int F>

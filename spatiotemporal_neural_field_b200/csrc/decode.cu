@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
                                                              const float2* __restrict__ gate_cr,
                                                              const float* __restrict__ latent, GradPtrs go,
                                                              float* __restrict__ grad_tables,
+                                                             float* __restrict__ grad_pos,
                                                              float* __restrict__ ws, int n_params) {
   extern __shared__ float smem[];
   const int H = m.hidden, IN = m.in_dim, NH = m.n_hidden;
@@ -253,13 +254,21 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
       __syncthreads();
       float* t = dA; dA = dB; dB = t;
     }
-    // ---- scatter dz into the tables ----
+    // ---- scatter dz into the tables; position gradient ----
     if (valid) {
+      float gx[4] = {0.f, 0.f, 0.f, 0.f};
       for (int l = 0; l < g.L; ++l) {
         float dz[F];
 #pragma unroll
         for (int f = 0; f < F; ++f) dz[f] = dA[(l * F + f) * kBwdBlock + col];
         scatter_level<F>(xt, g, l, grad_tables, dz);
+        if (grad_pos) level_position_grad<T, F>(xt, g, l, tables, dz, gx);
+      }
+      if (grad_pos) {
+        float gp[3];
+        position_grad_chain(pos[n], g, gx, gp);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) grad_pos[3 * n + i] += gp[i];
       }
     }
     __syncthreads();
@@ -304,14 +313,15 @@ static int launch_fwd(const GridParams& gp, const MlpParams& mp, size_t smem, co
 template <typename T, int F, typename W>
 static int launch_bwd(const GridParams& gp, const MlpParams& mp, size_t smem, const float* pos, int64_t N,
                       const void* tables, const void* weights, const float* gate_cr, const float* latent, GradPtrs go,
-                      float* grad_tables, float* grad_weights, float* ws, int n_params, cudaStream_t s) {
+                      float* grad_tables, float* grad_pos, float* grad_weights, float* ws, int n_params,
+                      cudaStream_t s) {
   auto k = decode_bwd_simt<T, F, W>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
   int blocks = bwd_blocks(N);
   k<<<blocks, kBwdBlock, smem, s>>>(gp, mp, reinterpret_cast<const float4*>(pos), N,
                                     static_cast<const T*>(tables), static_cast<const W*>(weights),
-                                    reinterpret_cast<const float2*>(gate_cr), latent, go, grad_tables, ws, n_params);
+                                    reinterpret_cast<const float2*>(gate_cr), latent, go, grad_tables, grad_pos, ws, n_params);
   SPIN4D_CHECK(launch_status());
   int rb = (n_params + 255) / 256;
   reduce_slots<<<rb, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
@@ -377,7 +387,7 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
 int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* m);
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                   const void* tables, const void* weights, const float* gate_cr, const float* latent,
-                  const spin4d_output_grads* go, float* grad_tables, float* grad_weights, float* ws, int n_params,
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* ws, int n_params,
                   int blocks, cudaStream_t s);
 
 // Thread blocks (= workspace slots) the backward launches for N positions.
@@ -415,35 +425,57 @@ extern "C" size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const s
   return (size_t)bwd_slots(g, m, N) * slot_stride((int)spin4d_mlp_param_count(m)) * sizeof(float);
 }
 
-extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
-                                 const void* tables, const void* weights, const float* gate_cr, const float* latent,
-                                 const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
-                                 void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
+namespace spin4d {
+
+// spin4d_decode_bwd with an optional position gradient (grad_pos may be NULL).
+static int decode_bwd_impl(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
+                           const void* tables, const void* weights, const float* gate_cr, const float* latent,
+                           const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
+                           float* grad_pos, void* workspace, size_t ws_bytes, cudaStream_t s, const char* name) {
   SPIN4D_CHECK(check_common(g, m, pos, N, tables, weights, gate_cr));
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_tables || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_tables, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256) ||
-      (latent && !aligned(latent, 16)))
+      (latent && !aligned(latent, 16)) || (grad_pos && !aligned(grad_pos, 4)))
     return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_decode_bwd_workspace(g, m, N)) return SPIN4D_ERR_INVALID;
   if (grad_out->rot && !aligned(grad_out->rot, 4)) return SPIN4D_ERR_INVALID;
   const bool tc = decode_bwd_tc_ctas_per_sm(g, m) > 0;
   if (!tc && bwd_smem(m) > 220 * 1024) return SPIN4D_ERR_UNSUPPORTED;
-  if (fault_injected("spin4d_decode_bwd")) return SPIN4D_ERR_INJECTED;
+  if (fault_injected(name)) return SPIN4D_ERR_INJECTED;
   int n_params = (int)spin4d_mlp_param_count(m);
   if (tc) {
-    cudaStream_t s = (cudaStream_t)stream;
     const int blocks = bwd_slots(g, m, N);
     float* ws = static_cast<float*>(workspace);
-    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
-                               ws, n_params, blocks, s));
+    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_pos, ws,
+                               n_params, blocks, s));
     reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
     return launch_status();
   }
   GradPtrs go{grad_out->scale, grad_out->rot, grad_out->rgb, grad_out->opacity, grad_out->cov};
   return dispatch<BwdFn>(g->table_dtype, g->F, m->w_dtype, make_grid_params(g), make_mlp(m), bwd_smem(m), pos,
-                         N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
-                         static_cast<float*>(workspace), n_params, (cudaStream_t)stream);
+                         N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, grad_weights,
+                         static_cast<float*>(workspace), n_params, s);
+}
+
+}  // namespace spin4d
+
+extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
+                                 const void* tables, const void* weights, const float* gate_cr, const float* latent,
+                                 const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
+                                 void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
+  return decode_bwd_impl(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
+                         nullptr, workspace, ws_bytes, (cudaStream_t)stream, "spin4d_decode_bwd");
+}
+
+extern "C" int spin4d_decode_bwd_pos(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos,
+                                     int64_t N, const void* tables, const void* weights, const float* gate_cr,
+                                     const float* latent, const spin4d_output_grads* grad_out, float* grad_tables,
+                                     float* grad_weights, float* grad_pos, void* workspace, size_t ws_bytes,
+                                     spin4d_stream_t stream) {
+  if (N > 0 && !grad_pos) return SPIN4D_ERR_INVALID;
+  return decode_bwd_impl(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
+                         grad_pos, workspace, ws_bytes, (cudaStream_t)stream, "spin4d_decode_bwd_pos");
 }
 
 // ---------------------------------------------------------------------------

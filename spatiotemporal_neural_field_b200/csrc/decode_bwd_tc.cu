@@ -266,7 +266,7 @@ template <int F, int IN, int H>
 __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kernel(
     GridParams g, int gate, float tau, const float4* __restrict__ pos, int64_t N, const __half* __restrict__ tables,
     const __half* __restrict__ weights, const float2* __restrict__ gate_cr, const float* __restrict__ latent, GradIn go,
-    float* __restrict__ grad_tables, float* __restrict__ ws, int n_params) {
+    float* __restrict__ grad_tables, float* __restrict__ grad_pos, float* __restrict__ ws, int n_params) {
   using Lay = BLayout<IN, H>;
   // TMEM columns: two per-tile regions of H, then the weight-gradient
   // accumulators dW1 (IN), dW2 (H), dWh^T (16)
@@ -544,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
       }
       tc::fence_before_sync();
       const float id1 = 1.0f / s_d1;
+      float gx[4] = {0.f, 0.f, 0.f, 0.f};
       if (valid) {
         constexpr int LV = HALF_IN / F;
 #pragma unroll 1
@@ -552,6 +553,22 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 #pragma unroll
           for (int f = 0; f < F; ++f) dz[f] = dzv[q * F + f] * id1;
           scatter_level_paired<F>(xt, g, half * LV + q, grad_tables, dz);
+          if (grad_pos) level_position_grad<__half, F>(xt, g, half * LV + q, tables, dz, gx);
+        }
+      }
+      if (grad_pos) {
+        // the two halves' level sums meet in the (now free) dy tile; half 0
+        // applies Eq. 7's Jacobian and owns the position's output
+        float4* part = reinterpret_cast<float4*>(sm + Lay::dyt);
+        part[half * kTile + row] = make_float4(gx[0], gx[1], gx[2], gx[3]);
+        __syncthreads();
+        if (half == 0 && valid) {
+          const float4 o = part[kTile + row];
+          const float sum[4] = {gx[0] + o.x, gx[1] + o.y, gx[2] + o.z, gx[3] + o.w};
+          float gp[3];
+          position_grad_chain(pos[n], g, sum, gp);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) grad_pos[3 * n + i] += gp[i];
         }
       }
     }
@@ -574,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 template <int F, int IN, int H>
 int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* pos, int64_t N, const void* tables,
                   const void* weights, const float* gate_cr, const float* latent, const spin4d_output_grads* go,
-                  float* grad_tables, float* grad_weights, float* ws, int n_params, int blocks, cudaStream_t s) {
+                  float* grad_tables, float* grad_pos, float* ws, int n_params, int blocks, cudaStream_t s) {
   using Lay = BLayout<IN, H>;
   auto k = decode_bwd_tc_kernel<F, IN, H>;
   const int smem = align_up(Lay::bytes, 128);
@@ -593,7 +610,8 @@ int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* p
   GradIn gi{go->scale, go->rot, go->rgb, go->opacity, go->cov};
   k<<<blocks, kThreads, smem, s>>>(gp, m->gate, m->tau, reinterpret_cast<const float4*>(pos), N,
                                    static_cast<const __half*>(tables), static_cast<const __half*>(weights),
-                                   reinterpret_cast<const float2*>(gate_cr), latent, gi, grad_tables, ws, n_params);
+                                   reinterpret_cast<const float2*>(gate_cr), latent, gi, grad_tables, grad_pos, ws,
+                                   n_params);
   return launch_status();
 }
 
@@ -622,15 +640,15 @@ int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* 
 
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                   const void* tables, const void* weights, const float* gate_cr, const float* latent,
-                  const spin4d_output_grads* go, float* grad_tables, float* grad_weights, float* ws, int n_params,
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* ws, int n_params,
                   int blocks, cudaStream_t s) {
   const GridParams gp = make_grid_params(g);
   if (g->F == 2 && m->in_dim == 32 && m->hidden == 64)
-    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
-                                    ws, n_params, blocks, s);
+    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, ws,
+                                    n_params, blocks, s);
   if (g->F == 4 && m->in_dim == 64 && m->hidden == 128)
-    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_weights,
-                                     ws, n_params, blocks, s);
+    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, ws,
+                                     n_params, blocks, s);
   return SPIN4D_ERR_UNSUPPORTED;
 }
 

@@ -73,6 +73,8 @@ _SIGS = {
     "spin4d_decode_bwd_workspace": (c_sz, [P(GridDesc), P(MlpDesc), c_i64]),
     "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
                                   c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_decode_bwd_pos": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
+                                      c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_decode_bwd_noalloc": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
                                           P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
@@ -220,17 +222,22 @@ def decode_bwd_workspace(g: GridDesc, m: MlpDesc, N: int) -> int:
 def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
                grad_tables: torch.Tensor, grad_weights: torch.Tensor, gate_cr=None,
                workspace: Optional[torch.Tensor] = None, latent: Optional[torch.Tensor] = None,
-               stream=None) -> None:
-    """latent: the z saved by decode_fwd for the same positions (optional)."""
+               grad_pos: Optional[torch.Tensor] = None, stream=None) -> None:
+    """latent: the z saved by decode_fwd for the same positions (optional);
+    grad_pos: N x 3 fp32 accumulating the position gradient (optional)."""
     N = pos.shape[0]
     need = decode_bwd_workspace(g, m, N)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
     go = OutputGrads(*(_ptr(grads.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov")))
-    _check("spin4d_decode_bwd", lib.spin4d_decode_bwd(ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables),
-                                                      _ptr(weights), _ptr(gate_cr), _ptr(latent), ctypes.byref(go),
-                                                      _ptr(grad_tables), _ptr(grad_weights), _ptr(workspace),
-                                                      workspace.numel(), _stream(stream)))
+    common = (ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables), _ptr(weights), _ptr(gate_cr),
+              _ptr(latent), ctypes.byref(go), _ptr(grad_tables), _ptr(grad_weights))
+    if grad_pos is None:
+        _check("spin4d_decode_bwd", lib.spin4d_decode_bwd(*common, _ptr(workspace), workspace.numel(),
+                                                          _stream(stream)))
+    else:
+        _check("spin4d_decode_bwd_pos", lib.spin4d_decode_bwd_pos(*common, _ptr(grad_pos), _ptr(workspace),
+                                                                  workspace.numel(), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -105,6 +105,11 @@ def test_invalid_arguments_rejected_on_host(sp):
     # misaligned saved latent
     assert lib.spin4d_decode_fwd(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None,
                                  sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4), None) == sp.ERR_INVALID
+    # position gradient: grad_pos must be given, 4-byte aligned
+    assert lib.spin4d_decode_bwd_pos(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, None,
+                                     FAKE, 1 << 30, None) == sp.ERR_INVALID
+    assert lib.spin4d_decode_bwd_pos(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, FAKE + 2,
+                                     FAKE, 1 << 30, None) == sp.ERR_INVALID
     # adam
     assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 0, 1e-3, 0.9, 0.99, 1e-15, 0, None,
                                 None) == sp.ERR_INVALID

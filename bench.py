@@ -590,7 +590,14 @@ def run_workloads(args):
             sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr, workspace=ws, latent=out["latent"])
 
         emit(name, "fwd+bwd (saved latent)", n, timed(fb, reps))
-        del P, T, W, out, fwd_out, grads, gt, gw, ws
+        gpos = torch.zeros((n, 3), device=dev)
+
+        def fbp():
+            sp.decode_fwd(g, m, P, T, W, cr, out=out)
+            sp.decode_bwd(g, m, P, T, W, grads, gt, gw, gate_cr=cr, workspace=ws, latent=out["latent"], grad_pos=gpos)
+
+        emit(name, "fwd+bwd+position gradient (saved latent)", n, timed(fbp, reps))
+        del P, T, W, out, fwd_out, grads, gt, gw, ws, gpos
         torch.cuda.empty_cache()
 
     # HexPlane

@@ -357,6 +357,39 @@ int spin4d_debug_corners(const spin4d_grid_desc* g, const float* pos, int64_t N,
 int spin4d_check_device_errors(int clear);
 
 /*
+ * Z-order (Morton) ordering of the Gaussians, for gather locality (the
+ * KineticGS notes serialise particles onto a Z-order space-filling curve to
+ * keep spatial neighbours adjacent).  Decoding the Gaussians in this order
+ * makes each tile's positions neighbours, so their hash-table corners
+ * overlap in the caches.
+ *
+ * keys[n]: the 30-bit Z-order code of Gaussian n's normalised spatial
+ * coordinates (Eq. 7, the same fp32 arithmetic and SPIN4D_INPUT_NORMALISED
+ * handling as the decoder), 10 bits per axis, q = min(floor(mu_bar * 1024),
+ * 1023), bit b of axis d at bit 3b + d.  The time coordinate is not used.
+ * On return `keys` holds the codes sorted ascending and perm[i] is the input
+ * index of the i-th smallest, equal codes in input order (a stable sort: the
+ * result is deterministic).  pos N x 4 fp32 (16-byte aligned), keys and perm
+ * N uint32 (device, 4-byte aligned), workspace >=
+ * spin4d_morton_order_workspace(N) bytes (device, 256-byte aligned).
+ * 0 <= N <= SPIN4D_MAX_SORT.  Apply perm to every per-Gaussian array with
+ * spin4d_permute_rows; decoding then returns attributes in sorted order.
+ */
+#define SPIN4D_MAX_SORT (1ll << 30)
+size_t spin4d_morton_order_workspace(int64_t N);
+int spin4d_morton_order(const spin4d_grid_desc* g, const float* pos, int64_t N, uint32_t* keys, uint32_t* perm,
+                        void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
+ * dst row i = src row perm[i], i < N, rows of row_bytes bytes (a multiple of
+ * 4).  src has src_rows rows; a row whose perm entry is not below src_rows
+ * is left unwritten.  src and dst (device, 4-byte aligned, 16-byte aligned
+ * for the vectorised path) must not overlap.
+ */
+int spin4d_permute_rows(const void* src, int64_t src_rows, void* dst, const uint32_t* perm, int64_t N,
+                        int64_t row_bytes, spin4d_stream_t stream);
+
+/*
  * Measurement helper (not part of the decoder): the gather-rate ceiling.
  * Launches `blocks` x 256 threads; each issues `loads_per_thread` (a multiple
  * of 8) independent loads at pseudo-random, width-aligned offsets of `buf`

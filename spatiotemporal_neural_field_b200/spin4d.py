@@ -91,6 +91,9 @@ _SIGS = {
     "spin4d_selftest_wait_timeout": (c_i32, [c_u32, c_vp]),
     "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
     "spin4d_probe_stream": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i32, c_vp, c_vp]),
+    "spin4d_morton_order_workspace": (c_sz, [c_i64]),
+    "spin4d_morton_order": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_permute_rows": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp]),
     "spin4d_probe_atomic": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
@@ -341,6 +344,30 @@ def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: i
                                                           loads_per_thread, blocks, seed, _ptr(sink),
                                                           _stream(stream)))
     return blocks * 256 * loads_per_thread // (8 if width == 128 else 1)
+
+
+def morton_order(g: GridDesc, pos: torch.Tensor, workspace: Optional[torch.Tensor] = None, stream=None):
+    """(sorted 30-bit Z-order keys, permutation), both N int32 holding uint32 values."""
+    N = pos.shape[0]
+    keys = torch.empty(N, dtype=torch.int32, device=pos.device)
+    perm = torch.empty(N, dtype=torch.int32, device=pos.device)
+    need = int(lib.spin4d_morton_order_workspace(N))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
+    _check("spin4d_morton_order", lib.spin4d_morton_order(ctypes.byref(g), _ptr(pos), N, _ptr(keys), _ptr(perm),
+                                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+    return keys, perm
+
+
+def permute_rows(src: torch.Tensor, perm: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """out[i] = src[perm[i]] along the first dimension (contiguous tensors)."""
+    N = perm.shape[0]
+    if out is None:
+        out = torch.empty((N,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    row_bytes = src[0].numel() * src.element_size() if src.dim() > 1 else src.element_size()
+    _check("spin4d_permute_rows", lib.spin4d_permute_rows(_ptr(src), src.shape[0], _ptr(out), _ptr(perm), N,
+                                                          row_bytes, _stream(stream)))
+    return out
 
 
 def probe_atomic(buf: torch.Tensor, width: int, ops_per_thread: int, blocks: int, seed: int = 1, stream=None) -> int:

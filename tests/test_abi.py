@@ -110,6 +110,16 @@ def test_invalid_arguments_rejected_on_host(sp):
                                      FAKE, 1 << 30, None) == sp.ERR_INVALID
     assert lib.spin4d_decode_bwd_pos(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, FAKE + 2,
                                      FAKE, 1 << 30, None) == sp.ERR_INVALID
+    # ordering
+    assert lib.spin4d_morton_order_workspace(0) == 0
+    assert lib.spin4d_morton_order_workspace(1000) > 0
+    assert lib.spin4d_morton_order(ref(g), FAKE, 10, FAKE, FAKE, FAKE, 16, None) == sp.ERR_INVALID   # workspace
+    assert lib.spin4d_morton_order(ref(g), FAKE + 8, 10, FAKE, FAKE, FAKE, 1 << 30, None) == sp.ERR_INVALID
+    assert lib.spin4d_morton_order(ref(g), FAKE, -1, FAKE, FAKE, FAKE, 1 << 30, None) == sp.ERR_INVALID
+    assert lib.spin4d_morton_order(ref(g), None, 0, None, None, None, 0, None) == sp.OK
+    assert lib.spin4d_permute_rows(FAKE, 10, FAKE, FAKE, 10, 6, None) == sp.ERR_INVALID       # row bytes
+    assert lib.spin4d_permute_rows(FAKE, 10, FAKE, FAKE, 10, 8, None) == sp.ERR_INVALID       # src == dst
+    assert lib.spin4d_permute_rows(None, 0, None, None, 0, 8, None) == sp.OK
     # adam
     assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 0, 1e-3, 0.9, 0.99, 1e-15, 0, None,
                                 None) == sp.ERR_INVALID

@@ -439,6 +439,40 @@ def run_ours(args):
         train = train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, tables, weights, grid, mlp,
                                        g, m, flush, stream)
 
+    # ---- the same frame decoded in Z-order (spin4d_morton_order + spin4d_permute_rows) ----
+    morton = None
+    if not args.no_fwd_bwd:
+        ws_sort = torch.empty(max(sp.lib.spin4d_morton_order_workspace(N), 1), dtype=torch.uint8, device=dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            flush.zero_()
+            a.record(stream)
+            _, perm = sp.morton_order(g, pos, workspace=ws_sort, stream=stream)
+            pos_sorted = sp.permute_rows(pos, perm, stream=stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+        sort_ms = a.elapsed_time(b)
+
+        def step_sorted():
+            sp.decode_fwd(g, m, pos_sorted, tables, weights, out=out, stream=stream)
+
+        for _ in range(args.warmup):
+            step_sorted()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step_sorted()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms_s = dp.max_over_ranks(sum(x.elapsed_time(y) for x, y in evs), device=dev) / args.steps
+        morton = {"value": N * world / (ms_s * 1e-3), "unit": UNIT, "ms_per_step": ms_s,
+                  "sort_ms": sort_ms,
+                  "note": "the same frame with the Gaussians in Z-order of their normalised positions (sorted once, "
+                          "outside the timed steps: the order is per scene, every frame reuses it); "
+                          "sort_ms = spin4d_morton_order + spin4d_permute_rows of the positions"}
+
     gather = None
     if not args.no_probe:
         rates = probe_sector_rates(sp, torch, dev)
@@ -473,6 +507,8 @@ def run_ours(args):
             line["gather_roofline"] = gather
         if train:
             line["train_step"] = train
+        if morton:
+            line["morton_sorted"] = morton
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.cpu_sample)
         print(json.dumps(line), flush=True)
@@ -577,6 +613,21 @@ def run_workloads(args):
         where = "hbm" if name == "stress_fp16_gate" else "l2"
         emit(name, "fwd", n, ms, table_sectors_per_position=spp, sector_rate=rate,
              frac_of_random_sector_ceiling=rate / ceil[where + "_random_sector_per_s"], ceiling=where)
+        if name in ("sports_frame_fp16", "stress_fp16_gate"):
+            ws_sort = torch.empty(max(sp.lib.spin4d_morton_order_workspace(n), 1), dtype=torch.uint8, device=dev)
+            for _ in range(2):   # the first call allocates the outputs; time the second
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.zero_()
+                a.record()
+                _, perm = sp.morton_order(g, P, workspace=ws_sort)
+                Ps = sp.permute_rows(P, perm)
+                crs = sp.permute_rows(cr, perm) if cr is not None else None
+                b.record()
+                torch.cuda.synchronize()
+            ms_s = timed(lambda: sp.decode_fwd(g, m, Ps, T, W, crs, out=fwd_out), reps)
+            emit(name, "fwd (Z-order sorted)", n, ms_s, sort_and_permute_ms=a.elapsed_time(b),
+                 table_sectors_per_position=spp, sector_rate=spp * n / (ms_s * 1e-3))
+            del Ps, crs, perm, ws_sort
         if name == "sports_frame_fp16":
             continue
         grads = {k: torch.randn((n, wd), device=dev) * (1e-2 if grid.dtype == "f16" else 1.0)

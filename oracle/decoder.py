@@ -148,6 +148,17 @@ def temporal_gate(t: np.ndarray, c: np.ndarray, r: np.ndarray, tau: float) -> np
     return sigmoid((t - (c - r)) / tau) * sigmoid(((c + r) - t) / tau)
 
 
+def temporal_gate_grad(t: np.ndarray, c: np.ndarray, r: np.ndarray, tau: float) -> Tuple[np.ndarray, np.ndarray]:
+    """(dw/dc, dw/dr) of w = a b, a = sigma((t - (c - r))/tau), b = sigma(((c + r) - t)/tau).
+
+    sigma' = sigma (1 - sigma): da/dc = -a(1-a)/tau, db/dc = b(1-b)/tau, so
+    dw/dc = a b (a - b)/tau; da/dr = a(1-a)/tau, db/dr = b(1-b)/tau, so
+    dw/dr = a b (2 - a - b)/tau."""
+    a = sigmoid((t - (c - r)) / tau)
+    b = sigmoid(((c + r) - t) / tau)
+    return a * b * (a - b) / tau, a * b * (2.0 - a - b) / tau
+
+
 # ---------------------------------------------------------------------------
 # Network
 # ---------------------------------------------------------------------------
@@ -239,14 +250,17 @@ def decode_forward(pos, tables, weights, grid, mlp, gate_cr=None, normalised_inp
 
 
 def decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=None, normalised_input=False,
-                    want_pos=False):
+                    want_pos=False, want_gate=False):
     """Gradients of sum_k <grads[k], output_k> w.r.t. the tables and weights.
 
     Returns (grad_tables L x T x F, grad_weights packed like ``weights``), and
     with ``want_pos`` also grad_pos N x 3: the gradient w.r.t. the spatial
     position (x, y, z) through the interpolation weights and Eq. 7 (w.r.t. the
     normalised coordinates themselves when ``normalised_input``).  The
-    timestamp is data, not a parameter, and gets none."""
+    timestamp is data, not a parameter, and gets none.  With ``want_gate``
+    (gated decoders) also grad_cr N x 2, the gradient w.r.t. the window
+    centre c and half-width r of the KineticGS gate: o = sigma(o^) w, so
+    dloss/dw = g_o sigma(o^), times (dw/dc, dw/dr)."""
     res, xt = _prepare(pos, grid, normalised_input)
     z = hashgrid.encode(xt, tables, res, grid.log2_T)
     layers = unpack_layers(weights, mlp.layer_shapes())
@@ -255,15 +269,23 @@ def decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=None, normal
     dy = heads_backward(y, g64, _gate_for(xt, mlp, gate_cr))
     dz, wgrads = mlp_backward(dy, layers, acts, pres)
     gt = hashgrid.scatter_table_grad(dz, xt, res, grid.log2_T, grid.L, grid.F)
-    if not want_pos:
-        return gt, pack_layers(wgrads)
-    gx = hashgrid.encode_position_grad(dz, xt, tables, res, grid.log2_T)[:, :3]
-    p32 = np.asarray(pos, np.float32)
-    if normalised_input:
-        gpos = gx * hashgrid.clamp_passes(p32[:, :3])
-    else:
-        gpos = np.einsum("ni,nij->nj", gx, hashgrid.contraction_jacobian(p32))
-    return gt, pack_layers(wgrads), gpos
+    result = [gt, pack_layers(wgrads)]
+    if want_pos:
+        gx = hashgrid.encode_position_grad(dz, xt, tables, res, grid.log2_T)[:, :3]
+        p32 = np.asarray(pos, np.float32)
+        if normalised_input:
+            gpos = gx * hashgrid.clamp_passes(p32[:, :3])
+        else:
+            gpos = np.einsum("ni,nij->nj", gx, hashgrid.contraction_jacobian(p32))
+        result.append(gpos)
+    if want_gate:
+        assert mlp.gate, "the gate gradient needs a gated decoder"
+        t = xt[:, 3].astype(np.float64)
+        cr = np.asarray(gate_cr, np.float64)
+        dc, dr = temporal_gate_grad(t, cr[:, 0], cr[:, 1], float(np.float32(mlp.tau)))
+        gw = g64["opacity"][:, 0] * sigmoid(y[:, 10])
+        result.append(np.stack([gw * dc, gw * dr], axis=1))
+    return tuple(result)
 
 
 def adam_step(p, g, m, v, step: int, lr: float, b1: float, b2: float, eps: float):

@@ -163,3 +163,45 @@ def test_decode_backward_position_gradient_composes_the_contraction():
     _, _, g_norm = dec.decode_backward(xt, tables, weights, TINY, S.MLP_TINY, grads, normalised_input=True,
                                        want_pos=True)
     np.testing.assert_allclose(g_raw, 0.25 * g_norm, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Gate parameters (the KineticGS window centre c and half-width r)
+# ---------------------------------------------------------------------------
+def test_gate_gradient_closed_forms():
+    """At the centre (t = c) the window is symmetric: dw/dc = 0 and
+    dw/dr = 2 a^2 (1 - a)/tau with a = sigma(r/tau); far outside, both vanish."""
+    tau = 0.02
+    r = np.array([0.05, 0.1, 0.3])
+    t = np.array([0.4, 0.5, 0.9])
+    dc, dr = dec.temporal_gate_grad(t, t, r, tau)
+    a = 1 / (1 + np.exp(-r / tau))
+    np.testing.assert_allclose(dc, 0.0, atol=1e-15)
+    np.testing.assert_allclose(dr, 2 * a * a * (1 - a) / tau, rtol=1e-12, atol=1e-12)
+    dc, dr = dec.temporal_gate_grad(np.array([0.0]), np.array([0.9]), np.array([0.05]), tau)
+    assert abs(dc[0]) < 1e-12 and abs(dr[0]) < 1e-12
+
+
+def test_gate_gradient_matches_central_differences():
+    w = S.WORKLOADS["stress_fp16_gate"]
+    grid, mlp = w["grid"], w["mlp"]
+    n = 64
+    xt = np.random.default_rng(20).uniform(0.05, 0.95, size=(n, 4)).astype(np.float32)
+    tables = S.hash_tables(grid, seed=21, scale=1.0)
+    weights = S.mlp_weights(mlp, seed=22, bias_scale=0.5)
+    cr = S.gate_params(n, seed=23).astype(np.float64)
+    cr[:, 0] = xt[:, 3] + np.random.default_rng(24).uniform(-0.2, 0.2, n)   # windows near each t
+    grads = S.upstream_grads(n, S.DECODE_OUT_WIDTHS, 1.0, seed=25)
+    _, _, gcr = dec.decode_backward(xt, tables, weights, grid, mlp, grads, gate_cr=cr, normalised_input=True,
+                                    want_gate=True)
+
+    def loss(c):
+        out = dec.decode_forward(xt, tables, weights, grid, mlp, gate_cr=c, normalised_input=True)
+        return sum(np.sum(np.asarray(grads[k], np.float64) * out[k], axis=1) for k in grads)
+
+    h = 1e-6
+    for j in range(2):
+        e = np.zeros(2)
+        e[j] = h
+        fd = (loss(cr + e) - loss(cr - e)) / (2 * h)
+        np.testing.assert_allclose(gcr[:, j], fd, rtol=1e-6, atol=1e-7)

@@ -189,25 +189,38 @@ int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                       void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 
 /*
- * spin4d_decode_bwd that also accumulates the gradient w.r.t. the Gaussian
- * means (SPIN-4DGS section 3.3 trains the positions jointly with the
- * decoder):
- *   grad_pos += dloss/d(x, y, z)   (N x 3 fp32, 4-byte aligned, not NULL)
- * through the quadrilinear interpolation weights of every level (the
- * derivative inside the cell the position falls in, times res - 1 per axis)
- * and the Jacobian of Eq. 7 (I/4 inside the unit ball; outside, the
- * contracted point 2 - 1/|mu| along the ray of mu).  With
- * SPIN4D_INPUT_NORMALISED it is the gradient w.r.t. the normalised
- * coordinates, zero where the clamp to [0, 1] bound.  The timestamp is data,
- * not a parameter: it gets no gradient.  The corner entries are gathered
- * again for this even when `latent` is given.  Each position's three values
- * are written by one thread (no atomics).  Other arguments, results and
- * errors are those of spin4d_decode_bwd.
+ * Optional extra gradients of spin4d_decode_bwd_ext (a NULL member is not
+ * computed).  Both are accumulated (+=) and each position's values are
+ * written by one thread (no atomics), so repeated calls add identically.
+ *
+ * pos (N x 3 fp32, 4-byte aligned): dloss/d(x, y, z) of the Gaussian means
+ *   (SPIN-4DGS section 3.3 trains the positions jointly with the decoder),
+ *   through the quadrilinear interpolation weights of every level (the
+ *   derivative inside the cell the position falls in, times res - 1 per
+ *   axis) and the Jacobian of Eq. 7 (I/4 inside the unit ball; outside, the
+ *   contracted point 2 - 1/|mu| along the ray of mu).  With
+ *   SPIN4D_INPUT_NORMALISED it is the gradient w.r.t. the normalised
+ *   coordinates, zero where the clamp to [0, 1] bound.  The timestamp is
+ *   data, not a parameter: it gets no gradient.  The corner entries are
+ *   gathered again for this even when `latent` is given.
+ * gate_cr (N x 2 fp32, 4-byte aligned; gated decoders only): dloss/d(c, r)
+ *   of the KineticGS window (a learned gate: c and r come from the caller's
+ *   own predictor).  o = sigma(o^) w, w = a b, a = sigma((t - (c - r))/tau),
+ *   b = sigma(((c + r) - t)/tau): dloss/dw = g_o sigma(o^), dw/dc =
+ *   a b (a - b)/tau, dw/dr = a b (2 - a - b)/tau.
  */
-int spin4d_decode_bwd_pos(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
+typedef struct spin4d_extra_grads {
+    float* pos;
+    float* gate_cr;
+} spin4d_extra_grads;
+
+/* spin4d_decode_bwd plus the gradients `extra` asks for (extra not NULL;
+ * SPIN4D_ERR_INVALID for extra->gate_cr on an ungated decoder).  Other
+ * arguments, results and errors are those of spin4d_decode_bwd. */
+int spin4d_decode_bwd_ext(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                           const float* pos, int64_t N, const void* tables, const void* weights,
                           const float* gate_cr, const float* latent, const spin4d_output_grads* grad_out,
-                          float* grad_tables, float* grad_weights, float* grad_pos,
+                          float* grad_tables, float* grad_weights, const spin4d_extra_grads* extra,
                           void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 
 /*

@@ -447,6 +447,16 @@ __device__ __forceinline__ float temporal_gate(float t, float c, float r, float 
   return sigmoidf_((t - (c - r)) / tau) * sigmoidf_(((c + r) - t) / tau);
 }
 
+// Gradient w.r.t. the window centre c and half-width r of the gate, given
+// dloss/dw: w = a b with a = sigma((t - (c - r))/tau), b = sigma(((c + r) - t)/tau),
+// dw/dc = a b (a - b)/tau and dw/dr = a b (2 - a - b)/tau.
+__device__ __forceinline__ void temporal_gate_backward(float t, float c, float r, float tau, float dw, float out[2]) {
+  const float a = sigmoidf_((t - (c - r)) / tau), b = sigmoidf_(((c + r) - t) / tau);
+  const float k = dw * a * b / tau;
+  out[0] = k * (a - b);
+  out[1] = k * (2.0f - a - b);
+}
+
 // Decoded attributes of one Gaussian from its 11 head outputs.
 struct Attr {
   float s[3], r[4], rgb[3], o, cov[6];

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
                                                              const float* __restrict__ latent, GradPtrs go,
                                                              float* __restrict__ grad_tables,
                                                              float* __restrict__ grad_pos,
+                                                             float* __restrict__ grad_gate,
                                                              float* __restrict__ ws, int n_params) {
   extern __shared__ float smem[];
   const int H = m.hidden, IN = m.in_dim, NH = m.n_hidden;
@@ -203,8 +204,9 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
         for (int k = 0; k < head_in; ++k) acc = fmaf(ldw(wh + o * head_in, k), cur[k * kBwdBlock + col], acc);
         y[o] = acc;
       }
+      float2 cr = make_float2(0.f, 0.f);
       if (m.gate) {
-        float2 cr = gate_cr[n];
+        cr = gate_cr[n];
         gate = temporal_gate(xt[3], cr.x, cr.y, m.tau);
       }
       AttrGrad ag;
@@ -219,6 +221,12 @@ __global__ void __launch_bounds__(kBwdBlock) decode_bwd_simt(GridParams g, MlpPa
       for (int i = 0; i < 6; ++i) ag.cov[i] = ld_or0(go.cov, 6 * n + i);
       float dy[kHeadRows];
       heads_backward(y, gate, ag, dy);
+      if (grad_gate && m.gate) {   // o = sigma(o^) w: dloss/dw = g_o sigma(o^)
+        float gcr[2];
+        temporal_gate_backward(xt[3], cr.x, cr.y, m.tau, ag.o * sigmoidf_(y[10]), gcr);
+        grad_gate[2 * n] += gcr[0];
+        grad_gate[2 * n + 1] += gcr[1];
+      }
 #pragma unroll
       for (int o = 0; o < kHeadRows; ++o) dy_s[o * kBwdBlock + col] = dy[o];
     } else {
@@ -313,15 +321,16 @@ static int launch_fwd(const GridParams& gp, const MlpParams& mp, size_t smem, co
 template <typename T, int F, typename W>
 static int launch_bwd(const GridParams& gp, const MlpParams& mp, size_t smem, const float* pos, int64_t N,
                       const void* tables, const void* weights, const float* gate_cr, const float* latent, GradPtrs go,
-                      float* grad_tables, float* grad_pos, float* grad_weights, float* ws, int n_params,
-                      cudaStream_t s) {
+                      float* grad_tables, float* grad_pos, float* grad_gate, float* grad_weights, float* ws,
+                      int n_params, cudaStream_t s) {
   auto k = decode_bwd_simt<T, F, W>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
   int blocks = bwd_blocks(N);
   k<<<blocks, kBwdBlock, smem, s>>>(gp, mp, reinterpret_cast<const float4*>(pos), N,
                                     static_cast<const T*>(tables), static_cast<const W*>(weights),
-                                    reinterpret_cast<const float2*>(gate_cr), latent, go, grad_tables, grad_pos, ws, n_params);
+                                    reinterpret_cast<const float2*>(gate_cr), latent, go, grad_tables, grad_pos, grad_gate, ws,
+                                    n_params);
   SPIN4D_CHECK(launch_status());
   int rb = (n_params + 255) / 256;
   reduce_slots<<<rb, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
@@ -387,8 +396,8 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
 int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* m);
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                   const void* tables, const void* weights, const float* gate_cr, const float* latent,
-                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* ws, int n_params,
-                  int blocks, cudaStream_t s);
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* grad_gate, float* ws,
+                  int n_params, int blocks, cudaStream_t s);
 
 // Thread blocks (= workspace slots) the backward launches for N positions.
 static int bwd_slots(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, int64_t N) {
@@ -427,17 +436,20 @@ extern "C" size_t spin4d_decode_bwd_workspace(const spin4d_grid_desc* g, const s
 
 namespace spin4d {
 
-// spin4d_decode_bwd with an optional position gradient (grad_pos may be NULL).
+// spin4d_decode_bwd with optional extra gradients (members of `extra` may be NULL).
 static int decode_bwd_impl(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                            const void* tables, const void* weights, const float* gate_cr, const float* latent,
                            const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
-                           float* grad_pos, void* workspace, size_t ws_bytes, cudaStream_t s, const char* name) {
+                           const spin4d_extra_grads& extra, void* workspace, size_t ws_bytes, cudaStream_t s,
+                           const char* name) {
   SPIN4D_CHECK(check_common(g, m, pos, N, tables, weights, gate_cr));
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_tables || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_tables, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256) ||
-      (latent && !aligned(latent, 16)) || (grad_pos && !aligned(grad_pos, 4)))
+      (latent && !aligned(latent, 16)) || (extra.pos && !aligned(extra.pos, 4)) ||
+      (extra.gate_cr && !aligned(extra.gate_cr, 4)))
     return SPIN4D_ERR_INVALID;
+  if (extra.gate_cr && !m->gate) return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_decode_bwd_workspace(g, m, N)) return SPIN4D_ERR_INVALID;
   if (grad_out->rot && !aligned(grad_out->rot, 4)) return SPIN4D_ERR_INVALID;
   const bool tc = decode_bwd_tc_ctas_per_sm(g, m) > 0;
@@ -447,15 +459,15 @@ static int decode_bwd_impl(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, 
   if (tc) {
     const int blocks = bwd_slots(g, m, N);
     float* ws = static_cast<float*>(workspace);
-    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_pos, ws,
-                               n_params, blocks, s));
+    SPIN4D_CHECK(decode_bwd_tc(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, extra.pos,
+                               extra.gate_cr, ws, n_params, blocks, s));
     reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
     return launch_status();
   }
   GradPtrs go{grad_out->scale, grad_out->rot, grad_out->rgb, grad_out->opacity, grad_out->cov};
   return dispatch<BwdFn>(g->table_dtype, g->F, m->w_dtype, make_grid_params(g), make_mlp(m), bwd_smem(m), pos,
-                         N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, grad_weights,
-                         static_cast<float*>(workspace), n_params, s);
+                         N, tables, weights, gate_cr, latent, go, grad_tables, extra.pos, extra.gate_cr,
+                         grad_weights, static_cast<float*>(workspace), n_params, s);
 }
 
 }  // namespace spin4d
@@ -465,17 +477,18 @@ extern "C" int spin4d_decode_bwd(const spin4d_grid_desc* g, const spin4d_mlp_des
                                  const spin4d_output_grads* grad_out, float* grad_tables, float* grad_weights,
                                  void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
   return decode_bwd_impl(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
-                         nullptr, workspace, ws_bytes, (cudaStream_t)stream, "spin4d_decode_bwd");
+                         spin4d_extra_grads{nullptr, nullptr}, workspace, ws_bytes, (cudaStream_t)stream,
+                         "spin4d_decode_bwd");
 }
 
-extern "C" int spin4d_decode_bwd_pos(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos,
+extern "C" int spin4d_decode_bwd_ext(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos,
                                      int64_t N, const void* tables, const void* weights, const float* gate_cr,
                                      const float* latent, const spin4d_output_grads* grad_out, float* grad_tables,
-                                     float* grad_weights, float* grad_pos, void* workspace, size_t ws_bytes,
-                                     spin4d_stream_t stream) {
-  if (N > 0 && !grad_pos) return SPIN4D_ERR_INVALID;
+                                     float* grad_weights, const spin4d_extra_grads* extra, void* workspace,
+                                     size_t ws_bytes, spin4d_stream_t stream) {
+  if (!extra) return SPIN4D_ERR_INVALID;
   return decode_bwd_impl(g, m, pos, N, tables, weights, gate_cr, latent, grad_out, grad_tables, grad_weights,
-                         grad_pos, workspace, ws_bytes, (cudaStream_t)stream, "spin4d_decode_bwd_pos");
+                         *extra, workspace, ws_bytes, (cudaStream_t)stream, "spin4d_decode_bwd_ext");
 }
 
 // ---------------------------------------------------------------------------

@@ -266,7 +266,8 @@ template <int F, int IN, int H>
 __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kernel(
     GridParams g, int gate, float tau, const float4* __restrict__ pos, int64_t N, const __half* __restrict__ tables,
     const __half* __restrict__ weights, const float2* __restrict__ gate_cr, const float* __restrict__ latent, GradIn go,
-    float* __restrict__ grad_tables, float* __restrict__ grad_pos, float* __restrict__ ws, int n_params) {
+    float* __restrict__ grad_tables, float* __restrict__ grad_pos, float* __restrict__ grad_gate,
+    float* __restrict__ ws, int n_params) {
   using Lay = BLayout<IN, H>;
   // TMEM columns: two per-tile regions of H, then the weight-gradient
   // accumulators dW1 (IN), dW2 (H), dWh^T (16)
@@ -455,8 +456,9 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 #pragma unroll
         for (int i = 0; i < kHeadRows; ++i) y[i] = fmaf(v[i], ih2, bias[2 * H + i]);
         float gw = 1.0f;
+        float2 cr = make_float2(0.f, 0.f);
         if (gate) {
-          const float2 cr = gate_cr[n];
+          cr = gate_cr[n];
           gw = temporal_gate(xt[3], cr.x, cr.y, tau);
         }
         AttrGrad ag;
@@ -470,6 +472,12 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 #pragma unroll
         for (int i = 0; i < 6; ++i) ag.cov[i] = g_or0(go.cov, 6 * n + i);
         heads_backward(y, gw, ag, dy);
+        if (grad_gate && gate) {   // o = sigma(o^) w: dloss/dw = g_o sigma(o^)
+          float gcr[2];
+          temporal_gate_backward(xt[3], cr.x, cr.y, tau, ag.o * sigmoidf_(y[10]), gcr);
+          grad_gate[2 * n] += gcr[0];
+          grad_gate[2 * n + 1] += gcr[1];
+        }
       }
     }
     float dm = 0.f;
@@ -591,7 +599,8 @@ __global__ void __launch_bounds__(kThreads, H <= 64 ? 2 : 1) decode_bwd_tc_kerne
 template <int F, int IN, int H>
 int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* pos, int64_t N, const void* tables,
                   const void* weights, const float* gate_cr, const float* latent, const spin4d_output_grads* go,
-                  float* grad_tables, float* grad_pos, float* ws, int n_params, int blocks, cudaStream_t s) {
+                  float* grad_tables, float* grad_pos, float* grad_gate, float* ws, int n_params, int blocks,
+                  cudaStream_t s) {
   using Lay = BLayout<IN, H>;
   auto k = decode_bwd_tc_kernel<F, IN, H>;
   const int smem = align_up(Lay::bytes, 128);
@@ -610,8 +619,8 @@ int launch_bwd_tc(const GridParams& gp, const spin4d_mlp_desc* m, const float* p
   GradIn gi{go->scale, go->rot, go->rgb, go->opacity, go->cov};
   k<<<blocks, kThreads, smem, s>>>(gp, m->gate, m->tau, reinterpret_cast<const float4*>(pos), N,
                                    static_cast<const __half*>(tables), static_cast<const __half*>(weights),
-                                   reinterpret_cast<const float2*>(gate_cr), latent, gi, grad_tables, grad_pos, ws,
-                                   n_params);
+                                   reinterpret_cast<const float2*>(gate_cr), latent, gi, grad_tables, grad_pos,
+                                   grad_gate, ws, n_params);
   return launch_status();
 }
 
@@ -640,15 +649,15 @@ int decode_bwd_tc_ctas_per_sm(const spin4d_grid_desc* g, const spin4d_mlp_desc* 
 
 int decode_bwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos, int64_t N,
                   const void* tables, const void* weights, const float* gate_cr, const float* latent,
-                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* ws, int n_params,
-                  int blocks, cudaStream_t s) {
+                  const spin4d_output_grads* go, float* grad_tables, float* grad_pos, float* grad_gate, float* ws,
+                  int n_params, int blocks, cudaStream_t s) {
   const GridParams gp = make_grid_params(g);
   if (g->F == 2 && m->in_dim == 32 && m->hidden == 64)
-    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, ws,
-                                    n_params, blocks, s);
+    return launch_bwd_tc<2, 32, 64>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos,
+                                    grad_gate, ws, n_params, blocks, s);
   if (g->F == 4 && m->in_dim == 64 && m->hidden == 128)
-    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos, ws,
-                                     n_params, blocks, s);
+    return launch_bwd_tc<4, 64, 128>(gp, m, pos, N, tables, weights, gate_cr, latent, go, grad_tables, grad_pos,
+                                     grad_gate, ws, n_params, blocks, s);
   return SPIN4D_ERR_UNSUPPORTED;
 }
 

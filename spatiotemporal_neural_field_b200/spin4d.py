@@ -51,6 +51,10 @@ class OutputGrads(ctypes.Structure):
     _fields_ = [("scale", c_vp), ("rot", c_vp), ("rgb", c_vp), ("opacity", c_vp), ("cov", c_vp)]
 
 
+class ExtraGrads(ctypes.Structure):
+    _fields_ = [("pos", c_vp), ("gate_cr", c_vp)]
+
+
 class HexDesc(ctypes.Structure):
     _fields_ = [("n_scales", c_i32), ("scales", c_i32 * 4), ("time_res", c_i32), ("channels", c_i32),
                 ("n_frames", c_i32), ("hidden", c_i32), ("n_hidden", c_i32)]
@@ -73,8 +77,8 @@ _SIGS = {
     "spin4d_decode_bwd_workspace": (c_sz, [P(GridDesc), P(MlpDesc), c_i64]),
     "spin4d_decode_bwd": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
                                   c_vp, c_vp, c_vp, c_sz, c_vp]),
-    "spin4d_decode_bwd_pos": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
-                                      c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_decode_bwd_ext": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
+                                      c_vp, c_vp, P(ExtraGrads), c_vp, c_sz, c_vp]),
     "spin4d_decode_bwd_noalloc": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
                                           P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
@@ -225,9 +229,12 @@ def decode_bwd_workspace(g: GridDesc, m: MlpDesc, N: int) -> int:
 def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
                grad_tables: torch.Tensor, grad_weights: torch.Tensor, gate_cr=None,
                workspace: Optional[torch.Tensor] = None, latent: Optional[torch.Tensor] = None,
-               grad_pos: Optional[torch.Tensor] = None, stream=None) -> None:
+               grad_pos: Optional[torch.Tensor] = None, grad_gate: Optional[torch.Tensor] = None,
+               stream=None) -> None:
     """latent: the z saved by decode_fwd for the same positions (optional);
-    grad_pos: N x 3 fp32 accumulating the position gradient (optional)."""
+    grad_pos: N x 3 fp32 accumulating the position gradient (optional);
+    grad_gate: N x 2 fp32 accumulating the gradient w.r.t. the gate's (c, r)
+    (optional, gated decoders)."""
     N = pos.shape[0]
     need = decode_bwd_workspace(g, m, N)
     if workspace is None:
@@ -235,11 +242,12 @@ def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, t
     go = OutputGrads(*(_ptr(grads.get(k)) for k in ("scale", "rot", "rgb", "opacity", "cov")))
     common = (ctypes.byref(g), ctypes.byref(m), _ptr(pos), N, _ptr(tables), _ptr(weights), _ptr(gate_cr),
               _ptr(latent), ctypes.byref(go), _ptr(grad_tables), _ptr(grad_weights))
-    if grad_pos is None:
+    if grad_pos is None and grad_gate is None:
         _check("spin4d_decode_bwd", lib.spin4d_decode_bwd(*common, _ptr(workspace), workspace.numel(),
                                                           _stream(stream)))
     else:
-        _check("spin4d_decode_bwd_pos", lib.spin4d_decode_bwd_pos(*common, _ptr(grad_pos), _ptr(workspace),
+        extra = ExtraGrads(_ptr(grad_pos), _ptr(grad_gate))
+        _check("spin4d_decode_bwd_ext", lib.spin4d_decode_bwd_ext(*common, ctypes.byref(extra), _ptr(workspace),
                                                                   workspace.numel(), _stream(stream)))
 
 

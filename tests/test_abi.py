@@ -105,10 +105,14 @@ def test_invalid_arguments_rejected_on_host(sp):
     # misaligned saved latent
     assert lib.spin4d_decode_fwd(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None,
                                  sp.Outputs(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4), None) == sp.ERR_INVALID
-    # position gradient: grad_pos must be given, 4-byte aligned
-    assert lib.spin4d_decode_bwd_pos(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, None,
+    # extra gradients: the struct must be given, members aligned, the gate gradient only for a gated decoder
+    assert lib.spin4d_decode_bwd_ext(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, None,
                                      FAKE, 1 << 30, None) == sp.ERR_INVALID
-    assert lib.spin4d_decode_bwd_pos(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, FAKE + 2,
+    ex = sp.ExtraGrads(FAKE + 2, None)
+    assert lib.spin4d_decode_bwd_ext(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, ref(ex),
+                                     FAKE, 1 << 30, None) == sp.ERR_INVALID
+    ex = sp.ExtraGrads(None, FAKE)
+    assert lib.spin4d_decode_bwd_ext(ref(g), ref(m), FAKE, 10, FAKE, FAKE, None, None, ref(go), FAKE, FAKE, ref(ex),
                                      FAKE, 1 << 30, None) == sp.ERR_INVALID
     # ordering
     assert lib.spin4d_morton_order_workspace(0) == 0

@@ -14,6 +14,8 @@ here against things other than its own formula:
   differences, on positions exactly representable in fp32 so that the
   perturbed corner decisions and weights are exact.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -183,8 +185,8 @@ def test_gate_gradient_closed_forms():
 
 
 def test_gate_gradient_matches_central_differences():
-    w = S.WORKLOADS["stress_fp16_gate"]
-    grid, mlp = w["grid"], w["mlp"]
+    grid = TINY
+    mlp = dataclasses.replace(S.MLP_TINY, gate=True, tau=0.02)     # the tiny decoder with the gate
     n = 64
     xt = np.random.default_rng(20).uniform(0.05, 0.95, size=(n, 4)).astype(np.float32)
     tables = S.hash_tables(grid, seed=21, scale=1.0)

@@ -1,5 +1,7 @@
-"""GPU parity of the position gradient (spin4d_decode_bwd_pos) against the
-oracle (B200 only)."""
+"""GPU parity of the extra gradients of spin4d_decode_bwd_ext (position and
+gate parameters) against the oracle (B200 only)."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -134,3 +136,54 @@ def test_position_gradient_normalised_input(sp):
     out_of_range = (xt[:, :3] < 0) | (xt[:, :3] > 1)
     assert out_of_range.any() and np.all(host(gp)[out_of_range] == 0)
 
+
+
+# ---------------------------------------------------------------------------
+# gradient w.r.t. the gate's window centre and half-width
+# ---------------------------------------------------------------------------
+def _gate_case(sp, grid, mlp, pos, n, tscale, gstd, latent=False):
+    tables = S.hash_tables(grid, scale=tscale)
+    weights = S.mlp_weights(mlp, bias_scale=0.5)
+    cr = S.gate_params(n, seed=31)
+    grads = S.upstream_grads(n, S.DECODE_OUT_WIDTHS, gstd, seed=32)
+    g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+    P, T, W, CR = dev(pos), dev(tables), dev(weights), dev(cr)
+    lat = None
+    if latent:
+        out = sp.alloc_outputs(n, "cuda", latent_dim=grid.L * grid.F)
+        sp.decode_fwd(g, m, P, T, W, CR, out=out)
+        lat = out["latent"]
+    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
+    gw = torch.zeros(mlp.n_params(), device="cuda")
+    gp = torch.zeros((n, 3), device="cuda")
+    gg = torch.zeros((n, 2), device="cuda")
+    sp.decode_bwd(g, m, P, T, W, {k: dev(v) for k, v in grads.items()}, gt, gw, gate_cr=CR, latent=lat, grad_pos=gp,
+                  grad_gate=gg)
+    sp.check_device_errors()
+    _, _, wp, wg = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr, want_pos=True,
+                                       want_gate=True)
+    return host(gp), host(gg), wp, wg
+
+
+def test_gate_gradient_stress_tensor_core_path(sp):
+    w = S.WORKLOADS["stress_fp16_gate"]
+    n = 6007
+    gp, gg, wp, wg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0)
+    tol.normwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate")
+    tol.normwise(gp, wp, tol.FP16_GRAD_RTOL, "grad_pos alongside grad_gate")
+
+
+def test_gate_gradient_stress_saved_latent(sp):
+    w = S.WORKLOADS["stress_fp16_gate"]
+    n = 3001
+    _, gg, _, wg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0, latent=True)
+    tol.normwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate (saved latent)")
+
+
+def test_gate_gradient_fp32_simt_path(sp):
+    mlp = dataclasses.replace(S.MLP_TINY, gate=True, tau=0.05)
+    n = 4099
+    pos = S.uniform_positions(n, seed=33)
+    gp, gg, wp, wg = _gate_case(sp, S.GRID_TINY, mlp, pos, n, 1.0, 1.0)
+    tol.normwise(gg, wg, tol.FP32_GRAD_RTOL, "grad_gate (fp32)")
+    tol.normwise(gp, wp, tol.FP32_GRAD_RTOL, "grad_pos (fp32, gated)")

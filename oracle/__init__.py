@@ -20,4 +20,4 @@ Every function here is pinned by ``tests/test_oracle_*.py`` against values
 and properties fixed by the pages or by mathematics (closed forms, brute
 force, finite differences), not against itself.
 """
-from . import hashgrid, decoder, hexplane, ordering  # noqa: F401
+from . import hashgrid, decoder, hexplane, ordering, heads  # noqa: F401

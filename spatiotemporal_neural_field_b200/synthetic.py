@@ -135,6 +135,36 @@ MLP_STRESS = MlpSpec(in_dim=64, hidden=128, n_hidden=2, dtype="f16", gate=True, 
 
 HEX = HexSpec()
 
+
+@dataclasses.dataclass(frozen=True)
+class HeadsSpec:
+    """The paper's decoder: four heads (scale, rotation, SH colour, opacity),
+    each a three-layer MLP in_dim -> hidden -> hidden -> rows."""
+    in_dim: int
+    hidden: int = 64
+    sh_dim: int = 48
+    dtype: str = "f16"
+
+    def head_rows(self) -> Tuple[int, int, int, int]:
+        return (3, 4, self.sh_dim, 1)
+
+    def layer_shapes(self, head: int) -> List[Tuple[int, int]]:
+        return [(self.hidden, self.in_dim), (self.hidden, self.hidden), (self.head_rows()[head], self.hidden)]
+
+    def n_params(self) -> int:
+        return sum(o * i + o for h in range(4) for o, i in self.layer_shapes(h))
+
+
+# The paper's configuration (SPIN-4DGS section 4): hidden 64, L = 16, F = 4,
+# hash tables of 2^21 entries; resolutions as the sports grid (the page gives
+# none).
+GRID_PAPER = GridSpec(L=16, F=4, log2_T=21, nmin_s=16, nmax_s=2048, nmin_t=8, nmax_t=150,
+                      dtype="f16", t_min=0.0, t_max=float(N_FRAMES - 1))
+HEADS_PAPER = HeadsSpec(in_dim=64)
+GRID_TINY4 = GridSpec(L=4, F=4, log2_T=12, nmin_s=4, nmax_s=32, nmin_t=4, nmax_t=32,
+                      dtype="f32", t_min=0.0, t_max=1.0)
+HEADS_TINY = HeadsSpec(in_dim=16, hidden=16, sh_dim=12, dtype="f32")
+
 WORKLOADS: Dict[str, dict] = {
     "tiny_fp32": dict(N=4096, grid=GRID_TINY, mlp=MLP_TINY, grad_std=1.0),
     "sports_frame_fp16": dict(N=300_000, grid=GRID_SPORTS, mlp=MLP_SPORTS, frame=75),
@@ -143,6 +173,8 @@ WORKLOADS: Dict[str, dict] = {
                               eps=1e-15),
     "hexplane_fp32": dict(N=500_000, hex=HEX, grad_std=1.0),
     "stress_fp16_gate": dict(N=4_000_000, grid=GRID_STRESS, mlp=MLP_STRESS, grad_std=1.0),
+    # the paper's decoder: one 1M-position training launch of sports frames 0-3
+    "paper_heads_fp16": dict(N=1_000_000, grid=GRID_PAPER, heads=HEADS_PAPER, grad_std=1e-2),
 }
 
 
@@ -301,6 +333,34 @@ def mlp_weights(mlp: MlpSpec, seed: int = 0, head_bias: bool = True,
                 b = b + g.uniform(-bias_scale, bias_scale, size=o)
         parts += [W.reshape(-1), b]
     return _store(np.concatenate(parts), mlp.dtype)
+
+
+# Final-layer biases of the paper's heads (section 3.3): scale -5, rotation
+# (1, 0, 0, 0), SH colour none, opacity logit(0.1).
+HEADS_BIAS = ([-5.0, -5.0, -5.0], [1.0, 0.0, 0.0, 0.0], None, [math.log(0.1 / 0.9)])
+
+
+def heads_weights(spec: HeadsSpec, seed: int = 0, bias_scale: float = 0.0) -> np.ndarray:
+    """Packed weights of the four heads in order (scale, rotation, SH,
+    opacity), each [W1 b1 W2 b2 W3 b3] with W[out][in] row-major:
+    Xavier-uniform weights, hidden biases zero, final biases as the page
+    initialises them; U(+-bias_scale) added to every bias when > 0."""
+    g = rng(seed + 909)
+    parts = []
+    for h in range(4):
+        shapes = spec.layer_shapes(h)
+        for li, (o, i) in enumerate(shapes):
+            W = _xavier(g, o, i)
+            b = np.zeros(o)
+            if li == 2 and HEADS_BIAS[h] is not None:
+                b = np.array(HEADS_BIAS[h], np.float64)
+            if bias_scale > 0:
+                b = b + g.uniform(-bias_scale, bias_scale, size=o)
+            parts += [W.reshape(-1), b]
+    return _store(np.concatenate(parts), spec.dtype)
+
+
+HEADS_OUT_WIDTHS = {"scale": 3, "rot": 4, "sh": 48, "opacity": 1, "cov": 6}
 
 
 def hexplane_planes(hx: HexSpec, seed: int = 0, lo: float = 0.1, hi: float = 0.5) -> np.ndarray:

@@ -370,6 +370,83 @@ int spin4d_debug_corners(const spin4d_grid_desc* g, const float* pos, int64_t N,
 int spin4d_check_device_errors(int clear);
 
 /*
+ * The paper's attribute-aware decoder (SPIN-4DGS section 3.3, Eqs. 9-11):
+ * four heads -- scale, rotation, spherical-harmonic colour, opacity -- each a
+ * three-layer MLP in_dim -> hidden -> hidden -> rows (3, 4, sh_dim, 1) with
+ * exact GELU (x Phi(x)) after the first two layers, on the shared latent z
+ * of the hash encoder; s = exp(min(s^, 20)) (gradient zero above 20),
+ * r = r^/max(|r^|, 1e-12), sh = sh^, o = sigma(o^); Sigma by Eq. 2.
+ * Weights (fp32 or fp16, 4-byte aligned) are packed head by head in that
+ * order, each [W1 b1 W2 b2 W3 b3] with W[out][in] row-major.
+ * in_dim = L*F; in_dim, hidden and sh_dim at most 64
+ * (SPIN4D_ERR_UNSUPPORTED above).  fp32 arithmetic.
+ */
+typedef struct spin4d_heads_desc {
+    int32_t in_dim;
+    int32_t hidden;         /* 64 in the paper */
+    int32_t sh_dim;         /* 48: degree-3 SH, three colour channels */
+    int32_t w_dtype;        /* SPIN4D_F32 or SPIN4D_F16 */
+} spin4d_heads_desc;
+
+/* scale N x 3, rot N x 4 (16-byte aligned), sh N x sh_dim, opacity N x 1,
+ * cov N x 6 (fp32); latent (optional) N x in_dim receives z. */
+typedef struct spin4d_heads_outputs {
+    float* scale;
+    float* rot;
+    float* sh;
+    float* opacity;
+    float* cov;
+    float* latent;
+} spin4d_heads_outputs;
+
+typedef struct spin4d_heads_output_grads {
+    const float* scale;
+    const float* rot;
+    const float* sh;
+    const float* opacity;
+    const float* cov;
+} spin4d_heads_output_grads;
+
+/* Values in the packed weight vector (-1 if invalid). */
+int64_t spin4d_heads_param_count(const spin4d_heads_desc* h);
+
+int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
+                     const void* tables, const void* weights, spin4d_heads_outputs out, spin4d_stream_t stream);
+
+size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N);
+
+/* Backward of spin4d_heads_fwd for loss = sum_k <grad_out.k, output_k>
+ * (NULL members are zero): grad_tables += (L x T x F fp32, atomics),
+ * grad_weights += (packed like weights, fp32, summed in a fixed order).
+ * latent (optional) is the z spin4d_heads_fwd saved; workspace as for
+ * spin4d_decode_bwd, >= spin4d_heads_bwd_workspace bytes. */
+int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
+                     const void* tables, const void* weights, const float* latent,
+                     const spin4d_heads_output_grads* grad_out, float* grad_tables, float* grad_weights,
+                     void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
+ * Adam with per-group learning rates (SPIN-4DGS section 4 uses separate
+ * rates for the encoder and each decoder head): spin4d_adam_step over
+ * params[0..n) where element i takes the learning rate of the first group
+ * whose `end` exceeds i (groups sorted by end, the last end = n, at most
+ * SPIN4D_MAX_ADAM_GROUPS; host array).  Other arguments as spin4d_adam_step.
+ */
+#define SPIN4D_MAX_ADAM_GROUPS 16
+typedef struct spin4d_adam_group {
+    int64_t end;
+    float lr;
+} spin4d_adam_group;
+int spin4d_adam_step_groups(float* params, void* params_work, float* grad, float* m, float* v, int64_t n,
+                            const spin4d_adam_group* groups, int n_groups, int step, float b1, float b2, float eps,
+                            int zero_grad, int32_t* nonfinite_flag, spin4d_stream_t stream);
+
+/* Learning rate at optimiser step `step` (from 1): linear warm-up from 0 to
+ * lr_max over `warmup` steps, then cosine decay to lr_min at step `total`
+ * (lr_min afterwards).  Host function. */
+double spin4d_lr_warmup_cosine(int64_t step, double lr_max, double lr_min, int64_t warmup, int64_t total);
+
+/*
  * Z-order (Morton) ordering of the Gaussians, for gather locality (the
  * KineticGS notes serialise particles onto a Z-order space-filling curve to
  * keep spatial neighbours adjacent).  Decoding the Gaussians in this order

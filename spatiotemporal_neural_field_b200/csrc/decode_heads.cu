@@ -1,0 +1,460 @@
+// The paper's attribute-aware decoder: four heads (scale, rotation, SH
+// colour, opacity), each a three-layer MLP in -> hidden -> hidden -> rows
+// with GELU after the first two layers, on the shared latent z of the 4D
+// hash encoder (SPIN-4DGS section 3.3, Eqs. 9-11; Sigma by Eq. 2).
+//
+// fp32 SIMT kernels, one thread per position, activations in shared memory
+// [feature][position] so that the weight reads are block-wide broadcasts.
+// At the paper's size (L = 16, F = 4, T = 2^21: 256 MiB of fp16 tables) the
+// corner gathers come from HBM and the four 64-wide MLPs run beside them.
+//
+// Forward: gather z, then per head two GELU layers and the output layer,
+// four output rows per pass (independent accumulators), then Eq. 11 and Eq. 2.
+// Backward: forward again keeping the raw outputs of all heads (scale and
+// rotation couple through Sigma), the activations' adjoint, then per head
+// the forward again with its pre-activations, the data gradient through the
+// three layers into dz and the weight gradient summed over the block's
+// positions into the block's workspace slot (a second kernel adds the slots
+// in a fixed order); dz is scattered into the tables with fp32 atomics.
+#include <type_traits>
+
+#include "host.h"
+
+namespace spin4d {
+namespace {
+
+constexpr int kHeadsBlock = 64;      // forward: positions per block
+constexpr int kHeadsBwdBlock = 32;   // backward: positions per block
+constexpr int kMaxDim = 64;          // in_dim, hidden and sh_dim limit of the shared-memory layout
+
+struct HeadsParams {
+  int in_dim, hidden, sh_dim;
+  int rows[4];        // 3, 4, sh_dim, 1
+  int off[4];         // parameter offset of each head
+};
+
+struct HeadsOut {
+  float *scale, *rot, *sh, *opacity, *cov, *latent;
+};
+struct HeadsGrads {
+  const float *scale, *rot, *sh, *opacity, *cov;
+};
+
+template <typename W>
+__device__ __forceinline__ float wv(const W* __restrict__ w, int i) {
+  return to_f32<W>(__ldg(w + i));
+}
+
+// Exact GELU, x Phi(x), and its derivative Phi(x) + x phi(x).
+__device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_grad(float x) {
+  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * expf(-0.5f * x * x);
+}
+
+// out[o] = b[o] + sum_k W[o][k] in[k] for o < n_out, this thread's column;
+// pre (when given) keeps the value, out receives gelu of it when `act`.
+template <typename W>
+__device__ __forceinline__ void layer(const W* __restrict__ Wp, int n_out, int n_in, const float* in, float* out,
+                                      float* pre, bool act, int blk, int col) {
+  const W* bp = Wp + n_out * n_in;
+  int o = 0;
+  for (; o + 4 <= n_out; o += 4) {
+    float a0 = wv(bp, o), a1 = wv(bp, o + 1), a2 = wv(bp, o + 2), a3 = wv(bp, o + 3);
+    const W* w0 = Wp + o * n_in;
+    for (int k = 0; k < n_in; ++k) {
+      const float x = in[k * blk + col];
+      a0 = fmaf(wv(w0, k), x, a0);
+      a1 = fmaf(wv(w0 + n_in, k), x, a1);
+      a2 = fmaf(wv(w0 + 2 * n_in, k), x, a2);
+      a3 = fmaf(wv(w0 + 3 * n_in, k), x, a3);
+    }
+    const float a[4] = {a0, a1, a2, a3};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (pre) pre[(o + i) * blk + col] = a[i];
+      out[(o + i) * blk + col] = act ? gelu(a[i]) : a[i];
+    }
+  }
+  for (; o < n_out; ++o) {
+    float a = wv(bp, o);
+    const W* wr = Wp + o * n_in;
+    for (int k = 0; k < n_in; ++k) a = fmaf(wv(wr, k), in[k * blk + col], a);
+    if (pre) pre[o * blk + col] = a;
+    out[o * blk + col] = act ? gelu(a) : a;
+  }
+}
+
+// raw[0..2] scale^, raw[3..6] rot^, raw[7] opacity^ -> Eq. 11 and Eq. 2.
+__device__ __forceinline__ void store_heads(const HeadsOut& out, int64_t n, const float raw[8]) {
+  float s[3], r[4], cov[6];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
+  normalise_quat(raw + 3, r);
+  covariance(s, r, cov);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) out.scale[3 * n + i] = s[i];
+  reinterpret_cast<float4*>(out.rot)[n] = make_float4(r[0], r[1], r[2], r[3]);
+  out.opacity[n] = sigmoidf_(raw[7]);
+#pragma unroll
+  for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
+}
+
+template <typename T, int F>
+__device__ __forceinline__ void gather_z(const float xt[4], const GridParams& g, const T* __restrict__ tables,
+                                         float* z, int blk, int col, float* latent, int64_t n, int in_dim) {
+  for (int l = 0; l < g.L; ++l) {
+    float acc[F];
+    if constexpr (std::is_same<T, __half>::value && (F == 2 || F == 4))
+      encode_level_f16_paired<F>(xt, g, l, tables, acc);
+    else
+      encode_level<T, F>(xt, g, l, tables, acc);
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+      z[(l * F + f) * blk + col] = acc[f];
+      if (latent) latent[n * in_dim + l * F + f] = acc[f];
+    }
+  }
+}
+
+template <typename T, int F, typename W>
+__global__ void __launch_bounds__(kHeadsBlock) heads_fwd_kernel(GridParams g, HeadsParams hp,
+                                                                const float4* __restrict__ pos, int64_t N,
+                                                                const T* __restrict__ tables,
+                                                                const W* __restrict__ weights, HeadsOut out) {
+  __shared__ float z[kMaxDim * kHeadsBlock], a[kMaxDim * kHeadsBlock], b[kMaxDim * kHeadsBlock];
+  const int col = threadIdx.x;
+  const int IN = hp.in_dim, H = hp.hidden;
+  for (int64_t n0 = (int64_t)blockIdx.x * kHeadsBlock; n0 < N; n0 += (int64_t)gridDim.x * kHeadsBlock) {
+    const int64_t n = n0 + col;
+    if (n >= N) continue;   // no block-level synchronisation below
+    float xt[4];
+    normalise_position(pos[n], g, xt);
+    gather_z<T, F>(xt, g, tables, z, kHeadsBlock, col, out.latent, n, IN);
+    float raw[8];
+    for (int h = 0; h < 4; ++h) {
+      const W* w = weights + hp.off[h];
+      layer<W>(w, H, IN, z, a, nullptr, true, kHeadsBlock, col);
+      w += H * IN + H;
+      layer<W>(w, H, H, a, b, nullptr, true, kHeadsBlock, col);
+      w += H * H + H;
+      const int rows = hp.rows[h];
+      layer<W>(w, rows, H, b, a, nullptr, false, kHeadsBlock, col);   // raw outputs over a
+      if (h == 2) {
+        for (int i = 0; i < rows; ++i) out.sh[(int64_t)hp.sh_dim * n + i] = a[i * kHeadsBlock + col];
+      } else {
+        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+        for (int i = 0; i < rows; ++i) raw[base + i] = a[i * kHeadsBlock + col];
+      }
+    }
+    store_heads(out, n, raw);
+  }
+}
+
+__device__ __forceinline__ float g0(const float* p, int64_t i) { return p ? __ldg(p + i) : 0.0f; }
+
+// slot[p] += sum over the block's positions of d[o][t] * x[k][t] (weights)
+// and d[o][t] (biases) of one layer; each thread owns fixed parameters.
+__device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out, int n_in, float* slot, int blk) {
+  const int nW = n_out * n_in;
+  for (int p = threadIdx.x; p < nW + n_out; p += blockDim.x) {
+    float s = 0.0f;
+    if (p < nW) {
+      const int o = p / n_in, k = p - o * n_in;
+      for (int t = 0; t < blk; ++t) s = fmaf(d[o * blk + t], x[k * blk + t], s);
+    } else {
+      for (int t = 0; t < blk; ++t) s += d[(p - nW) * blk + t];
+    }
+    slot[p] += s;
+  }
+}
+
+// dx[k] (+)= sum_o W[o][k] d[o] for this column; times gelu'(pre[k]) when pre is given.
+template <typename W>
+__device__ __forceinline__ void dgrad(const W* __restrict__ Wp, int n_out, int n_in, const float* d, float* dx,
+                                      const float* pre, bool accumulate, int blk, int col) {
+  for (int k = 0; k < n_in; ++k) {
+    float s = 0.0f;
+    for (int o = 0; o < n_out; ++o) s = fmaf(wv(Wp + o * n_in, k), d[o * blk + col], s);
+    if (pre) s *= gelu_grad(pre[k * blk + col]);
+    dx[k * blk + col] = accumulate ? dx[k * blk + col] + s : s;
+  }
+}
+
+template <typename T, int F, typename W>
+__global__ void __launch_bounds__(kHeadsBwdBlock) heads_bwd_kernel(GridParams g, HeadsParams hp,
+                                                                   const float4* __restrict__ pos, int64_t N,
+                                                                   const T* __restrict__ tables,
+                                                                   const W* __restrict__ weights,
+                                                                   const float* __restrict__ latent, HeadsGrads go,
+                                                                   float* __restrict__ grad_tables,
+                                                                   float* __restrict__ ws, int n_params) {
+  constexpr int B = kHeadsBwdBlock;
+  extern __shared__ float sm[];
+  float* z = sm;                       // [IN][B]
+  float* p1 = z + kMaxDim * B;         // pre-activations of layer 1, later d(pre 1)
+  float* h1 = p1 + kMaxDim * B;
+  float* p2 = h1 + kMaxDim * B;        // pre-activations of layer 2, later d(pre 2)
+  float* h2 = p2 + kMaxDim * B;
+  float* dy = h2 + kMaxDim * B;        // one head's output adjoint
+  float* dz = dy + kMaxDim * B;
+  const int col = threadIdx.x;
+  const int IN = hp.in_dim, H = hp.hidden;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
+  for (int p = threadIdx.x; p < n_params; p += blockDim.x) slot[p] = 0.0f;
+
+  for (int64_t n0 = (int64_t)blockIdx.x * B; n0 < N; n0 += (int64_t)gridDim.x * B) {
+    const int64_t n = n0 + col;
+    const bool valid = n < N;
+    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    float dy_attr[8];   // adjoint of raw scale (3), rot (4), opacity (1)
+    if (valid) {
+      normalise_position(pos[n], g, xt);
+      if (latent) {
+        for (int k = 0; k < IN; ++k) z[k * B + col] = __ldg(latent + n * IN + k);
+      } else {
+        gather_z<T, F>(xt, g, tables, z, B, col, nullptr, n, IN);
+      }
+      // raw outputs of the scale, rotation and opacity heads
+      float raw[8];
+      for (int h = 0; h < 4; ++h) {
+        if (h == 2) continue;
+        const W* w = weights + hp.off[h];
+        layer<W>(w, H, IN, z, h1, nullptr, true, B, col);
+        w += H * IN + H;
+        layer<W>(w, H, H, h1, h2, nullptr, true, B, col);
+        w += H * H + H;
+        layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, B, col);
+        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+        for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[i * B + col];
+      }
+      // adjoint of Eq. 11 and Eq. 2
+      float s[3], r[4], cov_g[6], gs[3], gr[4];
+#pragma unroll
+      for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
+      const float nrm = normalise_quat(raw + 3, r);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) cov_g[i] = g0(go.cov, 6 * n + i);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) gs[i] = g0(go.scale, 3 * n + i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) gr[i] = g0(go.rot, 4 * n + i);
+      covariance_backward(s, r, cov_g, gs, gr);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) dy_attr[i] = raw[i] <= 20.0f ? gs[i] * s[i] : 0.0f;
+      normalise_quat_backward(r, nrm, gr, dy_attr + 3);
+      const float o = sigmoidf_(raw[7]);
+      dy_attr[7] = g0(go.opacity, n) * o * (1.0f - o);
+    } else {
+      for (int k = 0; k < IN; ++k) z[k * B + col] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dy_attr[i] = 0.0f;
+    }
+    for (int k = 0; k < IN; ++k) dz[k * B + col] = 0.0f;
+    // ---- per head: forward with pre-activations, then the three layers' gradients ----
+    for (int h = 0; h < 4; ++h) {
+      const int rows = hp.rows[h];
+      const W* w1 = weights + hp.off[h];
+      const W* w2 = w1 + H * IN + H;
+      const W* w3 = w2 + H * H + H;
+      float* s1 = slot + hp.off[h];
+      float* s2 = s1 + H * IN + H;
+      float* s3 = s2 + H * H + H;
+      if (valid) {
+        layer<W>(w1, H, IN, z, h1, p1, true, B, col);
+        layer<W>(w2, H, H, h1, h2, p2, true, B, col);
+        if (h == 2) {
+          for (int i = 0; i < rows; ++i) dy[i * B + col] = g0(go.sh, (int64_t)hp.sh_dim * n + i);
+        } else {
+          const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+          for (int i = 0; i < rows; ++i) dy[i * B + col] = dy_attr[base + i];
+        }
+      } else {
+        for (int k = 0; k < H; ++k) h1[k * B + col] = h2[k * B + col] = p1[k * B + col] = p2[k * B + col] = 0.0f;
+        for (int i = 0; i < rows; ++i) dy[i * B + col] = 0.0f;
+      }
+      __syncthreads();
+      wgrad(dy, h2, rows, H, s3, B);
+      dgrad<W>(w3, rows, H, dy, p2, p2, false, B, col);      // p2 <- d(pre 2)
+      __syncthreads();
+      wgrad(p2, h1, H, H, s2, B);
+      dgrad<W>(w2, H, H, p2, p1, p1, false, B, col);         // p1 <- d(pre 1)
+      __syncthreads();
+      wgrad(p1, z, H, IN, s1, B);
+      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, B, col);    // dz += W1^T d(pre 1)
+      __syncthreads();
+    }
+    if (valid) {
+      for (int l = 0; l < g.L; ++l) {
+        float d[F];
+#pragma unroll
+        for (int f = 0; f < F; ++f) d[f] = dz[(l * F + f) * B + col];
+        scatter_level<F>(xt, g, l, grad_tables, d);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
+    float s = 0.0f;
+    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * slot_stride(n_params) + p];
+    out[p] += s;
+  }
+}
+
+constexpr size_t kBwdSmem = (size_t)7 * kMaxDim * kHeadsBwdBlock * sizeof(float);
+
+int validate_heads(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
+  if (!h) return SPIN4D_ERR_INVALID;
+  if (h->in_dim != g->L * g->F) return SPIN4D_ERR_INVALID;
+  if (h->hidden < 1 || h->sh_dim < 1 || h->w_dtype < 0 || h->w_dtype > 1) return SPIN4D_ERR_INVALID;
+  if (h->in_dim > kMaxDim || h->hidden > kMaxDim || h->sh_dim > kMaxDim) return SPIN4D_ERR_UNSUPPORTED;
+  return SPIN4D_OK;
+}
+
+HeadsParams make_heads(const spin4d_heads_desc* h) {
+  HeadsParams p;
+  p.in_dim = h->in_dim;
+  p.hidden = h->hidden;
+  p.sh_dim = h->sh_dim;
+  const int rows[4] = {3, 4, h->sh_dim, 1};
+  int o = 0;
+  for (int k = 0; k < 4; ++k) {
+    p.rows[k] = rows[k];
+    p.off[k] = o;
+    o += h->hidden * h->in_dim + h->hidden + h->hidden * h->hidden + h->hidden + rows[k] * h->hidden + rows[k];
+  }
+  return p;
+}
+
+int64_t param_count(const spin4d_heads_desc* h) {
+  int64_t n = 0;
+  const int rows[4] = {3, 4, h->sh_dim, 1};
+  for (int k = 0; k < 4; ++k)
+    n += (int64_t)h->hidden * h->in_dim + h->hidden + (int64_t)h->hidden * h->hidden + h->hidden +
+         (int64_t)rows[k] * h->hidden + rows[k];
+  return n;
+}
+
+int bwd_blocks(int64_t N) { return persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 6); }
+
+template <typename T, int F, typename W>
+struct HeadsLaunch {
+  static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
+                 const void* weights, const HeadsOut& o, cudaStream_t s) {
+    const int blocks = persistent_blocks((N + kHeadsBlock - 1) / kHeadsBlock, 6);
+    heads_fwd_kernel<T, F, W><<<blocks, kHeadsBlock, 0, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                                             static_cast<const T*>(tables),
+                                                             static_cast<const W*>(weights), o);
+    return launch_status();
+  }
+  static int bwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
+                 const void* weights, const float* latent, const HeadsGrads& go, float* grad_tables,
+                 float* grad_weights, float* ws, int n_params, cudaStream_t s) {
+    auto k = heads_bwd_kernel<T, F, W>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int blocks = bwd_blocks(N);
+    k<<<blocks, kHeadsBwdBlock, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                              static_cast<const T*>(tables), static_cast<const W*>(weights), latent,
+                                              go, grad_tables, ws, n_params);
+    SPIN4D_CHECK(launch_status());
+    heads_reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
+    return launch_status();
+  }
+};
+
+template <typename T, int F>
+int dispatch_w(int wdt, bool bwd, const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N,
+               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+               float* gt, float* gw, float* ws, int n_params, cudaStream_t s) {
+  if (wdt == SPIN4D_F16) {
+    if (bwd) return HeadsLaunch<T, F, __half>::bwd(gp, hp, pos, N, tables, weights, latent, *go, gt, gw, ws, n_params, s);
+    return HeadsLaunch<T, F, __half>::fwd(gp, hp, pos, N, tables, weights, *o, s);
+  }
+  if (bwd) return HeadsLaunch<T, F, float>::bwd(gp, hp, pos, N, tables, weights, latent, *go, gt, gw, ws, n_params, s);
+  return HeadsLaunch<T, F, float>::fwd(gp, hp, pos, N, tables, weights, *o, s);
+}
+
+template <typename T>
+int dispatch_f(int F, int wdt, bool bwd, const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N,
+               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+               float* gt, float* gw, float* ws, int n_params, cudaStream_t s) {
+  switch (F) {
+    case 1: return dispatch_w<T, 1>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
+    case 2: return dispatch_w<T, 2>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
+    case 4: return dispatch_w<T, 4>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
+    case 8: return dispatch_w<T, 8>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
+    default: return SPIN4D_ERR_UNSUPPORTED;
+  }
+}
+
+int run(const spin4d_grid_desc* g, const spin4d_heads_desc* h, bool bwd, const float* pos, int64_t N,
+        const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+        float* gt, float* gw, float* ws, cudaStream_t s) {
+  const GridParams gp = make_grid_params(g);
+  const HeadsParams hp = make_heads(h);
+  const int n_params = (int)param_count(h);
+  if (g->table_dtype == SPIN4D_F16)
+    return dispatch_f<__half>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws,
+                              n_params, s);
+  return dispatch_f<float>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws,
+                           n_params, s);
+}
+
+int check_inputs(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
+                 const void* tables, const void* weights) {
+  SPIN4D_CHECK(validate_grid(g));
+  SPIN4D_CHECK(validate_heads(g, h));
+  if (N < 0) return SPIN4D_ERR_INVALID;
+  if (N == 0) return SPIN4D_OK;
+  const size_t esz = g->table_dtype == SPIN4D_F16 ? 2 : 4;
+  const size_t talign = esz * g->F > 16 ? 16 : esz * g->F;
+  if (!pos || !tables || !weights || !aligned(pos, 16) || !aligned(tables, talign) || !aligned(weights, 4))
+    return SPIN4D_ERR_INVALID;
+  return SPIN4D_OK;
+}
+
+}  // namespace
+}  // namespace spin4d
+
+using namespace spin4d;
+
+extern "C" int64_t spin4d_heads_param_count(const spin4d_heads_desc* h) {
+  if (!h || h->in_dim < 1 || h->hidden < 1 || h->sh_dim < 1) return -1;
+  return param_count(h);
+}
+
+extern "C" int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
+                                const void* tables, const void* weights, spin4d_heads_outputs out,
+                                spin4d_stream_t stream) {
+  SPIN4D_CHECK(check_inputs(g, h, pos, N, tables, weights));
+  if (N == 0) return SPIN4D_OK;
+  if (!out.scale || !out.rot || !out.sh || !out.opacity || !out.cov || !aligned(out.rot, 16)) return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_heads_fwd")) return SPIN4D_ERR_INJECTED;
+  const HeadsOut o{out.scale, out.rot, out.sh, out.opacity, out.cov, out.latent};
+  return run(g, h, false, pos, N, tables, weights, &o, nullptr, nullptr, nullptr, nullptr, nullptr,
+             (cudaStream_t)stream);
+}
+
+extern "C" size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N) {
+  if (validate_grid(g) != SPIN4D_OK || validate_heads(g, h) != SPIN4D_OK || N <= 0) return 0;
+  return (size_t)bwd_blocks(N) * slot_stride((int)param_count(h)) * sizeof(float);
+}
+
+extern "C" int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
+                                const void* tables, const void* weights, const float* latent,
+                                const spin4d_heads_output_grads* grad_out, float* grad_tables, float* grad_weights,
+                                void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
+  SPIN4D_CHECK(check_inputs(g, h, pos, N, tables, weights));
+  if (N == 0) return SPIN4D_OK;
+  if (!grad_out || !grad_tables || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
+  if (!aligned(grad_tables, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256) ||
+      ws_bytes < spin4d_heads_bwd_workspace(g, h, N))
+    return SPIN4D_ERR_INVALID;
+  if (fault_injected("spin4d_heads_bwd")) return SPIN4D_ERR_INJECTED;
+  const HeadsGrads go{grad_out->scale, grad_out->rot, grad_out->sh, grad_out->opacity, grad_out->cov};
+  return run(g, h, true, pos, N, tables, weights, nullptr, latent, &go, grad_tables, grad_weights,
+             static_cast<float*>(workspace), (cudaStream_t)stream);
+}

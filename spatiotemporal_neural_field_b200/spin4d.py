@@ -68,6 +68,22 @@ class HexOutputGrads(ctypes.Structure):
     _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp)]
 
 
+class HeadsDesc(ctypes.Structure):
+    _fields_ = [("in_dim", c_i32), ("hidden", c_i32), ("sh_dim", c_i32), ("w_dtype", c_i32)]
+
+
+class HeadsOutputs(ctypes.Structure):
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("sh", c_vp), ("opacity", c_vp), ("cov", c_vp), ("latent", c_vp)]
+
+
+class HeadsOutputGrads(ctypes.Structure):
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("sh", c_vp), ("opacity", c_vp), ("cov", c_vp)]
+
+
+class AdamGroup(ctypes.Structure):
+    _fields_ = [("end", c_i64), ("lr", c_f32)]
+
+
 P = ctypes.POINTER
 _SIGS = {
     "spin4d_grid_init": (c_i32, [P(GridDesc), c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_f32, c_f32]),
@@ -82,6 +98,14 @@ _SIGS = {
     "spin4d_decode_bwd_noalloc": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
                                           P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "spin4d_heads_param_count": (c_i64, [P(HeadsDesc)]),
+    "spin4d_heads_fwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, HeadsOutputs, c_vp]),
+    "spin4d_heads_bwd_workspace": (c_sz, [P(GridDesc), P(HeadsDesc), c_i64]),
+    "spin4d_heads_bwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, c_vp, P(HeadsOutputGrads), c_vp,
+                                 c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_adam_step_groups": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, P(AdamGroup), c_i32, c_i32, c_f32,
+                                        c_f32, c_f32, c_i32, c_vp, c_vp]),
+    "spin4d_lr_warmup_cosine": (ctypes.c_double, [c_i64, ctypes.c_double, ctypes.c_double, c_i64, c_i64]),
     "spin4d_adam_step": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i32, c_f32, c_f32, c_f32, c_f32, c_i32,
                                  c_vp, c_vp]),
     "spin4d_hexplane_plane_count": (c_i64, [P(HexDesc)]),
@@ -281,6 +305,62 @@ def adam_step(params, grad, m, v, step: int, lr: float, b1: float, b2: float, ep
     _check("spin4d_adam_step", lib.spin4d_adam_step(_ptr(params), _ptr(params_work), _ptr(grad), _ptr(m), _ptr(v),
                                                     params.numel(), step, lr, b1, b2, eps, 1 if zero_grad else 0,
                                                     _ptr(nonfinite_flag), _stream(stream)))
+
+
+def adam_step_groups(params, grad, m, v, step: int, groups, b1: float, b2: float, eps: float,
+                     params_work: Optional[torch.Tensor] = None, zero_grad: bool = False,
+                     nonfinite_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """groups: [(end, lr), ...] with increasing ends, the last = params.numel()."""
+    arr = (AdamGroup * len(groups))(*[AdamGroup(int(e), float(lr)) for e, lr in groups])
+    _check("spin4d_adam_step_groups", lib.spin4d_adam_step_groups(
+        _ptr(params), _ptr(params_work), _ptr(grad), _ptr(m), _ptr(v), params.numel(), arr, len(groups), step, b1, b2,
+        eps, 1 if zero_grad else 0, _ptr(nonfinite_flag), _stream(stream)))
+
+
+def lr_warmup_cosine(step: int, lr_max: float, lr_min: float, warmup: int, total: int) -> float:
+    return float(lib.spin4d_lr_warmup_cosine(step, lr_max, lr_min, warmup, total))
+
+
+# ---- the paper's four-head decoder ----
+HEADS_KEYS = ("scale", "rot", "sh", "opacity", "cov")
+
+
+def heads_desc(in_dim: int, hidden: int = 64, sh_dim: int = 48, w_dtype: str = "f16") -> HeadsDesc:
+    return HeadsDesc(in_dim, hidden, sh_dim, F16 if w_dtype == "f16" else F32)
+
+
+def heads_from_spec(spec) -> HeadsDesc:
+    return heads_desc(spec.in_dim, spec.hidden, spec.sh_dim, spec.dtype)
+
+
+def heads_param_count(h: HeadsDesc) -> int:
+    return int(lib.spin4d_heads_param_count(ctypes.byref(h)))
+
+
+def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent: bool = False, stream=None):
+    N = pos.shape[0]
+    widths = {"scale": 3, "rot": 4, "sh": h.sh_dim, "opacity": 1, "cov": 6}
+    if out is None:
+        out = {k: torch.empty((N, w), dtype=torch.float32, device=pos.device) for k, w in widths.items()}
+        if latent:
+            out["latent"] = torch.empty((N, h.in_dim), dtype=torch.float32, device=pos.device)
+    o = HeadsOutputs(*(_ptr(out[k]) for k in HEADS_KEYS), _ptr(out.get("latent")))
+    _check("spin4d_heads_fwd", lib.spin4d_heads_fwd(ctypes.byref(g), ctypes.byref(h), _ptr(pos), N, _ptr(tables),
+                                                    _ptr(weights), o, _stream(stream)))
+    return out
+
+
+def heads_bwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, grads, grad_tables, grad_weights, latent=None,
+              workspace=None, stream=None) -> None:
+    N = pos.shape[0]
+    if workspace is None:
+        need = int(lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), N))
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
+    go = HeadsOutputGrads(*(_ptr(grads.get(k)) for k in HEADS_KEYS))
+    _check("spin4d_heads_bwd", lib.spin4d_heads_bwd(ctypes.byref(g), ctypes.byref(h), _ptr(pos), N, _ptr(tables),
+                                                    _ptr(weights), _ptr(latent), ctypes.byref(go), _ptr(grad_tables),
+                                                    _ptr(grad_weights), _ptr(workspace), workspace.numel(),
+                                                    _stream(stream)))
 
 
 def hexplane_plane_count(h: HexDesc) -> int:

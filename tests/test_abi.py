@@ -124,6 +124,23 @@ def test_invalid_arguments_rejected_on_host(sp):
     assert lib.spin4d_permute_rows(FAKE, 10, FAKE, FAKE, 10, 6, None) == sp.ERR_INVALID       # row bytes
     assert lib.spin4d_permute_rows(FAKE, 10, FAKE, FAKE, 10, 8, None) == sp.ERR_INVALID       # src == dst
     assert lib.spin4d_permute_rows(None, 0, None, None, 0, 8, None) == sp.OK
+    # the paper's decoder
+    hs = sp.heads_desc(64)
+    assert sp.heads_param_count(hs) == S.HEADS_PAPER.n_params()
+    gp4 = sp.grid_from_spec(S.GRID_PAPER)
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(63)), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_INVALID
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(64, hidden=128)), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE + 4, FAKE, FAKE, FAKE, None), None) == sp.ERR_INVALID
+    # grouped Adam: ends must increase to n
+    grp = (sp.AdamGroup * 2)(sp.AdamGroup(60, 1e-3), sp.AdamGroup(50, 1e-4))
+    assert lib.spin4d_adam_step_groups(FAKE, None, FAKE, FAKE, FAKE, 100, grp, 2, 1, 0.9, 0.99, 1e-15, 0, None,
+                                       None) == sp.ERR_INVALID
+    grp = (sp.AdamGroup * 2)(sp.AdamGroup(60, 1e-3), sp.AdamGroup(90, 1e-4))
+    assert lib.spin4d_adam_step_groups(FAKE, None, FAKE, FAKE, FAKE, 100, grp, 2, 1, 0.9, 0.99, 1e-15, 0, None,
+                                       None) == sp.ERR_INVALID
     # adam
     assert lib.spin4d_adam_step(FAKE, None, FAKE, FAKE, FAKE, 100, 0, 1e-3, 0.9, 0.99, 1e-15, 0, None,
                                 None) == sp.ERR_INVALID
@@ -163,3 +180,10 @@ print(r1, r2)
     r1, r2 = map(int, out.stdout.split())
     assert r1 == -5          # injected after validation, before any launch
     assert r2 == -1          # other entry points unaffected (still validated)
+
+
+def test_learning_rate_schedule_matches_oracle(sp):
+    from oracle import heads as hd
+    for args in ((8e-3, 1e-7, 100, 1100), (1e-3, 1e-7, 0, 40000), (3e-5, 1e-7, 500, 500)):
+        for step in (1, 2, 50, 99, 100, 101, 600, 1099, 1100, 1101, 40000, 50000):
+            assert abs(sp.lr_warmup_cosine(step, *args) - hd.lr_warmup_cosine(step, *args)) <= 1e-12 * args[0]

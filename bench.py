@@ -13,6 +13,7 @@ the tables and the weight gradients).
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -650,6 +651,35 @@ def run_workloads(args):
         emit(name, "fwd+bwd+position gradient (saved latent)", n, timed(fbp, reps))
         del P, T, W, out, fwd_out, grads, gt, gw, ws, gpos
         torch.cuda.empty_cache()
+
+    # the paper's four-head GELU decoder, one 1M-position training launch
+    w = S.WORKLOADS["paper_heads_fp16"]
+    grid, spec, n = w["grid"], w["heads"], w["N"]
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
+    P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
+    T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+    W = torch.from_numpy(S.heads_weights(spec)).to(dev)
+    out = sp.heads_fwd(g, h, P, T, W, latent=True)
+    fwd_out = {k: v for k, v in out.items() if k != "latent"}
+    ms = timed(lambda: sp.heads_fwd(g, h, P, T, W, out=fwd_out), 10)
+    spp = table_sectors_per_position(sp, g, P, grid.F, 2)
+    emit("paper_heads_fp16", "fwd", n, ms, table_sectors_per_position=spp, sector_rate=spp * n / (ms * 1e-3),
+         frac_of_hbm_random_sector_ceiling=spp * n / (ms * 1e-3) / ceil["hbm_random_sector_per_s"],
+         mlp_flop_per_position=2 * sum(o * i for hd_ in range(4) for o, i in spec.layer_shapes(hd_)))
+    grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
+             for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim).items()}
+    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
+    gw = torch.zeros(spec.n_params(), device=dev)
+    ws = torch.empty(max(sp.lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), n), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def hfb():
+        sp.heads_fwd(g, h, P, T, W, out=out)
+        sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], workspace=ws)
+
+    emit("paper_heads_fp16", "fwd (saving z) + bwd", n, timed(hfb, 5))
+    del P, T, W, out, fwd_out, grads, gt, gw, ws
+    torch.cuda.empty_cache()
 
     # HexPlane
     w = S.WORKLOADS["hexplane_fp32"]

@@ -3,8 +3,10 @@
 // with GELU after the first two layers, on the shared latent z of the 4D
 // hash encoder (SPIN-4DGS section 3.3, Eqs. 9-11; Sigma by Eq. 2).
 //
-// fp32 SIMT kernels, one thread per position, activations in shared memory
-// [feature][position] so that the weight reads are block-wide broadcasts.
+// fp32 SIMT kernels, four threads per position (each a quarter of every
+// layer's output rows, and a quarter of the hash levels), activations in
+// shared memory [feature][position] so that the weight reads are warp-wide
+// broadcasts.
 // At the paper's size (L = 16, F = 4, T = 2^21: 256 MiB of fp16 tables) the
 // corner gathers come from HBM and the four 64-wide MLPs run beside them.
 //
@@ -51,36 +53,38 @@ __device__ __forceinline__ float gelu_grad(float x) {
   return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * expf(-0.5f * x * x);
 }
 
-// out[o] = b[o] + sum_k W[o][k] in[k] for o < n_out, this thread's column;
+// kParts threads serve each position; part p takes the output rows of the
+// 4-row groups p, p + kParts, ...  (all lanes of a warp share a part, so the
+// weight reads are warp-wide broadcasts).  Rows past n_out are computed on a
+// clamped row and not stored.
+constexpr int kParts = 4;
+
+// out[o] = b[o] + sum_k W[o][k] in[k] for this part's rows, this column;
 // pre (when given) keeps the value, out receives gelu of it when `act`.
 template <typename W>
 __device__ __forceinline__ void layer(const W* __restrict__ Wp, int n_out, int n_in, const float* in, float* out,
-                                      float* pre, bool act, int blk, int col) {
+                                      float* pre, bool act, int blk, int col, int part) {
   const W* bp = Wp + n_out * n_in;
-  int o = 0;
-  for (; o + 4 <= n_out; o += 4) {
-    float a0 = wv(bp, o), a1 = wv(bp, o + 1), a2 = wv(bp, o + 2), a3 = wv(bp, o + 3);
-    const W* w0 = Wp + o * n_in;
+  for (int o = 4 * part; o < n_out; o += 4 * kParts) {
+    int r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = min(o + i, n_out - 1);
+    float a0 = wv(bp, r[0]), a1 = wv(bp, r[1]), a2 = wv(bp, r[2]), a3 = wv(bp, r[3]);
+    const W *w0 = Wp + r[0] * n_in, *w1 = Wp + r[1] * n_in, *w2 = Wp + r[2] * n_in, *w3 = Wp + r[3] * n_in;
     for (int k = 0; k < n_in; ++k) {
       const float x = in[k * blk + col];
       a0 = fmaf(wv(w0, k), x, a0);
-      a1 = fmaf(wv(w0 + n_in, k), x, a1);
-      a2 = fmaf(wv(w0 + 2 * n_in, k), x, a2);
-      a3 = fmaf(wv(w0 + 3 * n_in, k), x, a3);
+      a1 = fmaf(wv(w1, k), x, a1);
+      a2 = fmaf(wv(w2, k), x, a2);
+      a3 = fmaf(wv(w3, k), x, a3);
     }
-    const float a[4] = {a0, a1, a2, a3};
+    const float v[4] = {a0, a1, a2, a3};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      if (pre) pre[(o + i) * blk + col] = a[i];
-      out[(o + i) * blk + col] = act ? gelu(a[i]) : a[i];
+      if (o + i >= n_out) break;
+      if (pre) pre[(o + i) * blk + col] = v[i];
+      out[(o + i) * blk + col] = act ? gelu(v[i]) : v[i];
     }
-  }
-  for (; o < n_out; ++o) {
-    float a = wv(bp, o);
-    const W* wr = Wp + o * n_in;
-    for (int k = 0; k < n_in; ++k) a = fmaf(wv(wr, k), in[k * blk + col], a);
-    if (pre) pre[o * blk + col] = a;
-    out[o * blk + col] = act ? gelu(a) : a;
   }
 }
 
@@ -99,10 +103,12 @@ __device__ __forceinline__ void store_heads(const HeadsOut& out, int64_t n, cons
   for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
 }
 
+// This part's levels of z (levels part, part + kParts, ...).
 template <typename T, int F>
 __device__ __forceinline__ void gather_z(const float xt[4], const GridParams& g, const T* __restrict__ tables,
-                                         float* z, int blk, int col, float* latent, int64_t n, int in_dim) {
-  for (int l = 0; l < g.L; ++l) {
+                                         float* z, int blk, int col, int part, float* latent, int64_t n,
+                                         int in_dim) {
+  for (int l = part; l < g.L; l += kParts) {
     float acc[F];
     if constexpr (std::is_same<T, __half>::value && (F == 2 || F == 4))
       encode_level_f16_paired<F>(xt, g, l, tables, acc);
@@ -117,43 +123,56 @@ __device__ __forceinline__ void gather_z(const float xt[4], const GridParams& g,
 }
 
 template <typename T, int F, typename W>
-__global__ void __launch_bounds__(kHeadsBlock) heads_fwd_kernel(GridParams g, HeadsParams hp,
-                                                                const float4* __restrict__ pos, int64_t N,
-                                                                const T* __restrict__ tables,
-                                                                const W* __restrict__ weights, HeadsOut out) {
-  __shared__ float z[kMaxDim * kHeadsBlock], a[kMaxDim * kHeadsBlock], b[kMaxDim * kHeadsBlock];
-  const int col = threadIdx.x;
+__global__ void __launch_bounds__(kHeadsBlock * kParts) heads_fwd_kernel(GridParams g, HeadsParams hp,
+                                                                         const float4* __restrict__ pos, int64_t N,
+                                                                         const T* __restrict__ tables,
+                                                                         const W* __restrict__ weights, HeadsOut out) {
+  constexpr int B = kHeadsBlock;
+  __shared__ float z[kMaxDim * B], a[kMaxDim * B], b[kMaxDim * B];
+  const int col = threadIdx.x % B, part = threadIdx.x / B;
   const int IN = hp.in_dim, H = hp.hidden;
-  for (int64_t n0 = (int64_t)blockIdx.x * kHeadsBlock; n0 < N; n0 += (int64_t)gridDim.x * kHeadsBlock) {
+  for (int64_t n0 = (int64_t)blockIdx.x * B; n0 < N; n0 += (int64_t)gridDim.x * B) {
     const int64_t n = n0 + col;
-    if (n >= N) continue;   // no block-level synchronisation below
-    float xt[4];
-    normalise_position(pos[n], g, xt);
-    gather_z<T, F>(xt, g, tables, z, kHeadsBlock, col, out.latent, n, IN);
+    const bool valid = n < N;
+    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) {
+      normalise_position(pos[n], g, xt);
+      gather_z<T, F>(xt, g, tables, z, B, col, part, out.latent, n, IN);
+    } else {
+      for (int k = part; k < IN; k += kParts) z[k * B + col] = 0.0f;
+    }
+    __syncthreads();
     float raw[8];
     for (int h = 0; h < 4; ++h) {
       const W* w = weights + hp.off[h];
-      layer<W>(w, H, IN, z, a, nullptr, true, kHeadsBlock, col);
+      layer<W>(w, H, IN, z, a, nullptr, true, B, col, part);
+      __syncthreads();
       w += H * IN + H;
-      layer<W>(w, H, H, a, b, nullptr, true, kHeadsBlock, col);
+      layer<W>(w, H, H, a, b, nullptr, true, B, col, part);
+      __syncthreads();
       w += H * H + H;
       const int rows = hp.rows[h];
-      layer<W>(w, rows, H, b, a, nullptr, false, kHeadsBlock, col);   // raw outputs over a
+      layer<W>(w, rows, H, b, a, nullptr, false, B, col, part);   // raw outputs over a
+      __syncthreads();
       if (h == 2) {
-        for (int i = 0; i < rows; ++i) out.sh[(int64_t)hp.sh_dim * n + i] = a[i * kHeadsBlock + col];
-      } else {
+        if (valid)
+          for (int i = part; i < rows; i += kParts) out.sh[(int64_t)hp.sh_dim * n + i] = a[i * B + col];
+      } else if (part == 0) {
         const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = 0; i < rows; ++i) raw[base + i] = a[i * kHeadsBlock + col];
+        for (int i = 0; i < rows; ++i) raw[base + i] = a[i * B + col];
       }
+      __syncthreads();   // a is layer 1's output of the next head
     }
-    store_heads(out, n, raw);
+    if (part == 0 && valid) store_heads(out, n, raw);
   }
 }
 
 __device__ __forceinline__ float g0(const float* p, int64_t i) { return p ? __ldg(p + i) : 0.0f; }
 
 // slot[p] += sum over the block's positions of d[o][t] * x[k][t] (weights)
-// and d[o][t] (biases) of one layer; each thread owns fixed parameters.
+// and d[o][t] (biases) of one layer, as fp32 reductions (no load to wait
+// for); each thread owns fixed parameters, so each slot element's adds come
+// from one thread in program order and the sum does not depend on scheduling.
 __device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out, int n_in, float* slot, int blk) {
   const int nW = n_out * n_in;
   for (int p = threadIdx.x; p < nW + n_out; p += blockDim.x) {
@@ -164,15 +183,16 @@ __device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out,
     } else {
       for (int t = 0; t < blk; ++t) s += d[(p - nW) * blk + t];
     }
-    slot[p] += s;
+    atomicAdd(slot + p, s);
   }
 }
 
-// dx[k] (+)= sum_o W[o][k] d[o] for this column; times gelu'(pre[k]) when pre is given.
+// dx[k] (+)= sum_o W[o][k] d[o] for this part's k (part, part + kParts, ...),
+// this column; times gelu'(pre[k]) when pre is given.
 template <typename W>
 __device__ __forceinline__ void dgrad(const W* __restrict__ Wp, int n_out, int n_in, const float* d, float* dx,
-                                      const float* pre, bool accumulate, int blk, int col) {
-  for (int k = 0; k < n_in; ++k) {
+                                      const float* pre, bool accumulate, int blk, int col, int part) {
+  for (int k = part; k < n_in; k += kParts) {
     float s = 0.0f;
     for (int o = 0; o < n_out; ++o) s = fmaf(wv(Wp + o * n_in, k), d[o * blk + col], s);
     if (pre) s *= gelu_grad(pre[k * blk + col]);
@@ -181,13 +201,10 @@ __device__ __forceinline__ void dgrad(const W* __restrict__ Wp, int n_out, int n
 }
 
 template <typename T, int F, typename W>
-__global__ void __launch_bounds__(kHeadsBwdBlock) heads_bwd_kernel(GridParams g, HeadsParams hp,
-                                                                   const float4* __restrict__ pos, int64_t N,
-                                                                   const T* __restrict__ tables,
-                                                                   const W* __restrict__ weights,
-                                                                   const float* __restrict__ latent, HeadsGrads go,
-                                                                   float* __restrict__ grad_tables,
-                                                                   float* __restrict__ ws, int n_params) {
+__global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
+    GridParams g, HeadsParams hp, const float4* __restrict__ pos, int64_t N, const T* __restrict__ tables,
+    const W* __restrict__ weights, const float* __restrict__ latent, HeadsGrads go, float* __restrict__ grad_tables,
+    float* __restrict__ ws, int n_params) {
   constexpr int B = kHeadsBwdBlock;
   extern __shared__ float sm[];
   float* z = sm;                       // [IN][B]
@@ -197,7 +214,8 @@ __global__ void __launch_bounds__(kHeadsBwdBlock) heads_bwd_kernel(GridParams g,
   float* h2 = p2 + kMaxDim * B;
   float* dy = h2 + kMaxDim * B;        // one head's output adjoint
   float* dz = dy + kMaxDim * B;
-  const int col = threadIdx.x;
+  float* dattr = dz + kMaxDim * B;     // [8][B]: adjoint of raw scale, rot, opacity
+  const int col = threadIdx.x % B, part = threadIdx.x / B;
   const int IN = hp.in_dim, H = hp.hidden;
   float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
   for (int p = threadIdx.x; p < n_params; p += blockDim.x) slot[p] = 0.0f;
@@ -206,50 +224,60 @@ __global__ void __launch_bounds__(kHeadsBwdBlock) heads_bwd_kernel(GridParams g,
     const int64_t n = n0 + col;
     const bool valid = n < N;
     float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    float dy_attr[8];   // adjoint of raw scale (3), rot (4), opacity (1)
-    if (valid) {
-      normalise_position(pos[n], g, xt);
-      if (latent) {
-        for (int k = 0; k < IN; ++k) z[k * B + col] = __ldg(latent + n * IN + k);
-      } else {
-        gather_z<T, F>(xt, g, tables, z, B, col, nullptr, n, IN);
-      }
-      // raw outputs of the scale, rotation and opacity heads
-      float raw[8];
-      for (int h = 0; h < 4; ++h) {
-        if (h == 2) continue;
-        const W* w = weights + hp.off[h];
-        layer<W>(w, H, IN, z, h1, nullptr, true, B, col);
-        w += H * IN + H;
-        layer<W>(w, H, H, h1, h2, nullptr, true, B, col);
-        w += H * H + H;
-        layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, B, col);
+    if (valid) normalise_position(pos[n], g, xt);
+    if (valid && latent) {
+      for (int k = part; k < IN; k += kParts) z[k * B + col] = __ldg(latent + n * IN + k);
+    } else if (valid) {
+      gather_z<T, F>(xt, g, tables, z, B, col, part, nullptr, n, IN);
+    } else {
+      for (int k = part; k < IN; k += kParts) z[k * B + col] = 0.0f;
+    }
+    for (int k = part; k < IN; k += kParts) dz[k * B + col] = 0.0f;
+    __syncthreads();
+    // raw outputs of the scale, rotation and opacity heads, then (part 0) the
+    // adjoint of Eq. 11 and Eq. 2
+    float raw[8];
+    for (int h = 0; h < 4; ++h) {
+      if (h == 2) continue;
+      const W* w = weights + hp.off[h];
+      layer<W>(w, H, IN, z, h1, nullptr, true, B, col, part);
+      __syncthreads();
+      w += H * IN + H;
+      layer<W>(w, H, H, h1, h2, nullptr, true, B, col, part);
+      __syncthreads();
+      w += H * H + H;
+      layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, B, col, part);
+      __syncthreads();
+      if (part == 0) {
         const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
         for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[i * B + col];
       }
-      // adjoint of Eq. 11 and Eq. 2
-      float s[3], r[4], cov_g[6], gs[3], gr[4];
-#pragma unroll
-      for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
-      const float nrm = normalise_quat(raw + 3, r);
-#pragma unroll
-      for (int i = 0; i < 6; ++i) cov_g[i] = g0(go.cov, 6 * n + i);
-#pragma unroll
-      for (int i = 0; i < 3; ++i) gs[i] = g0(go.scale, 3 * n + i);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) gr[i] = g0(go.rot, 4 * n + i);
-      covariance_backward(s, r, cov_g, gs, gr);
-#pragma unroll
-      for (int i = 0; i < 3; ++i) dy_attr[i] = raw[i] <= 20.0f ? gs[i] * s[i] : 0.0f;
-      normalise_quat_backward(r, nrm, gr, dy_attr + 3);
-      const float o = sigmoidf_(raw[7]);
-      dy_attr[7] = g0(go.opacity, n) * o * (1.0f - o);
-    } else {
-      for (int k = 0; k < IN; ++k) z[k * B + col] = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) dy_attr[i] = 0.0f;
+      __syncthreads();
     }
-    for (int k = 0; k < IN; ++k) dz[k * B + col] = 0.0f;
+    if (part == 0) {
+      float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (valid) {
+        float s[3], r[4], cov_g[6], gs[3], gr[4];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
+        const float nrm = normalise_quat(raw + 3, r);
+#pragma unroll
+        for (int i = 0; i < 6; ++i) cov_g[i] = g0(go.cov, 6 * n + i);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) gs[i] = g0(go.scale, 3 * n + i);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) gr[i] = g0(go.rot, 4 * n + i);
+        covariance_backward(s, r, cov_g, gs, gr);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) d[i] = raw[i] <= 20.0f ? gs[i] * s[i] : 0.0f;
+        normalise_quat_backward(r, nrm, gr, d + 3);
+        const float o = sigmoidf_(raw[7]);
+        d[7] = g0(go.opacity, n) * o * (1.0f - o);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dattr[i * B + col] = d[i];
+    }
+    __syncthreads();
     // ---- per head: forward with pre-activations, then the three layers' gradients ----
     for (int h = 0; h < 4; ++h) {
       const int rows = hp.rows[h];
@@ -259,32 +287,29 @@ __global__ void __launch_bounds__(kHeadsBwdBlock) heads_bwd_kernel(GridParams g,
       float* s1 = slot + hp.off[h];
       float* s2 = s1 + H * IN + H;
       float* s3 = s2 + H * H + H;
-      if (valid) {
-        layer<W>(w1, H, IN, z, h1, p1, true, B, col);
-        layer<W>(w2, H, H, h1, h2, p2, true, B, col);
-        if (h == 2) {
-          for (int i = 0; i < rows; ++i) dy[i * B + col] = g0(go.sh, (int64_t)hp.sh_dim * n + i);
-        } else {
-          const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-          for (int i = 0; i < rows; ++i) dy[i * B + col] = dy_attr[base + i];
-        }
+      layer<W>(w1, H, IN, z, h1, p1, true, B, col, part);
+      __syncthreads();
+      layer<W>(w2, H, H, h1, h2, p2, true, B, col, part);
+      if (h == 2) {
+        for (int i = part; i < rows; i += kParts)
+          dy[i * B + col] = valid ? g0(go.sh, (int64_t)hp.sh_dim * n + i) : 0.0f;
       } else {
-        for (int k = 0; k < H; ++k) h1[k * B + col] = h2[k * B + col] = p1[k * B + col] = p2[k * B + col] = 0.0f;
-        for (int i = 0; i < rows; ++i) dy[i * B + col] = 0.0f;
+        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+        for (int i = part; i < rows; i += kParts) dy[i * B + col] = dattr[(base + i) * B + col];
       }
       __syncthreads();
       wgrad(dy, h2, rows, H, s3, B);
-      dgrad<W>(w3, rows, H, dy, p2, p2, false, B, col);      // p2 <- d(pre 2)
+      dgrad<W>(w3, rows, H, dy, p2, p2, false, B, col, part);      // p2 <- d(pre 2)
       __syncthreads();
       wgrad(p2, h1, H, H, s2, B);
-      dgrad<W>(w2, H, H, p2, p1, p1, false, B, col);         // p1 <- d(pre 1)
+      dgrad<W>(w2, H, H, p2, p1, p1, false, B, col, part);         // p1 <- d(pre 1)
       __syncthreads();
       wgrad(p1, z, H, IN, s1, B);
-      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, B, col);    // dz += W1^T d(pre 1)
+      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, B, col, part);    // dz += W1^T d(pre 1)
       __syncthreads();
     }
     if (valid) {
-      for (int l = 0; l < g.L; ++l) {
+      for (int l = part; l < g.L; l += kParts) {
         float d[F];
 #pragma unroll
         for (int f = 0; f < F; ++f) d[f] = dz[(l * F + f) * B + col];
@@ -303,7 +328,7 @@ __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, in
   }
 }
 
-constexpr size_t kBwdSmem = (size_t)7 * kMaxDim * kHeadsBwdBlock * sizeof(float);
+constexpr size_t kBwdSmem = ((size_t)7 * kMaxDim + 8) * kHeadsBwdBlock * sizeof(float);
 
 int validate_heads(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
   if (!h) return SPIN4D_ERR_INVALID;
@@ -344,7 +369,7 @@ struct HeadsLaunch {
   static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const HeadsOut& o, cudaStream_t s) {
     const int blocks = persistent_blocks((N + kHeadsBlock - 1) / kHeadsBlock, 6);
-    heads_fwd_kernel<T, F, W><<<blocks, kHeadsBlock, 0, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+    heads_fwd_kernel<T, F, W><<<blocks, kHeadsBlock * kParts, 0, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
                                                              static_cast<const T*>(tables),
                                                              static_cast<const W*>(weights), o);
     return launch_status();
@@ -356,7 +381,7 @@ struct HeadsLaunch {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
     if (e != cudaSuccess) return cuda_status(e);
     const int blocks = bwd_blocks(N);
-    k<<<blocks, kHeadsBwdBlock, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+    k<<<blocks, kHeadsBwdBlock * kParts, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
                                               static_cast<const T*>(tables), static_cast<const W*>(weights), latent,
                                               go, grad_tables, ws, n_params);
     SPIN4D_CHECK(launch_status());

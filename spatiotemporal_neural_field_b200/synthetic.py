@@ -408,3 +408,82 @@ def upstream_grads(n: int, widths: Dict[str, int], std: float, seed: int = 0) ->
 
 DECODE_OUT_WIDTHS = {"scale": 3, "rot": 4, "rgb": 3, "opacity": 1, "cov": 6}
 HEX_OUT_WIDTHS = {"mu": 3, "rot": 4, "scale": 3, "sh": 48, "cov": 6}
+
+
+# ---------------------------------------------------------------------------
+# Rendering inputs
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class CameraSpec:
+    """A pinhole camera: view is the 3 x 4 world -> camera matrix [R | t]
+    (camera looking along +z, y down the image), intrinsics in pixels."""
+    view: Tuple[Tuple[float, ...], ...]
+    fx: float
+    fy: float
+    cx: float
+    cy: float
+    width: int
+    height: int
+    z_near: float = 0.2
+
+
+def orbit_camera(width: int = 640, height: int = 360, focal: float = 560.0, distance: float = 2.8,
+                 azimuth_deg: float = 30.0, elevation_deg: float = 15.0, z_near: float = 0.2) -> CameraSpec:
+    """A camera on a sphere of radius ``distance`` around the origin, looking
+    at it (the Panoptic Sports cameras ring the dome at 640 x 360)."""
+    az, el = math.radians(azimuth_deg), math.radians(elevation_deg)
+    eye = distance * np.array([math.cos(el) * math.sin(az), -math.sin(el), -math.cos(el) * math.cos(az)])
+    fwd = -eye / np.linalg.norm(eye)
+    up = np.array([0.0, -1.0, 0.0])
+    right = np.cross(up, fwd)
+    right /= np.linalg.norm(right)
+    down = np.cross(fwd, right)
+    R = np.stack([right, down, fwd])                # rows: camera x, y, z axes in world coordinates
+    t = -R @ eye
+    view = np.concatenate([R, t[:, None]], axis=1).astype(np.float32)
+    return CameraSpec(view=tuple(map(tuple, view.tolist())), fx=float(focal), fy=float(focal),
+                      cx=width / 2.0, cy=height / 2.0, width=int(width), height=int(height), z_near=float(z_near))
+
+
+def random_spd(n: int, sigmas: np.ndarray, g: np.random.Generator) -> np.ndarray:
+    """n x 6 packed (xx, xy, xz, yy, yz, zz) symmetric positive-definite
+    matrices U diag(sigmas^2) U^T, U a random orthogonal matrix (QR of a
+    normal matrix)."""
+    U, _ = np.linalg.qr(g.normal(size=(n, 3, 3)))
+    M = U * (sigmas ** 2)[:, None, :]
+    S = M @ np.transpose(U, (0, 2, 1))
+    return np.stack([S[:, 0, 0], S[:, 0, 1], S[:, 0, 2], S[:, 1, 1], S[:, 1, 2], S[:, 2, 2]], axis=1)
+
+
+def render_scene(n: int, seed: int = 0, positions: Optional[np.ndarray] = None, sh_degree: int = 3,
+                 scale_factor: float = 0.5, opacity_lo: float = 0.05) -> Dict[str, np.ndarray]:
+    """Attributes shaped like a trained scene: per-axis standard deviations
+    log-normal around ``scale_factor`` x the mean spacing (8/n)^(1/3) of n
+    points in the [-1,1]^3 box, random orientations, opacity = sigmoid(N(0, 2^2))
+    floored at ``opacity_lo``, SH coefficients with the degree-0 term
+    U(0.4, 3.2) and the higher ones N(0, 0.1^2) (sh_degree -1: RGB U(0.05, 1)).
+    Positions default to frame 75 of the sports scene."""
+    g = rng(seed + 909)
+    if positions is None:
+        positions = sports_scene(n, seed).frame(75)
+    mu = np.ascontiguousarray(positions[:, :3], np.float32)
+    n = mu.shape[0]
+    s0 = scale_factor * (8.0 / max(n, 1)) ** (1.0 / 3.0)
+    sig = s0 * np.exp(g.normal(0.0, 0.4, size=(n, 3)))
+    cov = random_spd(n, sig, g).astype(np.float32)
+    op = 1.0 / (1.0 + np.exp(-g.normal(0.0, 2.0, size=n)))
+    op = np.maximum(op, opacity_lo).astype(np.float32)
+    if sh_degree < 0:
+        col = g.uniform(0.05, 1.0, size=(n, 3)).astype(np.float32)
+    else:
+        K = (sh_degree + 1) ** 2
+        col = g.normal(0.0, 0.1, size=(n, K, 3))
+        col[:, 0, :] = g.uniform(0.4, 3.2, size=(n, 3))
+        col = col.reshape(n, 3 * K).astype(np.float32)
+    return dict(mu=mu, cov=cov, opacity=op, colours=col)
+
+
+def image_grads(cam: CameraSpec, std: float = 1.0, seed: int = 0) -> np.ndarray:
+    """3 x H x W float32 upstream image gradients ~ N(0, std^2)."""
+    g = rng(seed + 1010)
+    return g.normal(0.0, std, size=(3, cam.height, cam.width)).astype(np.float32)

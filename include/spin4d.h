@@ -480,6 +480,94 @@ int spin4d_permute_rows(const void* src, int64_t src_rows, void* dst, const uint
                         int64_t row_bytes, spin4d_stream_t stream);
 
 /*
+ * Rendering of the decoded Gaussians (SPIN-4DGS section 3.1): each Gaussian
+ * exp(-(x-mu)^T Sigma^-1 (x-mu)/2) (Eq. 1) is projected to the image with
+ * Sigma_2D = J W Sigma W^T J^T (Eq. 3, W the view rotation, J the Jacobian
+ * of the pinhole projection at the camera-space mean), and every pixel
+ * blends the Gaussians covering it front to back,
+ * C = sum_i c_i a_i prod_{j<i} (1 - a_j), a_i = o_i G_2D,i(pixel) (Eq. 4).
+ *
+ * Where the pages are silent the library fixes:
+ *  - pixel (i, j) (column i, row j) is evaluated at image point
+ *    (i + 1/2, j + 1/2); a camera-space point (x, y, z) maps to
+ *    (fx x/z + cx, fy y/z + cy); Gaussians with z <= z_near are culled;
+ *  - `lowpass` (pixels^2) is added to the diagonal of Sigma_2D (EWA's
+ *    screen-space filter; 0 gives Eq. 3 exactly) and a Gaussian whose
+ *    filtered Sigma_2D is not positive definite is culled;
+ *  - a Gaussian covers a pixel when its Mahalanobis distance d^2 <= 9;
+ *    a = min(alpha_max, o exp(-d^2/2)); a pixel skips a Gaussian with
+ *    a < alpha_min; blending stops before the first Gaussian that would take
+ *    the transmittance below t_stop; the remaining transmittance times
+ *    `background` is added last;
+ *  - order: camera depth z ascending (fp32), equal depths by index;
+ *  - colour: sh_degree -1 reads RGB (N x 3); degree D in 0..3 reads
+ *    (D+1)^2 real spherical-harmonic coefficients per channel,
+ *    coefficient-major (N x 3(D+1)^2, value [n][3 (l*l + l + m) + channel]),
+ *    evaluates the real SH without Condon-Shortley phase in the direction
+ *    from the camera centre (-R^T t) to mu, and clamps the sum at 0.
+ */
+#define SPIN4D_MAX_IMAGE_SIDE 16384
+#define SPIN4D_MAX_RENDER_GAUSSIANS (1ll << 31)
+#define SPIN4D_MAX_RENDER_PAIRS (1ll << 31)
+
+typedef struct spin4d_camera {
+    float view[12];          /* world -> camera [R | t], row-major 3 x 4: x_c = R mu + t; looks along +z */
+    float fx, fy, cx, cy;    /* pinhole intrinsics in pixels, fx, fy > 0 */
+    int32_t width, height;   /* 1..SPIN4D_MAX_IMAGE_SIDE */
+    float z_near;            /* > 0 */
+} spin4d_camera;
+
+typedef struct spin4d_render_desc {
+    int32_t sh_degree;       /* -1 (RGB) or 0..3 */
+    float lowpass;           /* >= 0, pixels^2 (e.g. 0.3) */
+    float alpha_max;         /* in (0, 1) (e.g. 0.99) */
+    float alpha_min;         /* in [0, alpha_max) (e.g. 1/255) */
+    float t_stop;            /* in [0, 1) (e.g. 1e-4; 0 blends every covering Gaussian) */
+    float background[3];
+    int32_t mean_stride;     /* floats from one mean to the next: 3, or 4 for (x, y, z, t) rows */
+    int32_t reserved;        /* must be 0 */
+} spin4d_render_desc;
+
+/*
+ * Bytes of the render state for N Gaussians, an image of width x height and
+ * room for max_pairs (Gaussian, 16x16 tile) pairs; 0 for invalid sizes.  The
+ * state is owned by the caller (device, 256-byte aligned); the forward
+ * fills it and the backward reads it.  Its first 8 bytes hold, after a
+ * forward, the number of pairs the frame needed (uint64): a value above
+ * max_pairs means the pairs did not fit, the image is incomplete and the call
+ * must be repeated with a larger max_pairs.  Bytes 8..11 hold the pairs kept
+ * (max_pairs when they did not fit; 0 if the total exceeds 2^32 - 1).
+ */
+size_t spin4d_render_state_bytes(int64_t N, int width, int height, int64_t max_pairs);
+
+/*
+ * Forward: means N rows of mean_stride floats (x, y, z first), cov N x 6
+ * packed (xx, xy, xz, yy, yz, zz), opacity N, colours as sh_degree says (all
+ * fp32, device, 4-byte aligned; may be NULL when N = 0).  Writes image
+ * (3 x height x width fp32, channel planes) and, if final_T is not NULL, the
+ * final transmittance (height x width fp32); both are overwritten, not
+ * accumulated.  0 <= N <= SPIN4D_MAX_RENDER_GAUSSIANS.
+ */
+int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_desc* desc, int64_t N, const float* means,
+                      const float* cov, const float* opacity, const float* colours, float* image, float* final_T,
+                      void* state, size_t state_bytes, int64_t max_pairs, spin4d_stream_t stream);
+
+/*
+ * Backward of spin4d_render_fwd for loss = sum(grad_image * image)
+ * (grad_image 3 x height x width fp32): the same camera, desc, inputs,
+ * state and max_pairs as the forward it follows.  ACCUMULATES into
+ * grad_means (N x 3), grad_cov (N x 6, the gradient w.r.t. each packed
+ * value), grad_opacity (N) and grad_colours (shaped like colours); any of
+ * them may be NULL.  The culling, support, alpha_min and termination
+ * decisions are those of the forward; a clamped alpha (o G > alpha_max) has
+ * zero derivative.  Culled Gaussians get no gradient.
+ */
+int spin4d_render_bwd(const spin4d_camera* cam, const spin4d_render_desc* desc, int64_t N, const float* means,
+                      const float* cov, const float* opacity, const float* colours, const float* grad_image,
+                      void* state, size_t state_bytes, int64_t max_pairs, float* grad_means, float* grad_cov,
+                      float* grad_opacity, float* grad_colours, spin4d_stream_t stream);
+
+/*
  * Measurement helper (not part of the decoder): the gather-rate ceiling.
  * Launches `blocks` x 256 threads; each issues `loads_per_thread` (a multiple
  * of 8) independent loads at pseudo-random, width-aligned offsets of `buf`

@@ -55,9 +55,9 @@ SUPPORT_D2 = 9.0            # 3-sigma ellipse
 PACK3 = ((0, 0), (0, 1), (0, 2), (1, 1), (1, 2), (2, 2))
 
 # margins below which a decision is called ambiguous (see module docstring)
-D2_MARGIN = 0.02            # absolute, on d^2 near 9
+D2_MARGIN = 2.5e-3          # absolute, on d^2 near 9 (fp32 error <= 1.3e-3 at the narrowest filtered footprint)
 REL_MARGIN = 2e-3           # relative, on alpha vs alpha_min / alpha_max and T vs t_stop
-DEPTH_MARGIN = 1e-5         # relative gap between two contributors' depths
+DEPTH_MARGIN = 1e-6         # relative gap between two contributors' depths (fp32 depth: <= 3e-7)
 
 
 @dataclass
@@ -211,38 +211,48 @@ def _depth_order(pr) -> np.ndarray:
 
 def composite_pixel(px: float, py: float, pr, order, st: Settings):
     """One pixel: returns (rgb, T_final, contributors in order, their alphas,
-    the transmittance before each, margin_ok, grad_margin_ok)."""
+    the transmittance before each, margin_ok, grad_margin_ok).
+
+    A margin counts only where the decision can change the result: Gaussians
+    up to the one that ends the blending, the 3-sigma edge only where alpha
+    there would still reach alpha_min."""
     m = pr["mean2d"][order]
     q = pr["conic"][order]
+    o = pr["opacity"][order]
     dx, dy = px - m[:, 0], py - m[:, 1]
     d2 = q[:, 0] * dx * dx + 2.0 * q[:, 1] * dx * dy + q[:, 2] * dy * dy
-    ok = True
-    gok = True
-    if np.any(np.abs(d2 - SUPPORT_D2) < D2_MARGIN):
-        ok = False
     cover = d2 <= SUPPORT_D2
-    idx = order[cover]
-    a_raw = pr["opacity"][idx] * np.exp(-0.5 * d2[cover])
+    a_raw = o * np.exp(-0.5 * d2)
     a = np.minimum(a_raw, st.alpha_max)
-    if np.any(np.abs(a_raw - st.alpha_max) < REL_MARGIN * st.alpha_max):
-        gok = False
-    if st.alpha_min > 0 and np.any(np.abs(a - st.alpha_min) < REL_MARGIN * st.alpha_min):
-        ok = False
-    keep = a >= st.alpha_min
-    idx, a = idx[keep], a[keep]
-    Tb = np.concatenate([[1.0], np.cumprod(1.0 - a)])     # T before each, then after the last
+    blend = cover & (a >= st.alpha_min)
+    pos = np.flatnonzero(blend)                           # positions in `order` that blend
+    ab = a[pos]
+    Tb = np.concatenate([[1.0], np.cumprod(1.0 - ab)])   # T before each, then after the last
+    n_eval = len(order)
+    k = len(pos)
     if st.t_stop > 0:
-        if np.any(np.abs(Tb[1:] - st.t_stop) < REL_MARGIN * st.t_stop):
-            ok = False
         stop = np.flatnonzero(Tb[1:] < st.t_stop)
         if stop.size:
-            k = stop[0]
-            idx, a, Tb = idx[:k], a[:k], Tb[:k + 1]
+            k = int(stop[0])
+            n_eval = int(pos[k]) + 1                      # the ending Gaussian was evaluated
+    ev = slice(0, n_eval)
+    ok = True
+    edge_matters = o[ev] * math.exp(-0.5 * SUPPORT_D2) >= st.alpha_min * (1.0 - REL_MARGIN)
+    if np.any((np.abs(d2[ev] - SUPPORT_D2) < D2_MARGIN) & edge_matters):
+        ok = False
+    if st.alpha_min > 0 and np.any(cover[ev] & (np.abs(a[ev] - st.alpha_min) < REL_MARGIN * st.alpha_min)):
+        ok = False
+    if st.t_stop > 0 and np.any(np.abs(Tb[1:min(k + 1, len(pos)) + 1] - st.t_stop) < REL_MARGIN * st.t_stop):
+        ok = False
+    sel = pos[:k]
+    idx = order[sel]
+    a_k, Tb_k = ab[:k], Tb[:k + 1]
     z = pr["depth"][idx]
     if z.size > 1 and np.any(np.diff(z) < DEPTH_MARGIN * z[1:]):
         ok = False
-    rgb = (pr["rgb"][idx] * (a * Tb[:-1])[:, None]).sum(axis=0) + Tb[-1] * np.asarray(st.background, np.float64)
-    return rgb, Tb[-1], idx, a, Tb[:-1], ok, ok and gok
+    gok = not np.any(np.abs(a_raw[sel] - st.alpha_max) < REL_MARGIN * st.alpha_max)
+    rgb = (pr["rgb"][idx] * (a_k * Tb_k[:-1])[:, None]).sum(axis=0) + Tb_k[-1] * np.asarray(st.background, np.float64)
+    return rgb, Tb_k[-1], idx, a_k, Tb_k[:-1], ok, ok and gok
 
 
 def render_pixels(cam: Camera, st: Settings, mu, cov6, opacity, colours, pixels: np.ndarray):
@@ -299,6 +309,8 @@ def render_backward(cam: Camera, st: Settings, mu, cov6, opacity, colours, grad_
     gok = np.ones((cam.height, cam.width), bool)
     for j in range(cam.height):
         for i in range(cam.width):
+            if not np.any(grad_image[:, j, i]):
+                continue                                          # contributes nothing
             px, py = i + 0.5, j + 0.5
             _, Tf, idx, a, Tb, _, ok = composite_pixel(px, py, pr, order, st)
             gok[j, i] = ok

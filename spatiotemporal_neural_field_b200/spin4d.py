@@ -84,6 +84,16 @@ class AdamGroup(ctypes.Structure):
     _fields_ = [("end", c_i64), ("lr", c_f32)]
 
 
+class Camera(ctypes.Structure):
+    _fields_ = [("view", c_f32 * 12), ("fx", c_f32), ("fy", c_f32), ("cx", c_f32), ("cy", c_f32),
+                ("width", c_i32), ("height", c_i32), ("z_near", c_f32)]
+
+
+class RenderDesc(ctypes.Structure):
+    _fields_ = [("sh_degree", c_i32), ("lowpass", c_f32), ("alpha_max", c_f32), ("alpha_min", c_f32),
+                ("t_stop", c_f32), ("background", c_f32 * 3), ("mean_stride", c_i32), ("reserved", c_i32)]
+
+
 P = ctypes.POINTER
 _SIGS = {
     "spin4d_grid_init": (c_i32, [P(GridDesc), c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_f32, c_f32]),
@@ -125,6 +135,11 @@ _SIGS = {
     "spin4d_probe_atomic": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
     "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
+    "spin4d_render_state_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i64]),
+    "spin4d_render_fwd": (c_i32, [P(Camera), P(RenderDesc), c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
+                                  c_i64, c_vp]),
+    "spin4d_render_bwd": (c_i32, [P(Camera), P(RenderDesc), c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_i64,
+                                  c_vp, c_vp, c_vp, c_vp, c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
     "spin4d_version": (ctypes.c_char_p, []),
@@ -495,3 +510,95 @@ def probe_fma(iters: int, blocks: int, device, sink: Optional[torch.Tensor] = No
 
 def version() -> str:
     return lib.spin4d_version().decode()
+
+
+# ---------------------------------------------------------------------------
+# Rendering (EWA projection + tile alpha compositing)
+# ---------------------------------------------------------------------------
+def camera(view, fx: float, fy: float, cx: float, cy: float, width: int, height: int,
+           z_near: float = 0.2) -> Camera:
+    """view: 3 x 4 world -> camera [R | t] (nested sequence or array)."""
+    flat = [float(v) for row in view for v in row]
+    if len(flat) != 12:
+        raise ValueError("view must be 3 x 4")
+    return Camera((c_f32 * 12)(*flat), fx, fy, cx, cy, int(width), int(height), z_near)
+
+
+def camera_from_spec(spec) -> Camera:
+    return camera(spec.view, spec.fx, spec.fy, spec.cx, spec.cy, spec.width, spec.height, spec.z_near)
+
+
+def render_desc(sh_degree: int = 3, lowpass: float = 0.3, alpha_max: float = 0.99, alpha_min: float = 1.0 / 255.0,
+                t_stop: float = 1e-4, background=(0.0, 0.0, 0.0), mean_stride: int = 3) -> RenderDesc:
+    return RenderDesc(sh_degree, lowpass, alpha_max, alpha_min, t_stop, (c_f32 * 3)(*background), mean_stride, 0)
+
+
+class RenderState:
+    """Caller-owned state between ``render_fwd`` and ``render_bwd``."""
+
+    def __init__(self, N: int, width: int, height: int, max_pairs: int, device):
+        need = int(lib.spin4d_render_state_bytes(N, width, height, max_pairs))
+        if need == 0:
+            raise ValueError("invalid render sizes")
+        self.N, self.width, self.height, self.max_pairs = N, width, height, max_pairs
+        self.buf = torch.empty(need, dtype=torch.uint8, device=device)
+
+    def pairs_needed(self) -> int:
+        """(Gaussian, tile) pairs the last forward needed; synchronises."""
+        return int(self.buf[:8].view(torch.int64).item())
+
+    def pairs_kept(self) -> int:
+        return int(self.buf[8:12].view(torch.int32).item())
+
+
+def default_max_pairs(N: int, width: int, height: int) -> int:
+    return max(16 * N, ((width + 15) // 16) * ((height + 15) // 16), 1 << 16)
+
+
+def render_fwd(cam: Camera, desc: RenderDesc, means, cov, opacity, colours, image=None, final_T=None,
+               state: Optional[RenderState] = None, stream=None):
+    """Forward render; returns (image 3 x H x W, state).  Asynchronous: check
+    ``state.pairs_needed() <= state.max_pairs`` (or use ``render``)."""
+    N = means.shape[0]
+    dev = means.device
+    if state is None:
+        state = RenderState(N, cam.width, cam.height, default_max_pairs(N, cam.width, cam.height), dev)
+    if image is None:
+        image = torch.empty((3, cam.height, cam.width), dtype=torch.float32, device=dev)
+    _check("spin4d_render_fwd", lib.spin4d_render_fwd(ctypes.byref(cam), ctypes.byref(desc), N, _ptr(means),
+                                                      _ptr(cov), _ptr(opacity), _ptr(colours), _ptr(image),
+                                                      _ptr(final_T), _ptr(state.buf), state.buf.numel(),
+                                                      state.max_pairs, _stream(stream)))
+    return image, state
+
+
+def render(cam: Camera, desc: RenderDesc, means, cov, opacity, colours, final_T=None,
+           state: Optional[RenderState] = None, stream=None):
+    """Forward render that grows the pair capacity until the frame fits
+    (one host synchronisation per attempt)."""
+    image, state = render_fwd(cam, desc, means, cov, opacity, colours, final_T=final_T, state=state, stream=stream)
+    need = state.pairs_needed()
+    if need > state.max_pairs:
+        state = RenderState(means.shape[0], cam.width, cam.height, need, means.device)
+        image, state = render_fwd(cam, desc, means, cov, opacity, colours, image=image, final_T=final_T,
+                                  state=state, stream=stream)
+    return image, state
+
+
+def render_bwd(cam: Camera, desc: RenderDesc, means, cov, opacity, colours, grad_image, state: RenderState,
+               grad_means=None, grad_cov=None, grad_opacity=None, grad_colours=None, stream=None):
+    """Accumulates the render's gradients into the given tensors (allocating
+    zeroed ones for those left None); returns them as a dict."""
+    N = means.shape[0]
+    dev = means.device
+    z = lambda shape: torch.zeros(shape, dtype=torch.float32, device=dev)   # noqa: E731
+    grad_means = z((N, 3)) if grad_means is None else grad_means
+    grad_cov = z((N, 6)) if grad_cov is None else grad_cov
+    grad_opacity = z((N,)) if grad_opacity is None else grad_opacity
+    grad_colours = z(tuple(colours.shape)) if grad_colours is None else grad_colours
+    _check("spin4d_render_bwd", lib.spin4d_render_bwd(ctypes.byref(cam), ctypes.byref(desc), N, _ptr(means),
+                                                      _ptr(cov), _ptr(opacity), _ptr(colours), _ptr(grad_image),
+                                                      _ptr(state.buf), state.buf.numel(), state.max_pairs,
+                                                      _ptr(grad_means), _ptr(grad_cov), _ptr(grad_opacity),
+                                                      _ptr(grad_colours), _stream(stream)))
+    return dict(mu=grad_means, cov=grad_cov, opacity=grad_opacity, colours=grad_colours)

@@ -55,7 +55,8 @@ def parse():
                    help="time the oracle on every workload (1 thread and all cores); one JSON line each")
     p.add_argument("--ncu-case", default=None,
                    help="profiling driver: run a few untimed launches of one workload and exit "
-                        "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32)")
+                        "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32, "
+                        "render_sports_frame)")
     return p.parse_args()
 
 
@@ -707,7 +708,76 @@ def run_workloads(args):
     emit("hexplane_fp32", "fwd+bwd (saved latent)", n, timed(hfb, 10))
     emit("hexplane_fp32", "bwd (gathering again)", n,
          timed(lambda: sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws), 10))
+    del inp, planes, weights, out, lat, grads, gp, gw, ws, out_l
+    torch.cuda.empty_cache()
+    render_workloads(sp, torch, dev, timed)
     sp.check_device_errors()
+
+
+def render_workloads(sp, torch, dev, timed):
+    """EWA projection + tile compositing of one sports frame (300k Gaussians,
+    SH degree 3) at the Panoptic Sports resolution 640 x 360: forward as
+    separate launches and as one CUDA graph, forward+backward, and the
+    paper's decoder followed by the render (a whole decoded frame)."""
+    spec = S.orbit_camera(640, 360)
+    sc = S.render_scene(300_000, seed=0)
+    n = sc["mu"].shape[0]
+    cam, desc = sp.camera_from_spec(spec), sp.render_desc(sh_degree=3)
+    args = [torch.from_numpy(sc[k]).to(dev) for k in ("mu", "cov", "opacity", "colours")]
+    img, st = sp.render(cam, desc, *args)
+    T = torch.empty((360, 640), device=dev)
+    pairs = st.pairs_needed()
+
+    def fwd():
+        sp.render_fwd(cam, desc, *args, image=img, final_T=T, state=st)
+
+    def line(what, ms, **extra):
+        d = {"workload": "render_sports_frame", "pass": what, "gaussians": n, "width": 640, "height": 360,
+             "ms": ms, "frames_per_s": 1e3 / ms, "gaussians_per_s": n / (ms * 1e-3), "tile_pairs": pairs}
+        d.update(extra)
+        print(json.dumps(d), flush=True)
+
+    line("fwd (separate launches)", timed(fwd, 20))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fwd()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            fwd()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    line("fwd (one CUDA graph)", timed(graph.replay, 20))
+    G = torch.from_numpy(S.image_grads(spec)).to(dev)
+    grads = [torch.zeros((n, 3), device=dev), torch.zeros((n, 6), device=dev), torch.zeros(n, device=dev),
+             torch.zeros((n, 48), device=dev)]
+
+    def fb():
+        fwd()
+        sp.render_bwd(cam, desc, *args, G, st, *grads)
+
+    line("fwd+bwd (separate launches)", timed(fb, 20))
+    del graph
+
+    # the paper's decoder on the same frame, then the render of its output
+    grid, spec_h = S.GRID_PAPER, S.HEADS_PAPER
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec_h)
+    P = torch.from_numpy(S.sports_scene(n).frame(75)).to(dev)
+    Tb = torch.from_numpy(S.hash_tables(grid)).to(dev)
+    W = torch.from_numpy(S.heads_weights(spec_h)).to(dev)
+    out = sp.heads_fwd(g, h, P, Tb, W)
+    desc4 = sp.render_desc(sh_degree=3, mean_stride=4)
+    dimg, dst = sp.render(cam, desc4, P, out["cov"], out["opacity"], out["sh"])
+
+    def dr():
+        sp.heads_fwd(g, h, P, Tb, W, out=out)
+        sp.render_fwd(cam, desc4, P, out["cov"], out["opacity"], out["sh"], image=dimg, state=dst)
+
+    ms = timed(dr, 10)
+    print(json.dumps({"workload": "decode_and_render_frame", "pass": "paper decoder fwd + render fwd",
+                      "gaussians": n, "width": 640, "height": 360, "ms": ms, "frames_per_s": 1e3 / ms,
+                      "tile_pairs": dst.pairs_needed(),
+                      "note": "decoder at its initial state (scale e^-5, opacity 0.1, SH 0)"}), flush=True)
 
 
 def _oracle_chunk(task):
@@ -723,9 +793,18 @@ def _oracle_chunk(task):
 
 
 def _oracle_job(name, what, n, seed):
-    """The oracle's forward (or forward+backward) on n positions of a workload."""
-    from oracle import decoder as dec, hexplane as hxo
+    """The oracle's forward (or forward+backward) on n positions of a workload
+    (for the render: n sampled pixels of the frame)."""
+    from oracle import decoder as dec, hexplane as hxo, render as rdo
     rng = np.random.default_rng(seed)
+    if name == "render_sports_frame":
+        spec = S.orbit_camera(640, 360)
+        sc = S.render_scene(300_000, seed=0)
+        cam = rdo.Camera(view=np.array(spec.view, np.float64), fx=spec.fx, fy=spec.fy, cx=spec.cx, cy=spec.cy,
+                         width=spec.width, height=spec.height, z_near=spec.z_near)
+        pix = np.stack([rng.integers(0, 640, n), rng.integers(0, 360, n)], axis=1)
+        return lambda: rdo.render_pixels(cam, rdo.Settings(sh_degree=3), sc["mu"], sc["cov"], sc["opacity"],
+                                         sc["colours"], pix)
     if name == "hexplane_fp32":
         hx = S.WORKLOADS[name]["hex"]
         inp = S.hexplane_inputs(n, seed)
@@ -762,7 +841,8 @@ def run_cpu_workloads(args):
     procs = min(os.cpu_count() or 1, 32)
     jobs = [("tiny_fp32", "fwd", 4096), ("tiny_fp32", "fwd+bwd", 4096), ("sports_frame_fp16", "fwd", 20_000),
             ("sports_train_fp16", "fwd+bwd", 10_000), ("stress_fp16_gate", "fwd", 10_000),
-            ("hexplane_fp32", "fwd", 2_000), ("hexplane_fp32", "fwd+bwd", 1_000)]
+            ("hexplane_fp32", "fwd", 2_000), ("hexplane_fp32", "fwd+bwd", 1_000),
+            ("render_sports_frame", "fwd", 64)]
     ctx = mp.get_context("spawn")
     with ctx.Pool(procs) as pool:
         pool.map(_oracle_chunk, [("tiny_fp32", "fwd", i, 64) for i in range(procs)])   # start every worker
@@ -770,6 +850,15 @@ def run_cpu_workloads(args):
             one = _oracle_chunk((name, what, 1, n))
             line = {"workload": name, "pass": what, "kind": "oracle", "sample": n,
                     "positions_per_s_1_thread": n / one, "host_cores": os.cpu_count()}
+            if name == "render_sports_frame":
+                # the projection of all 300k Gaussians is paid once per frame, the blend per pixel
+                proj = _oracle_chunk((name, what, 1, 0))
+                frame = proj + (one - proj) * 640 * 360 / n
+                line = {"workload": name, "pass": what, "kind": "oracle", "sample_pixels": n,
+                        "sample_s": one, "projection_s": proj, "frame_s_1_thread_extrapolated": frame,
+                        "host_cores": os.cpu_count()}
+                print(json.dumps(line), flush=True)
+                continue
             if name != "stress_fp16_gate":
                 t0 = time.perf_counter()
                 pool.map(_oracle_chunk, [(name, what, 100 + i, n) for i in range(procs)])
@@ -785,7 +874,21 @@ def run_ncu_case(name):
     _b.build()
     from spatiotemporal_neural_field_b200 import spin4d as sp
     dev = torch.device("cuda", 0)
-    w = S.WORKLOADS[name]
+    w = S.WORKLOADS.get(name)
+    if name == "render_sports_frame":
+        spec = S.orbit_camera(640, 360)
+        sc = S.render_scene(300_000, seed=0)
+        cam, desc = sp.camera_from_spec(spec), sp.render_desc(sh_degree=3)
+        args = [torch.from_numpy(sc[k]).to(dev) for k in ("mu", "cov", "opacity", "colours")]
+        G = torch.from_numpy(S.image_grads(spec)).to(dev)
+        img, st = sp.render(cam, desc, *args)
+        for _ in range(3):
+            sp.render_fwd(cam, desc, *args, image=img, state=st)
+            sp.render_bwd(cam, desc, *args, G, st)
+        torch.cuda.synchronize()
+        sp.check_device_errors()
+        print("ncu case done:", name)
+        return
     if name == "hexplane_fp32":
         hx = w["hex"]
         n = w["N"]

@@ -1,12 +1,16 @@
 // Stable least-significant-digit radix sort of 32-bit keys with 32-bit
-// values, 8-bit digits: per pass a histogram kernel, an exclusive scan of the
-// (digit, block) counts and a scatter kernel that ranks each block's keys
-// stably (warp match on the digit, then a prefix over the warps), so equal
-// keys keep their input order and the result is deterministic.
+// values, 8-bit digits.  Each pass: a histogram kernel, a two-kernel
+// exclusive scan of the (digit, block) counts and a scatter kernel that
+// ranks each block's keys stably (warp match on the digit, then a prefix
+// over the warps), so equal keys keep their input order and the result is
+// deterministic.
 //
-// The key count may live on the device (n_dev, read by the kernels and
-// clamped to the capacity N the launch is sized for), so a sort can follow a
-// kernel that produced a data-dependent number of keys without a host sync.
+// The grid is fixed by the capacity (at most kMaxSortBlocks blocks, a few per
+// SM); each block owns one contiguous chunk of the keys, sized from the key
+// count at run time.  That count may live on the device (n_dev, clamped to
+// the capacity), so a sort can follow a kernel that produced a
+// data-dependent number of keys without a host sync, and the scan stays
+// sized by the grid, not by the capacity.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -16,28 +20,43 @@ namespace spin4d {
 namespace radix {
 namespace {   // every translation unit that sorts gets its own copy of the kernels
 
-constexpr int kSortThreads = 256;
-constexpr int kSortPerThread = 8;
-constexpr int kSortTile = kSortThreads * kSortPerThread;   // keys per block
+constexpr int kSortThreads = 256;              // keys ranked per round
+constexpr int kMinKeysPerBlock = 2048;
+constexpr int kMaxSortBlocks = 640;
 constexpr int kDigits = 256;
 constexpr int kScanThreads = 1024;
 constexpr int kScanPerThread = 8;
 constexpr int kScanChunk = kScanThreads * kScanPerThread;
+constexpr int kFusedScanMaxChunks = 1024;      // above this the chunk partials get their own scan kernel
+
+inline int sort_blocks(int64_t N) {
+  const int64_t b = (N + kMinKeysPerBlock - 1) / kMinKeysPerBlock;
+  return (int)(b < 1 ? 1 : (b > kMaxSortBlocks ? kMaxSortBlocks : b));
+}
+inline int64_t scan_len(int64_t N) { return (int64_t)sort_blocks(N) * kDigits; }
+inline int64_t scan_chunks(int64_t len) { return (len + kScanChunk - 1) / kScanChunk; }
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Block b's keys: [b * chunk, min((b + 1) * chunk, n)), chunk a multiple of
+// kSortThreads.
+__device__ __forceinline__ void block_chunk(int64_t N, const uint32_t* n_dev, int64_t& lo, int64_t& hi) {
+  const int64_t n = n_dev ? min(N, (int64_t)*n_dev) : N;
+  int64_t chunk = (n + gridDim.x - 1) / gridDim.x;
+  chunk = (chunk + kSortThreads - 1) / kSortThreads * kSortThreads;
+  lo = min((int64_t)blockIdx.x * chunk, n);
+  hi = min(lo + chunk, n);
+}
 
 // counts[d * B + b] = keys of block b whose digit is d.
 __global__ void __launch_bounds__(kSortThreads) radix_histogram(const uint32_t* __restrict__ keys, int64_t N,
                                                                 const uint32_t* __restrict__ n_dev, int shift,
                                                                 uint32_t* __restrict__ counts) {
-  if (n_dev) N = min(N, (int64_t)*n_dev);
   __shared__ uint32_t h[kDigits];
   h[threadIdx.x] = 0;
   __syncthreads();
-  const int64_t t0 = (int64_t)blockIdx.x * kSortTile;
-#pragma unroll
-  for (int r = 0; r < kSortPerThread; ++r) {
-    const int64_t i = t0 + r * kSortThreads + threadIdx.x;
-    if (i < N) atomicAdd(&h[(keys[i] >> shift) & 0xFFu], 1u);
-  }
+  int64_t lo, hi;
+  block_chunk(N, n_dev, lo, hi);
+  for (int64_t i = lo + threadIdx.x; i < hi; i += kSortThreads) atomicAdd(&h[(keys[i] >> shift) & 0xFFu], 1u);
   __syncthreads();
   counts[(size_t)threadIdx.x * gridDim.x + blockIdx.x] = h[threadIdx.x];
 }
@@ -83,7 +102,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_reduce(const uint32_t* __re
   if (threadIdx.x == 0) partial[blockIdx.x] = total;
 }
 
-// Scan step 2 (one block): partial[] -> its exclusive scan, in place.
+// Scan step 2 for many chunks (one block): partial[] -> its exclusive scan, in place.
 __global__ void __launch_bounds__(kScanThreads) scan_partials(uint32_t* __restrict__ partial, int n) {
   __shared__ uint32_t s_warp[32];
   uint32_t carry = 0;
@@ -97,11 +116,25 @@ __global__ void __launch_bounds__(kScanThreads) scan_partials(uint32_t* __restri
   }
 }
 
-// Scan step 3: out = exclusive scan of a, chunk c starting at partial[c].
+// Last step: out = exclusive scan of a.  FUSED: chunk c's start is the sum of
+// partial[0..c) (the raw chunk sums), added up here; otherwise partial[c]
+// already holds it.
+template <bool FUSED>
 __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __restrict__ a, int64_t n,
                                                            const uint32_t* __restrict__ partial,
                                                            uint32_t* __restrict__ out) {
   __shared__ uint32_t s_warp[32];
+  __shared__ uint32_t s_base;
+  if (FUSED) {
+    if (threadIdx.x < 32) {
+      uint32_t acc = 0;
+      for (int c = threadIdx.x; c < (int)blockIdx.x; c += 32) acc += partial[c];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (threadIdx.x == 0) s_base = acc;
+    }
+    __syncthreads();
+  }
   const int64_t c0 = (int64_t)blockIdx.x * kScanChunk + (int64_t)threadIdx.x * kScanPerThread;
   uint32_t v[kScanPerThread];
   uint32_t s = 0;
@@ -111,7 +144,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __res
     s += v[k];
   }
   uint32_t total;
-  uint32_t run = partial[blockIdx.x] + block_exclusive_scan(s, s_warp, total);
+  uint32_t run = (FUSED ? s_base : partial[blockIdx.x]) + block_exclusive_scan(s, s_warp, total);
 #pragma unroll
   for (int k = 0; k < kScanPerThread; ++k) {
     if (c0 + k < n) out[c0 + k] = run;
@@ -119,10 +152,10 @@ __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __res
   }
 }
 
-// Stable scatter of one block's keys (and values) by digit: the rank of a key
-// among the block's keys of its digit counts the earlier rounds, the earlier
-// warps of its round and the earlier lanes of its warp.  vals_in == NULL
-// means the values are the input indices.
+// Stable scatter of one block's chunk by digit, kSortThreads keys per round:
+// the rank of a key among the block's keys of its digit counts the earlier
+// rounds, the earlier warps of its round and the earlier lanes of its warp.
+// vals_in == NULL means the values are the input indices.
 __global__ void __launch_bounds__(kSortThreads) radix_scatter(const uint32_t* __restrict__ keys_in,
                                                               const uint32_t* __restrict__ vals_in, int64_t N,
                                                               const uint32_t* __restrict__ n_dev,
@@ -130,19 +163,19 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter(const uint32_t* __
                                                               uint32_t* __restrict__ keys_out,
                                                               uint32_t* __restrict__ vals_out) {
   constexpr int kWarps = kSortThreads / 32;
-  __shared__ uint32_t base[kDigits];          // global position of this block's first key of each digit
+  __shared__ uint32_t base[kDigits];          // global position of this block's next key of each digit
   __shared__ uint32_t wcnt[kWarps][kDigits];  // per round: keys per (warp, digit), then their prefix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (n_dev) N = min(N, (int64_t)*n_dev);
+  int64_t lo, hi;
+  block_chunk(N, n_dev, lo, hi);
   base[tid] = offsets[(size_t)tid * gridDim.x + blockIdx.x];
   const uint32_t lt = (1u << lane) - 1u;
-  const int64_t t0 = (int64_t)blockIdx.x * kSortTile;
-  for (int r = 0; r < kSortPerThread; ++r) {
+  for (int64_t r0 = lo; r0 < hi; r0 += kSortThreads) {
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) wcnt[w][tid] = 0u;
     __syncthreads();
-    const int64_t i = t0 + r * kSortThreads + tid;
-    const bool valid = i < N;
+    const int64_t i = r0 + tid;
+    const bool valid = i < hi;
     uint32_t key = 0, val = 0, d = 0;
     if (valid) {
       key = keys_in[i];
@@ -175,54 +208,51 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter(const uint32_t* __
   }
 }
 
+// Scratch for an exclusive scan of n values.
+inline size_t exclusive_scan_scratch(int64_t n) { return align256((size_t)scan_chunks(n) * 4); }
 
-inline int64_t sort_blocks(int64_t N) { return (N + kSortTile - 1) / kSortTile; }
-inline int64_t scan_len(int64_t N) { return sort_blocks(N) * kDigits; }
-inline int64_t scan_chunks(int64_t N) { return (scan_len(N) + kScanChunk - 1) / kScanChunk; }
-inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+// out = exclusive scan of a[0..n) (n < 2^32 / 2, sums below 2^32).
+inline void exclusive_scan(const uint32_t* a, int64_t n, uint32_t* out, void* scratch, cudaStream_t s) {
+  const int chunks = (int)scan_chunks(n);
+  uint32_t* partial = static_cast<uint32_t*>(scratch);
+  scan_reduce<<<chunks, kScanThreads, 0, s>>>(a, n, partial);
+  if (chunks <= kFusedScanMaxChunks) {
+    scan_apply<true><<<chunks, kScanThreads, 0, s>>>(a, n, partial, out);
+  } else {
+    scan_partials<<<1, kScanThreads, 0, s>>>(partial, chunks);
+    scan_apply<false><<<chunks, kScanThreads, 0, s>>>(a, n, partial, out);
+  }
+}
 
 // Scratch for sorting up to N keys: the (digit, block) counts, their scan and
 // the scan's chunk partials.
 inline size_t scratch_bytes(int64_t N) {
-  return 2 * align256((size_t)scan_len(N) * 4) + align256((size_t)scan_chunks(N) * 4);
+  return 2 * align256((size_t)scan_len(N) * 4) + exclusive_scan_scratch(scan_len(N));
 }
 
 // Sorts (keys, vals) by bits [0, 8 * passes) of the keys, ping-ponging with
-// (keys_b, vals_b).  vals == nullptr on entry to the first pass means the
-// values are the input indices.  Returns true when the result is in
-// (keys, vals) (an even number of passes), false when in (keys_b, vals_b).
+// (keys_b, vals_b).  With vals_are_index the first pass takes the input
+// indices as values.  N is the capacity; n_dev (or N) the key count.
+// Returns true when the result is in (keys, vals) (an even number of
+// passes), false when in (keys_b, vals_b).
 inline bool sort_pairs(uint32_t* keys, uint32_t* vals, uint32_t* keys_b, uint32_t* vals_b, bool vals_are_index,
                        int64_t N, const uint32_t* n_dev, int passes, void* scratch, cudaStream_t s) {
   uint32_t* counts = static_cast<uint32_t*>(scratch);
   uint32_t* offsets = counts + align256((size_t)scan_len(N) * 4) / 4;
-  uint32_t* partial = offsets + align256((size_t)scan_len(N) * 4) / 4;
-  const int B = (int)sort_blocks(N);
+  void* scan_scratch = offsets + align256((size_t)scan_len(N) * 4) / 4;
+  const int B = sort_blocks(N);
   const int64_t len = scan_len(N);
-  const int chunks = (int)scan_chunks(N);
   uint32_t *ka = keys, *kb = keys_b, *va = vals, *vb = vals_b;
   for (int pass = 0; pass < passes; ++pass) {
     const int shift = 8 * pass;
     radix_histogram<<<B, kSortThreads, 0, s>>>(ka, N, n_dev, shift, counts);
-    scan_reduce<<<chunks, kScanThreads, 0, s>>>(counts, len, partial);
-    scan_partials<<<1, kScanThreads, 0, s>>>(partial, chunks);
-    scan_apply<<<chunks, kScanThreads, 0, s>>>(counts, len, partial, offsets);
+    exclusive_scan(counts, len, offsets, scan_scratch, s);
     radix_scatter<<<B, kSortThreads, 0, s>>>(ka, (pass == 0 && vals_are_index) ? nullptr : va, N, n_dev, shift,
                                              offsets, kb, vb);
     uint32_t* t = ka; ka = kb; kb = t;
     t = va; va = vb; vb = t;
   }
   return (passes % 2) == 0;
-}
-
-// Exclusive scan of n values (n <= 2^31) into out, with
-// exclusive_scan_scratch(n) bytes of scratch.
-inline size_t exclusive_scan_scratch(int64_t n) { return align256((size_t)((n + kScanChunk - 1) / kScanChunk) * 4); }
-inline void exclusive_scan(const uint32_t* a, int64_t n, uint32_t* out, void* scratch, cudaStream_t s) {
-  const int chunks = (int)((n + kScanChunk - 1) / kScanChunk);
-  uint32_t* partial = static_cast<uint32_t*>(scratch);
-  scan_reduce<<<chunks, kScanThreads, 0, s>>>(a, n, partial);
-  scan_partials<<<1, kScanThreads, 0, s>>>(partial, chunks);
-  scan_apply<<<chunks, kScanThreads, 0, s>>>(a, n, partial, out);
 }
 
 }  // namespace

@@ -14,11 +14,13 @@
 //     tile's list in depth order, ties by Gaussian index.
 //  4. tile_ranges_kernel marks each tile's run; rasterise_fwd runs one
 //     256-thread CTA per tile, stages batches of 256 Gaussians in shared
-//     memory and blends them into its 256 pixels, leaving early once every
-//     pixel's transmittance is spent.
+//     memory, skips per warp the Gaussians whose support box misses the
+//     warp's 8x4 block, and blends the rest into its pixels, leaving early
+//     once every pixel's transmittance is spent.
 // Backward: rasterise_bwd walks each pixel's list back to front, recovering
 // the transmittance by division, sums each Gaussian's screen-space gradient
-// over the warp's 32 pixels with shuffles and adds it with vector atomics;
+// over the warp's 32 pixels with a transposing shuffle reduction and adds it
+// with one atomic per value;
 // project_bwd_kernel chains it through the projection to the mean,
 // covariance, opacity and colour inputs.
 //
@@ -36,7 +38,6 @@ namespace spin4d {
 namespace {
 
 constexpr int kTileSide = 16;
-constexpr int kTilePixels = kTileSide * kTileSide;
 constexpr float kSupportD2 = 9.0f;    // 3-sigma ellipse
 
 struct Cam {
@@ -173,31 +174,62 @@ __device__ __forceinline__ void view_dir(const Cam& c, const float* __restrict__
   d[2] = v2 * inv;
 }
 
-__global__ void project_kernel(Cam c, Blend b, int64_t N, const float* __restrict__ means,
-                               const float* __restrict__ cov, const float* __restrict__ opacity,
-                               const float* __restrict__ colours, float4* __restrict__ conic_o,
-                               float2* __restrict__ xy, float4* __restrict__ rgb, uint2* __restrict__ rect,
-                               uint32_t* __restrict__ ntiles, uint32_t* __restrict__ dkey) {
-  for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
+constexpr int kProjThreads = 128;   // Gaussians per projection tile
+
+// Colour rows of DEG (3 (DEG+1)^2 floats; DEG -1: 3) of one tile of
+// Gaussians, staged through shared memory so global reads and writes are
+// coalesced; padded by one float so each thread's row sits in its own banks.
+template <int DEG>
+struct ColourTile {
+  static constexpr int kRow = DEG < 0 ? 3 : 3 * (DEG + 1) * (DEG + 1);
+  static constexpr int kPitch = kRow + 1;
+  static constexpr bool kStaged = DEG >= 0;
+};
+
+template <int DEG>
+__device__ __forceinline__ void stage_rows(const float* __restrict__ src, int64_t n0, int nb, float* sm) {
+  constexpr int R = ColourTile<DEG>::kRow, P = ColourTile<DEG>::kPitch;
+  const float* g = src + n0 * R;
+  for (int e = threadIdx.x; e < nb * R; e += kProjThreads) sm[(e / R) * P + e % R] = __ldg(g + e);
+}
+
+template <int DEG>
+__global__ void __launch_bounds__(kProjThreads) project_kernel(
+    Cam c, Blend b, int64_t N, const float* __restrict__ means, const float* __restrict__ cov,
+    const float* __restrict__ opacity, const float* __restrict__ colours, float4* __restrict__ conic_o,
+    float4* __restrict__ xy, float4* __restrict__ rgb, uint2* __restrict__ rect, uint32_t* __restrict__ ntiles,
+    uint32_t* __restrict__ dkey) {
+  using CT = ColourTile<DEG>;
+  constexpr int K = DEG < 0 ? 1 : (DEG + 1) * (DEG + 1);
+  __shared__ float s_col[CT::kStaged ? kProjThreads * CT::kPitch : 1];
+  for (int64_t n0 = (int64_t)blockIdx.x * kProjThreads; n0 < N; n0 += (int64_t)gridDim.x * kProjThreads) {
+    const int nb = (int)min((int64_t)kProjThreads, N - n0);
+    if (CT::kStaged) {
+      __syncthreads();
+      stage_rows<DEG>(colours, n0, nb, s_col);
+      __syncthreads();
+    }
+    const int64_t n = n0 + threadIdx.x;
+    if (threadIdx.x >= nb) continue;
     const float* mu = means + n * b.mean_stride;
     Proj p;
     project_one(c, b.lowpass, mu, cov + 6 * n, p);
     const float o = __ldg(opacity + n);
     uint32_t nt = 0, key = 0xFFFFFFFFu;
     float4 co = make_float4(0.f, 0.f, 0.f, 0.f), col = make_float4(0.f, 0.f, 0.f, 0.f);
-    float2 m = make_float2(0.f, 0.f);
+    float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
     uint2 r = make_uint2(0u, 0u);
     // a Gaussian whose opacity is below alpha_min is skipped at every pixel
     if (p.visible && o >= b.alpha_min) {
       const float inv = 1.0f / p.det;
       co = make_float4(p.C * inv, -p.B * inv, p.A * inv, o);
-      m = make_float2(p.mx, p.my);
       // support: d^2 <= 9 and o exp(-d^2/2) >= alpha_min; a slightly larger
       // box than the exact one keeps it a superset under fp32 rounding
       float r2 = kSupportD2;
       if (b.alpha_min > 0.0f) r2 = fminf(r2, 2.0f * (logf(o) - b.log_amin));
       r2 = r2 * 1.0001f + 0.01f;
       const float rx = sqrtf(r2 * p.A) + 0.01f, ry = sqrtf(r2 * p.C) + 0.01f;
+      m = make_float4(p.mx, p.my, rx, ry);
       // pixel i is sampled at i + 1/2
       const int i0 = max((int)ceilf(fmaxf(p.mx - rx - 0.5f, -1.0f)), 0);
       const int i1 = min((int)floorf(fminf(p.mx + rx - 0.5f, (float)c.W)), c.W - 1);
@@ -209,19 +241,20 @@ __global__ void project_kernel(Cam c, Blend b, int64_t N, const float* __restric
         r = make_uint2(tx0 | (tx1 << 16), ty0 | (ty1 << 16));
         key = __float_as_uint(p.xc[2]);   // z > z_near > 0
       }
-      if (b.sh_degree < 0) {
+      if (DEG < 0) {
         const float* cc = colours + 3 * n;
         col = make_float4(__ldg(cc), __ldg(cc + 1), __ldg(cc + 2), 0.f);
       } else {
         float d[3], nv, Y[16];
         view_dir(c, mu, d, nv);
-        sh_basis(b.sh_degree, d[0], d[1], d[2], Y);
-        const float* k = colours + (int64_t)3 * b.n_coef * n;
+        sh_basis(DEG, d[0], d[1], d[2], Y);
+        const float* k = s_col + threadIdx.x * CT::kPitch;
         float s0 = 0.f, s1 = 0.f, s2 = 0.f;
-        for (int i = 0; i < b.n_coef; ++i) {
-          s0 += Y[i] * __ldg(k + 3 * i);
-          s1 += Y[i] * __ldg(k + 3 * i + 1);
-          s2 += Y[i] * __ldg(k + 3 * i + 2);
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+          s0 += Y[i] * k[3 * i];
+          s1 += Y[i] * k[3 * i + 1];
+          s2 += Y[i] * k[3 * i + 2];
         }
         col = make_float4(fmaxf(s0, 0.f), fmaxf(s1, 0.f), fmaxf(s2, 0.f), 0.f);
       }
@@ -297,29 +330,94 @@ __device__ __forceinline__ float mahalanobis2(float4 co, float dx, float dy) {
   return __fmaf_rn(__fmul_rn(co.x, dx), dx, u);
 }
 
-__global__ void __launch_bounds__(kTilePixels) rasterise_fwd(Blend b, int W, int H, const uint2* __restrict__ ranges,
-                                                            const uint32_t* __restrict__ pair_id,
-                                                            const float4* __restrict__ conic_o,
-                                                            const float2* __restrict__ xy,
-                                                            const float4* __restrict__ rgb, float* __restrict__ image,
-                                                            float* __restrict__ final_T,
-                                                            uint32_t* __restrict__ n_contrib,
-                                                            float* __restrict__ final_T_out) {
-  __shared__ float4 s_co[kTilePixels];
-  __shared__ float2 s_xy[kTilePixels];
-  __shared__ float4 s_rgb[kTilePixels];
+// Rasterisers: one CTA of kRastThreads per 16x16 tile, one pixel a thread;
+// each warp owns an 8x4 block ((warp & 1, warp >> 1) in a 2x4 grid of
+// blocks), lane (lane & 7, lane >> 3) in it, and skips as a whole the
+// Gaussians whose support box misses its block.
+constexpr int kRastThreads = 256;
+
+struct TileGeom {
+  int px, py;                   // the lane's pixel
+  float wx0, wx1, wy0, wy1;     // the warp block's pixel centres, for the box test
+};
+
+__device__ __forceinline__ TileGeom tile_geom(const Blend& b) {
   const int tile = blockIdx.x;
   const int tx = tile % b.tiles_x, ty = tile / b.tiles_x;
-  const int px = tx * kTileSide + (threadIdx.x % kTileSide), py = ty * kTileSide + (threadIdx.x / kTileSide);
-  const bool inside = px < W && py < H;
-  const float fx = (float)px + 0.5f, fy = (float)py + 0.5f;
-  const uint2 range = ranges[tile];
-  float T = 1.0f, c0 = 0.f, c1 = 0.f, c2 = 0.f;
-  uint32_t last = 0;
-  bool done = !inside;
-  for (uint32_t base = range.x; base < range.y; base += kTilePixels) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int bx = tx * kTileSide + (warp & 1) * 8, by = ty * kTileSide + (warp >> 1) * 4;
+  TileGeom g;
+  g.px = bx + (lane & 7);
+  g.py = by + (lane >> 3);
+  g.wx0 = (float)bx + 0.5f;
+  g.wx1 = (float)bx + 7.5f;
+  g.wy0 = (float)by + 0.5f;
+  g.wy1 = (float)by + 3.5f;
+  return g;
+}
+
+// warp-uniform: the Gaussian's support box (centre m.xy, half-widths m.zw) misses the warp's block
+__device__ __forceinline__ bool box_misses(const float4& m, const TileGeom& g) {
+  return m.x + m.z < g.wx0 || m.x - m.z > g.wx1 || m.y + m.w < g.wy0 || m.y - m.w > g.wy1;
+}
+
+struct FwdPix {
+  float fx, fy, T, c0, c1, c2;
+  uint32_t last;
+  bool done;
+};
+
+__device__ __forceinline__ void blend_step(FwdPix& q, const float4& co, const float4& m, const float4& cc,
+                                           const Blend& b, uint32_t idx) {
+  const float dx = __fsub_rn(q.fx, m.x), dy = __fsub_rn(q.fy, m.y);
+  const float d2 = mahalanobis2(co, dx, dy);
+  if (d2 > kSupportD2) return;
+  const float a = fminf(b.alpha_max, __fmul_rn(co.w, __expf(__fmul_rn(-0.5f, d2))));
+  if (a < b.alpha_min) return;
+  const float Tn = __fmul_rn(q.T, __fsub_rn(1.0f, a));
+  if (Tn < b.t_stop) {
+    q.done = true;
+    return;
+  }
+  const float w = a * q.T;
+  q.c0 += cc.x * w;
+  q.c1 += cc.y * w;
+  q.c2 += cc.z * w;
+  q.T = Tn;
+  q.last = idx;
+}
+
+__device__ __forceinline__ void store_pixel(const FwdPix& q, int px, int py, int W, int H, const Blend& b,
+                                            float* __restrict__ image, float* __restrict__ final_T,
+                                            uint32_t* __restrict__ n_contrib, float* __restrict__ final_T_out) {
+  if (px >= W || py >= H) return;
+  const int64_t pix = (int64_t)py * W + px;
+  const int64_t plane = (int64_t)W * H;
+  image[pix] = q.c0 + q.T * b.bg[0];
+  image[plane + pix] = q.c1 + q.T * b.bg[1];
+  image[2 * plane + pix] = q.c2 + q.T * b.bg[2];
+  final_T[pix] = q.T;
+  n_contrib[pix] = q.last;
+  if (final_T_out) final_T_out[pix] = q.T;
+}
+
+__global__ void __launch_bounds__(kRastThreads) rasterise_fwd(Blend b, int W, int H, const uint2* __restrict__ ranges,
+                                                             const uint32_t* __restrict__ pair_id,
+                                                             const float4* __restrict__ conic_o,
+                                                             const float4* __restrict__ xy,
+                                                             const float4* __restrict__ rgb, float* __restrict__ image,
+                                                             float* __restrict__ final_T,
+                                                             uint32_t* __restrict__ n_contrib,
+                                                             float* __restrict__ final_T_out) {
+  __shared__ float4 s_co[kRastThreads];
+  __shared__ float4 s_xy[kRastThreads];
+  __shared__ float4 s_rgb[kRastThreads];
+  const TileGeom g = tile_geom(b);
+  FwdPix q{(float)g.px + 0.5f, (float)g.py + 0.5f, 1.0f, 0.f, 0.f, 0.f, 0u, !(g.px < W && g.py < H)};
+  const uint2 range = ranges[blockIdx.x];
+  for (uint32_t base = range.x; base < range.y; base += kRastThreads) {
     // also the barrier that frees the previous batch's shared memory
-    if (__syncthreads_count(done) == kTilePixels) break;
+    if (__syncthreads_count(q.done) == kRastThreads) break;
     const uint32_t i = base + threadIdx.x;
     if (i < range.y) {
       const uint32_t id = pair_id[i];
@@ -328,90 +426,118 @@ __global__ void __launch_bounds__(kTilePixels) rasterise_fwd(Blend b, int W, int
       s_rgb[threadIdx.x] = rgb[id];
     }
     __syncthreads();
-    const int cnt = (int)min((uint32_t)kTilePixels, range.y - base);
-    for (int j = 0; !done && j < cnt; ++j) {
-      const float4 co = s_co[j];
-      const float2 m = s_xy[j];
-      const float dx = __fsub_rn(fx, m.x), dy = __fsub_rn(fy, m.y);
-      const float d2 = mahalanobis2(co, dx, dy);
-      if (d2 > kSupportD2) continue;
-      const float a = fminf(b.alpha_max, __fmul_rn(co.w, __expf(__fmul_rn(-0.5f, d2))));
-      if (a < b.alpha_min) continue;
-      const float Tn = __fmul_rn(T, __fsub_rn(1.0f, a));
-      if (Tn < b.t_stop) {
-        done = true;
-        break;
-      }
-      const float w = a * T;
-      const float4 cc = s_rgb[j];
-      c0 += cc.x * w;
-      c1 += cc.y * w;
-      c2 += cc.z * w;
-      T = Tn;
-      last = base - range.x + j + 1;
+    const int cnt = (int)min((uint32_t)kRastThreads, range.y - base);
+    for (int j = 0; j < cnt && !q.done; ++j) {
+      const float4 m = s_xy[j];
+      if (box_misses(m, g)) continue;
+      blend_step(q, s_co[j], m, s_rgb[j], b, base - range.x + j + 1);
     }
   }
-  if (inside) {
-    const int64_t pix = (int64_t)py * W + px;
-    const int64_t plane = (int64_t)W * H;
-    image[pix] = c0 + T * b.bg[0];
-    image[plane + pix] = c1 + T * b.bg[1];
-    image[2 * plane + pix] = c2 + T * b.bg[2];
-    final_T[pix] = T;
-    n_contrib[pix] = last;
-    if (final_T_out) final_T_out[pix] = T;
-  }
+  store_pixel(q, g.px, g.py, W, H, b, image, final_T, n_contrib, final_T_out);
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
+// Sums each of v[0..15] over the warp with 16 shuffles instead of 80: every
+// level hands half of the values to the partner lane and keeps the other
+// half.  Lane L (and L ^ 1) ends with the total of value (L >> 1) & 15.
+__device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) {
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
-  return v;
+  for (int lvl = 0; lvl < 4; ++lvl) {
+    const int off = 16 >> lvl, half = 8 >> lvl;
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? v[i] : v[i + half];
+      const float keep = up ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
-// gacc per Gaussian: 3 float4 = (d xy.x, d xy.y, d conic.a, d conic.b),
-// (d conic.c, d opacity, d r, d g), (d b, -, -, -)
-__global__ void __launch_bounds__(kTilePixels) rasterise_bwd(Blend b, int W, int H, const uint2* __restrict__ ranges,
-                                                            const uint32_t* __restrict__ pair_id,
-                                                            const float4* __restrict__ conic_o,
-                                                            const float2* __restrict__ xy,
-                                                            const float4* __restrict__ rgb,
-                                                            const float* __restrict__ final_T,
-                                                            const uint32_t* __restrict__ n_contrib,
-                                                            const float* __restrict__ grad_image,
-                                                            float4* __restrict__ gacc) {
-  __shared__ float4 s_co[kTilePixels];
-  __shared__ float2 s_xy[kTilePixels];
-  __shared__ float4 s_rgb[kTilePixels];
-  __shared__ uint32_t s_id[kTilePixels];
-  __shared__ uint32_t s_max;
-  const int tile = blockIdx.x;
-  const int tx = tile % b.tiles_x, ty = tile / b.tiles_x;
-  const int px = tx * kTileSide + (threadIdx.x % kTileSide), py = ty * kTileSide + (threadIdx.x / kTileSide);
-  const bool inside = px < W && py < H;
-  const float fx = (float)px + 0.5f, fy = (float)py + 0.5f;
-  const uint2 range = ranges[tile];
-  const int64_t pix = (int64_t)py * W + px, plane = (int64_t)W * H;
-  float T = 1.0f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
-  uint32_t last = 0;
-  if (inside) {
-    T = final_T[pix];
-    last = n_contrib[pix];
-    g0 = grad_image[pix];
-    g1 = grad_image[plane + pix];
-    g2 = grad_image[2 * plane + pix];
+struct BwdPix {
+  float fx, fy, T, S, Tf, gbg, g0, g1, g2;
+  uint32_t last;
+};
+
+__device__ __forceinline__ BwdPix bwd_pixel(int px, int py, int W, int H, const Blend& b,
+                                            const float* __restrict__ final_T, const uint32_t* __restrict__ n_contrib,
+                                            const float* __restrict__ grad_image) {
+  BwdPix q{(float)px + 0.5f, (float)py + 0.5f, 1.0f, 0.f, 1.0f, 0.f, 0.f, 0.f, 0.f, 0u};
+  if (px < W && py < H) {
+    const int64_t pix = (int64_t)py * W + px, plane = (int64_t)W * H;
+    q.T = final_T[pix];
+    q.last = n_contrib[pix];
+    q.g0 = grad_image[pix];
+    q.g1 = grad_image[plane + pix];
+    q.g2 = grad_image[2 * plane + pix];
   }
-  const float Tf = T;
-  const float gbg = g0 * b.bg[0] + g1 * b.bg[1] + g2 * b.bg[2];
-  float S = 0.0f;   // sum over blended Gaussians behind: (g . c_k) a_k T_k
+  q.Tf = q.T;
+  q.gbg = q.g0 * b.bg[0] + q.g1 * b.bg[1] + q.g2 * b.bg[2];
+  return q;
+}
+
+// One pixel's share of Gaussian j's screen-space gradient, added to v:
+// (d x, d y, d conic a, b, c, d opacity, d r, d g, d b).  The decisions are
+// the forward's (same arithmetic); j beyond the pixel's last blended
+// Gaussian is skipped.  Returns whether the pixel blended Gaussian j.
+__device__ __forceinline__ bool grad_step(BwdPix& q, uint32_t jidx, const float4& co, const float4& m,
+                                          const float4& cc, const Blend& b, float (&v)[16]) {
+  if (jidx >= q.last) return false;
+  const float dx = __fsub_rn(q.fx, m.x), dy = __fsub_rn(q.fy, m.y);
+  const float d2 = mahalanobis2(co, dx, dy);
+  if (d2 > kSupportD2) return false;
+  const float G = __expf(__fmul_rn(-0.5f, d2));
+  const float raw = __fmul_rn(co.w, G);
+  const float a = fminf(b.alpha_max, raw);
+  if (a < b.alpha_min) return false;
+  const float oma = 1.0f - a;
+  const float Ti = q.T / oma;             // transmittance before Gaussian j
+  const float gc = q.g0 * cc.x + q.g1 * cc.y + q.g2 * cc.z;
+  float ga = Ti * gc - (q.S + q.Tf * q.gbg) / oma;
+  const float wgt = a * Ti;
+  v[6] += q.g0 * wgt;
+  v[7] += q.g1 * wgt;
+  v[8] += q.g2 * wgt;
+  q.S += gc * wgt;
+  q.T = Ti;
+  if (raw > b.alpha_max) ga = 0.0f;       // clamped: alpha does not move
+  v[5] += ga * G;
+  const float gd2 = -0.5f * ga * co.w * G;
+  v[2] += gd2 * dx * dx;
+  v[3] += gd2 * 2.0f * dx * dy;
+  v[4] += gd2 * dy * dy;
+  v[0] += -2.0f * gd2 * (co.x * dx + co.y * dy);
+  v[1] += -2.0f * gd2 * (co.y * dx + co.z * dy);
+  return true;
+}
+
+// gacc per Gaussian: 12 floats, the 9 of grad_step then 3 unused
+__global__ void __launch_bounds__(kRastThreads) rasterise_bwd(Blend b, int W, int H, const uint2* __restrict__ ranges,
+                                                             const uint32_t* __restrict__ pair_id,
+                                                             const float4* __restrict__ conic_o,
+                                                             const float4* __restrict__ xy,
+                                                             const float4* __restrict__ rgb,
+                                                             const float* __restrict__ final_T,
+                                                             const uint32_t* __restrict__ n_contrib,
+                                                             const float* __restrict__ grad_image,
+                                                             float4* __restrict__ gacc) {
+  __shared__ float4 s_co[kRastThreads];
+  __shared__ float4 s_xy[kRastThreads];
+  __shared__ float4 s_rgb[kRastThreads];
+  __shared__ uint32_t s_id[kRastThreads];
+  __shared__ uint32_t s_max;
+  const TileGeom g = tile_geom(b);
+  const int lane = threadIdx.x & 31;
+  BwdPix q = bwd_pixel(g.px, g.py, W, H, b, final_T, n_contrib, grad_image);
+  const uint2 range = ranges[blockIdx.x];
   if (threadIdx.x == 0) s_max = 0;
   __syncthreads();
-  atomicMax(&s_max, last);
+  atomicMax(&s_max, q.last);
   __syncthreads();
   const uint32_t max_last = s_max;
-  const int lane = threadIdx.x & 31;
+  const uint32_t warp_last = __reduce_max_sync(0xffffffffu, q.last);
   for (uint32_t hi = max_last; hi > 0;) {
-    const uint32_t lo = hi > (uint32_t)kTilePixels ? hi - kTilePixels : 0u;
+    const uint32_t lo = hi > (uint32_t)kRastThreads ? hi - kRastThreads : 0u;
     __syncthreads();
     const uint32_t i = lo + threadIdx.x;
     if (i < hi) {
@@ -423,145 +549,144 @@ __global__ void __launch_bounds__(kTilePixels) rasterise_bwd(Blend b, int W, int
     }
     __syncthreads();
     for (int j = (int)(hi - lo) - 1; j >= 0; --j) {
-      float v[9] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      bool hit = false;
-      if (lo + j < last) {
-        const float4 co = s_co[j];
-        const float2 m = s_xy[j];
-        const float dx = __fsub_rn(fx, m.x), dy = __fsub_rn(fy, m.y);
-        const float d2 = mahalanobis2(co, dx, dy);
-        if (d2 <= kSupportD2) {
-          const float G = __expf(__fmul_rn(-0.5f, d2));
-          const float raw = __fmul_rn(co.w, G);
-          const float a = fminf(b.alpha_max, raw);
-          if (a >= b.alpha_min) {
-            hit = true;
-            const float4 cc = s_rgb[j];
-            const float oma = 1.0f - a;
-            const float Ti = T / oma;
-            const float gc = g0 * cc.x + g1 * cc.y + g2 * cc.z;
-            float ga = Ti * gc - (S + Tf * gbg) / oma;
-            const float wgt = a * Ti;
-            v[6] = g0 * wgt;
-            v[7] = g1 * wgt;
-            v[8] = g2 * wgt;
-            S += gc * wgt;
-            T = Ti;
-            if (raw > b.alpha_max) ga = 0.0f;   // clamped: alpha does not move
-            v[5] = ga * G;
-            const float gd2 = -0.5f * ga * co.w * G;
-            v[2] = gd2 * dx * dx;
-            v[3] = gd2 * 2.0f * dx * dy;
-            v[4] = gd2 * dy * dy;
-            v[0] = -2.0f * gd2 * (co.x * dx + co.y * dy);
-            v[1] = -2.0f * gd2 * (co.y * dx + co.z * dy);
-          }
-        }
-      }
+      const uint32_t jidx = lo + j;
+      const float4 m = s_xy[j];
+      // warp-uniform: the support box misses the block, or no lane got this far
+      if (jidx >= warp_last || box_misses(m, g)) continue;
+      float v[16] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const bool hit = grad_step(q, jidx, s_co[j], m, s_rgb[j], b, v);
       if (__any_sync(0xffffffffu, hit)) {
-#pragma unroll
-        for (int k = 0; k < 9; ++k) v[k] = warp_sum(v[k]);
-        if (lane == 0) {
-          float4* gq = gacc + 3 * (int64_t)s_id[j];
-          atomicAdd(gq, make_float4(v[0], v[1], v[2], v[3]));
-          atomicAdd(gq + 1, make_float4(v[4], v[5], v[6], v[7]));
-          atomicAdd(&gq[2].x, v[8]);
-        }
+        const float total = warp_transpose_sum16(v, lane);
+        const int k = (lane >> 1) & 15;
+        if ((lane & 1) == 0 && k < 9) atomicAdd(reinterpret_cast<float*>(gacc + 3 * (int64_t)s_id[j]) + k, total);
       }
     }
     hi = lo;
   }
 }
 
-__global__ void project_bwd_kernel(Cam c, Blend b, int64_t N, const float* __restrict__ means,
-                                   const float* __restrict__ cov, const float* __restrict__ opacity,
-                                   const float* __restrict__ colours, const float4* __restrict__ gacc,
-                                   float* __restrict__ grad_means, float* __restrict__ grad_cov,
-                                   float* __restrict__ grad_opacity, float* __restrict__ grad_colours) {
-  for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
-    const float* mu = means + n * b.mean_stride;
+template <int DEG>
+__global__ void __launch_bounds__(kProjThreads) project_bwd_kernel(
+    Cam c, Blend b, int64_t N, const float* __restrict__ means, const float* __restrict__ cov,
+    const float* __restrict__ opacity, const float* __restrict__ colours, const float4* __restrict__ gacc,
+    float* __restrict__ grad_means, float* __restrict__ grad_cov, float* __restrict__ grad_opacity,
+    float* __restrict__ grad_colours) {
+  using CT = ColourTile<DEG>;
+  constexpr int K = DEG < 0 ? 1 : (DEG + 1) * (DEG + 1);
+  // the tile's SH rows; each thread overwrites its own row with its SH
+  // gradient, which is then added to grad_colours row-coalesced
+  __shared__ float s_col[CT::kStaged ? kProjThreads * CT::kPitch : 1];
+  for (int64_t n0 = (int64_t)blockIdx.x * kProjThreads; n0 < N; n0 += (int64_t)gridDim.x * kProjThreads) {
+    const int nb = (int)min((int64_t)kProjThreads, N - n0);
+    if (CT::kStaged) {
+      __syncthreads();
+      stage_rows<DEG>(colours, n0, nb, s_col);
+      __syncthreads();
+    }
+    const int64_t n = n0 + threadIdx.x;
+    bool live = threadIdx.x < nb;
     Proj p;
-    project_one(c, b.lowpass, mu, cov + 6 * n, p);
-    const float o = __ldg(opacity + n);
-    if (!(p.visible && o >= b.alpha_min)) continue;   // never blended: zero gradient
-    const float4 q0 = gacc[3 * n], q1 = gacc[3 * n + 1], q2 = gacc[3 * n + 2];
-    const float gx = q0.x, gy = q0.y, ga = q0.z, gb = q0.w, gc = q1.x;
-    const float grgb[3] = {q1.z, q1.w, q2.x};
-    if (grad_opacity) grad_opacity[n] += q1.y;
-    // conic (a, b, c) = (C, -B, A) / det, det = A C - B^2
-    const float A = p.A, B = p.B, C = p.C;
-    const float id = 1.0f / p.det, id2 = id * id;
-    const float gA = (-ga * C * C + gb * B * C - gc * B * B) * id2;
-    const float gB = (2.0f * ga * B * C - 2.0f * gc * (-A * B)) * id2 - gb * (id + 2.0f * B * B * id2);
-    const float gC = (-ga * B * B + gb * A * B - gc * A * A) * id2;
-    // G2 = [[gA, gB/2], [gB/2, gC]]: dL/dSigma = T^T G2 T
-    float U0[3], U1[3];
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      U0[k] = gA * p.T0[k] + 0.5f * gB * p.T1[k];
-      U1[k] = 0.5f * gB * p.T0[k] + gC * p.T1[k];
+    float o = 0.f;
+    const float* mu = means + n * b.mean_stride;
+    if (live) {
+      project_one(c, b.lowpass, mu, cov + 6 * n, p);
+      o = __ldg(opacity + n);
+      live = p.visible && o >= b.alpha_min;   // otherwise never blended: zero gradient
     }
-    if (grad_cov) {
-      float* gcv = grad_cov + 6 * n;
-      gcv[0] += p.T0[0] * U0[0] + p.T1[0] * U1[0];
-      gcv[1] += 2.0f * (p.T0[0] * U0[1] + p.T1[0] * U1[1]);
-      gcv[2] += 2.0f * (p.T0[0] * U0[2] + p.T1[0] * U1[2]);
-      gcv[3] += p.T0[1] * U0[1] + p.T1[1] * U1[1];
-      gcv[4] += 2.0f * (p.T0[1] * U0[2] + p.T1[1] * U1[2]);
-      gcv[5] += p.T0[2] * U0[2] + p.T1[2] * U1[2];
-    }
-    if (!grad_means && !grad_colours) continue;
-    // dL/d(J W) = 2 G2 (J W) Sigma; dL/dJ = that times W^T
-    float gT0[3], gT1[3];
+    float* krow = s_col + threadIdx.x * CT::kPitch;
+    if (live) {
+      const float4 q0 = gacc[3 * n], q1 = gacc[3 * n + 1], q2 = gacc[3 * n + 2];
+      const float gx = q0.x, gy = q0.y, ga = q0.z, gb = q0.w, gc = q1.x;
+      const float grgb[3] = {q1.z, q1.w, q2.x};
+      if (grad_opacity) grad_opacity[n] += q1.y;
+      // conic (a, b, c) = (C, -B, A) / det, det = A C - B^2
+      const float A = p.A, B = p.B, C = p.C;
+      const float id = 1.0f / p.det, id2 = id * id;
+      const float gA = (-ga * C * C + gb * B * C - gc * B * B) * id2;
+      const float gB = (2.0f * ga * B * C + 2.0f * gc * A * B) * id2 - gb * (id + 2.0f * B * B * id2);
+      const float gC = (-ga * B * B + gb * A * B - gc * A * A) * id2;
+      // G2 = [[gA, gB/2], [gB/2, gC]]: dL/dSigma = T^T G2 T
+      float U0[3], U1[3];
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      gT0[k] = 2.0f * (gA * p.M0[k] + 0.5f * gB * p.M1[k]);
-      gT1[k] = 2.0f * (0.5f * gB * p.M0[k] + gC * p.M1[k]);
-    }
-    const float gJ00 = gT0[0] * c.R[0] + gT0[1] * c.R[1] + gT0[2] * c.R[2];
-    const float gJ02 = gT0[0] * c.R[6] + gT0[1] * c.R[7] + gT0[2] * c.R[8];
-    const float gJ11 = gT1[0] * c.R[3] + gT1[1] * c.R[4] + gT1[2] * c.R[5];
-    const float gJ12 = gT1[0] * c.R[6] + gT1[1] * c.R[7] + gT1[2] * c.R[8];
-    const float x = p.xc[0], y = p.xc[1], z = p.xc[2];
-    const float iz = 1.0f / z, iz2 = iz * iz, iz3 = iz2 * iz;
-    float gxc[3];
-    gxc[0] = -c.fx * iz2 * gJ02 + gx * c.fx * iz;
-    gxc[1] = -c.fy * iz2 * gJ12 + gy * c.fy * iz;
-    gxc[2] = -c.fx * iz2 * gJ00 + 2.0f * c.fx * x * iz3 * gJ02 - c.fy * iz2 * gJ11 + 2.0f * c.fy * y * iz3 * gJ12 -
-             gx * c.fx * x * iz2 - gy * c.fy * y * iz2;
-    float gmu[3];
-#pragma unroll
-    for (int k = 0; k < 3; ++k) gmu[k] = c.R[k] * gxc[0] + c.R[3 + k] * gxc[1] + c.R[6 + k] * gxc[2];
-    if (b.sh_degree < 0) {
-      if (grad_colours)
-        for (int ch = 0; ch < 3; ++ch) grad_colours[3 * n + ch] += grgb[ch];
-    } else {
-      float d[3], nv, Y[16];
-      view_dir(c, mu, d, nv);
-      sh_basis(b.sh_degree, d[0], d[1], d[2], Y);
-      const float* k = colours + (int64_t)3 * b.n_coef * n;
-      float pre[3] = {0.f, 0.f, 0.f};
-      for (int i = 0; i < b.n_coef; ++i)
-        for (int ch = 0; ch < 3; ++ch) pre[ch] += Y[i] * __ldg(k + 3 * i + ch);
-      float gp[3];
-      for (int ch = 0; ch < 3; ++ch) gp[ch] = pre[ch] >= 0.0f ? grgb[ch] : 0.0f;
-      float gd[3] = {0.f, 0.f, 0.f};
-      float* gk = grad_colours ? grad_colours + (int64_t)3 * b.n_coef * n : nullptr;
-      for (int i = 0; i < b.n_coef; ++i) {
-        float w = 0.f;
-        for (int ch = 0; ch < 3; ++ch) {
-          if (gk) gk[3 * i + ch] += Y[i] * gp[ch];
-          w += gp[ch] * __ldg(k + 3 * i + ch);
-        }
-        sh_grad_acc(i, w, d[0], d[1], d[2], gd);
+      for (int k = 0; k < 3; ++k) {
+        U0[k] = gA * p.T0[k] + 0.5f * gB * p.T1[k];
+        U1[k] = 0.5f * gB * p.T0[k] + gC * p.T1[k];
       }
-      // d = v / |v|: dL/dv = (I - d d^T) dL/dd / |v|
-      const float dot = gd[0] * d[0] + gd[1] * d[1] + gd[2] * d[2];
-      const float inv = 1.0f / fmaxf(nv, 1e-30f);
-      for (int k2 = 0; k2 < 3; ++k2) gmu[k2] += (gd[k2] - d[k2] * dot) * inv;
+      if (grad_cov) {
+        float* gcv = grad_cov + 6 * n;
+        gcv[0] += p.T0[0] * U0[0] + p.T1[0] * U1[0];
+        gcv[1] += 2.0f * (p.T0[0] * U0[1] + p.T1[0] * U1[1]);
+        gcv[2] += 2.0f * (p.T0[0] * U0[2] + p.T1[0] * U1[2]);
+        gcv[3] += p.T0[1] * U0[1] + p.T1[1] * U1[1];
+        gcv[4] += 2.0f * (p.T0[1] * U0[2] + p.T1[1] * U1[2]);
+        gcv[5] += p.T0[2] * U0[2] + p.T1[2] * U1[2];
+      }
+      // dL/d(J W) = 2 G2 (J W) Sigma; dL/dJ = that times W^T
+      float gT0[3], gT1[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        gT0[k] = 2.0f * (gA * p.M0[k] + 0.5f * gB * p.M1[k]);
+        gT1[k] = 2.0f * (0.5f * gB * p.M0[k] + gC * p.M1[k]);
+      }
+      const float gJ00 = gT0[0] * c.R[0] + gT0[1] * c.R[1] + gT0[2] * c.R[2];
+      const float gJ02 = gT0[0] * c.R[6] + gT0[1] * c.R[7] + gT0[2] * c.R[8];
+      const float gJ11 = gT1[0] * c.R[3] + gT1[1] * c.R[4] + gT1[2] * c.R[5];
+      const float gJ12 = gT1[0] * c.R[6] + gT1[1] * c.R[7] + gT1[2] * c.R[8];
+      const float x = p.xc[0], y = p.xc[1], z = p.xc[2];
+      const float iz = 1.0f / z, iz2 = iz * iz, iz3 = iz2 * iz;
+      float gxc[3];
+      gxc[0] = -c.fx * iz2 * gJ02 + gx * c.fx * iz;
+      gxc[1] = -c.fy * iz2 * gJ12 + gy * c.fy * iz;
+      gxc[2] = -c.fx * iz2 * gJ00 + 2.0f * c.fx * x * iz3 * gJ02 - c.fy * iz2 * gJ11 + 2.0f * c.fy * y * iz3 * gJ12 -
+               gx * c.fx * x * iz2 - gy * c.fy * y * iz2;
+      float gmu[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) gmu[k] = c.R[k] * gxc[0] + c.R[3 + k] * gxc[1] + c.R[6 + k] * gxc[2];
+      if (DEG < 0) {
+        if (grad_colours)
+          for (int ch = 0; ch < 3; ++ch) grad_colours[3 * n + ch] += grgb[ch];
+      } else {
+        float d[3], nv, Y[16];
+        view_dir(c, mu, d, nv);
+        sh_basis(DEG, d[0], d[1], d[2], Y);
+        float pre[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < K; ++i)
+#pragma unroll
+          for (int ch = 0; ch < 3; ++ch) pre[ch] += Y[i] * krow[3 * i + ch];
+        float gp[3];
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) gp[ch] = pre[ch] >= 0.0f ? grgb[ch] : 0.0f;
+        float gd[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+          float w = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < 3; ++ch) {
+            w += gp[ch] * krow[3 * i + ch];
+            krow[3 * i + ch] = Y[i] * gp[ch];   // this row now holds the SH gradient
+          }
+          sh_grad_acc(i, w, d[0], d[1], d[2], gd);
+        }
+        // d = v / |v|: dL/dv = (I - d d^T) dL/dd / |v|
+        const float dot = gd[0] * d[0] + gd[1] * d[1] + gd[2] * d[2];
+        const float inv = 1.0f / fmaxf(nv, 1e-30f);
+#pragma unroll
+        for (int k2 = 0; k2 < 3; ++k2) gmu[k2] += (gd[k2] - d[k2] * dot) * inv;
+      }
+      if (grad_means)
+#pragma unroll
+        for (int k2 = 0; k2 < 3; ++k2) grad_means[3 * n + k2] += gmu[k2];
+    } else if (CT::kStaged && threadIdx.x < nb) {
+#pragma unroll
+      for (int i = 0; i < CT::kRow; ++i) krow[i] = 0.0f;
     }
-    if (grad_means)
-      for (int k2 = 0; k2 < 3; ++k2) grad_means[3 * n + k2] += gmu[k2];
+    if (CT::kStaged && grad_colours) {
+      __syncthreads();
+      constexpr int R = CT::kRow, P = CT::kPitch;
+      float* g = grad_colours + n0 * R;
+      for (int e = threadIdx.x; e < nb * R; e += kProjThreads) g[e] += s_col[(e / R) * P + e % R];
+    }
   }
 }
 
@@ -588,7 +713,7 @@ StateLayout state_layout(int64_t N, int W, int H, int64_t P) {
   const size_t tiles = (size_t)tiles_of(W) * tiles_of(H);
   L.header = take(256);
   L.conic_o = take(n * 16);
-  L.xy = take(n * 8);
+  L.xy = take(n * 16);
   L.rgb = take(n * 16);
   L.rect = take(n * 8);
   L.ntiles = take(n * 4);
@@ -717,10 +842,20 @@ extern "C" int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_d
   uint32_t* pair_id = at<uint32_t>(state, L.pair_id);
   if (N > 0) {
     const int blocks = persistent_blocks((N + 255) / 256, 8);
-    project_kernel<<<blocks, 256, 0, s>>>(c, b, N, means, cov, opacity, colours, at<float4>(state, L.conic_o),
-                                          at<float2>(state, L.xy), at<float4>(state, L.rgb),
-                                          at<uint2>(state, L.rect), at<uint32_t>(state, L.ntiles),
-                                          at<uint32_t>(state, L.dkey));
+    const int pblocks = persistent_blocks((N + kProjThreads - 1) / kProjThreads, 8);
+#define SPIN4D_PROJECT(DEG)                                                                                    \
+  project_kernel<DEG><<<pblocks, kProjThreads, 0, s>>>(c, b, N, means, cov, opacity, colours,                \
+                                                       at<float4>(state, L.conic_o), at<float4>(state, L.xy), \
+                                                       at<float4>(state, L.rgb), at<uint2>(state, L.rect),    \
+                                                       at<uint32_t>(state, L.ntiles), at<uint32_t>(state, L.dkey))
+    switch (b.sh_degree) {
+      case -1: SPIN4D_PROJECT(-1); break;
+      case 0: SPIN4D_PROJECT(0); break;
+      case 1: SPIN4D_PROJECT(1); break;
+      case 2: SPIN4D_PROJECT(2); break;
+      default: SPIN4D_PROJECT(3); break;
+    }
+#undef SPIN4D_PROJECT
     SPIN4D_CHECK(launch_status());
     uint32_t* dkey = at<uint32_t>(state, L.dkey);
     uint32_t* dperm = at<uint32_t>(state, L.dperm);
@@ -749,8 +884,8 @@ extern "C" int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_d
           pair_tile, header, max_pairs, (uint32_t)n_tiles, at<uint2>(state, L.ranges));
     SPIN4D_CHECK(launch_status());
   }
-  rasterise_fwd<<<n_tiles, kTilePixels, 0, s>>>(b, c.W, c.H, at<uint2>(state, L.ranges), pair_id,
-                                                at<float4>(state, L.conic_o), at<float2>(state, L.xy),
+  rasterise_fwd<<<n_tiles, kRastThreads, 0, s>>>(b, c.W, c.H, at<uint2>(state, L.ranges), pair_id,
+                                                at<float4>(state, L.conic_o), at<float4>(state, L.xy),
                                                 at<float4>(state, L.rgb), image, at<float>(state, L.final_T),
                                                 at<uint32_t>(state, L.n_contrib), final_T);
   return launch_status();
@@ -779,12 +914,22 @@ extern "C" int spin4d_render_bwd(const spin4d_camera* cam, const spin4d_render_d
   const int passes = tile_sort_passes(n_tiles);
   const bool in_b = passes > 0 && max_pairs > 0 && (passes % 2) == 1;
   const uint32_t* pair_id = at<uint32_t>(state, in_b ? L.pair_id_b : L.pair_id);
-  rasterise_bwd<<<n_tiles, kTilePixels, 0, s>>>(b, c.W, c.H, at<uint2>(state, L.ranges), pair_id,
-                                                at<float4>(state, L.conic_o), at<float2>(state, L.xy),
+  rasterise_bwd<<<n_tiles, kRastThreads, 0, s>>>(b, c.W, c.H, at<uint2>(state, L.ranges), pair_id,
+                                                at<float4>(state, L.conic_o), at<float4>(state, L.xy),
                                                 at<float4>(state, L.rgb), at<float>(state, L.final_T),
                                                 at<uint32_t>(state, L.n_contrib), grad_image, gacc);
   SPIN4D_CHECK(launch_status());
-  project_bwd_kernel<<<persistent_blocks((N + 255) / 256, 8), 256, 0, s>>>(
-      c, b, N, means, cov, opacity, colours, gacc, grad_means, grad_cov, grad_opacity, grad_colours);
+  const int pblocks = persistent_blocks((N + kProjThreads - 1) / kProjThreads, 8);
+#define SPIN4D_PROJECT_BWD(DEG)                                                                                  \
+  project_bwd_kernel<DEG><<<pblocks, kProjThreads, 0, s>>>(c, b, N, means, cov, opacity, colours, gacc, grad_means, \
+                                                           grad_cov, grad_opacity, grad_colours)
+  switch (b.sh_degree) {
+    case -1: SPIN4D_PROJECT_BWD(-1); break;
+    case 0: SPIN4D_PROJECT_BWD(0); break;
+    case 1: SPIN4D_PROJECT_BWD(1); break;
+    case 2: SPIN4D_PROJECT_BWD(2); break;
+    default: SPIN4D_PROJECT_BWD(3); break;
+  }
+#undef SPIN4D_PROJECT_BWD
   return launch_status();
 }

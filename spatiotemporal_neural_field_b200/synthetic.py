@@ -456,20 +456,28 @@ def random_spd(n: int, sigmas: np.ndarray, g: np.random.Generator) -> np.ndarray
 
 
 def render_scene(n: int, seed: int = 0, positions: Optional[np.ndarray] = None, sh_degree: int = 3,
-                 scale_factor: float = 0.5, opacity_lo: float = 0.05) -> Dict[str, np.ndarray]:
+                 scale_factor: float = 1.0, opacity_lo: float = 0.05) -> Dict[str, np.ndarray]:
     """Attributes shaped like a trained scene: per-axis standard deviations
-    log-normal around ``scale_factor`` x the mean spacing (8/n)^(1/3) of n
-    points in the [-1,1]^3 box, random orientations, opacity = sigmoid(N(0, 2^2))
-    floored at ``opacity_lo``, SH coefficients with the degree-0 term
-    U(0.4, 3.2) and the higher ones N(0, 0.1^2) (sh_degree -1: RGB U(0.05, 1)).
-    Positions default to frame 75 of the sports scene."""
+    log-normal (sigma 0.4) around ``scale_factor`` x the mean distance to the
+    3 nearest neighbours (the initial scale 3D Gaussian Splatting gives each
+    point, so dense regions get small Gaussians), random orientations,
+    opacity = sigmoid(N(0, 2^2)) floored at ``opacity_lo``, SH coefficients
+    with the degree-0 term U(0.4, 3.2) and the higher ones N(0, 0.1^2)
+    (sh_degree -1: RGB U(0.05, 1)).  Positions default to frame 75 of the
+    sports scene."""
+    from scipy.spatial import cKDTree
     g = rng(seed + 909)
     if positions is None:
         positions = sports_scene(n, seed).frame(75)
     mu = np.ascontiguousarray(positions[:, :3], np.float32)
     n = mu.shape[0]
-    s0 = scale_factor * (8.0 / max(n, 1)) ** (1.0 / 3.0)
-    sig = s0 * np.exp(g.normal(0.0, 0.4, size=(n, 3)))
+    k = min(3, n - 1)
+    if k >= 1:
+        dist, _ = cKDTree(mu.astype(np.float64)).query(mu.astype(np.float64), k=k + 1)
+        s0 = scale_factor * np.maximum(dist[:, 1:].mean(axis=1), 1e-6)
+    else:
+        s0 = np.full(n, scale_factor * 0.1)
+    sig = s0[:, None] * np.exp(g.normal(0.0, 0.4, size=(n, 3)))
     cov = random_spd(n, sig, g).astype(np.float32)
     op = 1.0 / (1.0 + np.exp(-g.normal(0.0, 2.0, size=n)))
     op = np.maximum(op, opacity_lo).astype(np.float32)

@@ -88,15 +88,32 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   return before + x - v;
 }
 
+// A scan chunk moves between global and shared memory with coalesced
+// accesses (thread t touches t, t + kScanThreads, ...); each thread then
+// works on its kScanPerThread consecutive values in shared memory, read with
+// a padded stride so the eight-apart rows fall in different banks.
+__device__ __forceinline__ int padded(int e) { return e + (e >> 5); }
+constexpr int kScanShared = kScanChunk + kScanChunk / 32;
+
+__device__ __forceinline__ void load_chunk(const uint32_t* __restrict__ a, int64_t n, uint32_t* sm) {
+  const int64_t c0 = (int64_t)blockIdx.x * kScanChunk;
+#pragma unroll
+  for (int k = 0; k < kScanPerThread; ++k) {
+    const int e = k * kScanThreads + threadIdx.x;
+    sm[padded(e)] = c0 + e < n ? a[c0 + e] : 0u;
+  }
+  __syncthreads();
+}
+
 // Scan step 1: partial[c] = sum of chunk c of a.
 __global__ void __launch_bounds__(kScanThreads) scan_reduce(const uint32_t* __restrict__ a, int64_t n,
                                                             uint32_t* __restrict__ partial) {
   __shared__ uint32_t s_warp[32];
-  const int64_t c0 = (int64_t)blockIdx.x * kScanChunk + (int64_t)threadIdx.x * kScanPerThread;
+  __shared__ uint32_t sm[kScanShared];
+  load_chunk(a, n, sm);
   uint32_t s = 0;
 #pragma unroll
-  for (int k = 0; k < kScanPerThread; ++k)
-    if (c0 + k < n) s += a[c0 + k];
+  for (int k = 0; k < kScanPerThread; ++k) s += sm[padded(threadIdx.x * kScanPerThread + k)];
   uint32_t total;
   block_exclusive_scan(s, s_warp, total);
   if (threadIdx.x == 0) partial[blockIdx.x] = total;
@@ -125,6 +142,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __res
                                                            uint32_t* __restrict__ out) {
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_base;
+  __shared__ uint32_t sm[kScanShared];
   if (FUSED) {
     if (threadIdx.x < 32) {
       uint32_t acc = 0;
@@ -133,22 +151,28 @@ __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __res
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (threadIdx.x == 0) s_base = acc;
     }
-    __syncthreads();
   }
-  const int64_t c0 = (int64_t)blockIdx.x * kScanChunk + (int64_t)threadIdx.x * kScanPerThread;
+  load_chunk(a, n, sm);   // its barrier also publishes s_base
   uint32_t v[kScanPerThread];
   uint32_t s = 0;
 #pragma unroll
   for (int k = 0; k < kScanPerThread; ++k) {
-    v[k] = c0 + k < n ? a[c0 + k] : 0u;
+    v[k] = sm[padded(threadIdx.x * kScanPerThread + k)];
     s += v[k];
   }
   uint32_t total;
   uint32_t run = (FUSED ? s_base : partial[blockIdx.x]) + block_exclusive_scan(s, s_warp, total);
 #pragma unroll
   for (int k = 0; k < kScanPerThread; ++k) {
-    if (c0 + k < n) out[c0 + k] = run;
+    sm[padded(threadIdx.x * kScanPerThread + k)] = run;
     run += v[k];
+  }
+  __syncthreads();
+  const int64_t c0 = (int64_t)blockIdx.x * kScanChunk;
+#pragma unroll
+  for (int k = 0; k < kScanPerThread; ++k) {
+    const int e = k * kScanThreads + threadIdx.x;
+    if (c0 + e < n) out[c0 + e] = sm[padded(e)];
   }
 }
 

@@ -27,6 +27,7 @@ namespace {
 
 constexpr int kHeadsBlock = 64;      // forward: positions per block
 constexpr int kHeadsBwdBlock = 32;   // backward: positions per block
+constexpr int kHeadsBwdPitch = kHeadsBwdBlock + 1;
 constexpr int kMaxDim = 64;          // in_dim, hidden and sh_dim limit of the shared-memory layout
 
 struct HeadsParams {
@@ -169,21 +170,41 @@ __global__ void __launch_bounds__(kHeadsBlock * kParts) heads_fwd_kernel(GridPar
 
 __device__ __forceinline__ float g0(const float* p, int64_t i) { return p ? __ldg(p + i) : 0.0f; }
 
-// slot[p] += sum over the block's positions of d[o][t] * x[k][t] (weights)
-// and d[o][t] (biases) of one layer, as fp32 reductions (no load to wait
-// for); each thread owns fixed parameters, so each slot element's adds come
-// from one thread in program order and the sum does not depend on scheduling.
-__device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out, int n_in, float* slot, int blk) {
-  const int nW = n_out * n_in;
-  for (int p = threadIdx.x; p < nW + n_out; p += blockDim.x) {
-    float s = 0.0f;
-    if (p < nW) {
-      const int o = p / n_in, k = p - o * n_in;
-      for (int t = 0; t < blk; ++t) s = fmaf(d[o * blk + t], x[k * blk + t], s);
-    } else {
-      for (int t = 0; t < blk; ++t) s += d[(p - nW) * blk + t];
+// slot += the block's weight gradient of one layer: W[o][k] += sum_t d[o][t]
+// x[k][t] and b[o] += sum_t d[o][t], as fp32 reductions (no load to wait
+// for).  Activations are [feature][position] with an odd pitch, so lanes on
+// consecutive columns k read different banks; each thread keeps 8 rows of
+// one column in registers (the d reads are warp-wide broadcasts).  The task
+// of every slot element is fixed, so its adds come from one thread in program
+// order and the sum does not depend on scheduling.
+__device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out, int n_in, float* slot, int pitch,
+                                      int npos) {
+  constexpr int RO = 8;
+  const int ob = (n_out + RO - 1) / RO;
+  const int kb = (n_in + 31) / 32 * 32;   // columns padded to whole warps: a warp shares its row block
+  for (int task = threadIdx.x; task < ob * kb; task += blockDim.x) {
+    const int k = task % kb, o0 = (task / kb) * RO;
+    if (k >= n_in) continue;
+    float acc[RO];
+#pragma unroll
+    for (int i = 0; i < RO; ++i) acc[i] = 0.0f;
+    const float* dr[RO];
+#pragma unroll
+    for (int i = 0; i < RO; ++i) dr[i] = d + min(o0 + i, n_out - 1) * pitch;
+    const float* xk = x + k * pitch;
+    for (int t = 0; t < npos; ++t) {
+      const float xv = xk[t];
+#pragma unroll
+      for (int i = 0; i < RO; ++i) acc[i] = fmaf(dr[i][t], xv, acc[i]);
     }
-    atomicAdd(slot + p, s);
+#pragma unroll
+    for (int i = 0; i < RO; ++i)
+      if (o0 + i < n_out) atomicAdd(slot + (o0 + i) * n_in + k, acc[i]);
+  }
+  for (int o = threadIdx.x; o < n_out; o += blockDim.x) {
+    float sb = 0.0f;
+    for (int t = 0; t < npos; ++t) sb += d[o * pitch + t];
+    atomicAdd(slot + n_out * n_in + o, sb);
   }
 }
 
@@ -206,15 +227,16 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
     const W* __restrict__ weights, const float* __restrict__ latent, HeadsGrads go, float* __restrict__ grad_tables,
     float* __restrict__ ws, int n_params) {
   constexpr int B = kHeadsBwdBlock;
+  constexpr int P = kHeadsBwdPitch;    // odd: a warp's column reads hit 32 different banks
   extern __shared__ float sm[];
-  float* z = sm;                       // [IN][B]
-  float* p1 = z + kMaxDim * B;         // pre-activations of layer 1, later d(pre 1)
-  float* h1 = p1 + kMaxDim * B;
-  float* p2 = h1 + kMaxDim * B;        // pre-activations of layer 2, later d(pre 2)
-  float* h2 = p2 + kMaxDim * B;
-  float* dy = h2 + kMaxDim * B;        // one head's output adjoint
-  float* dz = dy + kMaxDim * B;
-  float* dattr = dz + kMaxDim * B;     // [8][B]: adjoint of raw scale, rot, opacity
+  float* z = sm;                       // [IN][P]
+  float* p1 = z + kMaxDim * P;         // pre-activations of layer 1, later d(pre 1)
+  float* h1 = p1 + kMaxDim * P;
+  float* p2 = h1 + kMaxDim * P;        // pre-activations of layer 2, later d(pre 2)
+  float* h2 = p2 + kMaxDim * P;
+  float* dy = h2 + kMaxDim * P;        // one head's output adjoint
+  float* dz = dy + kMaxDim * P;
+  float* dattr = dz + kMaxDim * P;     // [8][P]: adjoint of raw scale, rot, opacity
   const int col = threadIdx.x % B, part = threadIdx.x / B;
   const int IN = hp.in_dim, H = hp.hidden;
   float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
@@ -226,13 +248,13 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
     float xt[4] = {0.f, 0.f, 0.f, 0.f};
     if (valid) normalise_position(pos[n], g, xt);
     if (valid && latent) {
-      for (int k = part; k < IN; k += kParts) z[k * B + col] = __ldg(latent + n * IN + k);
+      for (int k = part; k < IN; k += kParts) z[k * P + col] = __ldg(latent + n * IN + k);
     } else if (valid) {
-      gather_z<T, F>(xt, g, tables, z, B, col, part, nullptr, n, IN);
+      gather_z<T, F>(xt, g, tables, z, P, col, part, nullptr, n, IN);
     } else {
-      for (int k = part; k < IN; k += kParts) z[k * B + col] = 0.0f;
+      for (int k = part; k < IN; k += kParts) z[k * P + col] = 0.0f;
     }
-    for (int k = part; k < IN; k += kParts) dz[k * B + col] = 0.0f;
+    for (int k = part; k < IN; k += kParts) dz[k * P + col] = 0.0f;
     __syncthreads();
     // raw outputs of the scale, rotation and opacity heads, then (part 0) the
     // adjoint of Eq. 11 and Eq. 2
@@ -240,17 +262,17 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
     for (int h = 0; h < 4; ++h) {
       if (h == 2) continue;
       const W* w = weights + hp.off[h];
-      layer<W>(w, H, IN, z, h1, nullptr, true, B, col, part);
+      layer<W>(w, H, IN, z, h1, nullptr, true, P, col, part);
       __syncthreads();
       w += H * IN + H;
-      layer<W>(w, H, H, h1, h2, nullptr, true, B, col, part);
+      layer<W>(w, H, H, h1, h2, nullptr, true, P, col, part);
       __syncthreads();
       w += H * H + H;
-      layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, B, col, part);
+      layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, P, col, part);
       __syncthreads();
       if (part == 0) {
         const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[i * B + col];
+        for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[i * P + col];
       }
       __syncthreads();
     }
@@ -275,7 +297,7 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
         d[7] = g0(go.opacity, n) * o * (1.0f - o);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dattr[i * B + col] = d[i];
+      for (int i = 0; i < 8; ++i) dattr[i * P + col] = d[i];
     }
     __syncthreads();
     // ---- per head: forward with pre-activations, then the three layers' gradients ----
@@ -287,32 +309,32 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
       float* s1 = slot + hp.off[h];
       float* s2 = s1 + H * IN + H;
       float* s3 = s2 + H * H + H;
-      layer<W>(w1, H, IN, z, h1, p1, true, B, col, part);
+      layer<W>(w1, H, IN, z, h1, p1, true, P, col, part);
       __syncthreads();
-      layer<W>(w2, H, H, h1, h2, p2, true, B, col, part);
+      layer<W>(w2, H, H, h1, h2, p2, true, P, col, part);
       if (h == 2) {
         for (int i = part; i < rows; i += kParts)
-          dy[i * B + col] = valid ? g0(go.sh, (int64_t)hp.sh_dim * n + i) : 0.0f;
+          dy[i * P + col] = valid ? g0(go.sh, (int64_t)hp.sh_dim * n + i) : 0.0f;
       } else {
         const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = part; i < rows; i += kParts) dy[i * B + col] = dattr[(base + i) * B + col];
+        for (int i = part; i < rows; i += kParts) dy[i * P + col] = dattr[(base + i) * P + col];
       }
       __syncthreads();
-      wgrad(dy, h2, rows, H, s3, B);
-      dgrad<W>(w3, rows, H, dy, p2, p2, false, B, col, part);      // p2 <- d(pre 2)
+      wgrad(dy, h2, rows, H, s3, P, B);
+      dgrad<W>(w3, rows, H, dy, p2, p2, false, P, col, part);      // p2 <- d(pre 2)
       __syncthreads();
-      wgrad(p2, h1, H, H, s2, B);
-      dgrad<W>(w2, H, H, p2, p1, p1, false, B, col, part);         // p1 <- d(pre 1)
+      wgrad(p2, h1, H, H, s2, P, B);
+      dgrad<W>(w2, H, H, p2, p1, p1, false, P, col, part);         // p1 <- d(pre 1)
       __syncthreads();
-      wgrad(p1, z, H, IN, s1, B);
-      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, B, col, part);    // dz += W1^T d(pre 1)
+      wgrad(p1, z, H, IN, s1, P, B);
+      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, P, col, part);    // dz += W1^T d(pre 1)
       __syncthreads();
     }
     if (valid) {
       for (int l = part; l < g.L; l += kParts) {
         float d[F];
 #pragma unroll
-        for (int f = 0; f < F; ++f) d[f] = dz[(l * F + f) * B + col];
+        for (int f = 0; f < F; ++f) d[f] = dz[(l * F + f) * P + col];
         scatter_level<F>(xt, g, l, grad_tables, d);
       }
     }
@@ -328,7 +350,7 @@ __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, in
   }
 }
 
-constexpr size_t kBwdSmem = ((size_t)7 * kMaxDim + 8) * kHeadsBwdBlock * sizeof(float);
+constexpr size_t kBwdSmem = ((size_t)7 * kMaxDim + 8) * kHeadsBwdPitch * sizeof(float);
 
 int validate_heads(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
   if (!h) return SPIN4D_ERR_INVALID;

@@ -56,7 +56,7 @@ def parse():
     p.add_argument("--ncu-case", default=None,
                    help="profiling driver: run a few untimed launches of one workload and exit "
                         "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32, "
-                        "render_sports_frame)")
+                        "render_sports_frame, paper_heads_fp16)")
     return p.parse_args()
 
 
@@ -797,6 +797,25 @@ def _oracle_job(name, what, n, seed):
     (for the render: n sampled pixels of the frame)."""
     from oracle import decoder as dec, hexplane as hxo, render as rdo
     rng = np.random.default_rng(seed)
+    if name == "paper_heads_fp16":
+        # 200k positions (a small case of the 1M launch): forward saving z, then the backward
+        grid, spec_h = w["grid"], w["heads"]
+        n = 200_000
+        g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec_h)
+        P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
+        T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+        W = torch.from_numpy(S.heads_weights(spec_h)).to(dev)
+        grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
+                 for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec_h.sh_dim).items()}
+        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
+        gw = torch.zeros(spec_h.n_params(), device=dev)
+        for _ in range(2):
+            out = sp.heads_fwd(g, h, P, T, W, latent=True)
+            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"])
+        torch.cuda.synchronize()
+        sp.check_device_errors()
+        print("ncu case done:", name)
+        return
     if name == "render_sports_frame":
         spec = S.orbit_camera(640, 360)
         sc = S.render_scene(300_000, seed=0)
@@ -875,6 +894,25 @@ def run_ncu_case(name):
     from spatiotemporal_neural_field_b200 import spin4d as sp
     dev = torch.device("cuda", 0)
     w = S.WORKLOADS.get(name)
+    if name == "paper_heads_fp16":
+        # 200k positions (a small case of the 1M launch): forward saving z, then the backward
+        grid, spec_h = w["grid"], w["heads"]
+        n = 200_000
+        g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec_h)
+        P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
+        T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+        W = torch.from_numpy(S.heads_weights(spec_h)).to(dev)
+        grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
+                 for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec_h.sh_dim).items()}
+        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
+        gw = torch.zeros(spec_h.n_params(), device=dev)
+        for _ in range(2):
+            out = sp.heads_fwd(g, h, P, T, W, latent=True)
+            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"])
+        torch.cuda.synchronize()
+        sp.check_device_errors()
+        print("ncu case done:", name)
+        return
     if name == "render_sports_frame":
         spec = S.orbit_camera(640, 360)
         sc = S.render_scene(300_000, seed=0)

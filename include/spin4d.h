@@ -378,8 +378,8 @@ int spin4d_check_device_errors(int clear);
  * r = r^/max(|r^|, 1e-12), sh = sh^, o = sigma(o^); Sigma by Eq. 2.
  * Weights (fp32 or fp16, 4-byte aligned) are packed head by head in that
  * order, each [W1 b1 W2 b2 W3 b3] with W[out][in] row-major.
- * in_dim = L*F; in_dim, hidden and sh_dim at most 64
- * (SPIN4D_ERR_UNSUPPORTED above).  fp32 arithmetic.
+ * in_dim = L*F; in_dim, hidden and sh_dim at most 64, in_dim and hidden
+ * multiples of 4 (SPIN4D_ERR_UNSUPPORTED otherwise).  fp32 arithmetic.
  */
 typedef struct spin4d_heads_desc {
     int32_t in_dim;

@@ -27,7 +27,6 @@ namespace {
 
 constexpr int kHeadsBlock = 64;      // forward: positions per block
 constexpr int kHeadsBwdBlock = 32;   // backward: positions per block
-constexpr int kHeadsBwdPitch = kHeadsBwdBlock + 1;
 constexpr int kMaxDim = 64;          // in_dim, hidden and sh_dim limit of the shared-memory layout
 
 struct HeadsParams {
@@ -170,115 +169,231 @@ __global__ void __launch_bounds__(kHeadsBlock * kParts) heads_fwd_kernel(GridPar
 
 __device__ __forceinline__ float g0(const float* p, int64_t i) { return p ? __ldg(p + i) : 0.0f; }
 
-// slot += the block's weight gradient of one layer: W[o][k] += sum_t d[o][t]
-// x[k][t] and b[o] += sum_t d[o][t], as fp32 reductions (no load to wait
-// for).  Activations are [feature][position] with an odd pitch, so lanes on
-// consecutive columns k read different banks; each thread keeps 8 rows of
-// one column in registers (the d reads are warp-wide broadcasts).  The task
-// of every slot element is fixed, so its adds come from one thread in program
+// ---------------------------------------------------------------------------
+// Backward.  Activations live in shared memory [position][feature] with a
+// pitch of kQ = 68 floats (16-byte rows; 68 = 4 mod 32, so the eight
+// positions p, p + 8, ... of a thread group fall in different banks).  One
+// layer's weights at a time are staged as fp32 rows of the same pitch (rows
+// padded with zeros to a multiple of 4).  Every inner loop is register
+// blocked 4 x 4: one 16-byte shared load feeds four FMAs, so the loops are
+// bound by the FMA pipe rather than by loads.  Threads: 128 = 16 feature
+// groups x 8 position groups; position group g owns positions g, g + 8,
+// g + 16, g + 24 of the block's 32.
+// ---------------------------------------------------------------------------
+constexpr int kQ = 68;
+constexpr int kBwdThreads = 128;
+
+template <typename W>
+__device__ __forceinline__ void stage_layer(const W* __restrict__ src, int n_out, int n_in, float* __restrict__ Ws,
+                                            float* __restrict__ bs) {
+  const int n_out4 = (n_out + 3) & ~3;
+  for (int i = threadIdx.x; i < n_out4 * n_in; i += kBwdThreads) {
+    const int o = i / n_in, k = i - o * n_in;
+    Ws[o * kQ + k] = o < n_out ? to_f32<W>(__ldg(src + i)) : 0.0f;
+  }
+  for (int o = threadIdx.x; o < n_out4; o += kBwdThreads) bs[o] = o < n_out ? to_f32<W>(__ldg(src + n_out * n_in + o)) : 0.0f;
+}
+
+// out[t][o] = b[o] + sum_k W[o][k] in[t][k] for o < n_out; pre[t][o] keeps
+// the value when given, out receives gelu of it when `act`.  Thread (rg, pg)
+// computes rows rg, rg + 16, rg + 32, rg + 48 for its four positions.
+__device__ __forceinline__ void layer_q(const float* __restrict__ Ws, const float* __restrict__ bs, int n_out,
+                                        int n_in, const float* in, float* out, float* pre, bool act) {
+  const int pg = threadIdx.x & 7, rg = threadIdx.x >> 3;
+  if (rg >= n_out) return;
+  float acc[4][4];
+  int row[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    row[j] = min(rg + 16 * j, kMaxDim - 1);   // rows past n_out compute on a staged row and are not stored
+    const float bj = rg + 16 * j < n_out ? bs[rg + 16 * j] : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[j][i] = bj;
+  }
+  for (int k = 0; k < n_in; k += 4) {
+    float4 x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const float4*>(in + (pg + 8 * i) * kQ + k);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 w = *reinterpret_cast<const float4*>(Ws + row[j] * kQ + k);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        acc[j][i] = fmaf(w.x, x[i].x, fmaf(w.y, x[i].y, fmaf(w.z, x[i].z, fmaf(w.w, x[i].w, acc[j][i]))));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int o = rg + 16 * j;
+    if (o >= n_out) break;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = pg + 8 * i;
+      if (pre) pre[t * kQ + o] = acc[j][i];
+      out[t * kQ + o] = act ? gelu(acc[j][i]) : acc[j][i];
+    }
+  }
+}
+
+// acc[kk][i] = sum_o W[o][4 kg + kk] d[t_i][o] over o < n_out4 (d's columns
+// and W's rows past n_out are zero).  Thread (kg, pg), kg < n_in / 4.
+__device__ __forceinline__ void dgrad_q(const float* __restrict__ Ws, int n_out4, const float* d, int kg,
+                                        float (&acc)[4][4]) {
+  const int pg = threadIdx.x & 7;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[kk][i] = 0.0f;
+  for (int o = 0; o < n_out4; o += 4) {
+    float4 dv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dv[i] = *reinterpret_cast<const float4*>(d + (pg + 8 * i) * kQ + o);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const float4 w = *reinterpret_cast<const float4*>(Ws + (o + jj) * kQ + 4 * kg);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float dd = jj == 0 ? dv[i].x : (jj == 1 ? dv[i].y : (jj == 2 ? dv[i].z : dv[i].w));
+        acc[0][i] = fmaf(w.x, dd, acc[0][i]);
+        acc[1][i] = fmaf(w.y, dd, acc[1][i]);
+        acc[2][i] = fmaf(w.z, dd, acc[2][i]);
+        acc[3][i] = fmaf(w.w, dd, acc[3][i]);
+      }
+    }
+  }
+}
+
+// dx[t][k] = (sum_o W[o][k] d[t][o]) * gelu'(pre[t][k]), in place over pre.
+__device__ __forceinline__ void dgrad_gelu_q(const float* __restrict__ Ws, int n_out4, int n_in, const float* d,
+                                             float* pre_dx) {
+  const int pg = threadIdx.x & 7, kg = threadIdx.x >> 3;
+  if (4 * kg >= n_in) return;
+  float acc[4][4];
+  dgrad_q(Ws, n_out4, d, kg, acc);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float* q = pre_dx + (pg + 8 * i) * kQ + 4 * kg + kk;
+      *q = acc[kk][i] * gelu_grad(*q);
+    }
+}
+
+// slot += the block's gradient of one layer: W[o][k] += sum_t d[t][o] x[t][k],
+// b[o] += sum_t d[t][o], as fp32 reductions (no load to wait for).  Each slot
+// element belongs to one task of one thread, so its adds come in program
 // order and the sum does not depend on scheduling.
-__device__ __forceinline__ void wgrad(const float* d, const float* x, int n_out, int n_in, float* slot, int pitch,
-                                      int npos) {
-  constexpr int RO = 8;
-  const int ob = (n_out + RO - 1) / RO;
-  const int kb = (n_in + 31) / 32 * 32;   // columns padded to whole warps: a warp shares its row block
-  for (int task = threadIdx.x; task < ob * kb; task += blockDim.x) {
-    const int k = task % kb, o0 = (task / kb) * RO;
-    if (k >= n_in) continue;
-    float acc[RO];
+__device__ __forceinline__ void wgrad_q(const float* d, const float* x, int n_out, int n_in, float* slot, int npos) {
+  const int ogs = (n_out + 3) >> 2, kgs = n_in >> 2;
+  for (int task = threadIdx.x; task < ogs * kgs; task += kBwdThreads) {
+    const int kg = task % kgs, og = task / kgs;
+    float acc[4][4];
 #pragma unroll
-    for (int i = 0; i < RO; ++i) acc[i] = 0.0f;
-    const float* dr[RO];
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int i = 0; i < RO; ++i) dr[i] = d + min(o0 + i, n_out - 1) * pitch;
-    const float* xk = x + k * pitch;
+      for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
     for (int t = 0; t < npos; ++t) {
-      const float xv = xk[t];
+      const float4 dv = *reinterpret_cast<const float4*>(d + t * kQ + 4 * og);
+      const float4 xv = *reinterpret_cast<const float4*>(x + t * kQ + 4 * kg);
+      const float dd[4] = {dv.x, dv.y, dv.z, dv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-      for (int i = 0; i < RO; ++i) acc[i] = fmaf(dr[i][t], xv, acc[i]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(dd[a], xx[c], acc[a][c]);
     }
 #pragma unroll
-    for (int i = 0; i < RO; ++i)
-      if (o0 + i < n_out) atomicAdd(slot + (o0 + i) * n_in + k, acc[i]);
+    for (int a = 0; a < 4; ++a) {
+      const int o = 4 * og + a;
+      if (o >= n_out) break;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) atomicAdd(slot + o * n_in + 4 * kg + c, acc[a][c]);
+    }
   }
-  for (int o = threadIdx.x; o < n_out; o += blockDim.x) {
+  for (int o = threadIdx.x; o < n_out; o += kBwdThreads) {
     float sb = 0.0f;
-    for (int t = 0; t < npos; ++t) sb += d[o * pitch + t];
+    for (int t = 0; t < npos; ++t) sb += d[t * kQ + o];
     atomicAdd(slot + n_out * n_in + o, sb);
   }
 }
 
-// dx[k] (+)= sum_o W[o][k] d[o] for this part's k (part, part + kParts, ...),
-// this column; times gelu'(pre[k]) when pre is given.
-template <typename W>
-__device__ __forceinline__ void dgrad(const W* __restrict__ Wp, int n_out, int n_in, const float* d, float* dx,
-                                      const float* pre, bool accumulate, int blk, int col, int part) {
-  for (int k = part; k < n_in; k += kParts) {
-    float s = 0.0f;
-    for (int o = 0; o < n_out; ++o) s = fmaf(wv(Wp + o * n_in, k), d[o * blk + col], s);
-    if (pre) s *= gelu_grad(pre[k * blk + col]);
-    dx[k * blk + col] = accumulate ? dx[k * blk + col] + s : s;
-  }
-}
-
 template <typename T, int F, typename W>
-__global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
+__global__ void __launch_bounds__(kBwdThreads) heads_bwd_kernel(
     GridParams g, HeadsParams hp, const float4* __restrict__ pos, int64_t N, const T* __restrict__ tables,
     const W* __restrict__ weights, const float* __restrict__ latent, HeadsGrads go, float* __restrict__ grad_tables,
     float* __restrict__ ws, int n_params) {
-  constexpr int B = kHeadsBwdBlock;
-  constexpr int P = kHeadsBwdPitch;    // odd: a warp's column reads hit 32 different banks
+  constexpr int B = kHeadsBwdBlock;     // 32 positions
   extern __shared__ float sm[];
-  float* z = sm;                       // [IN][P]
-  float* p1 = z + kMaxDim * P;         // pre-activations of layer 1, later d(pre 1)
-  float* h1 = p1 + kMaxDim * P;
-  float* p2 = h1 + kMaxDim * P;        // pre-activations of layer 2, later d(pre 2)
-  float* h2 = p2 + kMaxDim * P;
-  float* dy = h2 + kMaxDim * P;        // one head's output adjoint
-  float* dz = dy + kMaxDim * P;
-  float* dattr = dz + kMaxDim * P;     // [8][P]: adjoint of raw scale, rot, opacity
-  const int col = threadIdx.x % B, part = threadIdx.x / B;
+  float* z = sm;                        // [B][kQ]; after the last head, dz
+  float* p1 = z + B * kQ;               // pre-activations of layer 1, later d(pre 1)
+  float* h1 = p1 + B * kQ;
+  float* p2 = h1 + B * kQ;              // pre-activations of layer 2, later d(pre 2)
+  float* h2 = p2 + B * kQ;
+  float* dy = h2 + B * kQ;              // one head's output (first pass) or output adjoint
+  float* Ws = dy + B * kQ;              // one staged layer: kMaxDim rows of kQ
+  float* bs = Ws + kMaxDim * kQ;        // its biases
+  float* dattr = bs + kMaxDim;          // [B][8]: adjoint of raw scale^, rot^, opacity^
   const int IN = hp.in_dim, H = hp.hidden;
+  const int pg = threadIdx.x & 7, fg = threadIdx.x >> 3;
   float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
-  for (int p = threadIdx.x; p < n_params; p += blockDim.x) slot[p] = 0.0f;
+  for (int p = threadIdx.x; p < n_params; p += kBwdThreads) slot[p] = 0.0f;
 
   for (int64_t n0 = (int64_t)blockIdx.x * B; n0 < N; n0 += (int64_t)gridDim.x * B) {
-    const int64_t n = n0 + col;
-    const bool valid = n < N;
-    float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) normalise_position(pos[n], g, xt);
-    if (valid && latent) {
-      for (int k = part; k < IN; k += kParts) z[k * P + col] = __ldg(latent + n * IN + k);
-    } else if (valid) {
-      gather_z<T, F>(xt, g, tables, z, P, col, part, nullptr, n, IN);
-    } else {
-      for (int k = part; k < IN; k += kParts) z[k * P + col] = 0.0f;
+    // z: thread (fg, pg) fills features of its positions; levels for the gather
+    for (int e = threadIdx.x; e < B * IN; e += kBwdThreads) {
+      const int t = e / IN, k = e - t * IN;
+      const int64_t n = n0 + t;
+      z[t * kQ + k] = (n < N && latent) ? __ldg(latent + n * IN + k) : 0.0f;
     }
-    for (int k = part; k < IN; k += kParts) dz[k * P + col] = 0.0f;
+    if (!latent) {
+      // one thread per (position, level group): the gather writes its levels of z
+      for (int e = threadIdx.x; e < B * kParts; e += kBwdThreads) {
+        const int t = e % B, part = e / B;
+        const int64_t n = n0 + t;
+        if (n >= N) continue;
+        float xt[4];
+        normalise_position(pos[n], g, xt);
+        for (int l = part; l < g.L; l += kParts) {
+          float acc[F];
+          if constexpr (std::is_same<T, __half>::value && (F == 2 || F == 4))
+            encode_level_f16_paired<F>(xt, g, l, tables, acc);
+          else
+            encode_level<T, F>(xt, g, l, tables, acc);
+#pragma unroll
+          for (int f = 0; f < F; ++f) z[t * kQ + l * F + f] = acc[f];
+        }
+      }
+    }
     __syncthreads();
-    // raw outputs of the scale, rotation and opacity heads, then (part 0) the
-    // adjoint of Eq. 11 and Eq. 2
+    // ---- first pass: raw outputs of the scale, rotation and opacity heads ----
     float raw[8];
     for (int h = 0; h < 4; ++h) {
       if (h == 2) continue;
       const W* w = weights + hp.off[h];
-      layer<W>(w, H, IN, z, h1, nullptr, true, P, col, part);
+      stage_layer<W>(w, H, IN, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, H, IN, z, h1, nullptr, true);
       __syncthreads();
       w += H * IN + H;
-      layer<W>(w, H, H, h1, h2, nullptr, true, P, col, part);
+      stage_layer<W>(w, H, H, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, H, H, h1, h2, nullptr, true);
       __syncthreads();
       w += H * H + H;
-      layer<W>(w, hp.rows[h], H, h2, dy, nullptr, false, P, col, part);
+      stage_layer<W>(w, hp.rows[h], H, Ws, bs);
       __syncthreads();
-      if (part == 0) {
+      layer_q(Ws, bs, hp.rows[h], H, h2, dy, nullptr, false);
+      __syncthreads();
+      if (threadIdx.x < B) {
         const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[i * P + col];
+        for (int i = 0; i < hp.rows[h]; ++i) raw[base + i] = dy[threadIdx.x * kQ + i];
       }
       __syncthreads();
     }
-    if (part == 0) {
+    // ---- the adjoint of Eq. 11 and Eq. 2, one thread per position ----
+    if (threadIdx.x < B) {
+      const int64_t n = n0 + threadIdx.x;
       float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (valid) {
+      if (n < N) {
         float s[3], r[4], cov_g[6], gs[3], gr[4];
 #pragma unroll
         for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
@@ -297,44 +412,85 @@ __global__ void __launch_bounds__(kHeadsBwdBlock * kParts) heads_bwd_kernel(
         d[7] = g0(go.opacity, n) * o * (1.0f - o);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dattr[i * P + col] = d[i];
+      for (int i = 0; i < 8; ++i) dattr[threadIdx.x * 8 + i] = d[i];
     }
     __syncthreads();
-    // ---- per head: forward with pre-activations, then the three layers' gradients ----
+    // ---- per head: forward keeping pre-activations, then the three layers' gradients ----
+    float dz[4][4];   // this thread's (feature group, position group) block of dz, summed over the heads
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dz[kk][i] = 0.0f;
     for (int h = 0; h < 4; ++h) {
-      const int rows = hp.rows[h];
+      const int rows = hp.rows[h], rows4 = (rows + 3) & ~3;
       const W* w1 = weights + hp.off[h];
       const W* w2 = w1 + H * IN + H;
       const W* w3 = w2 + H * H + H;
       float* s1 = slot + hp.off[h];
       float* s2 = s1 + H * IN + H;
       float* s3 = s2 + H * H + H;
-      layer<W>(w1, H, IN, z, h1, p1, true, P, col, part);
+      stage_layer<W>(w1, H, IN, Ws, bs);
       __syncthreads();
-      layer<W>(w2, H, H, h1, h2, p2, true, P, col, part);
-      if (h == 2) {
-        for (int i = part; i < rows; i += kParts)
-          dy[i * P + col] = valid ? g0(go.sh, (int64_t)hp.sh_dim * n + i) : 0.0f;
-      } else {
-        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = part; i < rows; i += kParts) dy[i * P + col] = dattr[(base + i) * P + col];
+      layer_q(Ws, bs, H, IN, z, h1, p1, true);
+      __syncthreads();
+      stage_layer<W>(w2, H, H, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, H, H, h1, h2, p2, true);
+      // the head's output adjoint, zero past its rows
+      for (int e = threadIdx.x; e < B * rows4; e += kBwdThreads) {
+        const int t = e / rows4, i = e - t * rows4;
+        const int64_t n = n0 + t;
+        float v = 0.0f;
+        if (i < rows && n < N) {
+          if (h == 2)
+            v = g0(go.sh, (int64_t)hp.sh_dim * n + i);
+          else
+            v = dattr[t * 8 + (h == 0 ? 0 : (h == 1 ? 3 : 7)) + i];
+        }
+        dy[t * kQ + i] = v;
       }
       __syncthreads();
-      wgrad(dy, h2, rows, H, s3, P, B);
-      dgrad<W>(w3, rows, H, dy, p2, p2, false, P, col, part);      // p2 <- d(pre 2)
+      stage_layer<W>(w3, rows, H, Ws, bs);
+      wgrad_q(dy, h2, rows, H, s3, B);
       __syncthreads();
-      wgrad(p2, h1, H, H, s2, P, B);
-      dgrad<W>(w2, H, H, p2, p1, p1, false, P, col, part);         // p1 <- d(pre 1)
+      dgrad_gelu_q(Ws, rows4, H, dy, p2);          // p2 <- d(pre 2)
       __syncthreads();
-      wgrad(p1, z, H, IN, s1, P, B);
-      dgrad<W>(w1, H, IN, p1, dz, nullptr, true, P, col, part);    // dz += W1^T d(pre 1)
+      stage_layer<W>(w2, H, H, Ws, bs);
+      wgrad_q(p2, h1, H, H, s2, B);
       __syncthreads();
+      dgrad_gelu_q(Ws, H, H, p2, p1);              // p1 <- d(pre 1)
+      __syncthreads();
+      stage_layer<W>(w1, H, IN, Ws, bs);
+      wgrad_q(p1, z, H, IN, s1, B);
+      __syncthreads();
+      if (4 * fg < IN) {                           // dz += W1^T d(pre 1)
+        float acc[4][4];
+        dgrad_q(Ws, H, p1, fg, acc);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dz[kk][i] += acc[kk][i];
+      }
+      __syncthreads();   // the next head restages the weights and rewrites the activations
     }
-    if (valid) {
+    // dz over z (free now), then the scatter into the tables
+    if (4 * fg < IN) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[(pg + 8 * i) * kQ + 4 * fg + kk] = dz[kk][i];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < B * kParts; e += kBwdThreads) {
+      const int t = e % B, part = e / B;
+      const int64_t n = n0 + t;
+      if (n >= N) continue;
+      float xt[4];
+      normalise_position(pos[n], g, xt);
       for (int l = part; l < g.L; l += kParts) {
         float d[F];
 #pragma unroll
-        for (int f = 0; f < F; ++f) d[f] = dz[(l * F + f) * P + col];
+        for (int f = 0; f < F; ++f) d[f] = z[t * kQ + l * F + f];
         scatter_level<F>(xt, g, l, grad_tables, d);
       }
     }
@@ -350,13 +506,16 @@ __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, in
   }
 }
 
-constexpr size_t kBwdSmem = ((size_t)7 * kMaxDim + 8) * kHeadsBwdPitch * sizeof(float);
+constexpr size_t kBwdSmem = ((size_t)6 * kHeadsBwdBlock * kQ + (size_t)kMaxDim * kQ + kMaxDim +
+                             (size_t)kHeadsBwdBlock * 8) * sizeof(float);
 
 int validate_heads(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
   if (!h) return SPIN4D_ERR_INVALID;
   if (h->in_dim != g->L * g->F) return SPIN4D_ERR_INVALID;
   if (h->hidden < 1 || h->sh_dim < 1 || h->w_dtype < 0 || h->w_dtype > 1) return SPIN4D_ERR_INVALID;
   if (h->in_dim > kMaxDim || h->hidden > kMaxDim || h->sh_dim > kMaxDim) return SPIN4D_ERR_UNSUPPORTED;
+  // the backward's register blocking takes features four at a time
+  if (h->in_dim % 4 || h->hidden % 4) return SPIN4D_ERR_UNSUPPORTED;
   return SPIN4D_OK;
 }
 
@@ -384,7 +543,8 @@ int64_t param_count(const spin4d_heads_desc* h) {
   return n;
 }
 
-int bwd_blocks(int64_t N) { return persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 6); }
+// three blocks fit an SM (shared memory): the grid is three per SM, so there is no second wave
+int bwd_blocks(int64_t N) { return persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 3); }
 
 template <typename T, int F, typename W>
 struct HeadsLaunch {
@@ -403,7 +563,7 @@ struct HeadsLaunch {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
     if (e != cudaSuccess) return cuda_status(e);
     const int blocks = bwd_blocks(N);
-    k<<<blocks, kHeadsBwdBlock * kParts, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+    k<<<blocks, kBwdThreads, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
                                               static_cast<const T*>(tables), static_cast<const W*>(weights), latent,
                                               go, grad_tables, ws, n_params);
     SPIN4D_CHECK(launch_status());

@@ -134,6 +134,8 @@ def test_invalid_arguments_rejected_on_host(sp):
                                 sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
     assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
                                 sp.HeadsOutputs(FAKE, FAKE + 4, FAKE, FAKE, FAKE, None), None) == sp.ERR_INVALID
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(64, hidden=62)), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
     # grouped Adam: ends must increase to n
     grp = (sp.AdamGroup * 2)(sp.AdamGroup(60, 1e-3), sp.AdamGroup(50, 1e-4))
     assert lib.spin4d_adam_step_groups(FAKE, None, FAKE, FAKE, FAKE, 100, grp, 2, 1, 0.9, 0.99, 1e-15, 0, None,

@@ -498,6 +498,81 @@ __global__ void __launch_bounds__(kBwdThreads) heads_bwd_kernel(
   }
 }
 
+// Forward with the backward's register-blocked layers: 32 positions per
+// block, 128 threads; the gather takes one (position, level group) per
+// thread, the layers run 4 x 4 blocks out of shared memory.
+template <typename T, int F, typename W>
+__global__ void __launch_bounds__(kBwdThreads) heads_fwd_q_kernel(GridParams g, HeadsParams hp,
+                                                                  const float4* __restrict__ pos, int64_t N,
+                                                                  const T* __restrict__ tables,
+                                                                  const W* __restrict__ weights, HeadsOut out) {
+  constexpr int B = kHeadsBwdBlock;
+  extern __shared__ float sm[];
+  float* z = sm;                        // [B][kQ]
+  float* h1 = z + B * kQ;
+  float* h2 = h1 + B * kQ;
+  float* y = h1;                        // one head's raw outputs (layer 3 no longer needs h1)
+  float* Ws = h2 + B * kQ;
+  float* bs = Ws + kMaxDim * kQ;
+  const int IN = hp.in_dim, H = hp.hidden;
+  for (int64_t n0 = (int64_t)blockIdx.x * B; n0 < N; n0 += (int64_t)gridDim.x * B) {
+    for (int e = threadIdx.x; e < B * kParts; e += kBwdThreads) {
+      const int t = e % B, part = e / B;
+      const int64_t n = n0 + t;
+      if (n >= N) {
+        for (int l = part; l < g.L; l += kParts)
+          for (int f = 0; f < F; ++f) z[t * kQ + l * F + f] = 0.0f;
+        continue;
+      }
+      float xt[4];
+      normalise_position(pos[n], g, xt);
+      for (int l = part; l < g.L; l += kParts) {
+        float acc[F];
+        if constexpr (std::is_same<T, __half>::value && (F == 2 || F == 4))
+          encode_level_f16_paired<F>(xt, g, l, tables, acc);
+        else
+          encode_level<T, F>(xt, g, l, tables, acc);
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+          z[t * kQ + l * F + f] = acc[f];
+          if (out.latent) out.latent[n * IN + l * F + f] = acc[f];
+        }
+      }
+    }
+    float raw[8];
+    for (int h = 0; h < 4; ++h) {
+      const W* w = weights + hp.off[h];
+      const int rows = hp.rows[h];
+      __syncthreads();   // z written / the previous head's outputs read
+      stage_layer<W>(w, H, IN, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, H, IN, z, h1, nullptr, true);
+      __syncthreads();
+      stage_layer<W>(w + H * IN + H, H, H, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, H, H, h1, h2, nullptr, true);
+      __syncthreads();
+      stage_layer<W>(w + H * IN + H + H * H + H, rows, H, Ws, bs);
+      __syncthreads();
+      layer_q(Ws, bs, rows, H, h2, y, nullptr, false);
+      __syncthreads();
+      if (h == 2) {
+        for (int e = threadIdx.x; e < B * rows; e += kBwdThreads) {
+          const int t = e / rows, i = e - t * rows;
+          const int64_t n = n0 + t;
+          if (n < N) out.sh[(int64_t)hp.sh_dim * n + i] = y[t * kQ + i];
+        }
+      } else if (threadIdx.x < B) {
+        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+        for (int i = 0; i < rows; ++i) raw[base + i] = y[threadIdx.x * kQ + i];
+      }
+    }
+    if (threadIdx.x < B && n0 + threadIdx.x < N) store_heads(out, n0 + threadIdx.x, raw);
+  }
+}
+
+constexpr size_t kFwdQSmem = ((size_t)3 * kHeadsBwdBlock * kQ + (size_t)kMaxDim * kQ + kMaxDim) * sizeof(float);
+
 __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
     float s = 0.0f;
@@ -550,6 +625,15 @@ template <typename T, int F, typename W>
 struct HeadsLaunch {
   static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const HeadsOut& o, cudaStream_t s) {
+    if (hp.in_dim % 4 == 0 && hp.hidden % 4 == 0) {
+      auto k = heads_fwd_q_kernel<T, F, W>;
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdQSmem);
+      if (e != cudaSuccess) return cuda_status(e);
+      const int qb = persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 5);   // 5 fit an SM
+      k<<<qb, kBwdThreads, kFwdQSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                           static_cast<const T*>(tables), static_cast<const W*>(weights), o);
+      return launch_status();
+    }
     const int blocks = persistent_blocks((N + kHeadsBlock - 1) / kHeadsBlock, 6);
     heads_fwd_kernel<T, F, W><<<blocks, kHeadsBlock * kParts, 0, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
                                                              static_cast<const T*>(tables),

@@ -3,21 +3,22 @@
 // with GELU after the first two layers, on the shared latent z of the 4D
 // hash encoder (SPIN-4DGS section 3.3, Eqs. 9-11; Sigma by Eq. 2).
 //
-// fp32 SIMT kernels, four threads per position (each a quarter of every
-// layer's output rows, and a quarter of the hash levels), activations in
-// shared memory [feature][position] so that the weight reads are warp-wide
-// broadcasts.
-// At the paper's size (L = 16, F = 4, T = 2^21: 256 MiB of fp16 tables) the
-// corner gathers come from HBM and the four 64-wide MLPs run beside them.
+// fp32 SIMT kernels, 32 positions and 128 threads per block.  The hash
+// gather takes one (position, level group) per thread.  The layers run out
+// of shared memory: activations [position][feature], one layer's weights
+// staged as fp32 rows, every product register-blocked 4 x 4 over 16-byte
+// loads.  At the paper's size (L = 16, F = 4, T = 2^21: 256 MiB of fp16
+// tables) the corner gathers come from HBM and bound the forward.
 //
 // Forward: gather z, then per head two GELU layers and the output layer,
-// four output rows per pass (independent accumulators), then Eq. 11 and Eq. 2.
-// Backward: forward again keeping the raw outputs of all heads (scale and
-// rotation couple through Sigma), the activations' adjoint, then per head
-// the forward again with its pre-activations, the data gradient through the
-// three layers into dz and the weight gradient summed over the block's
-// positions into the block's workspace slot (a second kernel adds the slots
-// in a fixed order); dz is scattered into the tables with fp32 atomics.
+// then Eq. 11 and Eq. 2.
+// Backward: forward again keeping the raw outputs of the scale, rotation
+// and opacity heads (they couple through Sigma), the activations' adjoint,
+// then per head the forward again with its pre-activations, the data
+// gradient through the three layers into dz (kept in registers across the
+// heads) and the weight gradient summed over the block's positions into the
+// block's workspace slot (a second kernel adds the slots in a fixed order);
+// dz is scattered into the tables with fp32 atomics.
 #include <type_traits>
 
 #include "host.h"
@@ -25,8 +26,7 @@
 namespace spin4d {
 namespace {
 
-constexpr int kHeadsBlock = 64;      // forward: positions per block
-constexpr int kHeadsBwdBlock = 32;   // backward: positions per block
+constexpr int kHeadsBwdBlock = 32;   // positions per block (forward and backward)
 constexpr int kMaxDim = 64;          // in_dim, hidden and sh_dim limit of the shared-memory layout
 
 struct HeadsParams {
@@ -42,51 +42,15 @@ struct HeadsGrads {
   const float *scale, *rot, *sh, *opacity, *cov;
 };
 
-template <typename W>
-__device__ __forceinline__ float wv(const W* __restrict__ w, int i) {
-  return to_f32<W>(__ldg(w + i));
-}
-
 // Exact GELU, x Phi(x), and its derivative Phi(x) + x phi(x).
 __device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 __device__ __forceinline__ float gelu_grad(float x) {
   return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * expf(-0.5f * x * x);
 }
 
-// kParts threads serve each position; part p takes the output rows of the
-// 4-row groups p, p + kParts, ...  (all lanes of a warp share a part, so the
-// weight reads are warp-wide broadcasts).  Rows past n_out are computed on a
-// clamped row and not stored.
+// kParts threads share the hash gather of each position (levels part,
+// part + kParts, ...).
 constexpr int kParts = 4;
-
-// out[o] = b[o] + sum_k W[o][k] in[k] for this part's rows, this column;
-// pre (when given) keeps the value, out receives gelu of it when `act`.
-template <typename W>
-__device__ __forceinline__ void layer(const W* __restrict__ Wp, int n_out, int n_in, const float* in, float* out,
-                                      float* pre, bool act, int blk, int col, int part) {
-  const W* bp = Wp + n_out * n_in;
-  for (int o = 4 * part; o < n_out; o += 4 * kParts) {
-    int r[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) r[i] = min(o + i, n_out - 1);
-    float a0 = wv(bp, r[0]), a1 = wv(bp, r[1]), a2 = wv(bp, r[2]), a3 = wv(bp, r[3]);
-    const W *w0 = Wp + r[0] * n_in, *w1 = Wp + r[1] * n_in, *w2 = Wp + r[2] * n_in, *w3 = Wp + r[3] * n_in;
-    for (int k = 0; k < n_in; ++k) {
-      const float x = in[k * blk + col];
-      a0 = fmaf(wv(w0, k), x, a0);
-      a1 = fmaf(wv(w1, k), x, a1);
-      a2 = fmaf(wv(w2, k), x, a2);
-      a3 = fmaf(wv(w3, k), x, a3);
-    }
-    const float v[4] = {a0, a1, a2, a3};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (o + i >= n_out) break;
-      if (pre) pre[(o + i) * blk + col] = v[i];
-      out[(o + i) * blk + col] = act ? gelu(v[i]) : v[i];
-    }
-  }
-}
 
 // raw[0..2] scale^, raw[3..6] rot^, raw[7] opacity^ -> Eq. 11 and Eq. 2.
 __device__ __forceinline__ void store_heads(const HeadsOut& out, int64_t n, const float raw[8]) {
@@ -101,70 +65,6 @@ __device__ __forceinline__ void store_heads(const HeadsOut& out, int64_t n, cons
   out.opacity[n] = sigmoidf_(raw[7]);
 #pragma unroll
   for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
-}
-
-// This part's levels of z (levels part, part + kParts, ...).
-template <typename T, int F>
-__device__ __forceinline__ void gather_z(const float xt[4], const GridParams& g, const T* __restrict__ tables,
-                                         float* z, int blk, int col, int part, float* latent, int64_t n,
-                                         int in_dim) {
-  for (int l = part; l < g.L; l += kParts) {
-    float acc[F];
-    if constexpr (std::is_same<T, __half>::value && (F == 2 || F == 4))
-      encode_level_f16_paired<F>(xt, g, l, tables, acc);
-    else
-      encode_level<T, F>(xt, g, l, tables, acc);
-#pragma unroll
-    for (int f = 0; f < F; ++f) {
-      z[(l * F + f) * blk + col] = acc[f];
-      if (latent) latent[n * in_dim + l * F + f] = acc[f];
-    }
-  }
-}
-
-template <typename T, int F, typename W>
-__global__ void __launch_bounds__(kHeadsBlock * kParts) heads_fwd_kernel(GridParams g, HeadsParams hp,
-                                                                         const float4* __restrict__ pos, int64_t N,
-                                                                         const T* __restrict__ tables,
-                                                                         const W* __restrict__ weights, HeadsOut out) {
-  constexpr int B = kHeadsBlock;
-  __shared__ float z[kMaxDim * B], a[kMaxDim * B], b[kMaxDim * B];
-  const int col = threadIdx.x % B, part = threadIdx.x / B;
-  const int IN = hp.in_dim, H = hp.hidden;
-  for (int64_t n0 = (int64_t)blockIdx.x * B; n0 < N; n0 += (int64_t)gridDim.x * B) {
-    const int64_t n = n0 + col;
-    const bool valid = n < N;
-    float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) {
-      normalise_position(pos[n], g, xt);
-      gather_z<T, F>(xt, g, tables, z, B, col, part, out.latent, n, IN);
-    } else {
-      for (int k = part; k < IN; k += kParts) z[k * B + col] = 0.0f;
-    }
-    __syncthreads();
-    float raw[8];
-    for (int h = 0; h < 4; ++h) {
-      const W* w = weights + hp.off[h];
-      layer<W>(w, H, IN, z, a, nullptr, true, B, col, part);
-      __syncthreads();
-      w += H * IN + H;
-      layer<W>(w, H, H, a, b, nullptr, true, B, col, part);
-      __syncthreads();
-      w += H * H + H;
-      const int rows = hp.rows[h];
-      layer<W>(w, rows, H, b, a, nullptr, false, B, col, part);   // raw outputs over a
-      __syncthreads();
-      if (h == 2) {
-        if (valid)
-          for (int i = part; i < rows; i += kParts) out.sh[(int64_t)hp.sh_dim * n + i] = a[i * B + col];
-      } else if (part == 0) {
-        const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
-        for (int i = 0; i < rows; ++i) raw[base + i] = a[i * B + col];
-      }
-      __syncthreads();   // a is layer 1's output of the next head
-    }
-    if (part == 0 && valid) store_heads(out, n, raw);
-  }
 }
 
 __device__ __forceinline__ float g0(const float* p, int64_t i) { return p ? __ldg(p + i) : 0.0f; }
@@ -625,19 +525,12 @@ template <typename T, int F, typename W>
 struct HeadsLaunch {
   static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const HeadsOut& o, cudaStream_t s) {
-    if (hp.in_dim % 4 == 0 && hp.hidden % 4 == 0) {
-      auto k = heads_fwd_q_kernel<T, F, W>;
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdQSmem);
-      if (e != cudaSuccess) return cuda_status(e);
-      const int qb = persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 5);   // 5 fit an SM
-      k<<<qb, kBwdThreads, kFwdQSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
-                                           static_cast<const T*>(tables), static_cast<const W*>(weights), o);
-      return launch_status();
-    }
-    const int blocks = persistent_blocks((N + kHeadsBlock - 1) / kHeadsBlock, 6);
-    heads_fwd_kernel<T, F, W><<<blocks, kHeadsBlock * kParts, 0, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
-                                                             static_cast<const T*>(tables),
-                                                             static_cast<const W*>(weights), o);
+    auto k = heads_fwd_q_kernel<T, F, W>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdQSmem);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int blocks = persistent_blocks((N + kHeadsBwdBlock - 1) / kHeadsBwdBlock, 5);   // 5 fit an SM
+    k<<<blocks, kBwdThreads, kFwdQSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                             static_cast<const T*>(tables), static_cast<const W*>(weights), o);
     return launch_status();
   }
   static int bwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,

@@ -110,3 +110,73 @@ def test_grouped_adam_matches_oracle(sp):
         tol.normwise(host(M)[start:end], wm, 1e-6, "grouped adam m")
         tol.normwise(host(V)[start:end], wv, 1e-6, "grouped adam v")
         start = end
+
+
+def test_heads_edge_sizes(sp):
+    """N = 0 launches nothing; N = 1 and N = 33 (one block and one more
+    position) match the oracle; the backward accumulates."""
+    grid, spec = S.GRID_PAPER, S.HEADS_PAPER
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
+    tables = S.hash_tables(grid, seed=8, scale=1.0)
+    weights = S.heads_weights(spec, seed=9, bias_scale=0.3)
+    T, W = dev(tables), dev(weights)
+    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
+    gw = torch.zeros(spec.n_params(), device="cuda")
+    empty = torch.zeros((0, 4), device="cuda")
+    out = sp.heads_fwd(g, h, empty, T, W)
+    assert all(v.numel() == 0 for v in out.values())
+    widths = dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim)
+    sp.heads_bwd(g, h, empty, T, W, {k: torch.zeros((0, w), device="cuda") for k, w in widths.items()}, gt, gw)
+    torch.cuda.synchronize()
+    assert not gt.any() and not gw.any()
+    for n in (1, 33):
+        pos = S.sports_scene(300_000).frame(75)[:n]
+        grads = S.upstream_grads(n, widths, 1e-2, seed=10 + n)
+        P = dev(pos)
+        out = sp.heads_fwd(g, h, P, T, W)
+        want = hd.decode_forward(pos, tables, weights, grid, spec)
+        for k in ("scale", "rot", "sh", "opacity", "cov"):
+            tol.absolute(host(out[k]), want[k], tol.FP16_ATOL, "%s (N=%d)" % (k, n))
+        gt.zero_()
+        gw.zero_()
+        G = {k: dev(v) for k, v in grads.items()}
+        sp.heads_bwd(g, h, P, T, W, G, gt, gw)
+        first = (gt.clone(), gw.clone())
+        sp.heads_bwd(g, h, P, T, W, G, gt, gw)
+        wt, ww = hd.decode_backward(pos, tables, weights, grid, spec, grads)
+        tol.normwise(host(first[0]), wt, tol.FP16_GRAD_RTOL, "grad_tables (N=%d)" % n)
+        tol.normwise(host(first[1]), ww, tol.FP16_GRAD_RTOL, "grad_weights (N=%d)" % n)
+        # a second call adds the same gradient again
+        tol.normwise(host(gt), 2 * host(first[0]), 1e-5, "accumulated grad_tables (N=%d)" % n)
+        tol.normwise(host(gw), 2 * host(first[1]), 1e-5, "accumulated grad_weights (N=%d)" % n)
+
+
+def test_heads_full_launch_sampled_and_by_halves(sp):
+    """The timed 1M-position launch: forward on 400 sampled positions against
+    the oracle; the backward of the whole launch equals that of its two
+    halves (linearity; atomics only reorder the fp32 sums)."""
+    w = S.WORKLOADS["paper_heads_fp16"]
+    grid, spec, n = w["grid"], w["heads"], w["N"]
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
+    pos = S.sports_scene(300_000).frames(range(4))[:n]
+    tables = S.hash_tables(grid, seed=11, scale=1.0)
+    weights = S.heads_weights(spec, seed=12, bias_scale=0.3)
+    P, T, W = dev(pos), dev(tables), dev(weights)
+    out = sp.heads_fwd(g, h, P, T, W, latent=True)
+    idx = np.random.default_rng(13).choice(n, 400, replace=False)
+    want = hd.decode_forward(pos[idx], tables, weights, grid, spec)
+    for k in ("scale", "rot", "sh", "opacity", "cov"):
+        tol.absolute(host(out[k])[idx], want[k], tol.FP16_ATOL, k + " (1M launch, sampled)")
+    widths = dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim)
+    G = {k: torch.randn((n, wd), device="cuda", generator=torch.Generator("cuda").manual_seed(14)) * 1e-2
+         for k, wd in widths.items()}
+    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
+    gw = torch.zeros(spec.n_params(), device="cuda")
+    sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=out["latent"])
+    gt2, gw2 = torch.zeros_like(gt), torch.zeros_like(gw)
+    half = n // 2
+    for a, b in ((0, half), (half, n)):
+        sp.heads_bwd(g, h, P[a:b], T, W, {k: v[a:b] for k, v in G.items()}, gt2, gw2, latent=out["latent"][a:b])
+    torch.cuda.synchronize()
+    tol.normwise(host(gt2), host(gt), 1e-4, "grad_tables by halves")
+    tol.normwise(host(gw2), host(gw), 1e-4, "grad_weights by halves")

@@ -194,18 +194,25 @@ def test_sports_frame_full_size_sampled(sp):
 # backward
 # ---------------------------------------------------------------------------
 BWD_CASES = {
-    "rgb": (400, 64, 48, dict(sh_degree=-1, background=(0.3, 0.1, 0.2))),
-    "sh3": (500, 72, 40, dict(sh_degree=3)),
+    # name: (n, width, height, desc overrides, means as (x, y, z, t) rows)
+    "rgb": (400, 64, 48, dict(sh_degree=-1, background=(0.3, 0.1, 0.2)), False),
+    "sh3": (500, 72, 40, dict(sh_degree=3), False),
+    "sh2_stride4_no_stop_no_lowpass": (300, 50, 37, dict(sh_degree=2, t_stop=0.0, lowpass=0.0), True),
+    "one_gaussian": (1, 24, 20, dict(sh_degree=1), False),
 }
 
 
 @pytest.mark.parametrize("case", list(BWD_CASES))
 def test_backward_matches_oracle(sp, case):
-    n, w, h, kw = BWD_CASES[case]
+    n, w, h, kw, stride4 = BWD_CASES[case]
     deg = kw.get("sh_degree", 3)
     spec = S.orbit_camera(w, h, focal=0.9 * w)
     sc = _scene(n, seed=20 + len(case), deg=deg, scale_factor=0.8)
-    cam, desc, args, img, T, state = _gpu_render(sp, spec, sc, kw)
+    if n == 1:
+        sc["mu"][:] = 0.0                      # in front of the camera, centred
+        sc["cov"][:] = np.array([0.02, 0.003, 0.001, 0.015, 0.002, 0.01], np.float32)
+        sc["opacity"][:] = 0.7
+    cam, desc, args, img, T, state = _gpu_render(sp, spec, sc, kw, stride4=stride4)
     G = S.image_grads(spec, seed=21)
     got = sp.render_bwd(cam, desc, *args, dev(G), state)
     torch.cuda.synchronize()
@@ -216,7 +223,7 @@ def test_backward_matches_oracle(sp, case):
 
 
 def test_backward_accumulates_and_accepts_null_outputs(sp):
-    n, w, h, kw = BWD_CASES["sh3"]
+    n, w, h, kw, _ = BWD_CASES["sh3"]
     spec = S.orbit_camera(w, h, focal=0.9 * w)
     sc = _scene(n, seed=30, deg=3, scale_factor=0.8)
     cam, desc, args, _, _, state = _gpu_render(sp, spec, sc, kw)

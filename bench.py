@@ -660,8 +660,8 @@ def run_workloads(args):
     P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
     T = torch.from_numpy(S.hash_tables(grid)).to(dev)
     W = torch.from_numpy(S.heads_weights(spec)).to(dev)
-    out = sp.heads_fwd(g, h, P, T, W, latent=True)
-    fwd_out = {k: v for k, v in out.items() if k != "latent"}
+    out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+    fwd_out = {k: v for k, v in out.items() if k not in ("latent", "raw")}
     ms = timed(lambda: sp.heads_fwd(g, h, P, T, W, out=fwd_out), 10)
     spp = table_sectors_per_position(sp, g, P, grid.F, 2)
     emit("paper_heads_fp16", "fwd", n, ms, table_sectors_per_position=spp, sector_rate=spp * n / (ms * 1e-3),
@@ -676,9 +676,9 @@ def run_workloads(args):
 
     def hfb():
         sp.heads_fwd(g, h, P, T, W, out=out)
-        sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], workspace=ws)
+        sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws)
 
-    emit("paper_heads_fp16", "fwd (saving z) + bwd", n, timed(hfb, 5))
+    emit("paper_heads_fp16", "fwd (saving z and raw head outputs) + bwd", n, timed(hfb, 5))
     del P, T, W, out, fwd_out, grads, gt, gw, ws
     torch.cuda.empty_cache()
 
@@ -810,8 +810,8 @@ def _oracle_job(name, what, n, seed):
         gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
         gw = torch.zeros(spec_h.n_params(), device=dev)
         for _ in range(2):
-            out = sp.heads_fwd(g, h, P, T, W, latent=True)
-            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"])
+            out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"])
         torch.cuda.synchronize()
         sp.check_device_errors()
         print("ncu case done:", name)
@@ -907,8 +907,8 @@ def run_ncu_case(name):
         gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
         gw = torch.zeros(spec_h.n_params(), device=dev)
         for _ in range(2):
-            out = sp.heads_fwd(g, h, P, T, W, latent=True)
-            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"])
+            out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"])
         torch.cuda.synchronize()
         sp.check_device_errors()
         print("ncu case done:", name)

@@ -389,7 +389,10 @@ typedef struct spin4d_heads_desc {
 } spin4d_heads_desc;
 
 /* scale N x 3, rot N x 4 (16-byte aligned), sh N x sh_dim, opacity N x 1,
- * cov N x 6 (fp32); latent (optional) N x in_dim receives z. */
+ * cov N x 6 (fp32); latent (optional) N x in_dim receives z; raw
+ * (optional) N x 8 receives the raw outputs of the scale, rotation and
+ * opacity heads (s^ 3, r^ 4, o^ 1), which spin4d_heads_bwd can take instead
+ * of recomputing those heads. */
 typedef struct spin4d_heads_outputs {
     float* scale;
     float* rot;
@@ -397,6 +400,7 @@ typedef struct spin4d_heads_outputs {
     float* opacity;
     float* cov;
     float* latent;
+    float* raw;
 } spin4d_heads_outputs;
 
 typedef struct spin4d_heads_output_grads {
@@ -418,10 +422,11 @@ size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_
 /* Backward of spin4d_heads_fwd for loss = sum_k <grad_out.k, output_k>
  * (NULL members are zero): grad_tables += (L x T x F fp32, atomics),
  * grad_weights += (packed like weights, fp32, summed in a fixed order).
- * latent (optional) is the z spin4d_heads_fwd saved; workspace as for
+ * latent and raw (optional, each may be NULL) are the z and the raw head
+ * outputs spin4d_heads_fwd saved for the same inputs; workspace as for
  * spin4d_decode_bwd, >= spin4d_heads_bwd_workspace bytes. */
 int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
-                     const void* tables, const void* weights, const float* latent,
+                     const void* tables, const void* weights, const float* latent, const float* raw,
                      const spin4d_heads_output_grads* grad_out, float* grad_tables, float* grad_weights,
                      void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 

@@ -36,7 +36,7 @@ struct HeadsParams {
 };
 
 struct HeadsOut {
-  float *scale, *rot, *sh, *opacity, *cov, *latent;
+  float *scale, *rot, *sh, *opacity, *cov, *latent, *raw;
 };
 struct HeadsGrads {
   const float *scale, *rot, *sh, *opacity, *cov;
@@ -219,8 +219,8 @@ __device__ __forceinline__ void wgrad_q(const float* d, const float* x, int n_ou
 template <typename T, int F, typename W>
 __global__ void __launch_bounds__(kBwdThreads) heads_bwd_kernel(
     GridParams g, HeadsParams hp, const float4* __restrict__ pos, int64_t N, const T* __restrict__ tables,
-    const W* __restrict__ weights, const float* __restrict__ latent, HeadsGrads go, float* __restrict__ grad_tables,
-    float* __restrict__ ws, int n_params) {
+    const W* __restrict__ weights, const float* __restrict__ latent, const float* __restrict__ raw_in, HeadsGrads go,
+    float* __restrict__ grad_tables, float* __restrict__ ws, int n_params) {
   constexpr int B = kHeadsBwdBlock;     // 32 positions
   extern __shared__ float sm[];
   float* z = sm;                        // [B][kQ]; after the last head, dz
@@ -264,9 +264,14 @@ __global__ void __launch_bounds__(kBwdThreads) heads_bwd_kernel(
       }
     }
     __syncthreads();
-    // ---- first pass: raw outputs of the scale, rotation and opacity heads ----
+    // ---- first pass: raw outputs of the scale, rotation and opacity heads
+    // (read from the forward's copy when given) ----
     float raw[8];
-    for (int h = 0; h < 4; ++h) {
+    if (raw_in && threadIdx.x < B && n0 + threadIdx.x < N) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) raw[i] = __ldg(raw_in + (n0 + threadIdx.x) * 8 + i);
+    }
+    for (int h = 0; h < 4 && !raw_in; ++h) {
       if (h == 2) continue;
       const W* w = weights + hp.off[h];
       stage_layer<W>(w, H, IN, Ws, bs);
@@ -467,7 +472,13 @@ __global__ void __launch_bounds__(kBwdThreads) heads_fwd_q_kernel(GridParams g, 
         for (int i = 0; i < rows; ++i) raw[base + i] = y[threadIdx.x * kQ + i];
       }
     }
-    if (threadIdx.x < B && n0 + threadIdx.x < N) store_heads(out, n0 + threadIdx.x, raw);
+    if (threadIdx.x < B && n0 + threadIdx.x < N) {
+      store_heads(out, n0 + threadIdx.x, raw);
+      if (out.raw) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out.raw[(n0 + threadIdx.x) * 8 + i] = raw[i];
+      }
+    }
   }
 }
 
@@ -534,14 +545,14 @@ struct HeadsLaunch {
     return launch_status();
   }
   static int bwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
-                 const void* weights, const float* latent, const HeadsGrads& go, float* grad_tables,
+                 const void* weights, const float* latent, const float* raw, const HeadsGrads& go, float* grad_tables,
                  float* grad_weights, float* ws, int n_params, cudaStream_t s) {
     auto k = heads_bwd_kernel<T, F, W>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
     if (e != cudaSuccess) return cuda_status(e);
     const int blocks = bwd_blocks(N);
     k<<<blocks, kBwdThreads, kBwdSmem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
-                                              static_cast<const T*>(tables), static_cast<const W*>(weights), latent,
+                                              static_cast<const T*>(tables), static_cast<const W*>(weights), latent, raw,
                                               go, grad_tables, ws, n_params);
     SPIN4D_CHECK(launch_status());
     heads_reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, n_params, grad_weights);
@@ -551,39 +562,39 @@ struct HeadsLaunch {
 
 template <typename T, int F>
 int dispatch_w(int wdt, bool bwd, const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N,
-               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const float* raw, const HeadsGrads* go,
                float* gt, float* gw, float* ws, int n_params, cudaStream_t s) {
   if (wdt == SPIN4D_F16) {
-    if (bwd) return HeadsLaunch<T, F, __half>::bwd(gp, hp, pos, N, tables, weights, latent, *go, gt, gw, ws, n_params, s);
+    if (bwd) return HeadsLaunch<T, F, __half>::bwd(gp, hp, pos, N, tables, weights, latent, raw, *go, gt, gw, ws, n_params, s);
     return HeadsLaunch<T, F, __half>::fwd(gp, hp, pos, N, tables, weights, *o, s);
   }
-  if (bwd) return HeadsLaunch<T, F, float>::bwd(gp, hp, pos, N, tables, weights, latent, *go, gt, gw, ws, n_params, s);
+  if (bwd) return HeadsLaunch<T, F, float>::bwd(gp, hp, pos, N, tables, weights, latent, raw, *go, gt, gw, ws, n_params, s);
   return HeadsLaunch<T, F, float>::fwd(gp, hp, pos, N, tables, weights, *o, s);
 }
 
 template <typename T>
 int dispatch_f(int F, int wdt, bool bwd, const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N,
-               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+               const void* tables, const void* weights, const HeadsOut* o, const float* latent, const float* raw, const HeadsGrads* go,
                float* gt, float* gw, float* ws, int n_params, cudaStream_t s) {
   switch (F) {
-    case 1: return dispatch_w<T, 1>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
-    case 2: return dispatch_w<T, 2>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
-    case 4: return dispatch_w<T, 4>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
-    case 8: return dispatch_w<T, 8>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws, n_params, s);
+    case 1: return dispatch_w<T, 1>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws, n_params, s);
+    case 2: return dispatch_w<T, 2>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws, n_params, s);
+    case 4: return dispatch_w<T, 4>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws, n_params, s);
+    case 8: return dispatch_w<T, 8>(wdt, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws, n_params, s);
     default: return SPIN4D_ERR_UNSUPPORTED;
   }
 }
 
 int run(const spin4d_grid_desc* g, const spin4d_heads_desc* h, bool bwd, const float* pos, int64_t N,
-        const void* tables, const void* weights, const HeadsOut* o, const float* latent, const HeadsGrads* go,
+        const void* tables, const void* weights, const HeadsOut* o, const float* latent, const float* raw, const HeadsGrads* go,
         float* gt, float* gw, float* ws, cudaStream_t s) {
   const GridParams gp = make_grid_params(g);
   const HeadsParams hp = make_heads(h);
   const int n_params = (int)param_count(h);
   if (g->table_dtype == SPIN4D_F16)
-    return dispatch_f<__half>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws,
+    return dispatch_f<__half>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws,
                               n_params, s);
-  return dispatch_f<float>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, go, gt, gw, ws,
+  return dispatch_f<float>(g->F, h->w_dtype, bwd, gp, hp, pos, N, tables, weights, o, latent, raw, go, gt, gw, ws,
                            n_params, s);
 }
 
@@ -617,8 +628,8 @@ extern "C" int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_de
   if (N == 0) return SPIN4D_OK;
   if (!out.scale || !out.rot || !out.sh || !out.opacity || !out.cov || !aligned(out.rot, 16)) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_heads_fwd")) return SPIN4D_ERR_INJECTED;
-  const HeadsOut o{out.scale, out.rot, out.sh, out.opacity, out.cov, out.latent};
-  return run(g, h, false, pos, N, tables, weights, &o, nullptr, nullptr, nullptr, nullptr, nullptr,
+  const HeadsOut o{out.scale, out.rot, out.sh, out.opacity, out.cov, out.latent, out.raw};
+  return run(g, h, false, pos, N, tables, weights, &o, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
              (cudaStream_t)stream);
 }
 
@@ -628,7 +639,7 @@ extern "C" size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const sp
 }
 
 extern "C" int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
-                                const void* tables, const void* weights, const float* latent,
+                                const void* tables, const void* weights, const float* latent, const float* raw,
                                 const spin4d_heads_output_grads* grad_out, float* grad_tables, float* grad_weights,
                                 void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
   SPIN4D_CHECK(check_inputs(g, h, pos, N, tables, weights));
@@ -639,6 +650,6 @@ extern "C" int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_de
     return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_heads_bwd")) return SPIN4D_ERR_INJECTED;
   const HeadsGrads go{grad_out->scale, grad_out->rot, grad_out->sh, grad_out->opacity, grad_out->cov};
-  return run(g, h, true, pos, N, tables, weights, nullptr, latent, &go, grad_tables, grad_weights,
+  return run(g, h, true, pos, N, tables, weights, nullptr, latent, raw, &go, grad_tables, grad_weights,
              static_cast<float*>(workspace), (cudaStream_t)stream);
 }

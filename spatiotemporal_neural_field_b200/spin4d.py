@@ -73,7 +73,8 @@ class HeadsDesc(ctypes.Structure):
 
 
 class HeadsOutputs(ctypes.Structure):
-    _fields_ = [("scale", c_vp), ("rot", c_vp), ("sh", c_vp), ("opacity", c_vp), ("cov", c_vp), ("latent", c_vp)]
+    _fields_ = [("scale", c_vp), ("rot", c_vp), ("sh", c_vp), ("opacity", c_vp), ("cov", c_vp), ("latent", c_vp),
+                ("raw", c_vp)]
 
 
 class HeadsOutputGrads(ctypes.Structure):
@@ -111,8 +112,8 @@ _SIGS = {
     "spin4d_heads_param_count": (c_i64, [P(HeadsDesc)]),
     "spin4d_heads_fwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, HeadsOutputs, c_vp]),
     "spin4d_heads_bwd_workspace": (c_sz, [P(GridDesc), P(HeadsDesc), c_i64]),
-    "spin4d_heads_bwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, c_vp, P(HeadsOutputGrads), c_vp,
-                                 c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_heads_bwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(HeadsOutputGrads),
+                                 c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_adam_step_groups": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, P(AdamGroup), c_i32, c_i32, c_f32,
                                         c_f32, c_f32, c_i32, c_vp, c_vp]),
     "spin4d_lr_warmup_cosine": (ctypes.c_double, [c_i64, ctypes.c_double, ctypes.c_double, c_i64, c_i64]),
@@ -352,28 +353,34 @@ def heads_param_count(h: HeadsDesc) -> int:
     return int(lib.spin4d_heads_param_count(ctypes.byref(h)))
 
 
-def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent: bool = False, stream=None):
+def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent: bool = False, raw: bool = False,
+              stream=None):
+    """Outputs dict; with latent / raw it also holds z (N x in_dim) and the
+    raw scale, rotation and opacity head outputs (N x 8) for heads_bwd."""
     N = pos.shape[0]
     widths = {"scale": 3, "rot": 4, "sh": h.sh_dim, "opacity": 1, "cov": 6}
     if out is None:
         out = {k: torch.empty((N, w), dtype=torch.float32, device=pos.device) for k, w in widths.items()}
         if latent:
             out["latent"] = torch.empty((N, h.in_dim), dtype=torch.float32, device=pos.device)
-    o = HeadsOutputs(*(_ptr(out[k]) for k in HEADS_KEYS), _ptr(out.get("latent")))
+        if raw:
+            out["raw"] = torch.empty((N, 8), dtype=torch.float32, device=pos.device)
+    o = HeadsOutputs(*(_ptr(out[k]) for k in HEADS_KEYS), _ptr(out.get("latent")), _ptr(out.get("raw")))
     _check("spin4d_heads_fwd", lib.spin4d_heads_fwd(ctypes.byref(g), ctypes.byref(h), _ptr(pos), N, _ptr(tables),
                                                     _ptr(weights), o, _stream(stream)))
     return out
 
 
 def heads_bwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, grads, grad_tables, grad_weights, latent=None,
-              workspace=None, stream=None) -> None:
+              workspace=None, stream=None, raw=None) -> None:
     N = pos.shape[0]
     if workspace is None:
         need = int(lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), N))
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=pos.device)
     go = HeadsOutputGrads(*(_ptr(grads.get(k)) for k in HEADS_KEYS))
     _check("spin4d_heads_bwd", lib.spin4d_heads_bwd(ctypes.byref(g), ctypes.byref(h), _ptr(pos), N, _ptr(tables),
-                                                    _ptr(weights), _ptr(latent), ctypes.byref(go), _ptr(grad_tables),
+                                                    _ptr(weights), _ptr(latent), _ptr(raw), ctypes.byref(go),
+                                                    _ptr(grad_tables),
                                                     _ptr(grad_weights), _ptr(workspace), workspace.numel(),
                                                     _stream(stream)))
 

@@ -56,18 +56,30 @@ def test_heads_forward_matches_oracle(sp, case):
         else:
             tol.absolute(host(out[k]), want[k], tol.FP16_ATOL, k)
     tol.rowwise(host(out["latent"]), want["z"], tol.FP32_RTOL, "latent")
+    # the raw head outputs the forward saves for the backward: Eq. 11 inverts them
+    raw = host(sp.heads_fwd(g, h, dev(pos), dev(tables), dev(weights), raw=True)["raw"]).astype(np.float64)
+    tol.absolute(np.exp(np.minimum(raw[:, :3], 20.0)), want["scale"], tol.FP16_ATOL, "raw scale")
+    tol.absolute(raw[:, 3:7] / np.linalg.norm(raw[:, 3:7], axis=1, keepdims=True), want["rot"], tol.FP16_ATOL,
+                 "raw rotation")
+    tol.absolute(1.0 / (1.0 + np.exp(-raw[:, 7])), want["opacity"][:, 0], tol.FP16_ATOL, "raw opacity")
 
 
-@pytest.mark.parametrize("case,latent", [("tiny_fp32", False), ("paper_fp16", False), ("paper_fp16", True),
-                                         ("paper_fp16_init", False)])
-def test_heads_backward_matches_oracle(sp, case, latent):
+@pytest.mark.parametrize("case,saved", [("tiny_fp32", ""), ("tiny_fp32", "latent+raw"), ("paper_fp16", ""),
+                                        ("paper_fp16", "latent"), ("paper_fp16", "raw"), ("paper_fp16", "latent+raw"),
+                                        ("paper_fp16_init", "")])
+def test_heads_backward_matches_oracle(sp, case, saved):
+    """With the forward's z and / or raw head outputs the backward skips the
+    gather and / or the first recompute of the scale, rotation and opacity
+    heads; the gradients are the same."""
     grid, spec, pos, tables, weights, grads = _setup(case)
     g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
     P, T, W = dev(pos), dev(tables), dev(weights)
-    lat = sp.heads_fwd(g, h, P, T, W, latent=True)["latent"] if latent else None
+    fw = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+    lat = fw["latent"] if "latent" in saved else None
+    raw = fw["raw"] if "raw" in saved else None
     gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
     gw = torch.zeros(spec.n_params(), device="cuda")
-    sp.heads_bwd(g, h, P, T, W, {k: dev(v) for k, v in grads.items()}, gt, gw, latent=lat)
+    sp.heads_bwd(g, h, P, T, W, {k: dev(v) for k, v in grads.items()}, gt, gw, latent=lat, raw=raw)
     wt, ww = hd.decode_backward(pos, tables, weights, grid, spec, grads)
     rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
     tol.normwise(host(gt), wt, rtol, "grad_tables")
@@ -162,7 +174,7 @@ def test_heads_full_launch_sampled_and_by_halves(sp):
     tables = S.hash_tables(grid, seed=11, scale=1.0)
     weights = S.heads_weights(spec, seed=12, bias_scale=0.3)
     P, T, W = dev(pos), dev(tables), dev(weights)
-    out = sp.heads_fwd(g, h, P, T, W, latent=True)
+    out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
     idx = np.random.default_rng(13).choice(n, 400, replace=False)
     want = hd.decode_forward(pos[idx], tables, weights, grid, spec)
     for k in ("scale", "rot", "sh", "opacity", "cov"):
@@ -172,11 +184,12 @@ def test_heads_full_launch_sampled_and_by_halves(sp):
          for k, wd in widths.items()}
     gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
     gw = torch.zeros(spec.n_params(), device="cuda")
-    sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=out["latent"])
+    sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=out["latent"], raw=out["raw"])
     gt2, gw2 = torch.zeros_like(gt), torch.zeros_like(gw)
     half = n // 2
     for a, b in ((0, half), (half, n)):
-        sp.heads_bwd(g, h, P[a:b], T, W, {k: v[a:b] for k, v in G.items()}, gt2, gw2, latent=out["latent"][a:b])
+        sp.heads_bwd(g, h, P[a:b], T, W, {k: v[a:b] for k, v in G.items()}, gt2, gw2, latent=out["latent"][a:b],
+                     raw=out["raw"][a:b])
     torch.cuda.synchronize()
     tol.normwise(host(gt2), host(gt), 1e-4, "grad_tables by halves")
     tol.normwise(host(gw2), host(gw), 1e-4, "grad_weights by halves")

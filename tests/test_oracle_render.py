@@ -334,3 +334,62 @@ def test_backward_matches_central_differences(deg):
             flat[p] = old
             fd = (lp - lm) / (2 * h)
             assert abs(got[p] - fd) <= 1e-6 * max(1.0, abs(fd)), (key, p, got[p], fd)
+
+
+def test_view_direction_runs_from_the_camera_centre():
+    """The camera centre is the point the view maps to the camera-space
+    origin; a degree-1 SH colour is sqrt(3/4pi) (k_y d_y + k_z d_z + k_x d_x)
+    in the direction from that centre to the Gaussian."""
+    spec = S.orbit_camera(32, 24, focal=30.0, azimuth_deg=40.0, elevation_deg=25.0)
+    cam = _cam(spec)
+    np.testing.assert_allclose(cam.R @ cam.centre + cam.t, 0.0, atol=1e-6)
+    eye = np.array([2.8 * math.cos(math.radians(25)) * math.sin(math.radians(40)), -2.8 * math.sin(math.radians(25)),
+                    -2.8 * math.cos(math.radians(25)) * math.cos(math.radians(40))])
+    np.testing.assert_allclose(cam.centre, eye, atol=1e-5)
+    mu = np.array([[0.1, -0.2, 0.05]])
+    k = np.zeros((1, 4, 3))
+    k[0, 1:4, 0] = [0.3, -0.2, 0.5]            # channel 0: Y_1,-1 (y), Y_1,0 (z), Y_1,1 (x)
+    k[0, 0, 1] = 1.0                           # channel 1: constant
+    rgb, pre, d, _ = rd.sh_colour(mu, k.reshape(1, 12), 1, cam.centre)
+    v = mu[0] - eye
+    v /= np.linalg.norm(v)
+    c1 = math.sqrt(3 / (4 * math.pi))
+    # the view matrix is stored in fp32, so the centre agrees with the exact eye to ~1e-7
+    np.testing.assert_allclose(pre[0, 0], c1 * (0.3 * v[1] - 0.2 * v[2] + 0.5 * v[0]), rtol=1e-6)
+    np.testing.assert_allclose(pre[0, 1], 1 / (2 * math.sqrt(math.pi)), rtol=1e-12)
+
+
+def test_backward_with_clamped_alpha_matches_central_differences():
+    """Opaque Gaussians (o = 1) reach alpha_max at their centres; where the
+    clamp holds, alpha does not move with o, the mean or Sigma."""
+    rng = np.random.default_rng(41)
+    cam = _cam(S.orbit_camera(20, 16, focal=18.0))
+    n = 10
+    sc = S.render_scene(n, seed=41, positions=rng.uniform(-0.35, 0.35, size=(n, 3)).astype(np.float32),
+                        sh_degree=-1, scale_factor=1.5)
+    sc = {k: v.astype(np.float64) for k, v in sc.items()}
+    sc["opacity"][:] = 1.0
+    st = rd.Settings(sh_degree=-1, alpha_max=0.99, t_stop=0.0, background=np.array([0.2, 0.5, 0.1]))
+    g = S.image_grads(S.orbit_camera(20, 16), seed=42).astype(np.float64)
+    pr = rd.project(cam, st, sc["mu"], sc["cov"], sc["opacity"], sc["colours"])
+    order = rd._depth_order(pr)
+    clamped = 0
+    for j in range(16):
+        for i in range(20):
+            _, _, idx, a, _, _, _ = rd.composite_pixel(i + 0.5, j + 0.5, pr, order, st)
+            clamped += int(np.sum(a == st.alpha_max))
+    assert clamped >= 3, "the scene must clamp some alphas"
+    grads = rd.render_backward(cam, st, sc["mu"], sc["cov"], sc["opacity"], sc["colours"], g)
+    h = 1e-6
+    for key in ("opacity", "mu", "cov"):
+        flat = sc[key].reshape(-1)
+        got = grads[key].reshape(-1)
+        for p in range(flat.size):
+            old = flat[p]
+            flat[p] = old + h
+            lp = _loss(cam, st, sc, g)
+            flat[p] = old - h
+            lm = _loss(cam, st, sc, g)
+            flat[p] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(got[p] - fd) <= 1e-6 * max(1.0, abs(fd)), (key, p, got[p], fd)

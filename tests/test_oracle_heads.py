@@ -118,3 +118,16 @@ def test_learning_rate_schedule():
     assert lr(1100) == 1e-7 and lr(5000) == 1e-7
     vals = [lr(s) for s in range(100, 1101)]
     assert all(a >= b for a, b in zip(vals, vals[1:]))
+
+
+def test_scale_clip_at_twenty():
+    """Eq. 11 with the page's clip: s = exp(min(s^, 20)), and no gradient to s^
+    where the clip holds."""
+    raw = dict(scale=np.array([[25.0, 19.0, 0.0]]), rot=np.array([[1.0, 0.0, 0.0, 0.0]]),
+               sh=np.zeros((1, 12)), opacity=np.zeros((1, 1)))
+    out = hd.activations(raw)
+    np.testing.assert_allclose(out["scale"][0], [math.exp(20.0), math.exp(19.0), 1.0], rtol=1e-15)
+    grads = dict(scale=np.ones((1, 3)), rot=np.zeros((1, 4)), sh=np.zeros((1, 12)), opacity=np.zeros((1, 1)),
+                 cov=np.zeros((1, 6)))
+    d = hd.activations_backward(raw, grads)["scale"][0]
+    np.testing.assert_allclose(d, [0.0, math.exp(19.0), 1.0], rtol=1e-15)

@@ -36,3 +36,14 @@ def test_z_order_locality_and_monotonicity():
 def test_order_is_a_stable_sort():
     keys = np.array([5, 3, 5, 0, 3, 3, 7], np.uint32)
     assert od.morton_order(keys).tolist() == [3, 1, 4, 5, 0, 2, 6]
+
+
+def test_keys_of_raw_positions():
+    """Through Eq. 7: inside the unit ball mu_bar = mu/4 + 1/2, so mu = (0.25, 0, -0.5)
+    and the origin have known cells; the timestamp does not enter the key."""
+    pos = np.array([[0.25, 0.0, -0.5, 0.0], [0.25, 0.0, -0.5, 0.9], [0.0, 0.0, 0.0, 0.3]], np.float32)
+    keys = od.morton_keys(pos, 0.0, 1.0)
+    # (0.25, 0, -0.5) -> mu_bar (0.5625, 0.5, 0.375) -> q (576, 512, 384)
+    want = od.interleave(np.array([[576, 512, 384]]))[0]
+    assert keys[0] == want and keys[1] == want
+    assert keys[2] == od.interleave(np.array([[512, 512, 512]]))[0]

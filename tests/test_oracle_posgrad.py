@@ -207,3 +207,31 @@ def test_gate_gradient_matches_central_differences():
         e[j] = h
         fd = (loss(cr + e) - loss(cr - e)) / (2 * h)
         np.testing.assert_allclose(gcr[:, j], fd, rtol=1e-6, atol=1e-7)
+
+
+def test_position_gradient_is_zero_where_the_clamp_holds():
+    """Normalised input outside [0, 1] is clamped, so the output does not move
+    with that coordinate: its central difference, and the gradient, are 0;
+    the in-range coordinates keep their central differences."""
+    h = 2.0 ** -18
+    base = _grid_positions(16, 14, h)
+    xt = base.copy()
+    xt[:8, 0] = -0.25                       # clamped below on x
+    xt[8:, 1] = 1.375                       # clamped above on y
+    tables = S.hash_tables(TINY, seed=15, scale=1.0)
+    weights = S.mlp_weights(S.MLP_TINY, seed=16, bias_scale=0.5)
+    grads = S.upstream_grads(len(xt), S.DECODE_OUT_WIDTHS, 1.0, seed=17)
+    _, _, gpos = dec.decode_backward(xt, tables, weights, TINY, S.MLP_TINY, grads, normalised_input=True,
+                                     want_pos=True)
+
+    def loss(x):
+        out = dec.decode_forward(x, tables, weights, TINY, S.MLP_TINY, normalised_input=True)
+        return sum(np.sum(np.asarray(grads[k], np.float64) * out[k], axis=1) for k in grads)
+
+    for d in range(3):
+        e = np.zeros(4, np.float32)
+        e[d] = h
+        fd = (loss(xt + e) - loss(xt - e)) / (2 * h)
+        np.testing.assert_allclose(gpos[:, d], fd, rtol=1e-6, atol=1e-6)
+    assert np.all(gpos[:8, 0] == 0.0) and np.all(gpos[8:, 1] == 0.0)
+    assert np.abs(gpos[:8, 1:]).max() > 1e-3 and np.abs(gpos[8:, [0, 2]]).max() > 1e-3

@@ -335,6 +335,7 @@ __device__ __forceinline__ float mahalanobis2(float4 co, float dx, float dy) {
 // blocks), lane (lane & 7, lane >> 3) in it, and skips as a whole the
 // Gaussians whose support box misses its block.
 constexpr int kRastThreads = 256;
+constexpr int kFewLanes = 10;   // backward: up to this many blending lanes add directly, more reduce first
 
 struct TileGeom {
   int px, py;                   // the lane's pixel
@@ -555,10 +556,20 @@ __global__ void __launch_bounds__(kRastThreads) rasterise_bwd(Blend b, int W, in
       if (jidx >= warp_last || box_misses(m, g)) continue;
       float v[16] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const bool hit = grad_step(q, jidx, s_co[j], m, s_rgb[j], b, v);
-      if (__any_sync(0xffffffffu, hit)) {
-        const float total = warp_transpose_sum16(v, lane);
-        const int k = (lane >> 1) & 15;
-        if ((lane & 1) == 0 && k < 9) atomicAdd(reinterpret_cast<float*>(gacc + 3 * (int64_t)s_id[j]) + k, total);
+      const uint32_t hits = __ballot_sync(0xffffffffu, hit);
+      if (hits) {
+        float* gq = reinterpret_cast<float*>(gacc + 3 * (int64_t)s_id[j]);
+        if (__popc(hits) <= kFewLanes) {
+          // a few lanes: each adds its own nine values (cheaper than the reduction)
+          if (hit) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) atomicAdd(gq + k, v[k]);
+          }
+        } else {
+          const float total = warp_transpose_sum16(v, lane);
+          const int k = (lane >> 1) & 15;
+          if ((lane & 1) == 0 && k < 9) atomicAdd(gq + k, total);
+        }
       }
     }
     hi = lo;

@@ -10,11 +10,14 @@
 // count at run time.  That count may live on the device (n_dev, clamped to
 // the capacity), so a sort can follow a kernel that produced a
 // data-dependent number of keys without a host sync, and the scan stays
-// sized by the grid, not by the capacity.
+// sized by the grid, not by the capacity.  The kernels of a sort are
+// launched as programmatic dependents of each other (pdl.cuh).
 #pragma once
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include "pdl.cuh"
 
 namespace spin4d {
 namespace radix {
@@ -51,6 +54,8 @@ __device__ __forceinline__ void block_chunk(int64_t N, const uint32_t* n_dev, in
 __global__ void __launch_bounds__(kSortThreads) radix_histogram(const uint32_t* __restrict__ keys, int64_t N,
                                                                 const uint32_t* __restrict__ n_dev, int shift,
                                                                 uint32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_release();
   __shared__ uint32_t h[kDigits];
   h[threadIdx.x] = 0;
   __syncthreads();
@@ -108,6 +113,8 @@ __device__ __forceinline__ void load_chunk(const uint32_t* __restrict__ a, int64
 // Scan step 1: partial[c] = sum of chunk c of a.
 __global__ void __launch_bounds__(kScanThreads) scan_reduce(const uint32_t* __restrict__ a, int64_t n,
                                                             uint32_t* __restrict__ partial) {
+  pdl_wait();
+  pdl_release();
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t sm[kScanShared];
   load_chunk(a, n, sm);
@@ -121,6 +128,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_reduce(const uint32_t* __re
 
 // Scan step 2 for many chunks (one block): partial[] -> its exclusive scan, in place.
 __global__ void __launch_bounds__(kScanThreads) scan_partials(uint32_t* __restrict__ partial, int n) {
+  pdl_wait();
+  pdl_release();
   __shared__ uint32_t s_warp[32];
   uint32_t carry = 0;
   for (int base = 0; base < n; base += kScanThreads) {
@@ -140,6 +149,8 @@ template <bool FUSED>
 __global__ void __launch_bounds__(kScanThreads) scan_apply(const uint32_t* __restrict__ a, int64_t n,
                                                            const uint32_t* __restrict__ partial,
                                                            uint32_t* __restrict__ out) {
+  pdl_wait();
+  pdl_release();
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_base;
   __shared__ uint32_t sm[kScanShared];
@@ -186,6 +197,8 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter(const uint32_t* __
                                                               int shift, const uint32_t* __restrict__ offsets,
                                                               uint32_t* __restrict__ keys_out,
                                                               uint32_t* __restrict__ vals_out) {
+  pdl_wait();
+  pdl_release();
   constexpr int kWarps = kSortThreads / 32;
   __shared__ uint32_t base[kDigits];          // global position of this block's next key of each digit
   __shared__ uint32_t wcnt[kWarps][kDigits];  // per round: keys per (warp, digit), then their prefix
@@ -239,12 +252,12 @@ inline size_t exclusive_scan_scratch(int64_t n) { return align256((size_t)scan_c
 inline void exclusive_scan(const uint32_t* a, int64_t n, uint32_t* out, void* scratch, cudaStream_t s) {
   const int chunks = (int)scan_chunks(n);
   uint32_t* partial = static_cast<uint32_t*>(scratch);
-  scan_reduce<<<chunks, kScanThreads, 0, s>>>(a, n, partial);
+  launch_pdl(scan_reduce, chunks, kScanThreads, 0, s, a, n, partial);
   if (chunks <= kFusedScanMaxChunks) {
-    scan_apply<true><<<chunks, kScanThreads, 0, s>>>(a, n, partial, out);
+    launch_pdl(scan_apply<true>, chunks, kScanThreads, 0, s, a, n, partial, out);
   } else {
-    scan_partials<<<1, kScanThreads, 0, s>>>(partial, chunks);
-    scan_apply<false><<<chunks, kScanThreads, 0, s>>>(a, n, partial, out);
+    launch_pdl(scan_partials, 1, kScanThreads, 0, s, partial, chunks);
+    launch_pdl(scan_apply<false>, chunks, kScanThreads, 0, s, a, n, partial, out);
   }
 }
 
@@ -269,10 +282,10 @@ inline bool sort_pairs(uint32_t* keys, uint32_t* vals, uint32_t* keys_b, uint32_
   uint32_t *ka = keys, *kb = keys_b, *va = vals, *vb = vals_b;
   for (int pass = 0; pass < passes; ++pass) {
     const int shift = 8 * pass;
-    radix_histogram<<<B, kSortThreads, 0, s>>>(ka, N, n_dev, shift, counts);
+    launch_pdl(radix_histogram, B, kSortThreads, 0, s, ka, N, n_dev, shift, counts);
     exclusive_scan(counts, len, offsets, scan_scratch, s);
-    radix_scatter<<<B, kSortThreads, 0, s>>>(ka, (pass == 0 && vals_are_index) ? nullptr : va, N, n_dev, shift,
-                                             offsets, kb, vb);
+    launch_pdl(radix_scatter, B, kSortThreads, 0, s, ka, (pass == 0 && vals_are_index) ? nullptr : va, N, n_dev,
+               shift, offsets, kb, vb);
     uint32_t* t = ka; ka = kb; kb = t;
     t = va; va = vb; vb = t;
   }

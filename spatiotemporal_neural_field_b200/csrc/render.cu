@@ -2,7 +2,9 @@
 // (SPIN-4DGS section 3.1: Eq. 1 Gaussian, Eq. 3 Sigma_2D = J W Sigma W^T J^T,
 // Eq. 4 front-to-back blending C = sum_i c_i a_i prod_{j<i} (1 - a_j)).
 //
-// Forward, all on one stream, no host synchronisation (graph-capturable):
+// Forward, all on one stream, no host synchronisation (graph-capturable;
+// every kernel after the projection is a programmatic dependent launch of
+// the one before it, see pdl.cuh):
 //  1. project_kernel, one thread per Gaussian: camera transform, Eq. 3 with
 //     the screen-space filter, conic, colour from the spherical harmonics,
 //     the box of pixels its support can reach and the 16x16 tiles it spans.
@@ -32,6 +34,7 @@
 #include <algorithm>
 
 #include "host.h"
+#include "pdl.cuh"
 #include "radix.cuh"
 
 namespace spin4d {
@@ -199,6 +202,8 @@ __global__ void __launch_bounds__(kProjThreads) project_kernel(
     const float* __restrict__ opacity, const float* __restrict__ colours, float4* __restrict__ conic_o,
     float4* __restrict__ xy, float4* __restrict__ rgb, uint2* __restrict__ rect, uint32_t* __restrict__ ntiles,
     uint32_t* __restrict__ dkey) {
+  pdl_wait();
+  pdl_release();
   using CT = ColourTile<DEG>;
   constexpr int K = DEG < 0 ? 1 : (DEG + 1) * (DEG + 1);
   __shared__ float s_col[CT::kStaged ? kProjThreads * CT::kPitch : 1];
@@ -272,6 +277,8 @@ __global__ void __launch_bounds__(kProjThreads) project_kernel(
 // exact 64-bit total (the 32-bit scan that follows may wrap; see emit_pairs)
 __global__ void counts_in_order(const uint32_t* __restrict__ perm, const uint32_t* __restrict__ ntiles, int64_t N,
                                 uint32_t* __restrict__ cnt, uint32_t* __restrict__ header) {
+  pdl_wait();
+  pdl_release();
   uint64_t local = 0;
   for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < N; k += (int64_t)gridDim.x * blockDim.x) {
     const uint32_t c = ntiles[perm[k]];
@@ -286,6 +293,8 @@ __global__ void counts_in_order(const uint32_t* __restrict__ perm, const uint32_
 // first `cap` when they do not, none when the total overflows 32 bits (the
 // scan's offsets would then wrap and could leave slots unwritten).
 __global__ void clamp_pair_count(uint32_t* header, uint32_t cap) {
+  pdl_wait();
+  pdl_release();
   const uint64_t need = *reinterpret_cast<const unsigned long long*>(header);
   header[2] = need > 0xFFFFFFFFull ? 0u : (need > cap ? cap : (uint32_t)need);
 }
@@ -296,6 +305,8 @@ __global__ void emit_pairs(const uint32_t* __restrict__ perm, const uint32_t* __
                            const uint32_t* __restrict__ offs, const uint2* __restrict__ rect, int64_t N, int tiles_x,
                            const uint32_t* __restrict__ header, uint32_t* __restrict__ pair_tile,
                            uint32_t* __restrict__ pair_id) {
+  pdl_wait();
+  pdl_release();
   const uint32_t kept = header[2];
   for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < N; k += (int64_t)gridDim.x * blockDim.x) {
     const uint32_t c = cnt[k];
@@ -314,6 +325,8 @@ __global__ void emit_pairs(const uint32_t* __restrict__ perm, const uint32_t* __
 
 __global__ void tile_ranges_kernel(const uint32_t* __restrict__ tile, const uint32_t* __restrict__ header,
                                    int64_t cap, uint32_t n_tiles, uint2* __restrict__ ranges) {
+  pdl_wait();
+  pdl_release();
   const int64_t n = min((int64_t)header[2], cap);
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const uint32_t t = tile[i];
@@ -410,6 +423,8 @@ __global__ void __launch_bounds__(kRastThreads) rasterise_fwd(Blend b, int W, in
                                                              float* __restrict__ final_T,
                                                              uint32_t* __restrict__ n_contrib,
                                                              float* __restrict__ final_T_out) {
+  pdl_wait();
+  pdl_release();
   __shared__ float4 s_co[kRastThreads];
   __shared__ float4 s_xy[kRastThreads];
   __shared__ float4 s_rgb[kRastThreads];
@@ -522,6 +537,7 @@ __global__ void __launch_bounds__(kRastThreads) rasterise_bwd(Blend b, int W, in
                                                              const uint32_t* __restrict__ n_contrib,
                                                              const float* __restrict__ grad_image,
                                                              float4* __restrict__ gacc) {
+  pdl_release();   // the projection backward may launch; it waits for this grid in its pdl_wait
   __shared__ float4 s_co[kRastThreads];
   __shared__ float4 s_xy[kRastThreads];
   __shared__ float4 s_rgb[kRastThreads];
@@ -582,6 +598,8 @@ __global__ void __launch_bounds__(kProjThreads) project_bwd_kernel(
     const float* __restrict__ opacity, const float* __restrict__ colours, const float4* __restrict__ gacc,
     float* __restrict__ grad_means, float* __restrict__ grad_cov, float* __restrict__ grad_opacity,
     float* __restrict__ grad_colours) {
+  pdl_wait();
+  pdl_release();
   using CT = ColourTile<DEG>;
   constexpr int K = DEG < 0 ? 1 : (DEG + 1) * (DEG + 1);
   // the tile's SH rows; each thread overwrites its own row with its SH
@@ -874,11 +892,11 @@ extern "C" int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_d
                       at<void>(state, L.scratch), s);
     uint32_t* cnt = at<uint32_t>(state, L.cnt);
     uint32_t* offs = at<uint32_t>(state, L.offs);
-    counts_in_order<<<blocks, 256, 0, s>>>(dperm, at<uint32_t>(state, L.ntiles), N, cnt, header);
-    clamp_pair_count<<<1, 1, 0, s>>>(header, (uint32_t)max_pairs);
+    launch_pdl(counts_in_order, blocks, 256, 0, s, dperm, at<uint32_t>(state, L.ntiles), N, cnt, header);
+    launch_pdl(clamp_pair_count, 1, 1, 0, s, header, (uint32_t)max_pairs);
     radix::exclusive_scan(cnt, N, offs, at<void>(state, L.scratch), s);
-    emit_pairs<<<blocks, 256, 0, s>>>(dperm, cnt, offs, at<uint2>(state, L.rect), N, b.tiles_x, header, pair_tile,
-                                      pair_id);
+    launch_pdl(emit_pairs, blocks, 256, 0, s, dperm, cnt, offs, at<uint2>(state, L.rect), N, b.tiles_x, header,
+               pair_tile, pair_id);
     SPIN4D_CHECK(launch_status());
     const int passes = tile_sort_passes(n_tiles);
     if (passes > 0 && max_pairs > 0) {
@@ -891,14 +909,14 @@ extern "C" int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_d
       }
     }
     if (max_pairs > 0)
-      tile_ranges_kernel<<<persistent_blocks((max_pairs + 255) / 256, 8), 256, 0, s>>>(
-          pair_tile, header, max_pairs, (uint32_t)n_tiles, at<uint2>(state, L.ranges));
+      launch_pdl(tile_ranges_kernel, persistent_blocks((max_pairs + 255) / 256, 8), 256, 0, s, pair_tile,
+                 (const uint32_t*)header, max_pairs, (uint32_t)n_tiles, at<uint2>(state, L.ranges));
     SPIN4D_CHECK(launch_status());
   }
-  rasterise_fwd<<<n_tiles, kRastThreads, 0, s>>>(b, c.W, c.H, at<uint2>(state, L.ranges), pair_id,
-                                                at<float4>(state, L.conic_o), at<float4>(state, L.xy),
-                                                at<float4>(state, L.rgb), image, at<float>(state, L.final_T),
-                                                at<uint32_t>(state, L.n_contrib), final_T);
+  launch_pdl(rasterise_fwd, n_tiles, kRastThreads, 0, s, b, c.W, c.H, (const uint2*)at<uint2>(state, L.ranges),
+             (const uint32_t*)pair_id, (const float4*)at<float4>(state, L.conic_o),
+             (const float4*)at<float4>(state, L.xy), (const float4*)at<float4>(state, L.rgb), image,
+             at<float>(state, L.final_T), at<uint32_t>(state, L.n_contrib), final_T);
   return launch_status();
 }
 
@@ -931,9 +949,9 @@ extern "C" int spin4d_render_bwd(const spin4d_camera* cam, const spin4d_render_d
                                                 at<uint32_t>(state, L.n_contrib), grad_image, gacc);
   SPIN4D_CHECK(launch_status());
   const int pblocks = persistent_blocks((N + kProjThreads - 1) / kProjThreads, 8);
-#define SPIN4D_PROJECT_BWD(DEG)                                                                                  \
-  project_bwd_kernel<DEG><<<pblocks, kProjThreads, 0, s>>>(c, b, N, means, cov, opacity, colours, gacc, grad_means, \
-                                                           grad_cov, grad_opacity, grad_colours)
+#define SPIN4D_PROJECT_BWD(DEG)                                                                                 \
+  launch_pdl(project_bwd_kernel<DEG>, pblocks, kProjThreads, 0, s, c, b, N, means, cov, opacity, colours,          \
+             (const float4*)gacc, grad_means, grad_cov, grad_opacity, grad_colours)
   switch (b.sh_degree) {
     case -1: SPIN4D_PROJECT_BWD(-1); break;
     case 0: SPIN4D_PROJECT_BWD(0); break;

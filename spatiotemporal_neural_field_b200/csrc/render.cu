@@ -375,6 +375,28 @@ __device__ __forceinline__ bool box_misses(const float4& m, const TileGeom& g) {
   return m.x + m.z < g.wx0 || m.x - m.z > g.wx1 || m.y + m.w < g.wy0 || m.y - m.w > g.wy1;
 }
 
+// Bit w set when the Gaussian's support box (centre m.xy, half-widths m.zw)
+// reaches warp w's block of this tile (pixel centres bx + 0.5 .. bx + 7.5,
+// by + 0.5 .. by + 3.5 for block (w & 1, w >> 1)); computed once per batch
+// entry, so each warp then tests one bit.
+__device__ __forceinline__ uint32_t block_mask(const float4& m, const Blend& b) {
+  const int tile = blockIdx.x;
+  const float x0 = (float)((tile % b.tiles_x) * kTileSide), y0 = (float)((tile / b.tiles_x) * kTileSide);
+  const float lx = m.x - m.z, hx = m.x + m.z, ly = m.y - m.w, hy = m.y + m.w;
+  uint32_t cols = 0, rows = 0;
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+    if (hx >= x0 + 8.0f * c + 0.5f && lx <= x0 + 8.0f * c + 7.5f) cols |= 1u << c;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    if (hy >= y0 + 4.0f * r + 0.5f && ly <= y0 + 4.0f * r + 3.5f) rows |= 1u << r;
+  uint32_t mask = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w)
+    if (((cols >> (w & 1)) & 1u) && ((rows >> (w >> 1)) & 1u)) mask |= 1u << w;
+  return mask;
+}
+
 struct FwdPix {
   float fx, fy, T, c0, c1, c2;
   uint32_t last;
@@ -428,7 +450,9 @@ __global__ void __launch_bounds__(kRastThreads) rasterise_fwd(Blend b, int W, in
   __shared__ float4 s_co[kRastThreads];
   __shared__ float4 s_xy[kRastThreads];
   __shared__ float4 s_rgb[kRastThreads];
+  __shared__ uint8_t s_mask[kRastThreads];
   const TileGeom g = tile_geom(b);
+  const uint32_t wbit = 1u << (threadIdx.x >> 5);
   FwdPix q{(float)g.px + 0.5f, (float)g.py + 0.5f, 1.0f, 0.f, 0.f, 0.f, 0u, !(g.px < W && g.py < H)};
   const uint2 range = ranges[blockIdx.x];
   for (uint32_t base = range.x; base < range.y; base += kRastThreads) {
@@ -438,15 +462,16 @@ __global__ void __launch_bounds__(kRastThreads) rasterise_fwd(Blend b, int W, in
     if (i < range.y) {
       const uint32_t id = pair_id[i];
       s_co[threadIdx.x] = conic_o[id];
-      s_xy[threadIdx.x] = xy[id];
+      const float4 m = xy[id];
+      s_xy[threadIdx.x] = m;
       s_rgb[threadIdx.x] = rgb[id];
+      s_mask[threadIdx.x] = (uint8_t)block_mask(m, b);
     }
     __syncthreads();
     const int cnt = (int)min((uint32_t)kRastThreads, range.y - base);
     for (int j = 0; j < cnt && !q.done; ++j) {
-      const float4 m = s_xy[j];
-      if (box_misses(m, g)) continue;
-      blend_step(q, s_co[j], m, s_rgb[j], b, base - range.x + j + 1);
+      if (!(s_mask[j] & wbit)) continue;   // the same for the whole warp
+      blend_step(q, s_co[j], s_xy[j], s_rgb[j], b, base - range.x + j + 1);
     }
   }
   store_pixel(q, g.px, g.py, W, H, b, image, final_T, n_contrib, final_T_out);

@@ -667,6 +667,14 @@ def run_workloads(args):
     emit("paper_heads_fp16", "fwd", n, ms, table_sectors_per_position=spp, sector_rate=spp * n / (ms * 1e-3),
          frac_of_hbm_random_sector_ceiling=spp * n / (ms * 1e-3) / ceil["hbm_random_sector_per_s"],
          mlp_flop_per_position=2 * sum(o * i for hd_ in range(4) for o, i in spec.layer_shapes(hd_)))
+    # the same launch decoded in Z-order (sorted once per scene; outputs in sorted order)
+    ws_sort = torch.empty(max(sp.lib.spin4d_morton_order_workspace(n), 1), dtype=torch.uint8, device=dev)
+    _, perm = sp.morton_order(g, P, workspace=ws_sort)
+    Ps = sp.permute_rows(P, perm)
+    ms_s = timed(lambda: sp.heads_fwd(g, h, Ps, T, W, out=fwd_out), 10)
+    emit("paper_heads_fp16", "fwd (Z-order sorted)", n, ms_s, table_sectors_per_position=spp,
+         sector_rate=spp * n / (ms_s * 1e-3))
+    del Ps, perm, ws_sort
     grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
              for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim).items()}
     gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)

@@ -853,13 +853,12 @@ T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
 }
 
-int check_inputs(const spin4d_render_desc* d, int64_t N, const float* means, const float* cov, const float* opacity,
-                 const float* colours, void* state, size_t state_bytes, size_t need) {
+int check_inputs(int64_t N, const float* means, const float* cov, const float* opacity, const float* colours,
+                 void* state, size_t state_bytes, size_t need) {
   if (N > 0 && (!means || !cov || !opacity || !colours)) return SPIN4D_ERR_INVALID;
   if (!state || !aligned(state, 256) || state_bytes < need) return SPIN4D_ERR_INVALID;
   if (N > 0 && (!aligned(means, 4) || !aligned(cov, 4) || !aligned(opacity, 4) || !aligned(colours, 4)))
     return SPIN4D_ERR_INVALID;
-  (void)d;
   return SPIN4D_OK;
 }
 
@@ -881,7 +880,7 @@ extern "C" int spin4d_render_fwd(const spin4d_camera* cam, const spin4d_render_d
                                  spin4d_stream_t stream) {
   SPIN4D_CHECK(validate_render(cam, desc, N, max_pairs));
   const StateLayout L = state_layout(N, cam->width, cam->height, max_pairs);
-  SPIN4D_CHECK(check_inputs(desc, N, means, cov, opacity, colours, state, state_bytes, L.total));
+  SPIN4D_CHECK(check_inputs(N, means, cov, opacity, colours, state, state_bytes, L.total));
   if (!image || !aligned(image, 4) || (final_T && !aligned(final_T, 4))) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_render_fwd")) return SPIN4D_ERR_INJECTED;
   cudaStream_t s = (cudaStream_t)stream;
@@ -952,7 +951,7 @@ extern "C" int spin4d_render_bwd(const spin4d_camera* cam, const spin4d_render_d
                                  spin4d_stream_t stream) {
   SPIN4D_CHECK(validate_render(cam, desc, N, max_pairs));
   const StateLayout L = state_layout(N, cam->width, cam->height, max_pairs);
-  SPIN4D_CHECK(check_inputs(desc, N, means, cov, opacity, colours, state, state_bytes, L.total));
+  SPIN4D_CHECK(check_inputs(N, means, cov, opacity, colours, state, state_bytes, L.total));
   if (!grad_image || !aligned(grad_image, 4)) return SPIN4D_ERR_INVALID;
   for (const float* g : {grad_means, grad_cov, grad_opacity, grad_colours})
     if (g && !aligned(g, 4)) return SPIN4D_ERR_INVALID;

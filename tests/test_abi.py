@@ -189,3 +189,49 @@ def test_learning_rate_schedule_matches_oracle(sp):
     for args in ((8e-3, 1e-7, 100, 1100), (1e-3, 1e-7, 0, 40000), (3e-5, 1e-7, 500, 500)):
         for step in (1, 2, 50, 99, 100, 101, 600, 1099, 1100, 1101, 40000, 50000):
             assert abs(sp.lr_warmup_cosine(step, *args) - hd.lr_warmup_cosine(step, *args)) <= 1e-12 * args[0]
+
+
+def test_render_arguments_rejected_on_host(sp):
+    """Every argument of the renderer is checked before a launch."""
+    from spatiotemporal_neural_field_b200 import synthetic as S
+    lib, ref = sp.lib, ctypes.byref
+    cam = sp.camera_from_spec(S.orbit_camera(64, 48))
+    desc = sp.render_desc(sh_degree=3)
+    need = lib.spin4d_render_state_bytes(100, 64, 48, 4096)
+    assert need > 0
+    assert lib.spin4d_render_state_bytes(100, 0, 48, 4096) == 0
+    assert lib.spin4d_render_state_bytes(-1, 64, 48, 4096) == 0
+    assert lib.spin4d_render_state_bytes(100, 64, 48, -5) == 0
+
+    def fwd(c=cam, d=desc, n=100, state=FAKE, nbytes=need, cap=4096, image=FAKE):
+        return lib.spin4d_render_fwd(ref(c), ref(d), n, FAKE, FAKE, FAKE, FAKE, image, None, state, nbytes, cap,
+                                     None)
+
+    def bad_cam(**kw):
+        c = sp.camera_from_spec(S.orbit_camera(64, 48))
+        for k, v in kw.items():
+            setattr(c, k, v)
+        return c
+
+    def bad_desc(**kw):
+        d = sp.render_desc(sh_degree=3)
+        for k, v in kw.items():
+            setattr(d, k, v)
+        return d
+
+    assert fwd(c=bad_cam(width=0)) == sp.ERR_INVALID
+    assert fwd(c=bad_cam(fx=0.0)) == sp.ERR_INVALID
+    assert fwd(c=bad_cam(z_near=0.0)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(sh_degree=4)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(alpha_max=1.0)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(alpha_min=0.99)) == sp.ERR_INVALID      # not below alpha_max
+    assert fwd(d=bad_desc(t_stop=1.0)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(lowpass=-1.0)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(mean_stride=5)) == sp.ERR_INVALID
+    assert fwd(d=bad_desc(reserved=1)) == sp.ERR_INVALID
+    assert fwd(n=-1) == sp.ERR_INVALID
+    assert fwd(nbytes=need - 1) == sp.ERR_INVALID                  # state too small
+    assert fwd(state=FAKE + 16) == sp.ERR_INVALID                  # state not 256-byte aligned
+    assert fwd(image=None) == sp.ERR_INVALID
+    assert lib.spin4d_render_bwd(ref(cam), ref(desc), 100, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, 4096,
+                                 None, None, None, None, None) == sp.ERR_INVALID   # no upstream gradient

@@ -46,7 +46,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fwd-bwd", action="store_true")
-    p.add_argument("--cpu-sample", type=int, default=150_000, help="positions the oracle decodes for cpu_baseline")
+    p.add_argument("--cpu-sample", type=int, default=300_000,
+                   help="positions the oracle decodes for cpu_baseline (the whole frame: ~10 s on one core)")
     p.add_argument("--no-probe", action="store_true", help="skip the random-gather ceiling measurement")
     p.add_argument("--workloads", action="store_true",
                    help="time every workload (fwd, and fwd+bwd where trained) and the device ceilings; "

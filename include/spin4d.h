@@ -379,7 +379,11 @@ int spin4d_check_device_errors(int clear);
  * Weights (fp32 or fp16, 4-byte aligned) are packed head by head in that
  * order, each [W1 b1 W2 b2 W3 b3] with W[out][in] row-major.
  * in_dim = L*F; in_dim, hidden and sh_dim at most 64, in_dim and hidden
- * multiples of 4 (SPIN4D_ERR_UNSUPPORTED otherwise).  fp32 arithmetic.
+ * multiples of 4 (SPIN4D_ERR_UNSUPPORTED otherwise).  fp32 arithmetic, except
+ * that the forward with fp16 tables and weights, F = 4, in_dim = hidden = 64,
+ * sh_dim a multiple of 16 up to 48 and 16-byte aligned sh and raw runs its
+ * layers on the tensor cores: z and the hidden activations are rounded to
+ * fp16, products accumulate in fp32 (the latent output stays fp32).
  */
 typedef struct spin4d_heads_desc {
     int32_t in_dim;

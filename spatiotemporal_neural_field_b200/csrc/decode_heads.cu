@@ -11,7 +11,10 @@
 // tables) the corner gathers come from HBM and bound the forward.
 //
 // Forward: gather z, then per head two GELU layers and the output layer,
-// then Eq. 11 and Eq. 2.
+// then Eq. 11 and Eq. 2.  With fp16 tables and weights, in_dim = hidden =
+// 64 and an SH head of 16, 32 or 48 rows (the paper's configuration) the
+// layers run on the tensor cores instead (heads_fwd_tc_kernel): z and the
+// hidden activations rounded to fp16, fp32 accumulation.
 // Backward: forward again keeping the raw outputs of the scale, rotation
 // and opacity heads (they couple through Sigma), the activations' adjoint,
 // then per head the forward again with its pre-activations, the data
@@ -22,8 +25,25 @@
 #include <type_traits>
 
 #include "host.h"
+#include "tc.cuh"
 
 namespace spin4d {
+
+// Set when a bounded wait of the tensor-core forward runs out.
+__device__ int g_heads_device_error = 0;
+
+int heads_device_error(int clear) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_heads_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (clear && v) {
+    int zero = 0;
+    e = cudaMemcpyToSymbol(g_heads_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return v ? SPIN4D_ERR_TIMEOUT : SPIN4D_OK;
+}
+
 namespace {
 
 constexpr int kHeadsBwdBlock = 32;   // positions per block (forward and backward)
@@ -484,6 +504,251 @@ __global__ void __launch_bounds__(kBwdThreads) heads_fwd_q_kernel(GridParams g, 
 
 constexpr size_t kFwdQSmem = ((size_t)3 * kHeadsBwdBlock * kQ + (size_t)kMaxDim * kQ + kMaxDim) * sizeof(float);
 
+// ---------------------------------------------------------------------------
+// Forward on the tensor cores, for fp16 tables and weights with in_dim =
+// hidden = 64 (the paper's configuration) and an SH head of 16, 32 or 48
+// rows.  Persistent CTAs of 256 threads take tiles of 128 positions, two
+// threads per position (each gathers half of the levels and handles half of
+// every layer's columns).  z is rounded to fp16 into a K-major operand tile;
+// then, head by head, three tcgen05.mma chains (M = 128, K = 64; N = 64,
+// 64 and the head's rows padded to 16) run with the fp32 accumulators in
+// tensor memory: columns 0-63 for the two hidden layers, 64 onwards for the
+// output layer.  Each hidden epilogue reads a thread's 32 columns, adds the
+// bias, applies the exact GELU and writes the next fp16 operand tile.  All
+// weights are staged once per CTA (112 KB of shared memory with the tiles,
+// so two CTAs share an SM and one gathers while the other multiplies).
+// Every mbarrier wait is bounded; one that runs out sets a device error word
+// and the CTA releases its tensor memory and exits.
+// ---------------------------------------------------------------------------
+constexpr int kHT = 128;
+constexpr int kHTThreads = 256;
+constexpr int kHTMaxSh = 48;
+constexpr uint32_t kHTWait = 1u << 24;
+constexpr uint32_t kHTCols = 128;
+
+struct HeadsTcLayout {
+  static constexpr int W1 = 0;                                   // 4 x [64][64] fp16, K-major
+  static constexpr int W2 = W1 + 4 * 64 * 64 * 2;                // 4 x [64][64]
+  static constexpr int W3 = W2 + 4 * 64 * 64 * 2;                // [16 | 16 | sh | 16 rows][64]
+  static constexpr int kW3Rows = 48 + kHTMaxSh;
+  static constexpr int BIAS = W3 + kW3Rows * 64 * 2;             // fp32: b1 4x64, b2 4x64, b3 kW3Rows
+  static constexpr int ZT = BIAS + (512 + kW3Rows) * 4;          // [128][64] fp16
+  static constexpr int HT = ZT + kHT * 64 * 2;                   // [128][64] fp16
+  static constexpr int MISC = HT + kHT * 64 * 2;                 // mbarrier, TMEM address
+  static constexpr int BYTES = MISC + 16;
+};
+static_assert(HeadsTcLayout::ZT % 128 == 0 && HeadsTcLayout::W3 % 128 == 0, "operand tiles 128-byte aligned");
+
+// W[rows][K] (fp16, row-major in global memory, any 2-byte alignment) -> a
+// K-major tile of `rows_pad` rows, the rows past `rows` zero.
+__device__ __forceinline__ void stage_kmajor(uint8_t* sm, int soff, const __half* __restrict__ w, int rows,
+                                             int rows_pad, int K) {
+  for (int i = threadIdx.x; i < rows_pad * K; i += kHTThreads) {
+    const int r = i / K, c = i - r * K;
+    const __half v = r < rows ? w[(size_t)r * K + c] : __float2half(0.0f);
+    *reinterpret_cast<__half*>(sm + soff + tc::kmaj_off(r, c >> 3, K) + (c & 7) * 2) = v;
+  }
+}
+
+// Output rows of head h padded to 16, and their first row in the W3 tile.
+__device__ __forceinline__ int tc_pad(int h, int sh_pad) { return h == 2 ? sh_pad : 16; }
+__device__ __forceinline__ int tc_row3(int h, int sh_pad) { return h < 3 ? 16 * h : 32 + sh_pad; }
+
+template <int F>
+__global__ void __launch_bounds__(kHTThreads, 2) heads_fwd_tc_kernel(GridParams g, HeadsParams hp,
+                                                                      const float4* __restrict__ pos, int64_t N,
+                                                                      const __half* __restrict__ tables,
+                                                                      const __half* __restrict__ weights,
+                                                                      HeadsOut out) {
+  using Lay = HeadsTcLayout;
+  constexpr int IN = 64;
+  extern __shared__ __align__(1024) uint8_t hsm[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kHT - 1), half = tid >> 7;
+  float* bias = reinterpret_cast<float*>(hsm + Lay::BIAS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hsm + Lay::MISC + 8);
+  const uint32_t mbar = tc::smem_u32(hsm + Lay::MISC);
+  const int sh_rows = hp.sh_dim, sh_pad = (sh_rows + 15) & ~15;
+  // ---- all weights and biases, once per CTA ----
+#pragma unroll 1
+  for (int h = 0; h < 4; ++h) {
+    const __half* w1 = weights + hp.off[h];
+    const __half* w2 = w1 + 64 * IN + 64;
+    const __half* w3 = w2 + 64 * 64 + 64;
+    const int rows = hp.rows[h], pad = tc_pad(h, sh_pad), r3 = tc_row3(h, sh_pad);
+    stage_kmajor(hsm, Lay::W1 + h * 8192, w1, 64, 64, IN);
+    stage_kmajor(hsm, Lay::W2 + h * 8192, w2, 64, 64, 64);
+    stage_kmajor(hsm, Lay::W3 + r3 * 128, w3, rows, pad, 64);
+    for (int o = tid; o < 64; o += kHTThreads) {
+      bias[h * 64 + o] = __half2float(w1[64 * IN + o]);
+      bias[256 + h * 64 + o] = __half2float(w2[64 * 64 + o]);
+    }
+    for (int o = tid; o < pad; o += kHTThreads) bias[512 + r3 + o] = o < rows ? __half2float(w3[rows * 64 + o]) : 0.0f;
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), kHTCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t sbase = tc::smem_u32(hsm);
+  uint32_t phase = 0;
+  bool failed = false;
+
+  // one K = 64 chain into TMEM column dcol: A rows = positions, B rows = outputs
+  auto mma_chain = [&](uint32_t a_tile, uint32_t b_tile, int n_out, uint32_t dcol) {
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        tc::mma_f16(tmem + dcol, tc::smem_desc(a_tile + k * 256, 128, 1024), tc::smem_desc(b_tile + k * 256, 128, 1024),
+                    tc::idesc_f16_f32(kHT, n_out), k > 0 ? 1u : 0u);
+      tc::mma_commit(mbar);
+    }
+    const bool ok = tc::mbar_wait_bounded(mbar, phase, kHTWait);
+    phase ^= 1u;
+    const bool bad = __syncthreads_or(!ok);
+    tc::fence_after_sync();
+    return !bad;
+  };
+  // hidden epilogue: this thread's 32 columns + bias, GELU, fp16 into HT
+  auto hidden_epilogue = [&](const float* b) {
+    float v[32];
+    tc::tmem_ld32(tmem + lane + half * 32, v);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = tc::pack_half2(gelu(v[2 * i] + b[half * 32 + 2 * i]), gelu(v[2 * i + 1] + b[half * 32 + 2 * i + 1]));
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<uint4*>(hsm + Lay::HT + tc::kmaj_off(row, half * 4 + q, 64)) =
+          make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+  };
+
+  for (int64_t tile = blockIdx.x; tile * kHT < N; tile += gridDim.x) {
+    const int64_t n = tile * kHT + row;
+    const bool valid = n < N;
+    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) normalise_position(pos[n], g, xt);
+    // ---- gather: chunks kc = 4 half .. 4 half + 3 (8 features, 8 / F levels each) ----
+#pragma unroll 1
+    for (int kc = half * 4; kc < half * 4 + 4; ++kc) {
+      float zv[8];
+#pragma unroll
+      for (int q = 0; q < 8 / F; ++q) {
+        float acc[F];
+        if (valid) {
+          encode_level_f16_paired<F>(xt, g, kc * (8 / F) + q, tables, acc);
+        } else {
+#pragma unroll
+          for (int f = 0; f < F; ++f) acc[f] = 0.f;
+        }
+#pragma unroll
+        for (int f = 0; f < F; ++f) zv[q * F + f] = acc[f];
+      }
+      if (out.latent && valid) {
+        float4* zl = reinterpret_cast<float4*>(out.latent + n * IN + kc * 8);
+        zl[0] = make_float4(zv[0], zv[1], zv[2], zv[3]);
+        zl[1] = make_float4(zv[4], zv[5], zv[6], zv[7]);
+      }
+      *reinterpret_cast<uint4*>(hsm + Lay::ZT + tc::kmaj_off(row, kc, IN)) =
+          make_uint4(tc::pack_half2(zv[0], zv[1]), tc::pack_half2(zv[2], zv[3]), tc::pack_half2(zv[4], zv[5]),
+                     tc::pack_half2(zv[6], zv[7]));
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    float raw[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int h = 0; h < 4; ++h) {
+      const int pad = tc_pad(h, sh_pad), r3 = tc_row3(h, sh_pad);
+      if (!mma_chain(sbase + Lay::ZT, sbase + Lay::W1 + h * 8192, 64, 0)) { failed = true; break; }
+      hidden_epilogue(bias + h * 64);
+      if (!mma_chain(sbase + Lay::HT, sbase + Lay::W2 + h * 8192, 64, 0)) { failed = true; break; }
+      hidden_epilogue(bias + 256 + h * 64);
+      if (!mma_chain(sbase + Lay::HT, sbase + Lay::W3 + r3 * 128, pad, 64)) { failed = true; break; }
+      const float* b3 = bias + 512 + r3;
+      if (h == 2) {
+        // SH rows 0-31 on warps 0-3, rows 32-47 on warps 4-7; rows are 16-byte aligned (sh_dim % 16 == 0)
+        float4* dst = reinterpret_cast<float4*>(out.sh + (int64_t)sh_rows * n);
+        if (half == 0) {
+          float v[32];
+          if (pad >= 32) {
+            tc::tmem_ld32(tmem + lane + 64, v);
+          } else {
+            tc::tmem_ld16(tmem + lane + 64, v);
+#pragma unroll
+            for (int i = 16; i < 32; ++i) v[i] = 0.0f;
+          }
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (4 * q < sh_rows)
+                dst[q] = make_float4(v[4 * q] + b3[4 * q], v[4 * q + 1] + b3[4 * q + 1], v[4 * q + 2] + b3[4 * q + 2],
+                                     v[4 * q + 3] + b3[4 * q + 3]);
+          }
+        } else if (pad > 32) {
+          float v[16];
+          tc::tmem_ld16(tmem + lane + 96, v);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[8 + q] = make_float4(v[4 * q] + b3[32 + 4 * q], v[4 * q + 1] + b3[33 + 4 * q],
+                                       v[4 * q + 2] + b3[34 + 4 * q], v[4 * q + 3] + b3[35 + 4 * q]);
+          }
+        }
+      } else if (half == 0) {
+        float v[16];
+        tc::tmem_ld16(tmem + lane + 64, v);
+        if (h == 0) {
+#pragma unroll
+          for (int i = 0; i < 3; ++i) raw[i] = v[i] + b3[i];
+        } else if (h == 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) raw[3 + i] = v[i] + b3[i];
+        } else {
+          raw[7] = v[0] + b3[0];
+        }
+      }
+      tc::fence_before_sync();
+      __syncthreads();   // TMEM columns and HT free for the next head
+    }
+    if (failed) break;
+    if (half == 0 && valid) {
+      store_heads(out, n, raw);
+      if (out.raw) {
+        float4* r = reinterpret_cast<float4*>(out.raw + n * 8);
+        r[0] = make_float4(raw[0], raw[1], raw[2], raw[3]);
+        r[1] = make_float4(raw[4], raw[5], raw[6], raw[7]);
+      }
+    }
+  }
+
+  // ---- teardown: nothing of ours may still be writing TMEM when it is freed ----
+  if (failed) {
+    if (tid == 0) atomicExch(&g_heads_device_error, 1);
+    tc::mbar_wait_bounded(mbar, phase ^ 1u, kHTWait);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kHTCols);
+  }
+}
+
 __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
     float s = 0.0f;
@@ -534,8 +799,38 @@ int bwd_blocks(int64_t N) { return persistent_blocks((N + kHeadsBwdBlock - 1) / 
 
 template <typename T, int F, typename W>
 struct HeadsLaunch {
+  // the tensor-core forward (fp16 tables and weights, in_dim = hidden = 64)
+  static int fwd_tc(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
+                    const void* weights, const HeadsOut& o, cudaStream_t s) {
+    auto k = heads_fwd_tc_kernel<F>;
+    const int smem = HeadsTcLayout::BYTES;
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kHTThreads, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      if (occ < 1 || occ * kHTCols > 512) return SPIN4D_ERR_UNSUPPORTED;   // TMEM would be oversubscribed
+      configured[dev] = true;
+    }
+    const int blocks = persistent_blocks((N + kHT - 1) / kHT, 2);
+    k<<<blocks, kHTThreads, smem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                      static_cast<const __half*>(tables), static_cast<const __half*>(weights), o);
+    return launch_status();
+  }
   static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const HeadsOut& o, cudaStream_t s) {
+    if constexpr (std::is_same<T, __half>::value && std::is_same<W, __half>::value && F == 4) {
+      // its vector stores want 16-byte rows of sh and raw
+      const bool vec = ((uintptr_t)o.sh & 15) == 0 && ((uintptr_t)o.raw & 15) == 0;
+      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim % 16 == 0 && hp.sh_dim <= kHTMaxSh && vec) {
+        const int st = fwd_tc(gp, hp, pos, N, tables, weights, o, s);
+        if (st != SPIN4D_ERR_UNSUPPORTED) return st;   // else the SIMT forward below
+      }
+    }
     auto k = heads_fwd_q_kernel<T, F, W>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdQSmem);
     if (e != cudaSuccess) return cuda_status(e);

@@ -309,8 +309,9 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
   return SPIN4D_OK;
 }
 
-int bwd_device_error(int clear);   // decode_bwd_tc.cu
-int hex_device_error(int clear);   // hexplane.cu
+int bwd_device_error(int clear);     // decode_bwd_tc.cu
+int hex_device_error(int clear);     // hexplane.cu
+int heads_device_error(int clear);   // decode_heads.cu
 
 namespace {
 // Waits on an mbarrier that nothing ever arrives at, with the same bounded
@@ -348,7 +349,9 @@ extern "C" int spin4d_check_device_errors(int clear) {
   }
   const int b = spin4d::bwd_device_error(clear);
   const int h = spin4d::hex_device_error(clear);
+  const int p = spin4d::heads_device_error(clear);
   if (b != SPIN4D_OK) return b;
   if (h != SPIN4D_OK) return h;
+  if (p != SPIN4D_OK) return p;
   return v ? SPIN4D_ERR_TIMEOUT : SPIN4D_OK;
 }

@@ -96,6 +96,18 @@ __device__ __forceinline__ PlaneSample plane_sample(const float xt[4], const Hex
   return s;
 }
 
+// The first corner's float offset and the bilinear fractions of sample k,
+// computed exactly as plane_sample does.
+__device__ __forceinline__ int64_t plane_corner(const float xt[4], const HexParams& hp, int k, float& wa, float& wb) {
+  float pa = __fmul_rn(pick_axis(xt, hp.axis_a[k]), hp.scale_a[k]);
+  float pb = __fmul_rn(pick_axis(xt, hp.axis_b[k]), hp.scale_b[k]);
+  int ia = min(max((int)floorf(pa), 0), hp.res_a[k] - 2);
+  int ib = min(max((int)floorf(pb), 0), hp.res_b[k] - 2);
+  wa = __fsub_rn(pa, (float)ia);
+  wb = __fsub_rn(pb, (float)ib);
+  return hp.off[k] + ((int64_t)ib * hp.res_a[k] + ia) * kHexC;
+}
+
 __device__ __forceinline__ float4 sample4(const float* __restrict__ planes, const PlaneSample& s, int c4) {
   float4 a = __ldg(reinterpret_cast<const float4*>(planes + s.o00) + c4);
   float4 b = __ldg(reinterpret_cast<const float4*>(planes + s.o01) + c4);
@@ -414,7 +426,8 @@ struct HexTcLayout {
   static constexpr int W3 = W2 + 3 * S_PLANE;                      // [64][64] x 3 planes (58 rows used)
   static constexpr int BIAS = W3 + 3 * S_PLANE;                    // b1 | b2 | b3 (64 each)
   static constexpr int MISC = BIAS + 3 * kHexH * 4;                // 2 mbarriers + TMEM address
-  static constexpr int BYTES = MISC + 32;
+  static constexpr int XT = MISC + 32;                             // forward: the tile's normalised (x, t)
+  static constexpr int BYTES = XT + kHexTile * 16;
   static __device__ __forceinline__ int z(int b) { return A + b * Z_STAGE; }
   static __device__ __forceinline__ int w(int b) { return B1 + b * W_STAGE; }
 };
@@ -466,6 +479,29 @@ __device__ __forceinline__ void store_split8(uint8_t* sm, int off, int plane, in
 __device__ __forceinline__ void store_split8(uint8_t* sm, int off, int plane, int r, int kc, int L, float4 a, float4 b) {
   const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
   store_split8(sm, off, plane, r, kc, L, v);
+}
+
+// Stores 4 consecutive values (columns c .. c + 3, c % 4 == 0) of row r as
+// their three bf16 planes.
+__device__ __forceinline__ void store_split4(uint8_t* sm, int off, int plane, int r, int c, int L, float4 v) {
+  const float x[4] = {v.x, v.y, v.z, v.w};
+  uint32_t p0[2], p1[2], p2[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+    const float2 f0 = __bfloat1622float2(h0);
+    const float r0 = x[2 * j] - f0.x, r1 = x[2 * j + 1] - f0.y;
+    const __nv_bfloat162 h1 = __floats2bfloat162_rn(r0, r1);
+    const float2 f1 = __bfloat1622float2(h1);
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(r0 - f1.x, r1 - f1.y);
+    p0[j] = bf2_bits(h0);
+    p1[j] = bf2_bits(h1);
+    p2[j] = bf2_bits(h2);
+  }
+  const uint32_t o = (uint32_t)off + tc::kmaj_off(r, c >> 3, L) + (c & 7) * 2;
+  *reinterpret_cast<uint2*>(sm + o) = make_uint2(p0[0], p0[1]);
+  *reinterpret_cast<uint2*>(sm + o + plane) = make_uint2(p1[0], p1[1]);
+  *reinterpret_cast<uint2*>(sm + o + 2 * plane) = make_uint2(p2[0], p2[1]);
 }
 
 // Stores this thread's 32 values (columns half*32 ..) of row r of a 64-column tile.
@@ -692,6 +728,107 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
   return true;
 }
 
+// Registers of one plane sample in the row-coalesced gather: this thread's
+// chunk of the W1 slice, and channels 4 (lane & 7) .. + 3 of the four corner
+// rows of four Gaussians with their bilinear fractions.
+struct RowRegs {
+  float w[8];
+  float4 c[4][4];   // [Gaussian j][corner 00, 01, 10, 11]
+  float wa[4], wb[4];
+};
+
+// hex_stream for sampling from the planes, with the corner rows read whole:
+// lane l of warp w takes channels 4 (l & 7) .. + 3 of Gaussians
+// 16 w + 4 j + (l >> 3), j = 0..3, so eight lanes read one 128-byte row and a
+// warp's load covers four rows.  (Reading a Gaussian's own row per lane makes
+// every 32-byte sector a separate L1 wavefront, which bounds that form.)
+// xt_s holds the tile's normalised coordinates, tile0 its first Gaussian.
+template <int DEPTH, class Issue, class Consume>
+__device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
+                                                const float* __restrict__ W1, float* __restrict__ zdst, int64_t tile0,
+                                                int64_t N, const float4* xt_s, HexBars& bars, Issue issue,
+                                                Consume consume) {
+  using Lay = HexTcLayout;
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int sub = lid >> 3, c4 = lid & 7;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  RowRegs ra, rb;
+  auto prefetch = [&](int k, RowRegs& r) {
+    ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
+    const int64_t down = (int64_t)hp.res_a[k] * (kHexC / 4);   // one row of the plane, in float4
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = 16 * warp + 4 * j + sub;
+      if (tile0 + g < N) {
+        const float4 x = xt_s[g];
+        const float xt[4] = {x.x, x.y, x.z, x.w};
+        const float4* p = reinterpret_cast<const float4*>(planes + plane_corner(xt, hp, k, r.wa[j], r.wb[j])) + c4;
+        r.c[j][0] = __ldg(p);
+        r.c[j][1] = __ldg(p + kHexC / 4);
+        r.c[j][2] = __ldg(p + down);
+        r.c[j][3] = __ldg(p + down + kHexC / 4);
+      } else {
+        r.wa[j] = r.wb[j] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) r.c[j][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  auto step = [&](int k, RowRegs& r) -> bool {
+    const int b = k & 1;
+    bool ok = true;
+    if (k >= 2) {   // as in hex_stream: take sample k-2's results, then refill the stage
+      ok = bars.wait(b);
+      tc::fence_after_sync();
+      if (ok) consume(k - 2, b);
+    }
+    store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, r.w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = 16 * warp + 4 * j + sub;
+      const float wa = r.wa[j], wb = r.wb[j];
+      const float w00 = (1.0f - wa) * (1.0f - wb), w01 = wa * (1.0f - wb), w10 = (1.0f - wa) * wb, w11 = wa * wb;
+      const float4 a = r.c[j][0], bb = r.c[j][1], c = r.c[j][2], d = r.c[j][3];
+      float4 z;
+      z.x = w00 * a.x + w01 * bb.x + w10 * c.x + w11 * d.x;
+      z.y = w00 * a.y + w01 * bb.y + w10 * c.y + w11 * d.y;
+      z.z = w00 * a.z + w01 * bb.z + w10 * c.z + w11 * d.z;
+      z.w = w00 * a.w + w01 * bb.w + w10 * c.w + w11 * d.w;
+      if (zdst && tile0 + g < N) reinterpret_cast<float4*>(zdst + (tile0 + g) * IN + k * kHexC)[c4] = z;
+      store_split4(sm, Lay::z(b), Lay::Z_PLANE, g, 4 * c4, kHexC, z);
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    if (__syncthreads_or(!ok)) return false;
+    if (tid == 0) {
+      tc::fence_after_sync();
+      issue(k, b);
+      tc::mma_commit(bars.addr(b));
+    }
+    if (k + DEPTH < NS) prefetch(k + DEPTH, r);
+    return true;
+  };
+  prefetch(0, ra);
+  if constexpr (DEPTH == 2) {
+    prefetch(1, rb);
+    for (int k = 0; k < NS; k += 2) {
+      if (!step(k, ra)) return false;
+      if (!step(k + 1, rb)) return false;
+    }
+  } else {
+    for (int k = 0; k < NS; ++k)
+      if (!step(k, ra)) return false;
+  }
+  for (int k = NS - 2; k < NS; ++k) {   // the last two samples
+    const int b = k & 1;
+    const bool ok = bars.wait(b);
+    if (__syncthreads_or(!ok)) return false;
+    tc::fence_after_sync();
+    consume(k, b);
+  }
+  return true;
+}
+
 // grad[0..63] += the 256 bytes at shared address src, asynchronously (one
 // bulk reduction); completion is tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_add_2rows(float* grad, uint32_t src) {
@@ -762,6 +899,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::MISC + 16);
   const uint32_t mbar0 = tc::smem_u32(sm + Lay::MISC), mbar1 = mbar0 + 8;
   const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
+  float4* xt_s = reinterpret_cast<float4*>(sm + Lay::XT);
 
   stage_small_layers(sm, Lay::BIAS, W2g, b1, b2, W3g, b3);
   if (warp == 0) {
@@ -788,10 +926,14 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   bool failed = false;
 
   for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
-    const int64_t n = tile * kHexTile + row;
+    const int64_t tile0 = tile * kHexTile, n = tile0 + row;
     const bool valid = n < N;
-    float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) hex_normalise(mu, frame, n, hp, xt);
+    if (half == 0) {
+      float xt[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) hex_normalise(mu, frame, n, hp, xt);
+      xt_s[row] = make_float4(xt[0], xt[1], xt[2], xt[3]);
+    }
+    __syncthreads();
     float acc1[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc1[i] = 0.f;
@@ -801,7 +943,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
-    if (!hex_stream<2, false>(sm, hp, planes, W1, nullptr, latent, n, valid, xt, bars, issue, consume)) {
+    if (!hex_stream_rows<2>(sm, hp, planes, W1, latent, tile0, N, xt_s, bars, issue, consume)) {
       failed = true;
       break;
     }

@@ -413,10 +413,19 @@ constexpr uint32_t kHexWait = 1u << 24;
 // Byte size of one bf16 plane of an R x L tile.
 constexpr int plane_bytes(int R, int L) { return R * L * 2; }
 
+// The forward's z tiles are K-major with the 8-row groups adjacent (128 B
+// apart) and the four 8-column chunks kZChunk = 2080 bytes apart: the 32-byte
+// skew sends a warp's stores of four rows x 32 columns to distinct banks.
+// (The backward keeps the plain layout, chunks adjacent; both fit Z_PLANE.)
+constexpr int kZChunk = (kHexTile / 8) * 128 + 32;
+__device__ __forceinline__ uint32_t zpad_off(int r, int c) {
+  return (uint32_t)((r >> 3) * 128 + (c >> 3) * kZChunk + (r & 7) * 16 + (c & 7) * 2);
+}
+
 struct HexTcLayout {
-  static constexpr int Z_PLANE = plane_bytes(kHexTile, kHexC);      // 8 KB
+  static constexpr int Z_PLANE = (kHexC / 8) * kZChunk;             // 8320 B (>= 8 KB of the plain layout)
   static constexpr int Z_STAGE = 3 * Z_PLANE;
-  static constexpr int A = 0;                                      // 2 z stages = 48 KB; later the H tile
+  static constexpr int A = 0;                                      // 2 z stages = 48.75 KB; later the H tile
   static constexpr int H_PLANE = plane_bytes(kHexTile, kHexH);     // 16 KB: the H tile fills region A
   static constexpr int W_PLANE = plane_bytes(kHexH, kHexC);        // 4 KB
   static constexpr int W_STAGE = 3 * W_PLANE;
@@ -426,12 +435,15 @@ struct HexTcLayout {
   static constexpr int W3 = W2 + 3 * S_PLANE;                      // [64][64] x 3 planes (58 rows used)
   static constexpr int BIAS = W3 + 3 * S_PLANE;                    // b1 | b2 | b3 (64 each)
   static constexpr int MISC = BIAS + 3 * kHexH * 4;                // 2 mbarriers + TMEM address
-  static constexpr int XT = MISC + 32;                             // forward: the tile's normalised (x, t)
-  static constexpr int BYTES = XT + kHexTile * 16;
+  // forward: per plane sample and Gaussian of the tile, {first corner row, wa, wb, 0}
+  static constexpr int SMP = MISC + 32;
+  static constexpr int BYTES = SMP + 24 * kHexTile * 16;
   static __device__ __forceinline__ int z(int b) { return A + b * Z_STAGE; }
   static __device__ __forceinline__ int w(int b) { return B1 + b * W_STAGE; }
 };
-static_assert(3 * HexTcLayout::H_PLANE == 2 * HexTcLayout::Z_STAGE, "H tile must fill the z stages");
+static_assert(3 * HexTcLayout::H_PLANE <= 2 * HexTcLayout::Z_STAGE, "the H tile must fit over the z stages");
+static_assert(HexTcLayout::B1 % 128 == 0 && HexTcLayout::SMP % 16 == 0, "tile alignment");
+static_assert(HexTcLayout::BYTES <= 227 * 1024, "forward tiles exceed the shared memory of one CTA");
 
 // Backward: the forward's z stages, W1 stages and W2 | W3 at the same
 // offsets, the scatter staging over W2 | W3, a second activation tile T1,
@@ -481,9 +493,9 @@ __device__ __forceinline__ void store_split8(uint8_t* sm, int off, int plane, in
   store_split8(sm, off, plane, r, kc, L, v);
 }
 
-// Stores 4 consecutive values (columns c .. c + 3, c % 4 == 0) of row r as
-// their three bf16 planes.
-__device__ __forceinline__ void store_split4(uint8_t* sm, int off, int plane, int r, int c, int L, float4 v) {
+// Stores 4 consecutive values (columns c .. c + 3, c % 4 == 0) of row r of
+// a z tile in the skewed layout (zpad_off) as their three bf16 planes.
+__device__ __forceinline__ void store_split4(uint8_t* sm, int off, int plane, int r, int c, float4 v) {
   const float x[4] = {v.x, v.y, v.z, v.w};
   uint32_t p0[2], p1[2], p2[2];
 #pragma unroll
@@ -498,7 +510,7 @@ __device__ __forceinline__ void store_split4(uint8_t* sm, int off, int plane, in
     p1[j] = bf2_bits(h1);
     p2[j] = bf2_bits(h2);
   }
-  const uint32_t o = (uint32_t)off + tc::kmaj_off(r, c >> 3, L) + (c & 7) * 2;
+  const uint32_t o = (uint32_t)off + zpad_off(r, c);
   *reinterpret_cast<uint2*>(sm + o) = make_uint2(p0[0], p0[1]);
   *reinterpret_cast<uint2*>(sm + o + plane) = make_uint2(p1[0], p1[1]);
   *reinterpret_cast<uint2*>(sm + o + 2 * plane) = make_uint2(p2[0], p2[1]);
@@ -519,6 +531,10 @@ struct SplitOp {
 // Tile with L columns read K-major (rows are M or N, columns are K).
 __device__ __forceinline__ SplitOp kmajor(uint32_t base, int plane, int L) {
   return {base, (uint32_t)plane, 128u, 16u * (uint32_t)L, 256u};
+}
+// A forward z tile (128 rows, skewed layout).
+__device__ __forceinline__ SplitOp kmajor_zpad(uint32_t base, int plane) {
+  return {base, (uint32_t)plane, (uint32_t)kZChunk, 128u, 2u * kZChunk};
 }
 // Tile with L columns read MN-major (columns are M or N, rows are K).
 __device__ __forceinline__ SplitOp mnmajor(uint32_t base, int plane, int L) {
@@ -734,7 +750,6 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
 struct RowRegs {
   float w[8];
   float4 c[4][4];   // [Gaussian j][corner 00, 01, 10, 11]
-  float wa[4], wb[4];
 };
 
 // hex_stream for sampling from the planes, with the corner rows read whole:
@@ -742,11 +757,13 @@ struct RowRegs {
 // 16 w + 4 j + (l >> 3), j = 0..3, so eight lanes read one 128-byte row and a
 // warp's load covers four rows.  (Reading a Gaussian's own row per lane makes
 // every 32-byte sector a separate L1 wavefront, which bounds that form.)
-// xt_s holds the tile's normalised coordinates, tile0 its first Gaussian.
+// smp[k * 128 + g] holds sample k of Gaussian g of the tile: its first
+// corner as a row index of the planes (rows of kHexC floats), wa and wb;
+// tile0 is the tile's first Gaussian.
 template <int DEPTH, class Issue, class Consume>
 __device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
                                                 const float* __restrict__ W1, float* __restrict__ zdst, int64_t tile0,
-                                                int64_t N, const float4* xt_s, HexBars& bars, Issue issue,
+                                                int64_t N, const float4* smp, HexBars& bars, Issue issue,
                                                 Consume consume) {
   using Lay = HexTcLayout;
   const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
@@ -760,15 +777,13 @@ __device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp
     for (int j = 0; j < 4; ++j) {
       const int g = 16 * warp + 4 * j + sub;
       if (tile0 + g < N) {
-        const float4 x = xt_s[g];
-        const float xt[4] = {x.x, x.y, x.z, x.w};
-        const float4* p = reinterpret_cast<const float4*>(planes + plane_corner(xt, hp, k, r.wa[j], r.wb[j])) + c4;
+        const uint32_t crow = __float_as_uint(smp[k * kHexTile + g].x);
+        const float4* p = reinterpret_cast<const float4*>(planes + (int64_t)crow * kHexC) + c4;
         r.c[j][0] = __ldg(p);
         r.c[j][1] = __ldg(p + kHexC / 4);
         r.c[j][2] = __ldg(p + down);
         r.c[j][3] = __ldg(p + down + kHexC / 4);
       } else {
-        r.wa[j] = r.wb[j] = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) r.c[j][c] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -786,7 +801,8 @@ __device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int g = 16 * warp + 4 * j + sub;
-      const float wa = r.wa[j], wb = r.wb[j];
+      const float4 rec = smp[k * kHexTile + g];
+      const float wa = rec.y, wb = rec.z;
       const float w00 = (1.0f - wa) * (1.0f - wb), w01 = wa * (1.0f - wb), w10 = (1.0f - wa) * wb, w11 = wa * wb;
       const float4 a = r.c[j][0], bb = r.c[j][1], c = r.c[j][2], d = r.c[j][3];
       float4 z;
@@ -795,7 +811,7 @@ __device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp
       z.z = w00 * a.z + w01 * bb.z + w10 * c.z + w11 * d.z;
       z.w = w00 * a.w + w01 * bb.w + w10 * c.w + w11 * d.w;
       if (zdst && tile0 + g < N) reinterpret_cast<float4*>(zdst + (tile0 + g) * IN + k * kHexC)[c4] = z;
-      store_split4(sm, Lay::z(b), Lay::Z_PLANE, g, 4 * c4, kHexC, z);
+      store_split4(sm, Lay::z(b), Lay::Z_PLANE, g, 4 * c4, z);
     }
     tc::fence_proxy_async();
     tc::fence_before_sync();
@@ -899,7 +915,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::MISC + 16);
   const uint32_t mbar0 = tc::smem_u32(sm + Lay::MISC), mbar1 = mbar0 + 8;
   const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
-  float4* xt_s = reinterpret_cast<float4*>(sm + Lay::XT);
+  float4* smp = reinterpret_cast<float4*>(sm + Lay::SMP);
 
   stage_small_layers(sm, Lay::BIAS, W2g, b1, b2, W3g, b3);
   if (warp == 0) {
@@ -928,10 +944,16 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
   for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
     const int64_t tile0 = tile * kHexTile, n = tile0 + row;
     const bool valid = n < N;
-    if (half == 0) {
+    {
+      // the tile's sample table: each half takes every other sample
       float xt[4] = {0.f, 0.f, 0.f, 0.f};
       if (valid) hex_normalise(mu, frame, n, hp, xt);
-      xt_s[row] = make_float4(xt[0], xt[1], xt[2], xt[3]);
+      for (int k = half; k < hp.n_samples; k += 2) {
+        float wa = 0.f, wb = 0.f;
+        uint32_t crow = 0;
+        if (valid) crow = (uint32_t)(plane_corner(xt, hp, k, wa, wb) / kHexC);
+        smp[k * kHexTile + row] = make_float4(__uint_as_float(crow), wa, wb, 0.f);
+      }
     }
     __syncthreads();
     float acc1[32];
@@ -939,11 +961,11 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
     for (int i = 0; i < 32; ++i) acc1[i] = 0.f;
     // ---- layer 1, streamed over the plane samples ----
     auto issue = [&](int, int b) {
-      mma6(tmem + 128 * b, tmem + 128 * b + 64, kmajor(sbase + Lay::z(b), Lay::Z_PLANE, kHexC),
+      mma6(tmem + 128 * b, tmem + 128 * b + 64, kmajor_zpad(sbase + Lay::z(b), Lay::Z_PLANE),
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
-    if (!hex_stream_rows<2>(sm, hp, planes, W1, latent, tile0, N, xt_s, bars, issue, consume)) {
+    if (!hex_stream_rows<2>(sm, hp, planes, W1, latent, tile0, N, smp, bars, issue, consume)) {
       failed = true;
       break;
     }

@@ -623,6 +623,24 @@ __device__ __forceinline__ void ld_nc_v8(const float* p, float v[8]) {
                : "l"(p));
 }
 
+// An L2 policy that evicts first: the latent streams through L2 (1.15 GB at
+// 500k Gaussians) and should not push out the planes or their gradients.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void ld_nc_v8_stream(const float* p, float v[8], uint64_t pol) {
+  asm volatile("ld.global.nc.L2::cache_hint.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "l"(p), "l"(pol));
+}
+__device__ __forceinline__ void st_v4_stream(float* p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w), "l"(pol)
+               : "memory");
+}
+
 // Global data of one plane sample for one thread: its chunk of the W1 slice
 // (row tid/4, 8 columns) and, for its Gaussian, either the 16 channels
 // (half*16 ..) of the four corner rows with their bilinear weights, or the
@@ -665,8 +683,9 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
     ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
     if (!valid) return;
     if constexpr (LATENT) {
-      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16, r.z);
-      ld_nc_v8(zsrc + n * IN + k * kHexC + half * 16 + 8, r.z + 8);
+      const uint64_t pol = l2_evict_first();
+      ld_nc_v8_stream(zsrc + n * IN + k * kHexC + half * 16, r.z, pol);
+      ld_nc_v8_stream(zsrc + n * IN + k * kHexC + half * 16 + 8, r.z + 8, pol);
     } else {
       const PlaneSample ps = plane_sample(xt, hp, k);
       r.wt[0] = ps.w00;
@@ -810,7 +829,7 @@ __device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp
       z.y = w00 * a.y + w01 * bb.y + w10 * c.y + w11 * d.y;
       z.z = w00 * a.z + w01 * bb.z + w10 * c.z + w11 * d.z;
       z.w = w00 * a.w + w01 * bb.w + w10 * c.w + w11 * d.w;
-      if (zdst && tile0 + g < N) reinterpret_cast<float4*>(zdst + (tile0 + g) * IN + k * kHexC)[c4] = z;
+      if (zdst && tile0 + g < N) st_v4_stream(zdst + (tile0 + g) * IN + k * kHexC + 4 * c4, z, l2_evict_first());
       store_split4(sm, Lay::z(b), Lay::Z_PLANE, g, 4 * c4, z);
     }
     tc::fence_proxy_async();

@@ -418,8 +418,21 @@ typedef struct spin4d_heads_output_grads {
 /* Values in the packed weight vector (-1 if invalid). */
 int64_t spin4d_heads_param_count(const spin4d_heads_desc* h);
 
+/* Bytes of the forward's optional workspace: N rows of 64 fp16 features for
+ * the configuration whose layers run on the tensor cores (see
+ * spin4d_heads_desc), 0 for every other configuration. */
+size_t spin4d_heads_fwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N);
+
+/* Forward of the four heads for N positions (device pointers; pos N x 4,
+ * tables and weights as above).  workspace (device, 256-byte aligned,
+ * >= spin4d_heads_fwd_workspace bytes; may be NULL) lets the tensor-core
+ * configuration run as two kernels: a full-occupancy hash gather that writes
+ * z (fp16) there, then the layers; with NULL the same arithmetic runs as one
+ * fused kernel, slower.  Other configurations ignore it.  Misaligned or too
+ * small a workspace returns SPIN4D_ERR_INVALID. */
 int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
-                     const void* tables, const void* weights, spin4d_heads_outputs out, spin4d_stream_t stream);
+                     const void* tables, const void* weights, spin4d_heads_outputs out, void* workspace,
+                     size_t ws_bytes, spin4d_stream_t stream);
 
 size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N);
 

@@ -25,6 +25,7 @@
 #include <type_traits>
 
 #include "host.h"
+#include "pdl.cuh"
 #include "tc.cuh"
 
 namespace spin4d {
@@ -57,6 +58,7 @@ struct HeadsParams {
 
 struct HeadsOut {
   float *scale, *rot, *sh, *opacity, *cov, *latent, *raw;
+  uint4* z16;   // workspace of the split tensor-core forward (N rows of 64 fp16), or null
 };
 struct HeadsGrads {
   const float *scale, *rot, *sh, *opacity, *cov;
@@ -554,7 +556,41 @@ __device__ __forceinline__ void stage_kmajor(uint8_t* sm, int soff, const __half
 __device__ __forceinline__ int tc_pad(int h, int sh_pad) { return h == 2 ? sh_pad : 16; }
 __device__ __forceinline__ int tc_row3(int h, int sh_pad) { return h < 3 ? 16 * h : 32 + sh_pad; }
 
+// Gather of the split forward: one thread per position, two levels (one
+// 16-byte chunk of 8 fp16 features, rounded as the fused kernel rounds them)
+// at a time, into z16 rows of 64 halves and into the fp32 latent when given.
+// At 64 warps per SM the corner loads keep far more requests in flight than
+// the fused kernel's 16 warps per SM.
 template <int F>
+__global__ void __launch_bounds__(128) heads_gather_kernel(GridParams g, const float4* __restrict__ pos, int64_t N,
+                                                          const __half* __restrict__ tables, uint4* __restrict__ z16,
+                                                          float* __restrict__ latent) {
+  static_assert(F == 4, "the split forward takes L = 16, F = 4");
+  pdl_release();
+  for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
+    float xt[4];
+    normalise_position(pos[n], g, xt);
+#pragma unroll 1
+    for (int kc = 0; kc < 8; ++kc) {
+      float a[4], b[4];
+      encode_level_f16_paired<4>(xt, g, 2 * kc, tables, a);
+      encode_level_f16_paired<4>(xt, g, 2 * kc + 1, tables, b);
+      z16[n * 8 + kc] = make_uint4(tc::pack_half2(a[0], a[1]), tc::pack_half2(a[2], a[3]), tc::pack_half2(b[0], b[1]),
+                                   tc::pack_half2(b[2], b[3]));
+      if (latent) {
+        float4* zl = reinterpret_cast<float4*>(latent + n * 64 + kc * 8);
+        zl[0] = make_float4(a[0], a[1], a[2], a[3]);
+        zl[1] = make_float4(b[0], b[1], b[2], b[3]);
+      }
+    }
+  }
+}
+
+// FROM_Z: the layers of the split forward, z read from the gather's z16
+// rows (launched programmatically dependent on the gather: weights and
+// tensor memory are set up before waiting for it); otherwise the fused
+// forward that gathers z itself.
+template <int F, bool FROM_Z>
 __global__ void __launch_bounds__(kHTThreads, 2) heads_fwd_tc_kernel(GridParams g, HeadsParams hp,
                                                                       const float4* __restrict__ pos, int64_t N,
                                                                       const __half* __restrict__ tables,
@@ -602,6 +638,7 @@ __global__ void __launch_bounds__(kHTThreads, 2) heads_fwd_tc_kernel(GridParams 
   const uint32_t sbase = tc::smem_u32(hsm);
   uint32_t phase = 0;
   bool failed = false;
+  if constexpr (FROM_Z) pdl_wait();   // the gather's z16 rows are complete and visible
 
   // one K = 64 chain into TMEM column dcol: A rows = positions, B rows = outputs
   auto mma_chain = [&](uint32_t a_tile, uint32_t b_tile, int n_out, uint32_t dcol) {
@@ -639,11 +676,22 @@ __global__ void __launch_bounds__(kHTThreads, 2) heads_fwd_tc_kernel(GridParams 
   for (int64_t tile = blockIdx.x; tile * kHT < N; tile += gridDim.x) {
     const int64_t n = tile * kHT + row;
     const bool valid = n < N;
+    if constexpr (FROM_Z) {
+      // the tile's z rows: a warp copies 8 rows x 4 chunks (64 contiguous
+      // bytes of each row), which land in distinct banks of the K-major tile
+      for (int i = tid; i < kHT * 8; i += kHTThreads) {
+        const int w = i >> 5, l = i & 31;
+        const int r = 8 * (w >> 1) + (l & 7), kc = 4 * (w & 1) + (l >> 3);
+        const int64_t nr = tile * kHT + r;
+        const uint4 v = nr < N ? __ldg(out.z16 + nr * 8 + kc) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(hsm + Lay::ZT + tc::kmaj_off(r, kc, IN)) = v;
+      }
+    }
     float xt[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) normalise_position(pos[n], g, xt);
+    if (!FROM_Z && valid) normalise_position(pos[n], g, xt);
     // ---- gather: chunks kc = 4 half .. 4 half + 3 (8 features, 8 / F levels each) ----
 #pragma unroll 1
-    for (int kc = half * 4; kc < half * 4 + 4; ++kc) {
+    for (int kc = half * 4; kc < (FROM_Z ? 0 : half * 4 + 4); ++kc) {
       float zv[8];
 #pragma unroll
       for (int q = 0; q < 8 / F; ++q) {
@@ -800,26 +848,39 @@ int bwd_blocks(int64_t N) { return persistent_blocks((N + kHeadsBwdBlock - 1) / 
 template <typename T, int F, typename W>
 struct HeadsLaunch {
   // the tensor-core forward (fp16 tables and weights, in_dim = hidden = 64)
-  static int fwd_tc(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
-                    const void* weights, const HeadsOut& o, cudaStream_t s) {
-    auto k = heads_fwd_tc_kernel<F>;
-    const int smem = HeadsTcLayout::BYTES;
+  template <bool FROM_Z>
+  static int configure_tc(int smem) {
     static bool configured[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (!configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      int occ = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kHTThreads, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      if (occ < 1 || occ * kHTCols > 512) return SPIN4D_ERR_UNSUPPORTED;   // TMEM would be oversubscribed
-      configured[dev] = true;
-    }
+    if (configured[dev]) return SPIN4D_OK;
+    auto k = heads_fwd_tc_kernel<F, FROM_Z>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kHTThreads, smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (occ < 1 || occ * kHTCols > 512) return SPIN4D_ERR_UNSUPPORTED;   // TMEM would be oversubscribed
+    configured[dev] = true;
+    return SPIN4D_OK;
+  }
+  static int fwd_tc(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
+                    const void* weights, const HeadsOut& o, cudaStream_t s) {
+    const int smem = HeadsTcLayout::BYTES;
     const int blocks = persistent_blocks((N + kHT - 1) / kHT, 2);
-    k<<<blocks, kHTThreads, smem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
-                                      static_cast<const __half*>(tables), static_cast<const __half*>(weights), o);
-    return launch_status();
+    const float4* P = reinterpret_cast<const float4*>(pos);
+    const __half* tab = static_cast<const __half*>(tables);
+    const __half* wts = static_cast<const __half*>(weights);
+    if (!o.z16) {
+      SPIN4D_CHECK(configure_tc<false>(smem));
+      heads_fwd_tc_kernel<F, false><<<blocks, kHTThreads, smem, s>>>(gp, hp, P, N, tab, wts, o);
+      return launch_status();
+    }
+    SPIN4D_CHECK(configure_tc<true>(smem));
+    heads_gather_kernel<F><<<persistent_blocks((N + 127) / 128, 16), 128, 0, s>>>(gp, P, N, tab, o.z16, o.latent);
+    SPIN4D_CHECK(launch_status());
+    return cuda_status(launch_pdl(heads_fwd_tc_kernel<F, true>, dim3(blocks), dim3(kHTThreads), (size_t)smem, s, gp,
+                                  hp, P, N, tab, wts, o));
   }
   static int fwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const HeadsOut& o, cudaStream_t s) {
@@ -893,6 +954,13 @@ int run(const spin4d_grid_desc* g, const spin4d_heads_desc* h, bool bwd, const f
                            n_params, s);
 }
 
+// The configuration whose forward splits into gather + tensor-core layers
+// when given a workspace (otherwise it runs the fused tensor-core kernel).
+bool split_forward(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
+  return g->table_dtype == SPIN4D_F16 && h->w_dtype == SPIN4D_F16 && g->F == 4 && h->in_dim == 64 &&
+         h->hidden == 64 && h->sh_dim % 16 == 0 && h->sh_dim <= kHTMaxSh;
+}
+
 int check_inputs(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
                  const void* tables, const void* weights) {
   SPIN4D_CHECK(validate_grid(g));
@@ -916,14 +984,22 @@ extern "C" int64_t spin4d_heads_param_count(const spin4d_heads_desc* h) {
   return param_count(h);
 }
 
+extern "C" size_t spin4d_heads_fwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N) {
+  if (validate_grid(g) != SPIN4D_OK || validate_heads(g, h) != SPIN4D_OK || N <= 0) return 0;
+  return split_forward(g, h) ? (size_t)N * 64 * sizeof(__half) : 0;
+}
+
 extern "C" int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
-                                const void* tables, const void* weights, spin4d_heads_outputs out,
-                                spin4d_stream_t stream) {
+                                const void* tables, const void* weights, spin4d_heads_outputs out, void* workspace,
+                                size_t ws_bytes, spin4d_stream_t stream) {
   SPIN4D_CHECK(check_inputs(g, h, pos, N, tables, weights));
   if (N == 0) return SPIN4D_OK;
   if (!out.scale || !out.rot || !out.sh || !out.opacity || !out.cov || !aligned(out.rot, 16)) return SPIN4D_ERR_INVALID;
+  const size_t need = spin4d_heads_fwd_workspace(g, h, N);
+  if (workspace && (!aligned(workspace, 256) || ws_bytes < need)) return SPIN4D_ERR_INVALID;
   if (fault_injected("spin4d_heads_fwd")) return SPIN4D_ERR_INJECTED;
-  const HeadsOut o{out.scale, out.rot, out.sh, out.opacity, out.cov, out.latent, out.raw};
+  uint4* z16 = workspace && need ? static_cast<uint4*>(workspace) : nullptr;
+  const HeadsOut o{out.scale, out.rot, out.sh, out.opacity, out.cov, out.latent, out.raw, z16};
   return run(g, h, false, pos, N, tables, weights, &o, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
              (cudaStream_t)stream);
 }

@@ -110,7 +110,9 @@ _SIGS = {
                                           P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "spin4d_heads_param_count": (c_i64, [P(HeadsDesc)]),
-    "spin4d_heads_fwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, HeadsOutputs, c_vp]),
+    "spin4d_heads_fwd_workspace": (c_sz, [P(GridDesc), P(HeadsDesc), c_i64]),
+    "spin4d_heads_fwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, HeadsOutputs, c_vp, c_sz,
+                                 c_vp]),
     "spin4d_heads_bwd_workspace": (c_sz, [P(GridDesc), P(HeadsDesc), c_i64]),
     "spin4d_heads_bwd": (c_i32, [P(GridDesc), P(HeadsDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(HeadsOutputGrads),
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
@@ -354,10 +356,15 @@ def heads_param_count(h: HeadsDesc) -> int:
 
 
 def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent: bool = False, raw: bool = False,
-              stream=None):
+              stream=None, workspace="auto"):
     """Outputs dict; with latent / raw it also holds z (N x in_dim) and the
-    raw scale, rotation and opacity head outputs (N x 8) for heads_bwd."""
+    raw scale, rotation and opacity head outputs (N x 8) for heads_bwd.
+    workspace: "auto" allocates what spin4d_heads_fwd_workspace asks for,
+    None passes none (the fused kernel), or a uint8 device tensor."""
     N = pos.shape[0]
+    if isinstance(workspace, str):
+        need = lib.spin4d_heads_fwd_workspace(ctypes.byref(g), ctypes.byref(h), N)
+        workspace = torch.empty(need, dtype=torch.uint8, device=pos.device) if need else None
     widths = {"scale": 3, "rot": 4, "sh": h.sh_dim, "opacity": 1, "cov": 6}
     if out is None:
         out = {k: torch.empty((N, w), dtype=torch.float32, device=pos.device) for k, w in widths.items()}
@@ -366,8 +373,9 @@ def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent:
         if raw:
             out["raw"] = torch.empty((N, 8), dtype=torch.float32, device=pos.device)
     o = HeadsOutputs(*(_ptr(out[k]) for k in HEADS_KEYS), _ptr(out.get("latent")), _ptr(out.get("raw")))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("spin4d_heads_fwd", lib.spin4d_heads_fwd(ctypes.byref(g), ctypes.byref(h), _ptr(pos), N, _ptr(tables),
-                                                    _ptr(weights), o, _stream(stream)))
+                                                    _ptr(weights), o, _ptr(workspace), ws_bytes, _stream(stream)))
     return out
 
 

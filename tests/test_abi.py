@@ -129,13 +129,21 @@ def test_invalid_arguments_rejected_on_host(sp):
     assert sp.heads_param_count(hs) == S.HEADS_PAPER.n_params()
     gp4 = sp.grid_from_spec(S.GRID_PAPER)
     assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(63)), FAKE, 10, FAKE, FAKE,
-                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_INVALID
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_INVALID
     assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(64, hidden=128)), FAKE, 10, FAKE, FAKE,
-                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_UNSUPPORTED
     assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
-                                sp.HeadsOutputs(FAKE, FAKE + 4, FAKE, FAKE, FAKE, None), None) == sp.ERR_INVALID
+                                sp.HeadsOutputs(FAKE, FAKE + 4, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_INVALID
+    # the split forward's workspace: 64 fp16 per position; misaligned or short is rejected
+    assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(hs), 10) == 10 * 128
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), FAKE, 10 * 128 - 1,
+                                None) == sp.ERR_INVALID
+    assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), FAKE + 16, 10 * 128,
+                                None) == sp.ERR_INVALID
     assert lib.spin4d_heads_fwd(ref(gp4), ref(sp.heads_desc(64, hidden=62)), FAKE, 10, FAKE, FAKE,
-                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None) == sp.ERR_UNSUPPORTED
+                                sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_UNSUPPORTED
     # grouped Adam: ends must increase to n
     grp = (sp.AdamGroup * 2)(sp.AdamGroup(60, 1e-3), sp.AdamGroup(50, 1e-4))
     assert lib.spin4d_adam_step_groups(FAKE, None, FAKE, FAKE, FAKE, 100, grp, 2, 1, 0.9, 0.99, 1e-15, 0, None,

@@ -62,6 +62,12 @@ def test_heads_forward_matches_oracle(sp, case):
     tol.absolute(raw[:, 3:7] / np.linalg.norm(raw[:, 3:7], axis=1, keepdims=True), want["rot"], tol.FP16_ATOL,
                  "raw rotation")
     tol.absolute(1.0 / (1.0 + np.exp(-raw[:, 7])), want["opacity"][:, 0], tol.FP16_ATOL, "raw opacity")
+    if grid.dtype != "f32":
+        # without a workspace the tensor-core configuration runs as one fused kernel
+        fused = sp.heads_fwd(g, h, dev(pos), dev(tables), dev(weights), latent=True, workspace=None)
+        for k in ("scale", "rot", "sh", "opacity", "cov"):
+            tol.absolute(host(fused[k]), want[k], tol.FP16_ATOL, "fused " + k)
+        tol.rowwise(host(fused["latent"]), want["z"], tol.FP32_RTOL, "fused latent")
 
 
 @pytest.mark.parametrize("case,saved", [("tiny_fp32", ""), ("tiny_fp32", "latent+raw"), ("paper_fp16", ""),

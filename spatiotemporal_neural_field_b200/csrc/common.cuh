@@ -507,4 +507,32 @@ template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
 
+// Sums over a warp: v[i] holds this lane's value of column i; on return the
+// lane holds the sum over the warp's 32 lanes of column `lane`.  Each of the
+// five exchange rounds halves the columns a lane is responsible for.
+__device__ __forceinline__ float warp_column_sum(float v[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+
+// Adds 32 consecutive floats to a workspace slot row with fp32 vector
+// reductions.  Only this thread ever updates these elements, so the adds land
+// in program order and the sum does not depend on scheduling.
+__device__ __forceinline__ void slot_add32(float* dst, const float a[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) atomicAdd(d + q, make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
+}
+
 }  // namespace spin4d

@@ -820,6 +820,373 @@ __global__ void __launch_bounds__(kHTThreads, 2) heads_fwd_tc_kernel(GridParams 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Backward on the tensor cores, for the configuration of heads_fwd_tc_kernel
+// when the forward's z (fp32 latent) and raw head outputs are given.  One
+// persistent CTA of 256 threads per SM takes tiles of 128 positions; thread
+// (row, half) owns position `row` and columns half*32 .. of every M = 128
+// product.  Per head, with fp16 operand tiles and fp32 accumulators in TMEM
+// (columns: P1 0-63, P2 64-127, D 128-191, dz 192-255):
+//   P1 = z W1^T, h1 = gelu(P1 + b1);  P2 = h1 W2^T, h2 = gelu(P2 + b2);
+//   dy = the head's output adjoint (Eq. 11 / Eq. 2 backward, or dL/dsh);
+//   D = dy W3, d2 = D * gelu'(P2 + b2);  D = d2 W2, d1 = D * gelu'(P1 + b1);
+//   dz += d1 W1 (accumulated over the heads);
+//   dW3 = dy^T h2, dW2 = d2^T h1, dW1 = d1^T z as M = 64 products over the
+//   tile's 128 positions (rows of dW3 padded to 64 with zero columns of dy),
+//   added to the CTA's workspace slot by vector reductions whose every element
+//   has one owning thread (so the sum does not depend on scheduling).
+// The slot is padded per head: [W1 64x64][b1][W2 64x64][b2][W3 64x64][b3 64]
+// so every row is 16-byte aligned; heads_reduce_slots_tc maps it back to the
+// packed order.  dz is then scattered into the tables as the SIMT kernel does.
+// GELU and its derivative use the rational erf of gelu_fast (the operands
+// they feed are fp16).
+// ---------------------------------------------------------------------------
+constexpr int kHBHead = 3 * (64 * 64 + 64);   // floats of one head in the padded slot
+constexpr int kHBSlot = 4 * kHBHead;
+constexpr int kHBW2 = 64 * 64 + 64, kHBW3 = 2 * (64 * 64 + 64), kHBB3 = kHBW3 + 64 * 64;
+
+__device__ __forceinline__ float gelu_grad_fast(float x) {
+  const float u = fabsf(x) * 0.70710678118654752f;
+  float p = fmaf(u, 0.0000430638f, 0.0002765672f);
+  p = fmaf(p, u, 0.0001520143f);
+  p = fmaf(p, u, 0.0092705272f);
+  p = fmaf(p, u, 0.0422820123f);
+  p = fmaf(p, u, 0.0705230784f);
+  p = fmaf(p, u, 1.0f);
+  p *= p;
+  p *= p;
+  p *= p;
+  p *= p;
+  const float he = 0.5f * __fdividef(1.0f, p);   // (1 - erf(|x| / sqrt 2)) / 2
+  const float Phi = x >= 0.0f ? 1.0f - he : he;
+  return Phi + x * 0.39894228040143268f * __expf(-0.5f * x * x);
+}
+
+struct HeadsBwdLayout {
+  static constexpr int W1 = HeadsTcLayout::W1, W2 = HeadsTcLayout::W2, W3 = HeadsTcLayout::W3;
+  static constexpr int BIAS = HeadsTcLayout::BIAS;
+  static constexpr int ZT = 81920;                    // [128][64] fp16 tiles, K-major
+  static constexpr int H1 = ZT + 16384;
+  static constexpr int H2 = H1 + 16384;
+  static constexpr int DY = H2 + 16384;               // dy, later d1
+  static constexpr int D2 = DY + 16384;
+  static constexpr int PART = D2 + 16384;             // [4][64] fp32 column partial sums
+  static constexpr int BACC = PART + 1024;            // [4 heads][3][64] fp32 bias gradients
+  static constexpr int MISC = BACC + 3072;
+  static constexpr int BYTES = MISC + 16;
+};
+static_assert(HeadsTcLayout::BIAS + (512 + HeadsTcLayout::kW3Rows) * 4 <= HeadsBwdLayout::ZT, "layout overlap");
+static_assert(HeadsBwdLayout::BYTES <= 227 * 1024, "backward tiles exceed one CTA's shared memory");
+
+template <int F>
+__global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
+    GridParams g, HeadsParams hp, const float4* __restrict__ pos, int64_t N, const __half* __restrict__ weights,
+    const float* __restrict__ latent, const float* __restrict__ raw_in, HeadsGrads go,
+    float* __restrict__ grad_tables, float* __restrict__ ws) {
+  using Lay = HeadsBwdLayout;
+  constexpr int IN = 64;
+  extern __shared__ __align__(1024) uint8_t bsm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int row = tid & (kHT - 1), half = tid >> 7;
+  float* bias = reinterpret_cast<float*>(bsm + Lay::BIAS);
+  float* part = reinterpret_cast<float*>(bsm + Lay::PART);
+  float* bacc = reinterpret_cast<float*>(bsm + Lay::BACC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bsm + Lay::MISC + 8);
+  const uint32_t mbar = tc::smem_u32(bsm + Lay::MISC);
+  const int sh_rows = hp.sh_dim, sh_pad = (sh_rows + 15) & ~15;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(kHBSlot);
+  for (int p = tid; p < kHBSlot; p += kHTThreads) slot[p] = 0.f;
+  for (int p = tid; p < 4 * 3 * 64; p += kHTThreads) bacc[p] = 0.f;
+#pragma unroll 1
+  for (int h = 0; h < 4; ++h) {
+    const __half* w1 = weights + hp.off[h];
+    const __half* w2 = w1 + 64 * IN + 64;
+    const __half* w3 = w2 + 64 * 64 + 64;
+    const int rows = hp.rows[h], pad = tc_pad(h, sh_pad), r3 = tc_row3(h, sh_pad);
+    stage_kmajor(bsm, Lay::W1 + h * 8192, w1, 64, 64, IN);
+    stage_kmajor(bsm, Lay::W2 + h * 8192, w2, 64, 64, 64);
+    stage_kmajor(bsm, Lay::W3 + r3 * 128, w3, rows, pad, 64);
+    for (int o = tid; o < 64; o += kHTThreads) {
+      bias[h * 64 + o] = __half2float(w1[64 * IN + o]);
+      bias[256 + h * 64 + o] = __half2float(w2[64 * 64 + o]);
+    }
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t sbase = tc::smem_u32(bsm);
+  const uint32_t P1 = tmem, P2 = tmem + 64, DD = tmem + 128, DZ = tmem + 192;
+  // Row m of a 64-row (M = 64) accumulator sits in TMEM lane (m % 16) + 32 (m / 16):
+  // warp w holds rows 16 (w % 4) + lane for lanes below 16, columns (w / 4) * 32 ..
+  const int wrow = (warp & 3) * 16 + lid;
+  const bool wrow_ok = lid < 16;
+  const int wcol = (warp >> 2) * 32;
+  uint32_t phase = 0;
+  bool failed = false;
+
+  // K-major tile with L columns; MN-major read of the same tile
+  auto kdesc = [&](uint32_t off, int L, int k) { return tc::smem_desc(sbase + off + k * 256, 128, 16 * L); };
+  auto mdesc = [&](uint32_t off, int L, int k) { return tc::smem_desc(sbase + off + k * 32 * L, 16 * L, 128); };
+  auto wait_mma = [&]() -> bool {
+    if (tid == 0) tc::mma_commit(mbar);
+    const bool ok = tc::mbar_wait_bounded(mbar, phase, kHTWait);
+    phase ^= 1u;
+    const bool bad = __syncthreads_or(!ok);
+    tc::fence_after_sync();
+    return !bad;
+  };
+  auto store_row = [&](int off, const float v[32]) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = tc::pack_half2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<uint4*>(bsm + off + tc::kmaj_off(row, half * 4 + q, 64)) =
+          make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  };
+  auto tiles_ready = [&]() {
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+  };
+  // column sums of this thread's 32 values over the tile's 128 rows: warp sums
+  // into part[warp % 4][col], then (after the next barrier) bias_add adds
+  // them in a fixed order
+  auto col_partial = [&](const float v[32]) {
+    float t[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = v[i];
+    part[(warp & 3) * 64 + half * 32 + lid] = warp_column_sum(t);
+  };
+  auto bias_add = [&](float* dst) {
+    if (tid < 64) dst[tid] += part[tid] + part[64 + tid] + part[128 + tid] + part[192 + tid];
+  };
+  auto flush64 = [&](uint32_t acc, float* dst, int nrows) {   // dst: 64 x 64 rows of the slot
+    float a[32];
+    tc::tmem_ld32(acc + lane + wcol, a);
+    if (wrow_ok && wrow < nrows) slot_add32(dst + wrow * 64 + wcol, a);
+  };
+
+  for (int64_t tile = blockIdx.x; tile * kHT < N && !failed; tile += gridDim.x) {
+    const int64_t n = tile * kHT + row;
+    const bool valid = n < N;
+    // ---- z (fp32 latent) -> fp16 K-major tile: a warp copies 8 rows x 4 float4 ----
+    for (int i = tid; i < kHT * 16; i += kHTThreads) {
+      const int w = i >> 5, l = i & 31;
+      const int r = 8 * (w >> 2) + (l & 7), c4 = 4 * (w & 3) + (l >> 3);
+      const int64_t nr = tile * kHT + r;
+      const float4 v = nr < N ? __ldg(reinterpret_cast<const float4*>(latent + nr * IN) + c4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<uint2*>(bsm + Lay::ZT + tc::kmaj_off(r, c4 >> 1, IN) + (c4 & 1) * 8) =
+          make_uint2(tc::pack_half2(v.x, v.y), tc::pack_half2(v.z, v.w));
+    }
+    // ---- the adjoint of Eq. 11 and Eq. 2 from the saved raw outputs ----
+    float da[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (half == 0 && valid) {
+      float raw[8], s[3], r[4], cov_g[6], gs[3], gr[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) raw[i] = __ldg(raw_in + n * 8 + i);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) s[i] = expf(fminf(raw[i], 20.0f));
+      const float nrm = normalise_quat(raw + 3, r);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) cov_g[i] = g0(go.cov, 6 * n + i);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) gs[i] = g0(go.scale, 3 * n + i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) gr[i] = g0(go.rot, 4 * n + i);
+      covariance_backward(s, r, cov_g, gs, gr);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) da[i] = raw[i] <= 20.0f ? gs[i] * s[i] : 0.0f;
+      normalise_quat_backward(r, nrm, gr, da + 3);
+      const float o = sigmoidf_(raw[7]);
+      da[7] = g0(go.opacity, n) * o * (1.0f - o);
+    }
+    tiles_ready();
+
+#pragma unroll 1
+    for (int h = 0; h < 4; ++h) {
+      const int rows = hp.rows[h], pad = tc_pad(h, sh_pad), r3 = tc_row3(h, sh_pad);
+      const float* b1 = bias + h * 64;
+      const float* b2 = bias + 256 + h * 64;
+      float* sh_slot = slot + h * kHBHead;
+      float* bh = bacc + h * 192;   // db1 | db2 | db3
+      // ---- P1 = z W1^T ----
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_f16(P1, kdesc(Lay::ZT, 64, k), kdesc(Lay::W1 + h * 8192, 64, k), tc::idesc_f16_f32(kHT, 64), k > 0);
+      }
+      if (!wait_mma()) { failed = true; break; }
+      {
+        float v[32];
+        tc::tmem_ld32(P1 + lane + half * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + b1[half * 32 + i]);
+        store_row(Lay::H1, v);
+      }
+      tiles_ready();
+      // ---- P2 = h1 W2^T ----
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_f16(P2, kdesc(Lay::H1, 64, k), kdesc(Lay::W2 + h * 8192, 64, k), tc::idesc_f16_f32(kHT, 64), k > 0);
+      }
+      if (!wait_mma()) { failed = true; break; }
+      {
+        float v[32];
+        tc::tmem_ld32(P2 + lane + half * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + b2[half * 32 + i]);
+        store_row(Lay::H2, v);
+        // the head's output adjoint, zero past its rows (64 columns: rows of dW3 pad to 64)
+        float dy[32];
+        if (h == 2) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = half * 32 + i;
+            dy[i] = (valid && c < rows && go.sh) ? __ldg(go.sh + (int64_t)sh_rows * n + c) : 0.f;
+          }
+        } else {
+          const int base = h == 0 ? 0 : (h == 1 ? 3 : 7);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dy[i] = 0.f;
+          if (half == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dy[i] = i < rows ? da[min(base + i, 7)] : 0.f;
+          }
+        }
+        store_row(Lay::DY, dy);
+        col_partial(dy);
+      }
+      tiles_ready();
+      bias_add(bh + 128);
+      // ---- D = dy W3 ----
+      if (tid == 0) {
+        tc::fence_after_sync();
+        for (int k = 0; k < pad / 16; ++k)
+          tc::mma_f16(DD, kdesc(Lay::DY, 64, k), mdesc(Lay::W3 + r3 * 128, 64, k), tc::idesc_f16t_f32(kHT, 64, false, true),
+                      k > 0);
+      }
+      if (!wait_mma()) { failed = true; break; }
+      {
+        float d[32], p[32];
+        tc::tmem_ld32(DD + lane + half * 32, d);
+        tc::tmem_ld32(P2 + lane + half * 32, p);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] *= gelu_grad_fast(p[i] + b2[half * 32 + i]);
+        store_row(Lay::D2, d);
+        col_partial(d);
+      }
+      tiles_ready();
+      bias_add(bh + 64);
+      // ---- dW3 = dy^T h2 (into P2's columns, free now); D = d2 W2 ----
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_f16(P2, mdesc(Lay::DY, 64, k), mdesc(Lay::H2, 64, k), tc::idesc_f16t_f32(64, 64, true, true), k > 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_f16(DD, kdesc(Lay::D2, 64, k), mdesc(Lay::W2 + h * 8192, 64, k), tc::idesc_f16t_f32(kHT, 64, false, true),
+                      k > 0);
+      }
+      if (!wait_mma()) { failed = true; break; }
+      flush64(P2, sh_slot + kHBW3, rows);
+      {
+        float d[32], p[32];
+        tc::tmem_ld32(DD + lane + half * 32, d);
+        tc::tmem_ld32(P1 + lane + half * 32, p);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] *= gelu_grad_fast(p[i] + b1[half * 32 + i]);
+        store_row(Lay::DY, d);   // d1 over dy (its products are done)
+        col_partial(d);
+      }
+      tiles_ready();
+      bias_add(bh);
+      // ---- dW2 = d2^T h1 (P2's columns), dW1 = d1^T z (P1's), dz += d1 W1 ----
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_f16(P2, mdesc(Lay::D2, 64, k), mdesc(Lay::H1, 64, k), tc::idesc_f16t_f32(64, 64, true, true), k > 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_f16(P1, mdesc(Lay::DY, 64, k), mdesc(Lay::ZT, 64, k), tc::idesc_f16t_f32(64, 64, true, true), k > 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_f16(DZ, kdesc(Lay::DY, 64, k), mdesc(Lay::W1 + h * 8192, 64, k), tc::idesc_f16t_f32(kHT, 64, false, true),
+                      (h > 0 || k > 0) ? 1u : 0u);
+      }
+      if (!wait_mma()) { failed = true; break; }
+      flush64(P2, sh_slot + kHBW2, 64);
+      flush64(P1, sh_slot, 64);
+      tc::fence_before_sync();
+      __syncthreads();   // the next head rewrites P1, P2 and the tiles
+    }
+    if (failed) break;
+    // ---- dz into the tables: this thread's levels half*8 .. half*8 + 7 ----
+    {
+      float dz[32];
+      tc::tmem_ld32(DZ + lane + half * 32, dz);
+      if (valid) {
+        float xt[4];
+        normalise_position(pos[n], g, xt);
+#pragma unroll 1
+        for (int q = 0; q < 8; ++q) scatter_level<F>(xt, g, half * 8 + q, grad_tables, dz + 4 * q);
+      }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+  }
+
+  if (failed) {
+    if (tid == 0) atomicExch(&g_heads_device_error, 1);
+    tc::mbar_wait_bounded(mbar, phase ^ 1u, kHTWait);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!failed)
+    for (int p = tid; p < 4 * 3 * 64; p += kHTThreads) {
+      const int h = p / 192, k = p - h * 192, which = k >> 6, o = k & 63;
+      float* dst = slot + h * kHBHead + (which == 0 ? 64 * 64 : which == 1 ? kHBW2 + 64 * 64 : kHBB3);
+      dst[o] += bacc[p];
+    }
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// grad_weights (packed) += the padded slots of heads_bwd_tc_kernel, summed
+// over the slots in a fixed order.
+__global__ void heads_reduce_slots_tc(const float* __restrict__ ws, int n_slots, HeadsParams hp, int n_params,
+                                      float* __restrict__ out) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
+    int h = 0;
+    while (h < 3 && p >= hp.off[h + 1]) ++h;
+    const int q = p - hp.off[h];
+    const int w3_end = kHBW3 + hp.rows[h] * 64;
+    const int src = h * kHBHead + (q < w3_end ? q : kHBB3 + (q - w3_end));
+    float s = 0.0f;
+    for (int c = 0; c < n_slots; ++c) s += ws[(size_t)c * slot_stride(kHBSlot) + src];
+    out[p] += s;
+  }
+}
+
 __global__ void heads_reduce_slots(const float* __restrict__ ws, int n_slots, int n_params, float* __restrict__ out) {
   for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_params; p += gridDim.x * blockDim.x) {
     float s = 0.0f;
@@ -923,9 +1290,41 @@ struct HeadsLaunch {
                                              static_cast<const T*>(tables), static_cast<const W*>(weights), o);
     return launch_status();
   }
+  // the tensor-core backward (the forward's configuration, given its saved z and raw outputs)
+  static int bwd_tc(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* weights,
+                    const float* latent, const float* raw, const HeadsGrads& go, float* grad_tables,
+                    float* grad_weights, float* ws, int n_params, cudaStream_t s) {
+    auto k = heads_bwd_tc_kernel<F>;
+    const int smem = HeadsBwdLayout::BYTES;
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kHTThreads, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      if (occ < 1 || occ * 256 > 512) return SPIN4D_ERR_UNSUPPORTED;   // TMEM would be oversubscribed
+      configured[dev] = true;
+    }
+    const int blocks = persistent_blocks((N + kHT - 1) / kHT, 1);
+    k<<<blocks, kHTThreads, smem, s>>>(gp, hp, reinterpret_cast<const float4*>(pos), N,
+                                      static_cast<const __half*>(weights), latent, raw, go, grad_tables, ws);
+    SPIN4D_CHECK(launch_status());
+    heads_reduce_slots_tc<<<(n_params + 255) / 256, 256, 0, s>>>(ws, blocks, hp, n_params, grad_weights);
+    return launch_status();
+  }
   static int bwd(const GridParams& gp, const HeadsParams& hp, const float* pos, int64_t N, const void* tables,
                  const void* weights, const float* latent, const float* raw, const HeadsGrads& go, float* grad_tables,
                  float* grad_weights, float* ws, int n_params, cudaStream_t s) {
+    if constexpr (std::is_same<T, __half>::value && std::is_same<W, __half>::value && F == 4) {
+      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim % 16 == 0 && hp.sh_dim <= kHTMaxSh && latent && raw &&
+          ((uintptr_t)latent & 15) == 0) {
+        const int st = bwd_tc(gp, hp, pos, N, weights, latent, raw, go, grad_tables, grad_weights, ws, n_params, s);
+        if (st != SPIN4D_ERR_UNSUPPORTED) return st;   // else the SIMT backward below
+      }
+    }
     auto k = heads_bwd_kernel<T, F, W>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
     if (e != cudaSuccess) return cuda_status(e);
@@ -1029,7 +1428,10 @@ extern "C" int spin4d_heads_fwd(const spin4d_grid_desc* g, const spin4d_heads_de
 
 extern "C" size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_desc* h, int64_t N) {
   if (validate_grid(g) != SPIN4D_OK || validate_heads(g, h) != SPIN4D_OK || N <= 0) return 0;
-  return (size_t)bwd_blocks(N) * slot_stride((int)param_count(h)) * sizeof(float);
+  const size_t simt = (size_t)bwd_blocks(N) * slot_stride((int)param_count(h)) * sizeof(float);
+  // the tensor-core backward: one padded slot per CTA, one CTA per SM
+  const size_t tcb = (size_t)persistent_blocks((N + kHT - 1) / kHT, 1) * slot_stride(kHBSlot) * sizeof(float);
+  return split_forward(g, h) && tcb > simt ? tcb : simt;
 }
 
 extern "C" int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,

@@ -72,11 +72,12 @@ def test_heads_forward_matches_oracle(sp, case):
 
 @pytest.mark.parametrize("case,saved", [("tiny_fp32", ""), ("tiny_fp32", "latent+raw"), ("paper_fp16", ""),
                                         ("paper_fp16", "latent"), ("paper_fp16", "raw"), ("paper_fp16", "latent+raw"),
-                                        ("paper_fp16_init", "")])
+                                        ("paper_fp16_init", ""), ("paper_fp16_init", "latent+raw")])
 def test_heads_backward_matches_oracle(sp, case, saved):
     """With the forward's z and / or raw head outputs the backward skips the
     gather and / or the first recompute of the scale, rotation and opacity
-    heads; the gradients are the same."""
+    heads; the gradients are the same.  With both, the paper's configuration
+    runs the tensor-core backward."""
     grid, spec, pos, tables, weights, grads = _setup(case)
     g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
     P, T, W = dev(pos), dev(tables), dev(weights)
@@ -131,8 +132,10 @@ def test_grouped_adam_matches_oracle(sp):
 
 
 def test_heads_edge_sizes(sp):
-    """N = 0 launches nothing; N = 1 and N = 33 (one block and one more
-    position) match the oracle; the backward accumulates."""
+    """N = 0 launches nothing; N = 1, 33 and 129 (one block and one more
+    position; one tensor-core tile and one more) match the oracle, with the
+    SIMT backward and with the tensor-core one (saved z and raw outputs);
+    the backward accumulates."""
     grid, spec = S.GRID_PAPER, S.HEADS_PAPER
     g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
     tables = S.hash_tables(grid, seed=8, scale=1.0)
@@ -147,7 +150,7 @@ def test_heads_edge_sizes(sp):
     sp.heads_bwd(g, h, empty, T, W, {k: torch.zeros((0, w), device="cuda") for k, w in widths.items()}, gt, gw)
     torch.cuda.synchronize()
     assert not gt.any() and not gw.any()
-    for n in (1, 33):
+    for n in (1, 33, 129):
         pos = S.sports_scene(300_000).frame(75)[:n]
         grads = S.upstream_grads(n, widths, 1e-2, seed=10 + n)
         P = dev(pos)
@@ -167,6 +170,16 @@ def test_heads_edge_sizes(sp):
         # a second call adds the same gradient again
         tol.normwise(host(gt), 2 * host(first[0]), 1e-5, "accumulated grad_tables (N=%d)" % n)
         tol.normwise(host(gw), 2 * host(first[1]), 1e-5, "accumulated grad_weights (N=%d)" % n)
+        saved = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+        gt.zero_()
+        gw.zero_()
+        sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=saved["latent"], raw=saved["raw"])
+        tc_first = (gt.clone(), gw.clone())
+        sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=saved["latent"], raw=saved["raw"])
+        tol.normwise(host(tc_first[0]), wt, tol.FP16_GRAD_RTOL, "tc grad_tables (N=%d)" % n)
+        tol.normwise(host(tc_first[1]), ww, tol.FP16_GRAD_RTOL, "tc grad_weights (N=%d)" % n)
+        tol.normwise(host(gt), 2 * host(tc_first[0]), 1e-5, "tc accumulated grad_tables (N=%d)" % n)
+        tol.normwise(host(gw), 2 * host(tc_first[1]), 1e-5, "tc accumulated grad_weights (N=%d)" % n)
 
 
 def test_heads_full_launch_sampled_and_by_halves(sp):

@@ -134,6 +134,10 @@ def test_invalid_arguments_rejected_on_host(sp):
                                 sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_UNSUPPORTED
     assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
                                 sp.HeadsOutputs(FAKE, FAKE + 4, FAKE, FAKE, FAKE, None), None, 0, None) == sp.ERR_INVALID
+    # the backward's workspace covers the tensor-core kernel's padded slot (12480 floats per head,
+    # one CTA) even where the SIMT kernel's packed slots are smaller
+    assert lib.spin4d_heads_bwd_workspace(ref(gp4), ref(hs), 1) >= 4 * 12480 * 4
+    assert lib.spin4d_heads_bwd_workspace(ref(gp4), ref(hs), 0) == 0
     # the split forward's workspace: 64 fp16 per position; misaligned or short is rejected
     assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(hs), 10) == 10 * 128
     assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,

@@ -3,18 +3,22 @@
 // with GELU after the first two layers, on the shared latent z of the 4D
 // hash encoder (SPIN-4DGS section 3.3, Eqs. 9-11; Sigma by Eq. 2).
 //
-// fp32 SIMT kernels, 32 positions and 128 threads per block.  The hash
-// gather takes one (position, level group) per thread.  The layers run out
-// of shared memory: activations [position][feature], one layer's weights
-// staged as fp32 rows, every product register-blocked 4 x 4 over 16-byte
-// loads.  At the paper's size (L = 16, F = 4, T = 2^21: 256 MiB of fp16
-// tables) the corner gathers come from HBM and bound the forward.
+// Two implementations.  With fp16 tables and weights, F = 4, in_dim =
+// hidden = 64 and an SH head of 16, 32 or 48 rows (the paper's
+// configuration) the layers run on the tensor cores: the forward as a
+// full-occupancy gather of z into a workspace followed by heads_fwd_tc_kernel
+// (or that kernel alone, gathering itself, without a workspace), and the
+// backward, given the forward's z and raw outputs, as heads_bwd_tc_kernel.
+// Operands are fp16 (z, activations, deltas), accumulation fp32.  Every other
+// case runs the fp32 SIMT kernels below.
+//
+// SIMT kernels: 32 positions and 128 threads per block.  The hash gather
+// takes one (position, level group) per thread.  The layers run out of
+// shared memory: activations [position][feature], one layer's weights staged
+// as fp32 rows, every product register-blocked 4 x 4 over 16-byte loads.
 //
 // Forward: gather z, then per head two GELU layers and the output layer,
-// then Eq. 11 and Eq. 2.  With fp16 tables and weights, in_dim = hidden =
-// 64 and an SH head of 16, 32 or 48 rows (the paper's configuration) the
-// layers run on the tensor cores instead (heads_fwd_tc_kernel): z and the
-// hidden activations rounded to fp16, fp32 accumulation.
+// then Eq. 11 and Eq. 2.
 // Backward: forward again keeping the raw outputs of the scale, rotation
 // and opacity heads (they couple through Sigma), the activations' adjoint,
 // then per head the forward again with its pre-activations, the data

@@ -698,6 +698,10 @@ def run_workloads(args):
         sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws)
 
     emit("paper_heads_fp16", "fwd (saving z and raw head outputs) + bwd", n, timed(hfb, 5))
+    sp.heads_fwd(g, h, P, T, W, out=out)
+    emit("paper_heads_fp16", "bwd (saved z and raw head outputs)", n,
+         timed(lambda: sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws),
+               5))
     del P, T, W, out, fwd_out, grads, gt, gw, ws
     torch.cuda.empty_cache()
 

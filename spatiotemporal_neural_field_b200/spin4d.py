@@ -381,6 +381,10 @@ def heads_fwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, out=None, latent:
 
 def heads_bwd(g: GridDesc, h: HeadsDesc, pos, tables, weights, grads, grad_tables, grad_weights, latent=None,
               workspace=None, stream=None, raw=None) -> None:
+    """grad_tables and grad_weights += the gradients of sum_k <grads[k], output_k>.
+    latent and raw are the forward's saved z and raw head outputs (optional);
+    with both, the paper's configuration runs on the tensor cores.  The
+    workspace (uint8 device tensor) is allocated when not given."""
     N = pos.shape[0]
     if workspace is None:
         need = int(lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), N))

@@ -441,7 +441,10 @@ size_t spin4d_heads_bwd_workspace(const spin4d_grid_desc* g, const spin4d_heads_
  * grad_weights += (packed like weights, fp32, summed in a fixed order).
  * latent and raw (optional, each may be NULL) are the z and the raw head
  * outputs spin4d_heads_fwd saved for the same inputs; workspace as for
- * spin4d_decode_bwd, >= spin4d_heads_bwd_workspace bytes. */
+ * spin4d_decode_bwd, >= spin4d_heads_bwd_workspace bytes.  With both given
+ * (latent 16-byte aligned) the tensor-core configuration of spin4d_heads_desc
+ * runs its layers on the tensor cores with fp16 operands (z, activations,
+ * output adjoints, deltas) and fp32 accumulation; otherwise fp32 SIMT. */
 int spin4d_heads_bwd(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,
                      const void* tables, const void* weights, const float* latent, const float* raw,
                      const spin4d_heads_output_grads* grad_out, float* grad_tables, float* grad_weights,

@@ -381,8 +381,8 @@ int spin4d_check_device_errors(int clear);
  * in_dim = L*F; in_dim, hidden and sh_dim at most 64, in_dim and hidden
  * multiples of 4 (SPIN4D_ERR_UNSUPPORTED otherwise).  fp32 arithmetic, except
  * that the forward with fp16 tables and weights, F = 4, in_dim = hidden = 64,
- * sh_dim a multiple of 16 up to 48 and 16-byte aligned sh and raw runs its
- * layers on the tensor cores: z and the hidden activations are rounded to
+ * sh_dim = 48 and 16-byte aligned sh and raw runs its layers on the tensor
+ * cores: z and the hidden activations are rounded to
  * fp16, products accumulate in fp32 (the latent output stays fp32).
  */
 typedef struct spin4d_heads_desc {

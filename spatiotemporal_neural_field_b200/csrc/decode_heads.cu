@@ -4,7 +4,7 @@
 // hash encoder (SPIN-4DGS section 3.3, Eqs. 9-11; Sigma by Eq. 2).
 //
 // Two implementations.  With fp16 tables and weights, F = 4, in_dim =
-// hidden = 64 and an SH head of 16, 32 or 48 rows (the paper's
+// hidden = 64 and the degree-3 SH head of 48 rows (the paper's
 // configuration) the layers run on the tensor cores: the forward as a
 // full-occupancy gather of z into a workspace followed by heads_fwd_tc_kernel
 // (or that kernel alone, gathering itself, without a workspace), and the
@@ -534,8 +534,9 @@ constexpr size_t kFwdQSmem = ((size_t)3 * kHeadsBwdBlock * kQ + (size_t)kMaxDim 
 
 // ---------------------------------------------------------------------------
 // Forward on the tensor cores, for fp16 tables and weights with in_dim =
-// hidden = 64 (the paper's configuration) and an SH head of 16, 32 or 48
-// rows.  Persistent CTAs of 256 threads take tiles of 128 positions, two
+// hidden = 64 (the paper's configuration) and an SH head of 48 rows (the
+// code takes 16 or 32 as well; only 48, the tested size, is dispatched).
+// Persistent CTAs of 256 threads take tiles of 128 positions, two
 // threads per position (each gathers half of the levels and handles half of
 // every layer's columns).  z is rounded to fp16 into a K-major operand tile;
 // then, head by head, three tcgen05.mma chains (M = 128, K = 64; N = 64,
@@ -1281,7 +1282,7 @@ struct HeadsLaunch {
     if constexpr (std::is_same<T, __half>::value && std::is_same<W, __half>::value && F == 4) {
       // its vector stores want 16-byte rows of sh and raw
       const bool vec = ((uintptr_t)o.sh & 15) == 0 && ((uintptr_t)o.raw & 15) == 0;
-      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim % 16 == 0 && hp.sh_dim <= kHTMaxSh && vec) {
+      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim == kHTMaxSh && vec) {
         const int st = fwd_tc(gp, hp, pos, N, tables, weights, o, s);
         if (st != SPIN4D_ERR_UNSUPPORTED) return st;   // else the SIMT forward below
       }
@@ -1323,7 +1324,7 @@ struct HeadsLaunch {
                  const void* weights, const float* latent, const float* raw, const HeadsGrads& go, float* grad_tables,
                  float* grad_weights, float* ws, int n_params, cudaStream_t s) {
     if constexpr (std::is_same<T, __half>::value && std::is_same<W, __half>::value && F == 4) {
-      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim % 16 == 0 && hp.sh_dim <= kHTMaxSh && latent && raw &&
+      if (hp.in_dim == 64 && hp.hidden == 64 && hp.sh_dim == kHTMaxSh && latent && raw &&
           ((uintptr_t)latent & 15) == 0) {
         const int st = bwd_tc(gp, hp, pos, N, weights, latent, raw, go, grad_tables, grad_weights, ws, n_params, s);
         if (st != SPIN4D_ERR_UNSUPPORTED) return st;   // else the SIMT backward below
@@ -1384,7 +1385,7 @@ int run(const spin4d_grid_desc* g, const spin4d_heads_desc* h, bool bwd, const f
 // when given a workspace (otherwise it runs the fused tensor-core kernel).
 bool split_forward(const spin4d_grid_desc* g, const spin4d_heads_desc* h) {
   return g->table_dtype == SPIN4D_F16 && h->w_dtype == SPIN4D_F16 && g->F == 4 && h->in_dim == 64 &&
-         h->hidden == 64 && h->sh_dim % 16 == 0 && h->sh_dim <= kHTMaxSh;
+         h->hidden == 64 && h->sh_dim == kHTMaxSh;
 }
 
 int check_inputs(const spin4d_grid_desc* g, const spin4d_heads_desc* h, const float* pos, int64_t N,

@@ -140,6 +140,10 @@ def test_invalid_arguments_rejected_on_host(sp):
     assert lib.spin4d_heads_bwd_workspace(ref(gp4), ref(hs), 0) == 0
     # the split forward's workspace: 64 fp16 per position; misaligned or short is rejected
     assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(hs), 10) == 10 * 128
+    # only the tensor-core configuration (fp16 weights, hidden 64, 48 SH rows) asks for one
+    assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(sp.heads_desc(64, sh_dim=32)), 10) == 0
+    assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(sp.heads_desc(64, hidden=32)), 10) == 0
+    assert lib.spin4d_heads_fwd_workspace(ref(gp4), ref(sp.heads_desc(64, w_dtype="f32")), 10) == 0
     assert lib.spin4d_heads_fwd(ref(gp4), ref(hs), FAKE, 10, FAKE, FAKE,
                                 sp.HeadsOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None), FAKE, 10 * 128 - 1,
                                 None) == sp.ERR_INVALID

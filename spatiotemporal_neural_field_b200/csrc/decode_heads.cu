@@ -878,9 +878,23 @@ struct HeadsBwdLayout {
   static constexpr int PART = D2 + 16384;             // [4][64] fp32 column partial sums
   static constexpr int BACC = PART + 1024;            // [4 heads][3][64] fp32 bias gradients
   static constexpr int MISC = BACC + 3072;
-  static constexpr int BYTES = MISC + 16;
+  static constexpr int SCL = MISC + 16;               // operand scales: [4][2] weight-bound exponents,
+                                                      // [8 warps][4 heads] tile maxima of |dy|
+  static constexpr int BYTES = SCL + 256;
 };
 static_assert(HeadsTcLayout::BIAS + (512 + HeadsTcLayout::kW3Rows) * 4 <= HeadsBwdLayout::ZT, "layout overlap");
+
+// Power of two that brings a magnitude m below 2^10 (into [2^9, 2^10)): the
+// fp16 gradient tiles of the tensor-core backward are stored scaled by such
+// factors, so that small gradients keep fp16's 11-bit precision instead of
+// going subnormal, and no scaled value comes near fp16's maximum (65504).
+// Exact; 1 for m = 0 or a non-finite m.
+__device__ __forceinline__ float heads_pow2_below(float m, int target) {
+  if (!(m > 0.f) || !isfinite(m)) return 1.0f;
+  int e;
+  frexpf(m, &e);   // m = f 2^e, f in [0.5, 1)
+  return ldexpf(1.0f, max(-100, min(100, target - e)));
+}
 static_assert(HeadsBwdLayout::BYTES <= 227 * 1024, "backward tiles exceed one CTA's shared memory");
 
 template <int F>
@@ -916,8 +930,35 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
       bias[256 + h * 64 + o] = __half2float(w2[64 * 64 + o]);
     }
   }
+  // Weight bounds of the dgrad chain, per head: |d2| <= max|dy| * B3 * 1.2 and
+  // |d1| <= max|d2| * B2 * 1.2, with B the largest absolute column sum of W3
+  // (W2) and 1.2 above GELU's largest slope (1.129).  Their powers of two
+  // rescale d2 and d1 so that both stay below 2^10 after dy is scaled there.
+  int* wexp = reinterpret_cast<int*>(bsm + Lay::SCL);         // [h][0] for d2, [h][1] for d1
+  float* dymax = reinterpret_cast<float*>(bsm + Lay::SCL + 32);
+  float* dzinv = reinterpret_cast<float*>(bsm + Lay::SCL + 160);   // [4] unscaling of each head's dz
+  if (tid < 8) wexp[tid] = 0;
+  __syncthreads();
+  {
+    const int h = tid >> 6, j = tid & 63;
+    const __half* w2 = weights + hp.off[h] + 64 * IN + 64;
+    const __half* w3 = w2 + 64 * 64 + 64;
+    float b3 = 0.f, b2 = 0.f;
+    for (int i = 0; i < hp.rows[h]; ++i) b3 += fabsf(__half2float(w3[i * 64 + j]));
+    for (int i = 0; i < 64; ++i) b2 += fabsf(__half2float(w2[i * 64 + j]));
+    // non-negative floats order like their bit patterns
+    atomicMax(wexp + 2 * h, __float_as_int(1.2f * b3));
+    atomicMax(wexp + 2 * h + 1, __float_as_int(1.2f * b2));
+  }
+  __syncthreads();
+  if (tid < 8) {
+    const float b = __int_as_float(wexp[tid]);
+    int e = 0;
+    if (b > 0.f && isfinite(b)) frexpf(b, &e);   // b < 2^e
+    wexp[tid] = max(-60, min(60, e));
+  }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
     tc::tmem_relinquish();
   }
   if (tid == 0) {
@@ -931,6 +972,7 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t sbase = tc::smem_u32(bsm);
+  // each head's dz has its own accumulator (its own operand scale): DZ + 64 h
   const uint32_t P1 = tmem, P2 = tmem + 64, DD = tmem + 128, DZ = tmem + 192;
   // Row m of a 64-row (M = 64) accumulator sits in TMEM lane (m % 16) + 32 (m / 16):
   // warp w holds rows 16 (w % 4) + lane for lanes below 16, columns (w / 4) * 32 ..
@@ -951,10 +993,10 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
     tc::fence_after_sync();
     return !bad;
   };
-  auto store_row = [&](int off, const float v[32]) {
+  auto store_row = [&](int off, const float v[32], float sc) {
     uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = tc::pack_half2(v[2 * i], v[2 * i + 1]);
+    for (int i = 0; i < 16; ++i) pk[i] = tc::pack_half2(v[2 * i] * sc, v[2 * i + 1] * sc);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       *reinterpret_cast<uint4*>(bsm + off + tc::kmaj_off(row, half * 4 + q, 64)) =
@@ -968,18 +1010,20 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
   // column sums of this thread's 32 values over the tile's 128 rows: warp sums
   // into part[warp % 4][col], then (after the next barrier) bias_add adds
   // them in a fixed order
-  auto col_partial = [&](const float v[32]) {
+  auto col_partial = [&](const float v[32], float inv) {
     float t[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) t[i] = v[i];
+    for (int i = 0; i < 32; ++i) t[i] = v[i] * inv;
     part[(warp & 3) * 64 + half * 32 + lid] = warp_column_sum(t);
   };
   auto bias_add = [&](float* dst) {
     if (tid < 64) dst[tid] += part[tid] + part[64 + tid] + part[128 + tid] + part[192 + tid];
   };
-  auto flush64 = [&](uint32_t acc, float* dst, int nrows) {   // dst: 64 x 64 rows of the slot
+  auto flush64 = [&](uint32_t acc, float* dst, int nrows, float inv) {   // dst: 64 x 64 rows of the slot
     float a[32];
     tc::tmem_ld32(acc + lane + wcol, a);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] *= inv;
     if (wrow_ok && wrow < nrows) slot_add32(dst + wrow * 64 + wcol, a);
   };
 
@@ -1018,6 +1062,19 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
       const float o = sigmoidf_(raw[7]);
       da[7] = g0(go.opacity, n) * o * (1.0f - o);
     }
+    {
+      // this tile's largest |dy| per head (scale, rotation, SH, opacity)
+      float m[4] = {fmaxf(fabsf(da[0]), fmaxf(fabsf(da[1]), fabsf(da[2]))),
+                    fmaxf(fmaxf(fabsf(da[3]), fabsf(da[4])), fmaxf(fabsf(da[5]), fabsf(da[6]))), 0.f, fabsf(da[7])};
+      if (valid && go.sh)
+        for (int c = half * 32; c < min(sh_rows, half * 32 + 32); ++c)
+          m[2] = fmaxf(m[2], fabsf(__ldg(go.sh + (int64_t)sh_rows * n + c)));
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float wm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m[h])));
+        if (lid == 0) dymax[warp * 4 + h] = wm;
+      }
+    }
     tiles_ready();
 
 #pragma unroll 1
@@ -1027,6 +1084,15 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
       const float* b2 = bias + 256 + h * 64;
       float* sh_slot = slot + h * kHBHead;
       float* bh = bacc + h * 192;   // db1 | db2 | db3
+      // operand scales of this head on this tile: dy below 2^10 by its tile
+      // maximum, d2 and d1 further by the weight bounds (all powers of two)
+      float mdy = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) mdy = fmaxf(mdy, dymax[w * 4 + h]);
+      const float s_dy = heads_pow2_below(mdy, 10);
+      const float s_d2 = s_dy * ldexpf(1.0f, -wexp[2 * h]);
+      const float s_d1 = s_d2 * ldexpf(1.0f, -wexp[2 * h + 1]);
+      const float i_dy = 1.0f / s_dy, i_d2 = 1.0f / s_d2, i_d1 = 1.0f / s_d1;
       // ---- P1 = z W1^T ----
       if (tid == 0) {
         tc::fence_after_sync();
@@ -1040,7 +1106,7 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
         tc::tmem_ld32(P1 + lane + half * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + b1[half * 32 + i]);
-        store_row(Lay::H1, v);
+        store_row(Lay::H1, v, 1.0f);
       }
       tiles_ready();
       // ---- P2 = h1 W2^T ----
@@ -1056,7 +1122,7 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
         tc::tmem_ld32(P2 + lane + half * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + b2[half * 32 + i]);
-        store_row(Lay::H2, v);
+        store_row(Lay::H2, v, 1.0f);
         // the head's output adjoint, zero past its rows (64 columns: rows of dW3 pad to 64)
         float dy[32];
         if (h == 2) {
@@ -1074,8 +1140,8 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
             for (int i = 0; i < 4; ++i) dy[i] = i < rows ? da[min(base + i, 7)] : 0.f;
           }
         }
-        store_row(Lay::DY, dy);
-        col_partial(dy);
+        store_row(Lay::DY, dy, s_dy);
+        col_partial(dy, 1.0f);
       }
       tiles_ready();
       bias_add(bh + 128);
@@ -1093,8 +1159,9 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
         tc::tmem_ld32(P2 + lane + half * 32, p);
 #pragma unroll
         for (int i = 0; i < 32; ++i) d[i] *= gelu_grad_fast(p[i] + b2[half * 32 + i]);
-        store_row(Lay::D2, d);
-        col_partial(d);
+        // d holds d2 s_dy; stored as d2 s_d2
+        store_row(Lay::D2, d, s_d2 * i_dy);
+        col_partial(d, i_dy);
       }
       tiles_ready();
       bias_add(bh + 64);
@@ -1110,15 +1177,16 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
                       k > 0);
       }
       if (!wait_mma()) { failed = true; break; }
-      flush64(P2, sh_slot + kHBW3, rows);
+      flush64(P2, sh_slot + kHBW3, rows, i_dy);
       {
         float d[32], p[32];
         tc::tmem_ld32(DD + lane + half * 32, d);
         tc::tmem_ld32(P1 + lane + half * 32, p);
 #pragma unroll
         for (int i = 0; i < 32; ++i) d[i] *= gelu_grad_fast(p[i] + b1[half * 32 + i]);
-        store_row(Lay::DY, d);   // d1 over dy (its products are done)
-        col_partial(d);
+        // d holds d1 s_d2; stored as d1 s_d1 over dy (its products are done)
+        store_row(Lay::DY, d, s_d1 * i_d2);
+        col_partial(d, i_d2);
       }
       tiles_ready();
       bias_add(bh);
@@ -1133,20 +1201,32 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
           tc::mma_f16(P1, mdesc(Lay::DY, 64, k), mdesc(Lay::ZT, 64, k), tc::idesc_f16t_f32(64, 64, true, true), k > 0);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tc::mma_f16(DZ, kdesc(Lay::DY, 64, k), mdesc(Lay::W1 + h * 8192, 64, k), tc::idesc_f16t_f32(kHT, 64, false, true),
-                      (h > 0 || k > 0) ? 1u : 0u);
+          tc::mma_f16(DZ + 64 * h, kdesc(Lay::DY, 64, k), mdesc(Lay::W1 + h * 8192, 64, k),
+                      tc::idesc_f16t_f32(kHT, 64, false, true), k > 0 ? 1u : 0u);
       }
       if (!wait_mma()) { failed = true; break; }
-      flush64(P2, sh_slot + kHBW2, 64);
-      flush64(P1, sh_slot, 64);
+      flush64(P2, sh_slot + kHBW2, 64, i_d2);
+      flush64(P1, sh_slot, 64, i_d1);
+      if (tid == 0) dzinv[h] = i_d1;   // read after the loop
       tc::fence_before_sync();
       __syncthreads();   // the next head rewrites P1, P2 and the tiles
     }
     if (failed) break;
-    // ---- dz into the tables: this thread's levels half*8 .. half*8 + 7 ----
+    // ---- dz (the heads' accumulators, each unscaled) into the tables: this
+    // thread's levels half*8 .. half*8 + 7 ----
     {
       float dz[32];
       tc::tmem_ld32(DZ + lane + half * 32, dz);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dz[i] *= dzinv[0];
+#pragma unroll 1
+      for (int h = 1; h < 4; ++h) {
+        float t[32];
+        tc::tmem_ld32(DZ + 64 * h + lane + half * 32, t);
+        const float inv = dzinv[h];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dz[i] = fmaf(t[i], inv, dz[i]);
+      }
       if (valid) {
         float xt[4];
         normalise_position(pos[n], g, xt);
@@ -1172,7 +1252,7 @@ __global__ void __launch_bounds__(kHTThreads, 1) heads_bwd_tc_kernel(
     }
   if (warp == 0) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1310,7 +1390,7 @@ struct HeadsLaunch {
       int occ = 0;
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kHTThreads, smem);
       if (e != cudaSuccess) return cuda_status(e);
-      if (occ < 1 || occ * 256 > 512) return SPIN4D_ERR_UNSUPPORTED;   // TMEM would be oversubscribed
+      if (occ != 1) return SPIN4D_ERR_UNSUPPORTED;   // one CTA holds all 512 TMEM columns
       configured[dev] = true;
     }
     const int blocks = persistent_blocks((N + kHT - 1) / kHT, 1);

@@ -11,6 +11,7 @@ import pytest
 from oracle import decoder as dec
 from oracle import hashgrid as hg
 from spatiotemporal_neural_field_b200 import synthetic as S
+from tests import magnitude as mag
 from tests import tol
 
 pytestmark = pytest.mark.gpu
@@ -102,23 +103,40 @@ def test_encode_matches_oracle(sp, grid, kind, n, scale):
     g = sp.grid_from_spec(grid)
     z = host(sp.encode_fwd(g, dev(pos), dev(tables)))
     res = hg.grid_resolutions(grid.L, grid.nmin_s, grid.nmax_s, grid.nmin_t, grid.nmax_t)
-    want = hg.encode(hg.normalise(pos, grid.t_min, grid.t_max), tables, res, grid.log2_T)
-    # fp32 accumulation of exactly-read table values: per-level 16-term sums
-    scale_row = np.max(np.abs(tables.astype(np.float64)))
-    err = np.max(np.abs(z - want)) / scale_row
-    assert err <= tol.FP32_RTOL, err
+    xt = hg.normalise(pos, grid.t_min, grid.t_max)
+    want = hg.encode(xt, tables, res, grid.log2_T)
+    # fp32 accumulation of exactly-read table values: per-level 16-term sums,
+    # held to the terms' root-sum-square where they cancel
+    tol.elementwise(z, want, tol.FP32_RTOL, "z", tol.column_groups(grid.L * grid.F),
+                    rho=mag.encode_mag(xt, tables, res, grid.log2_T))
 
 
 # ---------------------------------------------------------------------------
 # decode forward
 # ---------------------------------------------------------------------------
+def check_fp32_outputs(got, want, keys=KEYS, tag="", extra_mag=None):
+    """fp32 attributes, element-wise per attribute.  A rotation component is
+    r^_k / ||r^||, rounded relative to the unit row norm, so its magnitude is
+    1; a covariance entry is computed from R's O(1) entries, so its
+    magnitude is the spectral norm max_k s_k^2 (tests/magnitude.py);
+    ``extra_mag`` gives the magnitudes of further keys."""
+    for k in keys:
+        rho = None
+        if k == "rot":
+            rho = np.ones_like(want[k])
+        elif k == "cov":
+            rho = mag.cov_mag(want["scale"])
+        elif extra_mag and k in extra_mag:
+            rho = extra_mag[k]
+        tol.elementwise(got[k], want[k], tol.FP32_RTOL, tag + k, rho=rho)
+
+
 def _check_outputs(out, want, fp32: bool):
-    for k in KEYS:
-        got = host(out[k])
-        if fp32:
-            tol.rowwise(got, want[k], tol.FP32_RTOL, k)
-        else:
-            tol.absolute(got, want[k], tol.FP16_ATOL, k)
+    if fp32:
+        check_fp32_outputs({k: host(out[k]) for k in KEYS}, want)
+    else:
+        for k in KEYS:
+            tol.absolute(host(out[k]), want[k], tol.FP16_ATOL, k)
     np.testing.assert_allclose(np.linalg.norm(host(out["rot"]), axis=1), 1.0, atol=1e-5)
 
 
@@ -206,6 +224,13 @@ BWD_CASES = {
 }
 
 
+def check_decode_grads(gt, gw, wt, ww, grid, mlp, rtol, rho=(None, None), tag=""):
+    """Element-wise per table level and per weight block (see tests/tol.py)."""
+    tol.elementwise(gt, wt, rtol, tag + "grad_tables", tol.table_levels(grid.L, 1 << grid.log2_T, grid.F),
+                    rho=rho[0])
+    tol.elementwise(gw, ww, rtol, tag + "grad_weights", tol.weight_blocks(mlp.layer_shapes()), rho=rho[1])
+
+
 def _bwd(sp, grid, mlp, pos, tables, weights, cr, grads):
     g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
     gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), dtype=torch.float32, device="cuda")
@@ -223,15 +248,8 @@ def test_decode_bwd_matches_oracle(sp, case):
     gt, gw = _bwd(sp, grid, mlp, pos, tables, weights, cr, grads)
     wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr)
     rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
-    tol.normwise(gt, wt, rtol, "grad_tables")
-    # each layer's block of the packed weight gradient on its own scale
-    o = 0
-    for (out_d, in_d) in mlp.layer_shapes():
-        tol.normwise(gw[o:o + out_d * in_d], ww[o:o + out_d * in_d], rtol, "dW %dx%d" % (out_d, in_d))
-        o += out_d * in_d
-        tol.normwise(gw[o:o + out_d], ww[o:o + out_d], rtol, "db %d" % out_d)
-        o += out_d
-    assert o == gw.size
+    check_decode_grads(gt, gw, wt, ww, grid, mlp, rtol,
+                       mag.decoder_rss(pos, tables, weights, grid, mlp, grads, gate_cr=cr))
 
 
 @pytest.mark.parametrize("name,n", [("sports_frame_fp16", 20011), ("stress_fp16_gate", 3001)])
@@ -245,11 +263,8 @@ def test_decode_bwd_covariance_only_gradient(sp, name, n):
     zeros = {k: np.zeros_like(v) for k, v in full.items()}
     zeros["cov"] = full["cov"]
     wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, zeros, gate_cr=cr)
-    tol.normwise(gt, wt, tol.FP16_GRAD_RTOL, "grad_tables")
-    o = 0
-    for (out_d, in_d) in mlp.layer_shapes():
-        tol.normwise(gw[o:o + out_d * in_d], ww[o:o + out_d * in_d], tol.FP16_GRAD_RTOL, "dW %dx%d" % (out_d, in_d))
-        o += out_d * in_d + out_d
+    check_decode_grads(gt, gw, wt, ww, grid, mlp, tol.FP16_GRAD_RTOL,
+                       mag.decoder_rss(pos, tables, weights, grid, mlp, zeros, gate_cr=cr))
 
 
 @pytest.mark.parametrize("name,n", [("tiny_fp32", 4099), ("sports_frame_fp16", 20011), ("stress_fp16_gate", 3001)])
@@ -272,12 +287,14 @@ def test_saved_latent_matches_encoder_and_feeds_backward(sp, name, n):
         gw = torch.zeros(mlp.n_params(), dtype=torch.float32, device="cuda")
         sp.decode_bwd(g, m, P, T, W, G, gt, gw, gate_cr=C, latent=lat)
         res.append((host(gt), host(gw)))
-    tol.normwise(res[0][0], res[1][0], 1e-4, "tables: saved latent vs re-gather")
-    tol.normwise(res[0][1], res[1][1], 1e-4, "weights: saved latent vs re-gather")
+    levels = tol.table_levels(grid.L, 1 << grid.log2_T, grid.F)
+    blocks = tol.weight_blocks(mlp.layer_shapes())
+    tol.normwise(res[0][0], res[1][0], 1e-4, "tables: saved latent vs re-gather", levels)
+    tol.normwise(res[0][1], res[1][1], 1e-4, "weights: saved latent vs re-gather", blocks)
     wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr)
     rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
-    tol.normwise(res[0][0], wt, rtol, "grad_tables")
-    tol.normwise(res[0][1], ww, rtol, "grad_weights")
+    check_decode_grads(res[0][0], res[0][1], wt, ww, grid, mlp, rtol,
+                       mag.decoder_rss(pos, tables, weights, grid, mlp, grads, gate_cr=cr))
 
 
 def test_decode_bwd_null_upstream_means_zero(sp):
@@ -289,8 +306,8 @@ def test_decode_bwd_null_upstream_means_zero(sp):
     full = {k: np.zeros((1000, w), np.float32) for k, w in S.DECODE_OUT_WIDTHS.items()}
     full["rgb"] = grads["rgb"]
     wt, ww = dec.decode_backward(pos, tables, weights, grid, mlp, full)
-    tol.normwise(gt, wt, tol.FP32_GRAD_RTOL, "grad_tables")
-    tol.normwise(gw, ww, tol.FP32_GRAD_RTOL, "grad_weights")
+    check_decode_grads(gt, gw, wt, ww, grid, mlp, tol.FP32_GRAD_RTOL,
+                       mag.decoder_rss(pos, tables, weights, grid, mlp, full))
 
 
 def test_decode_bwd_accumulates_and_is_linear_at_full_batch(sp):
@@ -316,8 +333,10 @@ def test_decode_bwd_accumulates_and_is_linear_at_full_batch(sp):
     # Same arithmetic per position; only the fp32 accumulation order differs
     # (atomics, per-block weight slots).  A coarse-level entry receives up to
     # K ~ 10^3 additions here, so the rounding bound is ~K * 2^-24 ~ 6e-5.
-    tol.normwise(host(gt2), host(gt), 1e-4, "tables: halves vs whole")
-    tol.normwise(host(gw2), host(gw), 1e-4, "weights: halves vs whole")
+    levels = tol.table_levels(grid.L, 1 << grid.log2_T, grid.F)
+    blocks = tol.weight_blocks(mlp.layer_shapes())
+    tol.normwise(host(gt2), host(gt), 1e-4, "tables: halves vs whole", levels)
+    tol.normwise(host(gw2), host(gw), 1e-4, "weights: halves vs whole", blocks)
     # sampled oracle check: the head-bias gradient is a plain sum of dy over
     # positions; check it on a 4000-row subset launched alone
     rows = np.random.default_rng(2).choice(len(pos), 4000, replace=False)
@@ -326,8 +345,8 @@ def test_decode_bwd_accumulates_and_is_linear_at_full_batch(sp):
     sub = {k: v[rows] for k, v in grads.items()}
     sp.decode_bwd(g, m, dev(pos[rows]), T, W, {k: dev(v) for k, v in sub.items()}, gt3, gw3)
     wt, ww = dec.decode_backward(pos[rows], tables, weights, grid, mlp, sub)
-    tol.normwise(host(gt3), wt, tol.FP16_GRAD_RTOL, "grad_tables subset")
-    tol.normwise(host(gw3), ww, tol.FP16_GRAD_RTOL, "grad_weights subset")
+    check_decode_grads(host(gt3), host(gw3), wt, ww, grid, mlp, tol.FP16_GRAD_RTOL,
+                       mag.decoder_rss(pos[rows], tables, weights, grid, mlp, sub), tag="subset ")
 
 
 # ---------------------------------------------------------------------------
@@ -342,7 +361,7 @@ def test_cov_assemble_matches_oracle(sp):
     q32, s32 = q.astype(np.float32), s.astype(np.float32)
     cov = host(sp.cov_assemble(dev(s32), dev(q32)))
     want = dec.covariance(s32.astype(np.float64), q32.astype(np.float64))
-    tol.rowwise(cov, want, tol.FP32_RTOL, "cov")
+    tol.elementwise(cov, want, tol.FP32_RTOL, "cov", tol.column_groups(6), rho=mag.cov_mag(s32))
 
 
 def test_adam_matches_oracle(sp):

@@ -6,7 +6,9 @@ import pytest
 from oracle import decoder as dec
 from oracle import heads as hd
 from spatiotemporal_neural_field_b200 import synthetic as S
+from tests import magnitude as mag
 from tests import tol
+from tests.test_parity_decode import check_fp32_outputs
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -50,12 +52,17 @@ def test_heads_forward_matches_oracle(sp, case):
     g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
     out = sp.heads_fwd(g, h, dev(pos), dev(tables), dev(weights), latent=True)
     want = hd.decode_forward(pos, tables, weights, grid, spec)
-    for k in ("scale", "rot", "sh", "opacity", "cov"):
-        if grid.dtype == "f32":
-            tol.rowwise(host(out[k]), want[k], tol.FP32_RTOL, k)
-        else:
+    keys = ("scale", "rot", "sh", "opacity", "cov")
+    if grid.dtype == "f32":
+        check_fp32_outputs({k: host(out[k]) for k in keys}, want, keys,
+                           extra_mag=dict(sh=mag.heads_output_mag(pos, tables, weights, grid, spec)))
+    else:
+        for k in keys:
             tol.absolute(host(out[k]), want[k], tol.FP16_ATOL, k)
-    tol.rowwise(host(out["latent"]), want["z"], tol.FP32_RTOL, "latent")
+    res, xt = dec._prepare(pos, grid, False)
+    z_rho = mag.encode_mag(xt, tables, res, grid.log2_T)
+    tol.elementwise(host(out["latent"]), want["z"], tol.FP32_RTOL, "latent", tol.column_groups(grid.L * grid.F),
+                    rho=z_rho)
     # the raw head outputs the forward saves for the backward: Eq. 11 inverts them
     raw = host(sp.heads_fwd(g, h, dev(pos), dev(tables), dev(weights), raw=True)["raw"]).astype(np.float64)
     tol.absolute(np.exp(np.minimum(raw[:, :3], 20.0)), want["scale"], tol.FP16_ATOL, "raw scale")
@@ -67,7 +74,8 @@ def test_heads_forward_matches_oracle(sp, case):
         fused = sp.heads_fwd(g, h, dev(pos), dev(tables), dev(weights), latent=True, workspace=None)
         for k in ("scale", "rot", "sh", "opacity", "cov"):
             tol.absolute(host(fused[k]), want[k], tol.FP16_ATOL, "fused " + k)
-        tol.rowwise(host(fused["latent"]), want["z"], tol.FP32_RTOL, "fused latent")
+        tol.elementwise(host(fused["latent"]), want["z"], tol.FP32_RTOL, "fused latent",
+                        tol.column_groups(grid.L * grid.F), rho=z_rho)
 
 
 @pytest.mark.parametrize("case,saved", [("tiny_fp32", ""), ("tiny_fp32", "latent+raw"), ("paper_fp16", ""),
@@ -89,16 +97,21 @@ def test_heads_backward_matches_oracle(sp, case, saved):
     sp.heads_bwd(g, h, P, T, W, {k: dev(v) for k, v in grads.items()}, gt, gw, latent=lat, raw=raw)
     wt, ww = hd.decode_backward(pos, tables, weights, grid, spec, grads)
     rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
-    tol.normwise(host(gt), wt, rtol, "grad_tables")
-    gwh = host(gw)
-    o = 0
+    check_heads_grads(host(gt), host(gw), wt, ww, grid, spec, rtol,
+                      mag.heads_rss(pos, tables, weights, grid, spec, grads))
+
+
+def check_heads_grads(gt, gw, wt, ww, grid, spec, rtol, rho=(None, None), tag=""):
+    """Element-wise per table level and per weight block of each head."""
+    tol.elementwise(gt, wt, rtol, tag + "grad_tables", tol.table_levels(grid.L, 1 << grid.log2_T, grid.F),
+                    rho=rho[0])
+    blocks, o = [], 0
     for head in range(4):
-        for (out_d, in_d) in spec.layer_shapes(head):
-            tol.normwise(gwh[o:o + out_d * in_d], ww[o:o + out_d * in_d], rtol, "dW head %d %dx%d" % (head, out_d, in_d))
-            o += out_d * in_d
-            tol.normwise(gwh[o:o + out_d], ww[o:o + out_d], rtol, "db head %d %d" % (head, out_d))
-            o += out_d
-    assert o == gwh.size
+        hb = tol.weight_blocks(spec.layer_shapes(head), "head %d " % head, o)
+        blocks += hb
+        o = hb[-1][1].stop
+    assert o == spec.n_params()
+    tol.elementwise(gw, ww, rtol, tag + "grad_weights", blocks, rho=rho[1])
 
 
 def test_grouped_adam_matches_oracle(sp):
@@ -165,8 +178,9 @@ def test_heads_edge_sizes(sp):
         first = (gt.clone(), gw.clone())
         sp.heads_bwd(g, h, P, T, W, G, gt, gw)
         wt, ww = hd.decode_backward(pos, tables, weights, grid, spec, grads)
-        tol.normwise(host(first[0]), wt, tol.FP16_GRAD_RTOL, "grad_tables (N=%d)" % n)
-        tol.normwise(host(first[1]), ww, tol.FP16_GRAD_RTOL, "grad_weights (N=%d)" % n)
+        rho = mag.heads_rss(pos, tables, weights, grid, spec, grads)
+        check_heads_grads(host(first[0]), host(first[1]), wt, ww, grid, spec, tol.FP16_GRAD_RTOL, rho,
+                          "(N=%d) " % n)
         # a second call adds the same gradient again
         tol.normwise(host(gt), 2 * host(first[0]), 1e-5, "accumulated grad_tables (N=%d)" % n)
         tol.normwise(host(gw), 2 * host(first[1]), 1e-5, "accumulated grad_weights (N=%d)" % n)
@@ -176,8 +190,8 @@ def test_heads_edge_sizes(sp):
         sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=saved["latent"], raw=saved["raw"])
         tc_first = (gt.clone(), gw.clone())
         sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=saved["latent"], raw=saved["raw"])
-        tol.normwise(host(tc_first[0]), wt, tol.FP16_GRAD_RTOL, "tc grad_tables (N=%d)" % n)
-        tol.normwise(host(tc_first[1]), ww, tol.FP16_GRAD_RTOL, "tc grad_weights (N=%d)" % n)
+        check_heads_grads(host(tc_first[0]), host(tc_first[1]), wt, ww, grid, spec, tol.FP16_GRAD_RTOL, rho,
+                          "tc (N=%d) " % n)
         tol.normwise(host(gt), 2 * host(tc_first[0]), 1e-5, "tc accumulated grad_tables (N=%d)" % n)
         tol.normwise(host(gw), 2 * host(tc_first[1]), 1e-5, "tc accumulated grad_weights (N=%d)" % n)
 
@@ -210,5 +224,5 @@ def test_heads_full_launch_sampled_and_by_halves(sp):
         sp.heads_bwd(g, h, P[a:b], T, W, {k: v[a:b] for k, v in G.items()}, gt2, gw2, latent=out["latent"][a:b],
                      raw=out["raw"][a:b])
     torch.cuda.synchronize()
-    tol.normwise(host(gt2), host(gt), 1e-4, "grad_tables by halves")
+    tol.normwise(host(gt2), host(gt), 1e-4, "grad_tables by halves", tol.table_levels(grid.L, 1 << grid.log2_T, grid.F))
     tol.normwise(host(gw2), host(gw), 1e-4, "grad_weights by halves")

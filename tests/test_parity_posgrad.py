@@ -7,7 +7,9 @@ import pytest
 
 from oracle import decoder as dec
 from spatiotemporal_neural_field_b200 import synthetic as S
+from tests import magnitude as mag
 from tests import tol
+from tests.test_parity_decode import check_decode_grads
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -67,25 +69,28 @@ def _run(sp, case, latent=False):
     sp.decode_bwd(g, m, P, T, W, {k: dev(v) for k, v in grads.items()}, gt, gw, gate_cr=CR, latent=lat, grad_pos=gp)
     sp.check_device_errors()
     want = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr, want_pos=True)
-    return grid, host(gt), host(gw), host(gp), want
+    rho = mag.decoder_rss(pos, tables, weights, grid, mlp, grads, gate_cr=cr, want_pos=True)
+    return grid, mlp, host(gt), host(gw), host(gp), want, rho
+
+
+AXES = tol.column_groups(3, ["x", "y", "z"])
 
 
 @pytest.mark.parametrize("case", list(CASES))
 def test_position_gradient_matches_oracle(sp, case):
-    grid, gt, gw, gp, (wt, ww, wp) = _run(sp, case)
+    grid, mlp, gt, gw, gp, (wt, ww, wp), rho = _run(sp, case)
     rtol = tol.FP32_GRAD_RTOL if grid.dtype == "f32" else tol.FP16_GRAD_RTOL
-    tol.normwise(gp, wp, rtol, "grad_pos")
+    tol.elementwise(gp, wp, rtol, "grad_pos", AXES, rho=rho[2])
     # the table and weight gradients of the same call are unchanged by it
-    tol.normwise(gt, wt, rtol, "grad_tables")
-    tol.normwise(gw, ww, rtol, "grad_weights")
+    check_decode_grads(gt, gw, wt, ww, grid, mlp, rtol, rho[:2])
 
 
 @pytest.mark.parametrize("case", ["sports", "stress_gate"])
 def test_position_gradient_with_saved_latent(sp, case):
     """The corners are gathered again for the position gradient even when the
     forward's latent replaces the second gather of z."""
-    grid, _, _, gp, (_, _, wp) = _run(sp, case, latent=True)
-    tol.normwise(gp, wp, tol.FP16_GRAD_RTOL, "grad_pos (saved latent)")
+    grid, _, _, _, gp, (_, _, wp), rho = _run(sp, case, latent=True)
+    tol.elementwise(gp, wp, tol.FP16_GRAD_RTOL, "grad_pos (saved latent)", AXES, rho=rho[2])
 
 
 def test_position_gradient_accumulates_and_matches_plain_backward(sp):
@@ -107,7 +112,8 @@ def test_position_gradient_accumulates_and_matches_plain_backward(sp):
     sp.decode_bwd(g, m, P, T, W, G, gt2, gw2, grad_pos=gp)
     # weight gradients are summed in a fixed order: bit-identical to the plain call
     assert torch.equal(gw1, gw2)
-    tol.normwise(host(gt2), host(gt1), 1e-5, "tables with and without grad_pos")
+    tol.normwise(host(gt2), host(gt1), 1e-5, "tables with and without grad_pos",
+                 tol.table_levels(grid.L, 1 << grid.log2_T, grid.F))
     first = gp.clone()
     sp.decode_bwd(g, m, P, T, W, G, gt2, gw2, grad_pos=gp)
     # each position is written by one thread, so the second call adds the same values
@@ -132,7 +138,8 @@ def test_position_gradient_normalised_input(sp):
     sp.decode_bwd(g, m, dev(xt), dev(tables), dev(weights), {k: dev(v) for k, v in grads.items()}, gt, gw,
                   grad_pos=gp)
     _, _, wp = dec.decode_backward(xt, tables, weights, grid, mlp, grads, normalised_input=True, want_pos=True)
-    tol.normwise(host(gp), wp, tol.FP32_GRAD_RTOL, "grad_pos (normalised input)")
+    rho = mag.decoder_rss(xt, tables, weights, grid, mlp, grads, normalised_input=True, want_pos=True)[2]
+    tol.elementwise(host(gp), wp, tol.FP32_GRAD_RTOL, "grad_pos (normalised input)", AXES, rho=rho)
     out_of_range = (xt[:, :3] < 0) | (xt[:, :3] > 1)
     assert out_of_range.any() and np.all(host(gp)[out_of_range] == 0)
 
@@ -162,28 +169,33 @@ def _gate_case(sp, grid, mlp, pos, n, tscale, gstd, latent=False):
     sp.check_device_errors()
     _, _, wp, wg = dec.decode_backward(pos, tables, weights, grid, mlp, grads, gate_cr=cr, want_pos=True,
                                        want_gate=True)
-    return host(gp), host(gg), wp, wg
+    rho_pos = mag.decoder_rss(pos, tables, weights, grid, mlp, grads, gate_cr=cr, want_pos=True)[2]
+    rho_gate = mag.gate_rss(pos, tables, weights, grid, mlp, grads, cr)
+    return host(gp), host(gg), wp, wg, rho_pos, rho_gate
+
+
+GATE = tol.column_groups(2, ["c", "r"])
 
 
 def test_gate_gradient_stress_tensor_core_path(sp):
     w = S.WORKLOADS["stress_fp16_gate"]
     n = 6007
-    gp, gg, wp, wg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0)
-    tol.normwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate")
-    tol.normwise(gp, wp, tol.FP16_GRAD_RTOL, "grad_pos alongside grad_gate")
+    gp, gg, wp, wg, rp, rg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0)
+    tol.elementwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate", GATE, rho=rg)
+    tol.elementwise(gp, wp, tol.FP16_GRAD_RTOL, "grad_pos alongside grad_gate", AXES, rho=rp)
 
 
 def test_gate_gradient_stress_saved_latent(sp):
     w = S.WORKLOADS["stress_fp16_gate"]
     n = 3001
-    _, gg, _, wg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0, latent=True)
-    tol.normwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate (saved latent)")
+    _, gg, _, wg, _, rg = _gate_case(sp, w["grid"], w["mlp"], S.stress_positions(n), n, 1.0, 1.0, latent=True)
+    tol.elementwise(gg, wg, tol.FP16_GRAD_RTOL, "grad_gate (saved latent)", GATE, rho=rg)
 
 
 def test_gate_gradient_fp32_simt_path(sp):
     mlp = dataclasses.replace(S.MLP_TINY, gate=True, tau=0.05)
     n = 4099
     pos = S.uniform_positions(n, seed=33)
-    gp, gg, wp, wg = _gate_case(sp, S.GRID_TINY, mlp, pos, n, 1.0, 1.0)
-    tol.normwise(gg, wg, tol.FP32_GRAD_RTOL, "grad_gate (fp32)")
-    tol.normwise(gp, wp, tol.FP32_GRAD_RTOL, "grad_pos (fp32, gated)")
+    gp, gg, wp, wg, rp, rg = _gate_case(sp, S.GRID_TINY, mlp, pos, n, 1.0, 1.0)
+    tol.elementwise(gg, wg, tol.FP32_GRAD_RTOL, "grad_gate (fp32)", GATE, rho=rg)
+    tol.elementwise(gp, wp, tol.FP32_GRAD_RTOL, "grad_pos (fp32, gated)", AXES, rho=rp)

@@ -20,6 +20,18 @@ features; align-corners bilinear (p = x~ * (res - 1), cell clamped to
 [d_mu 3 | d_q 4 | d_logs 3 | d_sh 48]; outputs mu' = mu + d_mu,
 q' = (q + d_q)/||q + d_q||, s' = exp(log s + d_logs), sh' = sh + d_sh and
 Sigma(s', q').
+
+Optional energy-flow window (KineticGS notes, "learnable energy-flow
+activation"): each Gaussian carries a window centre c and half-width r, and
+w = sigma((t~ - (c - r))/tau) sigma(((c + r) - t~)/tau) on the normalised
+time t~.  The notes gate the spatial displacement with a binary H(w) in
+{0, 1}, so that a Gaussian moves only inside its window, and modulate the
+features and the scale continuously by w.  Readings: H(w) = [w >= 1/2] (the
+notes give no threshold; 1/2 is where the window's two edges sit);
+mu' = mu + H(w) d_mu, s' = exp(log s + w d_logs), sh' = sh + w d_sh; the
+rotation offset, which the notes do not name among the modulated
+quantities, is left as it is.  H has zero derivative, so c and r receive
+gradient only through w (d_logs and d_sh).
 """
 from __future__ import annotations
 
@@ -106,39 +118,79 @@ def scatter_plane_grad(dz: np.ndarray, xt: np.ndarray, hx) -> np.ndarray:
     return grad
 
 
-def _outputs(y, inp):
+def energy_window(xt: np.ndarray, gate_cr, tau: float) -> np.ndarray:
+    """The double-sigmoid window w on the normalised time t~ (fp64)."""
+    cr = np.asarray(gate_cr, np.float64)
+    return decoder.temporal_gate(xt[:, 3].astype(np.float64), cr[:, 0], cr[:, 1], float(np.float32(tau)))
+
+
+def displacement_gate(w: np.ndarray) -> np.ndarray:
+    """H(w) in {0, 1}: 1 inside the window, read as w >= 1/2."""
+    return (np.asarray(w) >= 0.5).astype(np.float64)
+
+
+def _outputs(y, inp, w=None):
+    """Deformed Gaussians from the head output y; with the window weight w
+    the displacement is gated by H(w) and the scale and SH offsets scaled by w."""
     mu = np.asarray(inp["mu"], np.float64)
+    ones = np.ones(y.shape[0])
+    wm = ones if w is None else w
+    hm = ones if w is None else displacement_gate(w)
     qh = np.asarray(inp["q_can"], np.float64) + y[:, 3:7]
     q, _ = decoder.normalise_quat(qh)
-    s = np.exp(np.asarray(inp["logs_can"], np.float64) + y[:, 7:10])
-    return dict(mu=mu + y[:, 0:3], rot=q, scale=s,
-                sh=np.asarray(inp["sh_can"], np.float64) + y[:, 10:58],
+    s = np.exp(np.asarray(inp["logs_can"], np.float64) + wm[:, None] * y[:, 7:10])
+    return dict(mu=mu + hm[:, None] * y[:, 0:3], rot=q, scale=s,
+                sh=np.asarray(inp["sh_can"], np.float64) + wm[:, None] * y[:, 10:58],
                 cov=decoder.covariance(s, q)), qh
 
 
-def forward(inp: Dict[str, np.ndarray], planes, weights, hx) -> Dict[str, np.ndarray]:
+def _window(xt, hx, gate):
+    if gate is None:
+        return None
+    return energy_window(xt, gate["cr"], gate["tau"])
+
+
+def forward(inp: Dict[str, np.ndarray], planes, weights, hx, gate=None) -> Dict[str, np.ndarray]:
+    """``gate``: None, or dict(cr=N x 2 (c, r), tau=...) for the energy-flow window."""
     xt = normalise(inp["mu"], inp["frame"], hx.n_frames)
     z = encode(xt, planes, hx)
     layers = decoder.unpack_layers(weights, hx.layer_shapes())
     y, _, _ = decoder.mlp_forward(z, layers)
-    out, _ = _outputs(y, inp)
+    w = _window(xt, hx, gate)
+    out, _ = _outputs(y, inp, w)
     out["z"] = z
+    if w is not None:
+        out["w"] = w
     return out
 
 
-def backward(inp, planes, weights, hx, grads) -> Tuple[np.ndarray, np.ndarray]:
-    """Gradients of sum_k <grads[k], output_k> w.r.t. planes and weights."""
+def backward(inp, planes, weights, hx, grads, gate=None, want_gate=False):
+    """Gradients of sum_k <grads[k], output_k> w.r.t. planes and weights, and
+    with ``want_gate`` (gated only) w.r.t. the window's (c, r), N x 2."""
     xt = normalise(inp["mu"], inp["frame"], hx.n_frames)
     z = encode(xt, planes, hx)
     layers = decoder.unpack_layers(weights, hx.layer_shapes())
     y, acts, pres = decoder.mlp_forward(z, layers)
-    out, qh = _outputs(y, inp)
+    w = _window(xt, hx, gate)
+    out, qh = _outputs(y, inp, w)
     g = {k: np.asarray(v, np.float64) for k, v in grads.items()}
     ds_cov, dq_cov = decoder.covariance_backward(out["scale"], out["rot"], g["cov"])
+    dlogs = (g["scale"] + ds_cov) * out["scale"]          # d loss / d (log s + w d_logs)
+    wm = np.ones(y.shape[0]) if w is None else w
+    hm = np.ones(y.shape[0]) if w is None else displacement_gate(w)
     dy = np.zeros_like(y)
-    dy[:, 0:3] = g["mu"]
+    dy[:, 0:3] = hm[:, None] * g["mu"]
     dy[:, 3:7] = decoder.normalise_quat_backward(qh, g["rot"] + dq_cov)
-    dy[:, 7:10] = (g["scale"] + ds_cov) * out["scale"]
-    dy[:, 10:58] = g["sh"]
+    dy[:, 7:10] = wm[:, None] * dlogs
+    dy[:, 10:58] = wm[:, None] * g["sh"]
     dz, wgrads = decoder.mlp_backward(dy, layers, acts, pres)
-    return scatter_plane_grad(dz, xt, hx), decoder.pack_layers(wgrads)
+    result = (scatter_plane_grad(dz, xt, hx), decoder.pack_layers(wgrads))
+    if want_gate:
+        assert w is not None, "the window gradient needs a gated call"
+        # H(w) is piecewise constant: only the w-scaled offsets carry d loss / d w
+        dw = np.sum(dlogs * y[:, 7:10], axis=1) + np.sum(g["sh"] * y[:, 10:58], axis=1)
+        cr = np.asarray(gate["cr"], np.float64)
+        dwdc, dwdr = decoder.temporal_gate_grad(xt[:, 3].astype(np.float64), cr[:, 0], cr[:, 1],
+                                                float(np.float32(gate["tau"])))
+        result = result + (np.stack([dw * dwdc, dw * dwdr], axis=1),)
+    return result

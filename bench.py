@@ -13,6 +13,7 @@ the tables and the weight gradients).
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
 import argparse
+import dataclasses
 import ctypes
 import datetime
 import hashlib
@@ -46,12 +47,16 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fwd-bwd", action="store_true")
-    p.add_argument("--cpu-sample", type=int, default=300_000,
-                   help="positions the oracle decodes for cpu_baseline (the whole frame: ~10 s on one core)")
+    p.add_argument("--cpu-sample", type=int, default=100_000,
+                   help="positions the oracle decodes on one core for cpu_baseline (~4 s); every core's process "
+                        "decodes a quarter of that for the all-cores figure")
     p.add_argument("--no-probe", action="store_true", help="skip the random-gather ceiling measurement")
     p.add_argument("--workloads", action="store_true",
                    help="time every workload (fwd, and fwd+bwd where trained) and the device ceilings; "
                         "one JSON line each")
+    p.add_argument("--l2-window", action="store_true",
+                   help="time the 45-launch training step without and with an L2 access-policy window over the "
+                        "fp16 tables and over the fp32 table gradients; one JSON line each")
     p.add_argument("--cpu-workloads", action="store_true",
                    help="time the oracle on every workload (1 thread and all cores); one JSON line each")
     p.add_argument("--ncu-case", default=None,
@@ -76,10 +81,13 @@ def workload_config(n_gpus):
 
 
 def algorithmic_bytes_per_position():
-    """Useful bytes a position needs: 16 levels x 16 corners x F fp16 features,
-    its 16-byte (x,y,z,t) input and 17 fp32 outputs."""
+    """Useful table bytes a position needs: 16 levels x 16 corners x F fp16
+    features (its 16-byte input and 17 fp32 outputs come on top)."""
     g = S.WORKLOADS[WORKLOAD]["grid"]
-    return g.L * 16 * g.F * 2 + 16 + 17 * 4
+    return g.L * 16 * g.F * 2
+
+
+IO_BYTES_PER_POSITION = 16 + 17 * 4
 
 
 def measured_peaks():
@@ -168,6 +176,7 @@ def table_sectors_per_position(sp, g, pos_dev, F, elem_bytes, sample=20_000):
 def probe_sector_rates(sp, torch, dev):
     """Random 16-byte loads (one sector each) from a 32 MiB L2-resident buffer
     and from a 4 GiB buffer (HBM): the gather ceilings, sectors/s."""
+    from spatiotemporal_neural_field_b200 import probe as pr
     out = {}
     blocks = 4 * torch.cuda.get_device_properties(dev).multi_processor_count
     for name, nbytes, lpt in (("l2", 32 << 20, 4096), ("hbm", 4 << 30, 1024)):
@@ -176,7 +185,7 @@ def probe_sector_rates(sp, torch, dev):
         for it in range(4):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            n = sp.probe_gather(buf, 16, lpt, blocks, seed=it + 1)
+            n = pr.probe_gather(buf, 16, lpt, blocks, seed=it + 1)
             b.record()
             torch.cuda.synchronize()
             if it:
@@ -188,7 +197,7 @@ def probe_sector_rates(sp, torch, dev):
 
 
 def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, tables16, weights16, grid, mlp, g, m,
-                           flush, stream):
+                           flush, stream, l2_window=None):
     """One training step over the whole 150-frame sequence (45M positions):
     45 launches of 1M positions, each decode_fwd (saving z) + decode_bwd
     (gradients accumulate), then fused Adam on the fp32 master tables and
@@ -212,6 +221,10 @@ def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, table
     ws = torch.empty(max(sp.decode_bwd_workspace(g, m, nb), 1), dtype=torch.uint8, device=dev)
     b1, b2 = wt["betas"]
     state = {"step": 0}
+    window = None
+    if l2_window is not None:
+        # opt-in L2 residency over the fp16 tables or the fp32 table gradients
+        window = sp.l2_window_set(stream, {"tables": tab16, "grads": gtab}[l2_window])
 
     def step():
         for b in range(n_batches):
@@ -239,57 +252,128 @@ def train_step_measurement(args, sp, torch, dist, dev, world, rank, scene, table
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), device=dev) / k
+    if window is not None:
+        sp.l2_window_clear(stream)
     return {"metric": "decoded spatiotemporal positions/s (training step: fwd+bwd+Adam)",
+            "l2_window": None if window is None else {"over": l2_window, "bytes": window},
             "value": total * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "launches_per_step": 2 * n_batches + 2,
             "workload": "sports_train_fp16: 150 frames x 300k = 45M positions, 45 launches of 1M (decode_fwd saving z "
                         "+ decode_bwd), then fused Adam (lr 1e-3, betas (0.9, 0.99), eps 1e-15) on 16.8M table and "
                         "6987 weight parameters (fp32 master, fp16 working copy)"}
 
 
-def cpu_baseline(n_sample):
-    """The oracle, as it stands, on a bounded sample of the same workload."""
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+_WORKER = {}
+
+
+def _init_oracle_worker():
+    """Builds the frame, tables and weights once per spawned worker."""
+    sys.path.insert(0, ROOT)
+    w = S.WORKLOADS[WORKLOAD]
+    _WORKER["frame"] = S.sports_scene(w["N"]).frame(w["frame"])
+    _WORKER["tables"] = S.hash_tables(w["grid"])
+    _WORKER["weights"] = S.mlp_weights(w["mlp"])
+
+
+def _frame_decode_chunk(task):
+    """One worker's share of the oracle's frame decode: (seed, n) -> seconds
+    for n positions of the frame, single-threaded (0.2 s of sleep for n = 0,
+    which lines every worker up)."""
+    seed, n = task
+    if n == 0:
+        time.sleep(0.2)
+        return 0.0
+    if not _WORKER:
+        _init_oracle_worker()
     from threadpoolctl import threadpool_limits
     from oracle import decoder as dec
     w = S.WORKLOADS[WORKLOAD]
-    frame = S.sports_scene(w["N"]).frame(w["frame"])
-    rows = np.random.default_rng(7).choice(len(frame), n_sample, replace=False)
-    tables = S.hash_tables(w["grid"])
-    weights = S.mlp_weights(w["mlp"])
+    frame = _WORKER["frame"]
+    rows = np.random.default_rng(seed).choice(len(frame), n, replace=False)
     with threadpool_limits(limits=1):
         t0 = time.perf_counter()
-        dec.decode_forward(frame[rows], tables, weights, w["grid"], w["mlp"])
-        dt = time.perf_counter() - t0
-    return {"value": n_sample / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d positions of the same frame (numpy fp64, BLAS limited to 1 thread)" % n_sample,
-            "seconds": dt}
+        dec.decode_forward(frame[rows], _WORKER["tables"], _WORKER["weights"], w["grid"], w["mlp"])
+        return time.perf_counter() - t0
+
+
+class OraclePool:
+    """Spawned single-threaded worker processes, one per host core (spawn:
+    safe after the GPU work of the parent); each builds the workload's inputs
+    once, before anything is timed."""
+
+    def __init__(self):
+        import multiprocessing as mp
+        self.procs = os.cpu_count() or 1
+        self.pool = mp.get_context("spawn").Pool(self.procs, initializer=_init_oracle_worker)
+        for _ in range(2):   # every worker initialised and busy at once
+            self.pool.map(_frame_decode_chunk, [(i, 0) for i in range(self.procs)], chunksize=1)
+        self.pool.map(_frame_decode_chunk, [(i, 64) for i in range(self.procs)], chunksize=1)
+
+    def rate(self, per_proc, seed0=100):
+        """Positions/s of all workers decoding per_proc positions each."""
+        t0 = time.perf_counter()
+        self.pool.map(_frame_decode_chunk, [(seed0 + i, per_proc) for i in range(self.procs)], chunksize=1)
+        return per_proc * self.procs / (time.perf_counter() - t0)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(n_sample):
+    """The oracle, as it stands, on bounded samples of the same workload: one
+    thread, and one single-threaded spawned process per host core, each
+    decoding an equal share."""
+    one = _frame_decode_chunk((7, n_sample))
+    pool = OraclePool()
+    try:
+        per = max(n_sample // 4, 1000)
+        all_rate = pool.rate(per)
+    finally:
+        pool.close()
+    return {"value": all_rate, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
+            "sample": "%d processes x %d positions of the same frame (numpy fp64, one thread each)" % (pool.procs, per),
+            "host_cores": os.cpu_count(), "cpu_model": _cpu_model(),
+            "single_core": {"value": n_sample / one, "unit": UNIT, "cores": 1,
+                            "sample": "%d positions of the same frame (numpy fp64, BLAS limited to 1 thread)"
+                                      % n_sample, "seconds": one}}
 
 
 def run_reference(args):
+    """The reference arm: the oracle, as it stands, on the host's cores (one
+    single-threaded spawned process per core, each decoding its own sample of
+    the frame every step)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from threadpoolctl import threadpool_limits
-    from oracle import decoder as dec
-    w = S.WORKLOADS[WORKLOAD]
-    frame = S.sports_scene(w["N"]).frame(w["frame"])
-    tables = S.hash_tables(w["grid"])
-    weights = S.mlp_weights(w["mlp"])
-    sample = 10_000
-    rng = np.random.default_rng(11)
-    with threadpool_limits(limits=1):
-        for _ in range(args.warmup):
-            dec.decode_forward(frame[rng.choice(len(frame), sample, replace=False)], tables, weights, w["grid"], w["mlp"])
+    per = 10_000   # the oracle widens every table column per call: larger samples amortise that
+    pool = OraclePool()
+    try:
+        for i in range(args.warmup):
+            pool.rate(per, seed0=1000 * (i + 1))
         t0 = time.perf_counter()
-        for _ in range(args.steps):
-            dec.decode_forward(frame[rng.choice(len(frame), sample, replace=False)], tables, weights, w["grid"], w["mlp"])
+        for i in range(args.steps):
+            pool.rate(per, seed0=1000 * (args.warmup + i + 1))
         dt = time.perf_counter() - t0
-    value = sample * args.steps / dt
+    finally:
+        pool.close()
+    value = per * pool.procs * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(args.gpus),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": "%d positions of the frame per step" % sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
+                             "sample": "%d processes x %d positions of the frame per step" % (pool.procs, per),
+                             "cpu_model": _cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -500,9 +584,13 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": workload_config(world),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "roofline": {"bound": "l2_random_sector", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                         "bytes_per_position": bpp, "kernel": "decode_fwd"},
+                         "bytes_per_position": bpp, "io_bytes_per_position": IO_BYTES_PER_POSITION,
+                         "kernel": "decode_fwd_tc_kernel<2,32,64>",
+                         "note": "achieved = useful table bytes (16 levels x 16 corners x 2 fp16) per position x "
+                                 "positions / event time, against the driver's HBM copy peak; the tables (32 MiB) "
+                                 "are L2-resident, so the bound is the random 32-byte-sector rate of L2: see frac_l2"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clk,
@@ -511,6 +599,11 @@ def run_ours(args):
             line["fwd_bwd"] = fwd_bwd
         if gather:
             line["gather_roofline"] = gather
+            line["roofline"]["frac_l2"] = gather["frac_of_l2_random"]
+            line["roofline"]["l2_probe"] = (
+                "spin4d_probe_gather: 4 x SMs blocks of random 16-byte loads (one 32-byte sector each) over a "
+                "32 MiB L2-resident buffer, best of 3 timed runs; frac_l2 = the decoder's distinct table sectors "
+                "per position (from its own corner indices) x positions/s / that rate")
         if train:
             line["train_step"] = train
         if morton:
@@ -528,6 +621,7 @@ def device_ceilings(sp, torch, dev):
     line gather rates and sequential read bandwidth for an L2-resident
     (32 MiB) and an HBM-resident (4 GiB) buffer, the random-sector rate of a
     256 MiB buffer, and the fp32 FMA rate."""
+    from spatiotemporal_neural_field_b200 import probe as pr
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     def best(fn, reps=4):
@@ -545,25 +639,50 @@ def device_ceilings(sp, torch, dev):
     out = {}
     for name, nbytes, lpt in (("l2", 32 << 20, 4096), ("hbm", 4 << 30, 1024)):
         buf = torch.ones(nbytes // 4, dtype=torch.int32, device=dev)
-        out[name + "_random_sector_per_s"] = best(lambda it: sp.probe_gather(buf, 16, lpt, 4 * sms, seed=it + 1))
-        out[name + "_random_line128_per_s"] = best(lambda it: sp.probe_gather(buf, 128, lpt, 4 * sms, seed=it + 1))
+        out[name + "_random_sector_per_s"] = best(lambda it: pr.probe_gather(buf, 16, lpt, 4 * sms, seed=it + 1))
+        out[name + "_random_line128_per_s"] = best(lambda it: pr.probe_gather(buf, 128, lpt, 4 * sms, seed=it + 1))
         passes = 64 if name == "l2" else 2
-        out[name + "_sequential_bytes_per_s"] = best(lambda it: sp.probe_stream(buf, passes, 4 * sms))
+        out[name + "_sequential_bytes_per_s"] = best(lambda it: pr.probe_stream(buf, passes, 4 * sms))
         ops = 512 if name == "l2" else 128
         for wdt in (8, 16):
             out["%s_random_red%d_per_s" % (name, wdt)] = best(
-                lambda it: sp.probe_atomic(buf, wdt, ops, 4 * sms, seed=it + 1))
+                lambda it: pr.probe_atomic(buf, wdt, ops, 4 * sms, seed=it + 1))
         for rb in (128, 256):
             out["%s_random_bulk_red%d_rows_per_s" % (name, rb)] = best(
-                lambda it: sp.probe_bulk_reduce(buf, ops // 4, 8 * sms, seed=it + 1, row_bytes=rb))
+                lambda it: pr.probe_bulk_reduce(buf, ops // 4, 8 * sms, seed=it + 1, row_bytes=rb))
         del buf
     # random sectors of a buffer the size of the paper's tables (256 MiB: about
     # twice the L2, so part of the reads hit it as they do in the decoder)
     buf = torch.ones((256 << 20) // 4, dtype=torch.int32, device=dev)
-    out["tables256_random_sector_per_s"] = best(lambda it: sp.probe_gather(buf, 16, 1024, 4 * sms, seed=it + 1))
+    out["tables256_random_sector_per_s"] = best(lambda it: pr.probe_gather(buf, 16, 1024, 4 * sms, seed=it + 1))
     del buf
-    out["fp32_fma_flop_per_s"] = best(lambda it: sp.probe_fma(1 << 16, 8 * sms, dev))
+    out["fp32_fma_flop_per_s"] = best(lambda it: pr.probe_fma(1 << 16, 8 * sms, dev))
     return out
+
+
+def run_l2_window(args):
+    """The training step on a created stream: no window, a persisting window
+    over the fp16 tables, one over the fp32 table gradients."""
+    import torch
+    import torch.distributed as dist
+    from spatiotemporal_neural_field_b200 import build as _b
+    _b.build()
+    from spatiotemporal_neural_field_b200 import spin4d as sp
+    dev = torch.device("cuda", 0)
+    w = S.WORKLOADS[WORKLOAD]
+    grid, mlp = w["grid"], w["mlp"]
+    g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)
+    scene = S.sports_scene(w["N"])
+    tables = torch.from_numpy(S.hash_tables(grid)).to(dev)
+    weights = torch.from_numpy(S.mlp_weights(mlp)).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for which in (None, "tables", "grads", None):
+            r = train_step_measurement(args, sp, torch, dist, dev, 1, 0, scene, tables, weights, grid, mlp, g, m,
+                                       flush, s, l2_window=which)
+            print(json.dumps({"workload": "sports_train_fp16 training step", "l2_window": r["l2_window"],
+                              "ms_per_step": r["ms_per_step"], "positions_per_s": r["value"]}), flush=True)
 
 
 def run_workloads(args):
@@ -663,47 +782,10 @@ def run_workloads(args):
         del P, T, W, out, fwd_out, grads, gt, gw, ws, gpos
         torch.cuda.empty_cache()
 
-    # the paper's four-head GELU decoder, one 1M-position training launch
-    w = S.WORKLOADS["paper_heads_fp16"]
-    grid, spec, n = w["grid"], w["heads"], w["N"]
-    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
-    P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
-    T = torch.from_numpy(S.hash_tables(grid)).to(dev)
-    W = torch.from_numpy(S.heads_weights(spec)).to(dev)
-    out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
-    fwd_out = {k: v for k, v in out.items() if k not in ("latent", "raw")}
-    ms = timed(lambda: sp.heads_fwd(g, h, P, T, W, out=fwd_out), 10)
-    spp = table_sectors_per_position(sp, g, P, grid.F, 2)
-    emit("paper_heads_fp16", "fwd", n, ms, table_sectors_per_position=spp, sector_rate=spp * n / (ms * 1e-3),
-         frac_of_256mib_random_sector_ceiling=spp * n / (ms * 1e-3) / ceil["tables256_random_sector_per_s"],
-         mlp_flop_per_position=2 * sum(o * i for hd_ in range(4) for o, i in spec.layer_shapes(hd_)))
-    # the same launch decoded in Z-order (sorted once per scene; outputs in sorted order)
-    ws_sort = torch.empty(max(sp.lib.spin4d_morton_order_workspace(n), 1), dtype=torch.uint8, device=dev)
-    _, perm = sp.morton_order(g, P, workspace=ws_sort)
-    Ps = sp.permute_rows(P, perm)
-    ms_s = timed(lambda: sp.heads_fwd(g, h, Ps, T, W, out=fwd_out), 10)
-    emit("paper_heads_fp16", "fwd (Z-order sorted)", n, ms_s, table_sectors_per_position=spp,
-         sector_rate=spp * n / (ms_s * 1e-3),
-         frac_of_256mib_random_sector_ceiling=spp * n / (ms_s * 1e-3) / ceil["tables256_random_sector_per_s"])
-    del Ps, perm, ws_sort
-    grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
-             for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim).items()}
-    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
-    gw = torch.zeros(spec.n_params(), device=dev)
-    ws = torch.empty(max(sp.lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), n), 1),
-                     dtype=torch.uint8, device=dev)
-
-    def hfb():
-        sp.heads_fwd(g, h, P, T, W, out=out)
-        sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws)
-
-    emit("paper_heads_fp16", "fwd (saving z and raw head outputs) + bwd", n, timed(hfb, 5))
-    sp.heads_fwd(g, h, P, T, W, out=out)
-    emit("paper_heads_fp16", "bwd (saved z and raw head outputs)", n,
-         timed(lambda: sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws),
-               5))
-    del P, T, W, out, fwd_out, grads, gt, gw, ws
-    torch.cuda.empty_cache()
+    # the paper's four-head GELU decoder, one 1M-position training launch, at
+    # the measured table size 2^21 and at 2^23 (SPIN-4DGS section 4, Table 5)
+    for log2_T in (21, 23):
+        paper_heads_workload(sp, torch, dev, timed, emit, ceil, log2_T)
 
     # HexPlane
     w = S.WORKLOADS["hexplane_fp32"]
@@ -735,6 +817,51 @@ def run_workloads(args):
     torch.cuda.empty_cache()
     render_workloads(sp, torch, dev, timed)
     sp.check_device_errors()
+
+
+def paper_heads_workload(sp, torch, dev, timed, emit, ceil, log2_T):
+    """Times the paper decoder's 1M-position launch at table size 2^log2_T."""
+    w = S.WORKLOADS["paper_heads_fp16"]
+    grid, spec, n = dataclasses.replace(w["grid"], log2_T=log2_T), w["heads"], w["N"]
+    name = "paper_heads_fp16" if log2_T == 21 else "paper_heads_fp16_T2^%d" % log2_T
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
+    P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
+    T = torch.from_numpy(S.hash_tables(grid)).to(dev)
+    W = torch.from_numpy(S.heads_weights(spec)).to(dev)
+    out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+    fwd_out = {k: v for k, v in out.items() if k not in ("latent", "raw")}
+    ms = timed(lambda: sp.heads_fwd(g, h, P, T, W, out=fwd_out), 10)
+    spp = table_sectors_per_position(sp, g, P, grid.F, 2)
+    emit(name, "fwd", n, ms, table_sectors_per_position=spp, sector_rate=spp * n / (ms * 1e-3),
+         frac_of_256mib_random_sector_ceiling=spp * n / (ms * 1e-3) / ceil["tables256_random_sector_per_s"],
+         mlp_flop_per_position=2 * sum(o * i for hd_ in range(4) for o, i in spec.layer_shapes(hd_)))
+    # the same launch decoded in Z-order (sorted once per scene; outputs in sorted order)
+    ws_sort = torch.empty(max(sp.lib.spin4d_morton_order_workspace(n), 1), dtype=torch.uint8, device=dev)
+    _, perm = sp.morton_order(g, P, workspace=ws_sort)
+    Ps = sp.permute_rows(P, perm)
+    ms_s = timed(lambda: sp.heads_fwd(g, h, Ps, T, W, out=fwd_out), 10)
+    emit(name, "fwd (Z-order sorted)", n, ms_s, table_sectors_per_position=spp,
+         sector_rate=spp * n / (ms_s * 1e-3),
+         frac_of_256mib_random_sector_ceiling=spp * n / (ms_s * 1e-3) / ceil["tables256_random_sector_per_s"])
+    del Ps, perm, ws_sort
+    grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
+             for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim).items()}
+    gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
+    gw = torch.zeros(spec.n_params(), device=dev)
+    ws = torch.empty(max(sp.lib.spin4d_heads_bwd_workspace(ctypes.byref(g), ctypes.byref(h), n), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def hfb():
+        sp.heads_fwd(g, h, P, T, W, out=out)
+        sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws)
+
+    emit(name, "fwd (saving z and raw head outputs) + bwd", n, timed(hfb, 5))
+    sp.heads_fwd(g, h, P, T, W, out=out)
+    emit(name, "bwd (saved z and raw head outputs)", n,
+         timed(lambda: sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"], workspace=ws),
+               5))
+    del P, T, W, out, fwd_out, grads, gt, gw, ws
+    torch.cuda.empty_cache()
 
 
 def render_workloads(sp, torch, dev, timed):
@@ -820,25 +947,6 @@ def _oracle_job(name, what, n, seed):
     (for the render: n sampled pixels of the frame)."""
     from oracle import decoder as dec, hexplane as hxo, render as rdo
     rng = np.random.default_rng(seed)
-    if name == "paper_heads_fp16":
-        # 200k positions (a small case of the 1M launch): forward saving z, then the backward
-        grid, spec_h = w["grid"], w["heads"]
-        n = 200_000
-        g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec_h)
-        P = torch.from_numpy(S.sports_scene(300_000).frames(range(4))[:n]).to(dev)
-        T = torch.from_numpy(S.hash_tables(grid)).to(dev)
-        W = torch.from_numpy(S.heads_weights(spec_h)).to(dev)
-        grads = {k: torch.randn((n, wd), device=dev) * w["grad_std"]
-                 for k, wd in dict(S.HEADS_OUT_WIDTHS, sh=spec_h.sh_dim).items()}
-        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device=dev)
-        gw = torch.zeros(spec_h.n_params(), device=dev)
-        for _ in range(2):
-            out = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
-            sp.heads_bwd(g, h, P, T, W, grads, gt, gw, latent=out["latent"], raw=out["raw"])
-        torch.cuda.synchronize()
-        sp.check_device_errors()
-        print("ncu case done:", name)
-        return
     if name == "render_sports_frame":
         spec = S.orbit_camera(640, 360)
         sc = S.render_scene(300_000, seed=0)
@@ -1004,6 +1112,8 @@ def main():
     if args.ncu_case:
         run_ncu_case(args.ncu_case)
         return
+    if args.l2_window:
+        return run_l2_window(args)
     if args.cpu_workloads:
         run_cpu_workloads(args)
         return

@@ -53,7 +53,8 @@ typedef enum spin4d_status {
     SPIN4D_ERR_CUDA = -3,         /* a CUDA launch or query failed */
     SPIN4D_ERR_NONFINITE = -4,    /* a kernel met a non-finite value (see spin4d_adam_step) */
     SPIN4D_ERR_INJECTED = -5,     /* SPIN4D_FAULT selected this call */
-    SPIN4D_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out (see spin4d_check_device_errors) */
+    SPIN4D_ERR_TIMEOUT = -6,      /* a kernel's bounded wait ran out (see spin4d_check_device_errors) */
+    SPIN4D_ERR_BOUNDS = -7        /* checked build: a device bounds check failed */
 } spin4d_status;
 
 typedef enum spin4d_dtype { SPIN4D_F32 = 0, SPIN4D_F16 = 1 } spin4d_dtype;
@@ -235,14 +236,19 @@ int spin4d_decode_bwd_ext(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
  * process exits.  Returns SPIN4D_ERR_INVALID, launching nothing, when the
  * scratch this (g, m, N) needs (spin4d_decode_bwd_workspace) is larger.
  * The first call on each device looks the array's device address up
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  All calls share the one array: calls that
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the life
+ * of the process; make that first call before any stream capture.  A device
+ * reset (cudaDeviceReset, or the primary context destroyed and created again)
+ * can move the array, and the kept address is then stale: do not call this
+ * entry point after resetting a device it has already run on.  All calls share the one array: calls that
  * overlap on the GPU (different streams, or different host threads) race and
  * corrupt each other's weight gradients; serialise them.  Each call writes
  * every part of the scratch it reads, so nothing needs clearing between calls.
  * Other arguments, results and errors are those of spin4d_decode_bwd.
  */
 #define SPIN4D_NOALLOC_SCRATCH_BYTES (16u << 20)
+/* The size of that array as this library was compiled (bytes). */
+size_t spin4d_decode_bwd_noalloc_scratch_bytes(void);
 int spin4d_decode_bwd_noalloc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m,
                               const float* pos, int64_t N, const void* tables, const void* weights,
                               const float* gate_cr, const float* latent, const spin4d_output_grads* grad_out,
@@ -352,6 +358,49 @@ int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const in
                         void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 
 /*
+ * The energy-flow window of the KineticGS notes ("learnable energy-flow
+ * activation") on the HexPlane deformation.  Each Gaussian carries a window
+ * centre c and half-width r; on the normalised time t~ = frame/(n_frames - 1)
+ *   w = sigma((t~ - (c - r))/tau) sigma(((c + r) - t~)/tau).
+ * The notes gate the spatial displacement with a binary H(w) in {0, 1}, so a
+ * Gaussian moves only inside its window, and modulate the scale and the
+ * features continuously by w.  Read here as H(w) = [w >= 1/2] and
+ *   mu' = mu + H(w) d_mu,  s' = exp(logs_can + w d_logs),  sh' = sh_can + w d_sh,
+ * with the rotation offset (not among the quantities the notes modulate)
+ * applied as without the window.  H has zero derivative: c and r receive
+ * gradient through w alone.
+ *   cr:      N x 2 (c, r) fp32, device, 8-byte aligned.
+ *   tau:     > 0 and finite.
+ *   grad_cr: backward only: N x 2 fp32, 8-byte aligned, += d loss / d(c, r);
+ *            NULL for none.  Each Gaussian's pair is written by one thread.
+ */
+typedef struct spin4d_hex_gate {
+    const float* cr;
+    float tau;
+    float* grad_cr;
+} spin4d_hex_gate;
+
+/* spin4d_hexplane_fwd with the window (gate not NULL).  Other arguments,
+ * results and errors are those of spin4d_hexplane_fwd; SPIN4D_ERR_INVALID for
+ * a bad gate or a non-NULL gate->grad_cr. */
+int spin4d_hexplane_fwd_gated(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                              int64_t N, const float* planes, const float* weights,
+                              const float* q_can, const float* logs_can, const float* sh_can,
+                              const spin4d_hex_gate* gate, spin4d_hex_outputs out, spin4d_stream_t stream);
+
+/* spin4d_hexplane_bwd with the window (gate not NULL), and d loss / d(c, r)
+ * into gate->grad_cr when given.  Other arguments, results and errors are
+ * those of spin4d_hexplane_bwd; SPIN4D_ERR_UNSUPPORTED where only the fp32
+ * SIMT kernels could run. */
+int spin4d_hexplane_bwd_gated(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                              int64_t N, const float* planes, const float* weights,
+                              const float* q_can, const float* logs_can, const float* sh_can,
+                              const float* latent, const spin4d_hex_gate* gate,
+                              const spin4d_hex_output_grads* grad_out,
+                              float* grad_planes, float* grad_weights,
+                              void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/*
  * Test hook: the interpolation cell of every position at every level, as the
  * kernels compute it.  idx N x L x 16 uint32 (corner c selects vertex
  * base_d + bit d of c, d = 0 x, 1 y, 2 z, 3 t); frac N x L x 4 fp32
@@ -364,8 +413,10 @@ int spin4d_debug_corners(const spin4d_grid_desc* g, const float* pos, int64_t N,
  * Synchronous: reads the library's device error word, set by a kernel whose
  * bounded wait for its own tensor-core work ran out (the kernel then frees
  * its tensor memory and exits early, leaving its outputs incomplete).
- * Returns SPIN4D_OK or SPIN4D_ERR_TIMEOUT; clear != 0 resets the word.
- * Waits for the current device's legacy default stream.
+ * Returns SPIN4D_OK or SPIN4D_ERR_TIMEOUT; clear != 0 resets the word.  In
+ * the checked build (spin4d_checked_build) also SPIN4D_ERR_BOUNDS when a
+ * device bounds check failed (it takes precedence; clear resets those
+ * words too).  Waits for the current device's legacy default stream.
  */
 int spin4d_check_device_errors(int clear);
 
@@ -593,68 +644,33 @@ int spin4d_render_bwd(const spin4d_camera* cam, const spin4d_render_desc* desc, 
                       float* grad_opacity, float* grad_colours, spin4d_stream_t stream);
 
 /*
- * Measurement helper (not part of the decoder): the gather-rate ceiling.
- * Launches `blocks` x 256 threads; each issues `loads_per_thread` (a multiple
- * of 8) independent loads at pseudo-random, width-aligned offsets of `buf`
- * (device, `buf_bytes` long, 16-byte aligned; 128-byte aligned for width
- * 128), eight in flight per thread.  width 4 or 16: every load is its own
- * 4- or 16-byte access inside one 32-byte sector, so loads / elapsed time is
- * the random-sector rate of wherever `buf` lives (L2 for a buffer well under
- * the L2 size, HBM for one far above it).  width 128: each group of 8
- * consecutive lanes reads one random 128-byte line, 16 bytes per lane, so
- * (blocks x 256 x loads_per_thread / 8) / elapsed time is the random-line
- * rate.  `sink` (device, 4 bytes) is written only to keep the loads alive.
+ * Opt-in L2 residency for one buffer (the hash tables, say) on one stream:
+ * the stream's access-policy window covers [base, base + bytes) with the
+ * persisting property, and the current context's persisting-L2 set-aside
+ * (cudaLimitPersistingL2CacheSize) is raised to the window's size, at most
+ * cudaDevAttrMaxPersistingL2CacheSize.  Kernels later launched on `stream`
+ * keep that range in L2 ahead of streaming data.  The library never sets a
+ * window by itself.
+ *   stream: a created stream (not NULL: the legacy stream takes no window).
+ *   bytes is clipped to cudaDevAttrMaxAccessPolicyWindowSize; the clipped
+ *   size goes to *applied_bytes when that is not NULL.
+ * SPIN4D_ERR_UNSUPPORTED where the device has no persisting L2.
+ * spin4d_l2_window_clear removes the stream's window, returns persisting
+ * lines to normal (cudaCtxResetPersistingL2Cache) and restores the
+ * context's set-aside to its value before the first spin4d_l2_window_set.
+ * Both calls are host-synchronous configuration, not stream work.
  */
-int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int width, int64_t loads_per_thread, int blocks,
-                        uint32_t seed, uint32_t* sink, spin4d_stream_t stream);
+int spin4d_l2_window_set(spin4d_stream_t stream, const void* base, size_t bytes, size_t* applied_bytes);
+int spin4d_l2_window_clear(spin4d_stream_t stream);
 
 /*
- * Measurement helper: the scatter-add ceiling.  `blocks` x 256 threads each
- * issue `ops_per_thread` (a multiple of 8) fp32 reductions (red.global.add,
- * `width` = 4, 8 or 16 bytes: 1, 2 or 4 floats of +1.0) at pseudo-random,
- * width-aligned offsets of `buf` (device, 16-byte aligned, `buf_bytes`
- * long, modified); operations / elapsed time is the random-atomic rate of
- * wherever `buf` lives.
+ * 1 if this library was compiled with SPIN4D_CHECKED (libspin4d_checked.so),
+ * else 0.  The checked build verifies on the device that every hash-table
+ * index is below T and every HexPlane cell lies inside its plane; a failed
+ * check is recorded and the access redirected to a valid address (nothing
+ * traps), and spin4d_check_device_errors then returns SPIN4D_ERR_BOUNDS.
  */
-int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int64_t ops_per_thread, int blocks,
-                        uint32_t seed, spin4d_stream_t stream);
-
-/*
- * Measurement helper: the row scatter-add ceiling.  `blocks` x 128 threads
- * each add a row of fp32 ones (`row_bytes` = 128 or 256) to
- * `rows_per_thread` pseudo-random, row-aligned rows of `buf` (device,
- * 128-byte aligned, modified) with bulk asynchronous reductions
- * (cp.reduce.async.bulk .add.f32), up to 8 in flight per thread; rows /
- * elapsed time is the rate.
- */
-int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int row_bytes, int64_t rows_per_thread, int blocks,
-                             uint32_t seed, spin4d_stream_t stream);
-
-/*
- * Measurement helper: reads `buf` (device, 16-byte aligned, buf_bytes a
- * multiple of 16) front to back `passes` times with 16-byte loads from
- * `blocks` x 256 threads; passes x buf_bytes / elapsed time is the
- * sequential read bandwidth of wherever `buf` lives.
- */
-int spin4d_probe_stream(const void* buf, uint64_t buf_bytes, int passes, int blocks, uint32_t* sink,
-                        spin4d_stream_t stream);
-
-/*
- * Measurement helper: `blocks` x 256 threads each run 8 independent fp32 FMA
- * chains for `iters` steps; 16 x iters x blocks x 256 / elapsed time is the
- * CUDA-core fp32 rate in FLOP/s.
- */
-int spin4d_probe_fma(int64_t iters, int blocks, uint32_t* sink, spin4d_stream_t stream);
-
-/*
- * Test hook for failure detection: one block waits (at most max_iters polls,
- * 1..2^24) on a barrier that nothing ever arrives at, through the same
- * bounded-wait path the tensor-core kernels use; the wait runs out, the
- * kernel sets the device error word and exits.  A following
- * spin4d_check_device_errors returns SPIN4D_ERR_TIMEOUT.  Nothing hangs and
- * the context stays usable.
- */
-int spin4d_selftest_wait_timeout(uint32_t max_iters, spin4d_stream_t stream);
+int spin4d_checked_build(void);
 
 /* Static string for a status code. */
 const char* spin4d_status_string(int status);

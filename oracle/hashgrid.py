@@ -155,20 +155,29 @@ def encode(xt: np.ndarray, tables: np.ndarray, res: np.ndarray, log2_T: int) -> 
     return z
 
 
-def scatter_table_grad(dz: np.ndarray, xt: np.ndarray, res: np.ndarray, log2_T: int,
-                       L: int, F: int) -> np.ndarray:
-    """Adjoint of ``encode`` w.r.t. the tables: grad[l, idx_c, f] += weight_c * dz."""
+def scatter_table_grad_level(dz: np.ndarray, xt: np.ndarray, res: np.ndarray, log2_T: int, l: int,
+                             F: int) -> np.ndarray:
+    """Level l of the adjoint of ``encode`` w.r.t. the tables, T x F:
+    grad[idx_c, f] += weight_c * dz[:, l*F + f] (for tables too large to hold
+    every level's fp64 gradient at once)."""
     T = 1 << log2_T
     _, frac, idx = corner_select(xt, res, log2_T)
     wts = corner_weights(frac)
-    grad = np.zeros((L, T, F), np.float64)
+    grad = np.zeros((T, F), np.float64)
+    for f in range(F):
+        g = dz[:, l * F + f]
+        # all 16 corners of every position in one serial histogram
+        grad[:, f] = np.bincount(idx[:, l, :].astype(np.int64).reshape(-1),
+                                 weights=(wts[:, l, :] * g[:, None]).reshape(-1), minlength=T)
+    return grad
+
+
+def scatter_table_grad(dz: np.ndarray, xt: np.ndarray, res: np.ndarray, log2_T: int,
+                       L: int, F: int) -> np.ndarray:
+    """Adjoint of ``encode`` w.r.t. the tables: grad[l, idx_c, f] += weight_c * dz."""
+    grad = np.zeros((L, 1 << log2_T, F), np.float64)
     for l in range(L):
-        for f in range(F):
-            g = dz[:, l * F + f]
-            # all 16 corners of every position in one serial histogram
-            grad[l, :, f] = np.bincount(idx[:, l, :].astype(np.int64).reshape(-1),
-                                        weights=(wts[:, l, :] * g[:, None]).reshape(-1),
-                                        minlength=T)
+        grad[l] = scatter_table_grad_level(dz, xt, res, log2_T, l, F)
     return grad
 
 

@@ -123,8 +123,10 @@ def decode_forward(pos, tables, weights, grid, spec, normalised_input=False) -> 
     return out
 
 
-def decode_backward(pos, tables, weights, grid, spec, grads, normalised_input=False):
-    """(grad_tables L x T x F, grad_weights packed like ``weights``)."""
+def latent_backward(pos, tables, weights, grid, spec, grads, normalised_input=False):
+    """(res, xt, dz N x LF, grad_weights packed): the backward up to the
+    latent's adjoint dz, which ``hashgrid.scatter_table_grad`` (or, a level
+    at a time, ``scatter_table_grad_level``) spreads over the tables."""
     res, xt, z = _latent(pos, tables, grid, normalised_input)
     heads = unpack(weights, spec)
     fw = [head_forward(z, heads[h]) for h in range(4)]
@@ -136,8 +138,13 @@ def decode_backward(pos, tables, weights, grid, spec, grads, normalised_input=Fa
         d, g = head_backward(dy[name], heads[h], fw[h][1], fw[h][2])
         dz += d
         wgrads.append(g)
-    gt = hashgrid.scatter_table_grad(dz, xt, res, grid.log2_T, grid.L, grid.F)
-    return gt, pack(wgrads)
+    return res, xt, dz, pack(wgrads)
+
+
+def decode_backward(pos, tables, weights, grid, spec, grads, normalised_input=False):
+    """(grad_tables L x T x F, grad_weights packed like ``weights``)."""
+    res, xt, dz, gw = latent_backward(pos, tables, weights, grid, spec, grads, normalised_input)
+    return hashgrid.scatter_table_grad(dz, xt, res, grid.log2_T, grid.L, grid.F), gw
 
 
 def lr_warmup_cosine(step: int, lr_max: float, lr_min: float, warmup: int, total: int) -> float:

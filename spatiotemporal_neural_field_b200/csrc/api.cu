@@ -135,6 +135,30 @@ __global__ void cov_assemble_kernel(const float* __restrict__ scale, const float
 
 using namespace spin4d;
 
+namespace spin4d {
+// Readers of the translation units' bounds words (checked build only; they
+// register themselves while the library loads).
+static int (*g_bounds_readers[32])(int) = {nullptr};
+static int g_n_bounds_readers = 0;
+
+int register_bounds_word(int (*reader)(int clear)) {
+  if (g_n_bounds_readers < 32) g_bounds_readers[g_n_bounds_readers++] = reader;
+  return g_n_bounds_readers;
+}
+
+// SPIN4D_ERR_BOUNDS if a checked-build bounds check failed since the last
+// clear, SPIN4D_ERR_CUDA if a word could not be read, else SPIN4D_OK.
+int bounds_status(int clear) {
+  int st = SPIN4D_OK;
+  for (int i = 0; i < g_n_bounds_readers; ++i) {
+    const int v = g_bounds_readers[i](clear);
+    if (v < 0) return SPIN4D_ERR_CUDA;
+    if (v) st = SPIN4D_ERR_BOUNDS;
+  }
+  return st;
+}
+}  // namespace spin4d
+
 extern "C" {
 
 int spin4d_grid_init(spin4d_grid_desc* g, int L, int F, int log2_T, int table_dtype, int nmin_s,
@@ -196,11 +220,86 @@ const char* spin4d_status_string(int s) {
     case SPIN4D_ERR_NONFINITE: return "non-finite value";
     case SPIN4D_ERR_INJECTED: return "injected fault";
     case SPIN4D_ERR_TIMEOUT: return "device wait timed out";
+    case SPIN4D_ERR_BOUNDS: return "device bounds check failed (checked build)";
     default: return "unknown status";
   }
 }
 
 int spin4d_last_cuda_error(void) { return g_last_cuda_error; }
+
+int spin4d_checked_build(void) {
+#ifdef SPIN4D_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+// The persisting-L2 limit of the current context before the first window was
+// set (restored by spin4d_l2_window_clear), per device.
+static std::mutex g_l2_mu;
+static bool g_l2_saved[64] = {false};
+static size_t g_l2_prev[64] = {0};
+
+int spin4d_l2_window_set(spin4d_stream_t stream, const void* base, size_t bytes, size_t* applied_bytes) {
+  if (!stream || !base || bytes == 0) return SPIN4D_ERR_INVALID;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= 64) return SPIN4D_ERR_UNSUPPORTED;
+  int max_persist = 0, max_window = 0;
+  e = cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (max_persist <= 0 || max_window <= 0) return SPIN4D_ERR_UNSUPPORTED;
+  const size_t window = bytes < (size_t)max_window ? bytes : (size_t)max_window;
+  const size_t setaside = window < (size_t)max_persist ? window : (size_t)max_persist;
+  {
+    std::lock_guard<std::mutex> lock(g_l2_mu);
+    if (!g_l2_saved[dev]) {
+      e = cudaDeviceGetLimit(&g_l2_prev[dev], cudaLimitPersistingL2CacheSize);
+      if (e != cudaSuccess) return cuda_status(e);
+      g_l2_saved[dev] = true;
+    }
+  }
+  e = cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, setaside);
+  if (e != cudaSuccess) return cuda_status(e);
+  cudaStreamAttrValue attr;
+  memset(&attr, 0, sizeof(attr));
+  attr.accessPolicyWindow.base_ptr = const_cast<void*>(base);
+  attr.accessPolicyWindow.num_bytes = window;
+  attr.accessPolicyWindow.hitRatio = (float)((double)setaside / (double)window);
+  attr.accessPolicyWindow.hitProp = cudaAccessPropertyPersisting;
+  attr.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
+  e = cudaStreamSetAttribute((cudaStream_t)stream, cudaStreamAttributeAccessPolicyWindow, &attr);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (applied_bytes) *applied_bytes = window;
+  return SPIN4D_OK;
+}
+
+int spin4d_l2_window_clear(spin4d_stream_t stream) {
+  if (!stream) return SPIN4D_ERR_INVALID;
+  cudaStreamAttrValue attr;
+  memset(&attr, 0, sizeof(attr));
+  attr.accessPolicyWindow.num_bytes = 0;
+  attr.accessPolicyWindow.hitProp = cudaAccessPropertyNormal;
+  attr.accessPolicyWindow.missProp = cudaAccessPropertyNormal;
+  cudaError_t e = cudaStreamSetAttribute((cudaStream_t)stream, cudaStreamAttributeAccessPolicyWindow, &attr);
+  if (e != cudaSuccess) return cuda_status(e);
+  // lines already marked persisting return to normal
+  e = cudaCtxResetPersistingL2Cache();
+  if (e != cudaSuccess) return cuda_status(e);
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  std::lock_guard<std::mutex> lock(g_l2_mu);
+  if (dev >= 0 && dev < 64 && g_l2_saved[dev]) {
+    e = cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, g_l2_prev[dev]);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return SPIN4D_OK;
+}
 
 const char* spin4d_version(void) { return "0.1.0"; }
 

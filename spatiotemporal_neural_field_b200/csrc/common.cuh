@@ -74,6 +74,33 @@ __device__ __forceinline__ void level_cell(const float xt[4], const GridParams& 
 }
 
 // Table index of the 16 corners (bit d of c selects base_d + 1).
+// ---------------------------------------------------------------------------
+// Checked build (compiled with SPIN4D_CHECKED): device-side bounds checks on
+// every table index and HexPlane cell.  A failed check records itself in this
+// translation unit's bounds word and the access is redirected to a valid
+// address (entry 0 of the level, the plane's first row): nothing traps, and
+// spin4d_check_device_errors reports SPIN4D_ERR_BOUNDS.  Each translation
+// unit registers a reader of its word with the library at load time.
+// ---------------------------------------------------------------------------
+#ifdef SPIN4D_CHECKED
+static __device__ int g_bounds_error = 0;
+__device__ __forceinline__ bool bounds_ok(bool ok) {
+  if (!ok) atomicExch(&g_bounds_error, 1);
+  return ok;
+}
+int register_bounds_word(int (*reader)(int clear));   // api.cu
+static int read_bounds_word(int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bounds_error, sizeof(int)) != cudaSuccess) return -1;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_bounds_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+static const int g_bounds_registered = register_bounds_word(read_bounds_word);
+#endif
+
 __device__ __forceinline__ void level_indices(const uint32_t base[4], const GridParams& g, int l,
                                               uint32_t idx[16]) {
   if ((g.dense_bits >> l) & 1u) {
@@ -92,6 +119,11 @@ __device__ __forceinline__ void level_indices(const uint32_t base[4], const Grid
     for (int c = 0; c < 16; ++c)
       idx[c] = (hx[c & 1] ^ hy[(c >> 1) & 1] ^ hz[(c >> 2) & 1] ^ ht[(c >> 3) & 1]) & g.mask;
   }
+#ifdef SPIN4D_CHECKED
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    if (!bounds_ok(idx[c] <= g.mask)) idx[c] = 0;   // index < T
+#endif
 }
 
 // Quadrilinear weights prod_d (bit_d ? w_d : 1 - w_d), fp32.

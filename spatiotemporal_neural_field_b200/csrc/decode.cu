@@ -505,7 +505,10 @@ extern "C" int spin4d_decode_bwd_ext(const spin4d_grid_desc* g, const spin4d_mlp
 
 namespace spin4d {
 
-constexpr size_t kStaticScratchBytes = (size_t)16 << 20;   // 16 MiB
+// The one definition of the size is the header's, so the documented limit is
+// the enforced one.
+constexpr size_t kStaticScratchBytes = (size_t)SPIN4D_NOALLOC_SCRATCH_BYTES;   // 16 MiB
+static_assert(kStaticScratchBytes % 256 == 0, "scratch size must keep 256-byte slots aligned");
 static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 
 // Device address of g_static_scratch on the current device, looked up once
@@ -529,6 +532,8 @@ static int static_scratch_address(void** out) {
 }
 
 }  // namespace spin4d
+
+extern "C" size_t spin4d_decode_bwd_noalloc_scratch_bytes(void) { return spin4d::kStaticScratchBytes; }
 
 extern "C" int spin4d_decode_bwd_noalloc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const float* pos,
                                          int64_t N, const void* tables, const void* weights, const float* gate_cr,

@@ -312,31 +312,9 @@ int decode_fwd_tc(const spin4d_grid_desc* g, const spin4d_mlp_desc* m, const flo
 int bwd_device_error(int clear);     // decode_bwd_tc.cu
 int hex_device_error(int clear);     // hexplane.cu
 int heads_device_error(int clear);   // decode_heads.cu
-
-namespace {
-// Waits on an mbarrier that nothing ever arrives at, with the same bounded
-// wait and error path as the decoder kernels: the wait runs out, the kernel
-// records the timeout in the device error word and returns.
-__global__ void selftest_wait_timeout_kernel(uint32_t max_iters) {
-  __shared__ __align__(8) uint64_t bar;
-  const uint32_t mbar = tc::smem_u32(&bar);
-  if (threadIdx.x == 0) {
-    tc::mbar_init(mbar, 1);
-    tc::mbar_fence_init();
-  }
-  __syncthreads();
-  const bool ok = tc::mbar_wait_bounded(mbar, 0, max_iters);
-  if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicExch(&g_device_error, 1);
-}
-}  // namespace
+int bounds_status(int clear);        // api.cu (checked build: SPIN4D_ERR_BOUNDS)
 
 }  // namespace spin4d
-
-extern "C" int spin4d_selftest_wait_timeout(uint32_t max_iters, spin4d_stream_t stream) {
-  if (max_iters < 1 || max_iters > (1u << 24)) return SPIN4D_ERR_INVALID;
-  spin4d::selftest_wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(max_iters);
-  return spin4d::launch_status();
-}
 
 extern "C" int spin4d_check_device_errors(int clear) {
   int v = 0;
@@ -350,6 +328,8 @@ extern "C" int spin4d_check_device_errors(int clear) {
   const int b = spin4d::bwd_device_error(clear);
   const int h = spin4d::hex_device_error(clear);
   const int p = spin4d::heads_device_error(clear);
+  const int c = spin4d::bounds_status(clear);
+  if (c != SPIN4D_OK) return c;
   if (b != SPIN4D_OK) return b;
   if (h != SPIN4D_OK) return h;
   if (p != SPIN4D_OK) return p;

@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <string.h>
 
+#include <cmath>
+
 #include "host.h"
 #include "tc.cuh"
 
@@ -51,7 +53,29 @@ struct HexParams {
   int res_a[24], res_b[24];
   float scale_a[24], scale_b[24];
   int64_t off[24];        // float offset of each plane
+  // KineticGS energy-flow window (NULL gate_cr: no window): w from the
+  // per-Gaussian (c, r) on the normalised time, H(w) = [w >= 1/2] gates the
+  // displacement, w scales the log-scale and SH offsets; gate_grad (N x 2,
+  // may be NULL) receives d loss / d(c, r) in the backward
+  const float* gate_cr;
+  float* gate_grad;
+  float gate_tau;
 };
+
+// The window weight w and the displacement gate H(w) of Gaussian n (1, 1
+// without a window).
+__device__ __forceinline__ void hex_window(const HexParams& hp, const int32_t* __restrict__ frame, int64_t n,
+                                          float& w, float& hgate, float& t, float2& cr) {
+  w = 1.0f;
+  hgate = 1.0f;
+  t = 0.0f;
+  cr = make_float2(0.f, 0.f);
+  if (!hp.gate_cr) return;
+  t = clamp01(__fdiv_rn((float)__ldg(frame + n), hp.frames_m1));
+  cr = __ldg(reinterpret_cast<const float2*>(hp.gate_cr) + n);
+  w = temporal_gate(t, cr.x, cr.y, hp.gate_tau);
+  hgate = w >= 0.5f ? 1.0f : 0.0f;
+}
 
 struct HexOutPtrs {
   float *mu, *rot, *scale, *sh, *cov;
@@ -86,6 +110,10 @@ __device__ __forceinline__ PlaneSample plane_sample(const float xt[4], const Hex
   PlaneSample s;
   const int64_t row = (int64_t)hp.res_a[k] * kHexC;
   s.o00 = hp.off[k] + ((int64_t)ib * hp.res_a[k] + ia) * kHexC;
+#ifdef SPIN4D_CHECKED
+  // the cell's four rows inside plane k
+  if (!bounds_ok(ia >= 0 && ib >= 0 && ia + 1 < hp.res_a[k] && ib + 1 < hp.res_b[k])) s.o00 = hp.off[k];
+#endif
   s.o01 = s.o00 + kHexC;
   s.o10 = s.o00 + row;
   s.o11 = s.o10 + kHexC;
@@ -105,6 +133,9 @@ __device__ __forceinline__ int64_t plane_corner(const float xt[4], const HexPara
   int ib = min(max((int)floorf(pb), 0), hp.res_b[k] - 2);
   wa = __fsub_rn(pa, (float)ia);
   wb = __fsub_rn(pb, (float)ib);
+#ifdef SPIN4D_CHECKED
+  if (!bounds_ok(ia >= 0 && ib >= 0 && ia + 1 < hp.res_a[k] && ib + 1 < hp.res_b[k])) return hp.off[k];
+#endif
   return hp.off[k] + ((int64_t)ib * hp.res_a[k] + ia) * kHexC;
 }
 
@@ -460,7 +491,8 @@ struct HexBwdLayout {
   static constexpr int BIAS = T1 + 3 * HexTcLayout::H_PLANE;  // b1 | b2 | b3
   static constexpr int BACC = BIAS + 3 * kHexH * 4;           // db1 | db2 | db3 over the CTA's tiles
   static constexpr int MISC = BACC + 3 * kHexH * 4;           // 2 mbarriers + TMEM address
-  static constexpr int BYTES = MISC + 32;
+  static constexpr int GSUM = MISC + 32;                      // [128]: the SH half of d loss / d w (window)
+  static constexpr int BYTES = GSUM + kHexTile * 4;
 };
 static_assert(HexBwdLayout::BYTES <= 227 * 1024, "backward tiles exceed the shared memory of one CTA");
 
@@ -1010,15 +1042,21 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
       add_partial(tmem + 128 + lane + col, tmem + 192 + lane + col, y);
       tc::fence_before_sync();
       if (valid) {
+        float gw, gh, gt;
+        float2 gcr;
+        hex_window(hp, frame, n, gw, gh, gt, gcr);
         if (half == 0) {
           float qh[4], q[4], s[3], cov[6];
 #pragma unroll
-          for (int i = 0; i < 3; ++i) out.mu[3 * n + i] = __ldg(mu + 3 * n + i) + y[i];
+          for (int i = 0; i < 3; ++i) {
+            const float m0 = __ldg(mu + 3 * n + i);
+            out.mu[3 * n + i] = gh != 0.0f ? m0 + y[i] : m0;
+          }
 #pragma unroll
           for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + y[3 + i];
           normalise_quat(qh, q);
 #pragma unroll
-          for (int i = 0; i < 3; ++i) s[i] = expf(__ldg(logs_can + 3 * n + i) + y[7 + i]);
+          for (int i = 0; i < 3; ++i) s[i] = expf(__ldg(logs_can + 3 * n + i) + gw * y[7 + i]);
           covariance(s, q, cov);
           reinterpret_cast<float4*>(out.rot)[n] = make_float4(q[0], q[1], q[2], q[3]);
 #pragma unroll
@@ -1026,10 +1064,11 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
 #pragma unroll
           for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
 #pragma unroll
-          for (int i = 10; i < 32; ++i) out.sh[48 * n + (i - 10)] = __ldg(sh_can + 48 * n + (i - 10)) + y[i];
+          for (int i = 10; i < 32; ++i) out.sh[48 * n + (i - 10)] = __ldg(sh_can + 48 * n + (i - 10)) + gw * y[i];
         } else {
 #pragma unroll
-          for (int i = 0; i < kHexHead - 32; ++i) out.sh[48 * n + 22 + i] = __ldg(sh_can + 48 * n + 22 + i) + y[i];
+          for (int i = 0; i < kHexHead - 32; ++i)
+            out.sh[48 * n + 22 + i] = __ldg(sh_can + 48 * n + 22 + i) + gw * y[i];
         }
       }
     }
@@ -1164,20 +1203,32 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     for (int i = 0; i < 32; ++i) h2[i] = fmaxf(h2[i] + bias[kHexH + half * 32 + i], 0.f);
     store_row32(sm, BL::T1, row, half, h2);
     tiles_ready();
-    // head rows 0..15 (d_mu, d_q, d_logs) into stage 1's columns
+    // head rows 0..15 (d_mu, d_q, d_logs) into stage 1's columns; with the
+    // energy-flow window all 64 (d loss / d w needs the SH offsets too)
+    const bool gated = hp.gate_cr != nullptr;
     if (tid == 0) {
       tc::fence_after_sync();
-      mma6(tmem + 128, tmem + 192, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, 16, false, false));
+      mma6(tmem + 128, tmem + 192, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, gated ? kHexH : 16, false, false));
       tc::mma_commit(mbar0);
     }
     if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
     tc::fence_after_sync();
     // ---- 2. head adjoint ----
     float dy[32];
+    float gw = 1.0f, gh = 1.0f, gt = 0.0f;
+    float2 gcr = make_float2(0.f, 0.f);
+    if (valid) hex_window(hp, frame, n, gw, gh, gt, gcr);
+    float* gsum = reinterpret_cast<float*>(sm + BL::GSUM);
+    float dldw = 0.0f;   // d loss / d w: this thread's part of the w-scaled offsets
     if (half == 0) {
-      float a[16], c[16];
-      tc::tmem_ld16(tmem + 128 + lane, a);
-      tc::tmem_ld16(tmem + 192 + lane, c);
+      float a[32], c[32];
+      if (gated) {
+        tc::tmem_ld32(tmem + 128 + lane, a);
+        tc::tmem_ld32(tmem + 192 + lane, c);
+      } else {
+        tc::tmem_ld16(tmem + 128 + lane, a);
+        tc::tmem_ld16(tmem + 192 + lane, c);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) dy[i] = 0.f;
       if (valid) {
@@ -1185,9 +1236,12 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
 #pragma unroll
         for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + (a[3 + i] + c[3 + i] + bias[2 * kHexH + 3 + i]);
         const float nrm = normalise_quat(qh, q);
+        float dlogs_off[3];
 #pragma unroll
-        for (int i = 0; i < 3; ++i)
-          s[i] = expf(__ldg(logs_can + 3 * n + i) + (a[7 + i] + c[7 + i] + bias[2 * kHexH + 7 + i]));
+        for (int i = 0; i < 3; ++i) {
+          dlogs_off[i] = a[7 + i] + c[7 + i] + bias[2 * kHexH + 7 + i];
+          s[i] = expf(__ldg(logs_can + 3 * n + i) + gw * dlogs_off[i]);
+        }
 #pragma unroll
         for (int i = 0; i < 6; ++i) gc[i] = g_or0(go.cov, 6 * n + i);
 #pragma unroll
@@ -1197,22 +1251,48 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
         covariance_backward(s, q, gc, ds, dq);
         normalise_quat_backward(q, nrm, dq, dqh);
 #pragma unroll
-        for (int i = 0; i < 3; ++i) dy[i] = g_or0(go.mu, 3 * n + i);
+        for (int i = 0; i < 3; ++i) dy[i] = gh != 0.0f ? g_or0(go.mu, 3 * n + i) : 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) dy[3 + i] = dqh[i];
 #pragma unroll
-        for (int i = 0; i < 3; ++i) dy[7 + i] = ds[i] * s[i];
+        for (int i = 0; i < 3; ++i) {
+          const float dl = ds[i] * s[i];   // d loss / d(log s + w d_logs)
+          dy[7 + i] = gw * dl;
+          dldw += dl * dlogs_off[i];
+        }
 #pragma unroll
-        for (int i = 10; i < 32; ++i) dy[i] = g_or0(go.sh, 48 * n + (i - 10));
+        for (int i = 10; i < 32; ++i) {
+          const float g = g_or0(go.sh, 48 * n + (i - 10));
+          dy[i] = gw * g;
+          if (gated) dldw += g * (a[i] + c[i] + bias[2 * kHexH + i]);
+        }
       }
     } else {
+      float a[32], c[32];
+      if (gated) {
+        tc::tmem_ld32(tmem + 128 + lane + 32, a);
+        tc::tmem_ld32(tmem + 192 + lane + 32, c);
+      }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) dy[i] = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
+      for (int i = 0; i < 32; ++i) {
+        const float g = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
+        dy[i] = gw * g;
+        if (gated && i < kHexHead - 32) dldw += g * (a[i] + c[i] + bias[2 * kHexH + 32 + i]);
+      }
+      if (gated) gsum[row] = dldw;
     }
     tc::fence_before_sync();
     store_row32(sm, T0, row, half, dy);
     atomicAdd(bacc + 2 * kHexH + half * 32 + lid, warp_column_sum(dy));
     tiles_ready();
+    if (gated && half == 0 && valid && hp.gate_grad) {
+      // H(w) is piecewise constant: c and r receive gradient through w alone
+      float gcr_out[2];
+      temporal_gate_backward(gt, gcr.x, gcr.y, hp.gate_tau, dldw + gsum[row], gcr_out);
+      float2* dst = reinterpret_cast<float2*>(hp.gate_grad) + n;
+      const float2 prev = *dst;
+      *dst = make_float2(prev.x + gcr_out[0], prev.y + gcr_out[1]);
+    }
     // ---- 3. dh2 = dy W3 (masked), dW3 = dy^T h2 ----
     if (tid == 0) {
       tc::fence_after_sync();
@@ -1419,17 +1499,37 @@ extern "C" int64_t spin4d_hexplane_param_count(const spin4d_hexplane_desc* h) {
   return n + (int64_t)kHexHead * d + kHexHead;
 }
 
-extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
-                                   const float* planes, const float* weights, const float* q_can,
-                                   const float* logs_can, const float* sh_can, spin4d_hex_outputs out,
-                                   spin4d_stream_t stream) {
+namespace spin4d {
+// The window's arguments: cr N x 2 (8-byte aligned), tau > 0 and finite;
+// grad_cr (backward only) N x 2, 8-byte aligned, or NULL.
+static int hex_gate_check(const spin4d_hex_gate* gate, bool backward) {
+  if (!gate || !gate->cr || !aligned(gate->cr, 8)) return SPIN4D_ERR_INVALID;
+  if (!(gate->tau > 0.0f) || !std::isfinite(gate->tau)) return SPIN4D_ERR_INVALID;
+  if (gate->grad_cr && (!backward || !aligned(gate->grad_cr, 8))) return SPIN4D_ERR_INVALID;
+  return SPIN4D_OK;
+}
+
+static void hex_set_gate(HexParams& p, const spin4d_hex_gate* gate) {
+  if (!gate) return;
+  p.gate_cr = gate->cr;
+  p.gate_grad = gate->grad_cr;
+  p.gate_tau = gate->tau;
+}
+}  // namespace spin4d
+
+static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
+                             const float* planes, const float* weights, const float* q_can, const float* logs_can,
+                             const float* sh_can, const spin4d_hex_gate* gate, spin4d_hex_outputs out,
+                             spin4d_stream_t stream, const char* name) {
   SPIN4D_CHECK(hex_check(h, mu, frame, N, planes, weights, q_can, logs_can));
   if (N == 0) return SPIN4D_OK;
   if (!sh_can || !out.mu || !out.rot || !out.scale || !out.sh || !out.cov || !aligned(out.rot, 16))
     return SPIN4D_ERR_INVALID;
   if (out.latent && !aligned(out.latent, 32)) return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_hexplane_fwd")) return SPIN4D_ERR_INJECTED;
+  if (gate) SPIN4D_CHECK(hex_gate_check(gate, false));
+  if (fault_injected(name)) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
+  hex_set_gate(p, gate);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
   if (h->n_scales * 6 <= 24) {
     // tensor cores, bf16x3 split
@@ -1451,10 +1551,28 @@ extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* m
                                                                                logs_can, sh_can, o, out.latent);
     return launch_status();
   }
+  if (gate) return SPIN4D_ERR_UNSUPPORTED;   // the window is built into the tensor-core kernels only
   int blocks = persistent_blocks((N + 127) / 128, 4);
   hexplane_fwd_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can, logs_can,
                                                                 sh_can, o);
   return launch_status();
+}
+
+extern "C" int spin4d_hexplane_fwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
+                                   const float* planes, const float* weights, const float* q_can,
+                                   const float* logs_can, const float* sh_can, spin4d_hex_outputs out,
+                                   spin4d_stream_t stream) {
+  return hexplane_fwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, sh_can, nullptr, out, stream,
+                           "spin4d_hexplane_fwd");
+}
+
+extern "C" int spin4d_hexplane_fwd_gated(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                                         int64_t N, const float* planes, const float* weights, const float* q_can,
+                                         const float* logs_can, const float* sh_can, const spin4d_hex_gate* gate,
+                                         spin4d_hex_outputs out, spin4d_stream_t stream) {
+  if (!gate) return SPIN4D_ERR_INVALID;
+  return hexplane_fwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, sh_can, gate, out, stream,
+                           "spin4d_hexplane_fwd_gated");
 }
 
 extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N) {
@@ -1462,20 +1580,21 @@ extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, i
   return (size_t)hex_bwd_blocks(N) * slot_stride((int)spin4d_hexplane_param_count(h)) * sizeof(float);
 }
 
-extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
-                                   const float* planes, const float* weights, const float* q_can,
-                                   const float* logs_can, const float* sh_can, const float* latent,
-                                   const spin4d_hex_output_grads* grad_out, float* grad_planes,
-                                   float* grad_weights, void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
-  (void)sh_can;   // sh' = sh_can + d_sh: the upstream sh gradient flows through unchanged
+static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
+                             const float* planes, const float* weights, const float* q_can, const float* logs_can,
+                             const float* latent, const spin4d_hex_gate* gate, const spin4d_hex_output_grads* grad_out,
+                             float* grad_planes, float* grad_weights, void* workspace, size_t ws_bytes,
+                             spin4d_stream_t stream, const char* name) {
   SPIN4D_CHECK(hex_check(h, mu, frame, N, planes, weights, q_can, logs_can));
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_planes || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_planes, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256)) return SPIN4D_ERR_INVALID;
   if (latent && !aligned(latent, 32)) return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_hexplane_bwd_workspace(h, N)) return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_hexplane_bwd")) return SPIN4D_ERR_INJECTED;
+  if (gate) SPIN4D_CHECK(hex_gate_check(gate, true));
+  if (fault_injected(name)) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
+  hex_set_gate(p, gate);
   HexGradPtrs go{grad_out->mu, grad_out->rot, grad_out->scale, grad_out->sh, grad_out->cov};
   const int n_params = (int)spin4d_hexplane_param_count(h);
   cudaStream_t s = (cudaStream_t)stream;
@@ -1509,6 +1628,7 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
     }
   }
   if (blocks == 0) {
+    if (gate) return SPIN4D_ERR_UNSUPPORTED;   // the window is built into the tensor-core kernels only
     // fp32 SIMT fallback (the saved latent is not used)
     blocks = hex_bwd_blocks(N);
     const int smem = (4 * kHexH + kHexHead + kHexC) * kHexBwdBlock * (int)sizeof(float);
@@ -1521,4 +1641,26 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
   hex_reduce_slots<<<(n_params + 255) / 256, 256, 0, s>>>(static_cast<float*>(workspace), blocks, n_params,
                                                           grad_weights);
   return launch_status();
+}
+
+extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
+                                   const float* planes, const float* weights, const float* q_can,
+                                   const float* logs_can, const float* sh_can, const float* latent,
+                                   const spin4d_hex_output_grads* grad_out, float* grad_planes,
+                                   float* grad_weights, void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
+  (void)sh_can;   // sh' = sh_can + d_sh: the upstream sh gradient flows through unchanged
+  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, nullptr, grad_out, grad_planes,
+                           grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd");
+}
+
+extern "C" int spin4d_hexplane_bwd_gated(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                                         int64_t N, const float* planes, const float* weights, const float* q_can,
+                                         const float* logs_can, const float* sh_can, const float* latent,
+                                         const spin4d_hex_gate* gate, const spin4d_hex_output_grads* grad_out,
+                                         float* grad_planes, float* grad_weights, void* workspace, size_t ws_bytes,
+                                         spin4d_stream_t stream) {
+  (void)sh_can;
+  if (!gate) return SPIN4D_ERR_INVALID;
+  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, gate, grad_out, grad_planes,
+                           grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd_gated");
 }

@@ -12,10 +12,40 @@
 // reads a buffer front to back (the sequential ceiling of
 // wherever it lives) and probe_fma runs independent fp32 FMA chains (the
 // CUDA-core arithmetic peak).
-#include "host.h"
+//
+// Built into libspin4d_probe.so, a measurement and test library beside the
+// decoder's libspin4d.so; it shares only the tensor-core helper header.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "spin4d_probe.h"
+#include "tc.cuh"
 
 namespace spin4d {
 namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? SPIN4D_OK : SPIN4D_ERR_CUDA; }
+
+// This library's device error word: set when a bounded wait runs out.
+__device__ int g_probe_error = 0;
+
+// Waits on an mbarrier that nothing ever arrives at, with the bounded wait
+// of the decoder's tensor-core kernels: the wait runs out, the kernel
+// records the timeout and returns.
+__global__ void selftest_wait_timeout_kernel(uint32_t max_iters) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t mbar = tc::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(mbar, 1);
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  const bool ok = tc::mbar_wait_bounded(mbar, 0, max_iters);
+  if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicExch(&g_probe_error, 1);
+}
 
 __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   // integer finaliser of MurmurHash3 (public domain)
@@ -148,7 +178,6 @@ extern "C" int spin4d_probe_gather(const void* buf, uint64_t buf_bytes, int widt
   if (!buf || !sink || (width != 4 && width != 16 && width != 128) || buf_bytes < (uint64_t)width ||
       loads_per_thread < 8 || loads_per_thread % 8 || blocks < 1 || !aligned(buf, width == 128 ? 128 : 16))
     return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_probe_gather")) return SPIN4D_ERR_INJECTED;
   const uint64_t slots = buf_bytes / (uint64_t)width;
   const uint8_t* b = static_cast<const uint8_t*>(buf);
   cudaStream_t s = (cudaStream_t)stream;
@@ -165,7 +194,6 @@ extern "C" int spin4d_probe_stream(const void* buf, uint64_t buf_bytes, int pass
                                    spin4d_stream_t stream) {
   if (!buf || !sink || buf_bytes < 16 || buf_bytes % 16 || passes < 1 || blocks < 1 || !aligned(buf, 16))
     return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_probe_stream")) return SPIN4D_ERR_INJECTED;
   probe_stream_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint4*>(buf), buf_bytes / 16, passes,
                                                                 sink);
   return launch_status();
@@ -173,7 +201,6 @@ extern "C" int spin4d_probe_stream(const void* buf, uint64_t buf_bytes, int pass
 
 extern "C" int spin4d_probe_fma(int64_t iters, int blocks, uint32_t* sink, spin4d_stream_t stream) {
   if (!sink || iters < 1 || blocks < 1) return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_probe_fma")) return SPIN4D_ERR_INJECTED;
   probe_fma_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(iters, 1.0f, sink);
   return launch_status();
 }
@@ -183,7 +210,6 @@ extern "C" int spin4d_probe_atomic(void* buf, uint64_t buf_bytes, int width, int
   if (!buf || (width != 4 && width != 8 && width != 16) || buf_bytes < (uint64_t)width || ops_per_thread < 8 ||
       ops_per_thread % 8 || blocks < 1 || !aligned(buf, 16))
     return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_probe_atomic")) return SPIN4D_ERR_INJECTED;
   const uint64_t slots = buf_bytes / (uint64_t)width;
   float* b = static_cast<float*>(buf);
   cudaStream_t s = (cudaStream_t)stream;
@@ -201,7 +227,6 @@ extern "C" int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int row_b
   if (!buf || (row_bytes != 128 && row_bytes != 256) || buf_bytes < (uint64_t)row_bytes || rows_per_thread < 1 ||
       blocks < 1 || !aligned(buf, 128))
     return SPIN4D_ERR_INVALID;
-  if (fault_injected("spin4d_probe_bulk_reduce")) return SPIN4D_ERR_INJECTED;
   float* b = static_cast<float*>(buf);
   cudaStream_t s = (cudaStream_t)stream;
   if (row_bytes == 128)
@@ -209,4 +234,20 @@ extern "C" int spin4d_probe_bulk_reduce(void* buf, uint64_t buf_bytes, int row_b
   else
     probe_bulk_reduce_kernel<256><<<blocks, 128, 0, s>>>(b, buf_bytes / 256, rows_per_thread, seed);
   return launch_status();
+}
+
+extern "C" int spin4d_selftest_wait_timeout(uint32_t max_iters, spin4d_stream_t stream) {
+  if (max_iters < 1 || max_iters > (1u << 24)) return SPIN4D_ERR_INVALID;
+  selftest_wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(max_iters);
+  return launch_status();
+}
+
+extern "C" int spin4d_probe_check_device_errors(int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_probe_error, sizeof(int)) != cudaSuccess) return SPIN4D_ERR_CUDA;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_probe_error, &zero, sizeof(int)) != cudaSuccess) return SPIN4D_ERR_CUDA;
+  }
+  return v ? SPIN4D_ERR_TIMEOUT : SPIN4D_OK;
 }

@@ -12,13 +12,16 @@ from typing import Dict, Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspin4d.so")
+# SPIN4D_CHECKED=1 selects the build with device-side bounds checks
+_LIB_NAME = "libspin4d_checked.so" if os.environ.get("SPIN4D_CHECKED") == "1" else "libspin4d.so"
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIB_NAME)
 if not os.path.exists(_LIB_PATH):
-    raise ImportError("libspin4d.so is not built (run `python -m spatiotemporal_neural_field_b200.build` "
-                      "or __graft_entry__.build()); spin4d has no CPU fallback")
+    raise ImportError("%s is not built (run `python -m spatiotemporal_neural_field_b200.build` "
+                      "or __graft_entry__.build()); spin4d has no CPU fallback" % _LIB_NAME)
 lib = ctypes.CDLL(_LIB_PATH)
 
-OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_INJECTED, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_INJECTED, ERR_TIMEOUT, ERR_BOUNDS = (
+    0, -1, -2, -3, -4, -5, -6, -7)
 F32, F16 = 0, 1
 INPUT_NORMALISED = 1
 MAX_LEVELS = 16
@@ -68,6 +71,10 @@ class HexOutputGrads(ctypes.Structure):
     _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp)]
 
 
+class HexGate(ctypes.Structure):
+    _fields_ = [("cr", c_vp), ("tau", c_f32), ("grad_cr", c_vp)]
+
+
 class HeadsDesc(ctypes.Structure):
     _fields_ = [("in_dim", c_i32), ("hidden", c_i32), ("sh_dim", c_i32), ("w_dtype", c_i32)]
 
@@ -106,6 +113,7 @@ _SIGS = {
                                   c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_decode_bwd_ext": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(OutputGrads),
                                       c_vp, c_vp, P(ExtraGrads), c_vp, c_sz, c_vp]),
+    "spin4d_decode_bwd_noalloc_scratch_bytes": (c_sz, []),
     "spin4d_decode_bwd_noalloc": (c_i32, [P(GridDesc), P(MlpDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
                                           P(OutputGrads), c_vp, c_vp, c_vp]),
     "spin4d_cov_assemble": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
@@ -124,25 +132,26 @@ _SIGS = {
     "spin4d_hexplane_plane_count": (c_i64, [P(HexDesc)]),
     "spin4d_hexplane_param_count": (c_i64, [P(HexDesc)]),
     "spin4d_hexplane_fwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, HexOutputs, c_vp]),
+    "spin4d_hexplane_fwd_gated": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, P(HexGate),
+                                          HexOutputs, c_vp]),
+    "spin4d_hexplane_bwd_gated": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                          P(HexGate), P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_hexplane_bwd_workspace": (c_sz, [P(HexDesc), c_i64]),
     "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                     P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_debug_corners": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp]),
     "spin4d_check_device_errors": (c_i32, [c_i32]),
-    "spin4d_selftest_wait_timeout": (c_i32, [c_u32, c_vp]),
-    "spin4d_probe_gather": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp, c_vp]),
-    "spin4d_probe_stream": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i32, c_vp, c_vp]),
     "spin4d_morton_order_workspace": (c_sz, [c_i64]),
     "spin4d_morton_order": (c_i32, [P(GridDesc), c_vp, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_permute_rows": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp]),
-    "spin4d_probe_atomic": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
-    "spin4d_probe_bulk_reduce": (c_i32, [c_vp, ctypes.c_uint64, c_i32, c_i64, c_i32, c_u32, c_vp]),
-    "spin4d_probe_fma": (c_i32, [c_i64, c_i32, c_vp, c_vp]),
     "spin4d_render_state_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i64]),
     "spin4d_render_fwd": (c_i32, [P(Camera), P(RenderDesc), c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
                                   c_i64, c_vp]),
     "spin4d_render_bwd": (c_i32, [P(Camera), P(RenderDesc), c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_i64,
                                   c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "spin4d_checked_build": (c_i32, []),
+    "spin4d_l2_window_set": (c_i32, [c_vp, c_vp, c_sz, P(c_sz)]),
+    "spin4d_l2_window_clear": (c_i32, [c_vp]),
     "spin4d_status_string": (ctypes.c_char_p, [c_i32]),
     "spin4d_last_cuda_error": (c_i32, []),
     "spin4d_version": (ctypes.c_char_p, []),
@@ -293,7 +302,8 @@ def decode_bwd(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, t
                                                                   workspace.numel(), _stream(stream)))
 
 
-NOALLOC_SCRATCH_BYTES = 16 << 20
+# the size of the library's built-in scratch, as the library was compiled
+NOALLOC_SCRATCH_BYTES = int(lib.spin4d_decode_bwd_noalloc_scratch_bytes())
 
 
 def decode_bwd_noalloc(g: GridDesc, m: MlpDesc, pos, tables, weights, grads: Dict[str, torch.Tensor],
@@ -408,15 +418,22 @@ def hexplane_param_count(h: HexDesc) -> int:
 HEX_KEYS = (("mu", 3), ("rot", 4), ("scale", 3), ("sh", 48), ("cov", 6))
 
 
-def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=None, stream=None):
+def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=None, stream=None,
+                 gate_cr: Optional[torch.Tensor] = None, tau: float = 0.02):
+    """With ``gate_cr`` (N x 2 window centre and half-width) the energy-flow
+    window gates the deformation (spin4d_hexplane_fwd_gated)."""
     N = inp["mu"].shape[0]
     if out is None:
         out = {k: torch.empty((N, w), dtype=torch.float32, device=planes.device) for k, w in HEX_KEYS}
     o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS), _ptr(out.get("latent")))
-    _check("spin4d_hexplane_fwd", lib.spin4d_hexplane_fwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
-                                                          _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
-                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), o,
-                                                          _stream(stream)))
+    common = (ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N, _ptr(planes), _ptr(weights),
+              _ptr(inp["q_can"]), _ptr(inp["logs_can"]), _ptr(inp["sh_can"]))
+    if gate_cr is None:
+        _check("spin4d_hexplane_fwd", lib.spin4d_hexplane_fwd(*common, o, _stream(stream)))
+    else:
+        gate = HexGate(_ptr(gate_cr), tau, None)
+        _check("spin4d_hexplane_fwd_gated", lib.spin4d_hexplane_fwd_gated(*common, ctypes.byref(gate), o,
+                                                                          _stream(stream)))
     return out
 
 
@@ -425,16 +442,23 @@ def hexplane_bwd_workspace(h: HexDesc, N: int) -> int:
 
 
 def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, latent=None,
-                 stream=None):
+                 stream=None, gate_cr: Optional[torch.Tensor] = None, tau: float = 0.02,
+                 grad_cr: Optional[torch.Tensor] = None):
+    """With ``gate_cr`` the backward of the windowed deformation
+    (spin4d_hexplane_bwd_gated); ``grad_cr`` (N x 2) += d loss / d(c, r)."""
     N = inp["mu"].shape[0]
     if workspace is None:
         workspace = torch.empty(max(hexplane_bwd_workspace(h, N), 1), dtype=torch.uint8, device=planes.device)
     go = HexOutputGrads(*(_ptr(grads.get(k)) for k, _ in HEX_KEYS))
-    _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N,
-                                                          _ptr(planes), _ptr(weights), _ptr(inp["q_can"]),
-                                                          _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), _ptr(latent),
-                                                          ctypes.byref(go), _ptr(grad_planes), _ptr(grad_weights),
-                                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+    common = (ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N, _ptr(planes), _ptr(weights),
+              _ptr(inp["q_can"]), _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), _ptr(latent))
+    tail = (ctypes.byref(go), _ptr(grad_planes), _ptr(grad_weights), _ptr(workspace), workspace.numel(),
+            _stream(stream))
+    if gate_cr is None:
+        _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(*common, *tail))
+    else:
+        gate = HexGate(_ptr(gate_cr), tau, _ptr(grad_cr))
+        _check("spin4d_hexplane_bwd_gated", lib.spin4d_hexplane_bwd_gated(*common, ctypes.byref(gate), *tail))
 
 
 def debug_corners(g: GridDesc, pos: torch.Tensor, stream=None):
@@ -449,23 +473,6 @@ def debug_corners(g: GridDesc, pos: torch.Tensor, stream=None):
 def check_device_errors(clear: bool = True) -> None:
     """Synchronous: raises if a kernel's bounded device wait ran out."""
     _check("spin4d_check_device_errors", lib.spin4d_check_device_errors(1 if clear else 0))
-
-
-def selftest_wait_timeout(max_iters: int = 4096, stream=None) -> None:
-    """Launches a kernel whose bounded wait must run out (failure-detection test)."""
-    _check("spin4d_selftest_wait_timeout", lib.spin4d_selftest_wait_timeout(max_iters, _stream(stream)))
-
-
-def probe_gather(buf: torch.Tensor, width: int, loads_per_thread: int, blocks: int, seed: int = 1,
-                 sink: Optional[torch.Tensor] = None, stream=None) -> int:
-    """Launches the random-gather probe; returns the number of `width`-byte
-    units read (sectors for width 4/16, 128-byte lines for width 128)."""
-    if sink is None:
-        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
-    _check("spin4d_probe_gather", lib.spin4d_probe_gather(_ptr(buf), buf.numel() * buf.element_size(), width,
-                                                          loads_per_thread, blocks, seed, _ptr(sink),
-                                                          _stream(stream)))
-    return blocks * 256 * loads_per_thread // (8 if width == 128 else 1)
 
 
 def morton_order(g: GridDesc, pos: torch.Tensor, workspace: Optional[torch.Tensor] = None, stream=None):
@@ -492,39 +499,18 @@ def permute_rows(src: torch.Tensor, perm: torch.Tensor, out: Optional[torch.Tens
     return out
 
 
-def probe_atomic(buf: torch.Tensor, width: int, ops_per_thread: int, blocks: int, seed: int = 1, stream=None) -> int:
-    """Random fp32 reductions of `width` bytes into `buf`; returns the count."""
-    _check("spin4d_probe_atomic", lib.spin4d_probe_atomic(_ptr(buf), buf.numel() * buf.element_size(), width,
-                                                          ops_per_thread, blocks, seed, _stream(stream)))
-    return blocks * 256 * ops_per_thread
+def l2_window_set(stream, buf: torch.Tensor, nbytes: Optional[int] = None) -> int:
+    """Keeps ``buf`` (or its first ``nbytes``) persisting in L2 for the
+    kernels launched on ``stream`` (a torch.cuda.Stream, not the default
+    stream); returns the window's size in bytes."""
+    applied = c_sz(0)
+    n = buf.numel() * buf.element_size() if nbytes is None else nbytes
+    _check("spin4d_l2_window_set", lib.spin4d_l2_window_set(_stream(stream), _ptr(buf), n, ctypes.byref(applied)))
+    return int(applied.value)
 
 
-def probe_bulk_reduce(buf: torch.Tensor, rows_per_thread: int, blocks: int, seed: int = 1, row_bytes: int = 128,
-                      stream=None) -> int:
-    """Random bulk fp32 row reductions into `buf`; returns the rows added."""
-    _check("spin4d_probe_bulk_reduce", lib.spin4d_probe_bulk_reduce(_ptr(buf), buf.numel() * buf.element_size(),
-                                                                    row_bytes, rows_per_thread, blocks, seed,
-                                                                    _stream(stream)))
-    return blocks * 128 * rows_per_thread
-
-
-def probe_stream(buf: torch.Tensor, passes: int, blocks: int, sink: Optional[torch.Tensor] = None,
-                 stream=None) -> int:
-    """Sequential-read probe; returns the bytes read."""
-    if sink is None:
-        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
-    nbytes = buf.numel() * buf.element_size()
-    _check("spin4d_probe_stream", lib.spin4d_probe_stream(_ptr(buf), nbytes, passes, blocks, _ptr(sink),
-                                                          _stream(stream)))
-    return passes * nbytes
-
-
-def probe_fma(iters: int, blocks: int, device, sink: Optional[torch.Tensor] = None, stream=None) -> int:
-    """fp32 FMA-chain probe; returns the FLOPs executed."""
-    if sink is None:
-        sink = torch.zeros(1, dtype=torch.int32, device=device)
-    _check("spin4d_probe_fma", lib.spin4d_probe_fma(iters, blocks, _ptr(sink), _stream(stream)))
-    return 16 * iters * blocks * 256
+def l2_window_clear(stream) -> None:
+    _check("spin4d_l2_window_clear", lib.spin4d_l2_window_clear(_stream(stream)))
 
 
 def version() -> str:

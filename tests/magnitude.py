@@ -222,8 +222,28 @@ def decoder_rss(pos, tables, weights, grid, mlp, grads, gate_cr=None, normalised
     return tuple(out)
 
 
+def table_mag_level(mdz, xt, res, log2_T, l, F):
+    """Level l of ``table_mag``, T x F."""
+    T = 1 << log2_T
+    _, frac, idx = hg.corner_select(xt, res, log2_T)
+    w2 = hg.corner_weights(frac) ** 2
+    out = np.zeros((T, F))
+    for f in range(F):
+        g2 = mdz[:, l * F + f] ** 2
+        out[:, f] = np.sqrt(np.bincount(idx[:, l, :].astype(np.int64).reshape(-1),
+                                        weights=(w2[:, l, :] * g2[:, None]).reshape(-1), minlength=T))
+    return out
+
+
 def heads_rss(pos, tables, weights, grid, spec, grads):
     """The paper's four GELU heads."""
+    xt, res, mdz, mw = heads_latent_mag(pos, tables, weights, grid, spec, grads)
+    return table_mag(mdz, xt, res, grid.log2_T, grid.L, grid.F), mw
+
+
+def heads_latent_mag(pos, tables, weights, grid, spec, grads):
+    """(xt, res, m(dz) N x LF, packed weight magnitudes) of the paper's four
+    GELU heads: the four heads' dz add up before the scatter."""
     res, xt = dec._prepare(pos, grid, False)
     z = hg.encode(xt, tables, res, grid.log2_T)
     mz = encode_mag(xt, tables, res, grid.log2_T)
@@ -245,8 +265,7 @@ def heads_rss(pos, tables, weights, grid, spec, grads):
         mdz, mdeltas = mlp_backward_mag(mdy[name], heads[h], fw[h][2], hd.gelu_grad)
         mdz2 += mdz * mdz
         wr.append(weight_mag(macts, mdeltas))
-    # the four heads' dz add up before the scatter
-    return table_mag(np.sqrt(mdz2), xt, res, grid.log2_T, grid.L, grid.F), np.concatenate(wr)
+    return xt, res, np.sqrt(mdz2), np.concatenate(wr)
 
 
 def heads_output_mag(pos, tables, weights, grid, spec):

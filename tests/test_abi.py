@@ -13,6 +13,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "spin4d.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "spin4d_probe.h")
 
 
 @pytest.fixture(scope="module")
@@ -23,8 +24,8 @@ def sp():
     return spin4d
 
 
-def declared_functions():
-    src = open(HEADER).read()
+def declared_functions(header=HEADER):
+    src = open(header).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(spin4d_[a-z0-9_]+)\s*\(", src)))
 
@@ -38,6 +39,18 @@ def test_every_declared_symbol_is_exported(sp):
     exported = set(re.findall(r" T (spin4d_\w+)", out))
     assert set(names) <= exported, set(names) - exported
     assert set(sp.EXPORTED) == set(names)
+    assert not any("probe" in n or "selftest" in n for n in exported), "measurement tools in the decoder library"
+
+
+def test_probe_library_exports_its_header(sp):
+    """The measurement probes and the self-test live in their own library."""
+    from spatiotemporal_neural_field_b200 import probe as pr
+    names = declared_functions(PROBE_HEADER)
+    assert len(names) == 7
+    out = subprocess.run(["nm", "-D", "--defined-only", pr._LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (spin4d_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(pr.EXPORTED) == set(names)
 
 
 def test_grid_init_matches_oracle_resolutions(sp):
@@ -251,3 +264,13 @@ def test_render_arguments_rejected_on_host(sp):
     assert fwd(image=None) == sp.ERR_INVALID
     assert lib.spin4d_render_bwd(ref(cam), ref(desc), 100, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, 4096,
                                  None, None, None, None, None) == sp.ERR_INVALID   # no upstream gradient
+
+
+def test_l2_window_arguments_rejected_on_host(sp):
+    """The opt-in L2 window refuses the legacy stream, a NULL base and an
+    empty range before touching the device."""
+    applied = ctypes.c_size_t(0)
+    assert sp.lib.spin4d_l2_window_set(None, 1 << 20, 1 << 20, ctypes.byref(applied)) == sp.ERR_INVALID
+    assert sp.lib.spin4d_l2_window_set(1, None, 1 << 20, ctypes.byref(applied)) == sp.ERR_INVALID
+    assert sp.lib.spin4d_l2_window_set(1, 1 << 20, 0, ctypes.byref(applied)) == sp.ERR_INVALID
+    assert sp.lib.spin4d_l2_window_clear(None) == sp.ERR_INVALID

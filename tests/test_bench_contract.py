@@ -34,10 +34,12 @@ def test_reference_arm_line():
     assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 1
     assert d["value"] > 0 and d["higher_is_better"] is True and d["vs_baseline"] is None
     assert "workload" in d["config"]
-    # value is the sample's positions per second of the timed steps (10k positions a step)
-    assert abs(d["ms_per_step"] - 1e3 * 10_000 / d["value"]) <= 1e-6 * d["ms_per_step"]
+    # value is the sample's positions per second of the timed steps: every
+    # core's process decodes 10000 positions a step
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert cb["kind"] == "oracle" and cb["cores"] == os.cpu_count() and cb["sample"] and cb["value"] == d["value"]
+    assert abs(d["ms_per_step"] - 1e3 * 10_000 * cb["cores"] / d["value"]) <= 1e-6 * d["ms_per_step"]
+    assert cb["cpu_model"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

@@ -19,13 +19,17 @@ def sp():
 
 
 def test_bounded_wait_times_out_and_is_reported(sp):
-    sp.check_device_errors(clear=True)                  # start clean
-    sp.selftest_wait_timeout(max_iters=4096)
+    """The self-test kernel (libspin4d_probe.so) waits, through the decoder
+    kernels' bounded mbarrier wait, on a barrier nothing arrives at."""
+    from spatiotemporal_neural_field_b200 import probe as pr
+    pr.check_device_errors(clear=True)                  # start clean
+    pr.selftest_wait_timeout(max_iters=4096)
     torch.cuda.synchronize()
     with pytest.raises(sp.Spin4dError) as e:
-        sp.check_device_errors(clear=True)
+        pr.check_device_errors(clear=True)
     assert e.value.status == sp.ERR_TIMEOUT
-    sp.check_device_errors(clear=False)                 # cleared: no error any more
+    pr.check_device_errors(clear=False)                 # cleared: no error any more
+    sp.check_device_errors(clear=False)                 # the decoder library's word is untouched
     # the context is still usable: a real decode runs and is correct
     x = torch.arange(16, dtype=torch.float32, device="cuda").reshape(4, 4)
     assert float(x.sum()) == 120.0

@@ -1,9 +1,12 @@
 """GPU parity of the paper's four-head GELU decoder and the grouped Adam
 against the oracle (B200 only)."""
+import dataclasses
+
 import numpy as np
 import pytest
 
 from oracle import decoder as dec
+from oracle import hashgrid
 from oracle import heads as hd
 from spatiotemporal_neural_field_b200 import synthetic as S
 from tests import magnitude as mag
@@ -226,3 +229,56 @@ def test_heads_full_launch_sampled_and_by_halves(sp):
     torch.cuda.synchronize()
     tol.normwise(host(gt2), host(gt), 1e-4, "grad_tables by halves", tol.table_levels(grid.L, 1 << grid.log2_T, grid.F))
     tol.normwise(host(gw2), host(gw), 1e-4, "grad_weights by halves")
+
+
+def test_heads_table_size_2_23(sp):
+    """SPIN-4DGS section 4, Table 5: T = 2^23 entries per level, the paper's
+    best setting (16 x 2^23 x 4 fp16 = 1 GiB of tables, 2 GiB of fp32
+    gradients).  Forward on sampled rows of a 200k-position launch; the
+    backward of a 3001-position launch, tensor-core and SIMT forms, level by
+    level against the oracle's per-level scatter (its whole fp64 gradient
+    would be 4 GiB)."""
+    grid = dataclasses.replace(S.GRID_PAPER, log2_T=23)
+    spec = S.HEADS_PAPER
+    g, h = sp.grid_from_spec(grid), sp.heads_from_spec(spec)
+    tables = S.hash_tables(grid, seed=21, scale=1.0)
+    weights = S.heads_weights(spec, seed=22, bias_scale=0.3)
+    T, W = dev(tables), dev(weights)
+    n = 200_000
+    pos = S.sports_scene(300_000).frames(range(4))[:n]
+    out = sp.heads_fwd(g, h, dev(pos), T, W, latent=True)
+    idx = np.sort(np.random.default_rng(23).choice(n, 500, replace=False))
+    want = hd.decode_forward(pos[idx], tables, weights, grid, spec)
+    for k in ("scale", "rot", "sh", "opacity", "cov"):
+        tol.absolute(host(out[k])[idx], want[k], tol.FP16_ATOL, k + " (T = 2^23, sampled)")
+    res, xt = dec._prepare(pos[idx], grid, False)
+    tol.elementwise(host(out["latent"])[idx], want["z"], tol.FP32_RTOL, "latent (T = 2^23)",
+                    tol.column_groups(grid.L * grid.F), rho=mag.encode_mag(xt, tables, res, grid.log2_T))
+    del out
+    nb = 3001
+    pb = pos[:nb]
+    widths = dict(S.HEADS_OUT_WIDTHS, sh=spec.sh_dim)
+    grads = S.upstream_grads(nb, widths, 1e-2, seed=24)
+    P, G = dev(pb), {k: dev(v) for k, v in grads.items()}
+    saved = sp.heads_fwd(g, h, P, T, W, latent=True, raw=True)
+    res, xt, dz, ww = hd.latent_backward(pb, tables, weights, grid, spec, grads)
+    mxt, mres, mdz, mw = mag.heads_latent_mag(pb, tables, weights, grid, spec, grads)
+    for form in ("tensor-core", "SIMT"):
+        gt = torch.zeros((grid.L, 1 << grid.log2_T, grid.F), device="cuda")
+        gw = torch.zeros(spec.n_params(), device="cuda")
+        if form == "tensor-core":
+            sp.heads_bwd(g, h, P, T, W, G, gt, gw, latent=saved["latent"], raw=saved["raw"])
+        else:
+            sp.heads_bwd(g, h, P, T, W, G, gt, gw)
+        blocks, o = [], 0
+        for head in range(4):
+            hb = tol.weight_blocks(spec.layer_shapes(head), "head %d " % head, o)
+            blocks += hb
+            o = hb[-1][1].stop
+        tol.elementwise(host(gw), ww, tol.FP16_GRAD_RTOL, form + " grad_weights (T = 2^23)", blocks, rho=mw)
+        for l in range(grid.L):
+            wl = hashgrid.scatter_table_grad_level(dz, xt, res, grid.log2_T, l, grid.F)
+            tol.elementwise(host(gt[l]), wl, tol.FP16_GRAD_RTOL, "%s grad_tables (T = 2^23) level %d" % (form, l),
+                            rho=mag.table_mag_level(mdz, mxt, mres, grid.log2_T, l, grid.F))
+        del gt, gw
+        torch.cuda.empty_cache()

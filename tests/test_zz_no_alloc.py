@@ -61,12 +61,14 @@ def test_noalloc_backward_matches_workspace_backward_twice(sp, name, n):
 
 def test_noalloc_rejects_scratch_beyond_its_size(sp):
     """A shape whose weight-gradient scratch exceeds the built-in array is
-    refused before any launch."""
+    refused before any launch.  Every data pointer is NULL: should the size
+    check ever let the call through, the backward's own argument checks
+    refuse it before launching anything."""
     g = sp.grid_desc(8, 8, 12, "f32", 4, 32, 4, 32, 0.0, 1.0)          # latent width 64
     m = sp.mlp_desc(64, 128, 4, "f32")                                 # ~58k weights
     need = sp.decode_bwd_workspace(g, m, 1_000_000)
+    assert sp.NOALLOC_SCRATCH_BYTES == sp.lib.spin4d_decode_bwd_noalloc_scratch_bytes()
     assert need > sp.NOALLOC_SCRATCH_BYTES
-    fake = 1 << 20
-    st = sp.lib.spin4d_decode_bwd_noalloc(ctypes.byref(g), ctypes.byref(m), fake, 1_000_000, fake, fake, None, None,
-                                          ctypes.byref(sp.OutputGrads()), fake, fake, None)
+    st = sp.lib.spin4d_decode_bwd_noalloc(ctypes.byref(g), ctypes.byref(m), None, 1_000_000, None, None, None, None,
+                                          ctypes.byref(sp.OutputGrads()), None, None, None)
     assert st == sp.ERR_INVALID

@@ -62,7 +62,7 @@ def parse():
     p.add_argument("--ncu-case", default=None,
                    help="profiling driver: run a few untimed launches of one workload and exit "
                         "(sports_frame_fp16, stress_fp16_gate, sports_train_fp16, hexplane_fp32, tiny_fp32, "
-                        "render_sports_frame, paper_heads_fp16)")
+                        "render_sports_frame, paper_heads_fp16, hexplane_fwd_fp32)")
     return p.parse_args()
 
 
@@ -1054,6 +1054,21 @@ def run_ncu_case(name):
         for _ in range(3):
             sp.render_fwd(cam, desc, *args, image=img, state=st)
             sp.render_bwd(cam, desc, *args, G, st)
+        torch.cuda.synchronize()
+        sp.check_device_errors()
+        print("ncu case done:", name)
+        return
+    if name == "hexplane_fwd_fp32":
+        # the forward alone (no saved latent), as the timed forward line runs it
+        w = S.WORKLOADS["hexplane_fp32"]
+        hx, n = w["hex"], w["N"]
+        inp = {k: torch.from_numpy(v).to(dev) for k, v in S.hexplane_inputs(n).items()}
+        planes = torch.from_numpy(S.hexplane_planes(hx)).to(dev)
+        weights = torch.from_numpy(S.hexplane_weights(hx)).to(dev)
+        h = sp.hex_from_spec(hx)
+        out = {k: torch.empty((n, wd), device=dev) for k, wd in sp.HEX_KEYS}
+        for _ in range(3):
+            sp.hexplane_fwd(h, inp, planes, weights, out=out)
         torch.cuda.synchronize()
         sp.check_device_errors()
         print("ncu case done:", name)

@@ -18,6 +18,7 @@
 #include <string.h>
 
 #include <cmath>
+#include <stdlib.h>
 
 #include "host.h"
 #include "tc.cuh"
@@ -654,6 +655,29 @@ __device__ __forceinline__ void st_v4_stream(float* p, float4 v, uint64_t pol) {
                "f"(v.w), "l"(pol)
                : "memory");
 }
+// The planes are the one data set worth keeping in L2 across a launch: their
+// rows are read with an evict-last policy, and the per-Gaussian inputs and
+// outputs (hundreds of MB that each pass exactly once) with evict-first.
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ float4 ld_nc_v4_hint(const float4* p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ float ld_nc_hint(const float* p, uint64_t pol) {
+  float v;
+  asm volatile("ld.global.nc.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_hint(float* p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
 
 // Global data of one plane sample for one thread: its chunk of the W1 slice
 // (row tid/4, 8 columns) and, for its Gaussian, either the 16 channels
@@ -1089,6 +1113,436 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
 }
 
 
+// ---------------------------------------------------------------------------
+// Forward, warp-specialised.  The same arithmetic as hexplane_fwd_tc_kernel
+// (the same split products, the same fp32 accumulation order), with the
+// per-sample chain taken apart so that no step waits for the whole CTA:
+//   * 8 producer warps gather the tile's corner rows into registers two plane
+//     samples ahead, interpolate, and write the split z_k into a two-stage
+//     shared-memory ring;
+//   * 4 consumer warps (one thread per Gaussian, TMEM lane = row): one lane
+//     issues each sample's split MMAs into a three-stage TMEM ring and
+//     commits them to the stage's "empty" and "ready" barriers; all 128 add
+//     the sample's two accumulators to their fp32 row, free the TMEM stage,
+//     and write the split W1 slice of the sample two ahead into the ring
+//     stage that sample's MMAs just released; after the last sample they run
+//     layers 2 and 3 (through the H tile and TMEM columns 384..511) and
+//     write the outputs, while the producers already gather the next tile.
+//   A ring stage is full once all 8 producer warps and all 4 consumer warps
+//   have arrived.
+// Every hand-off is an mbarrier with a bounded wait; the roles' own named
+// barriers reduce a failure flag, so a timed-out wait ends both roles at their
+// next barrier instead of leaving either waiting.
+// ---------------------------------------------------------------------------
+constexpr int kWsProducerWarps = 8;
+constexpr int kWsProducers = 32 * kWsProducerWarps;
+constexpr int kWsConsumers = kHexTile;
+constexpr int kWsThreads = kWsProducers + kWsConsumers;
+constexpr int kWsTStages = 3;
+// Polls of one mbarrier before a wait gives up: every legitimate wait here is
+// for work of microseconds (a sample's gather, its MMAs, a tile's epilogue)
+constexpr uint32_t kWsWait = 1u << 20;
+static_assert(2 * 4 * 32 * 176 + 4 * 32 * 152 == kWsThreads * 168, "the register split must equal the launch's total");
+
+// A producer's corner rows of one plane sample: [Gaussian j][corner 00, 01, 10, 11]
+struct CornerRegs {
+  float4 c[4][4];
+};
+
+struct HexWsLayout {
+  static constexpr int Z_STAGE = HexTcLayout::Z_STAGE;             // split z_k, skewed (24,960 B)
+  static constexpr int W_STAGE = HexTcLayout::W_STAGE;             // split W1 slice (12,288 B)
+  static constexpr int STAGE = Z_STAGE + W_STAGE;                  // one ring stage
+  static constexpr int H = 2 * STAGE;                              // split H tile, 3 x 16 KB
+  static constexpr int W2 = H + 3 * HexTcLayout::H_PLANE;          // split W2, 3 x 8 KB
+  static constexpr int W3 = W2 + 3 * HexTcLayout::S_PLANE;         // split W3 (58 rows, padded), 3 x 8 KB
+  static constexpr int BIAS = W3 + 3 * HexTcLayout::S_PLANE;       // b1 | b2 | b3
+  static constexpr int BARS = BIAS + 3 * kHexH * 4;                // 12 mbarriers, then the TMEM address
+  static constexpr int SMP = BARS + 128;                           // per sample and Gaussian {row, wa, wb, 0}
+  static constexpr int BYTES = SMP + 24 * kHexTile * 16;
+  static __device__ __forceinline__ int z(int s) { return s * STAGE; }
+  static __device__ __forceinline__ int w(int s) { return s * STAGE + Z_STAGE; }
+};
+static_assert(HexWsLayout::STAGE % 128 == 0 && HexWsLayout::W2 % 128 == 0 && HexWsLayout::SMP % 16 == 0,
+              "tile alignment");
+static_assert(HexWsLayout::W2 - HexWsLayout::H == 3 * HexTcLayout::H_PLANE, "H tile size");
+static_assert(HexWsLayout::BYTES <= 227 * 1024, "warp-specialised tiles exceed the shared memory of one CTA");
+
+// mbarriers of the warp-specialised forward
+enum : int { kBarFull = 0, kBarEmpty = 2, kBarReady = 4, kBarFree = 7, kBarLayer = 10, kBarFinal = 11, kNumWsBars = 12 };
+static_assert(8 * kNumWsBars + 4 <= 128, "the mbarriers and the TMEM address fit their 128 bytes");
+
+// bar.sync on a named barrier for `n` threads of one role
+__device__ __forceinline__ void role_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// The same with an OR over the role's predicates: true if any thread's p was.
+__device__ __forceinline__ bool role_sync_or(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Bounded wait by every lane of a warp, agreed across the warp.
+__device__ __forceinline__ bool warp_wait(uint32_t mbar, uint32_t parity) {
+  const bool ok = tc::mbar_wait_bounded(mbar, parity, kWsWait);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// acc[i] += main[i] + corr[i] for this thread's TMEM lane, 64 columns (four
+// rounds with a main and a correction load in flight per wait).
+__device__ __forceinline__ void add_partial64(uint32_t d_main, uint32_t d_corr, float acc[64]) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    float a[16], b[16];
+    tc::tmem_ld16x2(d_main + 16 * h, d_corr + 16 * h, a, b);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[16 * h + i] += a[i] + b[i];
+  }
+}
+
+// The consumers' share of a ring stage: the W1 slice of plane sample k
+// (64 rows x 32 columns), row c / 2, columns 16 (c % 2) .. + 15, loaded into
+// registers a sample ahead and stored split.
+__device__ __forceinline__ void load_w1_slice(const float* __restrict__ W1, int IN, int k, int c, float v[16]) {
+  const float* src = W1 + (size_t)(c >> 1) * IN + k * kHexC + (c & 1) * 16;
+  ld_nc_v8(src, v);
+  ld_nc_v8(src + 8, v + 8);
+}
+__device__ __forceinline__ void store_w1_slice(uint8_t* sm, int off, int c, const float v[16]) {
+  store_split8(sm, off, HexTcLayout::W_PLANE, c >> 1, (c & 1) * 2, kHexC, v);
+  store_split8(sm, off, HexTcLayout::W_PLANE, c >> 1, (c & 1) * 2 + 1, kHexC, v + 8);
+}
+
+__global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
+    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
+    const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
+    const float* __restrict__ logs_can, const float* __restrict__ sh_can, HexOutPtrs out, float* __restrict__ latent) {
+  using Lay = HexWsLayout;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  const float* W1 = W;
+  const float* b1 = W1 + kHexH * IN;
+  const float* W2g = b1 + kHexH;
+  const float* b2 = W2g + kHexH * kHexH;
+  const float* W3g = b2 + kHexH;
+  const float* b3 = W3g + kHexHead * kHexH;
+  const uint32_t sbase = tc::smem_u32(sm);
+  const uint32_t bar0 = sbase + Lay::BARS;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::BARS + 8 * kNumWsBars);
+  float4* smp = reinterpret_cast<float4*>(sm + Lay::SMP);
+  const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
+
+  if (tid < kHexThreads) {
+    // W2 | W3 split at the forward's offsets, relocated to this layout
+    for (int i = tid; i < kHexH * (kHexH / 8); i += kHexThreads) {
+      const int r = i / (kHexH / 8), kc = i % (kHexH / 8);
+      const float4* w2 = reinterpret_cast<const float4*>(W2g + r * kHexH) + 2 * kc;
+      store_split8(sm, Lay::W2, HexTcLayout::S_PLANE, r, kc, kHexH, __ldg(w2), __ldg(w2 + 1));
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+      if (r < kHexHead) {
+        const float4* w3 = reinterpret_cast<const float4*>(W3g + r * kHexH) + 2 * kc;
+        a = __ldg(w3);
+        b = __ldg(w3 + 1);
+      }
+      store_split8(sm, Lay::W3, HexTcLayout::S_PLANE, r, kc, kHexH, a, b);
+    }
+    float* bw = reinterpret_cast<float*>(sm + Lay::BIAS);
+    for (int o = tid; o < kHexH; o += kHexThreads) {
+      bw[o] = __ldg(b1 + o);
+      bw[kHexH + o] = __ldg(b2 + o);
+      bw[2 * kHexH + o] = o < kHexHead ? __ldg(b3 + o) : 0.f;
+    }
+  }
+  if (warp == kWsProducerWarps) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(kBarFull + s), kWsProducerWarps + kWsConsumers / 32);
+      tc::mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int t = 0; t < kWsTStages; ++t) {
+      tc::mbar_init(bar(kBarReady + t), 1);
+      tc::mbar_init(bar(kBarFree + t), kWsConsumers / 32);
+    }
+    tc::mbar_init(bar(kBarLayer), 1);
+    tc::mbar_init(bar(kBarFinal), 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
+
+  if (warp < kWsProducerWarps) {
+    // ------------------------------ producers ------------------------------
+    // two warpgroups at 176 registers, the consumers' one at 152: together
+    // exactly the 384 x 168 the block was launched with
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+    const int row = tid & (kHexTile - 1), half = tid >> 7;
+    const int sub = lid >> 3, c4 = lid & 7;
+    uint32_t G = 0;   // samples this CTA has produced so far
+    CornerRegs ra, rb;
+    int64_t tile0 = 0;
+    const uint64_t keep = l2_evict_last();
+    auto prefetch = [&](int k, CornerRegs& r) {
+      const int64_t down = (int64_t)hp.res_a[k] * (kHexC / 4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int g = 16 * warp + 4 * j + sub;
+        if (tile0 + g < N) {
+          const uint32_t crow = __float_as_uint(smp[k * kHexTile + g].x);
+          const float4* p = reinterpret_cast<const float4*>(planes + (int64_t)crow * kHexC) + c4;
+          r.c[j][0] = ld_nc_v4_hint(p, keep);
+          r.c[j][1] = ld_nc_v4_hint(p + kHexC / 4, keep);
+          r.c[j][2] = ld_nc_v4_hint(p + down, keep);
+          r.c[j][3] = ld_nc_v4_hint(p + down + kHexC / 4, keep);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) r.c[j][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    };
+    auto produce = [&](int k, CornerRegs& r) -> bool {
+      const int s = G & 1;
+      if (G >= 2 && !warp_wait(bar(kBarEmpty + s), ((G >> 1) + 1) & 1)) return false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int g = 16 * warp + 4 * j + sub;
+        const float4 rec = smp[k * kHexTile + g];
+        const float wa = rec.y, wb = rec.z;
+        const float w00 = (1.0f - wa) * (1.0f - wb), w01 = wa * (1.0f - wb), w10 = (1.0f - wa) * wb, w11 = wa * wb;
+        const float4 a = r.c[j][0], bb = r.c[j][1], c = r.c[j][2], d = r.c[j][3];
+        float4 z;
+        z.x = w00 * a.x + w01 * bb.x + w10 * c.x + w11 * d.x;
+        z.y = w00 * a.y + w01 * bb.y + w10 * c.y + w11 * d.y;
+        z.z = w00 * a.z + w01 * bb.z + w10 * c.z + w11 * d.z;
+        z.w = w00 * a.w + w01 * bb.w + w10 * c.w + w11 * d.w;
+        if (latent && tile0 + g < N) st_v4_stream(latent + (tile0 + g) * IN + k * kHexC + 4 * c4, z, l2_evict_first());
+        store_split4(sm, Lay::z(s), HexTcLayout::Z_PLANE, g, 4 * c4, z);
+      }
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
+      ++G;
+      return true;
+    };
+    for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
+      // the previous tile's sample table is no longer read; a failure anywhere ends every producer here
+      if (role_sync_or(1, kWsProducers, failed)) {
+        failed = true;
+        break;
+      }
+      tile0 = tile * kHexTile;
+      {
+        float xt[4] = {0.f, 0.f, 0.f, 0.f};
+        const int64_t n = tile0 + row;
+        const bool valid = n < N;
+        if (valid) hex_normalise(mu, frame, n, hp, xt);
+        for (int k = half; k < NS; k += 2) {
+          float wa = 0.f, wb = 0.f;
+          uint32_t crow = 0;
+          if (valid) crow = (uint32_t)(plane_corner(xt, hp, k, wa, wb) / kHexC);
+          smp[k * kHexTile + row] = make_float4(__uint_as_float(crow), wa, wb, 0.f);
+        }
+      }
+      role_sync(1, kWsProducers);
+      prefetch(0, ra);
+      prefetch(1, rb);
+      for (int k = 0; k < NS && !failed; k += 2) {
+        if (!produce(k, ra)) {
+          failed = true;
+          break;
+        }
+        if (k + 2 < NS) prefetch(k + 2, ra);
+        if (!produce(k + 1, rb)) {
+          failed = true;
+          break;
+        }
+        if (k + 3 < NS) prefetch(k + 3, rb);
+      }
+    }
+  } else {
+    // ------------------------------ consumers ------------------------------
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;" ::: "memory");
+    const int c = tid - kWsProducers;                  // the tile row (Gaussian) and TMEM lane
+    const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t L = tmem + 128 * kWsTStages;        // layers 2 and 3: main | correction
+    const SplitOp Hk = kmajor(sbase + Lay::H, HexTcLayout::H_PLANE, kHexH);
+    uint32_t G = 0, lph = 0;
+    // the first two ring stages' W1 slices (samples 0 and 1 of the first
+    // tile); wreg then holds the next slice to stage (sample 2)
+    float wreg[16];
+    for (int s = 0; s < 2; ++s) {
+      load_w1_slice(W1, IN, s, c, wreg);
+      store_w1_slice(sm, Lay::w(s), c, wreg);
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
+    }
+    load_w1_slice(W1, IN, 2 % NS, c, wreg);
+    for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
+      const int64_t n = tile * kHexTile + c;
+      const bool valid = n < N;
+      const bool has_next = (tile + gridDim.x) * kHexTile < N;
+      float acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      // ---- layer 1: issue sample k, then consume sample k - 1 ----
+      for (int k = 0; k <= NS && !failed; ++k) {
+        if (k < NS && c == 0) {
+          const uint32_t g = G + k, s = g & 1, t = g % kWsTStages;
+          bool ok = tc::mbar_wait_bounded(bar(kBarFull + s), (g >> 1) & 1, kWsWait);
+          if (ok && g >= (uint32_t)kWsTStages)
+            ok = tc::mbar_wait_bounded(bar(kBarFree + t), ((g / kWsTStages) - 1) & 1, kWsWait);
+          if (ok) {
+            tc::fence_after_sync();
+            mma6(tmem + 128 * t, tmem + 128 * t + 64, kmajor_zpad(sbase + Lay::z(s), HexTcLayout::Z_PLANE),
+                 kmajor(sbase + Lay::w(s), HexTcLayout::W_PLANE, kHexC), kHexC,
+                 tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+            tc::mma_commit(bar(kBarEmpty + s));
+            tc::mma_commit(bar(kBarReady + t));
+          } else {
+            failed = true;
+          }
+        }
+        __syncwarp();
+        failed = __any_sync(0xffffffffu, failed);   // the issuing lane's outcome, for its whole warp
+        if (k >= 1 && !failed) {
+          const uint32_t g = G + k - 1, t = g % kWsTStages;
+          if (!warp_wait(bar(kBarReady + t), (g / kWsTStages) & 1)) {
+            failed = true;
+          } else {
+            tc::fence_after_sync();
+            add_partial64(tmem + 128 * t + lane, tmem + 128 * t + 64 + lane, acc);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lid == 0) tc::mbar_arrive(bar(kBarFree + t));
+            // sample g's MMAs are done, so its ring stage is free: it takes the
+            // W1 slice of sample g + 2 (this tile's k + 1, or the next tile's first two)
+            if (k + 1 < NS || has_next) {
+              const int s2 = (int)(g & 1);
+              store_w1_slice(sm, Lay::w(s2), c, wreg);   // the slice of sample index (k + 1) % NS
+              tc::fence_proxy_async();
+              __syncwarp();
+              if (lid == 0) tc::mbar_arrive(bar(kBarFull + s2));
+              load_w1_slice(W1, IN, (k + 2) % NS, c, wreg);
+            }
+          }
+        }
+      }
+      G += NS;
+      // ---- h1 = relu(acc + b1) -> H; layer 2 ----
+      if (!failed) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = fmaxf(acc[i] + bias[i], 0.f);
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) store_split8(sm, Lay::H, HexTcLayout::H_PLANE, c, kc, kHexH, acc + 8 * kc);
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kWsConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      if (c == 0) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, Hk, kmajor(sbase + Lay::W2, HexTcLayout::S_PLANE, kHexH), kHexH,
+             tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      if (!failed) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+        add_partial64(L + lane, L + 64 + lane, acc);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = fmaxf(acc[i] + bias[kHexH + i], 0.f);
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) store_split8(sm, Lay::H, HexTcLayout::H_PLANE, c, kc, kHexH, acc + 8 * kc);
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kWsConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      // ---- the head (58 rows padded to 64) ----
+      if (c == 0) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, Hk, kmajor(sbase + Lay::W3, HexTcLayout::S_PLANE, kHexH), kHexH,
+             tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      if (failed) continue;   // the next role_sync_or ends every consumer
+      float* y = acc;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) y[i] = bias[2 * kHexH + i];
+      add_partial64(L + lane, L + 64 + lane, y);
+      tc::fence_before_sync();
+      if (valid) {
+        const uint64_t once = l2_evict_first();
+        float gw, gh, gt;
+        float2 gcr;
+        hex_window(hp, frame, n, gw, gh, gt, gcr);
+        float qh[4], q[4], s[3], cov[6];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const float m0 = ld_nc_hint(mu + 3 * n + i, once);
+          st_hint(out.mu + 3 * n + i, gh != 0.0f ? m0 + y[i] : m0, once);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qh[i] = ld_nc_hint(q_can + 4 * n + i, once) + y[3 + i];
+        normalise_quat(qh, q);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) s[i] = expf(ld_nc_hint(logs_can + 3 * n + i, once) + gw * y[7 + i]);
+        covariance(s, q, cov);
+        st_v4_stream(out.rot + 4 * n, make_float4(q[0], q[1], q[2], q[3]), once);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) st_hint(out.scale + 3 * n + i, s[i], once);
+#pragma unroll
+        for (int i = 0; i < 6; ++i) st_hint(out.cov + 6 * n + i, cov[i], once);
+#pragma unroll
+        for (int i = 0; i < kHexHead - 10; ++i)
+          st_hint(out.sh + 48 * n + i, ld_nc_hint(sh_can + 48 * n + i, once) + gw * y[10 + i], once);
+      }
+    }
+    // every MMA this CTA issued is complete before the tensor memory goes
+    if (c == 0) {
+      tc::mma_commit(bar(kBarFinal));
+      tc::mbar_wait_bounded(bar(kBarFinal), 0, kWsWait);
+    }
+  }
+
+  if (failed) atomicExch(&g_hex_device_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kWsProducerWarps) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
 // Backward, one 128-Gaussian tile per step of a persistent CTA:
 //   1. forward again (layer 1 streamed as in the forward, z from the saved
 //      latent when given), keeping h1 and h2 in registers;
@@ -1104,7 +1558,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
 // gradients are warp column sums gathered in shared memory, so they do not
 // depend on scheduling.  TMEM: stages as in the forward, plus the 64-row
 // weight-gradient accumulators at columns 256 (main) and 320 (correction).
-template <bool LATENT>
+template <bool LATENT, bool GATED>
 __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
@@ -1205,10 +1659,9 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     tiles_ready();
     // head rows 0..15 (d_mu, d_q, d_logs) into stage 1's columns; with the
     // energy-flow window all 64 (d loss / d w needs the SH offsets too)
-    const bool gated = hp.gate_cr != nullptr;
     if (tid == 0) {
       tc::fence_after_sync();
-      mma6(tmem + 128, tmem + 192, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, gated ? kHexH : 16, false, false));
+      mma6(tmem + 128, tmem + 192, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, GATED ? kHexH : 16, false, false));
       tc::mma_commit(mbar0);
     }
     if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
@@ -1217,12 +1670,14 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     float dy[32];
     float gw = 1.0f, gh = 1.0f, gt = 0.0f;
     float2 gcr = make_float2(0.f, 0.f);
-    if (valid) hex_window(hp, frame, n, gw, gh, gt, gcr);
-    float* gsum = reinterpret_cast<float*>(sm + BL::GSUM);
-    float dldw = 0.0f;   // d loss / d w: this thread's part of the w-scaled offsets
+    if constexpr (GATED) {
+      if (valid) hex_window(hp, frame, n, gw, gh, gt, gcr);
+    }
+    float dldw = 0.0f;   // d loss / d w: this thread's part of the w-scaled offsets (window only)
     if (half == 0) {
-      float a[32], c[32];
-      if (gated) {
+      constexpr int HC = GATED ? 32 : 16;   // head columns this half reads
+      float a[HC], c[HC];
+      if constexpr (GATED) {
         tc::tmem_ld32(tmem + 128 + lane, a);
         tc::tmem_ld32(tmem + 192 + lane, c);
       } else {
@@ -1258,37 +1713,41 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
         for (int i = 0; i < 3; ++i) {
           const float dl = ds[i] * s[i];   // d loss / d(log s + w d_logs)
           dy[7 + i] = gw * dl;
-          dldw += dl * dlogs_off[i];
+          if constexpr (GATED) dldw += dl * dlogs_off[i];
         }
 #pragma unroll
         for (int i = 10; i < 32; ++i) {
           const float g = g_or0(go.sh, 48 * n + (i - 10));
           dy[i] = gw * g;
-          if (gated) dldw += g * (a[i] + c[i] + bias[2 * kHexH + i]);
+          if constexpr (GATED) dldw += g * (a[i] + c[i] + bias[2 * kHexH + i]);
         }
       }
     } else {
-      float a[32], c[32];
-      if (gated) {
+      if constexpr (GATED) {
+        float a[32], c[32];
         tc::tmem_ld32(tmem + 128 + lane + 32, a);
         tc::tmem_ld32(tmem + 192 + lane + 32, c);
-      }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float g = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
-        dy[i] = gw * g;
-        if (gated && i < kHexHead - 32) dldw += g * (a[i] + c[i] + bias[2 * kHexH + 32 + i]);
+        for (int i = 0; i < 32; ++i) {
+          const float g = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
+          dy[i] = gw * g;
+          if (i < kHexHead - 32) dldw += g * (a[i] + c[i] + bias[2 * kHexH + 32 + i]);
+        }
+        reinterpret_cast<float*>(sm + BL::GSUM)[row] = dldw;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dy[i] = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
       }
-      if (gated) gsum[row] = dldw;
     }
     tc::fence_before_sync();
     store_row32(sm, T0, row, half, dy);
     atomicAdd(bacc + 2 * kHexH + half * 32 + lid, warp_column_sum(dy));
     tiles_ready();
-    if (gated && half == 0 && valid && hp.gate_grad) {
+    if (GATED && half == 0 && valid && hp.gate_grad) {
       // H(w) is piecewise constant: c and r receive gradient through w alone
       float gcr_out[2];
-      temporal_gate_backward(gt, gcr.x, gcr.y, hp.gate_tau, dldw + gsum[row], gcr_out);
+      temporal_gate_backward(gt, gcr.x, gcr.y, hp.gate_tau, dldw + reinterpret_cast<const float*>(sm + BL::GSUM)[row],
+                             gcr_out);
       float2* dst = reinterpret_cast<float2*>(hp.gate_grad) + n;
       const float2 prev = *dst;
       *dst = make_float2(prev.x + gcr_out[0], prev.y + gcr_out[1]);
@@ -1531,6 +1990,26 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
   HexParams p = make_hex_params(h);
   hex_set_gate(p, gate);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
+  if (h->n_scales * 6 <= 24 && !getenv("SPIN4D_HEX_FWD_TC")) {
+    // tensor cores, bf16x3 split, warp-specialised
+    static bool ws_configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int smem = HexWsLayout::BYTES;
+    if (!ws_configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(hexplane_fwd_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_fwd_ws_kernel, kWsThreads, smem);
+      if (e != cudaSuccess) return cuda_status(e);
+      if (occ != 1) return SPIN4D_ERR_UNSUPPORTED;   // one CTA holds all 512 TMEM columns
+      ws_configured[dev] = true;
+    }
+    const int blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
+    hexplane_fwd_ws_kernel<<<blocks, kWsThreads, smem, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can,
+                                                                             logs_can, sh_can, o, out.latent);
+    return launch_status();
+  }
   if (h->n_scales * 6 <= 24) {
     // tensor cores, bf16x3 split
     static bool configured[64] = {false};
@@ -1608,7 +2087,8 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     const int smem = HexBwdLayout::BYTES;
     if (!configured[dev]) {
       bool ok = true;
-      for (auto* kern : {hexplane_bwd_tc_kernel<false>, hexplane_bwd_tc_kernel<true>}) {
+      for (auto* kern : {hexplane_bwd_tc_kernel<false, false>, hexplane_bwd_tc_kernel<true, false>,
+                         hexplane_bwd_tc_kernel<false, true>, hexplane_bwd_tc_kernel<true, true>}) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e);
         int occ = 0;
@@ -1621,7 +2101,8 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     }
     if (usable[dev]) {
       blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
-      auto* kern = latent ? hexplane_bwd_tc_kernel<true> : hexplane_bwd_tc_kernel<false>;
+      auto* kern = gate ? (latent ? hexplane_bwd_tc_kernel<true, true> : hexplane_bwd_tc_kernel<false, true>)
+                        : (latent ? hexplane_bwd_tc_kernel<true, false> : hexplane_bwd_tc_kernel<false, false>);
       kern<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, latent, go, grad_planes,
                                              static_cast<float*>(workspace), n_params);
       SPIN4D_CHECK(launch_status());

@@ -20,6 +20,8 @@
 #include <cmath>
 #include <stdlib.h>
 
+#include <mutex>
+
 #include "host.h"
 #include "tc.cuh"
 
@@ -467,15 +469,11 @@ struct HexTcLayout {
   static constexpr int W3 = W2 + 3 * S_PLANE;                      // [64][64] x 3 planes (58 rows used)
   static constexpr int BIAS = W3 + 3 * S_PLANE;                    // b1 | b2 | b3 (64 each)
   static constexpr int MISC = BIAS + 3 * kHexH * 4;                // 2 mbarriers + TMEM address
-  // forward: per plane sample and Gaussian of the tile, {first corner row, wa, wb, 0}
-  static constexpr int SMP = MISC + 32;
-  static constexpr int BYTES = SMP + 24 * kHexTile * 16;
   static __device__ __forceinline__ int z(int b) { return A + b * Z_STAGE; }
   static __device__ __forceinline__ int w(int b) { return B1 + b * W_STAGE; }
 };
 static_assert(3 * HexTcLayout::H_PLANE <= 2 * HexTcLayout::Z_STAGE, "the H tile must fit over the z stages");
-static_assert(HexTcLayout::B1 % 128 == 0 && HexTcLayout::SMP % 16 == 0, "tile alignment");
-static_assert(HexTcLayout::BYTES <= 227 * 1024, "forward tiles exceed the shared memory of one CTA");
+static_assert(HexTcLayout::B1 % 128 == 0, "tile alignment");
 
 // Backward: the forward's z stages, W1 stages and W2 | W3 at the same
 // offsets, the scatter staging over W2 | W3, a second activation tile T1,
@@ -804,104 +802,6 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
 // Registers of one plane sample in the row-coalesced gather: this thread's
 // chunk of the W1 slice, and channels 4 (lane & 7) .. + 3 of the four corner
 // rows of four Gaussians with their bilinear fractions.
-struct RowRegs {
-  float w[8];
-  float4 c[4][4];   // [Gaussian j][corner 00, 01, 10, 11]
-};
-
-// hex_stream for sampling from the planes, with the corner rows read whole:
-// lane l of warp w takes channels 4 (l & 7) .. + 3 of Gaussians
-// 16 w + 4 j + (l >> 3), j = 0..3, so eight lanes read one 128-byte row and a
-// warp's load covers four rows.  (Reading a Gaussian's own row per lane makes
-// every 32-byte sector a separate L1 wavefront, which bounds that form.)
-// smp[k * 128 + g] holds sample k of Gaussian g of the tile: its first
-// corner as a row index of the planes (rows of kHexC floats), wa and wb;
-// tile0 is the tile's first Gaussian.
-template <int DEPTH, class Issue, class Consume>
-__device__ __forceinline__ bool hex_stream_rows(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
-                                                const float* __restrict__ W1, float* __restrict__ zdst, int64_t tile0,
-                                                int64_t N, const float4* smp, HexBars& bars, Issue issue,
-                                                Consume consume) {
-  using Lay = HexTcLayout;
-  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
-  const int sub = lid >> 3, c4 = lid & 7;
-  const int IN = hp.in_dim, NS = hp.n_samples;
-  RowRegs ra, rb;
-  auto prefetch = [&](int k, RowRegs& r) {
-    ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
-    const int64_t down = (int64_t)hp.res_a[k] * (kHexC / 4);   // one row of the plane, in float4
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = 16 * warp + 4 * j + sub;
-      if (tile0 + g < N) {
-        const uint32_t crow = __float_as_uint(smp[k * kHexTile + g].x);
-        const float4* p = reinterpret_cast<const float4*>(planes + (int64_t)crow * kHexC) + c4;
-        r.c[j][0] = __ldg(p);
-        r.c[j][1] = __ldg(p + kHexC / 4);
-        r.c[j][2] = __ldg(p + down);
-        r.c[j][3] = __ldg(p + down + kHexC / 4);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) r.c[j][c] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-  };
-  auto step = [&](int k, RowRegs& r) -> bool {
-    const int b = k & 1;
-    bool ok = true;
-    if (k >= 2) {   // as in hex_stream: take sample k-2's results, then refill the stage
-      ok = bars.wait(b);
-      tc::fence_after_sync();
-      if (ok) consume(k - 2, b);
-    }
-    store_split8(sm, Lay::w(b), Lay::W_PLANE, tid >> 2, tid & 3, kHexC, r.w);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = 16 * warp + 4 * j + sub;
-      const float4 rec = smp[k * kHexTile + g];
-      const float wa = rec.y, wb = rec.z;
-      const float w00 = (1.0f - wa) * (1.0f - wb), w01 = wa * (1.0f - wb), w10 = (1.0f - wa) * wb, w11 = wa * wb;
-      const float4 a = r.c[j][0], bb = r.c[j][1], c = r.c[j][2], d = r.c[j][3];
-      float4 z;
-      z.x = w00 * a.x + w01 * bb.x + w10 * c.x + w11 * d.x;
-      z.y = w00 * a.y + w01 * bb.y + w10 * c.y + w11 * d.y;
-      z.z = w00 * a.z + w01 * bb.z + w10 * c.z + w11 * d.z;
-      z.w = w00 * a.w + w01 * bb.w + w10 * c.w + w11 * d.w;
-      if (zdst && tile0 + g < N) st_v4_stream(zdst + (tile0 + g) * IN + k * kHexC + 4 * c4, z, l2_evict_first());
-      store_split4(sm, Lay::z(b), Lay::Z_PLANE, g, 4 * c4, z);
-    }
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    if (__syncthreads_or(!ok)) return false;
-    if (tid == 0) {
-      tc::fence_after_sync();
-      issue(k, b);
-      tc::mma_commit(bars.addr(b));
-    }
-    if (k + DEPTH < NS) prefetch(k + DEPTH, r);
-    return true;
-  };
-  prefetch(0, ra);
-  if constexpr (DEPTH == 2) {
-    prefetch(1, rb);
-    for (int k = 0; k < NS; k += 2) {
-      if (!step(k, ra)) return false;
-      if (!step(k + 1, rb)) return false;
-    }
-  } else {
-    for (int k = 0; k < NS; ++k)
-      if (!step(k, ra)) return false;
-  }
-  for (int k = NS - 2; k < NS; ++k) {   // the last two samples
-    const int b = k & 1;
-    const bool ok = bars.wait(b);
-    if (__syncthreads_or(!ok)) return false;
-    tc::fence_after_sync();
-    consume(k, b);
-  }
-  return true;
-}
-
 // grad[0..63] += the 256 bytes at shared address src, asynchronously (one
 // bulk reduction); completion is tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_add_2rows(float* grad, uint32_t src) {
@@ -954,169 +854,10 @@ __device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, co
   }
 }
 
-__global__ void __launch_bounds__(kHexThreads, 1) hexplane_fwd_tc_kernel(
-    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
-    const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
-    const float* __restrict__ logs_can, const float* __restrict__ sh_can, HexOutPtrs out, float* __restrict__ latent) {
-  using Lay = HexTcLayout;
-  extern __shared__ __align__(1024) uint8_t sm[];
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid & (kHexTile - 1), half = tid / kHexTile;
-  const int IN = hp.in_dim;
-  const float* W1 = W;
-  const float* b1 = W1 + kHexH * IN;
-  const float* W2g = b1 + kHexH;
-  const float* b2 = W2g + kHexH * kHexH;
-  const float* W3g = b2 + kHexH;
-  const float* b3 = W3g + kHexHead * kHexH;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::MISC + 16);
-  const uint32_t mbar0 = tc::smem_u32(sm + Lay::MISC), mbar1 = mbar0 + 8;
-  const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
-  float4* smp = reinterpret_cast<float4*>(sm + Lay::SMP);
-
-  stage_small_layers(sm, Lay::BIAS, W2g, b1, b2, W3g, b3);
-  if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
-    tc::tmem_relinquish();
-  }
-  if (tid == 0) {
-    tc::mbar_init(mbar0, 1);
-    tc::mbar_init(mbar1, 1);
-    tc::mbar_fence_init();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t col = (uint32_t)(half * 32);
-  const uint32_t sbase = tc::smem_u32(sm);
-  const SplitOp H = kmajor(sbase + Lay::A, Lay::H_PLANE, kHexH);
-  // TMEM: plane sample k accumulates into columns [128b, 128b + 128) of stage
-  // b = k & 1 (main, then correction); layer 2 reuses stage 0's columns and
-  // the head stage 1's.
-  HexBars bars{mbar0, mbar1, 0u, 0u};
-  bool failed = false;
-
-  for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
-    const int64_t tile0 = tile * kHexTile, n = tile0 + row;
-    const bool valid = n < N;
-    {
-      // the tile's sample table: each half takes every other sample
-      float xt[4] = {0.f, 0.f, 0.f, 0.f};
-      if (valid) hex_normalise(mu, frame, n, hp, xt);
-      for (int k = half; k < hp.n_samples; k += 2) {
-        float wa = 0.f, wb = 0.f;
-        uint32_t crow = 0;
-        if (valid) crow = (uint32_t)(plane_corner(xt, hp, k, wa, wb) / kHexC);
-        smp[k * kHexTile + row] = make_float4(__uint_as_float(crow), wa, wb, 0.f);
-      }
-    }
-    __syncthreads();
-    float acc1[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc1[i] = 0.f;
-    // ---- layer 1, streamed over the plane samples ----
-    auto issue = [&](int, int b) {
-      mma6(tmem + 128 * b, tmem + 128 * b + 64, kmajor_zpad(sbase + Lay::z(b), Lay::Z_PLANE),
-           kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
-    };
-    auto consume = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, acc1); };
-    if (!hex_stream_rows<2>(sm, hp, planes, W1, latent, tile0, N, smp, bars, issue, consume)) {
-      failed = true;
-      break;
-    }
-    // ---- h1 = relu(sum + b1) -> H tile (over the z stages) ----
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc1[i] = fmaxf(acc1[i] + bias[half * 32 + i], 0.f);
-    store_row32(sm, Lay::A, row, half, acc1);
-    tiles_ready();
-    // ---- layer 2 into stage 0's columns ----
-    if (tid == 0) {
-      tc::fence_after_sync();
-      mma6(tmem, tmem + 64, H, kmajor(sbase + Lay::W2, Lay::S_PLANE, kHexH), kHexH,
-           tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
-      tc::mma_commit(mbar0);
-    }
-    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
-    tc::fence_after_sync();
-    {
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      add_partial(tmem + lane + col, tmem + 64 + lane + col, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i] + bias[kHexH + half * 32 + i], 0.f);
-      store_row32(sm, Lay::A, row, half, v);
-    }
-    tiles_ready();
-    // ---- head (58 rows, padded to 64) into stage 1's columns ----
-    if (tid == 0) {
-      tc::fence_after_sync();
-      mma6(tmem + 128, tmem + 192, H, kmajor(sbase + Lay::W3, Lay::S_PLANE, kHexH), kHexH,
-           tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
-      tc::mma_commit(mbar0);
-    }
-    if (__syncthreads_or(!bars.wait(0))) { failed = true; break; }
-    tc::fence_after_sync();
-    {
-      float y[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = bias[2 * kHexH + half * 32 + i];
-      add_partial(tmem + 128 + lane + col, tmem + 192 + lane + col, y);
-      tc::fence_before_sync();
-      if (valid) {
-        float gw, gh, gt;
-        float2 gcr;
-        hex_window(hp, frame, n, gw, gh, gt, gcr);
-        if (half == 0) {
-          float qh[4], q[4], s[3], cov[6];
-#pragma unroll
-          for (int i = 0; i < 3; ++i) {
-            const float m0 = __ldg(mu + 3 * n + i);
-            out.mu[3 * n + i] = gh != 0.0f ? m0 + y[i] : m0;
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + y[3 + i];
-          normalise_quat(qh, q);
-#pragma unroll
-          for (int i = 0; i < 3; ++i) s[i] = expf(__ldg(logs_can + 3 * n + i) + gw * y[7 + i]);
-          covariance(s, q, cov);
-          reinterpret_cast<float4*>(out.rot)[n] = make_float4(q[0], q[1], q[2], q[3]);
-#pragma unroll
-          for (int i = 0; i < 3; ++i) out.scale[3 * n + i] = s[i];
-#pragma unroll
-          for (int i = 0; i < 6; ++i) out.cov[6 * n + i] = cov[i];
-#pragma unroll
-          for (int i = 10; i < 32; ++i) out.sh[48 * n + (i - 10)] = __ldg(sh_can + 48 * n + (i - 10)) + gw * y[i];
-        } else {
-#pragma unroll
-          for (int i = 0; i < kHexHead - 32; ++i)
-            out.sh[48 * n + 22 + i] = __ldg(sh_can + 48 * n + 22 + i) + gw * y[i];
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  if (failed) {
-    if (tid == 0) atomicExch(&g_hex_device_error, 1);
-    bars.wait(0);
-    bars.wait(1);
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
-  }
-}
-
-
 // ---------------------------------------------------------------------------
-// Forward, warp-specialised.  The same arithmetic as hexplane_fwd_tc_kernel
-// (the same split products, the same fp32 accumulation order), with the
-// per-sample chain taken apart so that no step waits for the whole CTA:
+// Forward, warp-specialised: the tensor-core form of the layers (bf16x3
+// split products, fresh accumulators per plane sample added in fp32), with
+// the per-sample chain taken apart so that no step waits for the whole CTA:
 //   * 8 producer warps gather the tile's corner rows into registers two plane
 //     samples ahead, interpolate, and write the split z_k into a two-stage
 //     shared-memory ring;
@@ -1990,7 +1731,7 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
   HexParams p = make_hex_params(h);
   hex_set_gate(p, gate);
   HexOutPtrs o{out.mu, out.rot, out.scale, out.sh, out.cov};
-  if (h->n_scales * 6 <= 24 && !getenv("SPIN4D_HEX_FWD_TC")) {
+  if (h->n_scales * 6 <= 24) {
     // tensor cores, bf16x3 split, warp-specialised
     static bool ws_configured[64] = {false};
     int dev = 0;
@@ -2008,26 +1749,6 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     const int blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
     hexplane_fwd_ws_kernel<<<blocks, kWsThreads, smem, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can,
                                                                              logs_can, sh_can, o, out.latent);
-    return launch_status();
-  }
-  if (h->n_scales * 6 <= 24) {
-    // tensor cores, bf16x3 split
-    static bool configured[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    const int smem = HexTcLayout::BYTES;
-    if (!configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(hexplane_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      int occ = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_fwd_tc_kernel, kHexThreads, smem);
-      if (e != cudaSuccess) return cuda_status(e);
-      if (occ < 1 || occ * 256 > 512) return SPIN4D_ERR_UNSUPPORTED;
-      configured[dev] = true;
-    }
-    const int blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
-    hexplane_fwd_tc_kernel<<<blocks, kHexThreads, smem, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can,
-                                                                               logs_can, sh_can, o, out.latent);
     return launch_status();
   }
   if (gate) return SPIN4D_ERR_UNSUPPORTED;   // the window is built into the tensor-core kernels only

@@ -799,9 +799,6 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
   return true;
 }
 
-// Registers of one plane sample in the row-coalesced gather: this thread's
-// chunk of the W1 slice, and channels 4 (lane & 7) .. + 3 of the four corner
-// rows of four Gaussians with their bilinear fractions.
 // grad[0..63] += the 256 bytes at shared address src, asynchronously (one
 // bulk reduction); completion is tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_add_2rows(float* grad, uint32_t src) {

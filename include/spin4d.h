@@ -346,7 +346,9 @@ size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N);
  * forward's saved latent for the same inputs; given, the plane samples are
  * read from it instead of being gathered again.  workspace: device memory
  * of at least spin4d_hexplane_bwd_workspace(h, N) bytes, 256-byte aligned,
- * owned by the caller, overwritten.  Plane gradients are accumulated with
+ * owned by the caller, overwritten (per-block weight-gradient partials, and
+ * with a saved latent N x 64 fp32 of hidden-layer gradients handed between
+ * the two kernels of that path).  Plane gradients are accumulated with
  * fp32 atomics (their order of summation is not fixed); weight gradients
  * are summed in a fixed order.
  */

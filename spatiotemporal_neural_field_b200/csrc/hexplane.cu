@@ -467,8 +467,6 @@ struct HexTcLayout {
   static constexpr int S_PLANE = plane_bytes(kHexH, kHexH);        // 8 KB
   static constexpr int W2 = B1 + 2 * W_STAGE;                      // [64][64] x 3 planes
   static constexpr int W3 = W2 + 3 * S_PLANE;                      // [64][64] x 3 planes (58 rows used)
-  static constexpr int BIAS = W3 + 3 * S_PLANE;                    // b1 | b2 | b3 (64 each)
-  static constexpr int MISC = BIAS + 3 * kHexH * 4;                // 2 mbarriers + TMEM address
   static __device__ __forceinline__ int z(int b) { return A + b * Z_STAGE; }
   static __device__ __forceinline__ int w(int b) { return B1 + b * W_STAGE; }
 };
@@ -643,11 +641,6 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-__device__ __forceinline__ void ld_nc_v8_stream(const float* p, float v[8], uint64_t pol) {
-  asm volatile("ld.global.nc.L2::cache_hint.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-               : "l"(p), "l"(pol));
-}
 __device__ __forceinline__ void st_v4_stream(float* p, float4 v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
                "f"(v.w), "l"(pol)
@@ -681,62 +674,47 @@ __device__ __forceinline__ void st_hint(float* p, float v, uint64_t pol) {
 // (row tid/4, 8 columns) and, for its Gaussian, either the 16 channels
 // (half*16 ..) of the four corner rows with their bilinear weights, or the
 // 16 values of a saved latent.
-template <bool LATENT>
+// One thread's share of a plane sample in flight: its W1 slice chunk, its
+// half of the four corner rows, and the bilinear weights.
 struct SampleRegs {
   float w[8];
   float c[4][16];
   float wt[4];
 };
-template <>
-struct SampleRegs<true> {
-  float w[8];
-  float z[16];
-};
 
 // Streams the plane samples of one tile through the two stages.  Stage
 // b = k & 1 receives sample k: the 64x32 slice of W1 for the sample and the
-// tile's 128x32 feature block z_k (split), z_k read from zsrc (a saved
-// latent) when LATENT, else sampled from the planes (and then copied to zdst
-// when given).  issue(k, b) runs on thread 0 once the stage is written and
-// its MMAs are committed to stage b's barrier; consume(k, b) runs on every
-// thread once they are done, before the stage takes sample k + 2.  Each
-// thread reads its half of its Gaussian's four corner rows (or latent row)
-// as 32-byte sectors.  Global loads run DEPTH samples ahead: with DEPTH = 2,
-// two register sets (even and odd samples) keep about 128 KB of row reads
-// per SM in flight while the tensor core and the barriers work.  The sample
-// count is even (6 per scale).  Returns false if a wait ran out.
-template <int DEPTH, bool LATENT, class Issue, class Consume>
+// tile's 128x32 feature block z_k (split), sampled from the planes.
+// issue(k, b) runs on thread 0 once the stage is written and its MMAs are
+// committed to stage b's barrier; consume(k, b) runs on every thread once
+// they are done, before the stage takes sample k + 2.  Each thread reads its
+// half of its Gaussian's four corner rows as 32-byte sectors, one sample
+// ahead.  The sample count is even (6 per scale).  Returns false if a wait
+// ran out.
+template <class Issue, class Consume>
 __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, const float* __restrict__ planes,
-                                           const float* __restrict__ W1, const float* __restrict__ zsrc,
-                                           float* __restrict__ zdst, int64_t n, bool valid, const float xt[4],
+                                           const float* __restrict__ W1, bool valid, const float xt[4],
                                            HexBars& bars, Issue issue, Consume consume) {
   using Lay = HexTcLayout;
-  using Regs = SampleRegs<LATENT>;
   const int tid = threadIdx.x, row = tid & (kHexTile - 1), half = tid / kHexTile;
   const int IN = hp.in_dim, NS = hp.n_samples;
-  Regs ra, rb;
-  auto prefetch = [&](int k, Regs& r) {
+  SampleRegs r;
+  auto prefetch = [&](int k) {
     ld_nc_v8(W1 + (size_t)(tid >> 2) * IN + k * kHexC + (tid & 3) * 8, r.w);
     if (!valid) return;
-    if constexpr (LATENT) {
-      const uint64_t pol = l2_evict_first();
-      ld_nc_v8_stream(zsrc + n * IN + k * kHexC + half * 16, r.z, pol);
-      ld_nc_v8_stream(zsrc + n * IN + k * kHexC + half * 16 + 8, r.z + 8, pol);
-    } else {
-      const PlaneSample ps = plane_sample(xt, hp, k);
-      r.wt[0] = ps.w00;
-      r.wt[1] = ps.w01;
-      r.wt[2] = ps.w10;
-      r.wt[3] = ps.w11;
-      const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
+    const PlaneSample ps = plane_sample(xt, hp, k);
+    r.wt[0] = ps.w00;
+    r.wt[1] = ps.w01;
+    r.wt[2] = ps.w10;
+    r.wt[3] = ps.w11;
+    const int64_t off[4] = {ps.o00, ps.o01, ps.o10, ps.o11};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        ld_nc_v8(planes + off[c] + half * 16, r.c[c]);
-        ld_nc_v8(planes + off[c] + half * 16 + 8, r.c[c] + 8);
-      }
+    for (int c = 0; c < 4; ++c) {
+      ld_nc_v8(planes + off[c] + half * 16, r.c[c]);
+      ld_nc_v8(planes + off[c] + half * 16 + 8, r.c[c] + 8);
     }
   };
-  auto step = [&](int k, Regs& r) -> bool {
+  auto step = [&](int k) -> bool {
     const int b = k & 1;
     bool ok = true;
     if (k >= 2) {   // sample k-2 used this stage: take its results, then refill
@@ -752,18 +730,7 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       z[i] = 0.f;
-      if constexpr (LATENT) {
-        if (valid) z[i] = r.z[i];
-      } else {
-        if (valid) z[i] = r.wt[0] * r.c[0][i] + r.wt[1] * r.c[1][i] + r.wt[2] * r.c[2][i] + r.wt[3] * r.c[3][i];
-      }
-    }
-    if constexpr (!LATENT) {
-      if (valid && zdst) {
-        float4* d = reinterpret_cast<float4*>(zdst + n * IN + k * kHexC + half * 16);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) d[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-      }
+      if (valid) z[i] = r.wt[0] * r.c[0][i] + r.wt[1] * r.c[1][i] + r.wt[2] * r.c[2][i] + r.wt[3] * r.c[3][i];
     }
     store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2, kHexC, z);
     store_split8(sm, Lay::z(b), Lay::Z_PLANE, row, half * 2 + 1, kHexC, z + 8);
@@ -775,20 +742,12 @@ __device__ __forceinline__ bool hex_stream(uint8_t* sm, const HexParams& hp, con
       issue(k, b);
       tc::mma_commit(bars.addr(b));
     }
-    if (k + DEPTH < NS) prefetch(k + DEPTH, r);
+    if (k + 1 < NS) prefetch(k + 1);
     return true;
   };
-  prefetch(0, ra);
-  if constexpr (DEPTH == 2) {
-    prefetch(1, rb);
-    for (int k = 0; k < NS; k += 2) {
-      if (!step(k, ra)) return false;
-      if (!step(k + 1, rb)) return false;
-    }
-  } else {
-    for (int k = 0; k < NS; ++k)
-      if (!step(k, ra)) return false;
-  }
+  prefetch(0);
+  for (int k = 0; k < NS; ++k)
+    if (!step(k)) return false;
   for (int k = NS - 2; k < NS; ++k) {   // the last two samples
     const int b = k & 1;
     const bool ok = bars.wait(b);
@@ -1281,27 +1240,27 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
   }
 }
 
-// Backward, one 128-Gaussian tile per step of a persistent CTA:
-//   1. forward again (layer 1 streamed as in the forward, z from the saved
-//      latent when given), keeping h1 and h2 in registers;
+// Backward without a saved latent (the planes sampled again), one
+// 128-Gaussian tile per step of a persistent CTA:
+//   1. forward again (layer 1 streamed through the two stages), keeping h1
+//      and h2 in registers;
 //   2. the head's rows 0..15 give q' and s', and with them the head adjoint
 //      dy (58 values, zero padded to 64);
 //   3. dh2 = (dy W3) * [h2 > 0] and dW3 += dy^T h2, then
 //      dh1 = (dh2 W2) * [h1 > 0] and dW2 += dh2^T h1 (one MMA group each);
-//   4. per plane sample k, dz_k = dh1 W1_k and dW1_k += dh1^T z_k; dz_k is
-//      spread over the sample's four bilinear corners with fp32 vector
-//      atomics.
+//   4. per plane sample k, dz_k = dh1 W1_k and dW1_k += dh1^T z_k; w_c dz_k
+//      goes to the sample's four bilinear corner rows by bulk reductions.
 // Weight gradients are partial sums over one tile (K = 128, fresh
 // accumulators) added in fp32 to the CTA's workspace slot, and bias
 // gradients are warp column sums gathered in shared memory, so they do not
 // depend on scheduling.  TMEM: stages as in the forward, plus the 64-row
 // weight-gradient accumulators at columns 256 (main) and 320 (correction).
-template <bool LATENT, bool GATED>
+template <bool GATED>
 __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
-    const float* __restrict__ logs_can, const float* __restrict__ latent, HexGradPtrs go,
-    float* __restrict__ grad_planes, float* __restrict__ ws, int n_params) {
+    const float* __restrict__ logs_can, HexGradPtrs go, float* __restrict__ grad_planes, float* __restrict__ ws,
+    int n_params) {
   using Lay = HexTcLayout;
   using BL = HexBwdLayout;
   extern __shared__ __align__(1024) uint8_t sm[];
@@ -1373,7 +1332,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
            kmajor(sbase + Lay::w(b), Lay::W_PLANE, kHexC), kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
     };
     auto consume1 = [&](int, int b) { add_partial(tmem + 128 * b + lane + col, tmem + 128 * b + 64 + lane + col, h1); };
-    if (!hex_stream<LATENT ? 2 : 1, LATENT>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue1, consume1)) {
+    if (!hex_stream(sm, hp, planes, W1, valid, xt, bars, issue1, consume1)) {
       failed = true;
       break;
     }
@@ -1599,7 +1558,7 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
         bulk_commit();
       }
     };
-    if (!hex_stream<LATENT ? 2 : 1, LATENT>(sm, hp, planes, W1, latent, nullptr, n, valid, xt, bars, issue2, consume2)) {
+    if (!hex_stream(sm, hp, planes, W1, valid, xt, bars, issue2, consume2)) {
       failed = true;
       break;
     }
@@ -1623,6 +1582,763 @@ __global__ void __launch_bounds__(kHexThreads, 1) hexplane_bwd_tc_kernel(
       if (o < kHexHead) sb3[o] += bacc[2 * kHexH + o];
     }
   if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward from a saved latent, warp-specialised, in two kernels per launch:
+//   A. hexplane_bwd_head_ws_kernel: per 128-Gaussian tile, layer 1 again
+//      from the latent, the head adjoint and the small layers' data and
+//      weight gradients; it writes the tile's dh1 = d loss / d(W1 z + b1)
+//      (N x 64 fp32) to the workspace;
+//   B. hexplane_bwd_dz_ws_kernel: per tile and plane sample, dz_k = dh1 W1_k
+//      and dW1_k = dh1^T z_k; dz_k's four bilinear corner rows go to the plane
+//      gradients by bulk reductions, dW1_k to the CTA's workspace slot.
+// In both, 4 producer warps read the tile's latent rows of each plane sample
+// into registers two samples ahead and write them split into a ring of z
+// stages, and 8 consumer warps (two threads per Gaussian, 32 columns each;
+// TMEM lane = tile row) stage the split W1 slices into the ring, issue the
+// MMAs from one lane into a ring of TMEM stages and take the results out.
+// Two kernels rather than one: the dz pass issues 72 small split-product
+// MMAs per sample, whose latency must be hidden two samples deep, and its
+// scatter staging needs 66 KB; with the small layers' tiles and weights
+// beside them the ring would have only two stages.  dh1 costs 256 bytes per
+// Gaussian written and read again.  Every hand-off is an mbarrier with a
+// bounded wait; the consumers' named barriers reduce a failure flag.
+// ---------------------------------------------------------------------------
+constexpr int kBwProducerWarps = 4;
+constexpr int kBwProducers = 32 * kBwProducerWarps;
+constexpr int kBwConsumers = 2 * kHexTile;
+constexpr int kBwThreads = kBwProducers + kBwConsumers;
+static_assert(kBwProducerWarps == 4 && 4 * 32 * 152 + 8 * 32 * 176 == kBwThreads * 168,
+              "the register split must equal the launch's total");
+
+// Kernel A: z ring | W1 ring | T0 | T1 | W2 | W3 | biases and sums.
+struct HexBwWsLayout {
+  static constexpr int Z_STAGE = HexTcLayout::Z_STAGE;             // split z_k, skewed (24,960 B)
+  static constexpr int W_STAGE = HexTcLayout::W_STAGE;             // split W1 slice (12,288 B)
+  static constexpr int ZR = 0;                                     // 2 z stages
+  static constexpr int WR = ZR + 2 * Z_STAGE;                      // 2 W1 stages
+  static constexpr int T0 = WR + 2 * W_STAGE;                      // [128][64] x 3 planes
+  static constexpr int T1 = T0 + 3 * HexTcLayout::H_PLANE;         // [128][64] x 3 planes
+  static constexpr int W2 = T1 + 3 * HexTcLayout::H_PLANE;         // split W2
+  static constexpr int W3 = W2 + 3 * HexTcLayout::S_PLANE;         // split W3 (58 rows, padded)
+  static constexpr int BIAS = W3 + 3 * HexTcLayout::S_PLANE;       // b1 | b2 | b3
+  static constexpr int BACC = BIAS + 3 * kHexH * 4;                // db1 | db2 | db3 over the CTA's tiles
+  static constexpr int GSUM = BACC + 3 * kHexH * 4;                // [128]: the SH half of d loss / d w
+  static constexpr int BARS = GSUM + kHexTile * 4;                 // 12 mbarriers, then the TMEM address
+  static constexpr int BYTES = BARS + 128;
+  static __device__ __forceinline__ int z(int s) { return ZR + s * Z_STAGE; }
+  static __device__ __forceinline__ int w(int s) { return WR + s * W_STAGE; }
+};
+static_assert(HexBwWsLayout::T0 % 128 == 0 && HexBwWsLayout::W2 % 128 == 0, "tile alignment");
+static_assert(HexBwWsLayout::BYTES <= 227 * 1024, "warp-specialised backward tiles exceed the shared memory of one CTA");
+
+// A z tile in the skewed layout read MN-major (its columns are N, its rows
+// K): the 8-row groups are adjacent, the 8-column chunks kZChunk apart.
+__device__ __forceinline__ SplitOp mnmajor_zpad(uint32_t base, int plane) {
+  return {base, (uint32_t)plane, 128u, (uint32_t)kZChunk, 256u};
+}
+
+// One of 256 threads' share of a split W1 slice (64 rows x 32 columns): row
+// c / 4, columns 8 (c % 4) .. + 7.
+__device__ __forceinline__ void load_w1_slice8(const float* __restrict__ W1, int IN, int k, int c, float v[8]) {
+  ld_nc_v8(W1 + (size_t)(c >> 2) * IN + k * kHexC + (c & 3) * 8, v);
+}
+__device__ __forceinline__ void store_w1_slice8(uint8_t* sm, int off, int c, const float v[8]) {
+  store_split8(sm, off, HexTcLayout::W_PLANE, c >> 2, c & 3, kHexC, v);
+}
+
+// W2 and W3 split (W3 padded with zero rows to 64) by threads t of nt.
+__device__ __forceinline__ void stage_w23_at(uint8_t* sm, int w2, int w3, const float* __restrict__ W2g,
+                                             const float* __restrict__ W3g, int t, int nt) {
+  for (int i = t; i < kHexH * (kHexH / 8); i += nt) {
+    const int r = i / (kHexH / 8), kc = i % (kHexH / 8);
+    const float4* a2 = reinterpret_cast<const float4*>(W2g + r * kHexH) + 2 * kc;
+    store_split8(sm, w2, HexTcLayout::S_PLANE, r, kc, kHexH, __ldg(a2), __ldg(a2 + 1));
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (r < kHexHead) {
+      const float4* a3 = reinterpret_cast<const float4*>(W3g + r * kHexH) + 2 * kc;
+      a = __ldg(a3);
+      b = __ldg(a3 + 1);
+    }
+    store_split8(sm, w3, HexTcLayout::S_PLANE, r, kc, kHexH, a, b);
+  }
+}
+
+
+// Kernel B: 3 z stages | 3 W1 stages | T0 (dh1) | scatter staging | barriers.
+constexpr int kDzIssuerWarp = kBwProducerWarps + kBwConsumers / 32;   // warp 12
+constexpr int kDzThreads = 32 * (kDzIssuerWarp + 1);
+struct HexDzWsLayout {
+  static constexpr int STAGES = 3;
+  static constexpr int TSTAGES = 4;
+  static constexpr int ZR = 0;
+  static constexpr int WR = ZR + STAGES * HexTcLayout::Z_STAGE;
+  static constexpr int T0 = WR + STAGES * HexTcLayout::W_STAGE;
+  static constexpr int SCAT = T0 + 3 * HexTcLayout::H_PLANE;       // per Gaussian its 4 corner rows, padded
+  static constexpr int SCAT_ROW = HexBwdLayout::SCAT_ROW;
+  static constexpr int BARS = SCAT + kHexTile * SCAT_ROW;           // 16 mbarriers, then the TMEM address
+  static constexpr int BYTES = BARS + 144;
+  static __device__ __forceinline__ int z(int s) { return ZR + s * HexTcLayout::Z_STAGE; }
+  static __device__ __forceinline__ int w(int s) { return WR + s * HexTcLayout::W_STAGE; }
+};
+static_assert(HexDzWsLayout::T0 % 128 == 0 && HexDzWsLayout::SCAT % 16 == 0 && HexDzWsLayout::SCAT_ROW % 16 == 0,
+              "tile alignment");
+static_assert(HexDzWsLayout::BYTES <= 227 * 1024, "dz-pass tiles exceed the shared memory of one CTA");
+static_assert(kWsTStages * 128 + 128 <= 512 && HexDzWsLayout::TSTAGES * 128 <= 512, "TMEM columns");
+// mbarriers of kernel B
+enum : int { kDzFull = 0, kDzEmpty = 3, kDzReady = 6, kDzFree = 10, kDzT0 = 14, kDzFinal = 15, kNumDzBars = 16 };
+static_assert(8 * kNumDzBars + 4 <= 144, "the mbarriers and the TMEM address fit their 144 bytes");
+
+// The producers of both backward kernels: the latent rows of every plane
+// sample of this CTA's tiles, in tile order, into a ring of S split z stages
+// at zring (with W_TOO, the sample's split W1 slice into the ring of W
+// stages at wring as well); a stage is written once the MMAs of the sample S
+// before it are done (its "empty" barrier) and then announced on its "full"
+// barrier.  Global loads run two samples ahead in registers.  Returns false
+// if a wait ran out.
+template <int S, bool W_TOO>
+__device__ __forceinline__ bool bw_stream_latent(uint8_t* sm, int zring, int wring, uint32_t full0, uint32_t empty0,
+                                                 const float* __restrict__ latent, const float* __restrict__ W1,
+                                                 int64_t N, int IN, int NS, uint32_t total) {
+  const int warp = threadIdx.x >> 5, lid = threadIdx.x & 31;
+  const int sub = lid >> 3, c4 = lid & 7;
+  const uint64_t once = l2_evict_first();
+  int64_t ptile = blockIdx.x;
+  int pk = 0;   // the next sample to read: tile ptile, plane sample pk
+  float4 ra[8], rb[8];
+  float wa[W_TOO ? 16 : 1], wb[W_TOO ? 16 : 1];
+  auto prefetch = [&](float4 (&r)[8], float (&w)[W_TOO ? 16 : 1]) {
+    if constexpr (W_TOO) load_w1_slice(W1, IN, pk, threadIdx.x, w);
+    const int64_t tile0 = ptile * kHexTile;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t n = tile0 + 32 * warp + 4 * j + sub;
+      r[j] = n < N ? ld_nc_v4_hint(reinterpret_cast<const float4*>(latent + n * IN + pk * kHexC) + c4, once)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (++pk == NS) {
+      pk = 0;
+      ptile += gridDim.x;
+    }
+  };
+  uint32_t G = 0;   // samples written so far
+  auto produce = [&](const float4 (&r)[8], const float (&w)[W_TOO ? 16 : 1]) -> bool {
+    const uint32_t s = G % S;
+    if (G >= (uint32_t)S && !warp_wait(empty0 + 8u * s, ((G / S) - 1) & 1)) return false;
+    if constexpr (W_TOO) store_w1_slice(sm, wring + (int)s * HexTcLayout::W_STAGE, threadIdx.x, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      store_split4(sm, zring + (int)s * HexTcLayout::Z_STAGE, HexTcLayout::Z_PLANE, 32 * warp + 4 * j + sub, 4 * c4,
+                   r[j]);
+    tc::fence_proxy_async();
+    __syncwarp();
+    if (lid == 0) tc::mbar_arrive(full0 + 8u * s);
+    ++G;
+    return true;
+  };
+  prefetch(ra, wa);
+  prefetch(rb, wb);
+  for (uint32_t g = 0; g < total; g += 2) {
+    if (!produce(ra, wa)) return false;
+    prefetch(ra, wa);
+    if (g + 1 < total) {
+      if (!produce(rb, wb)) return false;
+      prefetch(rb, wb);
+    }
+  }
+  return true;
+}
+
+// Kernel A, the head of the backward from a saved latent: per tile, layer 1
+// again (z from the latent through the two-stage ring), h1 and h2, the head
+// adjoint dy, dh2 = (dy W3) * [h2 > 0] with dW3 = dy^T h2, and
+// dh1 = (dh2 W2) * [h1 > 0] with dW2 = dh2^T h1; it writes dh1 to dh1_out
+// (N x 64) and adds the weight and bias gradients of W2, W3 and the biases to
+// the CTA's workspace slot, which it zeroes first.
+template <bool GATED>
+__global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
+    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
+    const float* __restrict__ W, const float* __restrict__ q_can, const float* __restrict__ logs_can,
+    const float* __restrict__ latent, HexGradPtrs go, float* __restrict__ dh1_out, float* __restrict__ ws,
+    int n_params) {
+  using Lay = HexBwWsLayout;
+  using TL = HexTcLayout;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  const float* W1 = W;
+  const float* b1 = W1 + kHexH * IN;
+  const float* W2g = b1 + kHexH;
+  const float* b2 = W2g + kHexH * kHexH;
+  const float* W3g = b2 + kHexH;
+  const float* b3 = W3g + kHexHead * kHexH;
+  float* slot = ws + (size_t)blockIdx.x * slot_stride(n_params);
+  const uint32_t sbase = tc::smem_u32(sm);
+  const uint32_t bar0 = sbase + Lay::BARS;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::BARS + 8 * kNumWsBars);
+  const float* bias = reinterpret_cast<const float*>(sm + Lay::BIAS);
+  float* bacc = reinterpret_cast<float*>(sm + Lay::BACC);
+  // tiles of this CTA and the samples they pass through the ring
+  const int64_t ntiles = (N + kHexTile - 1) / kHexTile;
+  const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  const uint32_t total = (uint32_t)(my_tiles * NS);
+
+  for (int p = tid; p < n_params; p += kBwThreads) slot[p] = 0.f;
+  stage_w23_at(sm, Lay::W2, Lay::W3, W2g, W3g, tid, kBwThreads);
+  {
+    float* bw = reinterpret_cast<float*>(sm + Lay::BIAS);
+    for (int o = tid; o < kHexH; o += kBwThreads) {
+      bw[o] = __ldg(b1 + o);
+      bw[kHexH + o] = __ldg(b2 + o);
+      bw[2 * kHexH + o] = o < kHexHead ? __ldg(b3 + o) : 0.f;
+    }
+    for (int o = tid; o < 3 * kHexH; o += kBwThreads) bacc[o] = 0.f;
+  }
+  if (warp == kBwProducerWarps) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(kBarFull + s), kBwProducerWarps + kBwConsumers / 32);
+      tc::mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int t = 0; t < kWsTStages; ++t) {
+      tc::mbar_init(bar(kBarReady + t), 1);
+      tc::mbar_init(bar(kBarFree + t), kBwConsumers / 32);
+    }
+    tc::mbar_init(bar(kBarLayer), 1);
+    tc::mbar_init(bar(kBarFinal), 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
+
+  if (warp < kBwProducerWarps) {
+    // ------------------------------ producers ------------------------------
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;" ::: "memory");
+    failed = !bw_stream_latent<2, false>(sm, Lay::ZR, 0, bar(kBarFull), bar(kBarEmpty), latent, nullptr, N, IN, NS,
+                                         total);
+  } else {
+    // ------------------------------ consumers ------------------------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+    const int ct = tid - kBwProducers;                 // 0 .. 255
+    const int row = ct & (kHexTile - 1), half = ct >> 7;
+    const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t col = (uint32_t)(half * 32);
+    const uint32_t L = tmem + 128 * kWsTStages;        // small layers: main | correction
+    const uint32_t RW = tmem;                          // their weight gradients (64-row layout): the ring is idle then
+    // Row m of a 64-row accumulator sits in TMEM lane (m % 16) + 32 (m / 16):
+    // lanes below 16 of warp w hold rows 16 (w % 4) + lane.
+    const int wrow = (warp & 3) * 16 + lid;
+    const bool wrow_ok = lid < 16;
+    const bool issuer = ct == 0;
+    float* sW1 = slot;
+    float* sW2 = sW1 + kHexH * IN + kHexH;
+    float* sW3 = sW2 + kHexH * kHexH + kHexH;
+    const SplitOp T0k = kmajor(sbase + Lay::T0, TL::H_PLANE, kHexH), T0t = mnmajor(sbase + Lay::T0, TL::H_PLANE, kHexH);
+    const SplitOp T1k = kmajor(sbase + Lay::T1, TL::H_PLANE, kHexH), T1t = mnmajor(sbase + Lay::T1, TL::H_PLANE, kHexH);
+    const SplitOp W2k = kmajor(sbase + Lay::W2, TL::S_PLANE, kHexH), W2t = mnmajor(sbase + Lay::W2, TL::S_PLANE, kHexH);
+    const SplitOp W3k = kmajor(sbase + Lay::W3, TL::S_PLANE, kHexH), W3t = mnmajor(sbase + Lay::W3, TL::S_PLANE, kHexH);
+    uint32_t G = 0, lph = 0;
+    // W1 slices of the first two ring samples; wreg then holds the next (sample 2)
+    float wreg[8];
+    for (int s = 0; s < 2; ++s) {
+      load_w1_slice8(W1, IN, s, ct, wreg);
+      store_w1_slice8(sm, Lay::w(s), ct, wreg);
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
+    }
+    load_w1_slice8(W1, IN, 2, ct, wreg);
+
+    // Ring sample g: its MMAs by the issuing lane once its stage is full and its TMEM stage free.
+    auto issue = [&](uint32_t g, auto&& mmas) {
+      const uint32_t s = g & 1, t = g % kWsTStages;
+      bool ok = tc::mbar_wait_bounded(bar(kBarFull + s), (g >> 1) & 1, kWsWait);
+      if (ok && g >= (uint32_t)kWsTStages)
+        ok = tc::mbar_wait_bounded(bar(kBarFree + t), ((g / kWsTStages) - 1) & 1, kWsWait);
+      if (ok) {
+        tc::fence_after_sync();
+        mmas(s, tmem + 128 * t);
+        tc::mma_commit(bar(kBarEmpty + s));
+        tc::mma_commit(bar(kBarReady + t));
+      }
+      return ok;
+    };
+    // After sample g's TMEM stage is read: free it, and put the W1 slice of
+    // sample g + 2 into g's ring stage (g's MMAs are done with it).
+    auto release = [&](uint32_t g) {
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lid == 0) tc::mbar_arrive(bar(kBarFree + g % kWsTStages));
+      if (g + 2 < total) {
+        store_w1_slice8(sm, Lay::w(g & 1), ct, wreg);
+        tc::fence_proxy_async();
+        __syncwarp();
+        if (lid == 0) tc::mbar_arrive(bar(kBarFull + (g & 1)));
+        load_w1_slice8(W1, IN, (int)((g + 3) % (uint32_t)NS), ct, wreg);
+      }
+    };
+
+    for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
+      const int64_t n = tile * kHexTile + row;
+      const bool valid = n < N;
+      float xt[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) hex_normalise(mu, frame, n, hp, xt);
+      // ---- 1. layer 1 again: issue sample k, then add sample k - 1 ----
+      float h1[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h1[i] = 0.f;
+      for (int k = 0; k <= NS && !failed; ++k) {
+        if (k < NS && issuer)
+          failed = !issue(G + k, [&](uint32_t s, uint32_t S) {
+            mma6(S, S + 64, kmajor_zpad(sbase + Lay::z(s), TL::Z_PLANE), kmajor(sbase + Lay::w(s), TL::W_PLANE, kHexC),
+                 kHexC, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+          });
+        __syncwarp();
+        failed = __any_sync(0xffffffffu, failed);
+        if (k >= 1 && !failed) {
+          const uint32_t g = G + k - 1, t = g % kWsTStages;
+          if (!warp_wait(bar(kBarReady + t), (g / kWsTStages) & 1)) {
+            failed = true;
+          } else {
+            tc::fence_after_sync();
+            add_partial(tmem + 128 * t + lane + col, tmem + 128 * t + 64 + lane + col, h1);
+            release(g);
+          }
+        }
+      }
+      G += NS;
+      // ---- 2. h1, h2 and the head ----
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h1[i] = fmaxf(h1[i] + bias[half * 32 + i], 0.f);
+      store_row32(sm, Lay::T0, row, half, h1);
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kBwConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      if (issuer) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, T0k, W2k, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, false));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      uint32_t m2 = 0;   // bit i: h2 column half * 32 + i is positive
+      {
+        float h2[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h2[i] = 0.f;
+        if (!failed) add_partial(L + lane + col, L + 64 + lane + col, h2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          h2[i] = fmaxf(h2[i] + bias[kHexH + half * 32 + i], 0.f);
+          m2 |= (h2[i] > 0.f ? 1u : 0u) << i;
+        }
+        store_row32(sm, Lay::T1, row, half, h2);
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kBwConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      // head rows 0..15 (d_mu, d_q, d_logs); with the energy-flow window all
+      // 64 (d loss / d w needs the SH offsets too)
+      if (issuer) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, T1k, W3k, kHexH, tc::idesc_bf16_f32(kHexTile, GATED ? kHexH : 16, false, false));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      // ---- 3. head adjoint ----
+      float dy[32];
+      float gw = 1.0f, gh = 1.0f, gt = 0.0f;
+      float2 gcr = make_float2(0.f, 0.f);
+      if constexpr (GATED) {
+        if (valid) hex_window(hp, frame, n, gw, gh, gt, gcr);
+      }
+      float dldw = 0.0f;   // d loss / d w: this thread's part of the w-scaled offsets (window only)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dy[i] = 0.f;
+      // this thread's head outputs: columns half * 32 .. (the first 16 of half 0 without the window)
+      constexpr int HC = GATED ? 32 : 16;
+      float y[HC];
+      if (GATED || half == 0) {
+#pragma unroll
+        for (int h = 0; h < HC / 16; ++h) {
+          float a[16], c[16];
+          tc::tmem_ld16x2(L + lane + col + 16 * h, L + 64 + lane + col + 16 * h, a, c);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[16 * h + i] = a[i] + c[i] + bias[2 * kHexH + half * 32 + 16 * h + i];
+        }
+      }
+      if (half == 0) {
+        if (valid && !failed) {
+          float qh[4], q[4], s[3], gc[6], ds[3], dq[4], dqh[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) qh[i] = __ldg(q_can + 4 * n + i) + y[3 + i];
+          const float nrm = normalise_quat(qh, q);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) s[i] = expf(__ldg(logs_can + 3 * n + i) + gw * y[7 + i]);
+#pragma unroll
+          for (int i = 0; i < 6; ++i) gc[i] = g_or0(go.cov, 6 * n + i);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) ds[i] = g_or0(go.scale, 3 * n + i);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dq[i] = g_or0(go.rot, 4 * n + i);
+          covariance_backward(s, q, gc, ds, dq);
+          normalise_quat_backward(q, nrm, dq, dqh);
+#pragma unroll
+          for (int i = 0; i < 3; ++i) dy[i] = gh != 0.0f ? g_or0(go.mu, 3 * n + i) : 0.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dy[3 + i] = dqh[i];
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const float dl = ds[i] * s[i];   // d loss / d(log s + w d_logs)
+            dy[7 + i] = gw * dl;
+            if constexpr (GATED) dldw += dl * y[7 + i];
+          }
+#pragma unroll
+          for (int i = 10; i < 32; ++i) {
+            const float g = g_or0(go.sh, 48 * n + (i - 10));
+            dy[i] = gw * g;
+            if constexpr (GATED) dldw += g * y[i];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float g = (valid && i < kHexHead - 32) ? g_or0(go.sh, 48 * n + 22 + i) : 0.f;
+          dy[i] = gw * g;
+          if constexpr (GATED) {
+            if (i < kHexHead - 32) dldw += g * y[i];
+          }
+        }
+        if constexpr (GATED) reinterpret_cast<float*>(sm + Lay::GSUM)[row] = dldw;
+      }
+      tc::fence_before_sync();
+      store_row32(sm, Lay::T0, row, half, dy);
+      atomicAdd(bacc + 2 * kHexH + half * 32 + lid, warp_column_sum(dy));
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kBwConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      if (GATED && half == 0 && valid && hp.gate_grad) {
+        // H(w) is piecewise constant: c and r receive gradient through w alone
+        float gcr_out[2];
+        temporal_gate_backward(gt, gcr.x, gcr.y, hp.gate_tau, dldw + reinterpret_cast<const float*>(sm + Lay::GSUM)[row],
+                               gcr_out);
+        float2* dst = reinterpret_cast<float2*>(hp.gate_grad) + n;
+        const float2 prev = *dst;
+        *dst = make_float2(prev.x + gcr_out[0], prev.y + gcr_out[1]);
+      }
+      // ---- 4. dh2 = (dy W3) * [h2 > 0], dW3 = dy^T h2 ----
+      if (issuer) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, T0k, W3t, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, true));
+        mma6(RW, RW + 64, T0t, T1t, kHexTile, tc::idesc_bf16_f32(64, kHexH, true, true));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      {
+        float d[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] = 0.f;
+        if (!failed) add_partial(L + lane + col, L + 64 + lane + col, d);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] = (m2 >> i) & 1u ? d[i] : 0.f;
+        {
+          float a[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = 0.f;
+          if (!failed) add_partial(RW + lane + col, RW + 64 + lane + col, a);
+          if (!failed && wrow_ok && wrow < kHexHead) slot_add32(sW3 + wrow * kHexH + half * 32, a);
+        }
+        tc::fence_before_sync();
+        store_row32(sm, Lay::T0, row, half, d);
+        store_row32(sm, Lay::T1, row, half, h1);
+        atomicAdd(bacc + kHexH + half * 32 + lid, warp_column_sum(d));
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      if (role_sync_or(2, kBwConsumers, failed)) {
+        failed = true;
+        break;
+      }
+      // ---- 5. dh1 = (dh2 W2) * [h1 > 0], dW2 = dh2^T h1 ----
+      if (issuer) {
+        tc::fence_after_sync();
+        mma6(L, L + 64, T0k, W2t, kHexH, tc::idesc_bf16_f32(kHexTile, kHexH, false, true));
+        mma6(RW, RW + 64, T0t, T1t, kHexTile, tc::idesc_bf16_f32(64, kHexH, true, true));
+        tc::mma_commit(bar(kBarLayer));
+      }
+      __syncwarp();
+      failed = !warp_wait(bar(kBarLayer), lph);
+      lph ^= 1u;
+      tc::fence_after_sync();
+      {
+        float d[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] = 0.f;
+        if (!failed) add_partial(L + lane + col, L + 64 + lane + col, d);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] = h1[i] > 0.f ? d[i] : 0.f;
+        {
+          float a[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = 0.f;
+          if (!failed) add_partial(RW + lane + col, RW + 64 + lane + col, a);
+          if (!failed && wrow_ok) slot_add32(sW2 + wrow * kHexH + half * 32, a);
+        }
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(dh1_out + n * kHexH + half * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]);
+        }
+        atomicAdd(bacc + half * 32 + lid, warp_column_sum(d));
+      }
+      // the weight-gradient columns (ring stage 0) are read before the next tile's MMAs
+      tc::fence_before_sync();
+      if (role_sync_or(2, kBwConsumers, failed)) {
+        failed = true;
+        break;
+      }
+    }
+    // every MMA this CTA issued is complete before the tensor memory goes
+    if (issuer) {
+      tc::mma_commit(bar(kBarFinal));
+      tc::mbar_wait_bounded(bar(kBarFinal), 0, kWsWait);
+    }
+  }
+
+  if (failed) atomicExch(&g_hex_device_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!failed) {
+    float* sb1 = slot + kHexH * IN;
+    float* sb2 = sb1 + kHexH + kHexH * kHexH;
+    float* sb3 = sb2 + kHexH + kHexHead * kHexH;
+    for (int o = tid; o < kHexH; o += kBwThreads) {
+      sb1[o] += bacc[o];
+      sb2[o] += bacc[kHexH + o];
+      if (o < kHexHead) sb3[o] += bacc[2 * kHexH + o];
+    }
+  }
+  if (warp == kBwProducerWarps) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// Kernel B, the W1 pass of the backward from a saved latent: per tile, T0 =
+// dh1 (from kernel A), then per plane sample k the split MMAs
+//   dz_k [128 x 32]  = dh1 W1_k        (TMEM stage columns 0..63)
+//   dW1_k [64 x 32]  = dh1^T z_k       (columns 64..127, 64-row layout)
+// Roles: 4 producer warps write z_k and the W1 slice into the three-stage
+// ring; one issuer warp issues each sample's MMAs as soon as its ring stage
+// is full and its TMEM stage (of four) free, so the tensor core runs up to
+// four samples ahead; 8 consumer warps take dz_k and dW1_k out of TMEM,
+// scatter w_c dz_k to the plane gradients by bulk reductions and add dW1_k to
+// the CTA's workspace slot (zeroed by kernel A, which ran first on the same
+// grid).  The consumers write T0 for the next tile once they have taken out
+// every sample of the last one, and announce it on the T0 barrier.
+__global__ void __launch_bounds__(kDzThreads, 1) hexplane_bwd_dz_ws_kernel(
+    HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
+    const float* __restrict__ W1, const float* __restrict__ latent, const float* __restrict__ dh1,
+    float* __restrict__ grad_planes, float* __restrict__ ws, int n_params) {
+  using Lay = HexDzWsLayout;
+  using TL = HexTcLayout;
+  constexpr int S = Lay::STAGES, TS = Lay::TSTAGES;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+  const int IN = hp.in_dim, NS = hp.n_samples;
+  float* sW1 = ws + (size_t)blockIdx.x * slot_stride(n_params);
+  const uint32_t sbase = tc::smem_u32(sm);
+  const uint32_t bar0 = sbase + Lay::BARS;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::BARS + 8 * kNumDzBars);
+  const int64_t ntiles = (N + kHexTile - 1) / kHexTile;
+  const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  const uint32_t total = (uint32_t)(my_tiles * NS);
+
+  if (warp == kDzIssuerWarp) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(bar(kDzFull + s), kBwProducerWarps);
+      tc::mbar_init(bar(kDzEmpty + s), 1);
+    }
+    for (int t = 0; t < TS; ++t) {
+      tc::mbar_init(bar(kDzReady + t), 1);
+      tc::mbar_init(bar(kDzFree + t), kBwConsumers / 32);
+    }
+    tc::mbar_init(bar(kDzT0), kBwConsumers / 32);
+    tc::mbar_init(bar(kDzFinal), 1);
+    tc::mbar_fence_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
+
+  if (warp < kBwProducerWarps) {
+    // ------------------------------ producers ------------------------------
+    failed = !bw_stream_latent<S, true>(sm, Lay::ZR, Lay::WR, bar(kDzFull), bar(kDzEmpty), latent, W1, N, IN, NS,
+                                        total);
+  } else if (warp == kDzIssuerWarp) {
+    // -------------------------------- issuer --------------------------------
+    if (lid == 0) {
+      const SplitOp T0k = kmajor(sbase + Lay::T0, TL::H_PLANE, kHexH);
+      const SplitOp T0t = mnmajor(sbase + Lay::T0, TL::H_PLANE, kHexH);
+      uint32_t g = 0;
+      for (int64_t i = 0; i < my_tiles && !failed; ++i) {
+        if (!tc::mbar_wait_bounded(bar(kDzT0), (uint32_t)i & 1u, kWsWait)) {
+          failed = true;
+          break;
+        }
+        for (int k = 0; k < NS; ++k, ++g) {
+          const uint32_t s = g % S, t = g % TS;
+          bool ok = tc::mbar_wait_bounded(bar(kDzFull + s), (g / S) & 1, kWsWait);
+          if (ok && g >= (uint32_t)TS) ok = tc::mbar_wait_bounded(bar(kDzFree + t), ((g / TS) - 1) & 1, kWsWait);
+          if (!ok) {
+            failed = true;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t D = tmem + 128 * t;
+          mma6(D, D + 32, T0k, mnmajor(sbase + Lay::w(s), TL::W_PLANE, kHexC), kHexH,
+               tc::idesc_bf16_f32(kHexTile, kHexC, false, true));
+          mma6(D + 64, D + 96, T0t, mnmajor_zpad(sbase + Lay::z(s), TL::Z_PLANE), kHexTile,
+               tc::idesc_bf16_f32(64, kHexC, true, true));
+          tc::mma_commit(bar(kDzEmpty + s));
+          tc::mma_commit(bar(kDzReady + t));
+        }
+      }
+      // every MMA this CTA issued is complete before the tensor memory goes
+      tc::mma_commit(bar(kDzFinal));
+      tc::mbar_wait_bounded(bar(kDzFinal), 0, kWsWait);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------ consumers ------------------------------
+    const int ct = tid - kBwProducers;                 // 0 .. 255
+    const int row = ct & (kHexTile - 1), half = ct >> 7;
+    const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+    // Row m of a 64-row accumulator sits in TMEM lane (m % 16) + 32 (m / 16):
+    // lanes below 16 of warp w hold rows 16 (w % 4) + lane.
+    const int wrow = (warp & 3) * 16 + lid;
+    const bool wrow_ok = lid < 16;
+    uint8_t* rows = sm + Lay::SCAT + row * Lay::SCAT_ROW;
+    // this thread's half row of the next tile's dh1
+    float dn[32];
+    auto load_dh1 = [&](int64_t tile) {
+      const int64_t n = tile * kHexTile + row;
+      const bool ok = n < N;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = ok ? __ldg(reinterpret_cast<const float4*>(dh1 + n * kHexH + half * 32) + q)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        dn[4 * q] = v.x;
+        dn[4 * q + 1] = v.y;
+        dn[4 * q + 2] = v.z;
+        dn[4 * q + 3] = v.w;
+      }
+    };
+    uint32_t g = 0;
+    load_dh1(blockIdx.x);
+    for (int64_t tile = blockIdx.x; tile * kHexTile < N && !failed; tile += gridDim.x) {
+      const int64_t n = tile * kHexTile + row;
+      const bool valid = n < N;
+      float xt[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) hex_normalise(mu, frame, n, hp, xt);
+      // T0 = dh1 of this tile: this warp has taken out every sample of the
+      // last tile, so their MMAs, the last readers of T0, are done
+      store_row32(sm, Lay::T0, row, half, dn);
+      if ((tile + gridDim.x) * kHexTile < N) load_dh1(tile + gridDim.x);
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lid == 0) tc::mbar_arrive(bar(kDzT0));
+      for (int k = 0; k < NS; ++k, ++g) {
+        const uint32_t t = g % TS;
+        const uint32_t D = tmem + 128 * t;
+        if (!warp_wait(bar(kDzReady + t), (g / TS) & 1)) {
+          failed = true;
+          break;
+        }
+        tc::fence_after_sync();
+        float dz[32], wa[16], wc[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {   // both threads of a Gaussian read its whole dz row
+          float a[16], c[16];
+          tc::tmem_ld16x2(D + lane + 16 * h, D + 32 + lane + 16 * h, a, c);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) dz[16 * h + i] = a[i] + c[i];
+        }
+        tc::tmem_ld16x2(D + 64 + lane + half * 16, D + 96 + lane + half * 16, wa, wc);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lid == 0) tc::mbar_arrive(bar(kDzFree + t));
+        if (wrow_ok) {   // this thread alone updates these slot elements: see slot_add32
+          float4* dst = reinterpret_cast<float4*>(sW1 + (size_t)wrow * IN + k * kHexC + half * 16);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            atomicAdd(dst + q, make_float4(wa[4 * q] + wc[4 * q], wa[4 * q + 1] + wc[4 * q + 1],
+                                           wa[4 * q + 2] + wc[4 * q + 2], wa[4 * q + 3] + wc[4 * q + 3]));
+        }
+        if (valid) {
+          // corners 2 half and 2 half + 1 are neighbouring cells along the
+          // plane's first axis, so their gradient rows are contiguous: w_c dz
+          // is staged as those two 128-byte rows and added with one bulk
+          // reduction
+          const PlaneSample ps = plane_sample(xt, hp, k);
+          bulk_wait_read();   // this thread's rows of the previous sample have been read
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const float w = half ? (cc ? ps.w11 : ps.w10) : (cc ? ps.w01 : ps.w00);
+            float4* d = reinterpret_cast<float4*>(rows + (2 * half + cc) * (kHexC * 4));
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d[q] = make_float4(w * dz[4 * q], w * dz[4 * q + 1], w * dz[4 * q + 2], w * dz[4 * q + 3]);
+          }
+          tc::fence_proxy_async();
+          bulk_add_2rows(grad_planes + (half ? ps.o10 : ps.o00), tc::smem_u32(rows + 2 * half * (kHexC * 4)));
+          bulk_commit();
+        }
+      }
+    }
+    bulk_wait_all();
+  }
+
+  if (failed) atomicExch(&g_hex_device_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kDzIssuerWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
@@ -1772,9 +2488,22 @@ extern "C" int spin4d_hexplane_fwd_gated(const spin4d_hexplane_desc* h, const fl
                            "spin4d_hexplane_fwd_gated");
 }
 
+namespace spin4d {
+// Workspace: the per-block weight-gradient slots, then (from a 256-byte
+// boundary) N x 64 fp32 for dh1 between the two kernels of the backward from
+// a saved latent.
+static size_t hex_slots_bytes(const spin4d_hexplane_desc* h, int64_t N) {
+  const size_t b = (size_t)hex_bwd_blocks(N) * slot_stride((int)spin4d_hexplane_param_count(h)) * sizeof(float);
+  return (b + 255) & ~(size_t)255;
+}
+static float* hex_dh1_buffer(void* workspace, int64_t N, const spin4d_hexplane_desc* h) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + hex_slots_bytes(h, N));
+}
+}  // namespace spin4d
+
 extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, int64_t N) {
   if (validate_hex(h) != SPIN4D_OK || N <= 0) return 0;
-  return (size_t)hex_bwd_blocks(N) * slot_stride((int)spin4d_hexplane_param_count(h)) * sizeof(float);
+  return hex_slots_bytes(h, N) + (size_t)N * kHexH * sizeof(float);
 }
 
 static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
@@ -1805,12 +2534,29 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     const int smem = HexBwdLayout::BYTES;
     if (!configured[dev]) {
       bool ok = true;
-      for (auto* kern : {hexplane_bwd_tc_kernel<false, false>, hexplane_bwd_tc_kernel<true, false>,
-                         hexplane_bwd_tc_kernel<false, true>, hexplane_bwd_tc_kernel<true, true>}) {
+      for (auto* kern : {hexplane_bwd_tc_kernel<false>, hexplane_bwd_tc_kernel<true>}) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e);
         int occ = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kHexThreads, smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        ok = ok && occ == 1;
+      }
+      for (auto* kern : {hexplane_bwd_head_ws_kernel<false>, hexplane_bwd_head_ws_kernel<true>}) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, HexBwWsLayout::BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        int occ = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kBwThreads, HexBwWsLayout::BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        ok = ok && occ == 1;
+      }
+      {
+        cudaError_t e = cudaFuncSetAttribute(hexplane_bwd_dz_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             HexDzWsLayout::BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        int occ = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hexplane_bwd_dz_ws_kernel, kDzThreads,
+                                                          HexDzWsLayout::BYTES);
         if (e != cudaSuccess) return cuda_status(e);
         ok = ok && occ == 1;
       }
@@ -1819,10 +2565,20 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     }
     if (usable[dev]) {
       blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
-      auto* kern = gate ? (latent ? hexplane_bwd_tc_kernel<true, true> : hexplane_bwd_tc_kernel<false, true>)
-                        : (latent ? hexplane_bwd_tc_kernel<true, false> : hexplane_bwd_tc_kernel<false, false>);
-      kern<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, latent, go, grad_planes,
-                                             static_cast<float*>(workspace), n_params);
+      if (latent) {
+        // from the saved latent: warp-specialised, the head then the W1 pass
+        float* dh1 = hex_dh1_buffer(workspace, N, h);
+        auto* kern = gate ? hexplane_bwd_head_ws_kernel<true> : hexplane_bwd_head_ws_kernel<false>;
+        kern<<<blocks, kBwThreads, HexBwWsLayout::BYTES, s>>>(p, mu, frame, N, weights, q_can, logs_can, latent, go, dh1,
+                                                               static_cast<float*>(workspace), n_params);
+        SPIN4D_CHECK(launch_status());
+        hexplane_bwd_dz_ws_kernel<<<blocks, kDzThreads, HexDzWsLayout::BYTES, s>>>(
+            p, mu, frame, N, weights, latent, dh1, grad_planes, static_cast<float*>(workspace), n_params);
+      } else {
+        auto* kern = gate ? hexplane_bwd_tc_kernel<true> : hexplane_bwd_tc_kernel<false>;
+        kern<<<blocks, kHexThreads, smem, s>>>(p, mu, frame, N, planes, weights, q_can, logs_can, go, grad_planes,
+                                               static_cast<float*>(workspace), n_params);
+      }
       SPIN4D_CHECK(launch_status());
     }
   }

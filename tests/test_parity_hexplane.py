@@ -93,8 +93,11 @@ def test_hexplane_bwd_matches_oracle(sp, n):
     _check_grads(hx, gp, gw, wp, ww, tol.FP32_GRAD_RTOL, mag.hexplane_rss(inp, planes, weights, hx, grads))
 
 
-def test_hexplane_bwd_from_saved_latent_matches_oracle(sp):
-    n = 2001
+@pytest.mark.parametrize("n", [1, 129, 2001, 40_000])
+def test_hexplane_bwd_from_saved_latent_matches_oracle(sp, n):
+    """From the forward's saved latent: one Gaussian, a ragged second tile,
+    several tiles, and more tiles than SMs (the persistent CTAs run two, so
+    the sample ring carries across tiles)."""
     hx, inp, planes, weights = _inputs(n, 0.5, seed=1)
     grads = S.upstream_grads(n, S.HEX_OUT_WIDTHS, 1.0, seed=5)
     h = sp.hex_from_spec(hx)

@@ -805,15 +805,25 @@ def run_workloads(args):
     emit("hexplane_fp32", "fwd", n, ms, plane_lines_per_gaussian=lines,
          frac_of_l2_random_line_ceiling=lines * n / (ms * 1e-3) / ceil["l2_random_line128_per_s"])
     out_l = dict(out, latent=lat)
+    hid = torch.empty((n, hx.hidden), device=dev)
+    out_h = dict(out_l, hidden=hid)
 
     def hfb():
         sp.hexplane_fwd(h, inp, planes, weights, out=out_l)
         sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws, latent=lat)
 
+    def hfb_h1():
+        sp.hexplane_fwd(h, inp, planes, weights, out=out_h)
+        sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws, latent=lat, hidden=hid)
+
     emit("hexplane_fp32", "fwd+bwd (saved latent)", n, timed(hfb, 10))
+    emit("hexplane_fp32", "fwd+bwd (saved latent and h1)", n, timed(hfb_h1, 10))
+    emit("hexplane_fp32", "bwd (saved latent and h1)", n,
+         timed(lambda: sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws, latent=lat, hidden=hid),
+               10))
     emit("hexplane_fp32", "bwd (gathering again)", n,
          timed(lambda: sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, workspace=ws), 10))
-    del inp, planes, weights, out, lat, grads, gp, gw, ws, out_l
+    del inp, planes, weights, out, lat, grads, gp, gw, ws, out_l, hid, out_h
     torch.cuda.empty_cache()
     render_workloads(sp, torch, dev, timed)
     sp.check_device_errors()
@@ -1085,9 +1095,10 @@ def run_ncu_case(name):
         gw = torch.zeros(hx.n_params(), device=dev)
         out = {k: torch.empty((n, wd), device=dev) for k, wd in sp.HEX_KEYS}
         out["latent"] = torch.empty((n, hx.in_dim), device=dev)
-        for _ in range(3):   # a training step: forward saving the latent, backward reading it
+        out["hidden"] = torch.empty((n, hx.hidden), device=dev)
+        for _ in range(3):   # a training step: forward saving the latent and h1, backward reading them
             sp.hexplane_fwd(h, inp, planes, weights, out=out)
-            sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, latent=out["latent"])
+            sp.hexplane_bwd(h, inp, planes, weights, grads, gp, gw, latent=out["latent"], hidden=out["hidden"])
     else:
         grid, mlp = w["grid"], w["mlp"]
         g, m = sp.grid_from_spec(grid), sp.mlp_from_spec(mlp)

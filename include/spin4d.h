@@ -304,7 +304,10 @@ int64_t spin4d_hexplane_param_count(const spin4d_hexplane_desc* h);
 
 /* Deformed Gaussians: mu' N x 3, rot N x 4, scale N x 3, sh N x 48, cov N x 6 (fp32).
  * latent (optional, may be NULL): N x (n_scales*6*channels) fp32, 32-byte
- * aligned, receives the concatenated plane samples. */
+ * aligned, receives the concatenated plane samples.
+ * hidden (optional, may be NULL): N x hidden fp32, 16-byte aligned, receives
+ * the first trunk layer's output h1 = relu(W1 z + b1).  Saved beside the
+ * latent, it spares the backward the first layer (spin4d_hexplane_bwd_saved). */
 typedef struct spin4d_hex_outputs {
     float* mu;
     float* rot;
@@ -312,6 +315,7 @@ typedef struct spin4d_hex_outputs {
     float* sh;
     float* cov;
     float* latent;
+    float* hidden;
 } spin4d_hex_outputs;
 
 typedef struct spin4d_hex_output_grads {
@@ -399,6 +403,31 @@ int spin4d_hexplane_bwd_gated(const spin4d_hexplane_desc* h, const float* mu, co
                               const float* q_can, const float* logs_can, const float* sh_can,
                               const float* latent, const spin4d_hex_gate* gate,
                               const spin4d_hex_output_grads* grad_out,
+                              float* grad_planes, float* grad_weights,
+                              void* workspace, size_t ws_bytes, spin4d_stream_t stream);
+
+/* The forward's saved activations for spin4d_hexplane_bwd_saved: latent as
+ * in spin4d_hex_outputs (required), hidden the matching h1 (NULL: the
+ * backward computes h1 again from the latent). */
+typedef struct spin4d_hex_saved {
+    const float* latent;
+    const float* hidden;
+} spin4d_hex_saved;
+
+/*
+ * spin4d_hexplane_bwd (gate NULL) or spin4d_hexplane_bwd_gated (gate given)
+ * from the forward's saved latent and, when saved->hidden is given, its
+ * saved h1: the backward then starts at the second layer.  The results and
+ * every other argument are those of the two calls.  SPIN4D_ERR_INVALID for
+ * a NULL saved or saved->latent, a misaligned saved->hidden (16 bytes) or a
+ * bad gate; SPIN4D_ERR_UNSUPPORTED where only the fp32 SIMT kernels could
+ * run.  The saved arrays must come from a forward with the same inputs,
+ * planes and weights (and window): they are not checked.
+ */
+int spin4d_hexplane_bwd_saved(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                              int64_t N, const float* planes, const float* weights,
+                              const float* q_can, const float* logs_can, const spin4d_hex_saved* saved,
+                              const spin4d_hex_gate* gate, const spin4d_hex_output_grads* grad_out,
                               float* grad_planes, float* grad_weights,
                               void* workspace, size_t ws_bytes, spin4d_stream_t stream);
 

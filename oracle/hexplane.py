@@ -155,10 +155,11 @@ def forward(inp: Dict[str, np.ndarray], planes, weights, hx, gate=None) -> Dict[
     xt = normalise(inp["mu"], inp["frame"], hx.n_frames)
     z = encode(xt, planes, hx)
     layers = decoder.unpack_layers(weights, hx.layer_shapes())
-    y, _, _ = decoder.mlp_forward(z, layers)
+    y, acts, _ = decoder.mlp_forward(z, layers)
     w = _window(xt, hx, gate)
     out, _ = _outputs(y, inp, w)
     out["z"] = z
+    out["h1"] = acts[1]   # the first hidden layer, relu(W1 z + b1)
     if w is not None:
         out["w"] = w
     return out

@@ -921,7 +921,8 @@ __device__ __forceinline__ void store_w1_slice(uint8_t* sm, int off, int c, cons
 __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ planes, const float* __restrict__ W, const float* __restrict__ q_can,
-    const float* __restrict__ logs_can, const float* __restrict__ sh_can, HexOutPtrs out, float* __restrict__ latent) {
+    const float* __restrict__ logs_can, const float* __restrict__ sh_can, HexOutPtrs out, float* __restrict__ latent,
+    float* __restrict__ hidden) {
   using Lay = HexWsLayout;
   extern __shared__ __align__(1024) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
@@ -1148,6 +1149,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
         for (int i = 0; i < 64; ++i) acc[i] = fmaxf(acc[i] + bias[i], 0.f);
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) store_split8(sm, Lay::H, HexTcLayout::H_PLANE, c, kc, kHexH, acc + 8 * kc);
+        if (hidden && valid) {
+          float4* dst = reinterpret_cast<float4*>(hidden + n * kHexH);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+        }
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();
@@ -1612,8 +1618,9 @@ constexpr int kBwProducerWarps = 4;
 constexpr int kBwProducers = 32 * kBwProducerWarps;
 constexpr int kBwConsumers = 2 * kHexTile;
 constexpr int kBwThreads = kBwProducers + kBwConsumers;
-static_assert(kBwProducerWarps == 4 && 4 * 32 * 152 + 8 * 32 * 176 == kBwThreads * 168,
-              "the register split must equal the launch's total");
+static_assert(kBwProducerWarps == 4 && 4 * 32 * 152 + 8 * 32 * 176 == kBwThreads * 168 &&
+                  4 * 32 * 56 + 8 * 32 * 224 == kBwThreads * 168,
+              "the register splits must equal the launch's total");
 
 // Kernel A: z ring | W1 ring | T0 | T1 | W2 | W3 | biases and sums.
 struct HexBwWsLayout {
@@ -1759,12 +1766,12 @@ __device__ __forceinline__ bool bw_stream_latent(uint8_t* sm, int zring, int wri
 // dh1 = (dh2 W2) * [h1 > 0] with dW2 = dh2^T h1; it writes dh1 to dh1_out
 // (N x 64) and adds the weight and bias gradients of W2, W3 and the biases to
 // the CTA's workspace slot, which it zeroes first.
-template <bool GATED>
+template <bool GATED, bool HIDDEN>
 __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
     const float* __restrict__ W, const float* __restrict__ q_can, const float* __restrict__ logs_can,
-    const float* __restrict__ latent, HexGradPtrs go, float* __restrict__ dh1_out, float* __restrict__ ws,
-    int n_params) {
+    const float* __restrict__ latent, const float* __restrict__ hidden, HexGradPtrs go, float* __restrict__ dh1_out,
+    float* __restrict__ ws, int n_params) {
   using Lay = HexBwWsLayout;
   using TL = HexTcLayout;
   extern __shared__ __align__(1024) uint8_t sm[];
@@ -1825,12 +1832,21 @@ __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
 
   if (warp < kBwProducerWarps) {
     // ------------------------------ producers ------------------------------
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;" ::: "memory");
-    failed = !bw_stream_latent<2, false>(sm, Lay::ZR, 0, bar(kBarFull), bar(kBarEmpty), latent, nullptr, N, IN, NS,
-                                         total);
+    // with the saved h1 the producers have nothing to do: their registers go
+    // to the consumers (4 x 32 x 56 + 8 x 32 x 224 = 384 x 168)
+    if constexpr (HIDDEN)
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 152;" ::: "memory");
+    if constexpr (!HIDDEN)
+      failed = !bw_stream_latent<2, false>(sm, Lay::ZR, 0, bar(kBarFull), bar(kBarEmpty), latent, nullptr, N, IN, NS,
+                                           total);
   } else {
     // ------------------------------ consumers ------------------------------
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+    if constexpr (HIDDEN)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    else
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
     const int ct = tid - kBwProducers;                 // 0 .. 255
     const int row = ct & (kHexTile - 1), half = ct >> 7;
     const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
@@ -1852,14 +1868,33 @@ __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
     uint32_t G = 0, lph = 0;
     // W1 slices of the first two ring samples; wreg then holds the next (sample 2)
     float wreg[8];
-    for (int s = 0; s < 2; ++s) {
-      load_w1_slice8(W1, IN, s, ct, wreg);
-      store_w1_slice8(sm, Lay::w(s), ct, wreg);
-      tc::fence_proxy_async();
-      __syncwarp();
-      if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
+    if constexpr (!HIDDEN) {
+      for (int s = 0; s < 2; ++s) {
+        load_w1_slice8(W1, IN, s, ct, wreg);
+        store_w1_slice8(sm, Lay::w(s), ct, wreg);
+        tc::fence_proxy_async();
+        __syncwarp();
+        if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
+      }
+      load_w1_slice8(W1, IN, 2, ct, wreg);
     }
-    load_w1_slice8(W1, IN, 2, ct, wreg);
+    // with the saved h1: this thread's half row of the next tile's
+    float hn[HIDDEN ? 32 : 1];
+    auto load_h1 = [&](int64_t tile) {
+      if constexpr (HIDDEN) {
+        const int64_t m = tile * kHexTile + row;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = m < N ? __ldg(reinterpret_cast<const float4*>(hidden + m * kHexH + half * 32) + q)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          hn[4 * q] = v.x;
+          hn[4 * q + 1] = v.y;
+          hn[4 * q + 2] = v.z;
+          hn[4 * q + 3] = v.w;
+        }
+      }
+    };
+    load_h1(blockIdx.x);
 
     // Ring sample g: its MMAs by the issuing lane once its stage is full and its TMEM stage free.
     auto issue = [&](uint32_t g, auto&& mmas) {
@@ -1895,11 +1930,16 @@ __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
       const bool valid = n < N;
       float xt[4] = {0.f, 0.f, 0.f, 0.f};
       if (valid) hex_normalise(mu, frame, n, hp, xt);
-      // ---- 1. layer 1 again: issue sample k, then add sample k - 1 ----
+      // ---- 1. layer 1 again (or the saved h1): issue sample k, then add sample k - 1 ----
       float h1[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) h1[i] = 0.f;
-      for (int k = 0; k <= NS && !failed; ++k) {
+      if constexpr (HIDDEN) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h1[i] = hn[i];
+        if ((tile + gridDim.x) * kHexTile < N) load_h1(tile + gridDim.x);
+      }
+      for (int k = 0; !HIDDEN && k <= NS && !failed; ++k) {
         if (k < NS && issuer)
           failed = !issue(G + k, [&](uint32_t s, uint32_t S) {
             mma6(S, S + 64, kmajor_zpad(sbase + Lay::z(s), TL::Z_PLANE), kmajor(sbase + Lay::w(s), TL::W_PLANE, kHexC),
@@ -1920,8 +1960,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
       }
       G += NS;
       // ---- 2. h1, h2 and the head ----
+      if constexpr (!HIDDEN) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) h1[i] = fmaxf(h1[i] + bias[half * 32 + i], 0.f);
+        for (int i = 0; i < 32; ++i) h1[i] = fmaxf(h1[i] + bias[half * 32 + i], 0.f);
+      }
       store_row32(sm, Lay::T0, row, half, h1);
       tc::fence_proxy_async();
       tc::fence_before_sync();
@@ -2439,6 +2481,7 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
   if (!sh_can || !out.mu || !out.rot || !out.scale || !out.sh || !out.cov || !aligned(out.rot, 16))
     return SPIN4D_ERR_INVALID;
   if (out.latent && !aligned(out.latent, 32)) return SPIN4D_ERR_INVALID;
+  if (out.hidden && !aligned(out.hidden, 16)) return SPIN4D_ERR_INVALID;
   if (gate) SPIN4D_CHECK(hex_gate_check(gate, false));
   if (fault_injected(name)) return SPIN4D_ERR_INJECTED;
   HexParams p = make_hex_params(h);
@@ -2461,7 +2504,8 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
     }
     const int blocks = persistent_blocks((N + kHexTile - 1) / kHexTile, 1);
     hexplane_fwd_ws_kernel<<<blocks, kWsThreads, smem, (cudaStream_t)stream>>>(p, mu, frame, N, planes, weights, q_can,
-                                                                             logs_can, sh_can, o, out.latent);
+                                                                             logs_can, sh_can, o, out.latent,
+                                                                             out.hidden);
     return launch_status();
   }
   if (gate) return SPIN4D_ERR_UNSUPPORTED;   // the window is built into the tensor-core kernels only
@@ -2508,14 +2552,15 @@ extern "C" size_t spin4d_hexplane_bwd_workspace(const spin4d_hexplane_desc* h, i
 
 static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame, int64_t N,
                              const float* planes, const float* weights, const float* q_can, const float* logs_can,
-                             const float* latent, const spin4d_hex_gate* gate, const spin4d_hex_output_grads* grad_out,
-                             float* grad_planes, float* grad_weights, void* workspace, size_t ws_bytes,
-                             spin4d_stream_t stream, const char* name) {
+                             const float* latent, const float* hidden, const spin4d_hex_gate* gate,
+                             const spin4d_hex_output_grads* grad_out, float* grad_planes, float* grad_weights,
+                             void* workspace, size_t ws_bytes, spin4d_stream_t stream, const char* name) {
   SPIN4D_CHECK(hex_check(h, mu, frame, N, planes, weights, q_can, logs_can));
   if (N == 0) return SPIN4D_OK;
   if (!grad_out || !grad_planes || !grad_weights || !workspace) return SPIN4D_ERR_INVALID;
   if (!aligned(grad_planes, 16) || !aligned(grad_weights, 4) || !aligned(workspace, 256)) return SPIN4D_ERR_INVALID;
   if (latent && !aligned(latent, 32)) return SPIN4D_ERR_INVALID;
+  if (hidden && (!latent || !aligned(hidden, 16))) return SPIN4D_ERR_INVALID;
   if (ws_bytes < spin4d_hexplane_bwd_workspace(h, N)) return SPIN4D_ERR_INVALID;
   if (gate) SPIN4D_CHECK(hex_gate_check(gate, true));
   if (fault_injected(name)) return SPIN4D_ERR_INJECTED;
@@ -2542,7 +2587,8 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
         if (e != cudaSuccess) return cuda_status(e);
         ok = ok && occ == 1;
       }
-      for (auto* kern : {hexplane_bwd_head_ws_kernel<false>, hexplane_bwd_head_ws_kernel<true>}) {
+      for (auto* kern : {hexplane_bwd_head_ws_kernel<false, false>, hexplane_bwd_head_ws_kernel<true, false>,
+                         hexplane_bwd_head_ws_kernel<false, true>, hexplane_bwd_head_ws_kernel<true, true>}) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, HexBwWsLayout::BYTES);
         if (e != cudaSuccess) return cuda_status(e);
         int occ = 0;
@@ -2568,9 +2614,10 @@ static int hexplane_bwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
       if (latent) {
         // from the saved latent: warp-specialised, the head then the W1 pass
         float* dh1 = hex_dh1_buffer(workspace, N, h);
-        auto* kern = gate ? hexplane_bwd_head_ws_kernel<true> : hexplane_bwd_head_ws_kernel<false>;
-        kern<<<blocks, kBwThreads, HexBwWsLayout::BYTES, s>>>(p, mu, frame, N, weights, q_can, logs_can, latent, go, dh1,
-                                                               static_cast<float*>(workspace), n_params);
+        auto* kern = gate ? (hidden ? hexplane_bwd_head_ws_kernel<true, true> : hexplane_bwd_head_ws_kernel<true, false>)
+                          : (hidden ? hexplane_bwd_head_ws_kernel<false, true> : hexplane_bwd_head_ws_kernel<false, false>);
+        kern<<<blocks, kBwThreads, HexBwWsLayout::BYTES, s>>>(p, mu, frame, N, weights, q_can, logs_can, latent, hidden,
+                                                               go, dh1, static_cast<float*>(workspace), n_params);
         SPIN4D_CHECK(launch_status());
         hexplane_bwd_dz_ws_kernel<<<blocks, kDzThreads, HexDzWsLayout::BYTES, s>>>(
             p, mu, frame, N, weights, latent, dh1, grad_planes, static_cast<float*>(workspace), n_params);
@@ -2604,8 +2651,8 @@ extern "C" int spin4d_hexplane_bwd(const spin4d_hexplane_desc* h, const float* m
                                    const spin4d_hex_output_grads* grad_out, float* grad_planes,
                                    float* grad_weights, void* workspace, size_t ws_bytes, spin4d_stream_t stream) {
   (void)sh_can;   // sh' = sh_can + d_sh: the upstream sh gradient flows through unchanged
-  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, nullptr, grad_out, grad_planes,
-                           grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd");
+  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, nullptr, nullptr, grad_out,
+                           grad_planes, grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd");
 }
 
 extern "C" int spin4d_hexplane_bwd_gated(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
@@ -2616,6 +2663,18 @@ extern "C" int spin4d_hexplane_bwd_gated(const spin4d_hexplane_desc* h, const fl
                                          spin4d_stream_t stream) {
   (void)sh_can;
   if (!gate) return SPIN4D_ERR_INVALID;
-  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, gate, grad_out, grad_planes,
-                           grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd_gated");
+  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, latent, nullptr, gate, grad_out,
+                           grad_planes, grad_weights, workspace, ws_bytes, stream, "spin4d_hexplane_bwd_gated");
+}
+
+extern "C" int spin4d_hexplane_bwd_saved(const spin4d_hexplane_desc* h, const float* mu, const int32_t* frame,
+                                         int64_t N, const float* planes, const float* weights, const float* q_can,
+                                         const float* logs_can, const spin4d_hex_saved* saved,
+                                         const spin4d_hex_gate* gate, const spin4d_hex_output_grads* grad_out,
+                                         float* grad_planes, float* grad_weights, void* workspace, size_t ws_bytes,
+                                         spin4d_stream_t stream) {
+  if (!saved || !saved->latent) return SPIN4D_ERR_INVALID;
+  return hexplane_bwd_impl(h, mu, frame, N, planes, weights, q_can, logs_can, saved->latent, saved->hidden, gate,
+                           grad_out, grad_planes, grad_weights, workspace, ws_bytes, stream,
+                           "spin4d_hexplane_bwd_saved");
 }

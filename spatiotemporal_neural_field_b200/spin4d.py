@@ -64,7 +64,12 @@ class HexDesc(ctypes.Structure):
 
 
 class HexOutputs(ctypes.Structure):
-    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp), ("latent", c_vp)]
+    _fields_ = [("mu", c_vp), ("rot", c_vp), ("scale", c_vp), ("sh", c_vp), ("cov", c_vp), ("latent", c_vp),
+                ("hidden", c_vp)]
+
+
+class HexSaved(ctypes.Structure):
+    _fields_ = [("latent", c_vp), ("hidden", c_vp)]
 
 
 class HexOutputGrads(ctypes.Structure):
@@ -135,6 +140,8 @@ _SIGS = {
     "spin4d_hexplane_fwd_gated": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, P(HexGate),
                                           HexOutputs, c_vp]),
     "spin4d_hexplane_bwd_gated": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                          P(HexGate), P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "spin4d_hexplane_bwd_saved": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, P(HexSaved),
                                           P(HexGate), P(HexOutputGrads), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "spin4d_hexplane_bwd_workspace": (c_sz, [P(HexDesc), c_i64]),
     "spin4d_hexplane_bwd": (c_i32, [P(HexDesc), c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
@@ -425,7 +432,7 @@ def hexplane_fwd(h: HexDesc, inp: Dict[str, torch.Tensor], planes, weights, out=
     N = inp["mu"].shape[0]
     if out is None:
         out = {k: torch.empty((N, w), dtype=torch.float32, device=planes.device) for k, w in HEX_KEYS}
-    o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS), _ptr(out.get("latent")))
+    o = HexOutputs(*(_ptr(out[k]) for k, _ in HEX_KEYS), _ptr(out.get("latent")), _ptr(out.get("hidden")))
     common = (ctypes.byref(h), _ptr(inp["mu"]), _ptr(inp["frame"]), N, _ptr(planes), _ptr(weights),
               _ptr(inp["q_can"]), _ptr(inp["logs_can"]), _ptr(inp["sh_can"]))
     if gate_cr is None:
@@ -443,9 +450,11 @@ def hexplane_bwd_workspace(h: HexDesc, N: int) -> int:
 
 def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weights, workspace=None, latent=None,
                  stream=None, gate_cr: Optional[torch.Tensor] = None, tau: float = 0.02,
-                 grad_cr: Optional[torch.Tensor] = None):
+                 grad_cr: Optional[torch.Tensor] = None, hidden: Optional[torch.Tensor] = None):
     """With ``gate_cr`` the backward of the windowed deformation
-    (spin4d_hexplane_bwd_gated); ``grad_cr`` (N x 2) += d loss / d(c, r)."""
+    (spin4d_hexplane_bwd_gated); ``grad_cr`` (N x 2) += d loss / d(c, r).
+    ``hidden`` (the forward's saved h1, with ``latent``) selects
+    spin4d_hexplane_bwd_saved."""
     N = inp["mu"].shape[0]
     if workspace is None:
         workspace = torch.empty(max(hexplane_bwd_workspace(h, N), 1), dtype=torch.uint8, device=planes.device)
@@ -454,10 +463,15 @@ def hexplane_bwd(h: HexDesc, inp, planes, weights, grads, grad_planes, grad_weig
               _ptr(inp["q_can"]), _ptr(inp["logs_can"]), _ptr(inp["sh_can"]), _ptr(latent))
     tail = (ctypes.byref(go), _ptr(grad_planes), _ptr(grad_weights), _ptr(workspace), workspace.numel(),
             _stream(stream))
-    if gate_cr is None:
+    gate = None if gate_cr is None else HexGate(_ptr(gate_cr), tau, _ptr(grad_cr))
+    if hidden is not None:
+        saved = HexSaved(_ptr(latent), _ptr(hidden))
+        _check("spin4d_hexplane_bwd_saved",
+               lib.spin4d_hexplane_bwd_saved(*common[:-2], ctypes.byref(saved),
+                                             ctypes.byref(gate) if gate is not None else None, *tail))
+    elif gate is None:
         _check("spin4d_hexplane_bwd", lib.spin4d_hexplane_bwd(*common, *tail))
     else:
-        gate = HexGate(_ptr(gate_cr), tau, _ptr(grad_cr))
         _check("spin4d_hexplane_bwd_gated", lib.spin4d_hexplane_bwd_gated(*common, ctypes.byref(gate), *tail))
 
 

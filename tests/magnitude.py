@@ -288,6 +288,17 @@ def _hex_forward(inp, planes, weights, hx):
     return xt, layers, y, pres, macts, my
 
 
+def hexplane_hidden_mag(inp, planes, weights, hx):
+    """Magnitude for h1 = relu(W1 z + b1): that of its pre-activation's terms,
+    sqrt(|z|^2 (W1^2)^T + b1^2), on both sides of zero, since
+    |relu(a) - relu(b)| <= |a - b| holds where the rounding of W1 z + b1
+    carries it across."""
+    xt = hp.normalise(inp["mu"], inp["frame"], hx.n_frames)
+    z = hp.encode(xt, planes, hx)
+    W, b = dec.unpack_layers(weights, hx.layer_shapes())[0]
+    return np.sqrt((z * z) @ (W * W).T + b * b)
+
+
 def _hex_window(xt, hx, gate, n):
     """(w, H(w)) of the energy-flow window, ones without one."""
     if gate is None:

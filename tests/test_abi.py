@@ -192,6 +192,16 @@ def test_unsupported_hexplane_shape(sp):
     go = sp.HexOutputGrads()
     assert lib.spin4d_hexplane_bwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4,
                                    ctypes.byref(go), FAKE, FAKE, FAKE, 1 << 40, None) == sp.ERR_INVALID
+    # the saved activations: none, no latent, a misaligned h1
+    def saved(x):
+        return lib.spin4d_hexplane_bwd_saved(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, x, None,
+                                             ctypes.byref(go), FAKE, FAKE, FAKE, 1 << 40, None)
+    assert saved(None) == sp.ERR_INVALID
+    assert saved(ctypes.byref(sp.HexSaved(None, FAKE))) == sp.ERR_INVALID
+    assert saved(ctypes.byref(sp.HexSaved(FAKE, FAKE + 4))) == sp.ERR_INVALID
+    # a misaligned saved h1 in the forward
+    assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE + 4), None) == sp.ERR_INVALID
 
 
 def test_fault_injection_hook_in_subprocess(sp):

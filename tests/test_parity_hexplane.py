@@ -93,22 +93,45 @@ def test_hexplane_bwd_matches_oracle(sp, n):
     _check_grads(hx, gp, gw, wp, ww, tol.FP32_GRAD_RTOL, mag.hexplane_rss(inp, planes, weights, hx, grads))
 
 
+@pytest.mark.parametrize("saved_h1", [False, True])
 @pytest.mark.parametrize("n", [1, 129, 2001, 40_000])
-def test_hexplane_bwd_from_saved_latent_matches_oracle(sp, n):
-    """From the forward's saved latent: one Gaussian, a ragged second tile,
-    several tiles, and more tiles than SMs (the persistent CTAs run two, so
-    the sample ring carries across tiles)."""
+def test_hexplane_bwd_from_saved_latent_matches_oracle(sp, n, saved_h1):
+    """From the forward's saved latent (and its saved h1): one Gaussian, a
+    ragged second tile, several tiles, and more tiles than SMs (the
+    persistent CTAs run two, so the sample ring carries across tiles)."""
     hx, inp, planes, weights = _inputs(n, 0.5, seed=1)
     grads = S.upstream_grads(n, S.HEX_OUT_WIDTHS, 1.0, seed=5)
     h = sp.hex_from_spec(hx)
     I, P, W = {k: dev(v) for k, v in inp.items()}, dev(planes), dev(weights)
     out = {k: torch.empty((n, w), dtype=torch.float32, device="cuda") for k, w in sp.HEX_KEYS}
     out["latent"] = torch.empty((n, hx.in_dim), dtype=torch.float32, device="cuda")
+    if saved_h1:
+        out["hidden"] = torch.empty((n, hx.hidden), dtype=torch.float32, device="cuda")
     sp.hexplane_fwd(h, I, P, W, out=out)
     gp, gw = _zero_grads(hx)
-    sp.hexplane_bwd(h, I, P, W, {k: dev(v) for k, v in grads.items()}, gp, gw, latent=out["latent"])
+    sp.hexplane_bwd(h, I, P, W, {k: dev(v) for k, v in grads.items()}, gp, gw, latent=out["latent"],
+                    hidden=out.get("hidden"))
     wp, ww = hp.backward(inp, planes, weights, hx, grads)
     _check_grads(hx, gp, gw, wp, ww, tol.FP32_GRAD_RTOL, mag.hexplane_rss(inp, planes, weights, hx, grads))
+
+
+@pytest.mark.parametrize("n", [129, 3001])
+def test_hexplane_fwd_saved_h1_matches_oracle(sp, n):
+    """The forward's saved first hidden layer, relu(W1 z + b1), element-wise
+    against the oracle's (the magnitude of its pre-activation's terms where
+    it is positive); the other outputs are unchanged by saving it."""
+    hx, inp, planes, weights = _inputs(n, 0.5, seed=4)
+    h = sp.hex_from_spec(hx)
+    I, P, W = {k: dev(v) for k, v in inp.items()}, dev(planes), dev(weights)
+    out = {k: torch.empty((n, w), dtype=torch.float32, device="cuda") for k, w in sp.HEX_KEYS}
+    out["hidden"] = torch.empty((n, hx.hidden), dtype=torch.float32, device="cuda")
+    sp.hexplane_fwd(h, I, P, W, out=out)
+    want = hp.forward(inp, planes, weights, hx)
+    tol.elementwise(host(out["hidden"]), want["h1"], tol.FP32_RTOL, "h1", tol.column_groups(hx.hidden),
+                    rho=mag.hexplane_hidden_mag(inp, planes, weights, hx))
+    plain = sp.hexplane_fwd(h, I, P, W)
+    for k, _ in sp.HEX_KEYS:
+        assert torch.equal(plain[k], out[k]), k
 
 
 def test_hexplane_bwd_partial_upstream(sp):
@@ -156,6 +179,12 @@ def test_hexplane_bwd_full_batch_halves_latent_and_sample(sp):
     sp.hexplane_bwd(h, I, P, W, G, gp3, gw3, latent=out["latent"])
     tol.normwise(host(gp3), host(gp), 1e-4, "planes: saved latent vs gather", tol.plane_groups(hx))
     tol.normwise(host(gw3), host(gw), 1e-4, "weights: saved latent vs gather", tol.weight_blocks(hx.layer_shapes()))
+    out["hidden"] = torch.empty((n, hx.hidden), dtype=torch.float32, device="cuda")
+    sp.hexplane_fwd(h, I, P, W, out=out)
+    gp5, gw5 = _zero_grads(hx)
+    sp.hexplane_bwd(h, I, P, W, G, gp5, gw5, latent=out["latent"], hidden=out["hidden"])
+    tol.normwise(host(gp5), host(gp), 1e-4, "planes: saved h1 vs gather", tol.plane_groups(hx))
+    tol.normwise(host(gw5), host(gw), 1e-4, "weights: saved h1 vs gather", tol.weight_blocks(hx.layer_shapes()))
     rows = np.sort(np.random.default_rng(6).choice(n, 2000, replace=False))
     rows[-1] = n - 1
     sub_inp = {k: v[rows] for k, v in inp.items()}
@@ -243,6 +272,14 @@ def test_hexplane_gated_bwd_matches_oracle(sp, n):
     first = gcr.clone()
     sp.hexplane_bwd(h, I, P, W, G, gp2, gw2, latent=out["latent"], gate_cr=dev(cr), tau=TAU, grad_cr=gcr)
     _gated_bwd_check(hx, inp, planes, weights, grads, cr, gp2, gw2, gcr - first)
+    # and the saved latent with the saved h1
+    out["hidden"] = torch.empty((n, hx.hidden), dtype=torch.float32, device="cuda")
+    sp.hexplane_fwd(h, I, P, W, out=out, gate_cr=dev(cr), tau=TAU)
+    gp3, gw3 = _zero_grads(hx)
+    second = gcr.clone()
+    sp.hexplane_bwd(h, I, P, W, G, gp3, gw3, latent=out["latent"], hidden=out["hidden"], gate_cr=dev(cr), tau=TAU,
+                    grad_cr=gcr)
+    _gated_bwd_check(hx, inp, planes, weights, grads, cr, gp3, gw3, gcr - second)
 
 
 def test_hexplane_gated_full_size_sampled(sp):

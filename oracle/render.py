@@ -255,6 +255,104 @@ def composite_pixel(px: float, py: float, pr, order, st: Settings):
     return rgb, Tb_k[-1], idx, a_k, Tb_k[:-1], ok, ok and gok
 
 
+def _blend(px: float, py: float, pr, order, st: Settings, flip_cover=None, flip_alpha_min=None, stop_at=None,
+           swap=None):
+    """Colour and final transmittance of one pixel, decided as in
+    composite_pixel except for one forced change: the 3-sigma test
+    (flip_cover) or the alpha_min test (flip_alpha_min) of the Gaussian at that
+    position of ``order`` taken the other way; blending that stops after
+    exactly ``stop_at`` blending Gaussians; or the Gaussians at the two
+    positions ``swap`` of ``order`` exchanged."""
+    if swap is not None:
+        order = np.array(order, copy=True)
+        order[swap[0]], order[swap[1]] = order[swap[1]], order[swap[0]]
+    m = pr["mean2d"][order]
+    q = pr["conic"][order]
+    o = pr["opacity"][order]
+    dx, dy = px - m[:, 0], py - m[:, 1]
+    d2 = q[:, 0] * dx * dx + 2.0 * q[:, 1] * dx * dy + q[:, 2] * dy * dy
+    cover = d2 <= SUPPORT_D2
+    a = np.minimum(o * np.exp(-0.5 * d2), st.alpha_max)
+    passes = a >= st.alpha_min
+    if flip_cover is not None:
+        cover[flip_cover] = not cover[flip_cover]
+    if flip_alpha_min is not None:
+        passes[flip_alpha_min] = not passes[flip_alpha_min]
+    pos = np.flatnonzero(cover & passes)
+    ab = a[pos]
+    Tb = np.concatenate([[1.0], np.cumprod(1.0 - ab)])
+    k = len(pos)
+    if stop_at is not None:
+        k = min(stop_at, len(pos))
+    elif st.t_stop > 0:
+        stop = np.flatnonzero(Tb[1:] < st.t_stop)
+        if stop.size:
+            k = int(stop[0])
+    idx = order[pos[:k]]
+    rgb = (pr["rgb"][idx] * (ab[:k] * Tb[:k])[:, None]).sum(axis=0) + Tb[k] * np.asarray(st.background, np.float64)
+    return rgb, Tb[k]
+
+
+def pixel_flip_bound(px: float, py: float, pr, order, st: Settings):
+    """How far fp32 rounding can move one pixel: the sum, over the decisions
+    that composite_pixel finds within their margins, of the change in colour
+    (3) and final transmittance that taking that one decision the other way
+    makes (each computed by _blend).  Zero for a pixel clear of every margin.
+    Two decisions taken the other way together change the pixel by the sum of
+    their changes up to a product of two of the (small) alphas involved."""
+    base_rgb, base_T, _, _, _, ok, _ = composite_pixel(px, py, pr, order, st)
+    if ok:
+        return np.zeros(3), 0.0
+    m = pr["mean2d"][order]
+    q = pr["conic"][order]
+    o = pr["opacity"][order]
+    dx, dy = px - m[:, 0], py - m[:, 1]
+    d2 = q[:, 0] * dx * dx + 2.0 * q[:, 1] * dx * dy + q[:, 2] * dy * dy
+    cover = d2 <= SUPPORT_D2
+    a = np.minimum(o * np.exp(-0.5 * d2), st.alpha_max)
+    pos = np.flatnonzero(cover & (a >= st.alpha_min))
+    Tb = np.concatenate([[1.0], np.cumprod(1.0 - a[pos])])
+    k, n_eval = len(pos), len(order)
+    if st.t_stop > 0:
+        stop = np.flatnonzero(Tb[1:] < st.t_stop)
+        if stop.size:
+            k = int(stop[0])
+            n_eval = int(pos[k]) + 1
+    alts = []
+    edge_matters = o * math.exp(-0.5 * SUPPORT_D2) >= st.alpha_min * (1.0 - REL_MARGIN)
+    for g in np.flatnonzero((np.abs(d2[:n_eval] - SUPPORT_D2) < D2_MARGIN) & edge_matters[:n_eval]):
+        alts.append(_blend(px, py, pr, order, st, flip_cover=int(g)))
+    if st.alpha_min > 0:
+        near = cover[:n_eval] & (np.abs(a[:n_eval] - st.alpha_min) < REL_MARGIN * st.alpha_min)
+        for g in np.flatnonzero(near):
+            alts.append(_blend(px, py, pr, order, st, flip_alpha_min=int(g)))
+    if st.t_stop > 0:
+        for i in range(min(k + 1, len(pos))):
+            if abs(Tb[i + 1] - st.t_stop) < REL_MARGIN * st.t_stop:
+                # stopping before blending Gaussian i, or blending it too
+                alts.append(_blend(px, py, pr, order, st, stop_at=i if i < k else k + 1))
+    z = pr["depth"][order[pos[:k]]]
+    for i in np.flatnonzero(np.diff(z) < DEPTH_MARGIN * z[1:]) if z.size > 1 else []:
+        alts.append(_blend(px, py, pr, order, st, swap=(int(pos[i]), int(pos[i + 1]))))
+    rgb_b, T_b = np.zeros(3), 0.0
+    for rgb, T in alts:
+        rgb_b += np.abs(rgb - base_rgb)
+        T_b += abs(T - base_T)
+    return rgb_b, T_b
+
+
+def render_flip_bounds(cam: Camera, st: Settings, mu, cov6, opacity, colours, pixels: np.ndarray):
+    """pixel_flip_bound for the listed pixels (k x 2 integer (column, row)):
+    (k x 3 colour bounds, k transmittance bounds)."""
+    pr = project(cam, st, mu, cov6, opacity, colours)
+    order = _depth_order(pr)
+    rgb = np.zeros((len(pixels), 3))
+    T = np.zeros(len(pixels))
+    for k, (i, j) in enumerate(np.asarray(pixels)):
+        rgb[k], T[k] = pixel_flip_bound(i + 0.5, j + 0.5, pr, order, st)
+    return rgb, T
+
+
 def render_pixels(cam: Camera, st: Settings, mu, cov6, opacity, colours, pixels: np.ndarray):
     """Colour (k x 3), final transmittance (k) and margin flags (k) of the
     listed pixels (k x 2 integer (column, row))."""

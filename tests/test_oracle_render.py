@@ -393,3 +393,71 @@ def test_backward_with_clamped_alpha_matches_central_differences():
             flat[p] = old
             fd = (lp - lm) / (2 * h)
             assert abs(got[p] - fd) <= 1e-6 * max(1.0, abs(fd)), (key, p, got[p], fd)
+
+
+# ---------------------------------------------------------------------------
+# the bound on decisions within fp32 reach of their thresholds
+# ---------------------------------------------------------------------------
+def _pr(means, depths, opacities, rgbs, conic=(1.0, 0.0, 1.0)):
+    """A projected scene written out by hand: 2D means, unit conic."""
+    n = len(means)
+    return dict(mean2d=np.asarray(means, np.float64), conic=np.tile(np.asarray(conic, np.float64), (n, 1)),
+                opacity=np.asarray(opacities, np.float64), rgb=np.asarray(rgbs, np.float64),
+                depth=np.asarray(depths, np.float64), visible=np.ones(n, bool))
+
+
+def _bound(pr, st, px=0.5, py=0.5):
+    order = rd._depth_order(pr)
+    return rd.pixel_flip_bound(px, py, pr, order, st)
+
+
+def test_flip_bound_is_zero_on_a_clear_pixel():
+    st = rd.Settings(sh_degree=-1, background=np.zeros(3))
+    pr = _pr([[0.5, 0.5], [1.5, 0.5]], [1.0, 2.0], [0.6, 0.5], [[1, 0, 0], [0, 1, 0]])
+    rgb, T = _bound(pr, st)
+    assert np.all(rgb == 0.0) and T == 0.0
+
+
+def test_flip_bound_of_a_gaussian_on_its_three_sigma_edge():
+    """d^2 = 9 exactly at the pixel: the Gaussian may be dropped, which
+    removes its o e^-4.5 c from the colour and restores the transmittance."""
+    st = rd.Settings(sh_degree=-1, background=np.zeros(3))
+    o, c = 0.8, np.array([0.2, 0.5, 0.9])
+    pr = _pr([[3.5, 0.5]], [1.0], [o], [c])
+    rgb, T = _bound(pr, st)
+    a = o * math.exp(-4.5)
+    assert np.allclose(rgb, a * c, rtol=1e-12) and abs(T - a) < 1e-12
+
+
+def test_flip_bound_of_a_depth_tie():
+    """Two Gaussians at one depth on the pixel: either order may be taken;
+    the orders differ by a_1 a_2 (c_1 - c_2) in colour and not at all in the
+    transmittance."""
+    st = rd.Settings(sh_degree=-1, background=np.zeros(3))
+    c1, c2 = np.array([1.0, 0.0, 0.3]), np.array([0.0, 1.0, 0.3])
+    pr = _pr([[0.5, 0.5], [0.5, 0.5]], [2.0, 2.0], [0.6, 0.3], [c1, c2])
+    rgb, T = _bound(pr, st)
+    assert np.allclose(rgb, 0.6 * 0.3 * np.abs(c1 - c2), rtol=1e-12, atol=1e-15) and T < 1e-15
+
+
+def test_flip_bound_of_the_termination():
+    """One Gaussian that leaves the transmittance exactly at t_stop: blending
+    may stop before it (background, T = 1) instead."""
+    st = rd.Settings(sh_degree=-1, t_stop=0.05, alpha_max=0.99, background=np.array([0.1, 0.2, 0.3]))
+    c = np.array([0.9, 0.4, 0.2])
+    pr = _pr([[0.5, 0.5]], [1.0], [0.95], [c])
+    rgb, T = _bound(pr, st)
+    bg = np.array([0.1, 0.2, 0.3])
+    base = 0.95 * c + 0.05 * bg
+    assert np.allclose(rgb, np.abs(bg - base), rtol=1e-12) and abs(T - 0.95) < 1e-12
+
+
+def test_flip_bound_of_alpha_min():
+    """alpha exactly at alpha_min: the Gaussian may not blend."""
+    st = rd.Settings(sh_degree=-1, alpha_min=1 / 255, background=np.zeros(3))
+    c = np.array([0.3, 0.6, 0.9])
+    pr = _pr([[0.5, 0.5], [0.5, 0.5]], [1.0, 3.0], [1 / 255, 0.5], [c, [1.0, 1.0, 1.0]])
+    rgb, T = _bound(pr, st)
+    a = 1 / 255
+    # with it: a c + (1 - a) 0.5 (1, 1, 1); without it: 0.5 (1, 1, 1)
+    assert np.allclose(rgb, np.abs(a * c - a * 0.5), rtol=1e-12) and abs(T - a * 0.5) < 1e-12

@@ -187,3 +187,24 @@ def column_groups(ncols, labels=None):
 
 RENDER_ATOL = 2e-3
 RENDER_GRAD_RTOL = 1e-2
+# A pixel with decisions within fp32 reach of their thresholds may take any
+# of them the other way; the oracle bounds each single change
+# (oracle/render.py pixel_flip_bound) and several together change the pixel
+# by the sum of their changes up to products of two of the (small) alphas
+# involved, which this factor covers.
+RENDER_FLIP_SLACK = 1.5
+
+
+def absolute_with_bound(got, want, bound, atol, name=""):
+    """|g - o| <= atol + RENDER_FLIP_SLACK * bound element-wise; prints the
+    worst ratio and the number of entries that needed their bound."""
+    g, o = _pair(got, want, name)
+    b = np.asarray(bound, np.float64).reshape(g.shape)
+    err = np.abs(g - o)
+    lim = atol + RENDER_FLIP_SLACK * b
+    ratio = float(np.max(err / lim)) if g.size else 0.0
+    needed = int(np.count_nonzero(err > atol))
+    print("  %-40s worst |g-o|/bound %.3f, %d of %d entries beyond %.1e (within their flip bound)"
+          % (name, ratio, needed, g.size, atol))
+    assert ratio <= 1.0, "%s: |g-o| exceeds its bound by %.3fx" % (name, ratio)
+    return ratio

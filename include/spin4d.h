@@ -331,7 +331,7 @@ typedef struct spin4d_hex_output_grads {
  * s' = exp(logs_can + d_logs); sh' = sh_can + d_sh; Sigma(s', q').
  *   mu N x 3, frame N int32 in [0, n_frames), q_can N x 4, logs_can N x 3,
  *   sh_can N x 48 (all fp32).  planes and weights: device, 32-byte aligned;
- *   out.rot 16-byte aligned.  Misaligned or NULL arguments return
+ *   out.rot, out.sh and sh_can 16-byte aligned.  Misaligned or NULL arguments return
  *   SPIN4D_ERR_INVALID; channels other than 32, hidden other than 64 or
  *   n_hidden other than 2 return SPIN4D_ERR_UNSUPPORTED, before any launch.
  */

@@ -814,19 +814,17 @@ __device__ __forceinline__ void stage_small_layers(uint8_t* sm, int bias_off, co
 // Forward, warp-specialised: the tensor-core form of the layers (bf16x3
 // split products, fresh accumulators per plane sample added in fp32), with
 // the per-sample chain taken apart so that no step waits for the whole CTA:
-//   * 8 producer warps gather the tile's corner rows into registers two plane
-//     samples ahead, interpolate, and write the split z_k into a two-stage
-//     shared-memory ring;
+//   * 8 producer warps gather the tile's corner rows and the sample's W1
+//     slice into registers two plane samples ahead, interpolate, and write
+//     the split z_k and W1 slice into a two-stage shared-memory ring; a ring
+//     stage is full once all 8 have arrived;
 //   * 4 consumer warps (one thread per Gaussian, TMEM lane = row): one lane
 //     issues each sample's split MMAs into a three-stage TMEM ring and
 //     commits them to the stage's "empty" and "ready" barriers; all 128 add
-//     the sample's two accumulators to their fp32 row, free the TMEM stage,
-//     and write the split W1 slice of the sample two ahead into the ring
-//     stage that sample's MMAs just released; after the last sample they run
-//     layers 2 and 3 (through the H tile and TMEM columns 384..511) and
-//     write the outputs, while the producers already gather the next tile.
-//   A ring stage is full once all 8 producer warps and all 4 consumer warps
-//   have arrived.
+//     the sample's two accumulators to their fp32 row and free the TMEM
+//     stage; after the last sample they run layers 2 and 3 (through the H
+//     tile and TMEM columns 384..511) and write the outputs, while the
+//     producers already gather the next tile.
 // Every hand-off is an mbarrier with a bounded wait; the roles' own named
 // barriers reduce a failure flag, so a timed-out wait ends both roles at their
 // next barrier instead of leaving either waiting.
@@ -839,7 +837,7 @@ constexpr int kWsTStages = 3;
 // Polls of one mbarrier before a wait gives up: every legitimate wait here is
 // for work of microseconds (a sample's gather, its MMAs, a tile's epilogue)
 constexpr uint32_t kWsWait = 1u << 20;
-static_assert(2 * 4 * 32 * 176 + 4 * 32 * 152 == kWsThreads * 168, "the register split must equal the launch's total");
+static_assert(2 * 4 * 32 * 184 + 4 * 32 * 136 == kWsThreads * 168, "the register split must equal the launch's total");
 
 // A producer's corner rows of one plane sample: [Gaussian j][corner 00, 01, 10, 11]
 struct CornerRegs {
@@ -917,6 +915,14 @@ __device__ __forceinline__ void store_w1_slice(uint8_t* sm, int off, int c, cons
   store_split8(sm, off, HexTcLayout::W_PLANE, c >> 1, (c & 1) * 2, kHexC, v);
   store_split8(sm, off, HexTcLayout::W_PLANE, c >> 1, (c & 1) * 2 + 1, kHexC, v + 8);
 }
+// One of 256 threads' share of a split W1 slice (64 rows x 32 columns): row
+// c / 4, columns 8 (c % 4) .. + 7.
+__device__ __forceinline__ void load_w1_slice8(const float* __restrict__ W1, int IN, int k, int c, float v[8]) {
+  ld_nc_v8(W1 + (size_t)(c >> 2) * IN + k * kHexC + (c & 3) * 8, v);
+}
+__device__ __forceinline__ void store_w1_slice8(uint8_t* sm, int off, int c, const float v[8]) {
+  store_split8(sm, off, HexTcLayout::W_PLANE, c >> 2, c & 3, kHexC, v);
+}
 
 __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
@@ -967,7 +973,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
   }
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(bar(kBarFull + s), kWsProducerWarps + kWsConsumers / 32);
+      tc::mbar_init(bar(kBarFull + s), kWsProducerWarps);
       tc::mbar_init(bar(kBarEmpty + s), 1);
     }
     for (int t = 0; t < kWsTStages; ++t) {
@@ -987,15 +993,19 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
 
   if (warp < kWsProducerWarps) {
     // ------------------------------ producers ------------------------------
-    // two warpgroups at 176 registers, the consumers' one at 152: together
+    // two warpgroups at 184 registers, the consumers' one at 136: together
     // exactly the 384 x 168 the block was launched with
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
     const int row = tid & (kHexTile - 1), half = tid >> 7;
     const int sub = lid >> 3, c4 = lid & 7;
     uint32_t G = 0;   // samples this CTA has produced so far
     CornerRegs ra, rb;
     int64_t tile0 = 0;
     const uint64_t keep = l2_evict_last();
+    // this thread's part of the W1 slice of the next sample to write, read one sample ahead
+    float wnext[8];
+    int wk = 0;
+    load_w1_slice8(W1, IN, 0, tid, wnext);
     auto prefetch = [&](int k, CornerRegs& r) {
       const int64_t down = (int64_t)hp.res_a[k] * (kHexC / 4);
 #pragma unroll
@@ -1017,6 +1027,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
     auto produce = [&](int k, CornerRegs& r) -> bool {
       const int s = G & 1;
       if (G >= 2 && !warp_wait(bar(kBarEmpty + s), ((G >> 1) + 1) & 1)) return false;
+      store_w1_slice8(sm, Lay::w(s), tid, wnext);   // the slice of sample k
+      wk = wk + 1 == NS ? 0 : wk + 1;
+      load_w1_slice8(W1, IN, wk, tid, wnext);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int g = 16 * warp + 4 * j + sub;
@@ -1075,27 +1088,15 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
     }
   } else {
     // ------------------------------ consumers ------------------------------
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 136;" ::: "memory");
     const int c = tid - kWsProducers;                  // the tile row (Gaussian) and TMEM lane
     const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t L = tmem + 128 * kWsTStages;        // layers 2 and 3: main | correction
     const SplitOp Hk = kmajor(sbase + Lay::H, HexTcLayout::H_PLANE, kHexH);
     uint32_t G = 0, lph = 0;
-    // the first two ring stages' W1 slices (samples 0 and 1 of the first
-    // tile); wreg then holds the next slice to stage (sample 2)
-    float wreg[16];
-    for (int s = 0; s < 2; ++s) {
-      load_w1_slice(W1, IN, s, c, wreg);
-      store_w1_slice(sm, Lay::w(s), c, wreg);
-      tc::fence_proxy_async();
-      __syncwarp();
-      if (lid == 0) tc::mbar_arrive(bar(kBarFull + s));
-    }
-    load_w1_slice(W1, IN, 2 % NS, c, wreg);
     for (int64_t tile = blockIdx.x; tile * kHexTile < N; tile += gridDim.x) {
       const int64_t n = tile * kHexTile + c;
       const bool valid = n < N;
-      const bool has_next = (tile + gridDim.x) * kHexTile < N;
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
@@ -1129,16 +1130,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
             tc::fence_before_sync();
             __syncwarp();
             if (lid == 0) tc::mbar_arrive(bar(kBarFree + t));
-            // sample g's MMAs are done, so its ring stage is free: it takes the
-            // W1 slice of sample g + 2 (this tile's k + 1, or the next tile's first two)
-            if (k + 1 < NS || has_next) {
-              const int s2 = (int)(g & 1);
-              store_w1_slice(sm, Lay::w(s2), c, wreg);   // the slice of sample index (k + 1) % NS
-              tc::fence_proxy_async();
-              __syncwarp();
-              if (lid == 0) tc::mbar_arrive(bar(kBarFull + s2));
-              load_w1_slice(W1, IN, (k + 2) % NS, c, wreg);
-            }
           }
         }
       }
@@ -1225,9 +1216,19 @@ __global__ void __launch_bounds__(kWsThreads, 1) hexplane_fwd_ws_kernel(
         for (int i = 0; i < 3; ++i) st_hint(out.scale + 3 * n + i, s[i], once);
 #pragma unroll
         for (int i = 0; i < 6; ++i) st_hint(out.cov + 6 * n + i, cov[i], once);
+        // the 48 SH offsets as 16-byte vectors (sh_can and out.sh are 16-byte aligned)
+        const float4* shc = reinterpret_cast<const float4*>(sh_can + 48 * n);
+        float* sho = out.sh + 48 * n;
+        static_assert(kHexHead - 10 == 48, "48 SH coefficients");
 #pragma unroll
-        for (int i = 0; i < kHexHead - 10; ++i)
-          st_hint(out.sh + 48 * n + i, ld_nc_hint(sh_can + 48 * n + i, once) + gw * y[10 + i], once);
+        for (int q = 0; q < 12; ++q) {
+          float4 v = ld_nc_v4_hint(shc + q, once);
+          v.x += gw * y[10 + 4 * q];
+          v.y += gw * y[11 + 4 * q];
+          v.z += gw * y[12 + 4 * q];
+          v.w += gw * y[13 + 4 * q];
+          st_v4_stream(sho + 4 * q, v, once);
+        }
       }
     }
     // every MMA this CTA issued is complete before the tensor memory goes
@@ -1649,14 +1650,6 @@ __device__ __forceinline__ SplitOp mnmajor_zpad(uint32_t base, int plane) {
   return {base, (uint32_t)plane, 128u, (uint32_t)kZChunk, 256u};
 }
 
-// One of 256 threads' share of a split W1 slice (64 rows x 32 columns): row
-// c / 4, columns 8 (c % 4) .. + 7.
-__device__ __forceinline__ void load_w1_slice8(const float* __restrict__ W1, int IN, int k, int c, float v[8]) {
-  ld_nc_v8(W1 + (size_t)(c >> 2) * IN + k * kHexC + (c & 3) * 8, v);
-}
-__device__ __forceinline__ void store_w1_slice8(uint8_t* sm, int off, int c, const float v[8]) {
-  store_split8(sm, off, HexTcLayout::W_PLANE, c >> 2, c & 3, kHexC, v);
-}
 
 // W2 and W3 split (W3 padded with zero rows to 64) by threads t of nt.
 __device__ __forceinline__ void stage_w23_at(uint8_t* sm, int w2, int w3, const float* __restrict__ W2g,
@@ -2478,7 +2471,8 @@ static int hexplane_fwd_impl(const spin4d_hexplane_desc* h, const float* mu, con
                              spin4d_stream_t stream, const char* name) {
   SPIN4D_CHECK(hex_check(h, mu, frame, N, planes, weights, q_can, logs_can));
   if (N == 0) return SPIN4D_OK;
-  if (!sh_can || !out.mu || !out.rot || !out.scale || !out.sh || !out.cov || !aligned(out.rot, 16))
+  if (!sh_can || !out.mu || !out.rot || !out.scale || !out.sh || !out.cov || !aligned(out.rot, 16) ||
+      !aligned(sh_can, 16) || !aligned(out.sh, 16))
     return SPIN4D_ERR_INVALID;
   if (out.latent && !aligned(out.latent, 32)) return SPIN4D_ERR_INVALID;
   if (out.hidden && !aligned(out.hidden, 16)) return SPIN4D_ERR_INVALID;

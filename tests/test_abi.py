@@ -199,6 +199,11 @@ def test_unsupported_hexplane_shape(sp):
     assert saved(None) == sp.ERR_INVALID
     assert saved(ctypes.byref(sp.HexSaved(None, FAKE))) == sp.ERR_INVALID
     assert saved(ctypes.byref(sp.HexSaved(FAKE, FAKE + 4))) == sp.ERR_INVALID
+    # misaligned SH rows in the forward (canonical or output)
+    assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE + 4,
+                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None, None), None) == sp.ERR_INVALID
+    assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   sp.HexOutputs(FAKE, FAKE, FAKE, FAKE + 4, FAKE, None, None), None) == sp.ERR_INVALID
     # a misaligned saved h1 in the forward
     assert lib.spin4d_hexplane_fwd(ctypes.byref(h), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE,
                                    sp.HexOutputs(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE + 4), None) == sp.ERR_INVALID

@@ -1670,8 +1670,8 @@ __device__ __forceinline__ void stage_w23_at(uint8_t* sm, int w2, int w3, const 
 
 
 // Kernel B: 3 z stages | 3 W1 stages | T0 (dh1) | scatter staging | barriers.
-constexpr int kDzIssuerWarp = kBwProducerWarps + kBwConsumers / 32;   // warp 12
-constexpr int kDzThreads = 32 * (kDzIssuerWarp + 1);
+constexpr int kDzIssuerWarp = kBwProducerWarps + kBwConsumers / 32;   // warps 12 (dz) and 13 (dW1)
+constexpr int kDzThreads = 32 * (kDzIssuerWarp + 2);
 struct HexDzWsLayout {
   static constexpr int STAGES = 3;
   static constexpr int TSTAGES = 4;
@@ -2193,12 +2193,13 @@ __global__ void __launch_bounds__(kBwThreads, 1) hexplane_bwd_head_ws_kernel(
 //   dz_k [128 x 32]  = dh1 W1_k        (TMEM stage columns 0..63)
 //   dW1_k [64 x 32]  = dh1^T z_k       (columns 64..127, 64-row layout)
 // Roles: 4 producer warps write z_k and the W1 slice into the three-stage
-// ring; one issuer warp issues each sample's MMAs as soon as its ring stage
-// is full and its TMEM stage (of four) free, so the tensor core runs up to
-// four samples ahead; 8 consumer warps take dz_k and dW1_k out of TMEM,
-// scatter w_c dz_k to the plane gradients by bulk reductions and add dW1_k to
-// the CTA's workspace slot (zeroed by kernel A, which ran first on the same
-// grid).  The consumers write T0 for the next tile once they have taken out
+// ring; two issuer warps (the dz products and the dW1 products, so that the
+// single-thread issue of 72 small MMAs per sample is shared) issue each
+// sample's MMAs as soon as its ring stage is full and its TMEM stage (of
+// four) free, so the tensor core runs up to four samples ahead; 8 consumer
+// warps take dz_k and dW1_k out of TMEM, scatter w_c dz_k to the plane
+// gradients by bulk reductions and add dW1_k to the CTA's workspace slot
+// (zeroed by kernel A, which ran first on the same grid).  The consumers write T0 for the next tile once they have taken out
 // every sample of the last one, and announce it on the T0 barrier.
 __global__ void __launch_bounds__(kDzThreads, 1) hexplane_bwd_dz_ws_kernel(
     HexParams hp, const float* __restrict__ mu, const int32_t* __restrict__ frame, int64_t N,
@@ -2226,14 +2227,14 @@ __global__ void __launch_bounds__(kDzThreads, 1) hexplane_bwd_dz_ws_kernel(
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(bar(kDzFull + s), kBwProducerWarps);
-      tc::mbar_init(bar(kDzEmpty + s), 1);
+      tc::mbar_init(bar(kDzEmpty + s), 2);   // both issuers commit
     }
     for (int t = 0; t < TS; ++t) {
-      tc::mbar_init(bar(kDzReady + t), 1);
+      tc::mbar_init(bar(kDzReady + t), 2);
       tc::mbar_init(bar(kDzFree + t), kBwConsumers / 32);
     }
     tc::mbar_init(bar(kDzT0), kBwConsumers / 32);
-    tc::mbar_init(bar(kDzFinal), 1);
+    tc::mbar_init(bar(kDzFinal), 2);
     tc::mbar_fence_init();
   }
   tc::fence_before_sync();
@@ -2246,8 +2247,11 @@ __global__ void __launch_bounds__(kDzThreads, 1) hexplane_bwd_dz_ws_kernel(
     // ------------------------------ producers ------------------------------
     failed = !bw_stream_latent<S, true>(sm, Lay::ZR, Lay::WR, bar(kDzFull), bar(kDzEmpty), latent, W1, N, IN, NS,
                                         total);
-  } else if (warp == kDzIssuerWarp) {
-    // -------------------------------- issuer --------------------------------
+  } else if (warp >= kDzIssuerWarp) {
+    // ------------------------------- issuers -------------------------------
+    // One lane of each issuer warp: warp 12 issues the dz products, warp 13
+    // the dW1 products, and each commits its own to the stage's barriers (a
+    // commit tracks the MMAs its thread issued).
     if (lid == 0) {
       const SplitOp T0k = kmajor(sbase + Lay::T0, TL::H_PLANE, kHexH);
       const SplitOp T0t = mnmajor(sbase + Lay::T0, TL::H_PLANE, kHexH);
@@ -2267,10 +2271,12 @@ __global__ void __launch_bounds__(kDzThreads, 1) hexplane_bwd_dz_ws_kernel(
           }
           tc::fence_after_sync();
           const uint32_t D = tmem + 128 * t;
-          mma6(D, D + 32, T0k, mnmajor(sbase + Lay::w(s), TL::W_PLANE, kHexC), kHexH,
-               tc::idesc_bf16_f32(kHexTile, kHexC, false, true));
-          mma6(D + 64, D + 96, T0t, mnmajor_zpad(sbase + Lay::z(s), TL::Z_PLANE), kHexTile,
-               tc::idesc_bf16_f32(64, kHexC, true, true));
+          if (warp == kDzIssuerWarp)
+            mma6(D, D + 32, T0k, mnmajor(sbase + Lay::w(s), TL::W_PLANE, kHexC), kHexH,
+                 tc::idesc_bf16_f32(kHexTile, kHexC, false, true));
+          else
+            mma6(D + 64, D + 96, T0t, mnmajor_zpad(sbase + Lay::z(s), TL::Z_PLANE), kHexTile,
+                 tc::idesc_bf16_f32(64, kHexC, true, true));
           tc::mma_commit(bar(kDzEmpty + s));
           tc::mma_commit(bar(kDzReady + t));
         }

@@ -289,3 +289,19 @@ def test_l2_window_arguments_rejected_on_host(sp):
     assert sp.lib.spin4d_l2_window_set(1, None, 1 << 20, ctypes.byref(applied)) == sp.ERR_INVALID
     assert sp.lib.spin4d_l2_window_set(1, 1 << 20, 0, ctypes.byref(applied)) == sp.ERR_INVALID
     assert sp.lib.spin4d_l2_window_clear(None) == sp.ERR_INVALID
+
+
+def test_hexplane_empty_batch_is_a_no_op(sp):
+    """N = 0 returns success before any pointer is looked at or any launch,
+    for the forward and every backward entry point."""
+    lib = sp.lib
+    h = sp.hex_desc()
+    go = sp.HexOutputGrads()
+    out = sp.HexOutputs(None, None, None, None, None, None, None)
+    assert lib.spin4d_hexplane_fwd(ctypes.byref(h), None, None, 0, None, None, None, None, None, out, None) == 0
+    assert lib.spin4d_hexplane_bwd(ctypes.byref(h), None, None, 0, None, None, None, None, None, None,
+                                   ctypes.byref(go), None, None, None, 0, None) == 0
+    saved = sp.HexSaved(FAKE, FAKE)
+    assert lib.spin4d_hexplane_bwd_saved(ctypes.byref(h), None, None, 0, None, None, None, None, ctypes.byref(saved),
+                                         None, ctypes.byref(go), None, None, None, 0, None) == 0
+    assert lib.spin4d_hexplane_bwd_workspace(ctypes.byref(h), 0) == 0
